@@ -1,0 +1,167 @@
+"""Oracle host block manager (test infrastructure only), in plain Python.
+
+What the pages fix:
+  * the pool is a set of equal, fixed-size physical blocks; a free list holds
+    the unused ones and finished requests return theirs to it
+    [PagedAttention & Continuous Batching (study notes), "Block tables";
+    Batching and PagedAttention, "PagedAttention", item 1];
+  * each sequence has a block table of logical -> physical ids, filled left
+    to right, growing by one block when the current one fills; nothing is
+    reserved ahead [Batching and PagedAttention, "PagedAttention", items 2-3];
+  * on a fork the child takes the parent's block ids and every shared block's
+    reference count goes up; a block goes back to the pool when its count
+    reaches zero; a write into a shared block first gets a fresh block and a
+    copy [study notes, "Copy-on-write"; 7.8 PagedAttention & continuous
+    batching (LLM deep dive), "01 Concept"];
+  * allocation fails when the free list is empty [study notes, Q&A "What
+    fails if you page KV but never cap concurrency?"];
+  * waste is at most one partly filled block per request [Batching and
+    PagedAttention, "PagedAttention"].
+
+Readings where the pages say nothing (the GPU build's manager follows the
+same ones, so block tables can be compared bit for bit):
+  * free list order: first in, first out, starting as 0, 1, ..., N-1;
+    allocation takes the head, a block whose count reaches zero joins the tail;
+  * freeing a sequence releases its blocks from the last logical block to the
+    first;
+  * sequence ids count up from 0 over add_seq and fork, never reused;
+  * append_slots(seq, n) first copies a shared, partly filled last block
+    (the copy-on-write block is allocated before any new block), then takes
+    one new block each time a token starts a block; the slot id of a token is
+    physical block * block_size + offset;
+  * an allocation that cannot be met in full changes nothing and counts one
+    allocation failure;
+  * tail waste counts every physical block in use once: block_size minus the
+    slots written in it.
+"""
+
+from collections import deque
+
+
+class OracleOOM(Exception):
+    """The free list cannot supply the blocks a call needs."""
+
+
+class OracleBlockManager:
+    def __init__(self, num_blocks, block_size):
+        if num_blocks < 0 or block_size < 1:
+            raise ValueError("bad pool geometry")
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+        self.free_list = deque(range(num_blocks))
+        self.refcount = [0] * num_blocks
+        self.filled = [0] * num_blocks      # slots written in each physical block
+        self.tables = {}                    # seq id -> list of physical ids
+        self.lengths = {}                   # seq id -> tokens stored
+        self.next_seq = 0
+        self.alloc_failures = 0
+
+    # -- sequences -----------------------------------------------------
+    def add_seq(self):
+        sid = self.next_seq
+        self.next_seq += 1
+        self.tables[sid] = []
+        self.lengths[sid] = 0
+        return sid
+
+    def _take(self):
+        block = self.free_list.popleft()
+        self.refcount[block] = 1
+        self.filled[block] = 0
+        return block
+
+    def _release(self, block):
+        self.refcount[block] -= 1
+        if self.refcount[block] == 0:
+            self.filled[block] = 0
+            self.free_list.append(block)
+
+    def blocks_needed(self, seq, n):
+        """Blocks an append of n tokens to seq would take from the free list."""
+        length, table, bs = self.lengths[seq], self.tables[seq], self.block_size
+        if n <= 0:
+            return 0
+        cow = 1 if (length % bs != 0 and self.refcount[table[-1]] > 1) else 0
+        grow = -(-(length + n) // bs) - -(-length // bs)
+        return cow + grow
+
+    def append_slots(self, seq, n):
+        """Reserve slots for the next n tokens of seq.
+
+        Returns (slots, pairs): slot id of each new token in order, and the
+        (source, destination) block pairs that must be copied before the
+        tokens are written.  Raises OracleOOM with nothing changed.
+        """
+        if seq not in self.tables:
+            raise KeyError(seq)
+        if n < 0:
+            raise ValueError("negative token count")
+        if self.blocks_needed(seq, n) > len(self.free_list):
+            self.alloc_failures += 1
+            raise OracleOOM(seq)
+        table, bs = self.tables[seq], self.block_size
+        length = self.lengths[seq]
+        pairs, slots = [], []
+        if n > 0 and length % bs != 0 and self.refcount[table[-1]] > 1:
+            src = table[-1]
+            dst = self._take()
+            self.filled[dst] = self.filled[src]
+            self.refcount[src] -= 1
+            table[-1] = dst
+            pairs.append((src, dst))
+        for pos in range(length, length + n):
+            if pos % bs == 0:
+                table.append(self._take())
+            block = table[pos // bs]
+            offset = pos % bs
+            self.filled[block] = max(self.filled[block], offset + 1)
+            slots.append(block * bs + offset)
+        self.lengths[seq] = length + n
+        return slots, pairs
+
+    def fork(self, parent):
+        """New sequence sharing every block of parent (reference counts +1)."""
+        if parent not in self.tables:
+            raise KeyError(parent)
+        child = self.next_seq
+        self.next_seq += 1
+        self.tables[child] = list(self.tables[parent])
+        self.lengths[child] = self.lengths[parent]
+        for block in self.tables[child]:
+            self.refcount[block] += 1
+        return child
+
+    def free(self, seq):
+        """Drop seq; blocks whose count reaches zero return to the free list."""
+        table = self.tables.pop(seq)
+        del self.lengths[seq]
+        for block in reversed(table):
+            self._release(block)
+
+    # -- views ---------------------------------------------------------
+    def block_table(self, seq):
+        return list(self.tables[seq])
+
+    def length(self, seq):
+        return self.lengths[seq]
+
+    def num_free(self):
+        return len(self.free_list)
+
+    def num_used(self):
+        return self.num_blocks - len(self.free_list)
+
+    def tail_waste(self):
+        """Unwritten slots summed over every physical block in use (once each)."""
+        return sum(self.block_size - self.filled[b] for b in range(self.num_blocks)
+                   if self.refcount[b] > 0)
+
+    def stats(self):
+        return {
+            "num_blocks": self.num_blocks,
+            "free_blocks": self.num_free(),
+            "used_blocks": self.num_used(),
+            "alloc_failures": self.alloc_failures,
+            "tail_waste_slots": self.tail_waste(),
+            "num_seqs": len(self.tables),
+        }

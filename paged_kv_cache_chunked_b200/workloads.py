@@ -1,0 +1,147 @@
+"""Seeded synthetic inputs shared by the tests, the bench and the smoke check.
+
+This module only draws random numbers and lays them out; it holds none of the
+method's arithmetic (no attention, no allocation policy).  Physical block ids
+are a seeded random permutation of the pool, so a sequence's blocks are
+scattered the way an allocator under churn leaves them [Batching and
+PagedAttention, "PagedAttention": blocks live anywhere in GPU memory].
+
+Workloads (sizes as the spec configurations name them):
+  tiny_fp32      4 decode sequences, contexts {5, 16, 17, 40}, block 16, pool of
+                 32 blocks, 8 q / 8 kv heads, head dim 64, float32, scale 1/8
+  decode64_bf16  64 decode sequences, contexts uniform in [128, 4096], block 16,
+                 32 q / 8 kv heads, head dim 128, pool 1.25x the blocks needed
+  longdoc_bf16   8 decode sequences of 32,768 tokens, block 16, 16 q / 4 kv
+                 heads, head dim 256, pool 1.25x
+"""
+
+import math
+import random
+
+import torch
+
+WORKLOADS = {
+    "tiny_fp32": dict(context_lens=[5, 16, 17, 40], block_size=16, num_blocks=32, n_q_heads=8,
+                      n_kv_heads=8, head_dim=64, dtype=torch.float32, seed=1001),
+    "decode64_bf16": dict(num_seqs=64, ctx_range=(128, 4096), block_size=16, n_q_heads=32,
+                          n_kv_heads=8, head_dim=128, dtype=torch.bfloat16, pool_factor=1.25,
+                          seed=1002),
+    "longdoc_bf16": dict(context_lens=[32768] * 8, block_size=16, n_q_heads=16, n_kv_heads=4,
+                         head_dim=256, dtype=torch.bfloat16, pool_factor=1.25, seed=1003),
+}
+
+
+def page_toy_lengths(n=200, seed=7, mean=600, floor=50, max_len=4096):
+    """Final request lengths of the capacity toy [Batching and PagedAttention,
+    "Try it"]: seeded exponential draws (mean 600) shifted by 50 and capped at
+    the longest allowed request."""
+    rng = random.Random(seed)
+    return [min(max_len, int(rng.expovariate(1.0 / mean)) + floor) for _ in range(n)]
+
+
+def decode_context_lens(num_seqs, lo, hi, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randint(lo, hi + 1, (num_seqs,), generator=g).tolist()
+
+
+def make_batch(context_lens, query_lens=None, *, block_size, n_q_heads, n_kv_heads, head_dim,
+               dtype, seed, num_blocks=None, pool_factor=1.25, table_width=None,
+               poison_unused=True, device="cpu", values="normal"):
+    """A paged batch with scattered blocks.
+
+    context_lens[b] tokens are stored for sequence b (the step's new tokens
+    included); query_lens[b] (default 1: decode) of them are this step's
+    queries.  Returns a dict with q [T, Hq, d], k_pool / v_pool [N, Hkv, bs, d],
+    block_tables [B, W] int32 (-1 padded), context_lens [B] int32,
+    query_start_lens [B + 1] int32 and scale = 1/sqrt(d).
+
+    Unused pool blocks and the unwritten tail slots of each last block are
+    filled with NaN when poison_unused is set, so that a kernel that reads
+    past a sequence's context or through a wrong table entry cannot pass.
+    """
+    B = len(context_lens)
+    if query_lens is None:
+        query_lens = [1] * B
+    g = torch.Generator().manual_seed(seed)
+    nblk = [math.ceil(c / block_size) for c in context_lens]
+    needed = sum(nblk)
+    if num_blocks is None:
+        num_blocks = max(needed, math.ceil(pool_factor * needed))
+    if num_blocks < needed:
+        raise ValueError("pool too small for the batch")
+    width = table_width if table_width is not None else max(nblk + [1])
+    perm = torch.randperm(num_blocks, generator=g)
+    tables = torch.full((B, width), -1, dtype=torch.int32)
+    pos = 0
+    for b in range(B):
+        tables[b, :nblk[b]] = perm[pos:pos + nblk[b]].to(torch.int32)
+        pos += nblk[b]
+
+    shape = (num_blocks, n_kv_heads, block_size, head_dim)
+    if values == "normal":
+        k_pool = torch.randn(shape, generator=g, dtype=torch.float32)
+        v_pool = torch.randn(shape, generator=g, dtype=torch.float32)
+    else:
+        raise ValueError(values)
+    if poison_unused:
+        used = torch.zeros((num_blocks, block_size), dtype=torch.bool)
+        for b in range(B):
+            for j in range(nblk[b]):
+                n_in = min(block_size, context_lens[b] - j * block_size)
+                used[tables[b, j], :n_in] = True
+        mask = (~used)[:, None, :, None].expand(shape)
+        k_pool[mask] = float("nan")
+        v_pool[mask] = float("nan")
+    T = sum(query_lens)
+    q = torch.randn((T, n_q_heads, head_dim), generator=g, dtype=torch.float32)
+    qsl = torch.zeros(B + 1, dtype=torch.int32)
+    qsl[1:] = torch.cumsum(torch.tensor(query_lens, dtype=torch.int32), 0)
+    return {
+        "q": q.to(dtype).to(device),
+        "k_pool": k_pool.to(dtype).to(device),
+        "v_pool": v_pool.to(dtype).to(device),
+        "block_tables": tables.to(device),
+        "context_lens": torch.tensor(context_lens, dtype=torch.int32).to(device),
+        "query_start_lens": qsl.to(device),
+        "scale": 1.0 / math.sqrt(head_dim),
+        "block_size": block_size,
+        "num_blocks": num_blocks,
+    }
+
+
+def workload_batch(name, device="cpu", poison_unused=True):
+    """The named decode workload (see the module docstring) as a batch."""
+    w = dict(WORKLOADS[name])
+    seed = w.pop("seed")
+    if "num_seqs" in w:
+        lo, hi = w.pop("ctx_range")
+        ctx = decode_context_lens(w.pop("num_seqs"), lo, hi, seed)
+    else:
+        ctx = w.pop("context_lens")
+    return make_batch(ctx, None, seed=seed, device=device, poison_unused=poison_unused, **w)
+
+
+def contiguous_to_paged(k_seq, v_seq, block_size, seed, num_blocks=None):
+    """Scatter per-sequence contiguous K/V ([c_b, Hkv, d] each) into a pool
+    with randomly permuted physical blocks.  Used to test that paging leaves
+    attention unchanged.  Returns (k_pool, v_pool, block_tables)."""
+    g = torch.Generator().manual_seed(seed)
+    B = len(k_seq)
+    Hkv, d = k_seq[0].shape[1], k_seq[0].shape[2]
+    nblk = [math.ceil(k.shape[0] / block_size) for k in k_seq]
+    needed = sum(nblk)
+    num_blocks = num_blocks or needed + 3
+    perm = torch.randperm(num_blocks, generator=g)
+    k_pool = torch.full((num_blocks, Hkv, block_size, d), float("nan"), dtype=k_seq[0].dtype)
+    v_pool = torch.full_like(k_pool, float("nan"))
+    tables = torch.full((B, max(nblk)), -1, dtype=torch.int32)
+    pos = 0
+    for b in range(B):
+        for j in range(nblk[b]):
+            blk = int(perm[pos])
+            pos += 1
+            tables[b, j] = blk
+            lo, hi = j * block_size, min((j + 1) * block_size, k_seq[b].shape[0])
+            k_pool[blk, :, :hi - lo, :] = k_seq[b][lo:hi].transpose(0, 1)
+            v_pool[blk, :, :hi - lo, :] = v_seq[b][lo:hi].transpose(0, 1)
+    return k_pool, v_pool, tables
