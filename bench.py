@@ -1,0 +1,422 @@
+#!/usr/bin/env python
+"""Benchmark of one step of the paged-KV hot path on B200.
+
+A step is one decode iteration of the named workload: append each sequence's
+new token's K/V into its block (paged_kv_append), then paged attention of
+every sequence's query over its whole paged context (plan + attention +
+split-K reduce kernels).  The workload has no forks, so the copy-on-write
+block copy has no work in it.  Every step leaves the pool in the same state
+(the appended rows are the values already stored at those slots), so all
+steps are the same work.
+
+Prints one JSON line.  `value` is the step's algorithmic bytes (KV read once
+per sequence and kv head, Q and output, block tables, the append's reads and
+writes) per second over all GPUs; `roofline` is the attention call alone.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                       [--workload decode64_bf16|longdoc_bf16]
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_chunked_b200.workloads import WORKLOADS, workload_batch  # noqa: E402
+
+METRIC = "paged decode attention KV GB/s (% of HBM peak) and tokens/s per scheduler step"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SRC = os.path.join(ROOT, "paged_kv_cache_chunked_b200", "csrc", "attention_tc.cu")
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="decode64_bf16", choices=["decode64_bf16", "longdoc_bf16"])
+    p.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--profile-run", action="store_true",
+                   help="timed steps only: no clock window, no e2e leg, no CPU baseline")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------- work accounting
+def step_bytes(batch):
+    """Algorithmic bytes of one step: attention and append separately."""
+    q = batch["q"]
+    T, Hq, d = q.shape
+    _, Hkv, bs, _ = batch["k_pool"].shape
+    elt = q.element_size()
+    ctx = batch["context_lens"].to(torch.int64)
+    kv = int(ctx.sum()) * Hkv * d * elt * 2
+    tables = int(((ctx + bs - 1) // bs).sum()) * 4
+    attn = kv + 2 * T * Hq * d * elt + tables
+    append = 2 * (2 * T * Hkv * d * elt) + 8 * T
+    return attn, append, kv
+
+
+def last_token_slots(batch):
+    bs = batch["block_size"]
+    ctx = batch["context_lens"].to(torch.int64)
+    tables = batch["block_tables"].to(torch.int64)
+    pos = ctx - 1
+    blk = tables.gather(1, (pos // bs)[:, None])[:, 0]
+    return blk * bs + pos % bs
+
+
+def new_token_kv(batch, slots):
+    bs = batch["block_size"]
+    blk, off = slots // bs, slots % bs
+    return batch["k_pool"][blk, :, off].contiguous(), batch["v_pool"][blk, :, off].contiguous()
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_traffic(workload):
+    """DRAM bytes per attention call from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    with open(KERNEL_SRC, "rb") as f:
+        src_hash = hashlib.sha256(f.read()).hexdigest()[:16]
+    entry = rec.get(workload)
+    if not entry or entry.get("kernel_sha256_16") != src_hash:
+        return None
+    return entry.get("dram_bytes_per_call")
+
+
+# ---------------------------------------------------------------- CPU / oracle arm
+def oracle_step_seconds(batch, budget_s, min_runs=1):
+    """The oracle's attention over the whole workload batch, repeated for about
+    budget_s seconds; returns (seconds per run, runs, threads)."""
+    import oracle
+    runs, t0 = 0, time.perf_counter()
+    while runs < min_runs or time.perf_counter() - t0 < budget_s:
+        oracle.paged_attention(batch["q"], batch["k_pool"], batch["v_pool"], batch["block_tables"],
+                               batch["context_lens"], batch["query_start_lens"], batch["scale"])
+        runs += 1
+    return (time.perf_counter() - t0) / runs, runs, oracle.num_threads()
+
+
+def subset_batch(batch, n):
+    """The first n sequences of a batch (same pools)."""
+    qsl = batch["query_start_lens"]
+    t1 = int(qsl[n])
+    sub = dict(batch)
+    sub["q"] = batch["q"][:t1]
+    sub["block_tables"] = batch["block_tables"][:n]
+    sub["context_lens"] = batch["context_lens"][:n]
+    sub["query_start_lens"] = qsl[:n + 1]
+    return sub
+
+
+def run_reference(args, rank, world):
+    """The oracle, as it stands, on the host cores (rank 0 only).  Each step is
+    the oracle append plus float64 attention over a leading subset of the
+    workload's sequences, sized so that the whole run stays near two
+    minutes."""
+    if rank != 0:
+        return
+    import oracle
+    batch = workload_batch(args.workload, poison_unused=False)
+    slots = last_token_slots(batch)
+    k_new, v_new = new_token_kv(batch, slots)
+    kp, vp = batch["k_pool"].clone(), batch["v_pool"].clone()
+
+    def step(b, n):
+        oracle.kv_append(kp, vp, k_new[:n], v_new[:n], slots[:n])
+        oracle.paged_attention(b["q"], kp, vp, b["block_tables"], b["context_lens"],
+                               b["query_start_lens"], b["scale"])
+
+    B = batch["context_lens"].shape[0]
+    t0 = time.perf_counter()
+    step(batch, B)
+    t_full = time.perf_counter() - t0
+    frac = min(1.0, 120.0 / max(1, args.steps + args.warmup) / t_full)
+    ctx = batch["context_lens"].to(torch.int64)
+    cum = torch.cumsum(ctx, 0)
+    n = int(min(B, max(1, int((cum < frac * int(ctx.sum())).sum()) + 1)))
+    sample = subset_batch(batch, n)
+    attn_b, app_b, _ = step_bytes(sample)
+    for _ in range(args.warmup):
+        step(sample, n)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step(sample, n)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = (attn_b + app_b) / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": workload_config(args.workload, batch, "oracle on host cores: L2 not applicable"),
+        "tokens_per_s": n / dt,
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"each step: oracle append + float64 attention of the first "
+                                   f"{n} of {B} sequences of {args.workload} "
+                                   f"({int(sample['context_lens'].sum())} context tokens)"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(name, batch, l2_note):
+    w = WORKLOADS[name]
+    ctx = batch["context_lens"]
+    return {"workload": name, "num_seqs": int(ctx.shape[0]), "context_tokens": int(ctx.sum()),
+            "n_q_heads": w["n_q_heads"], "n_kv_heads": w["n_kv_heads"], "head_dim": w["head_dim"],
+            "block_size": w["block_size"], "num_blocks": int(batch["k_pool"].shape[0]),
+            "seed": w["seed"], "l2": l2_note, "parallelism": "replicas"}
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, rank, world, device):
+    from paged_kv_cache_chunked_b200 import api
+
+    batch = workload_batch(args.workload, poison_unused=False)
+    attn_b, app_b, kv_b = step_bytes(batch)
+    T, Hq, d = batch["q"].shape
+    N, Hkv, bs, _ = batch["k_pool"].shape
+    slots = last_token_slots(batch)
+    k_new, v_new = new_token_kv(batch, slots)
+
+    pool = api.kv_pool_create(N, bs, Hkv, d, torch.bfloat16, device)
+    pool.k_pool.copy_(batch["k_pool"])
+    pool.v_pool.copy_(batch["v_pool"])
+    dq = batch["q"].to(device)
+    dt_ = batch["block_tables"].to(device)
+    dctx = batch["context_lens"].to(device)
+    dqsl = batch["query_start_lens"].to(device)
+    dslots = slots.to(device)
+    dk, dv = k_new.to(device), v_new.to(device)
+    out = torch.empty_like(dq)
+    stream = torch.cuda.current_stream(device)
+
+    def step(ev=None):
+        api.paged_kv_append(dk, dv, dslots, pool=pool)
+        if ev is not None:
+            ev[0].record(stream)
+        api.paged_attention(dq, pool.k_pool, pool.v_pool, dt_, dctx, dqsl, batch["scale"], out=out)
+        if ev is not None:
+            ev[1].record(stream)
+
+    launches_per_step = 1 + (3 if pool.dtype == torch.bfloat16 and d in (64, 128, 256) and bs % 8 == 0 else 1)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(device)
+    assert pool.check_device_errors() == 0
+
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    if not args.profile_run:
+        clocks.start()
+        time.sleep(0.3)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        tdist.barrier()
+    torch.cuda.synchronize(device)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    if dist:
+        tdist.barrier()
+    total_ms = start.elapsed_time(end)
+    attn_ms = [a.elapsed_time(b) for a, b in evs]
+    # a long enough window for the clock sampler to see the load
+    t_extra = time.perf_counter()
+    while not args.profile_run and time.perf_counter() - t_extra < 1.0:
+        for _ in range(20):
+            step()
+        torch.cuda.synchronize(device)
+    clk = clocks.stop() if not args.profile_run else {"sm_mhz": None, "reasons": ["not sampled"]}
+    assert pool.check_device_errors() == 0
+
+    if dist:
+        t = torch.tensor([total_ms], device=device)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * (attn_b + app_b) / (ms_per_step * 1e-3) / 1e9
+
+    # end to end through the public API: pinned host inputs in, output back out
+    e2e = None
+    if not args.no_e2e and not args.profile_run:
+        h_q = batch["q"].pin_memory()
+        h_k, h_v = k_new.pin_memory(), v_new.pin_memory()
+        h_slots = slots.pin_memory()
+        h_t = batch["block_tables"].pin_memory()
+        h_ctx = batch["context_lens"].pin_memory()
+        h_qsl = batch["query_start_lens"].pin_memory()
+        h_out = torch.empty_like(batch["q"]).pin_memory()
+        bufs = [torch.empty_like(x, device=device) for x in (h_q, h_k, h_v, h_slots, h_t, h_ctx, h_qsl)]
+        h2d = sum(x.numel() * x.element_size() for x in (h_q, h_k, h_v, h_slots, h_t, h_ctx, h_qsl))
+        d2h = h_out.numel() * h_out.element_size()
+
+        def e2e_step():
+            for dst, src in zip(bufs, (h_q, h_k, h_v, h_slots, h_t, h_ctx, h_qsl)):
+                dst.copy_(src, non_blocking=True)
+            api.paged_kv_append(bufs[1], bufs[2], bufs[3], pool=pool)
+            o = api.paged_attention(bufs[0], pool.k_pool, pool.v_pool, bufs[4], bufs[5], bufs[6],
+                                    batch["scale"], out=out)
+            h_out.copy_(o, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if dist:
+            tdist.barrier()
+        torch.cuda.synchronize(device)
+        s2.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e2.record(stream)
+        torch.cuda.synchronize(device)
+        e_ms = s2.elapsed_time(e2)
+        if dist:
+            t = torch.tensor([e_ms], device=device)
+            tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e_ms /= args.steps
+        e2e = {"value": world * (attn_b + app_b) / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        assert torch.isfinite(h_out.float()).all()
+
+    if rank != 0:
+        return
+    peak, peak_kind = measured_peak()
+    attn_avg_ms = statistics.mean(attn_ms)
+    achieved = attn_b / (attn_avg_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(args.workload, batch,
+                                  f"no flush: the step reads {kv_b / 1e6:.0f} MB of KV, "
+                                  f"more than the 126 MB L2"),
+        "pct_hbm": 100.0 * value / world / peak,
+        "tokens_per_s": world * T / (ms_per_step * 1e-3),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": kernel_traffic(args.workload),
+                     "kernel": "paged_attention call (plan + attention_tc + reduce)",
+                     "algorithmic_bytes": attn_b, "avg_ms": attn_avg_ms,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_kind == "measured" else "fallback 6.65 TB/s"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": dict(clk, window="the timed region plus 1 s of the same steps right after it"),
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if world == 1 and args.cpu_baseline_seconds > 0 and not args.profile_run:
+        sec, runs, threads = oracle_step_seconds(batch, args.cpu_baseline_seconds)
+        line["cpu_baseline"] = {"value": attn_b / sec / 1e9, "unit": "GB/s", "cores": threads,
+                                "kind": "oracle",
+                                "sample": f"float64 oracle attention over the whole {args.workload} "
+                                          f"batch (attention bytes only), {runs} runs"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=device)
+    try:
+        run_ours(args, rank, world, device)
+    finally:
+        if world > 1:
+            import torch.distributed as tdist
+            tdist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,213 @@
+/*
+ * paged_kv.h -- C ABI of the paged KV cache library for NVIDIA B200 (sm_100a).
+ *
+ * The library implements the data path of PagedAttention with continuous
+ * batching: a pool of fixed-size physical KV blocks, per-sequence block
+ * tables, the attention kernel that gathers K/V through those tables
+ * (decode rows and causal chunked-prefill rows, GQA), the slot-mapped append
+ * of new tokens' K/V, the whole-block copy used by copy-on-write, and the
+ * host-side block manager that produces tables, slots and copy pairs.
+ *
+ * Sources for what each call computes:
+ *   [SN]  "PagedAttention & Continuous Batching" (study notes), sections
+ *         "Block tables", "Copy-on-write", "Continuous batching", "Flow".
+ *   [BP]  "Batching and PagedAttention", sections "Continuous batching",
+ *         "PagedAttention", "Sharing blocks", "When blocks run out",
+ *         "Choosing the block size".
+ *   [DD]  "7.8 PagedAttention & continuous batching" (LLM deep dive),
+ *         "01 Concept".
+ *
+ * Conventions (every call):
+ *   - Returns int status: PK_OK (0) or one of the PK_ERR_* codes below.  On
+ *     error nothing is launched and pk_last_error() describes the cause.
+ *   - Device pointers belong to the caller and must stay valid until the work
+ *     queued on `stream` has finished.  Calls are asynchronous on `stream`
+ *     (a cudaStream_t; NULL is the legacy default stream).  Nothing
+ *     synchronises except pk_check_device_errors.
+ *   - Integer metadata that lives on the device (tables, lengths, slots,
+ *     copy pairs) cannot be checked before launch.  Kernels check every
+ *     block id and slot they dereference; a bad one is skipped (or replaced
+ *     by block 0 in attention), never dereferenced, and
+ *     PK_ERR_BAD_INDEX is recorded in the pool's device error word, which
+ *     pk_check_device_errors reads.  Results of such a call are undefined.
+ *   - Bounded waits: a pipeline wait that exceeds its iteration limit records
+ *     PK_ERR_TIMEOUT in the same word and the kernel returns.
+ *   - Threading: calls on different pools may run concurrently; calls on
+ *     one pk_bm must be serialised by the caller.
+ */
+#ifndef PAGED_KV_H
+#define PAGED_KV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *pk_stream_t; /* same type as cudaStream_t */
+
+enum {
+    PK_OK = 0,
+    PK_ERR_INVALID_ARG = 1,  /* bad host-side argument (shape, pointer, alignment) */
+    PK_ERR_OOM = 2,          /* block manager: not enough free blocks; state unchanged */
+    PK_ERR_UNSUPPORTED = 3,  /* dtype / geometry this build does not handle */
+    PK_ERR_CUDA = 4,         /* a CUDA runtime call failed (message in pk_last_error) */
+    PK_ERR_BAD_INDEX = 5,    /* device: a block id or slot outside the pool was skipped */
+    PK_ERR_WORKSPACE = 6,    /* workspace smaller than pk_attention_workspace_size */
+    PK_ERR_TIMEOUT = 7       /* device: a bounded pipeline wait ran out */
+};
+
+enum { PK_F32 = 0, PK_BF16 = 1 };
+
+/* Thread-local description of the last error of this thread ("" if none). */
+const char *pk_last_error(void);
+
+/* Library version string. */
+const char *pk_version(void);
+
+/* ------------------------------------------------------------------------
+ * KV pool  [SN "Block tables"; BP "PagedAttention" item 1; DD]
+ *
+ * GPU memory for one layer's cache is divided into num_blocks equal physical
+ * blocks, each holding K and V of block_size tokens.  Layout (both pools):
+ *     [num_blocks][n_kv_heads][block_size][head_dim]   row-major, dtype
+ * so the K (or V) rows of one (block, kv head) are one contiguous chunk of
+ * block_size * head_dim elements.  Token slot s (0 <= s < num_blocks *
+ * block_size) is block s / block_size, offset s % block_size.
+ *
+ * k_base / v_base: device memory of that size, owned by the caller (e.g.
+ * torch tensors), 16-byte aligned.  The library owns only the descriptor and
+ * a 4-byte device error word, both released by pk_pool_destroy.
+ * dtype: PK_F32 or PK_BF16.  head_dim: 1..256 (fast tensor-core path: bf16,
+ * head_dim 64/128/256, block_size a multiple of 8; anything else runs a
+ * general CUDA kernel).  The current CUDA device at create time is the
+ * pool's device; later calls must be made with that device current.
+ * ------------------------------------------------------------------------ */
+typedef struct pk_pool pk_pool;
+
+int pk_pool_create(int num_blocks, int block_size, int n_kv_heads, int head_dim, int dtype,
+                   void *k_base, void *v_base, pk_pool **out);
+int pk_pool_destroy(pk_pool *pool);
+
+/* Reads and clears the pool's device error word (synchronises `stream`).
+ * *code_out = PK_OK or the first PK_ERR_BAD_INDEX / PK_ERR_TIMEOUT recorded. */
+int pk_check_device_errors(const pk_pool *pool, pk_stream_t stream, int *code_out);
+
+/* ------------------------------------------------------------------------
+ * KV append  [SN "Flow" step 4 "Append KV into mapped blocks"; BP
+ * "PagedAttention" item 3: blocks are filled on demand as tokens arrive]
+ *
+ * For every token t < num_tokens with slot = slot_mapping[t] >= 0:
+ *     Kpool[slot / bs][h][slot % bs][:] = k[t][h][:]   for every kv head h
+ *     Vpool[...] likewise from v.
+ * k, v: device [num_tokens][n_kv_heads][head_dim] of the pool's dtype,
+ * contiguous.  slot_mapping: device int64 [num_tokens]; a negative slot
+ * skips the token; slots must be distinct within one call (otherwise which
+ * token wins is undefined).  Bit-exact copy.
+ * ------------------------------------------------------------------------ */
+int pk_paged_kv_append(const pk_pool *pool, const void *k, const void *v,
+                       const int64_t *slot_mapping, int num_tokens, pk_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Block copy (copy-on-write)  [SN "Copy-on-write": a write into a shared
+ * block allocates a fresh block, copies, then writes; DD]
+ *
+ * For each pair i < n_pairs: block dst = src_dst_pairs[2i+1] receives a copy
+ * of block src = src_dst_pairs[2i] -- all heads, all slots, K and V.
+ * src_dst_pairs: device int32 [n_pairs][2].  Destinations must be distinct
+ * and no destination may be a source in the same call (the pairs the block
+ * manager emits satisfy both).  Bit-exact copy.
+ * ------------------------------------------------------------------------ */
+int pk_block_copy(const pk_pool *pool, const int32_t *src_dst_pairs, int n_pairs,
+                  pk_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Paged attention  [SN "Block tables": the kernel gathers through the table;
+ * BP "PagedAttention" item 4; BP "Continuous batching": one step mixes
+ * prefill chunks and decodes, long prompts are split into chunks]
+ *
+ * Batch of num_seqs sequences.  Sequence b has context_lens[b] = c_b tokens
+ * stored in the pool (this step's new tokens included: append first, then
+ * attend) and q_b = query_start_lens[b+1] - query_start_lens[b] >= 1 query
+ * tokens, the last q_b of its context (q_b = 1: decode; q_b > 1: a chunk).
+ * For query token i of b (logical position p = c_b - q_b + i) and q head h:
+ *     kvh = h / (n_q_heads / n_kv_heads)
+ *     K_j = Kpool[block_tables[b][j / bs]][kvh][j % bs][:]   (j = 0..p)
+ *     out[t][h][:] = sum_j softmax_j(scale * q[t][h] . K_j) * V_j
+ * computed with fp32 accumulation and an online softmax.
+ *
+ * q, out: device [num_tokens][n_q_heads][head_dim], the pool's dtype,
+ *   contiguous; num_tokens = query_start_lens[num_seqs].
+ * block_tables: device int32 [num_seqs][max_blocks_per_seq]; entries past
+ *   ceil(c_b / bs) are never read.  context_lens: device int32 [num_seqs],
+ *   1 <= c_b <= max_blocks_per_seq * bs.  query_start_lens: device int32
+ *   [num_seqs + 1], query_start_lens[0] = 0, 1 <= q_b <= c_b.
+ * n_q_heads % n_kv_heads == 0.
+ * workspace: device scratch of at least pk_attention_workspace_size bytes,
+ *   16-byte aligned, owned by the caller, not shared by calls in flight at the
+ *   same time; it holds the work list and the split-K partial results.
+ * ------------------------------------------------------------------------ */
+int pk_attention_workspace_size(const pk_pool *pool, int num_seqs, int num_tokens,
+                                int n_q_heads, int max_blocks_per_seq, size_t *bytes_out);
+
+int pk_paged_attention(const pk_pool *pool, const void *q, void *out,
+                       const int32_t *block_tables, int max_blocks_per_seq,
+                       const int32_t *context_lens, const int32_t *query_start_lens,
+                       int num_seqs, int num_tokens, int n_q_heads, float scale,
+                       void *workspace, size_t workspace_bytes, pk_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Host block manager  [SN "Block tables", "Copy-on-write"; BP
+ * "PagedAttention", "Sharing blocks", "When blocks run out"; DD]
+ *
+ * Free list, per-sequence block tables, reference counts, fork and
+ * copy-on-write, on the host.  Policy (fixed so that two implementations
+ * produce the same tables): the free list is first-in first-out starting as
+ * 0..num_blocks-1; a freed block joins its tail; freeing a sequence releases
+ * its blocks from the last logical block to the first; sequence ids count up
+ * from 0 over add_seq and fork.
+ * ------------------------------------------------------------------------ */
+typedef struct pk_bm pk_bm;
+
+typedef struct {
+    int64_t num_blocks;
+    int64_t free_blocks;
+    int64_t used_blocks;
+    int64_t alloc_failures;   /* append_slots calls refused with PK_ERR_OOM */
+    int64_t tail_waste_slots; /* unwritten slots over all blocks in use, each block once */
+    int64_t num_seqs;
+} pk_bm_stats;
+
+int pk_bm_create(int num_blocks, int block_size, pk_bm **out);
+int pk_bm_destroy(pk_bm *bm);
+/* New empty sequence; its id in *seq_out. */
+int pk_bm_add_seq(pk_bm *bm, int64_t *seq_out);
+/* Reserve slots for the next n tokens of seq.  slots_out[n] receives the slot
+ * id of each token.  If the sequence's last block is partly filled and shared
+ * (reference count > 1) a fresh block is taken first and the pair
+ * (old, new) is written to pairs_out (int32 [pairs_cap][2]); *n_pairs_out is
+ * the number of pairs (0 or 1).  The caller must run pk_block_copy on the
+ * pairs before appending.  PK_ERR_OOM: not enough free blocks; nothing
+ * changed. */
+int pk_bm_append_slots(pk_bm *bm, int64_t seq, int n, int64_t *slots_out, int32_t *pairs_out,
+                       int pairs_cap, int *n_pairs_out);
+/* Blocks append_slots(seq, n) would take from the free list. */
+int pk_bm_blocks_needed(const pk_bm *bm, int64_t seq, int n, int *needed_out);
+/* New sequence sharing all of parent's blocks (reference counts + 1). */
+int pk_bm_fork(pk_bm *bm, int64_t parent, int64_t *child_out);
+/* Drop seq; blocks no longer referenced return to the free list. */
+int pk_bm_free(pk_bm *bm, int64_t seq);
+/* Copy seq's block table (ceil(len / bs) ids) into out[cap]; *n_out = count. */
+int pk_bm_block_table(const pk_bm *bm, int64_t seq, int32_t *out, int cap, int *n_out);
+/* Fill out[n_seqs][width] (int32, row-major) with the tables of seqs[], -1 padded. */
+int pk_bm_fill_tables(const pk_bm *bm, const int64_t *seqs, int n_seqs, int32_t *out, int width);
+int pk_bm_seq_len(const pk_bm *bm, int64_t seq, int64_t *len_out);
+int pk_bm_refcount(const pk_bm *bm, int32_t block, int *count_out);
+int pk_bm_get_stats(const pk_bm *bm, pk_bm_stats *out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_KV_H */

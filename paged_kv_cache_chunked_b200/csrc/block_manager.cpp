@@ -1,0 +1,236 @@
+// Host block manager of the paged KV cache (C ABI pk_bm_*).
+//
+// What it keeps, from the pages:
+//  * a pool of equal physical blocks and a free list; finished requests
+//    return their blocks to it ["PagedAttention & Continuous Batching"
+//    (study notes), "Block tables"; "Batching and PagedAttention",
+//    "PagedAttention" items 1-3: blocks are allocated one at a time on demand,
+//    nothing is reserved for a maximum length];
+//  * a block table per sequence, logical block i -> physical id, filled left
+//    to right;
+//  * reference counts: a fork copies the parent's ids and increments the
+//    counts; a write into a shared block first takes a fresh block and a copy
+//    of the old one (copy-on-write); a block returns to the free list when its
+//    count reaches zero [study notes, "Copy-on-write"; "7.8 PagedAttention &
+//    continuous batching" (LLM deep dive), "01 Concept"];
+//  * allocation fails cleanly when the free list runs dry [study notes, Q&A
+//    on capping concurrency], leaving the state unchanged;
+//  * the operational counters the deep-dive page lists: free and used
+//    blocks, allocation failures, tail waste.
+//
+// Policy details the pages leave open, fixed so that tables are reproducible:
+// FIFO free list starting as 0..N-1 (a released block joins the tail);
+// a sequence's blocks are released from its last logical block to its first;
+// sequence ids count up from 0; in append_slots the copy-on-write block is
+// taken before any new block.
+#include <cstdint>
+#include <deque>
+#include <new>
+#include <unordered_map>
+#include <vector>
+
+#include "paged_kv.h"
+
+namespace pk {
+int fail(int code, const char *fmt, ...);
+}
+
+struct pk_bm {
+    int num_blocks;
+    int block_size;
+    std::deque<int32_t> free_list;
+    std::vector<int32_t> refcount;
+    std::vector<int32_t> filled;  // slots written in each physical block
+    struct Seq {
+        std::vector<int32_t> table;
+        int64_t len = 0;
+    };
+    std::unordered_map<int64_t, Seq> seqs;
+    int64_t next_seq = 0;
+    int64_t alloc_failures = 0;
+
+    int32_t take() {
+        const int32_t b = free_list.front();
+        free_list.pop_front();
+        refcount[b] = 1;
+        filled[b] = 0;
+        return b;
+    }
+    void release(int32_t b) {
+        if (--refcount[b] == 0) {
+            filled[b] = 0;
+            free_list.push_back(b);
+        }
+    }
+    int64_t needed(const Seq &s, int n) const {
+        if (n <= 0) return 0;
+        const int64_t bs = block_size;
+        const int cow = (s.len % bs != 0 && refcount[s.table.back()] > 1) ? 1 : 0;
+        const int64_t grow = (s.len + n + bs - 1) / bs - (s.len + bs - 1) / bs;
+        return cow + grow;
+    }
+};
+
+using pk::fail;
+
+extern "C" {
+
+int pk_bm_create(int num_blocks, int block_size, pk_bm **out) {
+    if (!out) return fail(PK_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (num_blocks < 0 || block_size < 1) return fail(PK_ERR_INVALID_ARG, "bad pool geometry");
+    pk_bm *bm = new (std::nothrow) pk_bm();
+    if (!bm) return fail(PK_ERR_INVALID_ARG, "out of host memory");
+    bm->num_blocks = num_blocks;
+    bm->block_size = block_size;
+    bm->refcount.assign(num_blocks, 0);
+    bm->filled.assign(num_blocks, 0);
+    for (int32_t b = 0; b < num_blocks; ++b) bm->free_list.push_back(b);
+    *out = bm;
+    return PK_OK;
+}
+
+int pk_bm_destroy(pk_bm *bm) {
+    delete bm;
+    return PK_OK;
+}
+
+int pk_bm_add_seq(pk_bm *bm, int64_t *seq_out) {
+    if (!bm || !seq_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    const int64_t id = bm->next_seq++;
+    bm->seqs.emplace(id, pk_bm::Seq());
+    *seq_out = id;
+    return PK_OK;
+}
+
+int pk_bm_blocks_needed(const pk_bm *bm, int64_t seq, int n, int *needed_out) {
+    if (!bm || !needed_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    auto it = bm->seqs.find(seq);
+    if (it == bm->seqs.end()) return fail(PK_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq);
+    if (n < 0) return fail(PK_ERR_INVALID_ARG, "negative token count");
+    *needed_out = (int)bm->needed(it->second, n);
+    return PK_OK;
+}
+
+int pk_bm_append_slots(pk_bm *bm, int64_t seq, int n, int64_t *slots_out, int32_t *pairs_out,
+                       int pairs_cap, int *n_pairs_out) {
+    if (!bm || !n_pairs_out || (n > 0 && !slots_out)) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    auto it = bm->seqs.find(seq);
+    if (it == bm->seqs.end()) return fail(PK_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq);
+    if (n < 0) return fail(PK_ERR_INVALID_ARG, "negative token count");
+    pk_bm::Seq &s = it->second;
+    *n_pairs_out = 0;
+    if (n == 0) return PK_OK;
+    const int64_t bs = bm->block_size;
+    const bool cow = s.len % bs != 0 && bm->refcount[s.table.back()] > 1;
+    if (cow && (pairs_cap < 1 || !pairs_out))
+        return fail(PK_ERR_INVALID_ARG, "copy-on-write pair needs pairs_out");
+    if (bm->needed(s, n) > (int64_t)bm->free_list.size()) {
+        ++bm->alloc_failures;
+        return fail(PK_ERR_OOM, "need %lld blocks, %zu free", (long long)bm->needed(s, n),
+                    bm->free_list.size());
+    }
+    if (cow) {
+        const int32_t src = s.table.back();
+        const int32_t dst = bm->take();
+        bm->filled[dst] = bm->filled[src];
+        --bm->refcount[src];
+        s.table.back() = dst;
+        pairs_out[0] = src;
+        pairs_out[1] = dst;
+        *n_pairs_out = 1;
+    }
+    for (int i = 0; i < n; ++i) {
+        const int64_t pos = s.len + i;
+        if (pos % bs == 0) s.table.push_back(bm->take());
+        const int32_t blk = s.table[pos / bs];
+        const int32_t off = (int32_t)(pos % bs);
+        if (bm->filled[blk] < off + 1) bm->filled[blk] = off + 1;
+        slots_out[i] = (int64_t)blk * bs + off;
+    }
+    s.len += n;
+    return PK_OK;
+}
+
+int pk_bm_fork(pk_bm *bm, int64_t parent, int64_t *child_out) {
+    if (!bm || !child_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    auto it = bm->seqs.find(parent);
+    if (it == bm->seqs.end()) return fail(PK_ERR_INVALID_ARG, "unknown sequence %lld", (long long)parent);
+    pk_bm::Seq child = it->second;  // copy before emplace can rehash
+    for (int32_t b : child.table) ++bm->refcount[b];
+    const int64_t id = bm->next_seq++;
+    bm->seqs.emplace(id, std::move(child));
+    *child_out = id;
+    return PK_OK;
+}
+
+int pk_bm_free(pk_bm *bm, int64_t seq) {
+    if (!bm) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    auto it = bm->seqs.find(seq);
+    if (it == bm->seqs.end()) return fail(PK_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq);
+    const std::vector<int32_t> &t = it->second.table;
+    for (auto b = t.rbegin(); b != t.rend(); ++b) bm->release(*b);
+    bm->seqs.erase(it);
+    return PK_OK;
+}
+
+int pk_bm_block_table(const pk_bm *bm, int64_t seq, int32_t *out, int cap, int *n_out) {
+    if (!bm || !n_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    auto it = bm->seqs.find(seq);
+    if (it == bm->seqs.end()) return fail(PK_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq);
+    const std::vector<int32_t> &t = it->second.table;
+    *n_out = (int)t.size();
+    if ((int)t.size() > cap || (!out && !t.empty()))
+        return fail(PK_ERR_INVALID_ARG, "table of %zu entries, capacity %d", t.size(), cap);
+    for (size_t i = 0; i < t.size(); ++i) out[i] = t[i];
+    return PK_OK;
+}
+
+int pk_bm_fill_tables(const pk_bm *bm, const int64_t *seqs, int n_seqs, int32_t *out, int width) {
+    if (!bm || (n_seqs > 0 && (!seqs || !out)) || n_seqs < 0 || width < 0)
+        return fail(PK_ERR_INVALID_ARG, "bad argument");
+    for (int i = 0; i < n_seqs; ++i) {
+        auto it = bm->seqs.find(seqs[i]);
+        if (it == bm->seqs.end())
+            return fail(PK_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seqs[i]);
+        const std::vector<int32_t> &t = it->second.table;
+        if ((int)t.size() > width)
+            return fail(PK_ERR_INVALID_ARG, "table of %zu entries, width %d", t.size(), width);
+        int32_t *row = out + (int64_t)i * width;
+        size_t j = 0;
+        for (; j < t.size(); ++j) row[j] = t[j];
+        for (; j < (size_t)width; ++j) row[j] = -1;
+    }
+    return PK_OK;
+}
+
+int pk_bm_seq_len(const pk_bm *bm, int64_t seq, int64_t *len_out) {
+    if (!bm || !len_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    auto it = bm->seqs.find(seq);
+    if (it == bm->seqs.end()) return fail(PK_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq);
+    *len_out = it->second.len;
+    return PK_OK;
+}
+
+int pk_bm_refcount(const pk_bm *bm, int32_t block, int *count_out) {
+    if (!bm || !count_out || block < 0 || block >= bm->num_blocks)
+        return fail(PK_ERR_INVALID_ARG, "bad argument");
+    *count_out = bm->refcount[block];
+    return PK_OK;
+}
+
+int pk_bm_get_stats(const pk_bm *bm, pk_bm_stats *out) {
+    if (!bm || !out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    out->num_blocks = bm->num_blocks;
+    out->free_blocks = (int64_t)bm->free_list.size();
+    out->used_blocks = bm->num_blocks - out->free_blocks;
+    out->alloc_failures = bm->alloc_failures;
+    int64_t waste = 0;
+    for (int b = 0; b < bm->num_blocks; ++b)
+        if (bm->refcount[b] > 0) waste += bm->block_size - bm->filled[b];
+    out->tail_waste_slots = waste;
+    out->num_seqs = (int64_t)bm->seqs.size();
+    return PK_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,190 @@
+// Slot-mapped KV append and whole-block copy (copy-on-write).
+//
+// Append ["PagedAttention & Continuous Batching" (study notes), "Flow" step 4:
+// new tokens' K/V go into the blocks their table maps them to]: token t's K
+// and V rows (all kv heads) are stored at slot slot_mapping[t] = block *
+// block_size + offset; negative slots are skipped.
+// Block copy [same page, "Copy-on-write": a write into a shared block takes a
+// fresh block and copies it first]: block dst receives all of block src, K
+// and V.
+//
+// Both are pure data movement, bound by HBM bandwidth: each thread moves
+// 16-byte vectors with streaming loads/stores, consecutive threads touch
+// consecutive 16-byte chunks of one (block, head) row so every warp access is
+// a full 512-byte coalesced segment.
+#include "pk_internal.h"
+
+namespace pk {
+namespace {
+
+struct alignas(16) Vec16 {
+    uint4 v;
+};
+
+// One thread per 16-byte chunk of one (token, head) row of K or V.
+// Grid-stride over num_tokens * n_kv_heads * row_chunks * 2.
+__global__ void kv_append_vec16(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
+                                uint4 *__restrict__ kp, uint4 *__restrict__ vp,
+                                const int64_t *__restrict__ slots, int num_tokens, int n_kv_heads,
+                                int block_size, int row_chunks, int64_t num_slots,
+                                int *err) {
+    const int64_t per_side = (int64_t)num_tokens * n_kv_heads * row_chunks;
+    const int64_t total = 2 * per_side;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const bool is_v = i >= per_side;
+        const int64_t j = is_v ? i - per_side : i;
+        const int c = (int)(j % row_chunks);
+        const int64_t th = j / row_chunks;  // token * n_kv_heads + head
+        const int h = (int)(th % n_kv_heads);
+        const int64_t t = th / n_kv_heads;
+        const int64_t slot = __ldg(slots + t);
+        if (slot < 0) continue;
+        if (slot >= num_slots) {
+            record_error(err, PK_ERR_BAD_INDEX);
+            continue;
+        }
+        const int64_t blk = slot / block_size;
+        const int off = (int)(slot % block_size);
+        const int64_t dst = ((blk * n_kv_heads + h) * block_size + off) * row_chunks + c;
+        const uint4 val = __ldcs((is_v ? v : k) + j);
+        __stcs((is_v ? vp : kp) + dst, val);
+    }
+}
+
+// Element-wise fallback for rows that are not a multiple of 16 bytes.
+template <typename T>
+__global__ void kv_append_scalar(const T *__restrict__ k, const T *__restrict__ v, T *kp, T *vp,
+                                 const int64_t *__restrict__ slots, int num_tokens,
+                                 int n_kv_heads, int block_size, int head_dim,
+                                 int64_t num_slots, int *err) {
+    const int64_t per_side = (int64_t)num_tokens * n_kv_heads * head_dim;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < 2 * per_side;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const bool is_v = i >= per_side;
+        const int64_t j = is_v ? i - per_side : i;
+        const int e = (int)(j % head_dim);
+        const int64_t th = j / head_dim;
+        const int h = (int)(th % n_kv_heads);
+        const int64_t t = th / n_kv_heads;
+        const int64_t slot = slots[t];
+        if (slot < 0) continue;
+        if (slot >= num_slots) {
+            record_error(err, PK_ERR_BAD_INDEX);
+            continue;
+        }
+        const int64_t dst = (((slot / block_size) * n_kv_heads + h) * block_size +
+                             slot % block_size) * head_dim + e;
+        (is_v ? vp : kp)[dst] = (is_v ? v : k)[j];
+    }
+}
+
+// One CTA per (pair, K or V); the block's bytes are copied as 16-byte vectors.
+__global__ void block_copy_vec16(uint4 *kp, uint4 *vp, const int32_t *__restrict__ pairs,
+                                 int n_pairs, int64_t block_chunks, int num_blocks, int *err) {
+    for (int64_t w = blockIdx.x; w < 2LL * n_pairs; w += gridDim.x) {
+        const int pr = (int)(w >> 1);
+        uint4 *pool = (w & 1) ? vp : kp;
+        const int src = __ldg(pairs + 2 * pr);
+        const int dst = __ldg(pairs + 2 * pr + 1);
+        if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+            if (threadIdx.x == 0) record_error(err, PK_ERR_BAD_INDEX);
+            continue;
+        }
+        const uint4 *s = pool + (int64_t)src * block_chunks;
+        uint4 *d = pool + (int64_t)dst * block_chunks;
+        // unrolled by 4 so that each thread keeps several loads in flight
+        int64_t i = threadIdx.x;
+        for (; i + 3 * blockDim.x < block_chunks; i += 4 * blockDim.x) {
+            uint4 a = __ldcs(s + i), b = __ldcs(s + i + blockDim.x);
+            uint4 c = __ldcs(s + i + 2 * blockDim.x), e = __ldcs(s + i + 3 * blockDim.x);
+            __stcs(d + i, a);
+            __stcs(d + i + blockDim.x, b);
+            __stcs(d + i + 2 * blockDim.x, c);
+            __stcs(d + i + 3 * blockDim.x, e);
+        }
+        for (; i < block_chunks; i += blockDim.x) __stcs(d + i, __ldcs(s + i));
+    }
+}
+
+template <typename T>
+__global__ void block_copy_scalar(T *kp, T *vp, const int32_t *__restrict__ pairs, int n_pairs,
+                                  int64_t block_elems, int num_blocks, int *err) {
+    for (int64_t w = blockIdx.x; w < 2LL * n_pairs; w += gridDim.x) {
+        const int pr = (int)(w >> 1);
+        T *pool = (w & 1) ? vp : kp;
+        const int src = pairs[2 * pr], dst = pairs[2 * pr + 1];
+        if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+            if (threadIdx.x == 0) record_error(err, PK_ERR_BAD_INDEX);
+            continue;
+        }
+        for (int64_t i = threadIdx.x; i < block_elems; i += blockDim.x)
+            pool[(int64_t)dst * block_elems + i] = pool[(int64_t)src * block_elems + i];
+    }
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15) == 0; }
+
+int grid_for(int64_t work, int threads, int sm_count) {
+    int64_t g = (work + threads - 1) / threads;
+    int64_t cap = (int64_t)sm_count * 16;
+    if (g > cap) g = cap;
+    return (int)(g < 1 ? 1 : g);
+}
+
+}  // namespace
+
+int launch_kv_append(const pk_pool *p, const void *k, const void *v, const int64_t *slots,
+                     int num_tokens, cudaStream_t st) {
+    if (num_tokens == 0) return PK_OK;
+    const int elt = p->dtype == PK_BF16 ? 2 : 4;
+    const int64_t row_bytes = (int64_t)p->head_dim * elt;
+    const int64_t num_slots = (int64_t)p->num_blocks * p->block_size;
+    if (row_bytes % 16 == 0 && aligned16(k) && aligned16(v)) {
+        const int row_chunks = (int)(row_bytes / 16);
+        const int64_t work = 2LL * num_tokens * p->n_kv_heads * row_chunks;
+        kv_append_vec16<<<grid_for(work, 256, p->sm_count), 256, 0, st>>>(
+            (const uint4 *)k, (const uint4 *)v, (uint4 *)p->k_base, (uint4 *)p->v_base, slots,
+            num_tokens, p->n_kv_heads, p->block_size, row_chunks, num_slots, p->d_err);
+    } else {
+        const int64_t work = 2LL * num_tokens * p->n_kv_heads * p->head_dim;
+        if (p->dtype == PK_BF16)
+            kv_append_scalar<uint16_t><<<grid_for(work, 256, p->sm_count), 256, 0, st>>>(
+                (const uint16_t *)k, (const uint16_t *)v, (uint16_t *)p->k_base,
+                (uint16_t *)p->v_base, slots, num_tokens, p->n_kv_heads, p->block_size,
+                p->head_dim, num_slots, p->d_err);
+        else
+            kv_append_scalar<float><<<grid_for(work, 256, p->sm_count), 256, 0, st>>>(
+                (const float *)k, (const float *)v, (float *)p->k_base, (float *)p->v_base,
+                slots, num_tokens, p->n_kv_heads, p->block_size, p->head_dim, num_slots,
+                p->d_err);
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PK_OK : cuda_fail(e, "kv append launch");
+}
+
+int launch_block_copy(const pk_pool *p, const int32_t *pairs, int n_pairs, cudaStream_t st) {
+    if (n_pairs == 0) return PK_OK;
+    const int elt = p->dtype == PK_BF16 ? 2 : 4;
+    const int64_t block_elems = (int64_t)p->n_kv_heads * p->block_size * p->head_dim;
+    const int64_t block_bytes = block_elems * elt;
+    const int64_t ctas = 2LL * n_pairs;
+    const int grid = (int)(ctas < (int64_t)p->sm_count * 32 ? ctas : (int64_t)p->sm_count * 32);
+    if (block_bytes % 16 == 0) {
+        block_copy_vec16<<<grid, 256, 0, st>>>((uint4 *)p->k_base, (uint4 *)p->v_base, pairs,
+                                               n_pairs, block_bytes / 16, p->num_blocks,
+                                               p->d_err);
+    } else if (p->dtype == PK_BF16) {
+        block_copy_scalar<uint16_t><<<grid, 256, 0, st>>>((uint16_t *)p->k_base,
+                                                          (uint16_t *)p->v_base, pairs, n_pairs,
+                                                          block_elems, p->num_blocks, p->d_err);
+    } else {
+        block_copy_scalar<float><<<grid, 256, 0, st>>>((float *)p->k_base, (float *)p->v_base,
+                                                       pairs, n_pairs, block_elems,
+                                                       p->num_blocks, p->d_err);
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PK_OK : cuda_fail(e, "block copy launch");
+}
+
+}  // namespace pk

@@ -1,0 +1,71 @@
+// Internal declarations of the paged KV library (not part of the C ABI).
+#pragma once
+
+#include <cuda.h>  // CUtensorMap (type only; the driver entry point is fetched at run time)
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "paged_kv.h"
+
+// Pool descriptor behind the opaque pk_pool handle.
+struct pk_pool {
+    int num_blocks;
+    int block_size;
+    int n_kv_heads;
+    int head_dim;
+    int dtype;  // PK_F32 / PK_BF16
+    void *k_base;
+    void *v_base;
+    int *d_err;       // device error word (first recorded PK_ERR_* code)
+    int device;
+    int sm_count;
+    bool tc_path;     // tensor-core + TMA attention applies to this geometry
+    int tc_ctas;      // resident CTAs of the tensor-core attention kernel (whole GPU)
+    alignas(64) CUtensorMap tmap_k;
+    alignas(64) CUtensorMap tmap_v;
+};
+
+namespace pk {
+
+// Sets the thread-local error message; returns `code`.
+int fail(int code, const char *fmt, ...);
+int cuda_fail(cudaError_t e, const char *what);
+
+// Records `code` in the device error word unless an earlier code is there.
+__device__ __forceinline__ void record_error(int *err, int code) {
+    if (err) atomicCAS(err, 0, code);
+}
+
+constexpr int kMaxHeadDim = 256;
+constexpr int kTile = 16;        // tokens per KV tile and rows per query tile
+constexpr int kConsumers = 4;    // consumer warps of the tensor-core attention kernel
+
+// ---- launchers (each returns PK_OK or an error code) ---------------------
+int launch_kv_append(const pk_pool *p, const void *k, const void *v, const int64_t *slots,
+                     int num_tokens, cudaStream_t st);
+int launch_block_copy(const pk_pool *p, const int32_t *pairs, int n_pairs, cudaStream_t st);
+
+struct AttnArgs {
+    const void *q;
+    void *out;
+    const int32_t *block_tables;
+    int max_blocks_per_seq;
+    const int32_t *context_lens;
+    const int32_t *query_start_lens;
+    int num_seqs;
+    int num_tokens;
+    int n_q_heads;
+    float scale;
+    void *workspace;
+    size_t workspace_bytes;
+};
+
+int launch_attention_generic(const pk_pool *p, const AttnArgs &a, cudaStream_t st);
+
+// Tensor-core path: workspace sizing and launch.
+size_t tc_workspace_bytes(const pk_pool *p, int num_seqs, int num_tokens, int n_q_heads,
+                          int max_blocks_per_seq);
+int tc_prepare_pool(pk_pool *p);  // occupancy query, once per pool
+int launch_attention_tc(const pk_pool *p, const AttnArgs &a, cudaStream_t st);
+
+}  // namespace pk

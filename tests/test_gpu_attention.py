@@ -1,0 +1,171 @@
+"""GPU parity of paged attention against the float64 oracle.
+
+Tolerance: |gpu - oracle| <= 2e-2 + 2e-2 |oracle| for bf16 inputs with fp32
+accumulation, 1e-4 + 1e-4 |oracle| for fp32 inputs, element by element.
+Pools are seeded N(0, 1); every slot no sequence owns (unused blocks, the
+tail of each last block) holds NaN, so reading past a context or through a
+wrong table entry fails the test.
+"""
+
+import math
+import os
+
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_chunked_b200 import api
+from paged_kv_cache_chunked_b200.workloads import make_batch, workload_batch, contiguous_to_paged
+
+from helpers import (assert_close, gpu_pool_from, oracle_attention, run_gpu_attention,
+                     sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+def _check(batch, Hq, Hkv, d, dtype, dev, what):
+    pool = gpu_pool_from(batch, Hkv, d, dtype, dev)
+    got = run_gpu_attention(batch, pool, dev)
+    ref = oracle_attention(batch)
+    err = assert_close(got, ref, dtype, what)
+    assert pool.check_device_errors() == 0
+    return got, err
+
+
+def test_tiny_fp32_decode(cuda_dev):
+    # 4 decode sequences, contexts {5, 16, 17, 40}, block 16, 32-block pool,
+    # 8 q / 8 kv heads, head dim 64, float32, scale 1/8
+    b = workload_batch("tiny_fp32")
+    _check(b, 8, 8, 64, torch.float32, cuda_dev, "tiny fp32")
+
+
+def test_tiny_fp32_as_causal_chunks(cuda_dev):
+    # the same contexts processed as 8-token causal chunks (the last 8 tokens
+    # of each context are queries; context 5 takes all 5)
+    ctx = [5, 16, 17, 40]
+    b = make_batch(ctx, [min(8, c) for c in ctx], block_size=16, num_blocks=32, n_q_heads=8,
+                   n_kv_heads=8, head_dim=64, dtype=torch.float32, seed=1001)
+    _check(b, 8, 8, 64, torch.float32, cuda_dev, "tiny fp32 chunks")
+
+
+DECODE_CASES = [
+    # contexts, Hq, Hkv, d, block size
+    ([1, 2, 15, 16, 17, 31, 33, 100, 257, 600], 32, 8, 128, 16),
+    ([5, 77, 300, 1029], 16, 4, 256, 16),
+    ([3, 64, 65, 900], 8, 8, 64, 16),
+    ([9, 120, 513], 32, 8, 128, 8),
+    ([40, 700, 1], 32, 8, 128, 32),
+    ([50, 333], 28, 4, 128, 16),      # group of 7
+    ([21, 400], 16, 1, 128, 16),      # group of 16
+    ([30, 250], 32, 1, 128, 16),      # group of 32: two row tiles per token
+    ([64, 1000], 8, 8, 128, 16),      # group of 1
+]
+
+
+@pytest.mark.parametrize("ctx,Hq,Hkv,d,bs", DECODE_CASES)
+def test_bf16_decode(cuda_dev, ctx, Hq, Hkv, d, bs):
+    b = make_batch(ctx, None, block_size=bs, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d,
+                   dtype=torch.bfloat16, seed=sum(ctx) + d)
+    _check(b, Hq, Hkv, d, torch.bfloat16, cuda_dev, f"decode {ctx}")
+
+
+CHUNK_CASES = [
+    # contexts, query lens, Hq, Hkv, d, block size
+    ([300, 200, 100, 50], [1, 64, 100, 3], 32, 8, 128, 16),
+    ([1000, 513], [512, 17], 32, 8, 128, 16),
+    ([129, 64], [129, 64], 16, 4, 256, 16),
+    ([90, 45], [33, 45], 8, 8, 64, 8),
+    ([600], [250], 28, 4, 128, 32),
+    ([70, 18], [70, 5], 32, 1, 128, 16),
+]
+
+
+@pytest.mark.parametrize("ctx,ql,Hq,Hkv,d,bs", CHUNK_CASES)
+def test_bf16_chunked_prefill_mixed_with_decode(cuda_dev, ctx, ql, Hq, Hkv, d, bs):
+    b = make_batch(ctx, ql, block_size=bs, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d,
+                   dtype=torch.bfloat16, seed=7 + sum(ql))
+    _check(b, Hq, Hkv, d, torch.bfloat16, cuda_dev, f"chunks {ctx}/{ql}")
+
+
+def test_permuted_block_ids_bit_identical(cuda_dev):
+    # paging must not change attention: same logical K/V under five different
+    # physical permutations gives bit-identical GPU output, equal to the oracle
+    ctx, ql, Hkv, Hq, d = [700, 90, 1500, 33], [1, 40, 1, 33], 8, 32, 128
+    g = torch.Generator().manual_seed(21)
+    k_seq = [torch.randn((c, Hkv, d), generator=g).to(torch.bfloat16) for c in ctx]
+    v_seq = [torch.randn((c, Hkv, d), generator=g).to(torch.bfloat16) for c in ctx]
+    q = torch.randn((sum(ql), Hq, d), generator=g).to(torch.bfloat16)
+    qsl = torch.tensor([0] + torch.cumsum(torch.tensor(ql), 0).tolist(), dtype=torch.int32)
+    outs = []
+    for seed in range(5):
+        kp, vp, tables = contiguous_to_paged(k_seq, v_seq, 16, seed=seed, num_blocks=200)
+        batch = {"q": q, "k_pool": kp, "v_pool": vp, "block_tables": tables,
+                 "context_lens": torch.tensor(ctx, dtype=torch.int32), "query_start_lens": qsl,
+                 "scale": 1 / math.sqrt(d), "block_size": 16}
+        got, _ = _check(batch, Hq, Hkv, d, torch.bfloat16, cuda_dev, f"perm {seed}")
+        outs.append(got.cpu())
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+
+
+def test_long_context_split_k(cuda_dev):
+    # two 8k-token sequences with head dim 256: many split-K partitions
+    b = make_batch([8192, 6000], None, block_size=16, n_q_heads=16, n_kv_heads=4, head_dim=256,
+                   dtype=torch.bfloat16, seed=33)
+    _check(b, 16, 4, 256, torch.bfloat16, cuda_dev, "long split-K")
+
+
+@pytest.mark.parametrize("name", ["decode64_bf16", "longdoc_bf16"])
+def test_full_size_workloads_sampled_rows(cuda_dev, name):
+    # the bench's workloads at full size: sampled rows against the oracle
+    b = workload_batch(name, poison_unused=False)
+    d = b["q"].shape[2]
+    Hq = b["q"].shape[1]
+    Hkv = b["k_pool"].shape[1]
+    pool = gpu_pool_from(b, Hkv, d, torch.bfloat16, cuda_dev)
+    got = run_gpu_attention(b, pool, cuda_dev).cpu()
+    rows = sample_rows(b["q"].shape[0], Hq, 48, seed=5)
+    ref = oracle.paged_attention_rows(b["q"], b["k_pool"], b["v_pool"], b["block_tables"],
+                                      b["context_lens"], b["query_start_lens"], b["scale"], rows)
+    got_rows = torch.stack([got[t, h] for t, h in rows])
+    assert_close(got_rows, ref, torch.bfloat16, name)
+    assert torch.isfinite(got).all()
+    assert pool.check_device_errors() == 0
+
+
+def test_single_token_context_returns_its_value(cuda_dev):
+    b = make_batch([1, 1, 1], None, block_size=16, n_q_heads=8, n_kv_heads=2, head_dim=128,
+                   dtype=torch.bfloat16, seed=4)
+    pool = gpu_pool_from(b, 2, 128, torch.bfloat16, cuda_dev)
+    got = run_gpu_attention(b, pool, cuda_dev).cpu()
+    for s in range(3):
+        blk = int(b["block_tables"][s, 0])
+        for h in range(8):
+            assert torch.equal(got[s, h], b["v_pool"][blk, h // 4, 0])
+
+
+@pytest.mark.parametrize("ctx,ql,bs,d", [([37, 5], [4, 5], 4, 40), ([19], [19], 1, 16)])
+def test_general_kernel_geometries(cuda_dev, ctx, ql, bs, d):
+    # block sizes and head dims outside the tensor-core tiling run the general kernel
+    b = make_batch(ctx, ql, block_size=bs, n_q_heads=4, n_kv_heads=2, head_dim=d,
+                   dtype=torch.bfloat16, seed=3)
+    _check(b, 4, 2, d, torch.bfloat16, cuda_dev, "general kernel")
+
+
+def test_general_kernel_forced_on_bf16(cuda_dev):
+    os.environ["PK_FORCE_GENERIC"] = "1"
+    try:
+        b = make_batch([300, 64], [1, 20], block_size=16, n_q_heads=32, n_kv_heads=8,
+                       head_dim=128, dtype=torch.bfloat16, seed=8)
+        _check(b, 32, 8, 128, torch.bfloat16, cuda_dev, "forced general")
+    finally:
+        del os.environ["PK_FORCE_GENERIC"]
+
+
+def test_bad_block_id_is_recorded_not_dereferenced(cuda_dev):
+    b = make_batch([40], None, block_size=16, n_q_heads=8, n_kv_heads=8, head_dim=128,
+                   dtype=torch.bfloat16, seed=2, poison_unused=False)
+    b["block_tables"][0, 1] = 10 ** 6
+    pool = gpu_pool_from(b, 8, 128, torch.bfloat16, cuda_dev)
+    run_gpu_attention(b, pool, cuda_dev)
+    assert pool.check_device_errors() == 5
