@@ -45,7 +45,8 @@ def parse():
     p.add_argument("--steps", type=int, default=2000)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="decode64_bf16", choices=["decode64_bf16", "longdoc_bf16"])
+    p.add_argument("--workload", default="decode64_bf16",
+                   choices=["decode64_bf16", "longdoc_bf16", "trace", "fork", "fork1028"])
     p.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--profile-run", action="store_true",
@@ -395,6 +396,66 @@ def run_ours(args, rank, world, device):
     print(json.dumps(line), flush=True)
 
 
+def run_serving(args, rank, world, device):
+    """Scheduler-driven workloads: the continuous-batching trace (300
+    iterations, Poisson arrivals, chunked prefill, preemption) or n-sample
+    forks with copy-on-write.  Reports tokens/s per scheduler step over the
+    GPU time of copy + append + attention, and KV GB/s."""
+    from paged_kv_cache_chunked_b200.drivers import ForkRunner, TraceRunner
+    peak, peak_kind = measured_peak()
+    kv_tok = 8 * 128 * 2 * 2          # K+V bytes per token per layer (8 kv heads, d 128, bf16)
+    recs = []
+    if args.workload == "trace":
+        r = TraceRunner(device)
+        while r.sched.step_no < 300 and (r.pending or r.sched.has_work()):
+            rec = r.step()
+            if rec is not None:
+                recs.append(rec)
+        skip = min(args.warmup, len(recs) // 2)
+        recs = recs[skip:]
+        cfg = {"workload": "trace", "steps_run": len(recs) + skip, "warmup_steps": skip,
+               "num_blocks": 8192, "block_size": 16, "n_q_heads": 32, "n_kv_heads": 8,
+               "head_dim": 128, "token_budget": 4096, "max_chunk": 512,
+               "preemptions": r.sched.metrics["preemptions"], "rejected": r.rejected,
+               "finished": len(r.sched.finished)}
+        ms = [x.gpu_ms for x in recs]
+        toks = [x.tokens for x in recs]
+        kvb = [x.context_tokens * kv_tok for x in recs]
+        copies = sum(x.copies for x in recs)
+    else:
+        plen = 1028 if args.workload == "fork1028" else 1024
+        r = ForkRunner(device, prompt_len=plen)
+        r.prefill()
+        for _ in range(min(args.warmup, 8)):
+            r.decode_step()
+        ms, toks, kvb, copies = [], [], [], 0
+        steps = min(args.steps, r.decode_steps - min(args.warmup, 8))
+        for _ in range(steps):
+            before_unique = r.unique_blocks()
+            t, c = r.decode_step()
+            ms.append(t)
+            toks.append(len(r.seqs))
+            kvb.append(before_unique * 16 * kv_tok)     # unique (physical) blocks read
+            copies += c
+        cfg = {"workload": args.workload, "prompts": 64, "prompt_len": plen, "samples": 4,
+               "block_size": 16, "n_q_heads": 32, "n_kv_heads": 8, "head_dim": 128,
+               "decode_steps_timed": steps, "unique_blocks": r.unique_blocks(),
+               "clone_blocks": r.clone_blocks(), "copies": copies}
+    tot_ms = sum(ms)
+    per_step = sorted(t / (m * 1e-3) for t, m in zip(toks, ms))
+    pct = lambda q: per_step[min(len(per_step) - 1, int(q * len(per_step)))]
+    line = {"metric": METRIC, "value": sum(toks) / (tot_ms * 1e-3), "unit": "tokens/s",
+            "n_gpus": world, "steps": len(ms), "warmup": args.warmup, "ms_per_step": tot_ms / len(ms),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": cfg,
+            "tokens_per_step_s": {"p10": pct(0.1), "p50": pct(0.5), "p90": pct(0.9)},
+            "kv_gbs": sum(kvb) / (tot_ms * 1e-3) / 1e9,
+            "pct_hbm": 100 * sum(kvb) / (tot_ms * 1e-3) / 1e9 / peak,
+            "timing": "per-step CUDA events around copy + append + attention; host scheduling excluded"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -411,7 +472,10 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                  device_id=device)
     try:
-        run_ours(args, rank, world, device)
+        if args.workload in ("trace", "fork", "fork1028"):
+            run_serving(args, rank, world, device)
+        else:
+            run_ours(args, rank, world, device)
     finally:
         if world > 1:
             import torch.distributed as tdist

@@ -1,0 +1,222 @@
+"""Drivers that run the paged-KV calls the way a serving engine does.
+
+TraceRunner   continuous batching over an arrival trace: each iteration the
+              scheduler plans a mixed batch (decodes first, then prefill
+              chunks), the kernels run copy -> append -> attention on one
+              stream, finished requests are freed ["PagedAttention &
+              Continuous Batching" (study notes), "Continuous batching" and
+              "Flow"; "Batching and PagedAttention", "Continuous batching"].
+ForkRunner    n parallel samples of each prompt: prefill, fork (children share
+              the prompt's blocks by reference count), then decode steps in
+              which the first write into a shared, partly filled tail block
+              triggers copy-on-write [study notes, "Copy-on-write";
+              "Batching and PagedAttention", "Sharing blocks"].
+
+Both generate queries and K/V with the counter-based generator of
+`workloads.token_values`, keyed by (request id, position), on the device.
+"""
+
+import torch
+
+from . import api
+from .scheduler import Request, Scheduler
+from .workloads import token_values, trace_requests
+
+
+class StepRecord:
+    __slots__ = ("step", "tokens", "decode_rows", "prefill_tokens", "copies", "gpu_ms",
+                 "context_tokens", "num_seqs")
+
+    def __init__(self, **kw):
+        for k, v in kw.items():
+            setattr(self, k, v)
+
+
+class TraceRunner:
+    """Runs the serving trace through the scheduler and the GPU kernels."""
+
+    def __init__(self, device, num_blocks=8192, block_size=16, n_q_heads=32, n_kv_heads=8,
+                 head_dim=128, token_budget=4096, max_chunk=512, trace=None, seed=1004,
+                 n_steps=300, dtype=torch.bfloat16):
+        self.device = torch.device(device)
+        self.Hq, self.Hkv, self.d, self.bs = n_q_heads, n_kv_heads, head_dim, block_size
+        self.dtype = dtype
+        self.seed = seed
+        self.n_steps = n_steps
+        self.pool = api.kv_pool_create(num_blocks, block_size, n_kv_heads, head_dim, dtype,
+                                       self.device)
+        self.bm = api.BlockManager(num_blocks, block_size)
+        self.sched = Scheduler(self.bm, token_budget, max_chunk)
+        trace = trace if trace is not None else trace_requests(n_steps=n_steps, seed=seed)
+        self.pending = [Request(i, a, p, o) for i, (a, p, o) in enumerate(trace)]
+        self.scale = head_dim ** -0.5
+        self.records = []
+        self.rejected = 0
+
+    def _admit_arrivals(self, step):
+        while self.pending and self.pending[0].arrival <= step:
+            req = self.pending.pop(0)
+            try:
+                self.sched.add_request(req)
+            except ValueError:
+                self.rejected += 1
+
+    def step(self, on_step=None, timed=True):
+        """One iteration.  on_step(plan, tensors, out) is called after the
+        kernels (for parity checks).  Returns the step's record, or None when
+        there was nothing to run."""
+        step = self.sched.step_no
+        self._admit_arrivals(step)
+        plan = self.sched.schedule()
+        if not plan.requests:
+            self.sched.complete(plan)
+            return None
+        dev = self.device
+        rids, pos = [], []
+        for req, s, n in zip(plan.requests, plan.starts, plan.counts):
+            rids.extend([req.rid] * n)
+            pos.extend(range(s, s + n))
+        meta = {
+            "slots": torch.tensor(plan.slots, dtype=torch.int64),
+            "tables": plan.tables,
+            "ctx": torch.tensor(plan.context_lens, dtype=torch.int32),
+            "qsl": torch.tensor(plan.query_start_lens(), dtype=torch.int32),
+            "pairs": torch.tensor(plan.copy_pairs, dtype=torch.int32).reshape(-1, 2),
+        }
+        d = {k: v.to(dev, non_blocking=True) for k, v in meta.items()}
+        q = token_values(self.seed, 0, rids, pos, self.Hq, self.d, self.dtype, dev)
+        k = token_values(self.seed, 1, rids, pos, self.Hkv, self.d, self.dtype, dev)
+        v = token_values(self.seed, 2, rids, pos, self.Hkv, self.d, self.dtype, dev)
+        stream = torch.cuda.current_stream(dev)
+        if timed:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        if d["pairs"].shape[0]:
+            api.block_copy(d["pairs"], pool=self.pool)
+        api.paged_kv_append(k, v, d["slots"], pool=self.pool)
+        out = api.paged_attention(q, self.pool.k_pool, self.pool.v_pool, d["tables"], d["ctx"],
+                                  d["qsl"], self.scale)
+        if timed:
+            e1.record(stream)
+        if on_step is not None:
+            on_step(plan, {"q": q, "k": k, "v": v, **meta}, out)
+        if timed:
+            e1.synchronize()
+        n_dec = sum(1 for r, s in zip(plan.requests, plan.starts) if s >= r.target)
+        rec = StepRecord(step=step, tokens=plan.num_tokens, decode_rows=n_dec,
+                         prefill_tokens=plan.num_tokens - n_dec, copies=len(plan.copy_pairs),
+                         gpu_ms=e0.elapsed_time(e1) if timed else None,
+                         context_tokens=sum(plan.context_lens), num_seqs=len(plan.requests))
+        self.sched.complete(plan)
+        self.records.append(rec)
+        return rec
+
+    def run(self, max_steps=None, on_step=None):
+        limit = max_steps if max_steps is not None else self.n_steps
+        while self.sched.step_no < limit and (self.pending or self.sched.has_work()):
+            self.step(on_step)
+        return self.records
+
+
+class ForkRunner:
+    """n parallel samples per prompt sharing the prompt's blocks (copy-on-write)."""
+
+    def __init__(self, device, n_prompts=64, prompt_len=1024, n_samples=4, block_size=16,
+                 n_q_heads=32, n_kv_heads=8, head_dim=128, decode_steps=256, seed=1005,
+                 dtype=torch.bfloat16, chunk=512):
+        self.device = torch.device(device)
+        self.Hq, self.Hkv, self.d, self.bs = n_q_heads, n_kv_heads, head_dim, block_size
+        self.dtype, self.seed, self.chunk = dtype, seed, chunk
+        self.n_prompts, self.prompt_len, self.n_samples = n_prompts, prompt_len, n_samples
+        self.decode_steps = decode_steps
+        per_seq = -(-(prompt_len + decode_steps) // block_size)
+        # shared prompt blocks + a private copy of the rest for every sample, with slack
+        self.num_blocks = n_prompts * n_samples * per_seq + 64
+        self.pool = api.kv_pool_create(self.num_blocks, block_size, n_kv_heads, head_dim, dtype,
+                                       self.device)
+        self.bm = api.BlockManager(self.num_blocks, block_size)
+        self.scale = head_dim ** -0.5
+        self.seqs = []       # (seq id, key id for the generator)
+        self.lengths = []
+        self.total_copies = 0
+
+    def _values(self, keys, pos):
+        dev = self.device
+        q = token_values(self.seed, 0, keys, pos, self.Hq, self.d, self.dtype, dev)
+        k = token_values(self.seed, 1, keys, pos, self.Hkv, self.d, self.dtype, dev)
+        v = token_values(self.seed, 2, keys, pos, self.Hkv, self.d, self.dtype, dev)
+        return q, k, v
+
+    def prefill(self):
+        """Prefill every prompt in chunks (causal), then fork n-1 children each."""
+        parents = [self.bm.add_seq() for _ in range(self.n_prompts)]
+        done = 0
+        while done < self.prompt_len:
+            n = min(self.chunk, self.prompt_len - done)
+            keys, pos, slots = [], [], []
+            for i, s in enumerate(parents):
+                sl, pairs = self.bm.append_slots(s, n)
+                assert not pairs
+                slots.extend(sl)
+                keys.extend([i * self.n_samples] * n)     # the parent's key: sample 0
+                pos.extend(range(done, done + n))
+            q, k, v = self._values(keys, pos)
+            dev = self.device
+            api.paged_kv_append(k, v, torch.tensor(slots, dtype=torch.int64, device=dev), pool=self.pool)
+            width = -(-(done + n) // self.bs)
+            tables = self.bm.fill_tables(parents, width).to(dev)
+            ctx = torch.full((len(parents),), done + n, dtype=torch.int32, device=dev)
+            qsl = torch.arange(0, (len(parents) + 1) * n, n, dtype=torch.int32, device=dev)
+            api.paged_attention(q, self.pool.k_pool, self.pool.v_pool, tables, ctx, qsl, self.scale)
+            done += n
+        for i, p in enumerate(parents):
+            self.seqs.append((p, i * self.n_samples))
+            for j in range(1, self.n_samples):
+                self.seqs.append((self.bm.fork(p), i * self.n_samples + j))
+        self.lengths = [self.prompt_len] * len(self.seqs)
+
+    def decode_step(self, on_step=None, timed=True):
+        """One decode token for every sample: copy-on-write pairs, append, attend.
+        Samples of one prompt diverge: each has its own key for new tokens."""
+        slots, pairs, keys, pos = [], [], [], []
+        for (s, key), L in zip(self.seqs, self.lengths):
+            sl, pr = self.bm.append_slots(s, 1)
+            slots.extend(sl)
+            pairs.extend(pr)
+            keys.append(key)
+            pos.append(L)
+        self.lengths = [L + 1 for L in self.lengths]
+        dev = self.device
+        q, k, v = self._values(keys, pos)
+        width = -(-max(self.lengths) // self.bs)
+        tables = self.bm.fill_tables([s for s, _ in self.seqs], width)
+        meta = {"slots": torch.tensor(slots, dtype=torch.int64), "tables": tables,
+                "ctx": torch.tensor(self.lengths, dtype=torch.int32),
+                "qsl": torch.arange(len(self.seqs) + 1, dtype=torch.int32),
+                "pairs": torch.tensor(pairs, dtype=torch.int32).reshape(-1, 2)}
+        dd = {kk: vv.to(dev, non_blocking=True) for kk, vv in meta.items()}
+        stream = torch.cuda.current_stream(dev)
+        if timed:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        if dd["pairs"].shape[0]:
+            api.block_copy(dd["pairs"], pool=self.pool)
+        api.paged_kv_append(k, v, dd["slots"], pool=self.pool)
+        out = api.paged_attention(q, self.pool.k_pool, self.pool.v_pool, dd["tables"], dd["ctx"],
+                                  dd["qsl"], self.scale)
+        if timed:
+            e1.record(stream)
+        if on_step is not None:
+            on_step({"q": q, "k": k, "v": v, **meta}, out)
+        self.total_copies += len(pairs)
+        if timed:
+            e1.synchronize()
+            return e0.elapsed_time(e1), len(pairs)
+        return None, len(pairs)
+
+    def unique_blocks(self):
+        return self.bm.num_used()
+
+    def clone_blocks(self):
+        """Blocks the same samples would hold if every fork cloned its prefix."""
+        return sum(-(-L // self.bs) for L in self.lengths)

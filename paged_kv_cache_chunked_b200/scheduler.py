@@ -1,0 +1,269 @@
+"""Iteration-level scheduler (continuous batching) driving the paged KV calls.
+
+What the pages fix:
+  * every iteration admits new work (a full prefill or one chunk of it),
+    drops finished requests and frees their blocks, and runs one mixed batch
+    of whatever remains ["PagedAttention & Continuous Batching" (study notes),
+    "Continuous batching"; "Batching and PagedAttention", "Continuous
+    batching"; "7.8 PagedAttention & continuous batching", "01 Concept"];
+  * long prompts are split into chunks so one prefill does not stall every
+    decode ["Batching and PagedAttention", "Continuous batching"];
+  * a cap on the tokens processed per step bounds the prefill work any step
+    absorbs ["Batching and PagedAttention", "Scheduling is a policy"];
+    admission reasons in blocks [deep dive, "01 Concept"];
+  * first come, first served; when blocks run out, the most recently arrived
+    requests are preempted first, all of their blocks together, and later
+    recomputed from the tokens they had ["Batching and PagedAttention",
+    "When blocks run out"].
+
+Readings where the pages give no number or order (listed in the design notes):
+  * token budget 4096 per step, prefill chunks of at most 512 tokens;
+  * decodes are scheduled first, one token each, in arrival order; then
+    prefill chunks, first come first served, while the budget lasts and the
+    chunk's blocks are free (no preemption to admit a prefill);
+  * a decode that cannot get a block preempts the latest-arrived running
+    request (possibly itself) until it fits;
+  * a preempted request goes back to the waiting queue in arrival order; its
+    recompute prefill covers its prompt and every generated token but the
+    last, which the next decode step appends;
+  * a request's K/V and queries are a deterministic function of (request id,
+    position), so recomputation reproduces the same bits.
+
+A request with prompt length P and output length O stores P + O - 1 tokens:
+the last prefill chunk yields the first output token, each decode step
+appends the previous output token and yields the next.
+"""
+
+from dataclasses import dataclass, field
+
+import torch
+
+
+@dataclass
+class Request:
+    rid: int
+    arrival: int
+    prompt_len: int
+    output_len: int
+    seq: int = -1            # block manager sequence, -1 when holding no blocks
+    stored: int = 0          # positions whose K/V is in the pool
+    target: int = 0          # positions to prefill before decoding
+    generated: int = 0       # output tokens produced
+    first_token_step: int = -1
+    admit_step: int = -1
+    finish_step: int = -1
+    preemptions: int = 0
+    token_steps: list = field(default_factory=list)
+
+    def __post_init__(self):
+        self.target = self.prompt_len
+
+    @property
+    def prefilling(self):
+        return self.stored < self.target
+
+
+@dataclass
+class StepPlan:
+    """One iteration's batch: per scheduled request, `n` new positions starting
+    at `start`; the device tensors the kernels take are built by `tensors()`."""
+    step: int
+    requests: list          # Request objects, batch order
+    starts: list            # first new position per request
+    counts: list            # new positions per request
+    slots: list             # slot id of every new position, batch order
+    copy_pairs: list        # (src, dst) copy-on-write pairs to run first
+    context_lens: list      # tokens stored per request after this step's append
+    tables: torch.Tensor    # int32 [B, W] block tables (host)
+    preempted: list         # requests preempted while planning this step
+
+    @property
+    def num_tokens(self):
+        return sum(self.counts)
+
+    def query_start_lens(self):
+        q = [0]
+        for n in self.counts:
+            q.append(q[-1] + n)
+        return q
+
+
+class Scheduler:
+    def __init__(self, bm, token_budget=4096, max_chunk=512):
+        self.bm = bm
+        self.block_size = bm.block_size
+        self.token_budget = token_budget
+        self.max_chunk = max_chunk
+        self.waiting = []    # arrival order
+        self.running = []    # arrival order; hold blocks
+        self.finished = []
+        self.step_no = 0
+        self.metrics = {"preemptions": 0, "alloc_failures": 0, "admitted": 0}
+
+    def add_request(self, req):
+        """Queue a request; one that could never fit in the whole pool is
+        rejected here, with the reason, instead of failing mid-generation."""
+        total = req.prompt_len + req.output_len - 1
+        if -(-total // self.block_size) > self.bm.num_blocks:
+            self.metrics["rejected"] = self.metrics.get("rejected", 0) + 1
+            raise ValueError(f"request {req.rid} needs {total} tokens, more than the pool holds")
+        self._requeue(req)
+
+    def _requeue(self, req):
+        self.waiting.append(req)
+        self.waiting.sort(key=lambda r: (r.arrival, r.rid))
+
+    def has_work(self):
+        return bool(self.waiting or self.running)
+
+    # -- preemption -------------------------------------------------------
+    def _preempt(self, req):
+        self.bm.free(req.seq)
+        req.seq = -1
+        req.stored = 0
+        req.target = req.prompt_len + max(req.generated - 1, 0)
+        req.preemptions += 1
+        self.metrics["preemptions"] += 1
+        self.running.remove(req)
+        self._requeue(req)
+
+    def _latest_running(self):
+        return max(self.running, key=lambda r: (r.arrival, r.rid))
+
+    # -- one iteration ------------------------------------------------------
+    def schedule(self):
+        """Plan the next step: reserve slots, emit copy pairs and tables.  If
+        requests hold blocks but none can advance (every one of them is
+        mid-prefill and the pool is full), the latest arrival is preempted
+        and the step planned again."""
+        plan = self._plan()
+        while not plan.requests and self.running:
+            victim = self._latest_running()
+            self._preempt(victim)
+            plan = self._plan()
+            plan.preempted.append(victim)
+        return plan
+
+    def _plan(self):
+        budget = self.token_budget
+        batch, starts, counts, slots, pairs, preempted = [], [], [], [], [], []
+
+        def reserve(req, n):
+            s, p = self.bm.append_slots(req.seq, n)
+            batch.append(req)
+            starts.append(req.stored)
+            counts.append(n)
+            slots.extend(s)
+            pairs.extend(p)
+
+        # decodes first, in arrival order
+        for req in sorted(self.running, key=lambda r: (r.arrival, r.rid)):
+            if req.prefilling or req not in self.running or budget == 0:
+                continue
+            while req in self.running and self.bm.blocks_needed(req.seq, 1) > self.bm.num_free():
+                victim = self._latest_running()
+                self.metrics["alloc_failures"] += 1
+                self._preempt(victim)
+                preempted.append(victim)
+            if req not in self.running:
+                continue
+            reserve(req, 1)
+            budget -= 1
+        # prefill chunks: running requests mid-prefill, then waiting ones (FCFS)
+        candidates = [r for r in sorted(self.running, key=lambda r: (r.arrival, r.rid))
+                      if r.prefilling and r not in batch]
+        candidates += [r for r in self.waiting if r not in preempted]
+        for req in candidates:
+            if budget == 0:
+                break
+            n = min(self.max_chunk, req.target - req.stored, budget)
+            if req.seq < 0:
+                # admission: reason in blocks before taking any
+                need = -(-n // self.block_size)
+                if need > self.bm.num_free():
+                    break        # FCFS: later arrivals wait behind this one
+                req.seq = self.bm.add_seq()
+                if req.admit_step < 0:
+                    req.admit_step = self.step_no
+                self.waiting.remove(req)
+                self.running.append(req)
+                self.running.sort(key=lambda r: (r.arrival, r.rid))
+                self.metrics["admitted"] += 1
+            if self.bm.blocks_needed(req.seq, n) > self.bm.num_free():
+                break
+            reserve(req, n)
+            budget -= n
+
+        seqs = [r.seq for r in batch]
+        ctx = [s + n for s, n in zip(starts, counts)]
+        width = max([-(-c // self.block_size) for c in ctx] + [1])
+        tables = self.bm.fill_tables(seqs, width) if seqs else torch.empty((0, 1), dtype=torch.int32)
+        return StepPlan(self.step_no, batch, starts, counts, slots, pairs, ctx, tables, preempted)
+
+    def complete(self, plan):
+        """Advance request state after the step's kernels ran; free finished."""
+        for req, n in zip(plan.requests, plan.counts):
+            was_prefill = req.stored < req.target
+            req.stored += n
+            if was_prefill:
+                if req.stored == req.target and req.generated == 0:
+                    req.generated = 1
+                    req.first_token_step = plan.step
+                    req.token_steps.append(plan.step)
+            else:
+                req.generated += 1
+                req.token_steps.append(plan.step)
+            if req.generated >= req.output_len and not req.prefilling:
+                req.finish_step = plan.step
+                self.bm.free(req.seq)
+                req.seq = -1
+                self.running.remove(req)
+                self.finished.append(req)
+        self.step_no += 1
+
+    def step_metrics(self):
+        s = self.bm.stats()
+        return {"free_blocks": s["free_blocks"], "used_blocks": s["used_blocks"],
+                "tail_waste_slots": s["tail_waste_slots"], "running": len(self.running),
+                "waiting": len(self.waiting), "preemptions": self.metrics["preemptions"],
+                "alloc_failures": self.metrics["alloc_failures"]}
+
+
+def summary(finished):
+    """Per-request serving metrics over finished requests, in scheduler steps
+    [7.8 PagedAttention & continuous batching, "01 Concept": queue delay, time
+    to first token, inter-token latency], split by request class (prompt
+    shorter or longer than 512 tokens) so throughput does not hide starvation."""
+    def stats(xs):
+        if not xs:
+            return None
+        xs = sorted(xs)
+        return {"mean": sum(xs) / len(xs), "p50": xs[len(xs) // 2], "p90": xs[int(0.9 * (len(xs) - 1))],
+                "max": xs[-1]}
+
+    out = {}
+    for name, sel in (("all", lambda r: True), ("short_prompt", lambda r: r.prompt_len <= 512),
+                      ("long_prompt", lambda r: r.prompt_len > 512)):
+        rs = [r for r in finished if sel(r)]
+        itl = []
+        for r in rs:
+            itl += [b - a for a, b in zip(r.token_steps, r.token_steps[1:])]
+        out[name] = {"requests": len(rs),
+                     "queue_delay": stats([r.admit_step - r.arrival for r in rs]),
+                     "ttft": stats([r.first_token_step - r.arrival for r in rs]),
+                     "itl": stats(itl),
+                     "preempted": sum(1 for r in rs if r.preemptions)}
+    return out
+
+
+def plan_inputs(plan, seed, n_q_heads, n_kv_heads, head_dim, dtype, device):
+    """q, k, v for a plan's new positions from the counter-based generator."""
+    from .workloads import token_values
+    rids, pos = [], []
+    for req, s, n in zip(plan.requests, plan.starts, plan.counts):
+        rids.extend([req.rid] * n)
+        pos.extend(range(s, s + n))
+    q = token_values(seed, 0, rids, pos, n_q_heads, head_dim, dtype, device)
+    k = token_values(seed, 1, rids, pos, n_kv_heads, head_dim, dtype, device)
+    v = token_values(seed, 2, rids, pos, n_kv_heads, head_dim, dtype, device)
+    return q, k, v

@@ -145,3 +145,56 @@ def contiguous_to_paged(k_seq, v_seq, block_size, seed, num_blocks=None):
             k_pool[blk, :, :hi - lo, :] = k_seq[b][lo:hi].transpose(0, 1)
             v_pool[blk, :, :hi - lo, :] = v_seq[b][lo:hi].transpose(0, 1)
     return k_pool, v_pool, tables
+
+
+# ---------------------------------------------------------------- trace inputs
+def _mix64(x):
+    """SplitMix64 finaliser on int64 tensors (wrapping arithmetic): a
+    counter-based generator, so a token's values depend only on its key."""
+    x = x ^ ((x >> 30) & 0x3FFFFFFFF)
+    x = x * -4658895280553007687          # 0xbf58476d1ce4e5b9 as a signed int64
+    x = x ^ ((x >> 27) & 0x1FFFFFFFFF)
+    x = x * -7723592293110705685          # 0x94d049bb133111eb as a signed int64
+    x = x ^ ((x >> 31) & 0x1FFFFFFFF)
+    return x
+
+
+def token_values(seed, stream, rids, positions, n_heads, head_dim, dtype, device="cpu"):
+    """Deterministic pseudo-normal values for (request id, position) pairs:
+    [len(positions), n_heads, head_dim].  stream separates q / k / v.
+
+    Each element is a sum of four 24-bit uniforms (Irwin-Hall), centred and
+    scaled to unit variance, computed with integer hashing and exact-order
+    float32 operations, so CPU and GPU produce the same bits.  Used so that a
+    preempted request recomputes exactly the K/V it had."""
+    rids = torch.as_tensor(rids, dtype=torch.int64, device=device).reshape(-1, 1, 1)
+    pos = torch.as_tensor(positions, dtype=torch.int64, device=device).reshape(-1, 1, 1)
+    h = torch.arange(n_heads, dtype=torch.int64, device=device).reshape(1, -1, 1)
+    e = torch.arange(head_dim, dtype=torch.int64, device=device).reshape(1, 1, -1)
+    key = (((seed * 1000003 + stream) * 1000003 + rids) * 1048576 + pos) * 4096 + h * head_dim + e
+    acc = torch.zeros(key.shape, dtype=torch.float32, device=device)
+    for j in range(4):
+        x = _mix64(key * 4 + j)
+        u = ((x >> 40) & 0xFFFFFF).to(torch.float32) * (1.0 / 16777216.0)
+        acc = acc + u
+    return ((acc - 2.0) * 1.7320508075688772).to(dtype)
+
+
+def trace_requests(n_steps=300, arrivals_per_step=4.0, prompt_median=512, prompt_sigma=1.0,
+                   prompt_max=8192, out_min=10, out_max=500, seed=1004):
+    """Continuous-batching trace: Poisson arrivals per step, lognormal prompt
+    lengths (median prompt_median, clipped to [1, prompt_max]), output lengths
+    uniform in [out_min, out_max].  Returns a list of (arrival_step, prompt_len,
+    output_len) in arrival order.  Lengths are mixed on purpose: equal lengths
+    hide what continuous batching is for ["Batching and PagedAttention",
+    "Common mistakes"]."""
+    import numpy as np
+    rng = np.random.Generator(np.random.PCG64(seed))
+    out = []
+    for step in range(n_steps):
+        for _ in range(int(rng.poisson(arrivals_per_step))):
+            p = int(round(float(rng.lognormal(math.log(prompt_median), prompt_sigma))))
+            p = min(max(p, 1), prompt_max)
+            o = int(rng.integers(out_min, out_max + 1))
+            out.append((step, p, o))
+    return out

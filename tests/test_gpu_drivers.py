@@ -1,0 +1,139 @@
+"""The serving drivers on the GPU, step by step against the oracle.
+
+TraceRunner: continuous batching with chunked prefill, preemption and
+recomputation; every step's decode rows and a sample of its prefill rows are
+compared with the float64 oracle run on a CPU mirror of the pool that the
+oracle's own append and copy keep up to date; the GPU pool itself is compared
+with the mirror bit for bit.
+
+ForkRunner: parallel samples share their prompt's blocks until a write
+["PagedAttention & Continuous Batching" (study notes), "Copy-on-write"]:
+siblings read identical K/V before the first decode, the first write into a
+shared, partly filled tail copies it (one copy per sharer but the last), and
+attention matches the oracle every step.
+"""
+
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_chunked_b200.drivers import ForkRunner, TraceRunner
+from paged_kv_cache_chunked_b200.workloads import trace_requests
+
+from helpers import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+class Mirror:
+    """CPU copy of the pool kept current with the oracle's append and copy."""
+
+    def __init__(self, pool):
+        self.k = pool.k_pool.cpu()
+        self.v = pool.v_pool.cpu()
+
+    def apply(self, pairs, k, v, slots):
+        if pairs.shape[0]:
+            oracle.block_copy(self.k, self.v, pairs)
+        oracle.kv_append(self.k, self.v, k.cpu(), v.cpu(), slots)
+
+
+def _check_rows(mirror, t, out, rows, scale, what):
+    ref = oracle.paged_attention_rows(t["q"].cpu(), mirror.k, mirror.v, t["tables"], t["ctx"],
+                                      t["qsl"], scale, rows)
+    got = torch.stack([out[r, h].cpu() for r, h in rows])
+    assert_close(got, ref, torch.bfloat16, what)
+
+
+def test_trace_steps_match_the_oracle(cuda_dev):
+    trace = trace_requests(n_steps=30, arrivals_per_step=3.0, prompt_median=256, prompt_max=1500,
+                           out_min=5, out_max=40, seed=17)
+    runner = TraceRunner(cuda_dev, num_blocks=700, n_steps=30, trace=trace, token_budget=1024,
+                         max_chunk=256)
+    mirror = Mirror(runner.pool)
+    gen = torch.Generator().manual_seed(0)
+
+    def on_step(plan, t, out):
+        mirror.apply(t["pairs"], t["k"], t["v"], t["slots"])
+        rows = []
+        qsl = t["qsl"].tolist()
+        for i, (req, s) in enumerate(zip(plan.requests, plan.starts)):
+            toks = list(range(qsl[i], qsl[i + 1]))
+            if s >= req.target:                       # decode row: every head
+                rows += [(toks[0], h) for h in range(runner.Hq)]
+            else:                                     # chunk: first, last and a random row
+                pick = {toks[0], toks[-1], toks[int(torch.randint(len(toks), (1,), generator=gen))]}
+                rows += [(tk, int(torch.randint(runner.Hq, (1,), generator=gen))) for tk in pick]
+        _check_rows(mirror, t, out, rows, runner.scale, f"trace step {plan.step}")
+        if plan.step % 10 == 0:
+            torch.cuda.synchronize()
+            assert torch.equal(runner.pool.k_pool.cpu(), mirror.k)
+            assert torch.equal(runner.pool.v_pool.cpu(), mirror.v)
+
+    runner.run(max_steps=60, on_step=on_step)
+    assert runner.sched.metrics["preemptions"] > 0     # the small pool forces recomputation
+    assert runner.pool.check_device_errors() == 0
+
+
+def test_recompute_reproduces_the_same_kv(cuda_dev):
+    # a request preempted and re-prefilled holds bit-identical K/V afterwards
+    trace = [(0, 40, 30), (0, 40, 30), (1, 40, 30)]
+    runner = TraceRunner(cuda_dev, num_blocks=9, block_size=16, n_steps=200, trace=trace,
+                         token_budget=256, max_chunk=64)
+
+    def logical_kv(req):
+        table = runner.bm.block_table(req.seq)
+        k = runner.pool.k_pool[table].transpose(1, 2).reshape(-1, runner.Hkv, runner.d)
+        return k[:req.stored].cpu()
+
+    before = {}
+    for _ in range(200):
+        for r in list(runner.sched.running):
+            if not r.prefilling:
+                before.setdefault(r.rid, {})[r.stored] = logical_kv(r)
+        if runner.step() is None and not runner.sched.has_work() and not runner.pending:
+            break
+        for r in list(runner.sched.running):
+            if r.preemptions and not r.prefilling and r.stored in before.get(r.rid, {}):
+                assert torch.equal(logical_kv(r), before[r.rid][r.stored])
+                r.checked = True
+    assert runner.sched.metrics["preemptions"] > 0
+    assert any(getattr(r, "checked", False) for r in runner.sched.finished + runner.sched.running)
+
+
+@pytest.mark.parametrize("prompt_len,bs,copies_per_prompt", [(100, 16, 3), (96, 16, 0), (37, 8, 3),
+                                                              (64, 32, 0)])
+def test_fork_copy_on_write(cuda_dev, prompt_len, bs, copies_per_prompt):
+    n_prompts, n_samples = 4, 4
+    runner = ForkRunner(cuda_dev, n_prompts=n_prompts, prompt_len=prompt_len,
+                        n_samples=n_samples, block_size=bs, decode_steps=6)
+    runner.prefill()
+    torch.cuda.synchronize()
+    shared = runner.unique_blocks()
+    assert shared == n_prompts * -(-prompt_len // bs)       # prompt blocks stored once
+    # siblings read identical K/V through identical tables before any write
+    for i in range(n_prompts):
+        tabs = [runner.bm.block_table(runner.seqs[i * n_samples + j][0]) for j in range(n_samples)]
+        assert all(t == tabs[0] for t in tabs)
+    mirror = Mirror(runner.pool)
+    copies = []
+
+    def on_step(t, out):
+        mirror.apply(t["pairs"], t["k"], t["v"], t["slots"])
+        rows = [(b, h) for b in range(len(runner.seqs)) for h in (0, runner.Hq - 1)]
+        _check_rows(mirror, t, out, rows, runner.scale, "fork decode")
+        copies.append(t["pairs"].shape[0])
+
+    for _ in range(runner.decode_steps):
+        runner.decode_step(on_step)
+    assert copies[0] == n_prompts * copies_per_prompt and sum(copies[1:]) == 0
+    # after diverging, siblings differ only in the blocks written since the fork
+    for i in range(n_prompts):
+        tabs = [runner.bm.block_table(runner.seqs[i * n_samples + j][0]) for j in range(n_samples)]
+        n_full = prompt_len // bs
+        assert all(t[:n_full] == tabs[0][:n_full] for t in tabs)
+        assert len({tuple(t[n_full:]) for t in tabs}) == n_samples
+    assert runner.unique_blocks() < runner.clone_blocks()
+    torch.cuda.synchronize()
+    assert torch.equal(runner.pool.k_pool.cpu(), mirror.k)
+    assert runner.pool.check_device_errors() == 0
