@@ -462,6 +462,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_consta
         if (ok && mbar_wait(&empty[stage], phase ^ 1)) {
             meta[stage] = make_int4(-1, 0, 0, 0);
             mbar_arrive(&full[stage]);
+            // the end marker completes a phase of this stage's barrier too
+            armed |= 1u << stage;
+            armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
         } else {
             record_error(prm.err, PK_ERR_TIMEOUT);
             *abort_flag = 1;
@@ -740,9 +743,13 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_consta
             break;
         }
         const int4 mt = meta[stage];
+        if (mt.x < 0) {  // end marker: no more stages from this CTA's producer
+            if (cur >= 0) finish_item();
+            break;
+        }
         if (mt.x != cur) {
             if (cur >= 0) finish_item();
-            if (!ok || mt.x < 0) break;
+            if (!ok) break;
             begin_item(mt.x);
             cur = mt.x;
         }
