@@ -158,6 +158,33 @@ int pk_paged_attention(const pk_pool *pool, const void *q, void *out,
                        void *workspace, size_t workspace_bytes, pk_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Paged attention without a caller workspace.  The pages have no
+ * counterpart to this call; it exists for callers that cannot allocate
+ * device memory, such as a C host program with no caching allocator, or a
+ * serving loop that has reserved all free HBM for the KV pool, where a
+ * cudaMalloc on the request path would fail or stall the device.
+ *
+ * Same arguments and results as pk_paged_attention, minus the workspace: the
+ * scratch comes from a fixed array of PK_NOALLOC_SCRATCH_BYTES in the
+ * library's own device memory, which every GPU that loads the library holds
+ * until the process exits.  The call allocates nothing (no cudaMalloc,
+ * cudaFree or allocating library routine).  A batch whose scratch need
+ * (pk_attention_workspace_size) exceeds the array is refused with
+ * PK_ERR_WORKSPACE before anything is launched.  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture.  All calls
+ * share the array: calls whose work overlaps on the GPU (two streams, two
+ * host threads) race and corrupt each other's results, so serialise them.
+ * ------------------------------------------------------------------------ */
+#define PK_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+int pk_paged_attention_noalloc(const pk_pool *pool, const void *q, void *out,
+                               const int32_t *block_tables, int max_blocks_per_seq,
+                               const int32_t *context_lens, const int32_t *query_start_lens,
+                               int num_seqs, int num_tokens, int n_q_heads, float scale,
+                               pk_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Host block manager  [SN "Block tables", "Copy-on-write"; BP
  * "PagedAttention", "Sharing blocks", "When blocks run out"; DD]
  *

@@ -52,6 +52,7 @@ SIGNATURES = {
     "pk_block_copy": ([_P, _P, _I, _P], _I),
     "pk_attention_workspace_size": ([_P, _I, _I, _I, _I, _PSZ], _I),
     "pk_paged_attention": ([_P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _F, _P, _SZ, _P], _I),
+    "pk_paged_attention_noalloc": ([_P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _F, _P], _I),
     "pk_bm_create": ([_I, _I, _PP], _I),
     "pk_bm_destroy": ([_P], _I),
     "pk_bm_add_seq": ([_P, _PI64], _I),
