@@ -46,7 +46,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="decode64_bf16",
-                   choices=["decode64_bf16", "longdoc_bf16", "trace", "fork", "fork1028"])
+                   choices=["decode64_bf16", "longdoc_bf16", "chunk512_bf16", "trace", "fork",
+                            "fork1028"])
     p.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--profile-run", action="store_true",
@@ -70,12 +71,29 @@ def step_bytes(batch):
 
 
 def last_token_slots(batch):
+    """Slots of every sequence's query tokens (its last q_b positions)."""
     bs = batch["block_size"]
     ctx = batch["context_lens"].to(torch.int64)
+    qsl = batch["query_start_lens"].to(torch.int64)
     tables = batch["block_tables"].to(torch.int64)
-    pos = ctx - 1
-    blk = tables.gather(1, (pos // bs)[:, None])[:, 0]
-    return blk * bs + pos % bs
+    slots = []
+    for b in range(ctx.shape[0]):
+        qn = int(qsl[b + 1] - qsl[b])
+        pos = torch.arange(int(ctx[b]) - qn, int(ctx[b]))
+        slots.append(tables[b, pos // bs] * bs + pos % bs)
+    return torch.cat(slots)
+
+
+def attention_flops(batch):
+    """4 * Hq * d per visible (query row, key) pair (QK^T and PV, 2 flops per MAC)."""
+    T, Hq, d = batch["q"].shape
+    ctx = batch["context_lens"].to(torch.int64).tolist()
+    qsl = batch["query_start_lens"].to(torch.int64).tolist()
+    keys = 0
+    for b, c in enumerate(ctx):
+        qn = qsl[b + 1] - qsl[b]
+        keys += qn * (c - qn) + qn * (qn + 1) // 2
+    return 4 * Hq * d * keys
 
 
 def new_token_kv(batch, slots):
@@ -235,6 +253,32 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback"
+
+
+def roofline_entry(workload, attn_b, flops, avg_ms, gbs, tflops, hbm_peak, hbm_kind):
+    """The attention call's roofline: HBM for decode (about 4 flop/byte at GQA 4),
+    the tensor pipe for prefill chunks (a dense contraction)."""
+    common = {"kernel": "paged_attention call (one attention_tc launch per 512 sequences)",
+              "algorithmic_bytes": attn_b, "algorithmic_flops": flops, "avg_ms": avg_ms,
+              "traffic": kernel_traffic(workload)}
+    if workload == "chunk512_bf16":
+        peak, kind = measured_tensor_peak()
+        return dict(common, bound="tensor", achieved=tflops, peak=peak, unit="TFLOP/s",
+                    frac=tflops / peak,
+                    peak_source=f"{kind} (MEASURED_PEAKS.json bf16_tflops, burst)")
+    return dict(common, bound="hbm", achieved=gbs, peak=hbm_peak, unit="GB/s",
+                frac=gbs / hbm_peak,
+                peak_source=f"{hbm_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                if hbm_kind == "measured" else "fallback 6.65 TB/s")
+
+
 def workload_config(name, batch, l2_note):
     w = WORKLOADS[name]
     ctx = batch["context_lens"]
@@ -275,7 +319,9 @@ def run_ours(args, rank, world, device):
         if ev is not None:
             ev[1].record(stream)
 
-    launches_per_step = 1 + (3 if pool.dtype == torch.bfloat16 and d in (64, 128, 256) and bs % 8 == 0 else 1)
+    # append + one attention kernel per window of 512 sequences (the general kernel: one launch)
+    tc = pool.dtype == torch.bfloat16 and d in (64, 128, 256) and bs % 8 == 0
+    launches_per_step = 1 + ((T + 511) // 512 if tc else 1)
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize(device)
@@ -367,6 +413,8 @@ def run_ours(args, rank, world, device):
     peak, peak_kind = measured_peak()
     attn_avg_ms = statistics.mean(attn_ms)
     achieved = attn_b / (attn_avg_ms * 1e-3) / 1e9
+    flops = attention_flops(batch)
+    tflops = flops / (attn_avg_ms * 1e-3) / 1e12
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -376,12 +424,9 @@ def run_ours(args, rank, world, device):
                                   f"more than the 126 MB L2"),
         "pct_hbm": 100.0 * value / world / peak,
         "tokens_per_s": world * T / (ms_per_step * 1e-3),
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": kernel_traffic(args.workload),
-                     "kernel": "paged_attention call (plan + attention_tc + reduce)",
-                     "algorithmic_bytes": attn_b, "avg_ms": attn_avg_ms,
-                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
-                     if peak_kind == "measured" else "fallback 6.65 TB/s"},
+        "roofline": roofline_entry(args.workload, attn_b, flops, attn_avg_ms, achieved, tflops,
+                                   peak, peak_kind),
+        "attention_tflops": tflops,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": dict(clk, window="the timed region plus 1 s of the same steps right after it"),
     }

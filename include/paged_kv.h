@@ -145,8 +145,12 @@ int pk_block_copy(const pk_pool *pool, const int32_t *src_dst_pairs, int n_pairs
  *   [num_seqs + 1], query_start_lens[0] = 0, 1 <= q_b <= c_b.
  * n_q_heads % n_kv_heads == 0.
  * workspace: device scratch of at least pk_attention_workspace_size bytes,
- *   16-byte aligned, owned by the caller, not shared by calls in flight at the
- *   same time; it holds the work list and the split-K partial results.
+ *   256-byte aligned, owned by the caller, not shared by calls in flight at
+ *   the same time; it holds the work-claim counter, the split-K arrival
+ *   counters and the split-K partial results.  It must be zero-filled before
+ *   its first use; every call that completes leaves the counters zeroed
+ *   again, so a workspace can be reused across calls, batches and pools.
+ *   After a call that recorded PK_ERR_TIMEOUT, zero it again.
  * ------------------------------------------------------------------------ */
 int pk_attention_workspace_size(const pk_pool *pool, int num_seqs, int num_tokens,
                                 int n_q_heads, int max_blocks_per_seq, size_t *bytes_out);
@@ -173,8 +177,10 @@ int pk_paged_attention(const pk_pool *pool, const void *q, void *out,
  * PK_ERR_WORKSPACE before anything is launched.  The first call on a device
  * looks up the array's device address (cudaGetSymbolAddress) with that
  * device current; make that first call before any stream capture.  All calls
- * share the array: calls whose work overlaps on the GPU (two streams, two
- * host threads) race and corrupt each other's results, so serialise them.
+ * share the array, which starts zeroed and which every completed call leaves
+ * with its counters zeroed: calls whose work overlaps on the GPU (two
+ * streams, two host threads) race and corrupt each other's results, so
+ * serialise them.
  * ------------------------------------------------------------------------ */
 #define PK_NOALLOC_SCRATCH_BYTES (32u << 20)
 

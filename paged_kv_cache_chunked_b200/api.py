@@ -98,7 +98,8 @@ class KVPool:
         check(lib().pk_attention_workspace_size(self.handle, num_seqs, num_tokens, n_q_heads,
                                                 max_blocks, ctypes.byref(n)))
         if self._workspace is None or self._workspace.numel() < n.value:
-            self._workspace = torch.empty(max(n.value, 256), dtype=torch.uint8, device=self.device)
+            # zero-filled once; every call leaves its counters zeroed again
+            self._workspace = torch.zeros(max(n.value, 256), dtype=torch.uint8, device=self.device)
         return self._workspace
 
     def check_device_errors(self):

@@ -1,8 +1,9 @@
 // pk_paged_attention_noalloc: paged attention for callers that cannot
 // allocate device memory.
 //
-// pk_paged_attention takes its scratch (the work list and the split-K partial
-// results) from a caller-provided workspace.  Some callers cannot provide
+// pk_paged_attention takes its scratch (the work-claim counter, the split-K
+// arrival counters and the split-K partial results) from a caller-provided
+// workspace.  Some callers cannot provide
 // one: a plain C host program with no caching allocator, or a serving loop
 // that reserves all free HBM for the KV pool up front, where a cudaMalloc on
 // the request path would fail or stall the whole device.  This entry point
@@ -18,12 +19,13 @@
 // that device current, and caches it; make that first call before any stream
 // capture.
 //
-// All calls share the array and it keeps the last call's contents.  Each call
-// rewrites everything it reads before reading it (the planner kernel writes
-// the work counts and resets the work counter at the start of every call), so
-// no state carries over; but two calls whose work overlaps on the GPU (on two
-// streams, or from two host threads) race on the array and corrupt each
-// other's results.  Serialise them.
+// All calls share the array and it keeps the last call's contents.  The only
+// state a call relies on at its start is the work-claim counter and the
+// split-K arrival counters, which must be zero: the array starts zeroed (a
+// __device__ variable is zero-initialised) and every completed call leaves
+// them zeroed; everything else is written before it is read.  Two calls whose
+// work overlaps on the GPU (on two streams, or from two host threads) race on
+// the array and corrupt each other's results.  Serialise them.
 #include <mutex>
 
 #include "pk_internal.h"

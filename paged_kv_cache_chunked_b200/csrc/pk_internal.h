@@ -38,7 +38,6 @@ __device__ __forceinline__ void record_error(int *err, int code) {
 
 constexpr int kMaxHeadDim = 256;
 constexpr int kTile = 16;        // tokens per KV tile and rows per query tile
-constexpr int kConsumers = 4;    // consumer warps of the tensor-core attention kernel
 
 // ---- launchers (each returns PK_OK or an error code) ---------------------
 int launch_kv_append(const pk_pool *p, const void *k, const void *v, const int64_t *slots,

@@ -13,6 +13,8 @@ Workloads (sizes as the spec configurations name them):
                  32 q / 8 kv heads, head dim 128, pool 1.25x the blocks needed
   longdoc_bf16   8 decode sequences of 32,768 tokens, block 16, 16 q / 4 kv
                  heads, head dim 256, pool 1.25x
+  chunk512_bf16  16 sequences at context 4096 whose last 512 tokens are this
+                 step's prefill chunk (causal), 32 q / 8 kv heads, head dim 128
 """
 
 import math
@@ -28,6 +30,10 @@ WORKLOADS = {
                           seed=1002),
     "longdoc_bf16": dict(context_lens=[32768] * 8, block_size=16, n_q_heads=16, n_kv_heads=4,
                          head_dim=256, dtype=torch.bfloat16, pool_factor=1.25, seed=1003),
+    # the last 512-token chunk of sixteen 4096-token prompts (chunked prefill)
+    "chunk512_bf16": dict(context_lens=[4096] * 16, query_lens=[512] * 16, block_size=16,
+                          n_q_heads=32, n_kv_heads=8, head_dim=128, dtype=torch.bfloat16,
+                          pool_factor=1.25, seed=1006),
 }
 
 
@@ -118,7 +124,8 @@ def workload_batch(name, device="cpu", poison_unused=True):
         ctx = decode_context_lens(w.pop("num_seqs"), lo, hi, seed)
     else:
         ctx = w.pop("context_lens")
-    return make_batch(ctx, None, seed=seed, device=device, poison_unused=poison_unused, **w)
+    ql = w.pop("query_lens", None)
+    return make_batch(ctx, ql, seed=seed, device=device, poison_unused=poison_unused, **w)
 
 
 def contiguous_to_paged(k_seq, v_seq, block_size, seed, num_blocks=None):

@@ -48,7 +48,7 @@ def _check_rows(mirror, t, out, rows, scale, what):
 def test_trace_steps_match_the_oracle(cuda_dev):
     trace = trace_requests(n_steps=30, arrivals_per_step=3.0, prompt_median=256, prompt_max=1500,
                            out_min=5, out_max=40, seed=17)
-    runner = TraceRunner(cuda_dev, num_blocks=700, n_steps=30, trace=trace, token_budget=1024,
+    runner = TraceRunner(cuda_dev, num_blocks=300, n_steps=30, trace=trace, token_budget=1024,
                          max_chunk=256)
     mirror = Mirror(runner.pool)
     gen = torch.Generator().manual_seed(0)

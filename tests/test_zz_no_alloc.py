@@ -63,11 +63,12 @@ def test_noalloc_refuses_batches_beyond_its_scratch(cuda_dev):
                    dtype=torch.bfloat16, seed=43, poison_unused=False)
     pool = gpu_pool_from(b, 8, 128, torch.bfloat16, cuda_dev)
     need = ctypes.c_size_t()
-    huge_tokens = 1 << 20                     # a million query tokens: far past 32 MiB
-    lib().pk_attention_workspace_size(pool.handle, 1, huge_tokens, 32, 4, ctypes.byref(need))
+    # 512 sequences with 16 q heads per kv head: split-K scratch past 32 MiB
+    n_seqs, n_q_heads = 512, 128
+    lib().pk_attention_workspace_size(pool.handle, n_seqs, n_seqs, n_q_heads, 4, ctypes.byref(need))
     assert need.value > 32 << 20
     dummy = ctypes.c_void_p(pool.k_pool.data_ptr())
-    rc = lib().pk_paged_attention_noalloc(pool.handle, dummy, dummy, dummy, 4, dummy, dummy, 1,
-                                          huge_tokens, 32, ctypes.c_float(1.0), None)
+    rc = lib().pk_paged_attention_noalloc(pool.handle, dummy, dummy, dummy, 4, dummy, dummy, n_seqs,
+                                          n_seqs, n_q_heads, ctypes.c_float(1.0), None)
     assert rc == 6                             # PK_ERR_WORKSPACE, nothing launched
     assert b"scratch" in lib().pk_last_error()
