@@ -36,7 +36,7 @@ from paged_kv_cache_chunked_b200.workloads import WORKLOADS, workload_batch  # n
 
 METRIC = "paged decode attention KV GB/s (% of HBM peak) and tokens/s per scheduler step"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SRC = os.path.join(ROOT, "paged_kv_cache_chunked_b200", "csrc", "attention_tc.cu")
+KERNEL_SRC = os.path.join(ROOT, "paged_kv_cache_chunked_b200", "csrc", "attention_decode.cu")
 
 
 def parse():
@@ -265,7 +265,7 @@ def measured_tensor_peak():
 def roofline_entry(workload, attn_b, flops, avg_ms, gbs, tflops, hbm_peak, hbm_kind):
     """The attention call's roofline: HBM for decode (about 4 flop/byte at GQA 4),
     the tensor pipe for prefill chunks (a dense contraction)."""
-    common = {"kernel": "paged_attention call (one attention_tc launch per 512 sequences)",
+    common = {"kernel": "paged_attention call (decode kernel; chunk kernel when chunks are present)",
               "algorithmic_bytes": attn_b, "algorithmic_flops": flops, "avg_ms": avg_ms,
               "traffic": kernel_traffic(workload)}
     if workload == "chunk512_bf16":
@@ -319,9 +319,12 @@ def run_ours(args, rank, world, device):
         if ev is not None:
             ev[1].record(stream)
 
-    # append + one attention kernel per window of 512 sequences (the general kernel: one launch)
+    # append + one decode kernel per window of 512 sequences, plus the chunk
+    # kernel when the step holds prefill chunks (the general kernel: one launch)
     tc = pool.dtype == torch.bfloat16 and d in (64, 128, 256) and bs % 8 == 0
-    launches_per_step = 1 + ((T + 511) // 512 if tc else 1)
+    B = batch["context_lens"].shape[0]
+    windows = (B + 511) // 512
+    launches_per_step = 1 + ((windows * (2 if T > B else 1)) if tc else 1)
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize(device)

@@ -1,0 +1,85 @@
+// Host side of the tensor-core attention path: workspace layout and the
+// dispatch of a call to the chunk kernel (sequences whose query rows need more
+// than one 16-row tile) and the decode kernel (all others).
+#include <algorithm>
+
+#include "pk_internal.h"
+
+namespace pk {
+namespace {
+
+constexpr size_t kHeaderBytes = 256;     // one scheduler header per kernel
+constexpr int kMaxSeqsPerLaunch = 512;   // window of sequences per kernel launch
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace: decode header | chunk header | split-K counters (fixed size) |
+// partial log2-sum-exp | partial O.  The headers and counters sit at offsets
+// that do not depend on the batch, so the zeros every call leaves there stay
+// valid when the next call's batch differs.
+struct Layout {
+    size_t hdr_decode, hdr_chunk, counters, partial_lse, partial_o, total;
+    int cap_rows;
+};
+
+Layout layout(const pk_pool *p, int num_seqs, int n_q_heads) {
+    Layout L{};
+    const int Hkv = p->n_kv_heads, D = p->head_dim;
+    const int g = std::max(1, n_q_heads / Hkv);
+    // split items: at most Hkv per sequence plus the ~items_per_cta per CTA that
+    // split-K adds; a decode item has g partial rows (the planner coarsens the
+    // partitions when a batch of short chunks needs more)
+    const long long items = (long long)Hkv * std::min(num_seqs, kMaxSeqsPerLaunch) +
+                            (long long)p->tc_ctas * decode_items_per_cta();
+    L.cap_rows = (int)std::min<long long>(items * std::min(g, kTile), 1LL << 30);
+    L.hdr_decode = 0;
+    L.hdr_chunk = kHeaderBytes;
+    size_t off = 2 * kHeaderBytes;
+    L.counters = off;
+    off = align_up(off + (size_t)kMaxSeqsPerLaunch * Hkv * sizeof(int), 256);
+    L.partial_lse = off;
+    off = align_up(off + (size_t)L.cap_rows * sizeof(float), 256);
+    L.partial_o = off;
+    off = align_up(off + (size_t)L.cap_rows * D * sizeof(float), 256);
+    L.total = off;
+    return L;
+}
+
+}  // namespace
+
+size_t tc_workspace_bytes(const pk_pool *p, int num_seqs, int num_tokens, int n_q_heads,
+                          int /*max_blocks_per_seq*/) {
+    (void)num_tokens;
+    return layout(p, num_seqs, n_q_heads).total;
+}
+
+int tc_prepare_pool(pk_pool *p) {
+    int rc = decode_prepare_pool(p);
+    if (rc == PK_OK) rc = chunk_prepare_pool(p);
+    return rc;
+}
+
+int launch_attention_tc(const pk_pool *p, const AttnArgs &a, cudaStream_t st) {
+    const Layout L = layout(p, a.num_seqs, a.n_q_heads);
+    if (a.workspace_bytes < L.total || a.workspace == nullptr)
+        return fail(PK_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", a.workspace_bytes, L.total);
+    if (((uintptr_t)a.workspace & 255) != 0)
+        return fail(PK_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    uint8_t *ws = (uint8_t *)a.workspace;
+    // the chunk kernel has work only if some sequence's rows (q_b tokens x g
+    // heads) exceed one 16-row tile: a chunk of several tokens, or g > 16
+    const int g = a.n_q_heads / p->n_kv_heads;
+    if (a.num_tokens > a.num_seqs || g > kTile) {
+        const int rc = launch_chunk(p, a, ws + L.hdr_chunk, st);
+        if (rc != PK_OK) return rc;
+    }
+    DecodeWs w;
+    w.header = ws + L.hdr_decode;
+    w.counters = (int *)(ws + L.counters);
+    w.partial_lse = (float *)(ws + L.partial_lse);
+    w.partial_o = (float *)(ws + L.partial_o);
+    w.cap_rows = L.cap_rows;
+    return launch_decode(p, a, w, st);
+}
+
+}  // namespace pk

@@ -19,8 +19,9 @@ struct pk_pool {
     int *d_err;       // device error word (first recorded PK_ERR_* code)
     int device;
     int sm_count;
-    bool tc_path;     // tensor-core + TMA attention applies to this geometry
-    int tc_ctas;      // resident CTAs of the tensor-core attention kernel (whole GPU)
+    bool tc_path;       // tensor-core + TMA attention applies to this geometry
+    int tc_ctas;        // resident CTAs of the decode attention kernel (whole GPU)
+    int tc_ctas_chunk;  // resident CTAs of the chunk attention kernel (whole GPU)
     alignas(64) CUtensorMap tmap_k;
     alignas(64) CUtensorMap tmap_v;
 };
@@ -64,7 +65,20 @@ int launch_attention_generic(const pk_pool *p, const AttnArgs &a, cudaStream_t s
 // Tensor-core path: workspace sizing and launch.
 size_t tc_workspace_bytes(const pk_pool *p, int num_seqs, int num_tokens, int n_q_heads,
                           int max_blocks_per_seq);
-int tc_prepare_pool(pk_pool *p);  // occupancy query, once per pool
+int tc_prepare_pool(pk_pool *p);  // occupancy queries, once per pool
 int launch_attention_tc(const pk_pool *p, const AttnArgs &a, cudaStream_t st);
+
+// The decode kernel's share of the workspace.
+struct DecodeWs {
+    void *header;
+    int *counters;
+    float *partial_o, *partial_lse;
+    int cap_rows;
+};
+int decode_prepare_pool(pk_pool *p);
+int decode_items_per_cta();
+int launch_decode(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, cudaStream_t st);
+int chunk_prepare_pool(pk_pool *p);
+int launch_chunk(const pk_pool *p, const AttnArgs &a, void *header, cudaStream_t st);
 
 }  // namespace pk
