@@ -33,14 +33,18 @@ constexpr int kFirst = 1, kLast = 2;
 
 template <int D>
 struct ChunkCfg;
+// One CTA per SM with 7 consumer warps: each KV tile that the producer warp
+// loads feeds 7 row tiles (112 query rows), so one issuing warp per SM (about
+// 14 GB/s of tile loads) keeps the tensor pipe busier than 2 CTAs of 3.
+// Eight warps keep 255 registers per thread available.
 template <>
 struct ChunkCfg<64> {
-    static constexpr int kStages = 16, kMinBlocks = 2, kConsumers = 3;
+    static constexpr int kStages = 24, kMinBlocks = 1, kConsumers = 7;
     static constexpr bool kQReg = true;
 };
 template <>
 struct ChunkCfg<128> {
-    static constexpr int kStages = 11, kMinBlocks = 2, kConsumers = 3;
+    static constexpr int kStages = 20, kMinBlocks = 1, kConsumers = 7;
     static constexpr bool kQReg = true;
 };
 template <>

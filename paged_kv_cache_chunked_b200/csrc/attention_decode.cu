@@ -95,7 +95,11 @@ struct DecParams {
     int *err;
 };
 
-template <int D>
+// T8: every item is one decode token of a group of at most 8 q heads.  The
+// heads then sit on the N = 8 side of the MMA (S^T = K Q^T, O^T = V^T P^T):
+// half the MMAs and half the accumulator registers of the 16-row layout,
+// with P^T moved into B-fragment order by movmatrix.
+template <int D, bool T8>
 __global__ void __launch_bounds__(dec_threads<D>(), DecCfg<D>::kMinBlocks)
 attention_decode_kernel(const __grid_constant__ CUtensorMap tmk,
                         const __grid_constant__ CUtensorMap tmv, const DecParams prm) {
@@ -151,8 +155,11 @@ attention_decode_kernel(const __grid_constant__ CUtensorMap tmk,
     const int nseq = prm.nseq, bs = prm.block_size, box = prm.box_rows;
 
     // ------------------------------------------------------------ producer side
-    // claims run one item ahead; the claimed item's table chunk is loaded
-    // when it is claimed, so both latencies hide behind the current item
+    // An item is staged (claimed, its Q rows bulk-copied, its descriptor and
+    // first table chunk taken) as soon as one of the warp's kQSlots Q slots is
+    // free, i.e. a whole item ahead of its use; its KV tiles are issued
+    // kStages ahead of the consumer in stream order.  The next claim is always
+    // in flight, so the atomic's latency hides too.
     auto claim = [&]() -> int {
         int v = 0;
         if (lane == 0) v = atomicAdd(&prm.hdr->next_item, 1);
@@ -163,18 +170,14 @@ attention_decode_kernel(const __grid_constant__ CUtensorMap tmk,
         const int e = blk_base + lane;
         return e < nblk ? __ldg(prm.tables + (long long)(prm.seq0 + b) * prm.max_blocks + e) : 0;
     };
-    int ready_idx = __shfl_sync(0xffffffffu, claim(), 0);
-    int ready_tab = 0;
-    if (ready_idx < n_items) {
-        const SplitItem r = decode_split(pa, nseq, g, Hkv, ready_idx);
-        ready_tab = chunk_entry(r.b, (r.kv_begin * kTile / bs) & ~31);
-    }
     int pending = claim();
-
-    bool ok = true, exhausted = ready_idx >= n_items;
-    int n_iss = 0, n_con = 0, n_staged = 0, n_begun = 0;
-    uint32_t qph = 0;  // parity bit per Q slot (consumer side)
-    // producer's current item
+    bool ok = true, exhausted = false;
+    int n_iss = 0, n_con = 0, n_staged = 0, n_begun = 0, n_started = 0;
+    uint32_t qph = 0;        // parity bit per Q slot (consumer side)
+    int tab_s0 = 0, tab_s1 = 0;  // each staged item's first table chunk (this lane's entry);
+                                 // loaded straight into the slot's register so the load
+                                 // stays in flight until the item starts
+    // producer cursor
     bool p_active = false;
     int p_b = 0, p_kvh = 0, p_kt = 0, p_ke = 0, p_c = 0;
     int cur_base = 0, cur_tab = 0, nxt_tab = 0;
@@ -192,22 +195,18 @@ attention_decode_kernel(const __grid_constant__ CUtensorMap tmk,
         }
         return phys;
     };
-    // take the next claimed item: stage its Q rows and descriptor
-    auto next_item = [&]() -> bool {
-        if (exhausted || n_staged - n_begun >= QS) return false;
-        const int idx = ready_idx;
-        const int tab = ready_tab;
-        ready_idx = __shfl_sync(0xffffffffu, pending, 0);
-        pending = claim();
-        if (ready_idx < n_items) {
-            const SplitItem r = decode_split(pa, nseq, g, Hkv, ready_idx);
-            ready_tab = chunk_entry(r.b, (r.kv_begin * kTile / bs) & ~31);
-        } else {
+    auto stage_next = [&]() {
+        const int idx = __shfl_sync(0xffffffffu, pending, 0);
+        if (idx >= n_items) {
             exhausted = true;
+            return;
         }
+        pending = claim();
         const SplitItem it = decode_split(pa, nseq, g, Hkv, idx);
         const int slot = n_staged % QS;
         const int qs0 = pa.s_qsl[it.b], qn = pa.s_qsl[it.b + 1] - qs0;
+        if (slot == 0) tab_s0 = chunk_entry(it.b, (it.kv_begin * kTile / bs) & ~31);
+        else tab_s1 = chunk_entry(it.b, (it.kv_begin * kTile / bs) & ~31);
         if (lane == 0) {
             Desc &d = descs[slot];
             d.seq = prm.seq0 + it.b;
@@ -232,16 +231,20 @@ attention_decode_kernel(const __grid_constant__ CUtensorMap tmk,
                       prm.q + ((long long)(qs0 + lane) * Hq + it.kvh * g) * D, (uint32_t)g * D * 2,
                       &qfull[slot]);
         ++n_staged;
+    };
+    auto start_item = [&]() {
+        const int slot = n_started % QS;
+        const Desc &d = descs[slot];
+        p_b = d.seq - prm.seq0;
+        p_kvh = d.kvh;
+        p_kt = d.kv_begin;
+        p_ke = d.kv_end;
+        p_c = d.c;
+        cur_base = (p_kt * kTile / bs) & ~31;
+        cur_tab = slot == 0 ? tab_s0 : tab_s1;
+        nxt_tab = chunk_entry(p_b, cur_base + 32);
         p_active = true;
-        p_b = it.b;
-        p_kvh = it.kvh;
-        p_kt = it.kv_begin;
-        p_ke = it.kv_end;
-        p_c = pa.s_ctx[it.b];
-        cur_base = (it.kv_begin * kTile / bs) & ~31;
-        cur_tab = tab;
-        nxt_tab = chunk_entry(it.b, cur_base + 32);
-        return true;
+        ++n_started;
     };
     auto issue_tile = [&]() {
         const int stage = n_iss % S;
@@ -270,9 +273,12 @@ attention_decode_kernel(const __grid_constant__ CUtensorMap tmk,
         if (++p_kt == p_ke) p_active = false;
     };
     auto refill = [&]() {
-        fence_proxy_async();  // stages / Q slots read since the last refill are rewritten below
+        while (!exhausted && n_staged - n_begun < QS) stage_next();
         while (n_iss - n_con < S) {
-            if (!p_active && !next_item()) break;
+            if (!p_active) {
+                if (n_started == n_staged) break;
+                start_item();
+            }
             issue_tile();
         }
     };
@@ -287,9 +293,13 @@ attention_decode_kernel(const __grid_constant__ CUtensorMap tmk,
     int c = 0, lim0 = 0, lim1 = 0, d_seq = 0, d_kvh = 0, d_nparts = 1, d_row = 0, d_base = 0,
         d_pstride = 0, d_qs0 = 0, d_rows = 0;
     long long orow0 = -1, orow1 = -1;
-    uint32_t qf[C::kQReg ? KS : 1][4];
-    float o[D / 8][4];
+    uint32_t qf[(C::kQReg && !T8) ? KS : 1][4];
+    float o[T8 ? 1 : D / 8][4];
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    // T8 state: Q^T as B fragments, O^T accumulators (16 d-rows x 8 heads per
+    // m-tile), running max / sum for heads qc and qc + 1
+    uint32_t qb[T8 ? KS : 1][2];
+    float ot[T8 ? KS : 1][4];
 
     auto begin_item = [&]() {
         const int slot = n_begun % QS;
@@ -317,7 +327,18 @@ attention_decode_kernel(const __grid_constant__ CUtensorMap tmk,
         orow0 = r0 < rows ? (long long)(d_qs0 + r0 / g) * Hq + d_kvh * g + r0 % g : -1;
         orow1 = r1 < rows ? (long long)(d_qs0 + r1 / g) * Hq + d_kvh * g + r1 % g : -1;
         const uint8_t *qs = qbuf + (size_t)slot * 32 * D;
-        if constexpr (C::kQReg) {
+        if constexpr (T8) {
+            const int h = lane >> 2;  // the B fragment's n index: head of the group
+            const uint8_t *qh = qs + h * D * 2;
+#pragma unroll
+            for (int kk = 0; kk < KS; ++kk) {
+                const int col = (kk * 16 + qc) * 2;
+                qb[kk][0] = h < rows ? *(const uint32_t *)(qh + col) : 0u;
+                qb[kk][1] = h < rows ? *(const uint32_t *)(qh + col + 16) : 0u;
+            }
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) ot[mt][0] = ot[mt][1] = ot[mt][2] = ot[mt][3] = 0.f;
+        } else if constexpr (C::kQReg) {
             const uint8_t *q0 = qs + qr * D * 2, *q1 = qs + (qr + 8) * D * 2;
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
@@ -351,9 +372,59 @@ attention_decode_kernel(const __grid_constant__ CUtensorMap tmk,
                 const int row = valid + ch / (D / 8), col = (ch % (D / 8)) * 8;
                 *(uint4 *)(vs + swz(row, col)) = make_uint4(0, 0, 0, 0);
             }
+            fence_proxy_async();  // the stage is rewritten by TMA later
             __syncwarp();
         }
         const uint32_t ka = smem_u32(ks), va = smem_u32(vs), qa = smem_u32(qpriv);
+        if constexpr (T8) {
+            // S^T (16 tokens x 8 heads): A = K rows, B = Q^T
+            float st[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < KS; ++kk) {
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(ka + swz(q_row, kk * 16 + q_col), a0, a1, a2, a3);
+                mma_bf16(st, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+            }
+            // st[0], st[1]: token qr, heads qc, qc + 1; st[2], st[3]: token qr + 8
+            const int tok0 = kt * kTile + qr;
+            float s0 = st[0] * prm.scale_log2, s1 = st[1] * prm.scale_log2;
+            float s2 = st[2] * prm.scale_log2, s3 = st[3] * prm.scale_log2;
+            if (tok0 >= c) s0 = s1 = -INFINITY;
+            if (tok0 + 8 >= c) s2 = s3 = -INFINITY;
+            float ma = fmaxf(s0, s2), mb = fmaxf(s1, s3);
+#pragma unroll
+            for (int x = 4; x < 32; x <<= 1) {
+                ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, x));
+                mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, x));
+            }
+            const float na = fmaxf(m0, ma), nb = fmaxf(m1, mb);
+            const float ba = na == -INFINITY ? 0.f : na, bb = nb == -INFINITY ? 0.f : nb;
+            const float ala = fast_exp2(m0 - ba), alb = fast_exp2(m1 - bb);
+            m0 = na;
+            m1 = nb;
+            const float p0 = fast_exp2(s0 - ba), p1 = fast_exp2(s1 - bb);
+            const float p2 = fast_exp2(s2 - ba), p3 = fast_exp2(s3 - bb);
+            l0 = l0 * ala + p0 + p2;
+            l1 = l1 * alb + p1 + p3;
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                ot[mt][0] *= ala;
+                ot[mt][1] *= alb;
+                ot[mt][2] *= ala;
+                ot[mt][3] *= alb;
+            }
+            // P^T as the B fragment: transpose the two 8x8 (token x head) blocks
+            const uint32_t b0 = movmatrix_trans(pack_bf16(p0, p1));
+            const uint32_t b1 = movmatrix_trans(pack_bf16(p2, p3));
+            // O^T (16 d-rows x 8 heads per m-tile) += V^T P^T
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_t(va + swz(k_row, mt * 16 + k_col), a0, a1, a2, a3);
+                mma_bf16(ot[mt], a0, a1, a2, a3, b0, b1);
+            }
+            return;
+        }
         float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
@@ -426,6 +497,53 @@ attention_decode_kernel(const __grid_constant__ CUtensorMap tmk,
     };
 
     auto finish_item = [&]() {
+        if constexpr (T8) {
+            // sums over the 16 token lanes of each head
+#pragma unroll
+            for (int x = 4; x < 32; x <<= 1) {
+                l0 += __shfl_xor_sync(0xffffffffu, l0, x);
+                l1 += __shfl_xor_sync(0xffffffffu, l1, x);
+            }
+            const float ia = l0 > 0.f ? 1.f / l0 : 0.f, ib = l1 > 0.f ? 1.f / l1 : 0.f;
+            const int ha = qc, hb = qc + 1;  // heads of this lane's accumulators
+            const bool va_ = ha < d_rows, vb_ = hb < d_rows;
+            if (d_nparts <= 1) {
+                __nv_bfloat16 *oa = prm.out + ((long long)d_qs0 * Hq + d_kvh * g + ha) * D;
+                __nv_bfloat16 *ob = oa + D;
+#pragma unroll
+                for (int mt = 0; mt < KS; ++mt) {
+                    const int d0 = mt * 16 + qr;
+                    if (va_) {
+                        oa[d0] = __float2bfloat16_rn(ot[mt][0] * ia);
+                        oa[d0 + 8] = __float2bfloat16_rn(ot[mt][2] * ia);
+                    }
+                    if (vb_) {
+                        ob[d0] = __float2bfloat16_rn(ot[mt][1] * ib);
+                        ob[d0 + 8] = __float2bfloat16_rn(ot[mt][3] * ib);
+                    }
+                }
+                return;
+            }
+            float *pa_ = prm.partial_o + (size_t)(d_row + ha) * D;
+            float *pb_ = pa_ + D;
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                const int d0 = mt * 16 + qr;
+                if (va_) {
+                    pa_[d0] = ot[mt][0] * ia;
+                    pa_[d0 + 8] = ot[mt][2] * ia;
+                }
+                if (vb_) {
+                    pb_[d0] = ot[mt][1] * ib;
+                    pb_[d0 + 8] = ot[mt][3] * ib;
+                }
+            }
+            if (qr == 0) {
+                float *pl = prm.partial_lse + (size_t)d_row;
+                if (va_) pl[ha] = l0 > 0.f ? m0 + __log2f(l0) : -INFINITY;
+                if (vb_) pl[hb] = l1 > 0.f ? m1 + __log2f(l1) : -INFINITY;
+            }
+        } else {
         l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
         l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
         l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
@@ -461,6 +579,7 @@ attention_decode_kernel(const __grid_constant__ CUtensorMap tmk,
             if (orow0 >= 0) pl[qr] = l0 > 0.f ? m0 + __log2f(l0) : -INFINITY;
             if (orow1 >= 0) pl[qr + 8] = l1 > 0.f ? m1 + __log2f(l1) : -INFINITY;
         }
+        }  // 16-row layout
         __threadfence();
         __syncwarp();
         int prev = 0;
@@ -468,33 +587,69 @@ attention_decode_kernel(const __grid_constant__ CUtensorMap tmk,
         if (lane == 0) prev = atomicAdd(cnt, 1);
         prev = __shfl_sync(0xffffffffu, prev, 0);
         if (prev != d_nparts - 1) return;
-        // last partition of (sequence, kv head): merge all partitions into the output
+        // last partition of (sequence, kv head): merge all partitions into the output,
+        // out = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M).  Rows go four at a
+        // time and loads are issued for all four rows (and two partitions) at
+        // once so their latencies overlap.
         __threadfence();
         const int nrows = min(kTile, d_rows);
-        for (int idx = lane; idx < nrows * (D / 4); idx += 32) {
-            const int row = idx / (D / 4), c4 = idx % (D / 4);
-            float M = -INFINITY;
-            for (int p = 0; p < d_nparts; ++p)
-                M = fmaxf(M, __ldcg(prm.partial_lse + (size_t)(d_base + p * d_pstride) + row));
-            float den = 0.f;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int p = 0; p < d_nparts; ++p) {
-                const size_t pr = (size_t)(d_base + p * d_pstride) + row;
-                const float lse = __ldcg(prm.partial_lse + pr);
-                const float wgt = lse == -INFINITY ? 0.f : fast_exp2(lse - M);
-                const float4 x = __ldcg((const float4 *)(prm.partial_o + pr * D) + c4);
-                den += wgt;
-                acc.x += wgt * x.x;
-                acc.y += wgt * x.y;
-                acc.z += wgt * x.z;
-                acc.w += wgt * x.w;
+        constexpr int RG = 4;
+        for (int r0 = 0; r0 < nrows; r0 += RG) {
+            float Mr[RG], den[RG];
+#pragma unroll
+            for (int r = 0; r < RG; ++r) {
+                float mx = -INFINITY;
+                if (r0 + r < nrows)
+                    for (int p = lane; p < d_nparts; p += 32)
+                        mx = fmaxf(mx, __ldcg(prm.partial_lse + (size_t)(d_base + p * d_pstride) + r0 + r));
+#pragma unroll
+                for (int o_ = 16; o_ > 0; o_ >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o_));
+                Mr[r] = mx;
             }
-            const float inv = den > 0.f ? 1.f / den : 0.f;
-            const long long orow = (long long)(d_qs0 + row / g) * Hq + d_kvh * g + row % g;
-            uint2 pk;
-            pk.x = pack_bf16(acc.x * inv, acc.y * inv);
-            pk.y = pack_bf16(acc.z * inv, acc.w * inv);
-            *(uint2 *)(prm.out + orow * D + c4 * 4) = pk;
+#pragma unroll
+            for (int r = 0; r < RG; ++r) {
+                float sm_ = 0.f;
+                if (r0 + r < nrows)
+                    for (int p = lane; p < d_nparts; p += 32) {
+                        const float lse = __ldcg(prm.partial_lse + (size_t)(d_base + p * d_pstride) + r0 + r);
+                        sm_ += lse == -INFINITY ? 0.f : fast_exp2(lse - Mr[r]);
+                    }
+#pragma unroll
+                for (int o_ = 16; o_ > 0; o_ >>= 1) sm_ += __shfl_xor_sync(0xffffffffu, sm_, o_);
+                den[r] = sm_ > 0.f ? 1.f / sm_ : 0.f;
+            }
+            for (int c4 = lane; c4 < D / 4; c4 += 32) {
+                float4 acc[RG];
+#pragma unroll
+                for (int r = 0; r < RG; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+                for (int p = 0; p < d_nparts; ++p) {
+                    const size_t prow = (size_t)(d_base + p * d_pstride) + r0;
+#pragma unroll
+                    for (int r = 0; r < RG; ++r) {
+                        if (r0 + r < nrows) {
+                            const float lse = __ldcg(prm.partial_lse + prow + r);
+                            const float wgt = lse == -INFINITY ? 0.f : fast_exp2(lse - Mr[r]);
+                            const float4 x = __ldcg((const float4 *)(prm.partial_o + (prow + r) * D) + c4);
+                            acc[r].x += wgt * x.x;
+                            acc[r].y += wgt * x.y;
+                            acc[r].z += wgt * x.z;
+                            acc[r].w += wgt * x.w;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < RG; ++r) {
+                    if (r0 + r < nrows) {
+                        const int row = r0 + r;
+                        const long long orow = (long long)(d_qs0 + row / g) * Hq + d_kvh * g + row % g;
+                        uint2 pk;
+                        pk.x = pack_bf16(acc[r].x * den[r], acc[r].y * den[r]);
+                        pk.y = pack_bf16(acc[r].z * den[r], acc[r].w * den[r]);
+                        *(uint2 *)(prm.out + orow * D + c4 * 4) = pk;
+                    }
+                }
+            }
         }
         if (lane == 0) *cnt = 0;  // leave the counter zeroed for the next call
     };
@@ -505,6 +660,7 @@ attention_decode_kernel(const __grid_constant__ CUtensorMap tmk,
         if (c_kt >= c_ke) {
             begin_item();
             if (!ok) break;
+            refill();  // stage the item after next now that a Q slot is free
         }
         const int stage = n_con % S;
         if (!mbar_wait(&full[stage], (uint32_t)(n_con / S) & 1)) {
@@ -538,16 +694,25 @@ int dec_threads_of(int D) {
     }
 }
 
-template <int D>
-static int dec_prepare(pk_pool *p) {
+template <int D, bool T8>
+static int dec_prepare_one(int *per_sm) {
     const int smem = (int)DecSmem<D>::kBytes;
-    cudaError_t e = cudaFuncSetAttribute(attention_decode_kernel<D>,
+    cudaError_t e = cudaFuncSetAttribute(attention_decode_kernel<D, T8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "set decode attention smem size");
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attention_decode_kernel<D>,
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, attention_decode_kernel<D, T8>,
                                                       dec_threads<D>(), smem);
     if (e != cudaSuccess) return cuda_fail(e, "decode attention occupancy");
+    return PK_OK;
+}
+
+template <int D>
+static int dec_prepare(pk_pool *p) {
+    int a = 0, b = 0;
+    int rc = dec_prepare_one<D, false>(&a);
+    if (rc == PK_OK) rc = dec_prepare_one<D, true>(&b);
+    if (rc != PK_OK) return rc;
+    const int per_sm = std::min(a, b);
     if (per_sm < 1) return fail(PK_ERR_UNSUPPORTED, "decode attention kernel does not fit on an SM");
     p->tc_ctas = per_sm * p->sm_count;
     return PK_OK;
@@ -588,11 +753,19 @@ static int dec_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, cu
     tp.partial_o = w.partial_o;
     tp.partial_lse = w.partial_lse;
     tp.err = p->d_err;
+    // every query token its sequence's only one and a group of <= 8 heads: the
+    // decode-specialised layout; anything else (short chunks, larger groups) the
+    // 16-row layout
+    const bool t8 = a.num_tokens == a.num_seqs && tp.group <= 8;
     for (int s0 = 0; s0 < a.num_seqs; s0 += kMaxSeqsPerLaunch) {
         tp.seq0 = s0;
         tp.nseq = std::min(kMaxSeqsPerLaunch, a.num_seqs - s0);
-        attention_decode_kernel<D><<<p->tc_ctas, dec_threads<D>(), DecSmem<D>::kBytes, st>>>(
-            p->tmap_k, p->tmap_v, tp);
+        if (t8)
+            attention_decode_kernel<D, true><<<p->tc_ctas, dec_threads<D>(), DecSmem<D>::kBytes, st>>>(
+                p->tmap_k, p->tmap_v, tp);
+        else
+            attention_decode_kernel<D, false><<<p->tc_ctas, dec_threads<D>(), DecSmem<D>::kBytes, st>>>(
+                p->tmap_k, p->tmap_v, tp);
     }
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? PK_OK : cuda_fail(e, "decode attention launch");
