@@ -48,6 +48,13 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+bool force_generic() {
+    const char *e = getenv("PK_FORCE_GENERIC");
+    return e && e[0] == '1';
+}
+
+}  // namespace
+
 // 2-D view of a pool: rows = num_blocks * n_kv_heads * block_size token rows of
 // head_dim bf16 each; box = 64 columns (128 bytes, the swizzle span) x box_rows.
 int encode_pool_map(CUtensorMap *map, void *base, const pk_pool *p, int box_rows) {
@@ -65,12 +72,6 @@ int encode_pool_map(CUtensorMap *map, void *base, const pk_pool *p, int box_rows
     return PK_OK;
 }
 
-bool force_generic() {
-    const char *e = getenv("PK_FORCE_GENERIC");
-    return e && e[0] == '1';
-}
-
-}  // namespace
 }  // namespace pk
 
 using namespace pk;

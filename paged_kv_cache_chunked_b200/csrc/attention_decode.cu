@@ -587,70 +587,10 @@ attention_decode_kernel(const __grid_constant__ CUtensorMap tmk,
         if (lane == 0) prev = atomicAdd(cnt, 1);
         prev = __shfl_sync(0xffffffffu, prev, 0);
         if (prev != d_nparts - 1) return;
-        // last partition of (sequence, kv head): merge all partitions into the output,
-        // out = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M).  Rows go four at a
-        // time and loads are issued for all four rows (and two partitions) at
-        // once so their latencies overlap.
+        // last partition of (sequence, kv head): merge all partitions into the output
         __threadfence();
-        const int nrows = min(kTile, d_rows);
-        constexpr int RG = 4;
-        for (int r0 = 0; r0 < nrows; r0 += RG) {
-            float Mr[RG], den[RG];
-#pragma unroll
-            for (int r = 0; r < RG; ++r) {
-                float mx = -INFINITY;
-                if (r0 + r < nrows)
-                    for (int p = lane; p < d_nparts; p += 32)
-                        mx = fmaxf(mx, __ldcg(prm.partial_lse + (size_t)(d_base + p * d_pstride) + r0 + r));
-#pragma unroll
-                for (int o_ = 16; o_ > 0; o_ >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o_));
-                Mr[r] = mx;
-            }
-#pragma unroll
-            for (int r = 0; r < RG; ++r) {
-                float sm_ = 0.f;
-                if (r0 + r < nrows)
-                    for (int p = lane; p < d_nparts; p += 32) {
-                        const float lse = __ldcg(prm.partial_lse + (size_t)(d_base + p * d_pstride) + r0 + r);
-                        sm_ += lse == -INFINITY ? 0.f : fast_exp2(lse - Mr[r]);
-                    }
-#pragma unroll
-                for (int o_ = 16; o_ > 0; o_ >>= 1) sm_ += __shfl_xor_sync(0xffffffffu, sm_, o_);
-                den[r] = sm_ > 0.f ? 1.f / sm_ : 0.f;
-            }
-            for (int c4 = lane; c4 < D / 4; c4 += 32) {
-                float4 acc[RG];
-#pragma unroll
-                for (int r = 0; r < RG; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 2
-                for (int p = 0; p < d_nparts; ++p) {
-                    const size_t prow = (size_t)(d_base + p * d_pstride) + r0;
-#pragma unroll
-                    for (int r = 0; r < RG; ++r) {
-                        if (r0 + r < nrows) {
-                            const float lse = __ldcg(prm.partial_lse + prow + r);
-                            const float wgt = lse == -INFINITY ? 0.f : fast_exp2(lse - Mr[r]);
-                            const float4 x = __ldcg((const float4 *)(prm.partial_o + (prow + r) * D) + c4);
-                            acc[r].x += wgt * x.x;
-                            acc[r].y += wgt * x.y;
-                            acc[r].z += wgt * x.z;
-                            acc[r].w += wgt * x.w;
-                        }
-                    }
-                }
-#pragma unroll
-                for (int r = 0; r < RG; ++r) {
-                    if (r0 + r < nrows) {
-                        const int row = r0 + r;
-                        const long long orow = (long long)(d_qs0 + row / g) * Hq + d_kvh * g + row % g;
-                        uint2 pk;
-                        pk.x = pack_bf16(acc[r].x * den[r], acc[r].y * den[r]);
-                        pk.y = pack_bf16(acc[r].z * den[r], acc[r].w * den[r]);
-                        *(uint2 *)(prm.out + orow * D + c4 * 4) = pk;
-                    }
-                }
-            }
-        }
+        merge_partials<D>(prm.partial_o, prm.partial_lse, d_base, d_pstride, d_nparts, 0,
+                          min(kTile, d_rows), prm.out, d_qs0, Hq, d_kvh, g, lane);
         if (lane == 0) *cnt = 0;  // leave the counter zeroed for the next call
     };
 

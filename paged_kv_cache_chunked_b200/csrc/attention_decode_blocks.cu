@@ -1,0 +1,799 @@
+// Paged decode attention for bf16 pools (head_dim 64/128/256) when every
+// sequence of the batch has exactly one query token and a kv head serves at
+// most 8 q heads: the decode step of continuous batching.
+//
+// What is computed ["PagedAttention & Continuous Batching" (study notes),
+// "Block tables"; "Batching and PagedAttention", "PagedAttention" item 4]:
+// for the query token of sequence b (position c_b - 1) and q head h, softmax
+// attention over keys 0..c_b - 1 of kv head h / g, key j read from physical
+// block table_b[j / bs] at slot j % bs.
+//
+// Structure.  Decode attention reads each cached K and V byte once and does
+// four flops per byte: it is bound by HBM.  A pool block holds the K (or V)
+// rows of all kv heads contiguously ([block][kv head][slot][d]), so a block
+// of HS heads is one run of HS * bs rows.  The kernel streams whole blocks:
+//   - one producer warp per CTA claims chunks of work, looks the blocks up in
+//     the block tables and loads each block's K and V rows for HS heads with
+//     128-row TMA boxes (128-byte swizzle) into a ring of NS shared-memory
+//     stages, a stage being NBS blocks (ST = NBS * bs tokens, up to 64 KiB);
+//     a few large copies per block keep HBM busy from one issuing warp;
+//   - eight consumer warps own one kv head each (or, for HS < 8, one of
+//     8 / HS phases of a head, taking every (8 / HS)-th 16-token tile of a
+//     stage).  Per tile: S^T = K Q^T (16 tokens x the head's <= 8 q heads) and
+//     O^T += V^T P^T on mma.sync m16n8k16 (bf16 in, fp32 accumulate), with P^T
+//     moved into operand order by movmatrix, and an online softmax in fp32.
+// Work split (flash-decoding-style split-K, balanced like stream-K): the
+// stages of all (sequence, head group) pairs are concatenated and cut into
+// chunks of CS stages, about kChunksPerCta per CTA; CTAs claim chunks from a
+// global counter.  The part of a pair inside one chunk is a partition; a pair
+// cut into several partitions writes (normalised O, log2-sum-exp) rows per
+// partition, and a second kernel, launched as a programmatic dependent of the
+// first, merges them with the whole GPU (no fence, atomic or wait in the
+// streaming kernel).
+//
+// Every wait is bounded (2 s); on expiry the kernel records PK_ERR_TIMEOUT,
+// waits (bounded) for its own copies in flight and returns.  Block ids are
+// range-checked before use.
+#include "tc_common.cuh"
+
+#include <algorithm>
+
+namespace pk {
+namespace {
+
+using namespace tc;
+
+constexpr int kNC = 8;                        // consumer warps
+constexpr int kBlkThreads = (kNC + 1) * 32;   // + one producer warp
+constexpr int kStageCap = 64 * 1024;          // K + V bytes of one stage
+constexpr int kChunksPerCta = 2;              // work chunks per CTA (dynamic claiming)
+constexpr int kMinChunkStages = 4;            // smallest chunk
+constexpr int kItemSlots = 2;                 // items staged ahead (Q rows + descriptor each)
+constexpr int kMergePlanHead = 8;             // merge plan: cs, total, then stage_pre, prow_pre
+
+enum : int { kFirst = 1, kLast = 2, kEnd = 4 };
+
+struct StageInfo {
+    int slot, st, flags, pad;
+};
+struct ItemDesc {
+    int b, hg, c, qs0, nparts, part, prow, pad;
+};
+
+struct BlkParams {
+    const __nv_bfloat16 *q;
+    __nv_bfloat16 *out;
+    const int32_t *tables, *ctx, *qsl;
+    int seq0, nseq, max_blocks, n_q_heads, n_kv_heads, group, block_size, num_blocks, num_tokens;
+    int HS, NBS, ST, NPH, NS;  // geometry: heads / blocks / tokens per stage, phases, stages
+    int ncta, cap_rows;
+    float scale_log2;
+    WsHeader *hdr;
+    int *mplan;                      // the plan, for the merge kernel
+    float *partial_o, *partial_lse;  // [row][D], [row]
+    int *err;
+    // shared-memory layout (byte offsets from the 1024-aligned base)
+    uint32_t stage_bytes, qslot_bytes, off_q, off_scr, off_plan, off_desc, off_info, off_bar, total;
+};
+
+// Shared-memory layout of one launch.
+template <int D>
+void blk_layout(BlkParams &p) {
+    constexpr int KS = D / 16;
+    auto up = [](uint32_t x, uint32_t a) { return (x + a - 1) / a * a; };
+    p.stage_bytes = (uint32_t)p.NBS * p.HS * p.block_size * D * 4;
+    p.qslot_bytes = up((uint32_t)p.HS * p.group * D * 2, 128);
+    uint32_t off = (uint32_t)p.NS * p.stage_bytes;
+    p.off_q = off;
+    off += kItemSlots * p.qslot_bytes;
+    p.off_scr = off;
+    if (p.NPH > 1) off += (uint32_t)(kNC - p.HS) * 32 * (KS * 4 + 4) * 4;
+    p.off_plan = off;
+    off += up(4 * kPlanLen * 4, 16);
+    p.off_desc = off;
+    off += kItemSlots * sizeof(ItemDesc);
+    p.off_info = off;
+    off += (uint32_t)p.NS * sizeof(StageInfo);
+    p.off_bar = up(off, 8);
+    off = p.off_bar + (uint32_t)(2 * p.NS + 2 * kItemSlots + 1) * 8;
+    p.total = off + 1024;  // + alignment slack
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBlkThreads, 1)
+attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
+                               const __grid_constant__ CUtensorMap tmv, const BlkParams prm) {
+    constexpr int KS = D / 16;
+    constexpr int NPN = D / 64;  // 64-column panels
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int NS = prm.NS, HS = prm.HS, NBS = prm.NBS, ST = prm.ST, NPH = prm.NPH;
+    const int g = prm.group, Hq = prm.n_q_heads, Hkv = prm.n_kv_heads, bs = prm.block_size;
+    const int NHG = Hkv / HS, nseq = prm.nseq;
+    const int PR = HS * bs;                                  // rows of a block's head group
+    const uint32_t panel_bytes = (uint32_t)PR * 128;         // one 64-column panel of a block
+    const uint32_t piece_bytes = panel_bytes * NPN;          // a block's K (or V) rows
+    int *stage_pre = (int *)(sm + prm.off_plan);  // stages of sequences 0..i-1 (all head groups)
+    int *prow_pre = stage_pre + kPlanLen;         // split-K partial rows of sequences 0..i-1
+    int *s_qsl = prow_pre + kPlanLen;
+    int *s_ctx = s_qsl + kPlanLen;
+    ItemDesc *descs = (ItemDesc *)(sm + prm.off_desc);
+    StageInfo *infos = (StageInfo *)(sm + prm.off_info);
+    uint64_t *full = (uint64_t *)(sm + prm.off_bar);
+    uint64_t *empty = full + NS;
+    uint64_t *qfull = empty + NS;
+    uint64_t *iempty = qfull + kItemSlots;
+    uint64_t *cbar = iempty + kItemSlots;  // barrier of the consumer warps
+    __shared__ int s_total, s_cs;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kNC);
+        }
+        for (int s = 0; s < kItemSlots; ++s) {
+            mbar_init(&qfull[s], 1);
+            mbar_init(&iempty[s], kNC);
+        }
+        mbar_init(cbar, kNC);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    // ---------------------------------------------------------------- plan
+    // per sequence: S_b = ceil(c_b / ST) stages per head group; chunk size CS;
+    // a (sequence, head group) spanning several chunks has one partition per
+    // chunk, each with HS * g partial rows
+    auto parts_of = [&](int start, int sb, int cs) { return (start + sb - 1) / cs - start / cs + 1; };
+    if (warp == 0) {
+        prefetch_tmap(&tmk);
+        prefetch_tmap(&tmv);
+        int run = 0;
+        for (int base = 0; base < nseq; base += 32) {
+            const int i = base + lane;
+            int ns = 0;
+            if (i < nseq) {
+                const int b = prm.seq0 + i;
+                const int s0 = __ldg(prm.qsl + b), s1 = __ldg(prm.qsl + b + 1), c = __ldg(prm.ctx + b);
+                s_qsl[i] = s0;
+                s_ctx[i] = c;
+                if (i == nseq - 1) s_qsl[nseq] = s1;
+                const bool ok = s0 >= 0 && s1 <= prm.num_tokens && s1 - s0 == 1 && c >= 1 &&
+                                (long long)(c + bs - 1) / bs <= prm.max_blocks;
+                if (!ok) record_error(prm.err, PK_ERR_BAD_INDEX);
+                else ns = NHG * ((c + ST - 1) / ST);
+            }
+            int inc = ns;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += y;
+            }
+            if (i < nseq) stage_pre[i + 1] = run + inc;
+            run += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (lane == 0) stage_pre[0] = 0;
+        __syncwarp();
+        const int total = run;
+        const long long want = (long long)prm.ncta * kChunksPerCta;
+        int cs = (int)std::max<long long>(kMinChunkStages, (total + want - 1) / want);
+        for (int attempt = 0; attempt < 8; ++attempt) {
+            int runp = 0;
+            for (int base = 0; base < nseq; base += 32) {
+                const int i = base + lane;
+                int np = 0;
+                if (i < nseq) {
+                    const int sb = (stage_pre[i + 1] - stage_pre[i]) / NHG;
+                    for (int hg = 0; hg < NHG && sb > 0; ++hg) {
+                        const int n = parts_of(stage_pre[i] + hg * sb, sb, cs);
+                        if (n > 1) np += n * HS * g;
+                    }
+                }
+                int inc = np;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, inc, o);
+                    if (lane >= o) inc += y;
+                }
+                if (i < nseq) prow_pre[i + 1] = runp + inc;
+                runp += __shfl_sync(0xffffffffu, inc, 31);
+            }
+            if (runp <= prm.cap_rows) break;
+            // more partial rows than the workspace holds: coarser chunks, finally
+            // one chunk for everything (no split)
+            cs = attempt < 6 ? 2 * cs : std::max(total, 1);
+        }
+        if (lane == 0) {
+            prow_pre[0] = 0;
+            s_total = total;
+            s_cs = cs;
+        }
+        __syncwarp();
+        if (blockIdx.x == 0) {  // the merge kernel's copy of the plan
+            if (lane == 0) {
+                prm.mplan[0] = cs;
+                prm.mplan[1] = total;
+            }
+            for (int i = lane; i <= nseq; i += 32) {
+                prm.mplan[kMergePlanHead + i] = stage_pre[i];
+                prm.mplan[kMergePlanHead + kPlanLen + i] = prow_pre[i];
+            }
+        }
+    }
+    // the merge kernel may be scheduled now; it waits for this grid to finish
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    __syncthreads();
+    const int total = s_total, cs = s_cs;
+    bool ok = true;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- producer
+        const int nchunks = (total + cs - 1) / cs;
+        auto claim = [&]() -> int {
+            int v = 0;
+            if (lane == 0) v = atomicAdd(&prm.hdr->next_item, 1);
+            return v;
+        };
+        int pending = claim();
+        int n_stage = 0, n_item = 0;
+        int cur_base = 0, cur_tab = 0, nxt_tab = 0, t_b = 0;
+        auto chunk_entry = [&](int b, int blk_base) -> int {
+            const int nblk = (s_ctx[b] + bs - 1) / bs;
+            const int e = blk_base + lane;
+            return e < nblk ? __ldg(prm.tables + (long long)(prm.seq0 + b) * prm.max_blocks + e) : 0;
+        };
+        auto table_get = [&](int blk) -> int {
+            while (blk >= cur_base + 32) {
+                cur_base += 32;
+                cur_tab = nxt_tab;
+                nxt_tab = chunk_entry(t_b, cur_base + 32);
+            }
+            int phys = __shfl_sync(0xffffffffu, cur_tab, blk - cur_base);
+            if (phys < 0 || phys >= prm.num_blocks) {
+                if (lane == 0) record_error(prm.err, PK_ERR_BAD_INDEX);
+                phys = 0;
+            }
+            return phys;
+        };
+        while (ok) {
+            const int chunk = __shfl_sync(0xffffffffu, pending, 0);
+            if (chunk >= nchunks) break;
+            pending = claim();
+            int g0 = chunk * cs;
+            const int g1 = min(total, g0 + cs);
+            while (ok && g0 < g1) {
+                // the partition of one (sequence, head group) inside this chunk
+                const int b = find_seq(stage_pre, nseq, g0);
+                const int sb = (stage_pre[b + 1] - stage_pre[b]) / NHG;
+                const int local = g0 - stage_pre[b];
+                const int hg = local / sb, st0 = local - hg * sb;
+                const int cnt = min(sb - st0, g1 - g0);
+                const int start = stage_pre[b] + hg * sb;
+                const int nparts = parts_of(start, sb, cs);
+                int prow = prow_pre[b];
+                for (int h = 0; h < hg; ++h) {
+                    const int n = parts_of(stage_pre[b] + h * sb, sb, cs);
+                    if (n > 1) prow += n * HS * g;
+                }
+                const int c = s_ctx[b];
+                const int slot = n_item % kItemSlots;
+                if (n_item >= kItemSlots &&
+                    !mbar_wait(&iempty[slot], (uint32_t)(n_item / kItemSlots - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    ItemDesc &d = descs[slot];
+                    d.b = b;
+                    d.hg = hg;
+                    d.c = c;
+                    d.qs0 = s_qsl[b];
+                    d.nparts = nparts;
+                    d.part = g0 / cs - start / cs;
+                    d.prow = prow;
+                    const uint32_t qb = (uint32_t)HS * g * D * 2;
+                    mbar_arrive_expect_tx(&qfull[slot], qb);
+                    bulk_load(sm + prm.off_q + slot * prm.qslot_bytes,
+                              prm.q + ((long long)s_qsl[b] * Hq + hg * HS * g) * D, qb, &qfull[slot]);
+                }
+                __syncwarp();
+                ++n_item;
+                // the sequence's block table from this partition's first block, 32 entries per lane chunk
+                t_b = b;
+                cur_base = (st0 * NBS) & ~31;
+                cur_tab = chunk_entry(b, cur_base);
+                nxt_tab = chunk_entry(b, cur_base + 32);
+                const int nblk = (c + bs - 1) / bs;
+                for (int st = st0; st < st0 + cnt; ++st) {
+                    const int s = n_stage % NS;
+                    if (n_stage >= NS && !mbar_wait(&empty[s], ((n_stage / NS) - 1) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    const int blk0 = st * NBS;
+                    const int np = min(NBS, nblk - blk0);  // blocks of this stage inside the context
+                    if (lane == 0) {
+                        StageInfo &inf = infos[s];
+                        inf.slot = slot;
+                        inf.st = st;
+                        inf.flags = (st == st0 ? kFirst : 0) | (st == st0 + cnt - 1 ? kLast : 0);
+                        mbar_arrive_expect_tx(&full[s], (uint32_t)np * piece_bytes * 2);
+                    }
+                    uint8_t *kst = sm + (size_t)s * prm.stage_bytes;
+                    uint8_t *vst = kst + (size_t)NBS * piece_bytes;
+                    for (int j = 0; j < np; ++j) {
+                        const int phys = table_get(blk0 + j);
+                        const int y = (phys * Hkv + hg * HS) * bs;
+                        if (lane == 0) {
+#pragma unroll
+                            for (int pn = 0; pn < NPN; ++pn) {
+                                tma_load_2d(kst + j * piece_bytes + pn * panel_bytes, &tmk, pn * 64, y, &full[s]);
+                                tma_load_2d(vst + j * piece_bytes + pn * panel_bytes, &tmv, pn * 64, y, &full[s]);
+                            }
+                        }
+                    }
+                    __syncwarp();
+                    ++n_stage;
+                }
+                g0 += cnt;
+            }
+        }
+        if (ok) {
+            // end marker
+            const int s = n_stage % NS;
+            if (n_stage >= NS && !mbar_wait(&empty[s], ((n_stage / NS) - 1) & 1)) ok = false;
+            if (ok) {
+                if (lane == 0) {
+                    infos[s].flags = kEnd;
+                    mbar_arrive(&full[s]);
+                }
+                ++n_stage;
+            }
+        }
+        if (!ok) {
+            if (lane == 0) record_error(prm.err, PK_ERR_TIMEOUT);
+            // never leave with a copy still writing into this CTA's shared memory
+            for (int n = max(0, n_stage - NS); n < n_stage; ++n)
+                mbar_wait(&full[n % NS], (uint32_t)(n / NS) & 1);
+            for (int k = max(0, n_item - kItemSlots); k < n_item; ++k)
+                mbar_wait(&qfull[k % kItemSlots], (uint32_t)(k / kItemSlots) & 1);
+        }
+    } else {
+        // ---------------------------------------------------------- consumers
+        const int cw = warp - 1, hl = cw % HS, ph = cw / HS;
+        const int qr = lane >> 2, qc = (lane & 3) * 2;
+        const int mi = lane >> 3, rr = lane & 7;
+        const int a_row = (mi & 1) * 8 + rr, a_col = (mi >> 1) * 8;  // K rows (A of S^T)
+        const int v_row = (mi >> 1) * 8 + rr, v_col = (mi & 1) * 8;  // V rows (A of O^T, transposed)
+        uint32_t qb[KS][2];
+        float ot[KS][4];
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads qc, qc + 1
+        int c = 0;
+        uint32_t qph = 0, cph = 0;
+        // all consumer warps meet (bounded: false after the wait limit)
+        auto consumer_sync = [&]() -> bool {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(cbar);
+            const bool r = mbar_wait(cbar, cph);
+            cph ^= 1u;
+            return r;
+        };
+        // byte offset of stage-relative token tau's row (head hl) in a K or V part, and its swizzle phase
+        auto row_of = [&](int tau, uint32_t &off, int &sw) {
+            const int pc = tau / bs, t = tau - pc * bs;
+            const int r = hl * bs + t;
+            off = (uint32_t)pc * piece_bytes + (uint32_t)r * 128;
+            sw = r & 7;
+        };
+        auto begin_item = [&](int slot) -> bool {
+            if (!mbar_wait(&qfull[slot], (qph >> slot) & 1)) return false;
+            qph ^= 1u << slot;
+            c = descs[slot].c;
+            const uint8_t *qh = sm + prm.off_q + slot * prm.qslot_bytes + (size_t)(hl * g + qr) * D * 2;
+#pragma unroll
+            for (int kk = 0; kk < KS; ++kk) {
+                const int col = (kk * 16 + qc) * 2;
+                qb[kk][0] = qr < g ? *(const uint32_t *)(qh + col) : 0u;
+                qb[kk][1] = qr < g ? *(const uint32_t *)(qh + col + 16) : 0u;
+            }
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) ot[mt][0] = ot[mt][1] = ot[mt][2] = ot[mt][3] = 0.f;
+            m0 = m1 = -INFINITY;
+            l0 = l1 = 0.f;
+            return true;
+        };
+        // one 16-token tile (stage-relative tokens tau0..tau0+15, sequence tokens tok0..)
+        auto tile = [&](uint8_t *kst, uint8_t *vst, int tau0, int tok0) {
+            const int valid = c - tok0;
+            if (valid < kTile) {
+                // tail: clear V rows past the context (stale or never-written slots)
+                for (int ch = lane; ch < (kTile - valid) * (D / 8); ch += 32) {
+                    const int row = valid + ch / (D / 8), col = (ch % (D / 8)) * 8;
+                    uint32_t off;
+                    int sw;
+                    row_of(tau0 + row, off, sw);
+                    *(uint4 *)(vst + off + (col >> 6) * panel_bytes + ((((col & 63) >> 3) ^ sw) << 4)) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async();  // the stage is rewritten by TMA later
+                __syncwarp();
+            }
+            uint32_t koff, voff;
+            int ksw, vsw;
+            row_of(tau0 + a_row, koff, ksw);
+            row_of(tau0 + v_row, voff, vsw);
+            const uint32_t ka = smem_u32(kst) + koff, va = smem_u32(vst) + voff;
+            float st[4] = {0.f, 0.f, 0.f, 0.f}, su[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < KS; ++kk) {
+                const int col = kk * 16 + a_col;
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(ka + (col >> 6) * panel_bytes + ((((col & 63) >> 3) ^ ksw) << 4), a0, a1, a2, a3);
+                if (kk & 1) mma_bf16(su, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+                else mma_bf16(st, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+            }
+            // st[0], st[1]: token qr, heads qc, qc + 1; st[2], st[3]: token qr + 8
+            float s0 = (st[0] + su[0]) * prm.scale_log2, s1 = (st[1] + su[1]) * prm.scale_log2;
+            float s2 = (st[2] + su[2]) * prm.scale_log2, s3 = (st[3] + su[3]) * prm.scale_log2;
+            if (qr >= valid) s0 = s1 = -INFINITY;
+            if (qr + 8 >= valid) s2 = s3 = -INFINITY;
+            float ma = fmaxf(s0, s2), mb = fmaxf(s1, s3);
+#pragma unroll
+            for (int x = 4; x < 32; x <<= 1) {
+                ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, x));
+                mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, x));
+            }
+            const float na = fmaxf(m0, ma), nb = fmaxf(m1, mb);
+            const float ba = na == -INFINITY ? 0.f : na, bb = nb == -INFINITY ? 0.f : nb;
+            const float ala = fast_exp2(m0 - ba), alb = fast_exp2(m1 - bb);
+            m0 = na;
+            m1 = nb;
+            const float p0 = fast_exp2(s0 - ba), p1 = fast_exp2(s1 - bb);
+            const float p2 = fast_exp2(s2 - ba), p3 = fast_exp2(s3 - bb);
+            l0 = l0 * ala + p0 + p2;
+            l1 = l1 * alb + p1 + p3;
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                ot[mt][0] *= ala;
+                ot[mt][1] *= alb;
+                ot[mt][2] *= ala;
+                ot[mt][3] *= alb;
+            }
+            // P^T as the B fragment: transpose the two 8x8 (token x head) blocks
+            const uint32_t b0 = movmatrix_trans(pack_bf16(p0, p1));
+            const uint32_t b1 = movmatrix_trans(pack_bf16(p2, p3));
+            // O^T (16 d-rows x 8 heads per m-tile) += V^T P^T
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                const int col = mt * 16 + v_col;
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_t(va + (col >> 6) * panel_bytes + ((((col & 63) >> 3) ^ vsw) << 4), a0, a1, a2, a3);
+                mma_bf16(ot[mt], a0, a1, a2, a3, b0, b1);
+            }
+        };
+        float *scr = (float *)(sm + prm.off_scr);
+        constexpr int kScr = KS * 4 + 4;  // floats per lane of one warp's state
+        auto finish_item = [&](int slot) -> bool {
+            const ItemDesc d = descs[slot];
+            if (NPH > 1) {
+                // phases of one head: fold phases 1.. into phase 0 through shared memory
+                if (ph > 0) {
+                    float *w = scr + (size_t)(cw - HS) * 32 * kScr;
+#pragma unroll
+                    for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) w[(mt * 4 + i) * 32 + lane] = ot[mt][i];
+                    w[(KS * 4 + 0) * 32 + lane] = m0;
+                    w[(KS * 4 + 1) * 32 + lane] = m1;
+                    w[(KS * 4 + 2) * 32 + lane] = l0;
+                    w[(KS * 4 + 3) * 32 + lane] = l1;
+                }
+                if (!consumer_sync()) return false;
+                if (ph == 0) {
+                    for (int q = 1; q < NPH; ++q) {
+                        const float *w = scr + (size_t)(hl + q * HS - HS) * 32 * kScr;
+                        const float xm0 = w[(KS * 4 + 0) * 32 + lane], xm1 = w[(KS * 4 + 1) * 32 + lane];
+                        const float xl0 = w[(KS * 4 + 2) * 32 + lane], xl1 = w[(KS * 4 + 3) * 32 + lane];
+                        const float n0 = fmaxf(m0, xm0), n1 = fmaxf(m1, xm1);
+                        const float b0 = n0 == -INFINITY ? 0.f : n0, b1 = n1 == -INFINITY ? 0.f : n1;
+                        const float a0 = fast_exp2(m0 - b0), x0 = fast_exp2(xm0 - b0);
+                        const float a1 = fast_exp2(m1 - b1), x1 = fast_exp2(xm1 - b1);
+                        l0 = l0 * a0 + xl0 * x0;
+                        l1 = l1 * a1 + xl1 * x1;
+                        m0 = n0;
+                        m1 = n1;
+#pragma unroll
+                        for (int mt = 0; mt < KS; ++mt) {
+                            ot[mt][0] = ot[mt][0] * a0 + w[(mt * 4 + 0) * 32 + lane] * x0;
+                            ot[mt][1] = ot[mt][1] * a1 + w[(mt * 4 + 1) * 32 + lane] * x1;
+                            ot[mt][2] = ot[mt][2] * a0 + w[(mt * 4 + 2) * 32 + lane] * x0;
+                            ot[mt][3] = ot[mt][3] * a1 + w[(mt * 4 + 3) * 32 + lane] * x1;
+                        }
+                    }
+                }
+                if (!consumer_sync()) return false;  // the scratch is free again
+            }
+            const bool split = d.nparts > 1;
+            if (ph == 0) {
+#pragma unroll
+                for (int x = 4; x < 32; x <<= 1) {  // sums over the token lanes of each head
+                    l0 += __shfl_xor_sync(0xffffffffu, l0, x);
+                    l1 += __shfl_xor_sync(0xffffffffu, l1, x);
+                }
+                const float ia = l0 > 0.f ? 1.f / l0 : 0.f, ib = l1 > 0.f ? 1.f / l1 : 0.f;
+                const int ha = qc, hb = qc + 1;  // heads of this lane's accumulators
+                const bool va_ = ha < g, vb_ = hb < g;
+                const int kvh = d.hg * HS + hl;
+                if (!split) {
+                    __nv_bfloat16 *oa = prm.out + ((long long)d.qs0 * Hq + kvh * g + ha) * D;
+                    __nv_bfloat16 *ob = oa + D;
+#pragma unroll
+                    for (int mt = 0; mt < KS; ++mt) {
+                        const int d0 = mt * 16 + qr;
+                        if (va_) {
+                            oa[d0] = __float2bfloat16_rn(ot[mt][0] * ia);
+                            oa[d0 + 8] = __float2bfloat16_rn(ot[mt][2] * ia);
+                        }
+                        if (vb_) {
+                            ob[d0] = __float2bfloat16_rn(ot[mt][1] * ib);
+                            ob[d0 + 8] = __float2bfloat16_rn(ot[mt][3] * ib);
+                        }
+                    }
+                } else {
+                    const int row = d.prow + d.part * HS * g + hl * g;
+                    float *pa_ = prm.partial_o + (size_t)(row + ha) * D;
+                    float *pb_ = pa_ + D;
+#pragma unroll
+                    for (int mt = 0; mt < KS; ++mt) {
+                        const int d0 = mt * 16 + qr;
+                        if (va_) {
+                            pa_[d0] = ot[mt][0] * ia;
+                            pa_[d0 + 8] = ot[mt][2] * ia;
+                        }
+                        if (vb_) {
+                            pb_[d0] = ot[mt][1] * ib;
+                            pb_[d0 + 8] = ot[mt][3] * ib;
+                        }
+                    }
+                    if (qr == 0) {
+                        float *pl = prm.partial_lse + (size_t)row;
+                        if (va_) pl[ha] = l0 > 0.f ? m0 + __log2f(l0) : -INFINITY;
+                        if (vb_) pl[hb] = l1 > 0.f ? m1 + __log2f(l1) : -INFINITY;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&iempty[slot]);
+            return true;
+        };
+
+        for (int n = 0;; ++n) {
+            const int s = n % NS;
+            if (!mbar_wait(&full[s], (uint32_t)(n / NS) & 1)) {
+                ok = false;
+                break;
+            }
+            const StageInfo inf = infos[s];
+            if (inf.flags & kEnd) break;
+            if ((inf.flags & kFirst) && !begin_item(inf.slot)) {
+                ok = false;
+                break;
+            }
+            uint8_t *kst = sm + (size_t)s * prm.stage_bytes;
+            uint8_t *vst = kst + (size_t)NBS * piece_bytes;
+            const int tok_stage = inf.st * ST;
+            for (int j = ph; j * kTile < ST; j += NPH) {
+                const int tok0 = tok_stage + j * kTile;
+                if (tok0 >= c) break;
+                tile(kst, vst, j * kTile, tok0);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+            if ((inf.flags & kLast) && !finish_item(inf.slot)) {
+                ok = false;
+                break;
+            }
+        }
+        if (!ok && lane == 0) record_error(prm.err, PK_ERR_TIMEOUT);
+    }
+    __syncthreads();
+    release_counter(prm.hdr);
+}
+
+// The largest dynamic shared memory a launch may ask for: the device's opt-in
+// limit per block less the kernel's static shared memory.
+// Merge of the split-K partitions [flash-decoding combination]: for every
+// (sequence, head group) that the streaming kernel cut into several
+// partitions, each output row (q head hg * HS * g + r of the sequence's token)
+// is out = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M), M = max_p lse_p, over
+// the partitions' normalised rows o_p and log2-sum-exps lse_p.  One thread per
+// (row, 4 columns); blockIdx.x = sequence * head groups + head group.
+struct MergeParams {
+    __nv_bfloat16 *out;
+    const int32_t *qsl;
+    const int *mplan;
+    const float *partial_o, *partial_lse;
+    int seq0, nseq, n_q_heads, n_kv_heads, group, HS;
+};
+
+constexpr int kMergeThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kMergeThreads) attention_merge_kernel(const MergeParams mp) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // the streaming kernel has finished
+    const int NHG = mp.n_kv_heads / mp.HS, HG = mp.HS * mp.group;
+    const int b = blockIdx.x / NHG, hg = blockIdx.x % NHG;
+    if (b >= mp.nseq) return;
+    const int *stage_pre = mp.mplan + kMergePlanHead, *prow_pre = stage_pre + kPlanLen;
+    const int cs = mp.mplan[0];
+    const int sb = (stage_pre[b + 1] - stage_pre[b]) / NHG;
+    if (sb == 0) return;
+    auto parts_of = [&](int start) { return (start + sb - 1) / cs - start / cs + 1; };
+    const int nparts = parts_of(stage_pre[b] + hg * sb);
+    if (nparts <= 1) return;
+    int prow = prow_pre[b];
+    for (int h = 0; h < hg; ++h) {
+        const int n = parts_of(stage_pre[b] + h * sb);
+        if (n > 1) prow += n * HG;
+    }
+    const int unit = blockIdx.y * kMergeThreads + threadIdx.x;
+    if (unit >= HG * (D / 4)) return;
+    const int r = unit / (D / 4), c4 = unit % (D / 4);
+    const float *lse = mp.partial_lse + prow + r;
+    float M = -INFINITY;
+#pragma unroll 8
+    for (int q = 0; q < nparts; ++q) M = fmaxf(M, __ldcg(lse + (size_t)q * HG));
+    float den = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 *po = (const float4 *)(mp.partial_o + (size_t)(prow + r) * D) + c4;
+#pragma unroll 8
+    for (int q = 0; q < nparts; ++q) {
+        const float l = __ldcg(lse + (size_t)q * HG);
+        const float4 x = __ldcg(po + (size_t)q * HG * (D / 4));
+        const float w = l == -INFINITY ? 0.f : fast_exp2(l - M);
+        den += w;
+        acc.x += w * x.x;
+        acc.y += w * x.y;
+        acc.z += w * x.z;
+        acc.w += w * x.w;
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    const long long orow = (long long)__ldg(mp.qsl + mp.seq0 + b) * mp.n_q_heads + hg * HG + r;
+    uint2 pk;
+    pk.x = pack_bf16(acc.x * inv, acc.y * inv);
+    pk.y = pack_bf16(acc.z * inv, acc.w * inv);
+    *(uint2 *)(mp.out + orow * D + c4 * 4) = pk;
+}
+
+template <int D>
+int blocks_prepare(pk_pool *p) {
+    int optin = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, p->device);
+    cudaFuncAttributes fa{};
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, attention_decode_blocks_kernel<D>);
+    if (e != cudaSuccess) return cuda_fail(e, "decode (block stream) attributes");
+    p->blk_smem_max = optin - (int)fa.sharedSizeBytes;
+    e = cudaFuncSetAttribute(attention_decode_blocks_kernel<D>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, p->blk_smem_max);
+    if (e != cudaSuccess) return cuda_fail(e, "set decode (block stream) smem size");
+    return PK_OK;
+}
+
+template <int D>
+int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, cudaStream_t st) {
+    BlkParams tp{};
+    tp.q = (const __nv_bfloat16 *)a.q;
+    tp.out = (__nv_bfloat16 *)a.out;
+    tp.tables = a.block_tables;
+    tp.ctx = a.context_lens;
+    tp.qsl = a.query_start_lens;
+    tp.max_blocks = a.max_blocks_per_seq;
+    tp.n_q_heads = a.n_q_heads;
+    tp.n_kv_heads = p->n_kv_heads;
+    tp.group = a.n_q_heads / p->n_kv_heads;
+    tp.block_size = p->block_size;
+    tp.num_blocks = p->num_blocks;
+    tp.num_tokens = a.num_tokens;
+    tp.HS = p->blk_hs;
+    tp.NBS = p->blk_nbs;
+    tp.ST = p->blk_nbs * p->block_size;
+    tp.NPH = kNC / p->blk_hs;
+    tp.ncta = p->sm_count;
+    tp.cap_rows = w.cap_rows;
+    tp.scale_log2 = a.scale * 1.4426950408889634f;
+    tp.hdr = (WsHeader *)w.header;
+    tp.mplan = w.merge_plan;
+    tp.partial_o = w.partial_o;
+    tp.partial_lse = w.partial_lse;
+    tp.err = p->d_err;
+    tp.NS = 3;
+    blk_layout<D>(tp);
+    if (tp.total > (uint32_t)p->blk_smem_max) {
+        tp.NS = 2;
+        blk_layout<D>(tp);
+    }
+    if (tp.total > (uint32_t)p->blk_smem_max)
+        return fail(PK_ERR_UNSUPPORTED, "decode attention: %u bytes of shared memory", tp.total);
+    for (int s0 = 0; s0 < a.num_seqs; s0 += kMaxSeqsPerLaunch) {
+        tp.seq0 = s0;
+        tp.nseq = std::min(kMaxSeqsPerLaunch, a.num_seqs - s0);
+        attention_decode_blocks_kernel<D><<<tp.ncta, kBlkThreads, tp.total, st>>>(p->tmap_kb, p->tmap_vb, tp);
+        MergeParams mp;
+        mp.out = tp.out;
+        mp.qsl = tp.qsl;
+        mp.mplan = tp.mplan;
+        mp.partial_o = tp.partial_o;
+        mp.partial_lse = tp.partial_lse;
+        mp.seq0 = tp.seq0;
+        mp.nseq = tp.nseq;
+        mp.n_q_heads = tp.n_q_heads;
+        mp.n_kv_heads = tp.n_kv_heads;
+        mp.group = tp.group;
+        mp.HS = tp.HS;
+        const int units = tp.HS * tp.group * (D / 4);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(tp.nseq * (tp.n_kv_heads / tp.HS), (units + kMergeThreads - 1) / kMergeThreads);
+        cfg.blockDim = dim3(kMergeThreads);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, attention_merge_kernel<D>, mp);
+        if (e != cudaSuccess) return cuda_fail(e, "split-K merge launch");
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PK_OK : cuda_fail(e, "decode attention launch");
+}
+
+}  // namespace
+
+// Stage geometry of a pool: HS = the largest power of two dividing n_kv_heads
+// (at most 8) whose block (K + V of HS heads) fits a stage, halved until a
+// stage of whole blocks holds a multiple of 16 tokens; NBS = blocks per stage.
+int decode_blocks_prepare_pool(pk_pool *p) {
+    p->blk_ok = false;
+    const int D = p->head_dim, bs = p->block_size;
+    int hs = 1;
+    while (hs < 8 && p->n_kv_heads % (hs * 2) == 0) hs *= 2;
+    for (; hs >= 1; hs /= 2) {
+        const long long per_block = (long long)hs * bs * D * 4;
+        if (per_block > kStageCap || hs * bs > 256) continue;
+        int nbs = (int)(kStageCap / per_block);
+        while (nbs >= 1 && (nbs * bs) % kTile != 0) --nbs;
+        if (nbs < 1) continue;
+        p->blk_hs = hs;
+        p->blk_nbs = nbs;
+        p->blk_ok = true;
+        break;
+    }
+    if (!p->blk_ok) return PK_OK;  // the other decode kernel serves this geometry
+    int rc;
+    switch (D) {
+        case 64: rc = blocks_prepare<64>(p); break;
+        case 128: rc = blocks_prepare<128>(p); break;
+        default: rc = blocks_prepare<256>(p); break;
+    }
+    if (rc != PK_OK) return rc;
+    rc = encode_pool_map(&p->tmap_kb, p->k_base, p, p->blk_hs * bs);
+    if (rc == PK_OK) rc = encode_pool_map(&p->tmap_vb, p->v_base, p, p->blk_hs * bs);
+    return rc;
+}
+
+int decode_blocks_chunks_per_cta() { return kChunksPerCta; }
+
+bool decode_blocks_applies(const pk_pool *p, const AttnArgs &a) {
+    return p->blk_ok && a.num_tokens == a.num_seqs && a.n_q_heads / p->n_kv_heads <= 8;
+}
+
+int launch_decode_blocks(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, cudaStream_t st) {
+    switch (p->head_dim) {
+        case 64: return blocks_launch<64>(p, a, w, st);
+        case 128: return blocks_launch<128>(p, a, w, st);
+        case 256: return blocks_launch<256>(p, a, w, st);
+        default: return fail(PK_ERR_UNSUPPORTED, "decode path: head_dim %d", p->head_dim);
+    }
+}
+
+}  // namespace pk

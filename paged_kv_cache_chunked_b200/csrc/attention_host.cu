@@ -1,6 +1,8 @@
 // Host side of the tensor-core attention path: workspace layout and the
 // dispatch of a call to the chunk kernel (sequences whose query rows need more
-// than one 16-row tile) and the decode kernel (all others).
+// than one 16-row tile), the block-streaming decode kernel (batches of one
+// query token per sequence and at most 8 q heads per kv head) and the
+// tile-streaming decode kernel (the remaining sequences of one 16-row tile).
 #include <algorithm>
 
 #include "pk_internal.h"
@@ -14,11 +16,11 @@ constexpr int kMaxSeqsPerLaunch = 512;   // window of sequences per kernel launc
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace: decode header | chunk header | split-K counters (fixed size) |
-// partial log2-sum-exp | partial O.  The headers and counters sit at offsets
+// merge plan (fixed size) | partial log2-sum-exp | partial O.  The headers and counters sit at offsets
 // that do not depend on the batch, so the zeros every call leaves there stay
 // valid when the next call's batch differs.
 struct Layout {
-    size_t hdr_decode, hdr_chunk, counters, partial_lse, partial_o, total;
+    size_t hdr_decode, hdr_chunk, counters, merge_plan, partial_lse, partial_o, total;
     int cap_rows;
 };
 
@@ -29,14 +31,19 @@ Layout layout(const pk_pool *p, int num_seqs, int n_q_heads) {
     // split items: at most Hkv per sequence plus the ~items_per_cta per CTA that
     // split-K adds; a decode item has g partial rows (the planner coarsens the
     // partitions when a batch of short chunks needs more)
-    const long long items = (long long)Hkv * std::min(num_seqs, kMaxSeqsPerLaunch) +
-                            (long long)p->tc_ctas * decode_items_per_cta();
+    // (the block-streaming kernel: chunks x heads per stage, rows of g each)
+    const long long per_cta =
+        std::max((long long)p->tc_ctas * decode_items_per_cta(),
+                 p->blk_ok ? (long long)p->sm_count * decode_blocks_chunks_per_cta() * p->blk_hs : 0LL);
+    const long long items = (long long)Hkv * std::min(num_seqs, kMaxSeqsPerLaunch) + per_cta;
     L.cap_rows = (int)std::min<long long>(items * std::min(g, kTile), 1LL << 30);
     L.hdr_decode = 0;
     L.hdr_chunk = kHeaderBytes;
     size_t off = 2 * kHeaderBytes;
     L.counters = off;
     off = align_up(off + (size_t)kMaxSeqsPerLaunch * Hkv * sizeof(int), 256);
+    L.merge_plan = off;  // 8 ints, then two arrays of kMaxSeqsPerLaunch + 1
+    off = align_up(off + (size_t)(8 + 2 * (kMaxSeqsPerLaunch + 1)) * sizeof(int), 256);
     L.partial_lse = off;
     off = align_up(off + (size_t)L.cap_rows * sizeof(float), 256);
     L.partial_o = off;
@@ -55,6 +62,7 @@ size_t tc_workspace_bytes(const pk_pool *p, int num_seqs, int num_tokens, int n_
 
 int tc_prepare_pool(pk_pool *p) {
     int rc = decode_prepare_pool(p);
+    if (rc == PK_OK) rc = decode_blocks_prepare_pool(p);
     if (rc == PK_OK) rc = chunk_prepare_pool(p);
     return rc;
 }
@@ -76,9 +84,11 @@ int launch_attention_tc(const pk_pool *p, const AttnArgs &a, cudaStream_t st) {
     DecodeWs w;
     w.header = ws + L.hdr_decode;
     w.counters = (int *)(ws + L.counters);
+    w.merge_plan = (int *)(ws + L.merge_plan);
     w.partial_lse = (float *)(ws + L.partial_lse);
     w.partial_o = (float *)(ws + L.partial_o);
     w.cap_rows = L.cap_rows;
+    if (decode_blocks_applies(p, a)) return launch_decode_blocks(p, a, w, st);
     return launch_decode(p, a, w, st);
 }
 

@@ -22,8 +22,13 @@ struct pk_pool {
     bool tc_path;       // tensor-core + TMA attention applies to this geometry
     int tc_ctas;        // resident CTAs of the decode attention kernel (whole GPU)
     int tc_ctas_chunk;  // resident CTAs of the chunk attention kernel (whole GPU)
+    bool blk_ok;        // the block-streaming decode kernel serves this geometry
+    int blk_hs, blk_nbs;  // its kv heads and blocks per pipeline stage
+    int blk_smem_max;     // its largest dynamic shared memory per launch
     alignas(64) CUtensorMap tmap_k;
     alignas(64) CUtensorMap tmap_v;
+    alignas(64) CUtensorMap tmap_kb;  // boxes of blk_hs * block_size rows (whole blocks)
+    alignas(64) CUtensorMap tmap_vb;
 };
 
 namespace pk {
@@ -72,12 +77,21 @@ int launch_attention_tc(const pk_pool *p, const AttnArgs &a, cudaStream_t st);
 struct DecodeWs {
     void *header;
     int *counters;
+    int *merge_plan;  // the block-streaming kernel's plan, for its merge kernel
     float *partial_o, *partial_lse;
     int cap_rows;
 };
 int decode_prepare_pool(pk_pool *p);
 int decode_items_per_cta();
 int launch_decode(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, cudaStream_t st);
+// Block-streaming decode kernel: batches whose sequences all have one query
+// token and groups of at most 8 q heads per kv head.
+int decode_blocks_prepare_pool(pk_pool *p);
+int decode_blocks_chunks_per_cta();
+bool decode_blocks_applies(const pk_pool *p, const AttnArgs &a);
+int launch_decode_blocks(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, cudaStream_t st);
+// 2-D TMA view of a pool (rows of head_dim bf16) with boxes of 64 columns x box_rows.
+int encode_pool_map(CUtensorMap *map, void *base, const pk_pool *p, int box_rows);
 int chunk_prepare_pool(pk_pool *p);
 int launch_chunk(const pk_pool *p, const AttnArgs &a, void *header, cudaStream_t st);
 

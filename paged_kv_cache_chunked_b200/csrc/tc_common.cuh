@@ -270,6 +270,82 @@ __device__ inline SplitItem decode_split(const PlanArrays &p, int nseq, int grou
     return it;
 }
 
+// Merges the split-K partitions of one (sequence, kv head) into the output
+// [flash-decoding combination of per-partition softmax results]:
+//   out_r = sum_p 2^(lse_p,r - M_r) o_p,r / sum_p 2^(lse_p,r - M_r),  M_r = max_p lse_p,r
+// where o_p,r is partition p's normalised output row r and lse_p,r its
+// log2-sum-exp (-inf for a partition with no key).  Partition p's rows sit at
+// partial rows base + p * pstride + r; row r is query token r / g (of the
+// tokens starting at qs0), q head kvh * g + r % g.  Merges rows row0 ..
+// row0 + nrows - 1.  Rows go four at a time, and
+// loads are issued for all four rows (and two partitions) at once so their
+// latencies overlap.  Executed by one full warp.
+template <int D, int UNROLL = 2>
+__device__ inline void merge_partials(const float *partial_o, const float *partial_lse, int base,
+                                      int pstride, int nparts, int row0, int nrows,
+                                      __nv_bfloat16 *out, int qs0, int Hq, int kvh, int g,
+                                      int lane) {
+    constexpr int RG = 4;
+    base += row0;
+    for (int r0 = 0; r0 < nrows; r0 += RG) {
+        float Mr[RG], den[RG];
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+            float mx = -INFINITY;
+            if (r0 + r < nrows)
+                for (int p = lane; p < nparts; p += 32)
+                    mx = fmaxf(mx, __ldcg(partial_lse + (size_t)(base + p * pstride) + r0 + r));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            Mr[r] = mx;
+        }
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+            float sm = 0.f;
+            if (r0 + r < nrows)
+                for (int p = lane; p < nparts; p += 32) {
+                    const float lse = __ldcg(partial_lse + (size_t)(base + p * pstride) + r0 + r);
+                    sm += lse == -INFINITY ? 0.f : fast_exp2(lse - Mr[r]);
+                }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
+            den[r] = sm > 0.f ? 1.f / sm : 0.f;
+        }
+        for (int c4 = lane; c4 < D / 4; c4 += 32) {
+            float4 acc[RG];
+#pragma unroll
+            for (int r = 0; r < RG; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll UNROLL
+            for (int p = 0; p < nparts; ++p) {
+                const size_t prow = (size_t)(base + p * pstride) + r0;
+#pragma unroll
+                for (int r = 0; r < RG; ++r) {
+                    if (r0 + r < nrows) {
+                        const float lse = __ldcg(partial_lse + prow + r);
+                        const float wgt = lse == -INFINITY ? 0.f : fast_exp2(lse - Mr[r]);
+                        const float4 x = __ldcg((const float4 *)(partial_o + (prow + r) * D) + c4);
+                        acc[r].x += wgt * x.x;
+                        acc[r].y += wgt * x.y;
+                        acc[r].z += wgt * x.z;
+                        acc[r].w += wgt * x.w;
+                    }
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < RG; ++r) {
+                if (r0 + r < nrows) {
+                    const int row = row0 + r0 + r;
+                    const long long orow = (long long)(qs0 + row / g) * Hq + kvh * g + row % g;
+                    uint2 pk;
+                    pk.x = pack_bf16(acc[r].x * den[r], acc[r].y * den[r]);
+                    pk.y = pack_bf16(acc[r].z * den[r], acc[r].w * den[r]);
+                    *(uint2 *)(out + orow * D + c4 * 4) = pk;
+                }
+            }
+        }
+    }
+}
+
 // The last CTA to finish resets the work counter for the next call (call
 // after a __syncthreads that every thread of the CTA reaches).
 __device__ inline void release_counter(WsHeader *hdr) {
