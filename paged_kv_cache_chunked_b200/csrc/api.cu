@@ -72,6 +72,25 @@ int encode_pool_map(CUtensorMap *map, void *base, const pk_pool *p, int box_rows
     return PK_OK;
 }
 
+// 3-D view of the same rows: x = column within a 64-column panel, y = row, z =
+// panel (stride 128 bytes).  A box {64, box_rows, head_dim / 64} lands in shared
+// memory as head_dim / 64 consecutive panels of box_rows 128-byte rows, the
+// layout of box_rows-row 2-D boxes placed panel after panel.
+int encode_pool_map3(CUtensorMap *map, void *base, const pk_pool *p, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(PK_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    const cuuint64_t dims[3] = {64, (cuuint64_t)p->num_blocks * p->n_kv_heads * p->block_size,
+                                (cuuint64_t)p->head_dim / 64};
+    const cuuint64_t strides[2] = {(cuuint64_t)p->head_dim * 2, 128};
+    const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)p->head_dim / 64};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PK_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (%d)", (int)r);
+    return PK_OK;
+}
+
 }  // namespace pk
 
 using namespace pk;

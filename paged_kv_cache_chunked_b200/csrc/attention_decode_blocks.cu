@@ -14,7 +14,7 @@
 // of HS heads is one run of HS * bs rows.  The kernel streams whole blocks:
 //   - one producer warp per CTA claims chunks of work, looks the blocks up in
 //     the block tables and loads each block's K and V rows for HS heads with
-//     128-row TMA boxes (128-byte swizzle) into a ring of NS shared-memory
+//     one TMA box each (all 64-column panels, 128-byte swizzle) into a ring of NS shared-memory
 //     stages, a stage being NBS blocks (ST = NBS * bs tokens, up to 64 KiB);
 //     a few large copies per block keep HBM busy from one issuing warp;
 //   - eight consumer warps own one kv head each (or, for HS < 8, one of
@@ -24,8 +24,9 @@
 //     moved into operand order by movmatrix, and an online softmax in fp32.
 // Work split (flash-decoding-style split-K, balanced like stream-K): the
 // stages of all (sequence, head group) pairs are concatenated and cut into
-// chunks of CS stages, about kChunksPerCta per CTA; CTAs claim chunks from a
-// global counter.  The part of a pair inside one chunk is a partition; a pair
+// chunks claimed from a global counter: first one large chunk per CTA
+// (kBigEighths / 8 of the work), then small ones (kSmallPerCta per CTA), so a
+// CTA that runs slow sheds the small chunks to the others.  The part of a pair inside one chunk is a partition; a pair
 // cut into several partitions writes (normalised O, log2-sum-exp) rows per
 // partition, and a second kernel, launched as a programmatic dependent of the
 // first, merges them with the whole GPU (no fence, atomic or wait in the
@@ -46,12 +47,40 @@ using namespace tc;
 constexpr int kNC = 8;                        // consumer warps
 constexpr int kBlkThreads = (kNC + 1) * 32;   // + one producer warp
 constexpr int kStageCap = 64 * 1024;          // K + V bytes of one stage
-constexpr int kChunksPerCta = 2;              // work chunks per CTA (dynamic claiming)
-constexpr int kMinChunkStages = 4;            // smallest chunk
+constexpr int kBigEighths = 8;                // share of the work in the first (large) chunks
+constexpr int kSmallPerCta = 4;               // small chunks per CTA for the rest
+constexpr int kMinChunkStages = 2;            // smallest chunk
 constexpr int kItemSlots = 2;                 // items staged ahead (Q rows + descriptor each)
-constexpr int kMergePlanHead = 8;             // merge plan: cs, total, then stage_pre, prow_pre
+constexpr int kMergeListHead = 4;             // merge list: count, pad, then int4 entries
+constexpr float kRescaleLog2 = 8.f;           // lazy softmax rescale threshold (log2 units)
 
 enum : int { kFirst = 1, kLast = 2, kEnd = 4 };
+
+// Chunks of the concatenated stages: nb large chunks of cb stages, then small
+// chunks of csm stages up to `total`.
+struct ChunkPlan {
+    int cb, nb, csm, total;
+    __device__ int of(int g) const {  // chunk holding stage g
+        const int big = nb * cb;
+        return g < big ? g / cb : nb + (g - big) / csm;
+    }
+    __device__ int begin(int k) const { return k < nb ? k * cb : nb * cb + (k - nb) * csm; }
+    __device__ int end(int k) const { return min(total, begin(k + 1)); }
+    __device__ int count() const { return nb + (total - nb * cb + csm - 1) / csm; }
+    // partitions of the stages [start, start + n)
+    __device__ int parts(int start, int n) const { return of(start + n - 1) - of(start) + 1; }
+};
+
+__device__ inline ChunkPlan make_chunk_plan(int total, int ncta, int scale) {
+    ChunkPlan c;
+    c.total = total;
+    c.cb = max(kMinChunkStages, (int)((long long)total * kBigEighths / (8LL * ncta))) * scale;
+    c.nb = min(ncta, total / c.cb);
+    const long long rest = total - (long long)c.nb * c.cb;
+    c.csm = max(kMinChunkStages, (int)((rest + (long long)ncta * kSmallPerCta - 1) /
+                                       ((long long)ncta * kSmallPerCta))) * scale;
+    return c;
+}
 
 struct StageInfo {
     int slot, st, flags, pad;
@@ -125,7 +154,7 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
     uint64_t *qfull = empty + NS;
     uint64_t *iempty = qfull + kItemSlots;
     uint64_t *cbar = iempty + kItemSlots;  // barrier of the consumer warps
-    __shared__ int s_total, s_cs;
+    __shared__ ChunkPlan s_cp;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -143,7 +172,6 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
     // per sequence: S_b = ceil(c_b / ST) stages per head group; chunk size CS;
     // a (sequence, head group) spanning several chunks has one partition per
     // chunk, each with HS * g partial rows
-    auto parts_of = [&](int start, int sb, int cs) { return (start + sb - 1) / cs - start / cs + 1; };
     if (warp == 0) {
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
@@ -174,8 +202,7 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
         if (lane == 0) stage_pre[0] = 0;
         __syncwarp();
         const int total = run;
-        const long long want = (long long)prm.ncta * kChunksPerCta;
-        int cs = (int)std::max<long long>(kMinChunkStages, (total + want - 1) / want);
+        ChunkPlan cp = make_chunk_plan(total, prm.ncta, 1);
         for (int attempt = 0; attempt < 8; ++attempt) {
             int runp = 0;
             for (int base = 0; base < nseq; base += 32) {
@@ -184,7 +211,7 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                 if (i < nseq) {
                     const int sb = (stage_pre[i + 1] - stage_pre[i]) / NHG;
                     for (int hg = 0; hg < NHG && sb > 0; ++hg) {
-                        const int n = parts_of(stage_pre[i] + hg * sb, sb, cs);
+                        const int n = cp.parts(stage_pre[i] + hg * sb, sb);
                         if (n > 1) np += n * HS * g;
                     }
                 }
@@ -200,142 +227,174 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
             if (runp <= prm.cap_rows) break;
             // more partial rows than the workspace holds: coarser chunks, finally
             // one chunk for everything (no split)
-            cs = attempt < 6 ? 2 * cs : std::max(total, 1);
+            if (attempt < 6) {
+                cp = make_chunk_plan(total, prm.ncta, 2 << attempt);
+            } else {
+                cp.cb = cp.csm = max(total, 1);
+                cp.nb = total > 0 ? 1 : 0;
+            }
         }
         if (lane == 0) {
             prow_pre[0] = 0;
-            s_total = total;
-            s_cs = cs;
+            s_cp = cp;
         }
         __syncwarp();
-        if (blockIdx.x == 0) {  // the merge kernel's copy of the plan
-            if (lane == 0) {
-                prm.mplan[0] = cs;
-                prm.mplan[1] = total;
+        if (blockIdx.x == 0) {
+            // the merge kernel's work list: (sequence, head group, first partial
+            // row, partitions) of every pair cut into several partitions
+            int n_split = 0;
+            for (int base = 0; base < nseq; base += 32) {
+                const int i = base + lane;
+                const int sb = i < nseq ? (stage_pre[i + 1] - stage_pre[i]) / NHG : 0;
+                int prow = i < nseq ? prow_pre[i] : 0;
+                for (int hg = 0; hg < NHG; ++hg) {
+                    const int n = sb > 0 ? cp.parts(stage_pre[i] + hg * sb, sb) : 1;
+                    const unsigned m = __ballot_sync(0xffffffffu, n > 1);
+                    if (n > 1) {
+                        int4 *e = (int4 *)(prm.mplan + kMergeListHead) + n_split + __popc(m & ((1u << lane) - 1));
+                        *e = make_int4(i, hg, prow, n);
+                        prow += n * HS * g;
+                    }
+                    n_split += __popc(m);
+                }
             }
-            for (int i = lane; i <= nseq; i += 32) {
-                prm.mplan[kMergePlanHead + i] = stage_pre[i];
-                prm.mplan[kMergePlanHead + kPlanLen + i] = prow_pre[i];
-            }
+            if (lane == 0) prm.mplan[0] = n_split;
         }
     }
     // the merge kernel may be scheduled now; it waits for this grid to finish
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __syncthreads();
-    const int total = s_total, cs = s_cs;
+    const ChunkPlan cp = s_cp;
     bool ok = true;
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
-        const int nchunks = (total + cs - 1) / cs;
+        // CTA i starts with chunk i; the chunks after the first gridDim.x go to
+        // whoever claims them (the claim for the next one is always in flight)
+        const int nchunks = cp.count();
         auto claim = [&]() -> int {
             int v = 0;
-            if (lane == 0) v = atomicAdd(&prm.hdr->next_item, 1);
+            if (lane == 0) v = (int)gridDim.x + atomicAdd(&prm.hdr->next_item, 1);
             return v;
         };
-        int pending = claim();
+        int pending = (int)blockIdx.x;
         int n_stage = 0, n_item = 0;
-        int cur_base = 0, cur_tab = 0, nxt_tab = 0, t_b = 0;
         auto chunk_entry = [&](int b, int blk_base) -> int {
             const int nblk = (s_ctx[b] + bs - 1) / bs;
             const int e = blk_base + lane;
             return e < nblk ? __ldg(prm.tables + (long long)(prm.seq0 + b) * prm.max_blocks + e) : 0;
         };
-        auto table_get = [&](int blk) -> int {
-            while (blk >= cur_base + 32) {
-                cur_base += 32;
-                cur_tab = nxt_tab;
-                nxt_tab = chunk_entry(t_b, cur_base + 32);
-            }
-            int phys = __shfl_sync(0xffffffffu, cur_tab, blk - cur_base);
-            if (phys < 0 || phys >= prm.num_blocks) {
-                if (lane == 0) record_error(prm.err, PK_ERR_BAD_INDEX);
-                phys = 0;
-            }
-            return phys;
+        // Items (partitions) in claim order.  The next item is found, and its
+        // first two table chunks requested, while the current one's stages
+        // are issued, so the table lookups of an item start without a wait.
+        struct PItem {
+            int b, hg, st0, cnt, nparts, part, prow, tab0, tab1;
         };
-        while (ok) {
-            const int chunk = __shfl_sync(0xffffffffu, pending, 0);
-            if (chunk >= nchunks) break;
-            pending = claim();
-            int g0 = chunk * cs;
-            const int g1 = min(total, g0 + cs);
-            while (ok && g0 < g1) {
-                // the partition of one (sequence, head group) inside this chunk
-                const int b = find_seq(stage_pre, nseq, g0);
-                const int sb = (stage_pre[b + 1] - stage_pre[b]) / NHG;
-                const int local = g0 - stage_pre[b];
-                const int hg = local / sb, st0 = local - hg * sb;
-                const int cnt = min(sb - st0, g1 - g0);
-                const int start = stage_pre[b] + hg * sb;
-                const int nparts = parts_of(start, sb, cs);
-                int prow = prow_pre[b];
-                for (int h = 0; h < hg; ++h) {
-                    const int n = parts_of(stage_pre[b] + h * sb, sb, cs);
-                    if (n > 1) prow += n * HS * g;
+        int g0 = 0, g1 = 0;
+        auto next_item = [&](PItem &it) -> bool {
+            while (g0 >= g1) {
+                const int chunk = __shfl_sync(0xffffffffu, pending, 0);
+                if (chunk >= nchunks) return false;
+                pending = claim();  // lane 0's value; broadcast when used
+                g0 = cp.begin(chunk);
+                g1 = cp.end(chunk);
+            }
+            // the partition of one (sequence, head group) inside the chunk
+            const int b = find_seq(stage_pre, nseq, g0);
+            const int sb = (stage_pre[b + 1] - stage_pre[b]) / NHG;
+            const int local = g0 - stage_pre[b];
+            it.b = b;
+            it.hg = local / sb;
+            it.st0 = local - it.hg * sb;
+            it.cnt = min(sb - it.st0, g1 - g0);
+            const int start = stage_pre[b] + it.hg * sb;
+            it.nparts = cp.parts(start, sb);
+            it.part = cp.of(g0) - cp.of(start);
+            it.prow = prow_pre[b];
+            for (int h = 0; h < it.hg; ++h) {
+                const int n = cp.parts(stage_pre[b] + h * sb, sb);
+                if (n > 1) it.prow += n * HS * g;
+            }
+            const int base = (it.st0 * NBS) & ~31;
+            it.tab0 = chunk_entry(b, base);
+            it.tab1 = chunk_entry(b, base + 32);
+            g0 += it.cnt;
+            return true;
+        };
+        PItem cur, nxt;
+        bool have = next_item(cur);
+        while (ok && have) {
+            const bool have_next = next_item(nxt);
+            const int b = cur.b, hg = cur.hg, c = s_ctx[b];
+            const int slot = n_item % kItemSlots;
+            if (n_item >= kItemSlots &&
+                !mbar_wait(&iempty[slot], (uint32_t)(n_item / kItemSlots - 1) & 1)) {
+                ok = false;
+                break;
+            }
+            if (lane == 0) {
+                ItemDesc &d = descs[slot];
+                d.b = b;
+                d.hg = hg;
+                d.c = c;
+                d.qs0 = s_qsl[b];
+                d.nparts = cur.nparts;
+                d.part = cur.part;
+                d.prow = cur.prow;
+                const uint32_t qb = (uint32_t)HS * g * D * 2;
+                mbar_arrive_expect_tx(&qfull[slot], qb);
+                bulk_load(sm + prm.off_q + slot * prm.qslot_bytes,
+                          prm.q + ((long long)s_qsl[b] * Hq + hg * HS * g) * D, qb, &qfull[slot]);
+            }
+            __syncwarp();
+            ++n_item;
+            // block table lookups: this lane holds entry cur_base + lane; the
+            // following 32 entries are in flight
+            int cur_base = (cur.st0 * NBS) & ~31, cur_tab = cur.tab0, nxt_tab = cur.tab1;
+            auto table_get = [&](int blk) -> int {
+                while (blk >= cur_base + 32) {
+                    cur_base += 32;
+                    cur_tab = nxt_tab;
+                    nxt_tab = chunk_entry(b, cur_base + 32);
                 }
-                const int c = s_ctx[b];
-                const int slot = n_item % kItemSlots;
-                if (n_item >= kItemSlots &&
-                    !mbar_wait(&iempty[slot], (uint32_t)(n_item / kItemSlots - 1) & 1)) {
+                int phys = __shfl_sync(0xffffffffu, cur_tab, blk - cur_base);
+                if (phys < 0 || phys >= prm.num_blocks) {
+                    if (lane == 0) record_error(prm.err, PK_ERR_BAD_INDEX);
+                    phys = 0;
+                }
+                return phys;
+            };
+            const int nblk = (c + bs - 1) / bs;
+            for (int st = cur.st0; st < cur.st0 + cur.cnt; ++st) {
+                const int s = n_stage % NS;
+                if (n_stage >= NS && !mbar_wait(&empty[s], ((n_stage / NS) - 1) & 1)) {
                     ok = false;
                     break;
                 }
+                const int blk0 = st * NBS;
+                const int np = min(NBS, nblk - blk0);  // blocks of this stage inside the context
                 if (lane == 0) {
-                    ItemDesc &d = descs[slot];
-                    d.b = b;
-                    d.hg = hg;
-                    d.c = c;
-                    d.qs0 = s_qsl[b];
-                    d.nparts = nparts;
-                    d.part = g0 / cs - start / cs;
-                    d.prow = prow;
-                    const uint32_t qb = (uint32_t)HS * g * D * 2;
-                    mbar_arrive_expect_tx(&qfull[slot], qb);
-                    bulk_load(sm + prm.off_q + slot * prm.qslot_bytes,
-                              prm.q + ((long long)s_qsl[b] * Hq + hg * HS * g) * D, qb, &qfull[slot]);
+                    StageInfo &inf = infos[s];
+                    inf.slot = slot;
+                    inf.st = st;
+                    inf.flags = (st == cur.st0 ? kFirst : 0) | (st == cur.st0 + cur.cnt - 1 ? kLast : 0);
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)np * piece_bytes * 2);
+                }
+                uint8_t *kst = sm + (size_t)s * prm.stage_bytes;
+                uint8_t *vst = kst + (size_t)NBS * piece_bytes;
+                for (int j = 0; j < np; ++j) {
+                    const int phys = table_get(blk0 + j);
+                    const int y = (phys * Hkv + hg * HS) * bs;
+                    if (lane == 0) {  // all panels of the block's rows: one box for K, one for V
+                        tma_load_3d(kst + j * piece_bytes, &tmk, 0, y, 0, &full[s]);
+                        tma_load_3d(vst + j * piece_bytes, &tmv, 0, y, 0, &full[s]);
+                    }
                 }
                 __syncwarp();
-                ++n_item;
-                // the sequence's block table from this partition's first block, 32 entries per lane chunk
-                t_b = b;
-                cur_base = (st0 * NBS) & ~31;
-                cur_tab = chunk_entry(b, cur_base);
-                nxt_tab = chunk_entry(b, cur_base + 32);
-                const int nblk = (c + bs - 1) / bs;
-                for (int st = st0; st < st0 + cnt; ++st) {
-                    const int s = n_stage % NS;
-                    if (n_stage >= NS && !mbar_wait(&empty[s], ((n_stage / NS) - 1) & 1)) {
-                        ok = false;
-                        break;
-                    }
-                    const int blk0 = st * NBS;
-                    const int np = min(NBS, nblk - blk0);  // blocks of this stage inside the context
-                    if (lane == 0) {
-                        StageInfo &inf = infos[s];
-                        inf.slot = slot;
-                        inf.st = st;
-                        inf.flags = (st == st0 ? kFirst : 0) | (st == st0 + cnt - 1 ? kLast : 0);
-                        mbar_arrive_expect_tx(&full[s], (uint32_t)np * piece_bytes * 2);
-                    }
-                    uint8_t *kst = sm + (size_t)s * prm.stage_bytes;
-                    uint8_t *vst = kst + (size_t)NBS * piece_bytes;
-                    for (int j = 0; j < np; ++j) {
-                        const int phys = table_get(blk0 + j);
-                        const int y = (phys * Hkv + hg * HS) * bs;
-                        if (lane == 0) {
-#pragma unroll
-                            for (int pn = 0; pn < NPN; ++pn) {
-                                tma_load_2d(kst + j * piece_bytes + pn * panel_bytes, &tmk, pn * 64, y, &full[s]);
-                                tma_load_2d(vst + j * piece_bytes + pn * panel_bytes, &tmv, pn * 64, y, &full[s]);
-                            }
-                        }
-                    }
-                    __syncwarp();
-                    ++n_stage;
-                }
-                g0 += cnt;
+                ++n_stage;
             }
+            cur = nxt;
+            have = have_next;
         }
         if (ok) {
             // end marker
@@ -422,42 +481,52 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
             row_of(tau0 + a_row, koff, ksw);
             row_of(tau0 + v_row, voff, vsw);
             const uint32_t ka = smem_u32(kst) + koff, va = smem_u32(vst) + voff;
-            float st[4] = {0.f, 0.f, 0.f, 0.f}, su[4] = {0.f, 0.f, 0.f, 0.f};
+            float sa[4][4] = {};
 #pragma unroll
             for (int kk = 0; kk < KS; ++kk) {
                 const int col = kk * 16 + a_col;
                 uint32_t a0, a1, a2, a3;
                 ldsm_x4(ka + (col >> 6) * panel_bytes + ((((col & 63) >> 3) ^ ksw) << 4), a0, a1, a2, a3);
-                if (kk & 1) mma_bf16(su, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
-                else mma_bf16(st, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+                mma_bf16(sa[kk & 3], a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
             }
-            // st[0], st[1]: token qr, heads qc, qc + 1; st[2], st[3]: token qr + 8
-            float s0 = (st[0] + su[0]) * prm.scale_log2, s1 = (st[1] + su[1]) * prm.scale_log2;
-            float s2 = (st[2] + su[2]) * prm.scale_log2, s3 = (st[3] + su[3]) * prm.scale_log2;
+            // four accumulator chains; s0, s1: token qr, heads qc, qc + 1; s2, s3: token qr + 8
+            auto sum4 = [&](int i) { return ((sa[0][i] + sa[1][i]) + (sa[2][i] + sa[3][i])) * prm.scale_log2; };
+            float s0 = sum4(0), s1 = sum4(1), s2 = sum4(2), s3 = sum4(3);
             if (qr >= valid) s0 = s1 = -INFINITY;
             if (qr + 8 >= valid) s2 = s3 = -INFINITY;
-            float ma = fmaxf(s0, s2), mb = fmaxf(s1, s3);
+            // Lazy rescaling: the running reference m moves (and O, l are
+            // rescaled) only when a score exceeds it by more than kRescaleLog2,
+            // so 2^(s - m) stays below 2^kRescaleLog2 (exact in the end: o = O / l
+            // and lse = m + log2 l hold for any reference).  The vote keeps the
+            // branch warp-uniform.
+            const float la = fmaxf(s0, s2), lb = fmaxf(s1, s3);
+            if (__any_sync(0xffffffffu, la > m0 + kRescaleLog2 || lb > m1 + kRescaleLog2)) {
+                float ma = la, mb = lb;
 #pragma unroll
-            for (int x = 4; x < 32; x <<= 1) {
-                ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, x));
-                mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, x));
+                for (int x = 4; x < 32; x <<= 1) {
+                    ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, x));
+                    mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, x));
+                }
+                const float na = fmaxf(m0, ma), nb = fmaxf(m1, mb);
+                const float ala = na == -INFINITY ? 1.f : fast_exp2(m0 - na);
+                const float alb = nb == -INFINITY ? 1.f : fast_exp2(m1 - nb);
+                m0 = na;
+                m1 = nb;
+                l0 *= ala;
+                l1 *= alb;
+#pragma unroll
+                for (int mt = 0; mt < KS; ++mt) {
+                    ot[mt][0] *= ala;
+                    ot[mt][1] *= alb;
+                    ot[mt][2] *= ala;
+                    ot[mt][3] *= alb;
+                }
             }
-            const float na = fmaxf(m0, ma), nb = fmaxf(m1, mb);
-            const float ba = na == -INFINITY ? 0.f : na, bb = nb == -INFINITY ? 0.f : nb;
-            const float ala = fast_exp2(m0 - ba), alb = fast_exp2(m1 - bb);
-            m0 = na;
-            m1 = nb;
+            const float ba = m0 == -INFINITY ? 0.f : m0, bb = m1 == -INFINITY ? 0.f : m1;
             const float p0 = fast_exp2(s0 - ba), p1 = fast_exp2(s1 - bb);
             const float p2 = fast_exp2(s2 - ba), p3 = fast_exp2(s3 - bb);
-            l0 = l0 * ala + p0 + p2;
-            l1 = l1 * alb + p1 + p3;
-#pragma unroll
-            for (int mt = 0; mt < KS; ++mt) {
-                ot[mt][0] *= ala;
-                ot[mt][1] *= alb;
-                ot[mt][2] *= ala;
-                ot[mt][3] *= alb;
-            }
+            l0 += p0 + p2;
+            l1 += p1 + p3;
             // P^T as the B fragment: transpose the two 8x8 (token x head) blocks
             const uint32_t b0 = movmatrix_trans(pack_bf16(p0, p1));
             const uint32_t b1 = movmatrix_trans(pack_bf16(p2, p3));
@@ -605,8 +674,13 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
 // (sequence, head group) that the streaming kernel cut into several
 // partitions, each output row (q head hg * HS * g + r of the sequence's token)
 // is out = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M), M = max_p lse_p, over
-// the partitions' normalised rows o_p and log2-sum-exps lse_p.  One thread per
-// (row, 4 columns); blockIdx.x = sequence * head groups + head group.
+// the partitions' normalised rows o_p and log2-sum-exps lse_p.
+// The streaming kernel lists the split pairs; an item is kMergeUnits (row,
+// 4 columns) outputs of one pair, and blocks stride over the items.  Each
+// output has kMergeSplit threads: thread s folds the
+// partitions s, s + kMergeSplit, ... eight at a time (all their loads issued
+// before the first is used), and the kMergeSplit partial folds are combined
+// through shared memory.
 struct MergeParams {
     __nv_bfloat16 *out;
     const int32_t *qsl;
@@ -616,52 +690,92 @@ struct MergeParams {
 };
 
 constexpr int kMergeThreads = 256;
+constexpr int kMergeSplit = 4;
+constexpr int kMergeUnits = kMergeThreads / kMergeSplit;
+constexpr int kMergeBatch = 8;
 
 template <int D>
 __global__ void __launch_bounds__(kMergeThreads) attention_merge_kernel(const MergeParams mp) {
     asm volatile("griddepcontrol.wait;" ::: "memory");  // the streaming kernel has finished
-    const int NHG = mp.n_kv_heads / mp.HS, HG = mp.HS * mp.group;
-    const int b = blockIdx.x / NHG, hg = blockIdx.x % NHG;
-    if (b >= mp.nseq) return;
-    const int *stage_pre = mp.mplan + kMergePlanHead, *prow_pre = stage_pre + kPlanLen;
-    const int cs = mp.mplan[0];
-    const int sb = (stage_pre[b + 1] - stage_pre[b]) / NHG;
-    if (sb == 0) return;
-    auto parts_of = [&](int start) { return (start + sb - 1) / cs - start / cs + 1; };
-    const int nparts = parts_of(stage_pre[b] + hg * sb);
-    if (nparts <= 1) return;
-    int prow = prow_pre[b];
-    for (int h = 0; h < hg; ++h) {
-        const int n = parts_of(stage_pre[b] + h * sb);
-        if (n > 1) prow += n * HG;
+    __shared__ float s_m[kMergeSplit][kMergeUnits], s_d[kMergeSplit][kMergeUnits];
+    __shared__ float4 s_a[kMergeSplit][kMergeUnits];
+    const int HG = mp.HS * mp.group;
+    const int nub = (HG * (D / 4) + kMergeUnits - 1) / kMergeUnits;  // unit blocks per pair
+    const int n_items = __ldcg(mp.mplan) * nub;
+    const int4 *list = (const int4 *)(mp.mplan + kMergeListHead);
+    const int u = threadIdx.x % kMergeUnits, sp = threadIdx.x / kMergeUnits;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const int4 e = __ldcg(list + item / nub);  // sequence, head group, first row, partitions
+        const int b = e.x, hg = e.y, prow = e.z, nparts = e.w;
+        const int unit = (item % nub) * kMergeUnits + u;
+        const bool live = unit < HG * (D / 4);
+        const int r = live ? unit / (D / 4) : 0, c4 = live ? unit % (D / 4) : 0;
+        const float *lse = mp.partial_lse + prow + r;
+        const float4 *po = (const float4 *)(mp.partial_o + (size_t)(prow + r) * D) + c4;
+        float M = -INFINITY, den = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int q0 = sp; live && q0 < nparts; q0 += kMergeSplit * kMergeBatch) {
+            float l[kMergeBatch];
+            float4 x[kMergeBatch];
+#pragma unroll
+            for (int i = 0; i < kMergeBatch; ++i) {
+                const int q = q0 + i * kMergeSplit;
+                l[i] = -INFINITY;
+                x[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (q < nparts) {
+                    l[i] = __ldcg(lse + (size_t)q * HG);
+                    x[i] = __ldcg(po + (size_t)q * HG * (D / 4));
+                }
+            }
+            float bm = M;
+#pragma unroll
+            for (int i = 0; i < kMergeBatch; ++i) bm = fmaxf(bm, l[i]);
+            if (bm == -INFINITY) continue;
+            const float a = M == -INFINITY ? 0.f : fast_exp2(M - bm);
+            den *= a;
+            acc.x *= a;
+            acc.y *= a;
+            acc.z *= a;
+            acc.w *= a;
+            M = bm;
+#pragma unroll
+            for (int i = 0; i < kMergeBatch; ++i) {
+                const float w = l[i] == -INFINITY ? 0.f : fast_exp2(l[i] - M);
+                den += w;
+                acc.x += w * x[i].x;
+                acc.y += w * x[i].y;
+                acc.z += w * x[i].z;
+                acc.w += w * x[i].w;
+            }
+        }
+        s_m[sp][u] = M;
+        s_d[sp][u] = den;
+        s_a[sp][u] = acc;
+        __syncthreads();
+        if (sp == 0 && live) {
+            float Mt = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < kMergeSplit; ++j) Mt = fmaxf(Mt, s_m[j][u]);
+            float dt = 0.f;
+            float4 at = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < kMergeSplit; ++j) {
+                const float w = s_m[j][u] == -INFINITY ? 0.f : fast_exp2(s_m[j][u] - Mt);
+                dt += w * s_d[j][u];
+                at.x += w * s_a[j][u].x;
+                at.y += w * s_a[j][u].y;
+                at.z += w * s_a[j][u].z;
+                at.w += w * s_a[j][u].w;
+            }
+            const float inv = dt > 0.f ? 1.f / dt : 0.f;
+            const long long orow = (long long)__ldg(mp.qsl + mp.seq0 + b) * mp.n_q_heads + hg * HG + r;
+            uint2 pk;
+            pk.x = pack_bf16(at.x * inv, at.y * inv);
+            pk.y = pack_bf16(at.z * inv, at.w * inv);
+            *(uint2 *)(mp.out + orow * D + c4 * 4) = pk;
+        }
+        __syncthreads();  // the shared arrays are rewritten by the next item
     }
-    const int unit = blockIdx.y * kMergeThreads + threadIdx.x;
-    if (unit >= HG * (D / 4)) return;
-    const int r = unit / (D / 4), c4 = unit % (D / 4);
-    const float *lse = mp.partial_lse + prow + r;
-    float M = -INFINITY;
-#pragma unroll 8
-    for (int q = 0; q < nparts; ++q) M = fmaxf(M, __ldcg(lse + (size_t)q * HG));
-    float den = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4 *po = (const float4 *)(mp.partial_o + (size_t)(prow + r) * D) + c4;
-#pragma unroll 8
-    for (int q = 0; q < nparts; ++q) {
-        const float l = __ldcg(lse + (size_t)q * HG);
-        const float4 x = __ldcg(po + (size_t)q * HG * (D / 4));
-        const float w = l == -INFINITY ? 0.f : fast_exp2(l - M);
-        den += w;
-        acc.x += w * x.x;
-        acc.y += w * x.y;
-        acc.z += w * x.z;
-        acc.w += w * x.w;
-    }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    const long long orow = (long long)__ldg(mp.qsl + mp.seq0 + b) * mp.n_q_heads + hg * HG + r;
-    uint2 pk;
-    pk.x = pack_bf16(acc.x * inv, acc.y * inv);
-    pk.y = pack_bf16(acc.z * inv, acc.w * inv);
-    *(uint2 *)(mp.out + orow * D + c4 * 4) = pk;
 }
 
 template <int D>
@@ -729,9 +843,8 @@ int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, cudaSt
         mp.n_kv_heads = tp.n_kv_heads;
         mp.group = tp.group;
         mp.HS = tp.HS;
-        const int units = tp.HS * tp.group * (D / 4);
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(tp.nseq * (tp.n_kv_heads / tp.HS), (units + kMergeThreads - 1) / kMergeThreads);
+        cfg.gridDim = dim3(2 * p->sm_count);
         cfg.blockDim = dim3(kMergeThreads);
         cfg.dynamicSmemBytes = 0;
         cfg.stream = st;
@@ -776,12 +889,12 @@ int decode_blocks_prepare_pool(pk_pool *p) {
         default: rc = blocks_prepare<256>(p); break;
     }
     if (rc != PK_OK) return rc;
-    rc = encode_pool_map(&p->tmap_kb, p->k_base, p, p->blk_hs * bs);
-    if (rc == PK_OK) rc = encode_pool_map(&p->tmap_vb, p->v_base, p, p->blk_hs * bs);
+    rc = encode_pool_map3(&p->tmap_kb, p->k_base, p, p->blk_hs * bs);
+    if (rc == PK_OK) rc = encode_pool_map3(&p->tmap_vb, p->v_base, p, p->blk_hs * bs);
     return rc;
 }
 
-int decode_blocks_chunks_per_cta() { return kChunksPerCta; }
+int decode_blocks_chunks_per_cta() { return 1 + kSmallPerCta; }
 
 bool decode_blocks_applies(const pk_pool *p, const AttnArgs &a) {
     return p->blk_ok && a.num_tokens == a.num_seqs && a.n_q_heads / p->n_kv_heads <= 8;

@@ -42,8 +42,8 @@ Layout layout(const pk_pool *p, int num_seqs, int n_q_heads) {
     size_t off = 2 * kHeaderBytes;
     L.counters = off;
     off = align_up(off + (size_t)kMaxSeqsPerLaunch * Hkv * sizeof(int), 256);
-    L.merge_plan = off;  // 8 ints, then two arrays of kMaxSeqsPerLaunch + 1
-    off = align_up(off + (size_t)(8 + 2 * (kMaxSeqsPerLaunch + 1)) * sizeof(int), 256);
+    L.merge_plan = off;  // a count, then an int4 per split (sequence, head group)
+    off = align_up(off + (size_t)(4 + 4 * kMaxSeqsPerLaunch * Hkv) * sizeof(int), 256);
     L.partial_lse = off;
     off = align_up(off + (size_t)L.cap_rows * sizeof(float), 256);
     L.partial_o = off;

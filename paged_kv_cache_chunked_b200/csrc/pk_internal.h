@@ -27,7 +27,7 @@ struct pk_pool {
     int blk_smem_max;     // its largest dynamic shared memory per launch
     alignas(64) CUtensorMap tmap_k;
     alignas(64) CUtensorMap tmap_v;
-    alignas(64) CUtensorMap tmap_kb;  // boxes of blk_hs * block_size rows (whole blocks)
+    alignas(64) CUtensorMap tmap_kb;  // 3-D boxes of blk_hs * block_size rows, all panels
     alignas(64) CUtensorMap tmap_vb;
 };
 
@@ -92,6 +92,8 @@ bool decode_blocks_applies(const pk_pool *p, const AttnArgs &a);
 int launch_decode_blocks(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, cudaStream_t st);
 // 2-D TMA view of a pool (rows of head_dim bf16) with boxes of 64 columns x box_rows.
 int encode_pool_map(CUtensorMap *map, void *base, const pk_pool *p, int box_rows);
+// 3-D TMA view (column in panel, row, 64-column panel) with boxes of all panels x box_rows.
+int encode_pool_map3(CUtensorMap *map, void *base, const pk_pool *p, int box_rows);
 int chunk_prepare_pool(pk_pool *p);
 int launch_chunk(const pk_pool *p, const AttnArgs &a, void *header, cudaStream_t st);
 
