@@ -36,7 +36,11 @@ from paged_kv_cache_chunked_b200.workloads import WORKLOADS, workload_batch  # n
 
 METRIC = "paged decode attention KV GB/s (% of HBM peak) and tokens/s per scheduler step"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SRC = os.path.join(ROOT, "paged_kv_cache_chunked_b200", "csrc", "attention_decode.cu")
+CSRC = os.path.join(ROOT, "paged_kv_cache_chunked_b200", "csrc")
+# the source of each workload's dominant kernel (the traffic record is valid for that source only)
+KERNEL_SRC = {"chunk512_bf16": os.path.join(CSRC, "attention_chunk.cu"),
+              "append_copy": os.path.join(CSRC, "kv_copy.cu")}
+DECODE_SRC = os.path.join(CSRC, "attention_decode_blocks.cu")
 
 
 def parse():
@@ -47,7 +51,7 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="decode64_bf16",
                    choices=["decode64_bf16", "longdoc_bf16", "chunk512_bf16", "trace", "fork",
-                            "fork1028"])
+                            "fork1028", "append_copy"])
     p.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--profile-run", action="store_true",
@@ -168,7 +172,7 @@ def kernel_traffic(workload):
             rec = json.load(f)
     except (OSError, ValueError):
         return None
-    with open(KERNEL_SRC, "rb") as f:
+    with open(KERNEL_SRC.get(workload, DECODE_SRC), "rb") as f:
         src_hash = hashlib.sha256(f.read()).hexdigest()[:16]
     entry = rec.get(workload)
     if not entry or entry.get("kernel_sha256_16") != src_hash:
@@ -209,6 +213,9 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     import oracle
+    if args.workload == "append_copy":
+        run_reference_kvops(args, world)
+        return
     batch = workload_batch(args.workload, poison_unused=False)
     slots = last_token_slots(batch)
     k_new, v_new = new_token_kv(batch, slots)
@@ -253,6 +260,39 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_reference_kvops(args, world):
+    """The oracle's append + block copy on the host, each step 1/16 of the
+    append_copy workload (4,096 tokens, 128 block pairs)."""
+    import oracle
+    w = KVOPS
+    slots, k, v, pairs = kvops_inputs()
+    n, m = w["tokens"] // 16, w["pairs"] // 16
+    kp = torch.zeros(w["num_blocks"], w["n_kv_heads"], w["block_size"], w["head_dim"], dtype=torch.bfloat16)
+    vp = torch.zeros_like(kp)
+    app_b, copy_b = kvops_bytes()
+
+    def step():
+        oracle.kv_append(kp, vp, k[:n], v[:n], slots[:n])
+        oracle.block_copy(kp, vp, pairs[:m])
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = (app_b + copy_b) / 16 / dt / 1e9
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "append_copy", **w, "l2": "oracle on host cores: L2 not applicable"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: oracle kv_append of {n} tokens + block_copy of {m} blocks"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 def measured_tensor_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -265,7 +305,10 @@ def measured_tensor_peak():
 def roofline_entry(workload, attn_b, flops, avg_ms, gbs, tflops, hbm_peak, hbm_kind):
     """The attention call's roofline: HBM for decode (about 4 flop/byte at GQA 4),
     the tensor pipe for prefill chunks (a dense contraction)."""
-    common = {"kernel": "paged_attention call (decode kernel; chunk kernel when chunks are present)",
+    kern = ("paged_attention call: chunk kernel + tile-streaming decode kernel"
+            if workload == "chunk512_bf16" else
+            "paged_attention call: block-streaming decode kernel + split-K merge kernel")
+    common = {"kernel": kern,
               "algorithmic_bytes": attn_b, "algorithmic_flops": flops, "avg_ms": avg_ms,
               "traffic": kernel_traffic(workload)}
     if workload == "chunk512_bf16":
@@ -319,12 +362,16 @@ def run_ours(args, rank, world, device):
         if ev is not None:
             ev[1].record(stream)
 
-    # append + one decode kernel per window of 512 sequences, plus the chunk
-    # kernel when the step holds prefill chunks (the general kernel: one launch)
+    # append, then per window of 512 sequences: for a batch of decodes only
+    # (groups of <= 8 q heads) the block-streaming kernel and its merge kernel,
+    # else the chunk kernel (when chunks are present) and the tile-streaming
+    # decode kernel; the general kernel is one launch
     tc = pool.dtype == torch.bfloat16 and d in (64, 128, 256) and bs % 8 == 0
     B = batch["context_lens"].shape[0]
     windows = (B + 511) // 512
-    launches_per_step = 1 + ((windows * (2 if T > B else 1)) if tc else 1)
+    blocks_path = tc and T == B and Hq // Hkv <= 8
+    per_window = 2 if blocks_path else (2 if T > B or Hq // Hkv > 16 else 1)
+    launches_per_step = 1 + (windows * per_window if tc else 1)
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize(device)
@@ -444,6 +491,162 @@ def run_ours(args, rank, world, device):
     print(json.dumps(line), flush=True)
 
 
+# KV append and block copy alone, at sizes well above L2: 65,536 new tokens
+# written to distinct random slots of a decode-64-shaped pool (8 kv heads, head
+# dim 128, 16-token blocks, bf16), then 2,048 whole blocks copied (the
+# copy-on-write step of a fork).
+KVOPS = dict(num_blocks=9594, n_kv_heads=8, block_size=16, head_dim=128, tokens=65536, pairs=2048,
+             seed=1007)
+
+
+def kvops_inputs():
+    w = KVOPS
+    g = torch.Generator().manual_seed(w["seed"])
+    N, H, bs, d = w["num_blocks"], w["n_kv_heads"], w["block_size"], w["head_dim"]
+    T = w["tokens"]
+    slots = torch.randperm(N * bs, generator=g)[:T]
+    k = torch.randn(T, H, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(T, H, d, generator=g).to(torch.bfloat16)
+    perm = torch.randperm(N, generator=g)
+    pairs = torch.stack([perm[:w["pairs"]], perm[w["pairs"]:2 * w["pairs"]]], 1).to(torch.int32)
+    return slots, k, v, pairs
+
+
+def kvops_bytes():
+    w = KVOPS
+    tok = w["n_kv_heads"] * w["head_dim"] * 2  # one token's K (or V) row set, bf16
+    append = 2 * (2 * w["tokens"] * tok) + 8 * w["tokens"]  # read new K, V; write them; slots
+    blk = w["n_kv_heads"] * w["block_size"] * w["head_dim"] * 2 * 2  # K + V of one block
+    copy = 2 * w["pairs"] * blk + 8 * w["pairs"]  # read + write each block; the pairs
+    return append, copy
+
+
+def run_kvops(args, rank, world, device):
+    from paged_kv_cache_chunked_b200 import api
+    w = KVOPS
+    slots, k, v, pairs = kvops_inputs()
+    app_b, copy_b = kvops_bytes()
+    pool = api.kv_pool_create(w["num_blocks"], w["block_size"], w["n_kv_heads"], w["head_dim"],
+                              torch.bfloat16, device)
+    ds, dk, dv, dp = slots.to(device), k.to(device), v.to(device), pairs.to(device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        api.paged_kv_append(dk, dv, ds, pool=pool)
+        if ev is not None:
+            ev[1].record(stream)
+        api.block_copy(dp, pool=pool)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(device)
+    assert pool.check_device_errors() == 0
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    if not args.profile_run:
+        clocks.start()
+        time.sleep(0.3)
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as tdist
+        tdist.barrier()
+    torch.cuda.synchronize(device)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    total_ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([total_ms], device=device)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    t_extra = time.perf_counter()
+    while not args.profile_run and time.perf_counter() - t_extra < 1.0:
+        for _ in range(20):
+            step()
+        torch.cuda.synchronize(device)
+    clk = clocks.stop() if not args.profile_run else {"sm_mhz": None, "reasons": ["not sampled"]}
+    assert pool.check_device_errors() == 0
+    app_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in evs)
+    copy_ms = statistics.mean(b.elapsed_time(c) for _, b, c in evs)
+    ms_per_step = total_ms / args.steps
+    value = world * (app_b + copy_b) / (ms_per_step * 1e-3) / 1e9
+
+    e2e = None
+    if not args.no_e2e and not args.profile_run:
+        hs, hk, hv, hp = (x.pin_memory() for x in (slots, k, v, pairs))
+        h_out = torch.empty(w["n_kv_heads"], w["block_size"], w["head_dim"], dtype=torch.bfloat16).pin_memory()
+        bufs = [torch.empty_like(x, device=device) for x in (hs, hk, hv, hp)]
+        h2d = sum(x.numel() * x.element_size() for x in (hs, hk, hv, hp))
+        d2h = h_out.numel() * h_out.element_size()
+        dst0 = int(pairs[0, 1])
+
+        def e2e_step():
+            for dst, src in zip(bufs, (hs, hk, hv, hp)):
+                dst.copy_(src, non_blocking=True)
+            api.paged_kv_append(bufs[1], bufs[2], bufs[0], pool=pool)
+            api.block_copy(bufs[3], pool=pool)
+            h_out.copy_(pool.k_pool[dst0], non_blocking=True)  # one copied block back
+
+        for _ in range(3):
+            e2e_step()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(device)
+        s2.record(stream)
+        n_e2e = max(1, min(args.steps, 200))
+        for _ in range(n_e2e):
+            e2e_step()
+        e2.record(stream)
+        torch.cuda.synchronize(device)
+        e_ms = s2.elapsed_time(e2) / n_e2e
+        e2e = {"value": world * (app_b + copy_b) / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    if rank != 0:
+        return
+    peak, peak_kind = measured_peak()
+    ach = app_b / (app_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "append_copy", **{k_: v_ for k_, v_ in w.items()},
+                   "l2": "no flush: each step moves 0.8 GB, more than the 126 MB L2",
+                   "parallelism": "replicas"},
+        "pct_hbm": 100.0 * value / world / peak,
+        "append_gbs": ach, "copy_gbs": copy_b / (copy_ms * 1e-3) / 1e9,
+        "roofline": {"kernel": "kv_append (paged_kv_append of 65,536 tokens)", "bound": "hbm",
+                     "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                     "algorithmic_bytes": app_b, "avg_ms": app_ms, "traffic": kernel_traffic("append_copy"),
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": dict(clk, window="the timed region plus 1 s of the same steps right after it"),
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if world == 1 and args.cpu_baseline_seconds > 0 and not args.profile_run:
+        import oracle
+        n = 4096  # bounded sample: 1/16 of the tokens, 1/16 of the pairs
+        kp = torch.zeros(w["num_blocks"], w["n_kv_heads"], w["block_size"], w["head_dim"],
+                         dtype=torch.bfloat16)
+        vp = torch.zeros_like(kp)
+        runs, t0 = 0, time.perf_counter()
+        while runs < 1 or time.perf_counter() - t0 < args.cpu_baseline_seconds:
+            oracle.kv_append(kp, vp, k[:n], v[:n], slots[:n])
+            oracle.block_copy(kp, vp, pairs[:w["pairs"] // 16])
+            runs += 1
+        sec = (time.perf_counter() - t0) / runs
+        line["cpu_baseline"] = {"value": (app_b + copy_b) / 16 / sec / 1e9, "unit": "GB/s", "cores": 1,
+                                "kind": "oracle",
+                                "sample": f"oracle kv_append of {n} tokens + block_copy of "
+                                          f"{w['pairs'] // 16} blocks (1/16 of a step), {runs} runs"}
+    print(json.dumps(line), flush=True)
+
+
 def run_serving(args, rank, world, device):
     """Scheduler-driven workloads: the continuous-batching trace (300
     iterations, Poisson arrivals, chunked prefill, preemption) or n-sample
@@ -522,6 +725,8 @@ def main():
     try:
         if args.workload in ("trace", "fork", "fork1028"):
             run_serving(args, rank, world, device)
+        elif args.workload == "append_copy":
+            run_kvops(args, rank, world, device)
         else:
             run_ours(args, rank, world, device)
     finally:
