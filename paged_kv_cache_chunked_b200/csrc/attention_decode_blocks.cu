@@ -135,6 +135,9 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
     constexpr int KS = D / 16;
     constexpr int NPN = D / 64;  // 64-column panels
     extern __shared__ uint8_t smem_raw[];
+    // launched as a programmatic dependent of the previous kernel on the stream
+    // (the KV append): nothing is read before that grid has finished
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int NS = prm.NS, HS = prm.HS, NBS = prm.NBS, ST = prm.ST, NPH = prm.NPH;
@@ -675,107 +678,75 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
 // partitions, each output row (q head hg * HS * g + r of the sequence's token)
 // is out = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M), M = max_p lse_p, over
 // the partitions' normalised rows o_p and log2-sum-exps lse_p.
-// The streaming kernel lists the split pairs; an item is kMergeUnits (row,
-// 4 columns) outputs of one pair, and blocks stride over the items.  Each
-// output has kMergeSplit threads: thread s folds the
-// partitions s, s + kMergeSplit, ... eight at a time (all their loads issued
-// before the first is used), and the kMergeSplit partial folds are combined
-// through shared memory.
+// The streaming kernel lists the split pairs.  blockIdx.x = list entry,
+// blockIdx.y = a block of kMergeThreads outputs (row, 4 columns) of that
+// pair; one thread per output folds the partitions eight at a time, all of a
+// batch's loads issued before the first is used.  No shared memory, no
+// barrier: a block past the list's end returns at once.
 struct MergeParams {
     __nv_bfloat16 *out;
     const int32_t *qsl;
     const int *mplan;
     const float *partial_o, *partial_lse;
-    int seq0, nseq, n_q_heads, n_kv_heads, group, HS;
+    int seq0, n_q_heads, group, HS;
 };
 
 constexpr int kMergeThreads = 256;
-constexpr int kMergeSplit = 4;
-constexpr int kMergeUnits = kMergeThreads / kMergeSplit;
 constexpr int kMergeBatch = 8;
 
 template <int D>
 __global__ void __launch_bounds__(kMergeThreads) attention_merge_kernel(const MergeParams mp) {
     asm volatile("griddepcontrol.wait;" ::: "memory");  // the streaming kernel has finished
-    __shared__ float s_m[kMergeSplit][kMergeUnits], s_d[kMergeSplit][kMergeUnits];
-    __shared__ float4 s_a[kMergeSplit][kMergeUnits];
     const int HG = mp.HS * mp.group;
-    const int nub = (HG * (D / 4) + kMergeUnits - 1) / kMergeUnits;  // unit blocks per pair
-    const int n_items = __ldcg(mp.mplan) * nub;
-    const int4 *list = (const int4 *)(mp.mplan + kMergeListHead);
-    const int u = threadIdx.x % kMergeUnits, sp = threadIdx.x / kMergeUnits;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const int4 e = __ldcg(list + item / nub);  // sequence, head group, first row, partitions
-        const int b = e.x, hg = e.y, prow = e.z, nparts = e.w;
-        const int unit = (item % nub) * kMergeUnits + u;
-        const bool live = unit < HG * (D / 4);
-        const int r = live ? unit / (D / 4) : 0, c4 = live ? unit % (D / 4) : 0;
-        const float *lse = mp.partial_lse + prow + r;
-        const float4 *po = (const float4 *)(mp.partial_o + (size_t)(prow + r) * D) + c4;
-        float M = -INFINITY, den = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int q0 = sp; live && q0 < nparts; q0 += kMergeSplit * kMergeBatch) {
-            float l[kMergeBatch];
-            float4 x[kMergeBatch];
+    const int unit = blockIdx.y * kMergeThreads + threadIdx.x;
+    const int n_split = __ldcg(mp.mplan);
+    const int4 e = __ldcg((const int4 *)(mp.mplan + kMergeListHead) + blockIdx.x);
+    if ((int)blockIdx.x >= n_split || unit >= HG * (D / 4)) return;
+    const int b = e.x, hg = e.y, prow = e.z, nparts = e.w;  // sequence, head group, first row, partitions
+    const int r = unit / (D / 4), c4 = unit % (D / 4);
+    const float *lse = mp.partial_lse + prow + r;
+    const float4 *po = (const float4 *)(mp.partial_o + (size_t)(prow + r) * D) + c4;
+    float M = -INFINITY, den = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q0 = 0; q0 < nparts; q0 += kMergeBatch) {
+        float l[kMergeBatch];
+        float4 x[kMergeBatch];
 #pragma unroll
-            for (int i = 0; i < kMergeBatch; ++i) {
-                const int q = q0 + i * kMergeSplit;
-                l[i] = -INFINITY;
-                x[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (q < nparts) {
-                    l[i] = __ldcg(lse + (size_t)q * HG);
-                    x[i] = __ldcg(po + (size_t)q * HG * (D / 4));
-                }
-            }
-            float bm = M;
-#pragma unroll
-            for (int i = 0; i < kMergeBatch; ++i) bm = fmaxf(bm, l[i]);
-            if (bm == -INFINITY) continue;
-            const float a = M == -INFINITY ? 0.f : fast_exp2(M - bm);
-            den *= a;
-            acc.x *= a;
-            acc.y *= a;
-            acc.z *= a;
-            acc.w *= a;
-            M = bm;
-#pragma unroll
-            for (int i = 0; i < kMergeBatch; ++i) {
-                const float w = l[i] == -INFINITY ? 0.f : fast_exp2(l[i] - M);
-                den += w;
-                acc.x += w * x[i].x;
-                acc.y += w * x[i].y;
-                acc.z += w * x[i].z;
-                acc.w += w * x[i].w;
+        for (int i = 0; i < kMergeBatch; ++i) {
+            l[i] = -INFINITY;
+            x[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (q0 + i < nparts) {
+                l[i] = __ldcg(lse + (size_t)(q0 + i) * HG);
+                x[i] = __ldcg(po + (size_t)(q0 + i) * HG * (D / 4));
             }
         }
-        s_m[sp][u] = M;
-        s_d[sp][u] = den;
-        s_a[sp][u] = acc;
-        __syncthreads();
-        if (sp == 0 && live) {
-            float Mt = -INFINITY;
+        float bm = M;
 #pragma unroll
-            for (int j = 0; j < kMergeSplit; ++j) Mt = fmaxf(Mt, s_m[j][u]);
-            float dt = 0.f;
-            float4 at = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < kMergeBatch; ++i) bm = fmaxf(bm, l[i]);
+        if (bm == -INFINITY) continue;
+        const float a = M == -INFINITY ? 0.f : fast_exp2(M - bm);
+        den *= a;
+        acc.x *= a;
+        acc.y *= a;
+        acc.z *= a;
+        acc.w *= a;
+        M = bm;
 #pragma unroll
-            for (int j = 0; j < kMergeSplit; ++j) {
-                const float w = s_m[j][u] == -INFINITY ? 0.f : fast_exp2(s_m[j][u] - Mt);
-                dt += w * s_d[j][u];
-                at.x += w * s_a[j][u].x;
-                at.y += w * s_a[j][u].y;
-                at.z += w * s_a[j][u].z;
-                at.w += w * s_a[j][u].w;
-            }
-            const float inv = dt > 0.f ? 1.f / dt : 0.f;
-            const long long orow = (long long)__ldg(mp.qsl + mp.seq0 + b) * mp.n_q_heads + hg * HG + r;
-            uint2 pk;
-            pk.x = pack_bf16(at.x * inv, at.y * inv);
-            pk.y = pack_bf16(at.z * inv, at.w * inv);
-            *(uint2 *)(mp.out + orow * D + c4 * 4) = pk;
+        for (int i = 0; i < kMergeBatch; ++i) {
+            const float w = l[i] == -INFINITY ? 0.f : fast_exp2(l[i] - M);
+            den += w;
+            acc.x += w * x[i].x;
+            acc.y += w * x[i].y;
+            acc.z += w * x[i].z;
+            acc.w += w * x[i].w;
         }
-        __syncthreads();  // the shared arrays are rewritten by the next item
     }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    const long long orow = (long long)__ldg(mp.qsl + mp.seq0 + b) * mp.n_q_heads + hg * HG + r;
+    uint2 pk;
+    pk.x = pack_bf16(acc.x * inv, acc.y * inv);
+    pk.y = pack_bf16(acc.z * inv, acc.w * inv);
+    *(uint2 *)(mp.out + orow * D + c4 * 4) = pk;
 }
 
 template <int D>
@@ -830,7 +801,20 @@ int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, cudaSt
     for (int s0 = 0; s0 < a.num_seqs; s0 += kMaxSeqsPerLaunch) {
         tp.seq0 = s0;
         tp.nseq = std::min(kMaxSeqsPerLaunch, a.num_seqs - s0);
-        attention_decode_blocks_kernel<D><<<tp.ncta, kBlkThreads, tp.total, st>>>(p->tmap_kb, p->tmap_vb, tp);
+        {
+            cudaLaunchConfig_t c0 = {};
+            c0.gridDim = dim3(tp.ncta);
+            c0.blockDim = dim3(kBlkThreads);
+            c0.dynamicSmemBytes = tp.total;
+            c0.stream = st;
+            cudaLaunchAttribute a0[1];
+            a0[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            a0[0].val.programmaticStreamSerializationAllowed = 1;
+            c0.attrs = a0;
+            c0.numAttrs = 1;
+            const cudaError_t e0 = cudaLaunchKernelEx(&c0, attention_decode_blocks_kernel<D>, p->tmap_kb, p->tmap_vb, tp);
+            if (e0 != cudaSuccess) return cuda_fail(e0, "decode attention launch");
+        }
         MergeParams mp;
         mp.out = tp.out;
         mp.qsl = tp.qsl;
@@ -838,13 +822,14 @@ int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, cudaSt
         mp.partial_o = tp.partial_o;
         mp.partial_lse = tp.partial_lse;
         mp.seq0 = tp.seq0;
-        mp.nseq = tp.nseq;
         mp.n_q_heads = tp.n_q_heads;
-        mp.n_kv_heads = tp.n_kv_heads;
         mp.group = tp.group;
         mp.HS = tp.HS;
+        const int units = tp.HS * tp.group * (D / 4);
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(2 * p->sm_count);
+        // one block row per possible split pair (sequence, head group); blocks past
+        // the list's end return at once
+        cfg.gridDim = dim3(tp.nseq * (tp.n_kv_heads / tp.HS), (units + kMergeThreads - 1) / kMergeThreads);
         cfg.blockDim = dim3(kMergeThreads);
         cfg.dynamicSmemBytes = 0;
         cfg.stream = st;

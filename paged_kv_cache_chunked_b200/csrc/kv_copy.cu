@@ -28,6 +28,9 @@ __global__ void kv_append_vec16(const uint4 *__restrict__ k, const uint4 *__rest
                                 const int64_t *__restrict__ slots, int num_tokens, int n_kv_heads,
                                 int block_size, int row_chunks, int64_t num_slots,
                                 int *err) {
+    // a dependent kernel (attention launched with programmatic serialisation)
+    // may start its launch now; it waits for this grid before reading
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t per_side = (int64_t)num_tokens * n_kv_heads * row_chunks;
     const int64_t total = 2 * per_side;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
@@ -58,6 +61,9 @@ __global__ void kv_append_scalar(const T *__restrict__ k, const T *__restrict__ 
                                  const int64_t *__restrict__ slots, int num_tokens,
                                  int n_kv_heads, int block_size, int head_dim,
                                  int64_t num_slots, int *err) {
+    // a dependent kernel (attention launched with programmatic serialisation)
+    // may start its launch now; it waits for this grid before reading
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t per_side = (int64_t)num_tokens * n_kv_heads * head_dim;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < 2 * per_side;
          i += (int64_t)gridDim.x * blockDim.x) {
@@ -82,6 +88,9 @@ __global__ void kv_append_scalar(const T *__restrict__ k, const T *__restrict__ 
 // One CTA per (pair, K or V); the block's bytes are copied as 16-byte vectors.
 __global__ void block_copy_vec16(uint4 *kp, uint4 *vp, const int32_t *__restrict__ pairs,
                                  int n_pairs, int64_t block_chunks, int num_blocks, int *err) {
+    // a dependent kernel (attention launched with programmatic serialisation)
+    // may start its launch now; it waits for this grid before reading
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     for (int64_t w = blockIdx.x; w < 2LL * n_pairs; w += gridDim.x) {
         const int pr = (int)(w >> 1);
         uint4 *pool = (w & 1) ? vp : kp;
@@ -110,6 +119,9 @@ __global__ void block_copy_vec16(uint4 *kp, uint4 *vp, const int32_t *__restrict
 template <typename T>
 __global__ void block_copy_scalar(T *kp, T *vp, const int32_t *__restrict__ pairs, int n_pairs,
                                   int64_t block_elems, int num_blocks, int *err) {
+    // a dependent kernel (attention launched with programmatic serialisation)
+    // may start its launch now; it waits for this grid before reading
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     for (int64_t w = blockIdx.x; w < 2LL * n_pairs; w += gridDim.x) {
         const int pr = (int)(w >> 1);
         T *pool = (w & 1) ? vp : kp;
