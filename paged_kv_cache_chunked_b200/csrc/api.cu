@@ -137,9 +137,16 @@ int pk_pool_create(int num_blocks, int block_size, int n_kv_heads, int head_dim,
     p->tc_path = dtype == PK_BF16 && (head_dim == 64 || head_dim == 128 || head_dim == 256) &&
                  block_size % 8 == 0 && rows < (1LL << 31) && !force_generic();
     if (p->tc_path) {
+        // 16-token tiles of one (block, kv head): one 3-D box brings all head-dim
+        // panels when a tile lies in one block (block_size a multiple of 16);
+        // else two 2-D boxes of 8 rows per panel
         const int box = block_size % kTile == 0 ? kTile : 8;
-        int rc = encode_pool_map(&p->tmap_k, k_base, p, box);
-        if (rc == PK_OK) rc = encode_pool_map(&p->tmap_v, v_base, p, box);
+        p->tile_map3d = box == kTile;
+        int rc = p->tile_map3d ? encode_pool_map3(&p->tmap_k, k_base, p, box)
+                               : encode_pool_map(&p->tmap_k, k_base, p, box);
+        if (rc == PK_OK)
+            rc = p->tile_map3d ? encode_pool_map3(&p->tmap_v, v_base, p, box)
+                               : encode_pool_map(&p->tmap_v, v_base, p, box);
         if (rc == PK_OK) rc = tc_prepare_pool(p);
         if (rc != PK_OK) {
             cudaFree(p->d_err);

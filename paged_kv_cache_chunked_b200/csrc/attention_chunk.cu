@@ -85,6 +85,7 @@ struct ChunkParams {
     const int32_t *ctx, *qsl;
     int seq0, nseq;
     int max_blocks, n_q_heads, n_kv_heads, group, block_size, box_rows, num_blocks, num_tokens;
+    bool map3d;  // tensor maps are 3-D: one box per 16-row tile
     float scale_log2;
     WsHeader *hdr;
     int *err;
@@ -236,7 +237,11 @@ attention_chunk_kernel(const __grid_constant__ CUtensorMap tmk,
                     mbar_arrive_expect_tx(&full[stage], (uint32_t)nsub * 2 * (D / 64) * box * 128);
                     uint8_t *ks = sm + L::kRing + (size_t)stage * L::kStageBytes;
                     uint8_t *vs = ks + 32 * D;
-                    for (int sb = 0; sb < nsub; ++sb) {
+                    if (prm.map3d) {  // one box per tile: 16 rows of every panel
+                        tma_load_3d(ks, &tmk, 0, y0, 0, &full[stage]);
+                        tma_load_3d(vs, &tmv, 0, y0, 0, &full[stage]);
+                    }
+                    for (int sb = 0; sb < (prm.map3d ? 0 : nsub); ++sb) {
                         const int y = sb == 0 ? y0 : y1;
 #pragma unroll
                         for (int pn = 0; pn < D / 64; ++pn) {
@@ -500,6 +505,7 @@ int chunk_launch_t(const pk_pool *p, const AttnArgs &a, void *header, cudaStream
     tp.group = a.n_q_heads / p->n_kv_heads;
     tp.block_size = p->block_size;
     tp.box_rows = p->block_size % kTile == 0 ? kTile : 8;
+    tp.map3d = p->tile_map3d;
     tp.num_blocks = p->num_blocks;
     tp.num_tokens = a.num_tokens;
     tp.scale_log2 = a.scale * 1.4426950408889634f;

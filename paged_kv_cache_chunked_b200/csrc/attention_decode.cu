@@ -88,6 +88,7 @@ struct DecParams {
     int seq0, nseq;
     int max_blocks, n_q_heads, n_kv_heads, group, block_size, box_rows, num_blocks, num_tokens;
     int ncta, cap_rows;
+    bool map3d;  // tensor maps are 3-D: one box per 16-row tile
     float scale_log2;
     WsHeader *hdr;
     int *counters;                   // per (sequence in the window, kv head)
@@ -259,7 +260,11 @@ attention_decode_kernel(const __grid_constant__ CUtensorMap tmk,
             mbar_arrive_expect_tx(&full[stage], (uint32_t)nsub * 2 * (D / 64) * box * 128);
             uint8_t *ks = ring + (size_t)stage * L::kStageBytes;
             uint8_t *vs = ks + 32 * D;
-            for (int sb = 0; sb < nsub; ++sb) {
+            if (prm.map3d) {  // one box per tile: 16 rows of every panel
+                tma_load_3d(ks, &tmk, 0, y0, 0, &full[stage]);
+                tma_load_3d(vs, &tmv, 0, y0, 0, &full[stage]);
+            }
+            for (int sb = 0; sb < (prm.map3d ? 0 : nsub); ++sb) {
                 const int y = sb == 0 ? y0 : y1;
 #pragma unroll
                 for (int pn = 0; pn < D / 64; ++pn) {
@@ -683,6 +688,7 @@ static int dec_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, cu
     tp.group = a.n_q_heads / p->n_kv_heads;
     tp.block_size = p->block_size;
     tp.box_rows = p->block_size % kTile == 0 ? kTile : 8;
+    tp.map3d = p->tile_map3d;
     tp.num_blocks = p->num_blocks;
     tp.num_tokens = a.num_tokens;
     tp.ncta = p->tc_ctas;

@@ -22,6 +22,7 @@ struct pk_pool {
     bool tc_path;       // tensor-core + TMA attention applies to this geometry
     int tc_ctas;        // resident CTAs of the decode attention kernel (whole GPU)
     int tc_ctas_chunk;  // resident CTAs of the chunk attention kernel (whole GPU)
+    bool tile_map3d;    // tmap_k / tmap_v are 3-D (16-row boxes of all panels), else 2-D (8 rows)
     bool blk_ok;        // the block-streaming decode kernel serves this geometry
     int blk_hs, blk_nbs;  // its kv heads and blocks per pipeline stage
     int blk_smem_max;     // its largest dynamic shared memory per launch
