@@ -31,6 +31,8 @@ constexpr int kTagAll = 15;  // stage consumed by every consumer warp
 constexpr int kTagEnd = -1;  // no more stages
 constexpr int kFirst = 1, kLast = 2;
 
+constexpr float kRescaleLog2 = 8.f;  // lazy softmax rescale threshold (log2 units)
+
 template <int D>
 struct ChunkCfg;
 // One CTA per SM with 7 consumer warps: each KV tile that the producer warp
@@ -374,7 +376,9 @@ attention_chunk_kernel(const __grid_constant__ CUtensorMap tmk,
                 __syncwarp();
             }
             const uint32_t ka = smem_u32(ks), va = smem_u32(vs), qa = smem_u32(qpriv);
+            // two accumulator chains per 8-key half (even / odd k-steps)
             float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            float sd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
             for (int kk = 0; kk < KS; ++kk) {
                 uint32_t a0, a1, a2, a3;
@@ -388,8 +392,13 @@ attention_chunk_kernel(const __grid_constant__ CUtensorMap tmk,
                 }
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4(ka + swz(k_row, kk * 16 + k_col), b0, b1, b2, b3);
-                mma_bf16(sc[0], a0, a1, a2, a3, b0, b1);
-                mma_bf16(sc[1], a0, a1, a2, a3, b2, b3);
+                if (kk & 1) {
+                    mma_bf16(sd[0], a0, a1, a2, a3, b0, b1);
+                    mma_bf16(sd[1], a0, a1, a2, a3, b2, b3);
+                } else {
+                    mma_bf16(sc[0], a0, a1, a2, a3, b0, b1);
+                    mma_bf16(sc[1], a0, a1, a2, a3, b2, b3);
+                }
             }
             const int key0 = kt * kTile + qc;
             const bool full_tile = kt * kTile + kTile - 1 <= min(lim0, lim1);
@@ -398,7 +407,7 @@ attention_chunk_kernel(const __grid_constant__ CUtensorMap tmk,
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    float s = sc[nt][i] * prm.scale_log2;
+                    float s = (sc[nt][i] + sd[nt][i]) * prm.scale_log2;
                     if (!full_tile) {
                         const int key = key0 + nt * 8 + (i & 1);
                         if (key > (i < 2 ? lim0 : lim1)) s = -INFINITY;
@@ -406,15 +415,31 @@ attention_chunk_kernel(const __grid_constant__ CUtensorMap tmk,
                     sc[nt][i] = s;
                     if (i < 2) mx0 = fmaxf(mx0, s); else mx1 = fmaxf(mx1, s);
                 }
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-            const float b0 = mn0 == -INFINITY ? 0.f : mn0, b1 = mn1 == -INFINITY ? 0.f : mn1;
-            const float al0 = fast_exp2(m0 - b0), al1 = fast_exp2(m1 - b1);
-            m0 = mn0;
-            m1 = mn1;
+            // Lazy rescaling: the row reference m moves (and O, l are rescaled) only
+            // when a score exceeds it by more than kRescaleLog2, so 2^(s - m) stays
+            // below 2^kRescaleLog2; o = O / l and lse are exact for any reference.
+            // The vote keeps the branch warp-uniform.
+            if (__any_sync(0xffffffffu, mx0 > m0 + kRescaleLog2 || mx1 > m1 + kRescaleLog2)) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+                const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+                const float al0 = mn0 == -INFINITY ? 1.f : fast_exp2(m0 - mn0);
+                const float al1 = mn1 == -INFINITY ? 1.f : fast_exp2(m1 - mn1);
+                m0 = mn0;
+                m1 = mn1;
+                l0 *= al0;
+                l1 *= al1;
+#pragma unroll
+                for (int n = 0; n < D / 8; ++n) {
+                    o[n][0] *= al0;
+                    o[n][1] *= al0;
+                    o[n][2] *= al1;
+                    o[n][3] *= al1;
+                }
+            }
+            const float b0 = m0 == -INFINITY ? 0.f : m0, b1 = m1 == -INFINITY ? 0.f : m1;
             float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
@@ -425,15 +450,8 @@ attention_chunk_kernel(const __grid_constant__ CUtensorMap tmk,
                 ps0 += sc[nt][0] + sc[nt][1];
                 ps1 += sc[nt][2] + sc[nt][3];
             }
-            l0 = l0 * al0 + ps0;
-            l1 = l1 * al1 + ps1;
-#pragma unroll
-            for (int n = 0; n < D / 8; ++n) {
-                o[n][0] *= al0;
-                o[n][1] *= al0;
-                o[n][2] *= al1;
-                o[n][3] *= al1;
-            }
+            l0 += ps0;
+            l1 += ps1;
             const uint32_t p0 = pack_bf16(sc[0][0], sc[0][1]), p1 = pack_bf16(sc[0][2], sc[0][3]);
             const uint32_t p2 = pack_bf16(sc[1][0], sc[1][1]), p3 = pack_bf16(sc[1][2], sc[1][3]);
 #pragma unroll
