@@ -59,6 +59,14 @@ DECODE_CASES = [
     ([21, 400], 16, 1, 128, 16),      # group of 16
     ([30, 250], 32, 1, 128, 16),      # group of 32: two row tiles per token
     ([64, 1000], 8, 8, 128, 16),      # group of 1
+    # decode batches on the block-streaming kernel: every stage geometry
+    ([30, 700, 2000], 8, 1, 128, 16),   # one kv head: eight phases per head, 8 blocks a stage
+    ([100, 1500, 7], 2, 1, 64, 16),     # one kv head, d 64: 16 blocks a stage
+    ([300, 50, 1200], 8, 2, 128, 16),   # two kv heads: four phases per head
+    ([100, 800], 24, 6, 128, 16),       # six kv heads: three head groups of two
+    ([500, 77], 32, 16, 64, 16),        # sixteen kv heads: two head groups of eight
+    ([200, 3000], 4, 2, 256, 64),       # block 64, d 256: one head a stage
+    ([90, 1000], 8, 8, 128, 256),       # block 256: too big for a stage, tile kernel instead
 ]
 
 
@@ -85,6 +93,14 @@ def test_bf16_chunked_prefill_mixed_with_decode(cuda_dev, ctx, ql, Hq, Hkv, d, b
     b = make_batch(ctx, ql, block_size=bs, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d,
                    dtype=torch.bfloat16, seed=7 + sum(ql))
     _check(b, Hq, Hkv, d, torch.bfloat16, cuda_dev, f"chunks {ctx}/{ql}")
+
+
+def test_decode_batch_over_several_launch_windows(cuda_dev):
+    # 600 sequences: the kernels take 512 sequences a launch, so two windows
+    ctx = [1 + (i * 37) % 90 for i in range(600)]
+    b = make_batch(ctx, None, block_size=16, n_q_heads=8, n_kv_heads=2, head_dim=64,
+                   dtype=torch.bfloat16, seed=77)
+    _check(b, 8, 2, 64, torch.bfloat16, cuda_dev, "600 sequences")
 
 
 def test_permuted_block_ids_bit_identical(cuda_dev):
