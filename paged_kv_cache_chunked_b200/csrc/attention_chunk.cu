@@ -9,13 +9,14 @@
 // tokens at context c sits at position c - q + i and attends to keys 0..c-q+i
 // of its kv head, each key read through the sequence's block table.
 //
-// Structure.  A work item is NC row tiles (16 rows each: pairs (query token,
-// head of the group), token-major) of one (sequence, kv head).  One producer
-// warp per CTA claims items from a global counter, stages each consumer
-// warp's Q rows by bulk copy, and streams every visible 16-token KV tile of
-// the item by TMA through a ring of shared-memory stages; all NC consumer
-// warps compute on every stage, each for its own 16 rows (the KV tile is read
-// from L2/HBM once per NC row tiles), masking causally by its own rows.
+// Structure.  A work item is NC x RT row tiles (16 rows each: pairs (query
+// token, head of the group), token-major) of one (sequence, kv head).  One
+// producer warp per CTA claims items from a global counter, stages each
+// consumer warp's Q rows by bulk copy, and streams every visible 16-token KV
+// tile of the item by TMA through a ring of shared-memory stages; all NC
+// consumer warps compute on every stage, each for its own RT row tiles (the KV
+// tile is loaded once per NC x RT row tiles, and each warp loads its K and V
+// fragments once for its RT tiles), masking causally by its own rows.
 // S = Q K^T and O += P V run on mma.sync m16n8k16 with an online softmax in
 // fp32 registers.  Bounded waits as in the decode kernel.
 #include "tc_common.cuh"
@@ -35,23 +36,24 @@ constexpr float kRescaleLog2 = 8.f;  // lazy softmax rescale threshold (log2 uni
 
 template <int D>
 struct ChunkCfg;
-// One CTA per SM with 7 consumer warps: each KV tile that the producer warp
-// loads feeds 7 row tiles (112 query rows), so one issuing warp per SM (about
-// 14 GB/s of tile loads) keeps the tensor pipe busier than 2 CTAs of 3.
-// Eight warps keep 255 registers per thread available.
+// One CTA per SM with 7 consumer warps of RT row tiles each: every KV tile
+// the producer warp loads feeds 7 x RT row tiles (224 query rows at RT = 2).
+// The producer's TMA issue rate, not the tensor pipe, bounds this kernel, so
+// the rows a tile feeds set its speed.  Eight warps keep 255 registers per
+// thread available; at RT = 2 the Q fragments come from shared memory.
 template <>
 struct ChunkCfg<64> {
-    static constexpr int kStages = 24, kMinBlocks = 1, kConsumers = 7;
-    static constexpr bool kQReg = true;
+    static constexpr int kStages = 16, kMinBlocks = 1, kConsumers = 7, kRowTiles = 2;
+    static constexpr bool kQReg = false;
 };
 template <>
 struct ChunkCfg<128> {
-    static constexpr int kStages = 20, kMinBlocks = 1, kConsumers = 7;
-    static constexpr bool kQReg = true;
+    static constexpr int kStages = 12, kMinBlocks = 1, kConsumers = 7, kRowTiles = 2;
+    static constexpr bool kQReg = false;
 };
 template <>
 struct ChunkCfg<256> {
-    static constexpr int kStages = 8, kMinBlocks = 1, kConsumers = 4;
+    static constexpr int kStages = 8, kMinBlocks = 1, kConsumers = 4, kRowTiles = 1;
     static constexpr bool kQReg = false;
 };
 
@@ -67,8 +69,9 @@ struct ChunkSmem {
     static constexpr int kStageBytes = 64 * D;
     static constexpr size_t kRing = 0;
     static constexpr size_t kQStage = kRing + (size_t)C::kStages * kStageBytes;
-    static constexpr size_t kQPriv = kQStage + (size_t)C::kConsumers * 32 * D;
-    static constexpr size_t kPlan = kQPriv + (C::kQReg ? 0 : (size_t)C::kConsumers * 32 * D);
+    static constexpr size_t kQPriv = kQStage + (size_t)C::kConsumers * C::kRowTiles * 32 * D;
+    static constexpr size_t kPlan =
+        kQPriv + (C::kQReg ? 0 : (size_t)C::kConsumers * C::kRowTiles * 32 * D);
     static constexpr size_t kDesc = kPlan + align_up(5 * (size_t)kPlanLen * 4, 16);
     static constexpr size_t kBars = kDesc + align_up(C::kConsumers * sizeof(RowDesc), 16);
     static constexpr size_t kMeta = kBars + (size_t)(2 * C::kStages + 2 * C::kConsumers) * 8;
@@ -99,7 +102,7 @@ attention_chunk_kernel(const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmv, const ChunkParams prm) {
     using C = ChunkCfg<D>;
     using L = ChunkSmem<D>;
-    constexpr int S = C::kStages, NC = C::kConsumers;
+    constexpr int S = C::kStages, NC = C::kConsumers, RT = C::kRowTiles;
     constexpr int KS = D / 16;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -149,7 +152,7 @@ attention_chunk_kernel(const __grid_constant__ CUtensorMap tmk,
         a.n_kv_heads = Hkv;
         a.ncta = 1;
         a.items_per_cta = 1;
-        a.rows_group = NC;
+        a.rows_group = NC * RT;
         a.cap_rows = 1 << 30;  // split items are not this kernel's work
         a.err = nullptr;       // the decode kernel reports bad sequences
         const PlanTotals t = plan_window(a, pa, lane);
@@ -170,7 +173,7 @@ attention_chunk_kernel(const __grid_constant__ CUtensorMap tmk,
             const int kvh = local % Hkv, grp = local / Hkv;
             const int c = pa.s_ctx[b], qs0 = pa.s_qsl[b], qn = pa.s_qsl[b + 1] - qs0;
             const int rows_total = qn * g;
-            const int last_row = min((grp + 1) * NC * kTile, rows_total) - 1;
+            const int last_row = min((grp + 1) * NC * RT * kTile, rows_total) - 1;
             const int kv_end = (c - qn + last_row / g) / kTile + 1;
             // Q rows and descriptor of each consumer warp's row tile
             for (int w = 0; w < NC && ok; ++w) {
@@ -179,8 +182,8 @@ attention_chunk_kernel(const __grid_constant__ CUtensorMap tmk,
                     break;
                 }
                 qphase ^= 1u << w;
-                const int tile = grp * NC + w, r0 = tile * kTile;
-                const int nrows = max(0, min(kTile, rows_total - r0));
+                const int tile = (grp * NC + w) * RT, r0 = tile * kTile;  // the warp's first row tile
+                const int nrows = max(0, min(RT * kTile, rows_total - r0));
                 if (lane == 0) {
                     RowDesc &d = descs[w];
                     d.seq = prm.seq0 + b;
@@ -199,7 +202,7 @@ attention_chunk_kernel(const __grid_constant__ CUtensorMap tmk,
                     const int t_first = r0 / g, t_last = (r0 + nrows - 1) / g;
                     for (int t = t_first + lane; t <= t_last; t += 32) {
                         const int ra = max(r0, t * g), rb = min(r0 + nrows, (t + 1) * g);
-                        bulk_load(sm + L::kQStage + (size_t)w * 32 * D + (size_t)(ra - r0) * D * 2,
+                        bulk_load(sm + L::kQStage + (size_t)w * RT * 32 * D + (size_t)(ra - r0) * D * 2,
                                   prm.q + ((long long)(qs0 + t) * Hq + kvh * g + (ra - t * g)) * D,
                                   (uint32_t)(rb - ra) * D * 2, &qfull[w]);
                     }
@@ -286,17 +289,19 @@ attention_chunk_kernel(const __grid_constant__ CUtensorMap tmk,
         const int k_row = (mi >> 1) * 8 + rr, k_col = (mi & 1) * 8;
         const int v_row = (mi & 1) * 8 + rr, v_col = (mi >> 1) * 8;
         const int q_row = (mi & 1) * 8 + rr, q_col = (mi >> 1) * 8;
-        const uint8_t *qstage = sm + L::kQStage + (size_t)w * 32 * D;
-        uint8_t *qpriv = sm + L::kQPriv + (size_t)w * 32 * D;
+        const uint8_t *qstage = sm + L::kQStage + (size_t)w * RT * 32 * D;
+        uint8_t *qpriv = sm + L::kQPriv + (size_t)w * RT * 32 * D;  // RT swizzled 16-row tiles
 
         int stage = 0;
         uint32_t phase = 0, qph = 0;
         bool active = false, ok = true;
-        int c = 0, max_lim = 0, lim0 = 0, lim1 = 0;
-        long long orow0 = -1, orow1 = -1;
+        int c = 0, max_lim = 0;
+        // per row tile t: rows qr and qr + 8 (limits, output rows, softmax state)
+        int lim0[RT], lim1[RT];
+        long long orow0[RT], orow1[RT];
         uint32_t qf[C::kQReg ? KS : 1][4];
-        float o[D / 8][4];
-        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+        float o[RT][D / 8][4];
+        float m0[RT], m1[RT], l0[RT], l1[RT];
 
         auto begin_item = [&]() {
             if (!mbar_wait(&qfull[w], qph)) {
@@ -308,59 +313,69 @@ attention_chunk_kernel(const __grid_constant__ CUtensorMap tmk,
             active = d.tile >= 0;
             c = d.c;
             const int rows = d.rows, qn = d.qn;
-            const int tile = max(d.tile, 0);
-            const int r0 = tile * kTile + qr, r1 = r0 + 8;
-            // rows past the last query row compute garbage that is never written
-            lim0 = r0 < rows ? c - qn + r0 / g : c - 1;
-            lim1 = r1 < rows ? c - qn + r1 / g : c - 1;
-            max_lim = c - qn + (min(tile * kTile + kTile, rows) - 1) / g;
-            orow0 = active && r0 < rows ? (long long)(d.qs0 + r0 / g) * Hq + d.kvh * g + r0 % g : -1;
-            orow1 = active && r1 < rows ? (long long)(d.qs0 + r1 / g) * Hq + d.kvh * g + r1 % g : -1;
-            const int nvalid = active ? min(kTile, rows - tile * kTile) : 0;
-            if constexpr (C::kQReg) {
-                const uint8_t *q0 = qstage + qr * D * 2, *q1 = qstage + (qr + 8) * D * 2;
+            const int tile0 = max(d.tile, 0);
+            max_lim = c - qn + (min((tile0 + RT) * kTile, rows) - 1) / g;
 #pragma unroll
-                for (int ks = 0; ks < KS; ++ks) {
-                    const int col = (ks * 16 + qc) * 2;
-                    qf[ks][0] = qr < nvalid ? *(const uint32_t *)(q0 + col) : 0u;
-                    qf[ks][1] = qr + 8 < nvalid ? *(const uint32_t *)(q1 + col) : 0u;
-                    qf[ks][2] = qr < nvalid ? *(const uint32_t *)(q0 + col + 16) : 0u;
-                    qf[ks][3] = qr + 8 < nvalid ? *(const uint32_t *)(q1 + col + 16) : 0u;
+            for (int t = 0; t < RT; ++t) {
+                const int tile = tile0 + t;
+                const int r0 = tile * kTile + qr, r1 = r0 + 8;
+                // rows past the last query row compute garbage that is never written
+                lim0[t] = r0 < rows ? c - qn + r0 / g : c - 1;
+                lim1[t] = r1 < rows ? c - qn + r1 / g : c - 1;
+                orow0[t] = active && r0 < rows ? (long long)(d.qs0 + r0 / g) * Hq + d.kvh * g + r0 % g : -1;
+                orow1[t] = active && r1 < rows ? (long long)(d.qs0 + r1 / g) * Hq + d.kvh * g + r1 % g : -1;
+                const int nvalid = active ? max(0, min(kTile, rows - tile * kTile)) : 0;
+                const uint8_t *qs = qstage + (size_t)t * 32 * D;
+                if constexpr (C::kQReg) {
+                    const uint8_t *q0 = qs + qr * D * 2, *q1 = qs + (qr + 8) * D * 2;
+#pragma unroll
+                    for (int ks = 0; ks < KS; ++ks) {
+                        const int col = (ks * 16 + qc) * 2;
+                        qf[ks][0] = qr < nvalid ? *(const uint32_t *)(q0 + col) : 0u;
+                        qf[ks][1] = qr + 8 < nvalid ? *(const uint32_t *)(q1 + col) : 0u;
+                        qf[ks][2] = qr < nvalid ? *(const uint32_t *)(q0 + col + 16) : 0u;
+                        qf[ks][3] = qr + 8 < nvalid ? *(const uint32_t *)(q1 + col + 16) : 0u;
+                    }
+                } else {
+                    uint8_t *qp = qpriv + (size_t)t * 32 * D;
+                    for (int ch = lane; ch < 16 * (D / 8); ch += 32) {
+                        const int row = ch / (D / 8), col = (ch % (D / 8)) * 8;
+                        uint4 v = make_uint4(0, 0, 0, 0);
+                        if (row < nvalid) v = *(const uint4 *)(qs + (row * D + col) * 2);
+                        *(uint4 *)(qp + swz(row, col)) = v;
+                    }
                 }
-            } else {
-                for (int ch = lane; ch < 16 * (D / 8); ch += 32) {
-                    const int row = ch / (D / 8), col = (ch % (D / 8)) * 8;
-                    uint4 v = make_uint4(0, 0, 0, 0);
-                    if (row < nvalid) v = *(const uint4 *)(qstage + (row * D + col) * 2);
-                    *(uint4 *)(qpriv + swz(row, col)) = v;
-                }
+#pragma unroll
+                for (int n = 0; n < D / 8; ++n) o[t][n][0] = o[t][n][1] = o[t][n][2] = o[t][n][3] = 0.f;
+                m0[t] = m1[t] = -INFINITY;
+                l0[t] = l1[t] = 0.f;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&qempty[w]);
-#pragma unroll
-            for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-            m0 = m1 = -INFINITY;
-            l0 = l1 = 0.f;
         };
 
         auto finish_item = [&]() {
             if (!active) return;
-            l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-            l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-            l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-            l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-            const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
-            if (orow0 >= 0) {
-                __nv_bfloat16 *dst = prm.out + orow0 * D;
 #pragma unroll
-                for (int n = 0; n < D / 8; ++n)
-                    *(uint32_t *)(dst + n * 8 + qc) = pack_bf16(o[n][0] * inv0, o[n][1] * inv0);
-            }
-            if (orow1 >= 0) {
-                __nv_bfloat16 *dst = prm.out + orow1 * D;
+            for (int t = 0; t < RT; ++t) {
+                float a0 = l0[t], a1 = l1[t];
+                a0 += __shfl_xor_sync(0xffffffffu, a0, 1);
+                a0 += __shfl_xor_sync(0xffffffffu, a0, 2);
+                a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
+                a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
+                const float inv0 = a0 > 0.f ? 1.f / a0 : 0.f, inv1 = a1 > 0.f ? 1.f / a1 : 0.f;
+                if (orow0[t] >= 0) {
+                    __nv_bfloat16 *dst = prm.out + orow0[t] * D;
 #pragma unroll
-                for (int n = 0; n < D / 8; ++n)
-                    *(uint32_t *)(dst + n * 8 + qc) = pack_bf16(o[n][2] * inv1, o[n][3] * inv1);
+                    for (int n = 0; n < D / 8; ++n)
+                        *(uint32_t *)(dst + n * 8 + qc) = pack_bf16(o[t][n][0] * inv0, o[t][n][1] * inv0);
+                }
+                if (orow1[t] >= 0) {
+                    __nv_bfloat16 *dst = prm.out + orow1[t] * D;
+#pragma unroll
+                    for (int n = 0; n < D / 8; ++n)
+                        *(uint32_t *)(dst + n * 8 + qc) = pack_bf16(o[t][n][2] * inv1, o[t][n][3] * inv1);
+                }
             }
         };
 
@@ -376,90 +391,109 @@ attention_chunk_kernel(const __grid_constant__ CUtensorMap tmk,
                 __syncwarp();
             }
             const uint32_t ka = smem_u32(ks), va = smem_u32(vs), qa = smem_u32(qpriv);
-            // two accumulator chains per 8-key half (even / odd k-steps)
-            float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            float sd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            // S = Q K^T per row tile; each K fragment serves all RT tiles; two
+            // accumulator chains per 8-key half (even / odd k-steps)
+            float sc[RT][2][4], sd[RT][2][4];
+#pragma unroll
+            for (int t = 0; t < RT; ++t)
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) sc[t][h][i] = sd[t][h][i] = 0.f;
 #pragma unroll
             for (int kk = 0; kk < KS; ++kk) {
-                uint32_t a0, a1, a2, a3;
-                if constexpr (C::kQReg) {
-                    a0 = qf[kk][0];
-                    a1 = qf[kk][1];
-                    a2 = qf[kk][2];
-                    a3 = qf[kk][3];
-                } else {
-                    ldsm_x4(qa + swz(q_row, kk * 16 + q_col), a0, a1, a2, a3);
-                }
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4(ka + swz(k_row, kk * 16 + k_col), b0, b1, b2, b3);
-                if (kk & 1) {
-                    mma_bf16(sd[0], a0, a1, a2, a3, b0, b1);
-                    mma_bf16(sd[1], a0, a1, a2, a3, b2, b3);
-                } else {
-                    mma_bf16(sc[0], a0, a1, a2, a3, b0, b1);
-                    mma_bf16(sc[1], a0, a1, a2, a3, b2, b3);
+#pragma unroll
+                for (int t = 0; t < RT; ++t) {
+                    uint32_t a0, a1, a2, a3;
+                    if constexpr (C::kQReg) {
+                        a0 = qf[kk][0];
+                        a1 = qf[kk][1];
+                        a2 = qf[kk][2];
+                        a3 = qf[kk][3];
+                    } else {
+                        ldsm_x4(qa + t * 32 * D + swz(q_row, kk * 16 + q_col), a0, a1, a2, a3);
+                    }
+                    if (kk & 1) {
+                        mma_bf16(sd[t][0], a0, a1, a2, a3, b0, b1);
+                        mma_bf16(sd[t][1], a0, a1, a2, a3, b2, b3);
+                    } else {
+                        mma_bf16(sc[t][0], a0, a1, a2, a3, b0, b1);
+                        mma_bf16(sc[t][1], a0, a1, a2, a3, b2, b3);
+                    }
                 }
             }
             const int key0 = kt * kTile + qc;
-            const bool full_tile = kt * kTile + kTile - 1 <= min(lim0, lim1);
-            float mx0 = -INFINITY, mx1 = -INFINITY;
+            uint32_t pf[RT][4];  // P as A fragments, per row tile
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+            for (int t = 0; t < RT; ++t) {
+                const bool full_tile = kt * kTile + kTile - 1 <= min(lim0[t], lim1[t]);
+                float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float s = (sc[nt][i] + sd[nt][i]) * prm.scale_log2;
-                    if (!full_tile) {
-                        const int key = key0 + nt * 8 + (i & 1);
-                        if (key > (i < 2 ? lim0 : lim1)) s = -INFINITY;
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        float sv = (sc[t][nt][i] + sd[t][nt][i]) * prm.scale_log2;
+                        if (!full_tile) {
+                            const int key = key0 + nt * 8 + (i & 1);
+                            if (key > (i < 2 ? lim0[t] : lim1[t])) sv = -INFINITY;
+                        }
+                        sc[t][nt][i] = sv;
+                        if (i < 2) mx0 = fmaxf(mx0, sv); else mx1 = fmaxf(mx1, sv);
                     }
-                    sc[nt][i] = s;
-                    if (i < 2) mx0 = fmaxf(mx0, s); else mx1 = fmaxf(mx1, s);
-                }
-            // Lazy rescaling: the row reference m moves (and O, l are rescaled) only
-            // when a score exceeds it by more than kRescaleLog2, so 2^(s - m) stays
-            // below 2^kRescaleLog2; o = O / l and lse are exact for any reference.
-            // The vote keeps the branch warp-uniform.
-            if (__any_sync(0xffffffffu, mx0 > m0 + kRescaleLog2 || mx1 > m1 + kRescaleLog2)) {
-                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-                const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-                const float al0 = mn0 == -INFINITY ? 1.f : fast_exp2(m0 - mn0);
-                const float al1 = mn1 == -INFINITY ? 1.f : fast_exp2(m1 - mn1);
-                m0 = mn0;
-                m1 = mn1;
-                l0 *= al0;
-                l1 *= al1;
+                // Lazy rescaling: the row reference m moves (and O, l are rescaled)
+                // only when a score exceeds it by more than kRescaleLog2, so
+                // 2^(s - m) stays below 2^kRescaleLog2; o = O / l is exact for any
+                // reference.  The vote keeps the branch warp-uniform.
+                if (__any_sync(0xffffffffu, mx0 > m0[t] + kRescaleLog2 || mx1 > m1[t] + kRescaleLog2)) {
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+                    const float mn0 = fmaxf(m0[t], mx0), mn1 = fmaxf(m1[t], mx1);
+                    const float al0 = mn0 == -INFINITY ? 1.f : fast_exp2(m0[t] - mn0);
+                    const float al1 = mn1 == -INFINITY ? 1.f : fast_exp2(m1[t] - mn1);
+                    m0[t] = mn0;
+                    m1[t] = mn1;
+                    l0[t] *= al0;
+                    l1[t] *= al1;
 #pragma unroll
-                for (int n = 0; n < D / 8; ++n) {
-                    o[n][0] *= al0;
-                    o[n][1] *= al0;
-                    o[n][2] *= al1;
-                    o[n][3] *= al1;
+                    for (int n = 0; n < D / 8; ++n) {
+                        o[t][n][0] *= al0;
+                        o[t][n][1] *= al0;
+                        o[t][n][2] *= al1;
+                        o[t][n][3] *= al1;
+                    }
                 }
-            }
-            const float b0 = m0 == -INFINITY ? 0.f : m0, b1 = m1 == -INFINITY ? 0.f : m1;
-            float ps0 = 0.f, ps1 = 0.f;
+                const float bb0 = m0[t] == -INFINITY ? 0.f : m0[t], bb1 = m1[t] == -INFINITY ? 0.f : m1[t];
+                float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                sc[nt][0] = fast_exp2(sc[nt][0] - b0);
-                sc[nt][1] = fast_exp2(sc[nt][1] - b0);
-                sc[nt][2] = fast_exp2(sc[nt][2] - b1);
-                sc[nt][3] = fast_exp2(sc[nt][3] - b1);
-                ps0 += sc[nt][0] + sc[nt][1];
-                ps1 += sc[nt][2] + sc[nt][3];
+                for (int nt = 0; nt < 2; ++nt) {
+                    sc[t][nt][0] = fast_exp2(sc[t][nt][0] - bb0);
+                    sc[t][nt][1] = fast_exp2(sc[t][nt][1] - bb0);
+                    sc[t][nt][2] = fast_exp2(sc[t][nt][2] - bb1);
+                    sc[t][nt][3] = fast_exp2(sc[t][nt][3] - bb1);
+                    ps0 += sc[t][nt][0] + sc[t][nt][1];
+                    ps1 += sc[t][nt][2] + sc[t][nt][3];
+                }
+                l0[t] += ps0;
+                l1[t] += ps1;
+                pf[t][0] = pack_bf16(sc[t][0][0], sc[t][0][1]);
+                pf[t][1] = pack_bf16(sc[t][0][2], sc[t][0][3]);
+                pf[t][2] = pack_bf16(sc[t][1][0], sc[t][1][1]);
+                pf[t][3] = pack_bf16(sc[t][1][2], sc[t][1][3]);
             }
-            l0 += ps0;
-            l1 += ps1;
-            const uint32_t p0 = pack_bf16(sc[0][0], sc[0][1]), p1 = pack_bf16(sc[0][2], sc[0][3]);
-            const uint32_t p2 = pack_bf16(sc[1][0], sc[1][1]), p3 = pack_bf16(sc[1][2], sc[1][3]);
+            // O += P V; each V fragment serves all RT tiles
 #pragma unroll
             for (int np = 0; np < KS; ++np) {
                 uint32_t v0, v1, v2, v3;
                 ldsm_x4_t(va + swz(v_row, np * 16 + v_col), v0, v1, v2, v3);
-                mma_bf16(o[2 * np], p0, p1, p2, p3, v0, v1);
-                mma_bf16(o[2 * np + 1], p0, p1, p2, p3, v2, v3);
+#pragma unroll
+                for (int t = 0; t < RT; ++t) {
+                    mma_bf16(o[t][2 * np], pf[t][0], pf[t][1], pf[t][2], pf[t][3], v0, v1);
+                    mma_bf16(o[t][2 * np + 1], pf[t][0], pf[t][1], pf[t][2], pf[t][3], v2, v3);
+                }
             }
         };
 
