@@ -64,6 +64,7 @@ int tc_prepare_pool(pk_pool *p) {
     int rc = decode_prepare_pool(p);
     if (rc == PK_OK) rc = decode_blocks_prepare_pool(p);
     if (rc == PK_OK) rc = chunk_prepare_pool(p);
+    if (rc == PK_OK) rc = chunk_umma_prepare_pool(p);
     return rc;
 }
 
@@ -78,7 +79,8 @@ int launch_attention_tc(const pk_pool *p, const AttnArgs &a, cudaStream_t st) {
     // heads) exceed one 16-row tile: a chunk of several tokens, or g > 16
     const int g = a.n_q_heads / p->n_kv_heads;
     if (a.num_tokens > a.num_seqs || g > kTile) {
-        const int rc = launch_chunk(p, a, ws + L.hdr_chunk, st);
+        const int rc = chunk_umma_applies(p, a) ? launch_chunk_umma(p, a, st)
+                                                : launch_chunk(p, a, ws + L.hdr_chunk, st);
         if (rc != PK_OK) return rc;
     }
     DecodeWs w;

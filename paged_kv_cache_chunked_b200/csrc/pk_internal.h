@@ -23,6 +23,7 @@ struct pk_pool {
     int tc_ctas;        // resident CTAs of the decode attention kernel (whole GPU)
     int tc_ctas_chunk;  // resident CTAs of the chunk attention kernel (whole GPU)
     bool tile_map3d;    // tmap_k / tmap_v are 3-D (16-row boxes of all panels), else 2-D (8 rows)
+    bool umma_ok;       // the tcgen05 chunk kernel serves this geometry
     bool blk_ok;        // the block-streaming decode kernel serves this geometry
     int blk_hs, blk_nbs;  // its kv heads and blocks per pipeline stage
     int blk_smem_max;     // its largest dynamic shared memory per launch
@@ -30,6 +31,7 @@ struct pk_pool {
     alignas(64) CUtensorMap tmap_v;
     alignas(64) CUtensorMap tmap_kb;  // 3-D boxes of blk_hs * block_size rows, all panels
     alignas(64) CUtensorMap tmap_vb;
+    alignas(64) CUtensorMap tmap_k2;  // 2-D, 16-row boxes: K tiles of the tcgen05 chunk kernel
 };
 
 namespace pk {
@@ -96,6 +98,10 @@ int encode_pool_map(CUtensorMap *map, void *base, const pk_pool *p, int box_rows
 // 3-D TMA view (column in panel, row, 64-column panel) with boxes of all panels x box_rows.
 int encode_pool_map3(CUtensorMap *map, void *base, const pk_pool *p, int box_rows);
 int chunk_prepare_pool(pk_pool *p);
+// tcgen05 chunk kernel (head_dim 128, block_size a multiple of 16, g dividing 128).
+int chunk_umma_prepare_pool(pk_pool *p);
+bool chunk_umma_applies(const pk_pool *p, const AttnArgs &a);
+int launch_chunk_umma(const pk_pool *p, const AttnArgs &a, cudaStream_t st);
 int launch_chunk(const pk_pool *p, const AttnArgs &a, void *header, cudaStream_t st);
 
 }  // namespace pk
