@@ -10,18 +10,20 @@
 // tokens at context c sits at position c - q + i and attends to keys 0..c-q+i
 // of its kv head, each key read through the sequence's block table.
 //
-// Structure.  A work item is 128 query rows (pairs (token, head of the
-// group), token-major) of one (sequence, kv head); CTA i takes items i,
-// i + gridDim.x, ...  Per 64-key stage:
-//   - four producer warps each load one 16-key block of the stage by TMA: K as
-//     two 2-D boxes (one per 64-column panel) into the canonical K-major
-//     128-byte-swizzled layout [panel][64 keys][128 B], V as one 3-D box
-//     [block][panel][16 keys][128 B];
-//   - one thread of the MMA warp issues S = Q K^T (M 128, N 64, eight K-steps
-//     of 16) into one of two tensor-memory buffers, then, when the softmax of
-//     the previous stage is done, O += P V (M 128, N 128, four K-steps; V read
-//     MN-major);
-//   - four softmax warps own one query row per thread: they read the row of S
+// Structure.  A work item is 256 query rows (pairs (token, head of the
+// group), token-major) of one (sequence, kv head), as two 128-row tiles; CTA i
+// takes items i, i + gridDim.x, ...  Per 64-key stage:
+//   - three producer warps load the stage's four 16-key blocks by TMA: K as two
+//     2-D boxes per block (one per 64-column panel; warps 0 and 1) into the
+//     canonical K-major 128-byte-swizzled layout [panel][64 keys][128 B], V as
+//     one 3-D box per block [block][panel][16 keys][128 B] (warp 2);
+//   - one thread of the MMA warp issues, per row tile, S = Q K^T (M 128, N 64,
+//     eight K-steps of 16) into one of two tensor-memory buffers, then, when
+//     both tiles' softmax of the previous stage are done, O += P V (M 128,
+//     N 128, four K-steps; V read MN-major);
+//   - per row tile, four softmax warps own one query row per thread (two
+//     warpgroups share each SM sub-partition and hide each other's latency):
+//     they read the row of S
 //     from tensor memory (no shuffles), mask causally, keep the running max m
 //     and sum l in fp32 (the reference m moves, and O is rescaled in tensor
 //     memory, only when a score exceeds it by more than 2^8), and write P as
@@ -40,29 +42,32 @@ namespace {
 using namespace tc;
 
 constexpr int kUD = 128;                // head dim
-constexpr int kURows = 128;             // query rows per item (UMMA M)
+constexpr int kURows = 128;             // query rows per row tile (UMMA M)
+constexpr int kUTiles = 2;              // row tiles per item: 256 query rows share each KV stage
+constexpr int kUItemRows = kURows * kUTiles;
 constexpr int kUKeys = 64;              // keys per stage
-constexpr int kUStages = 4;
-constexpr int kUProducers = 4;          // warps 0..3: one 16-key block of a stage each
-constexpr int kUSoft0 = 4;              // warps 4..7: softmax and epilogue
+constexpr int kUStages = 3;
 constexpr int kUMma = 8;                // warp 8: tensor memory and MMA issue
-constexpr int kUThreads = 9 * 32;
-constexpr uint32_t kUTmemCols = 256;    // S buffers at columns 0 and 64, O at 128
+constexpr int kUProd0 = 9;              // warps 9..11: producers (K panel 0, K panel 1, V)
+constexpr int kUProducers = 3;
+constexpr int kUThreads = 12 * 32;      // warps 0..3 and 4..7: softmax of row tile 0 and 1
+constexpr uint32_t kUTmemCols = 512;    // S[t][b] at 128 t + 64 b, O[t] at 256 + 128 t
 constexpr float kURescaleLog2 = 8.f;
 
-constexpr uint32_t kUQBytes = kURows * kUD * 2;       // [panel][128 rows][128 B]
+constexpr uint32_t kUQBytes = kURows * kUD * 2;       // per tile: [panel][128 rows][128 B]
 constexpr uint32_t kUKBytes = kUKeys * kUD * 2;       // [panel][64 keys][128 B]
 constexpr uint32_t kUVBytes = kUKeys * kUD * 2;       // [block][panel][16 keys][128 B]
 constexpr uint32_t kUStageBytes = kUKBytes + kUVBytes;
-constexpr uint32_t kUPBytes = kURows * kUKeys * 2;    // [128 rows][128 B]
+constexpr uint32_t kUPBytes = kURows * kUKeys * 2;    // per tile: [128 rows][128 B]
 constexpr uint32_t kUOffQ = 0;
-constexpr uint32_t kUOffKV = kUOffQ + kUQBytes;
+constexpr uint32_t kUOffKV = kUOffQ + kUTiles * kUQBytes;
 constexpr uint32_t kUOffP = kUOffKV + kUStages * kUStageBytes;
-constexpr uint32_t kUOffPlan = kUOffP + 2 * kUPBytes;
+constexpr uint32_t kUOffPlan = kUOffP + kUTiles * kUPBytes;
 constexpr uint32_t kUOffBar = kUOffPlan + (3 * kPlanLen * 4 + 15) / 16 * 16;
-// barriers: kv_full[stage][producer], kv_empty[stage], s_full[2], s_free[2],
-// p_full[2], pv_done[2], q_full, o_full, o_free, mma_done
-constexpr uint32_t kUNumBars = kUStages * kUProducers + kUStages + 8 + 4;
+// barriers: kv_full[stage][producer], kv_empty[stage]; per row tile: s_full[2],
+// s_free[2], p_full, pv_done, q_full, o_full, o_free; mma_done
+constexpr uint32_t kUPerTileBars = 9;
+constexpr uint32_t kUNumBars = kUStages * kUProducers + kUStages + kUTiles * kUPerTileBars + 1;
 constexpr uint32_t kUOffMisc = kUOffBar + kUNumBars * 8;  // tensor memory address, abort flag
 constexpr uint32_t kUSmem = kUOffMisc + 16 + 1024;        // + alignment slack
 
@@ -126,6 +131,11 @@ struct UItem {
     int b, kvh, rt, c, qn, qs0, rows, nkt;
 };
 
+// Per-row-tile barriers.
+struct UTileBars {
+    uint64_t *s_full, *s_free, *p_full, *pv_done, *q_full, *o_full, *o_free;
+};
+
 __global__ void __launch_bounds__(kUThreads, 1)
 attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D, 16-row boxes
                             const __grid_constant__ CUtensorMap tmv3,  // V: 3-D, 16 rows x 2 panels
@@ -140,14 +150,12 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
     int *s_ctx = s_qsl + kPlanLen;
     uint64_t *kv_full = (uint64_t *)(sm + kUOffBar);  // [stage][producer]
     uint64_t *kv_empty = kv_full + kUStages * kUProducers;
-    uint64_t *s_full = kv_empty + kUStages;
-    uint64_t *s_free = s_full + 2;
-    uint64_t *p_full = s_free + 2;
-    uint64_t *pv_done = p_full + 2;
-    uint64_t *q_full = pv_done + 2;
-    uint64_t *o_full = q_full + 1;
-    uint64_t *o_free = o_full + 1;
-    uint64_t *mma_done = o_free + 1;
+    uint64_t *tile_bars = kv_empty + kUStages;
+    uint64_t *mma_done = tile_bars + kUTiles * kUPerTileBars;
+    auto tb = [&](int t) {
+        uint64_t *q = tile_bars + t * kUPerTileBars;
+        return UTileBars{q, q + 2, q + 4, q + 5, q + 6, q + 7, q + 8};
+    };
     uint32_t *tmem_slot = (uint32_t *)(sm + kUOffMisc);
     volatile int *abort_flag = (volatile int *)(sm + kUOffMisc + 4);
     __shared__ int s_nitems;
@@ -155,15 +163,18 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
     if (threadIdx.x == 0) {
         for (int i = 0; i < kUStages * kUProducers; ++i) mbar_init(&kv_full[i], 1);
         for (int s = 0; s < kUStages; ++s) mbar_init(&kv_empty[s], 1);
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&s_full[b], 1);
-            mbar_init(&s_free[b], 4);
-            mbar_init(&p_full[b], 4);
-            mbar_init(&pv_done[b], 1);
+        for (int t = 0; t < kUTiles; ++t) {
+            const UTileBars B = tb(t);
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&B.s_full[b], 1);
+                mbar_init(&B.s_free[b], 4);
+            }
+            mbar_init(B.p_full, 4);
+            mbar_init(B.pv_done, 1);
+            mbar_init(B.q_full, 4);
+            mbar_init(B.o_full, 1);
+            mbar_init(B.o_free, 4);
         }
-        mbar_init(q_full, 4);
-        mbar_init(o_full, 1);
-        mbar_init(o_free, 4);
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -174,9 +185,9 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                      "r"(kUTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    if (warp == 0) {
+    if (warp == kUProd0) {
         // items: every sequence whose rows need more than one 16-row tile
-        // contributes ceil(rows / 128) row tiles per kv head
+        // contributes ceil(rows / 256) items per kv head
         int run = 0;
         for (int base = 0; base < nseq; base += 32) {
             const int i = base + lane;
@@ -190,7 +201,7 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                 const int qn = s1 - s0;
                 const bool ok = s0 >= 0 && s1 <= prm.num_tokens && qn >= 1 && c >= qn &&
                                 (long long)(c + bs - 1) / bs <= prm.max_blocks;
-                if (ok && qn * g > kTile) n = (qn * g + kURows - 1) / kURows * Hkv;
+                if (ok && qn * g > kTile) n = (qn * g + kUItemRows - 1) / kUItemRows * Hkv;
             }
             int inc = n;
 #pragma unroll
@@ -220,16 +231,17 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
         it.qn = s_qsl[b + 1] - it.qs0;
         it.c = s_ctx[b];
         it.rows = it.qn * g;
-        const int ntile = (it.rows + kURows - 1) / kURows;
-        it.kvh = local / ntile;
-        it.rt = local - it.kvh * ntile;
-        const int last_row = min((it.rt + 1) * kURows, it.rows) - 1;
+        const int nit = (it.rows + kUItemRows - 1) / kUItemRows;
+        it.kvh = local / nit;
+        it.rt = local - it.kvh * nit;
+        const int last_row = min((it.rt + 1) * kUItemRows, it.rows) - 1;
         it.nkt = (it.c - it.qn + last_row / g) / kUKeys + 1;
     };
 
-    if (warp < kUProducers) {
+    if (warp >= kUProd0) {
         // ------------------------------------------------------------ producers
-        const int p = warp;
+        // producer 0: K panel 0 of the stage's four 16-key blocks; 1: K panel 1; 2: V
+        const int p = warp - kUProd0;
         int n = 0;
         bool ok = true;
         for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
@@ -250,33 +262,42 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                     ok = false;
                     break;
                 }
-                const int k0 = j * kUKeys + p * kTile;  // this warp's 16 keys
-                int y = -1;
-                if (k0 < it.c) {
-                    const int blk = k0 / bs;
-                    while (blk >= base + 32) {
-                        base += 32;
-                        cur = nxt;
-                        nxt = base + 32 + lane < nblk ? __ldg(table + base + 32 + lane) : 0;
+                int ys[4];
+                int nload = 0;
+#pragma unroll
+                for (int jb = 0; jb < 4; ++jb) {
+                    const int k0 = j * kUKeys + jb * kTile;
+                    ys[jb] = -1;
+                    if (k0 < it.c) {  // warp-uniform
+                        const int blk = k0 / bs;
+                        while (blk >= base + 32) {
+                            base += 32;
+                            cur = nxt;
+                            nxt = base + 32 + lane < nblk ? __ldg(table + base + 32 + lane) : 0;
+                        }
+                        int phys = __shfl_sync(0xffffffffu, cur, blk - base);
+                        if (phys < 0 || phys >= prm.num_blocks) {
+                            if (lane == 0) record_error(prm.err, PK_ERR_BAD_INDEX);
+                            phys = 0;
+                        }
+                        ys[jb] = (phys * Hkv + it.kvh) * bs + k0 % bs;
+                        ++nload;
                     }
-                    int phys = __shfl_sync(0xffffffffu, cur, blk - base);
-                    if (phys < 0 || phys >= prm.num_blocks) {
-                        if (lane == 0) record_error(prm.err, PK_ERR_BAD_INDEX);
-                        phys = 0;
-                    }
-                    y = (phys * Hkv + it.kvh) * bs + k0 % bs;
                 }
                 uint64_t *bar = &kv_full[s * kUProducers + p];
                 if (lane == 0) {
-                    if (y >= 0) {
-                        uint8_t *ks = sm + kUOffKV + (size_t)s * kUStageBytes;
-                        uint8_t *vs = ks + kUKBytes;
-                        mbar_arrive_expect_tx(bar, 8192u);  // K: 2 boxes of 2 KiB; V: 4 KiB
-                        tma_load_2d(ks + p * 2048, &tmk2, 0, y, bar);
-                        tma_load_2d(ks + 8192 + p * 2048, &tmk2, 64, y, bar);
-                        tma_load_3d(vs + p * 4096, &tmv3, 0, y, 0, bar);
-                    } else {
+                    uint8_t *ks = sm + kUOffKV + (size_t)s * kUStageBytes;
+                    uint8_t *vs = ks + kUKBytes;
+                    if (nload == 0) {
                         mbar_arrive(bar);  // keys past the context: nothing to load
+                    } else {
+                        mbar_arrive_expect_tx(bar, (uint32_t)nload * (p == 2 ? 4096u : 2048u));
+#pragma unroll
+                        for (int jb = 0; jb < 4; ++jb) {
+                            if (ys[jb] < 0) continue;
+                            if (p == 2) tma_load_3d(vs + jb * 4096, &tmv3, 0, ys[jb], 0, bar);
+                            else tma_load_2d(ks + p * 8192 + jb * 2048, &tmk2, p * 64, ys[jb], bar);
+                        }
                     }
                 }
                 __syncwarp();
@@ -289,21 +310,26 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
         // never leave with a copy still writing into this CTA's shared memory
         for (int m = max(0, n - kUStages); m < n; ++m)
             mbar_wait(&kv_full[(m % kUStages) * kUProducers + p], (uint32_t)(m / kUStages) & 1);
-    } else if (warp >= kUSoft0 && warp < kUSoft0 + 4) {
+    } else if (warp < kUMma) {
         // ------------------------------------------------------------ softmax + epilogue
+        const int t = warp >> 2;             // row tile of this warpgroup
         const int sp = warp & 3;             // tensor-memory lane quarter of this warp
         const int r = sp * 32 + lane;        // the query row this thread owns
+        const UTileBars B = tb(t);
         const uint32_t row_t = tmem + ((uint32_t)(sp * 32) << 16);
+        const uint32_t s_col = (uint32_t)(t * 128), o_col = (uint32_t)(256 + t * 128);
+        uint8_t *qbuf = sm + kUOffQ + t * kUQBytes;
+        uint8_t *pbuf = sm + kUOffP + t * kUPBytes + r * 128;
         int n = 0, n_item = 0;
         bool ok = true;
         for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++n_item) {
             UItem it;
             item_of(idx, it);
-            const int R = it.rt * kURows + r;
+            const int R = it.rt * kUItemRows + t * kURows + r;
             const bool valid = R < it.rows;
-            const int t = valid ? R / g : 0, hh = valid ? R % g : 0;
-            const int pos = it.c - it.qn + t;
-            const long long qrow = ((long long)(it.qs0 + t) * Hq + it.kvh * g + hh) * kUD;
+            const int tok = valid ? R / g : 0, hh = valid ? R % g : 0;
+            const int pos = it.c - it.qn + tok;
+            const long long qrow = ((long long)(it.qs0 + tok) * Hq + it.kvh * g + hh) * kUD;
             // Q row into the K-major 128-byte-swizzled layout (the previous item's
             // MMAs have completed: its o_full was seen)
             {
@@ -312,26 +338,26 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                 for (int ch = 0; ch < 16; ++ch) {
                     const uint4 v = valid ? __ldg(src + ch) : make_uint4(0u, 0u, 0u, 0u);
                     const int pn = ch >> 3, c8 = ch & 7;
-                    *(uint4 *)(sm + kUOffQ + pn * (kURows * 128) + r * 128 + ((c8 ^ (r & 7)) << 4)) = v;
+                    *(uint4 *)(qbuf + pn * (kURows * 128) + r * 128 + ((c8 ^ (r & 7)) << 4)) = v;
                 }
             }
             fence_proxy_async();
             __syncwarp();
-            if (lane == 0) mbar_arrive(q_full);
+            if (lane == 0) mbar_arrive(B.q_full);
             float m = -INFINITY, l = 0.f;
             for (int j = 0; j < it.nkt; ++j, ++n) {
                 const int b = n & 1;
-                if (!mbar_wait(&s_full[b], (uint32_t)(n >> 1) & 1)) {
+                if (!mbar_wait(&B.s_full[b], (uint32_t)(n >> 1) & 1)) {
                     ok = false;
                     break;
                 }
                 tc_after();
                 uint32_t sv[64];
-                tmem_ld64(row_t + (uint32_t)(b * 64), sv);
+                tmem_ld64(row_t + s_col + (uint32_t)(b * 64), sv);
                 tmem_wait_ld();
                 tc_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&s_free[b]);
+                if (lane == 0) mbar_arrive(&B.s_free[b]);
                 const int k0 = j * kUKeys;
                 float mx = -INFINITY;
 #pragma unroll
@@ -340,24 +366,24 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                     sv[i] = __float_as_uint(sc);
                     mx = fmaxf(mx, sc);
                 }
+                // the P V of the previous stage has finished: P is free and O is final
+                if (n >= 1 && !mbar_wait(B.pv_done, (uint32_t)(n - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
                 if (__any_sync(0xffffffffu, mx > m + kURescaleLog2)) {
                     const float mn = fmaxf(m, mx);
                     const float alpha = mn == -INFINITY ? 1.f : fast_exp2(m - mn);
-                    if (j > 0) {
-                        // O holds earlier stages: wait for the last P V, rescale in place
-                        if (!mbar_wait(&pv_done[(n - 1) & 1], (uint32_t)((n - 1) >> 1) & 1)) {
-                            ok = false;
-                            break;
-                        }
+                    if (j > 0) {  // O holds earlier stages: rescale it in place
                         tc_after();
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4) {
                             uint32_t ov[32];
-                            tmem_ld32(row_t + 128u + (uint32_t)(q4 * 32), ov);
+                            tmem_ld32(row_t + o_col + (uint32_t)(q4 * 32), ov);
                             tmem_wait_ld();
 #pragma unroll
                             for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                            tmem_st32(row_t + 128u + (uint32_t)(q4 * 32), ov);
+                            tmem_st32(row_t + o_col + (uint32_t)(q4 * 32), ov);
                         }
                         tmem_wait_st();
                     }
@@ -367,30 +393,26 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                 const float bm = m == -INFINITY ? 0.f : m;
                 float ps = 0.f;
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    const float pv = fast_exp2(__uint_as_float(sv[i]) - bm);
-                    sv[i] = __float_as_uint(pv);
-                    ps += pv;
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    float pv[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        pv[i] = fast_exp2(__uint_as_float(sv[8 * c8 + i]) - bm);
+                        ps += pv[i];
+                    }
+                    uint4 w;
+                    w.x = pack_bf16(pv[0], pv[1]);
+                    w.y = pack_bf16(pv[2], pv[3]);
+                    w.z = pack_bf16(pv[4], pv[5]);
+                    w.w = pack_bf16(pv[6], pv[7]);
+                    *(uint4 *)(pbuf + ((c8 ^ (r & 7)) << 4)) = w;
                 }
                 l += ps;
-                // the P buffer was last read by the P V of stage n - 2
-                if (n >= 2 && !mbar_wait(&pv_done[b], (uint32_t)((n - 2) >> 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                uint8_t *pb = sm + kUOffP + b * kUPBytes + r * 128;
-#pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
-                    uint4 w;
-                    w.x = pack_bf16(__uint_as_float(sv[8 * c8 + 0]), __uint_as_float(sv[8 * c8 + 1]));
-                    w.y = pack_bf16(__uint_as_float(sv[8 * c8 + 2]), __uint_as_float(sv[8 * c8 + 3]));
-                    w.z = pack_bf16(__uint_as_float(sv[8 * c8 + 4]), __uint_as_float(sv[8 * c8 + 5]));
-                    w.w = pack_bf16(__uint_as_float(sv[8 * c8 + 6]), __uint_as_float(sv[8 * c8 + 7]));
-                    *(uint4 *)(pb + ((c8 ^ (r & 7)) << 4)) = w;
-                }
                 const int valid_keys = it.c - k0;
                 if (valid_keys < kUKeys) {
-                    // V rows past the context (stale or unloaded) must be zero: P is 0 there
+                    // V rows past the context (stale or unloaded) must be zero: P is 0
+                    // there.  Both warpgroups write the same zeros; the MMA thread
+                    // waits for both before either P V.
                     uint8_t *vs = sm + kUOffKV + (size_t)(n % kUStages) * kUStageBytes + kUKBytes;
                     for (int i = r; i < (kUKeys - valid_keys) * 16; i += kURows) {
                         const int key = valid_keys + i / 16, ch = i % 16;
@@ -401,11 +423,11 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                 fence_proxy_async();
                 tc_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&p_full[b]);
+                if (lane == 0) mbar_arrive(B.p_full);
             }
             if (!ok) break;
             // epilogue: O / l for this thread's row
-            if (!mbar_wait(o_full, (uint32_t)n_item & 1)) {
+            if (!mbar_wait(B.o_full, (uint32_t)n_item & 1)) {
                 ok = false;
                 break;
             }
@@ -415,7 +437,7 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
                 uint32_t ov[32];
-                tmem_ld32(row_t + 128u + (uint32_t)(q4 * 32), ov);
+                tmem_ld32(row_t + o_col + (uint32_t)(q4 * 32), ov);
                 tmem_wait_ld();
                 if (valid) {
 #pragma unroll
@@ -431,60 +453,67 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
             }
             tc_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(o_free);
+            if (lane == 0) mbar_arrive(B.o_free);
         }
         if (!ok) {
             if (lane == 0) record_error(prm.err, PK_ERR_TIMEOUT);
             *abort_flag = 1;
         }
-    } else if (warp == kUMma) {
+    } else {
         // ------------------------------------------------------------ MMA issue (one thread)
         if (lane == 0) {
             bool ok = true;
             int n = 0, n_item = 0;
-            const uint32_t qa = smem_u32(sm + kUOffQ);
+            // O += P V of stage nn for both row tiles (both softmax warpgroups done)
             auto pv = [&](int nn, bool first) -> bool {
-                const int bb = nn & 1;
-                if (!mbar_wait(&p_full[bb], (uint32_t)(nn >> 1) & 1)) return false;
-                if (first && n_item > 0 && !mbar_wait(o_free, (uint32_t)(n_item - 1) & 1)) return false;
+                for (int t = 0; t < kUTiles; ++t) {
+                    const UTileBars B = tb(t);
+                    if (!mbar_wait(B.p_full, (uint32_t)nn & 1)) return false;
+                    if (first && n_item > 0 && !mbar_wait(B.o_free, (uint32_t)(n_item - 1) & 1)) return false;
+                }
                 tc_after();
                 const int s = nn % kUStages;
                 const uint32_t va = smem_u32(sm + kUOffKV + (size_t)s * kUStageBytes + kUKBytes);
-                const uint32_t pa = smem_u32(sm + kUOffP + bb * kUPBytes);
+                for (int t = 0; t < kUTiles; ++t) {
+                    const uint32_t pa = smem_u32(sm + kUOffP + t * kUPBytes);
 #pragma unroll
-                for (int kp = 0; kp < 4; ++kp)
-                    umma_f16(tmem + 128u, sdesc(pa + kp * 32, 16, 1024), sdesc(va + kp * 4096, 2048, 1024), kIdescPV,
-                             (first && kp == 0) ? 0u : 1u);
-                umma_commit(&pv_done[bb]);
+                    for (int kp = 0; kp < 4; ++kp)
+                        umma_f16(tmem + 256u + (uint32_t)(t * 128), sdesc(pa + kp * 32, 16, 1024),
+                                 sdesc(va + kp * 4096, 2048, 1024), kIdescPV, (first && kp == 0) ? 0u : 1u);
+                    umma_commit(tb(t).pv_done);
+                }
                 umma_commit(&kv_empty[s]);
                 return true;
             };
             for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++n_item) {
                 UItem it;
                 item_of(idx, it);
-                if (!mbar_wait(q_full, (uint32_t)n_item & 1)) {
-                    ok = false;
-                    break;
-                }
+                for (int t = 0; t < kUTiles && ok; ++t) ok = mbar_wait(tb(t).q_full, (uint32_t)n_item & 1);
+                if (!ok) break;
                 tc_after();
                 for (int j = 0; j < it.nkt; ++j, ++n) {
                     const int s = n % kUStages, b = n & 1;
                     bool got = true;
                     for (int p = 0; p < kUProducers && got; ++p)
                         got = mbar_wait(&kv_full[s * kUProducers + p], (uint32_t)(n / kUStages) & 1);
-                    if (got && n >= 2) got = mbar_wait(&s_free[b], (uint32_t)((n >> 1) - 1) & 1);
+                    for (int t = 0; t < kUTiles && got; ++t)
+                        if (n >= 2) got = mbar_wait(&tb(t).s_free[b], (uint32_t)((n >> 1) - 1) & 1);
                     if (!got || *abort_flag) {
                         ok = false;
                         break;
                     }
                     tc_after();
                     const uint32_t ka = smem_u32(sm + kUOffKV + (size_t)s * kUStageBytes);
+                    for (int t = 0; t < kUTiles; ++t) {
+                        const uint32_t qa = smem_u32(sm + kUOffQ + t * kUQBytes);
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_f16(tmem + (uint32_t)(b * 64),
-                                 sdesc(qa + (kk >> 2) * (kURows * 128) + (kk & 3) * 32, 16, 1024),
-                                 sdesc(ka + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-                    umma_commit(&s_full[b]);
+                        for (int kk = 0; kk < 8; ++kk)
+                            umma_f16(tmem + (uint32_t)(t * 128 + b * 64),
+                                     sdesc(qa + (kk >> 2) * (kURows * 128) + (kk & 3) * 32, 16, 1024),
+                                     sdesc(ka + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), kIdescS,
+                                     kk > 0 ? 1u : 0u);
+                        umma_commit(&tb(t).s_full[b]);
+                    }
                     if (j > 0 && !pv(n - 1, j == 1)) {
                         ok = false;
                         break;
@@ -495,7 +524,7 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                     ok = false;
                     break;
                 }
-                umma_commit(o_full);
+                for (int t = 0; t < kUTiles; ++t) umma_commit(tb(t).o_full);
             }
             if (!ok) {
                 record_error(prm.err, PK_ERR_TIMEOUT);
