@@ -557,7 +557,8 @@ int chunk_umma_prepare_pool(pk_pool *p) {
     cudaError_t ce = cudaFuncSetAttribute(attention_chunk_umma_kernel,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kUSmem);
     if (ce != cudaSuccess) return cuda_fail(ce, "set chunk (tcgen05) smem size");
-    const int rc = encode_pool_map(&p->tmap_k2, p->k_base, p, kTile);
+    int rc = encode_pool_map(&p->tmap_k2, p->k_base, p, kTile);
+    if (rc == PK_OK) rc = encode_pool_map(&p->tmap_v2, p->v_base, p, kTile);
     if (rc != PK_OK) return rc;
     p->umma_ok = true;
     return PK_OK;

@@ -85,6 +85,12 @@ CHUNK_CASES = [
     ([90, 45], [33, 45], 8, 8, 64, 8),
     ([600], [250], 28, 4, 128, 32),
     ([70, 18], [70, 5], 32, 1, 128, 16),
+    # d 128, blocks of 16k: the tcgen05 chunk kernel, 256-row items of two 128-row tiles
+    ([512], [512], 8, 8, 128, 16),               # g 1, a whole prompt as one chunk (no prior context)
+    ([700, 300], [300, 129], 16, 8, 128, 16),    # g 2, ragged last row tile
+    ([1100, 96], [600, 96], 64, 8, 128, 32),     # g 8, block 32
+    ([2000, 40], [257, 40], 32, 2, 128, 64),     # g 16, block 64
+    ([333, 20], [200, 1], 64, 1, 128, 16),       # g 64: one token fills 64 rows; a decode in the batch
 ]
 
 
@@ -101,6 +107,17 @@ def test_decode_batch_over_several_launch_windows(cuda_dev):
     b = make_batch(ctx, None, block_size=16, n_q_heads=8, n_kv_heads=2, head_dim=64,
                    dtype=torch.bfloat16, seed=77)
     _check(b, 8, 2, 64, torch.bfloat16, cuda_dev, "600 sequences")
+
+
+def test_chunks_at_successive_offsets(cuda_dev):
+    # a 900-token prompt as one chunk, and 300-token chunks at offsets 0, 300 and
+    # 600 (each sees the earlier tokens as context): every row matches the oracle
+    ctx_total, d, Hq, Hkv = 900, 128, 32, 8
+    for start, qn in ((0, 900), (0, 300), (300, 300), (600, 300)):
+        c = start + qn
+        b = make_batch([c], [qn], block_size=16, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d,
+                       dtype=torch.bfloat16, seed=123)
+        _check(b, Hq, Hkv, d, torch.bfloat16, cuda_dev, f"chunk at {start}")
 
 
 def test_permuted_block_ids_bit_identical(cuda_dev):
