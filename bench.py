@@ -38,7 +38,7 @@ METRIC = "paged decode attention KV GB/s (% of HBM peak) and tokens/s per schedu
 FALLBACK_HBM_GBS = 6650.0
 CSRC = os.path.join(ROOT, "paged_kv_cache_chunked_b200", "csrc")
 # the source of each workload's dominant kernel (the traffic record is valid for that source only)
-KERNEL_SRC = {"chunk512_bf16": os.path.join(CSRC, "attention_chunk.cu"),
+KERNEL_SRC = {"chunk512_bf16": os.path.join(CSRC, "attention_chunk_umma.cu"),
               "append_copy": os.path.join(CSRC, "kv_copy.cu")}
 DECODE_SRC = os.path.join(CSRC, "attention_decode_blocks.cu")
 
@@ -305,7 +305,7 @@ def measured_tensor_peak():
 def roofline_entry(workload, attn_b, flops, avg_ms, gbs, tflops, hbm_peak, hbm_kind):
     """The attention call's roofline: HBM for decode (about 4 flop/byte at GQA 4),
     the tensor pipe for prefill chunks (a dense contraction)."""
-    kern = ("paged_attention call: chunk kernel + tile-streaming decode kernel"
+    kern = ("paged_attention call: tcgen05 chunk kernel (S and O accumulated in tensor memory)"
             if workload == "chunk512_bf16" else
             "paged_attention call: block-streaming decode kernel + split-K merge kernel")
     common = {"kernel": kern,

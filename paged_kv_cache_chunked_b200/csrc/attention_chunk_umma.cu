@@ -118,6 +118,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
                  : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+                 :
+                 : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+                 : "memory");
+}
 struct UParams {
     const __nv_bfloat16 *q;
     __nv_bfloat16 *out;
@@ -359,13 +370,22 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&B.s_free[b]);
                 const int k0 = j * kUKeys;
+                // scores in log2 units are s * scale_log2; the running max is kept in
+                // those units, the raw max (scale > 0) is taken first.  Stages wholly
+                // below every row's diagonal skip the mask.
                 float mx = -INFINITY;
+                if (__all_sync(0xffffffffu, valid && k0 + kUKeys - 1 <= pos)) {
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    const float sc = (valid && k0 + i <= pos) ? __uint_as_float(sv[i]) * prm.scale_log2 : -INFINITY;
-                    sv[i] = __float_as_uint(sc);
-                    mx = fmaxf(mx, sc);
+                    for (int i = 0; i < 64; ++i) mx = fmaxf(mx, __uint_as_float(sv[i]));
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) {
+                        const float sc = (valid && k0 + i <= pos) ? __uint_as_float(sv[i]) : -INFINITY;
+                        sv[i] = __float_as_uint(sc);
+                        mx = fmaxf(mx, sc);
+                    }
                 }
+                mx *= prm.scale_log2;
                 // the P V of the previous stage has finished: P is free and O is final
                 if (n >= 1 && !mbar_wait(B.pv_done, (uint32_t)(n - 1) & 1)) {
                     ok = false;
@@ -376,14 +396,14 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                     const float alpha = mn == -INFINITY ? 1.f : fast_exp2(m - mn);
                     if (j > 0) {  // O holds earlier stages: rescale it in place
                         tc_after();
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            uint32_t ov[32];
-                            tmem_ld32(row_t + o_col + (uint32_t)(q4 * 32), ov);
+#pragma unroll 1
+                        for (int q8 = 0; q8 < 8; ++q8) {
+                            uint32_t ov[16];
+                            tmem_ld16(row_t + o_col + (uint32_t)(q8 * 16), ov);
                             tmem_wait_ld();
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                            tmem_st32(row_t + o_col + (uint32_t)(q4 * 32), ov);
+                            for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                            tmem_st16(row_t + o_col + (uint32_t)(q8 * 16), ov);
                         }
                         tmem_wait_st();
                     }
@@ -391,13 +411,14 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                     l *= alpha;
                 }
                 const float bm = m == -INFINITY ? 0.f : m;
+                const float sl = prm.scale_log2;
                 float ps = 0.f;
 #pragma unroll
                 for (int c8 = 0; c8 < 8; ++c8) {
                     float pv[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        pv[i] = fast_exp2(__uint_as_float(sv[8 * c8 + i]) - bm);
+                        pv[i] = fast_exp2(fmaf(__uint_as_float(sv[8 * c8 + i]), sl, -bm));
                         ps += pv[i];
                     }
                     uint4 w;
