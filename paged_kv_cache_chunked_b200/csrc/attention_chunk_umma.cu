@@ -16,7 +16,10 @@
 //   - three producer warps load the stage's four 16-key blocks by TMA: K as two
 //     2-D boxes per block (one per 64-column panel; warps 0 and 1) into the
 //     canonical K-major 128-byte-swizzled layout [panel][64 keys][128 B], V as
-//     one 3-D box per block [block][panel][16 keys][128 B] (warp 2);
+//     one 3-D box per block [block][panel][16 keys][128 B] (warp 2).  K and V
+//     have rings of their own: a K slot is refilled as soon as the stage's S
+//     has completed, a V slot once its P V has, so each load is issued two to
+//     three stages before it is read;
 //   - one thread of the MMA warp issues, per row tile, S = Q K^T (M 128, N 64,
 //     eight K-steps of 16) into one of two tensor-memory buffers, then, when
 //     both tiles' softmax of the previous stage are done, O += P V (M 128,
@@ -46,10 +49,10 @@ constexpr int kURows = 128;             // query rows per row tile (UMMA M)
 constexpr int kUTiles = 2;              // row tiles per item: 256 query rows share each KV stage
 constexpr int kUItemRows = kURows * kUTiles;
 constexpr int kUKeys = 64;              // keys per stage
-constexpr int kUStages = 3;
+constexpr int kUKStages = 4;            // K ring: a slot is free once the stage's S = Q K^T has completed
+constexpr int kUVStages = 3;            // V ring: a slot is free once the stage's O += P V has completed
 constexpr int kUMma = 8;                // warp 8: tensor memory and MMA issue
-constexpr int kUProd0 = 9;              // warps 9..11: producers (K panel 0, K panel 1, V)
-constexpr int kUProducers = 3;
+constexpr int kUProd0 = 9;              // warps 9, 10: K panel 0, 1; warp 11: V
 constexpr int kUThreads = 12 * 32;      // warps 0..3 and 4..7: softmax of row tile 0 and 1
 constexpr uint32_t kUTmemCols = 512;    // S[t][b] at 128 t + 64 b, O[t] at 256 + 128 t
 constexpr float kURescaleLog2 = 8.f;
@@ -57,19 +60,20 @@ constexpr float kURescaleLog2 = 8.f;
 constexpr uint32_t kUQBytes = kURows * kUD * 2;       // per tile: [panel][128 rows][128 B]
 constexpr uint32_t kUKBytes = kUKeys * kUD * 2;       // [panel][64 keys][128 B]
 constexpr uint32_t kUVBytes = kUKeys * kUD * 2;       // [block][panel][16 keys][128 B]
-constexpr uint32_t kUStageBytes = kUKBytes + kUVBytes;
 constexpr uint32_t kUPBytes = kURows * kUKeys * 2;    // per tile: [128 rows][128 B]
 constexpr uint32_t kUOffQ = 0;
-constexpr uint32_t kUOffKV = kUOffQ + kUTiles * kUQBytes;
-constexpr uint32_t kUOffP = kUOffKV + kUStages * kUStageBytes;
+constexpr uint32_t kUOffK = kUOffQ + kUTiles * kUQBytes;
+constexpr uint32_t kUOffV = kUOffK + kUKStages * kUKBytes;
+constexpr uint32_t kUOffP = kUOffV + kUVStages * kUVBytes;
 constexpr uint32_t kUOffPlan = kUOffP + kUTiles * kUPBytes;
 constexpr uint32_t kUOffBar = kUOffPlan + (3 * kPlanLen * 4 + 15) / 16 * 16;
-// barriers: kv_full[stage][producer], kv_empty[stage]; per row tile: s_full[2],
-// s_free[2], p_full, pv_done, q_full, o_full, o_free; mma_done
+// barriers: k_full[K slot], k_empty[K slot], v_full[V slot], v_empty[V slot]; per
+// row tile: s_full[2], s_free[2], p_full, pv_done, q_full, o_full, o_free; mma_done
 constexpr uint32_t kUPerTileBars = 9;
-constexpr uint32_t kUNumBars = kUStages * kUProducers + kUStages + kUTiles * kUPerTileBars + 1;
+constexpr uint32_t kUNumBars = 2 * kUKStages + 2 * kUVStages + kUTiles * kUPerTileBars + 1;
 constexpr uint32_t kUOffMisc = kUOffBar + kUNumBars * 8;  // tensor memory address, abort flag
 constexpr uint32_t kUSmem = kUOffMisc + 16 + 1024;        // + alignment slack
+static_assert(kUSmem <= 227 * 1024 - 64, "chunk kernel shared memory");
 
 // instruction descriptors (kind::f16): fp32 accumulate, bf16 A and B, M = 128
 constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
@@ -111,13 +115,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
                  : "r"(taddr));
 }
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
-                 :
-                 : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-                 : "memory");
-}
-
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
@@ -159,9 +156,11 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
     int *item_pre = (int *)(sm + kUOffPlan);
     int *s_qsl = item_pre + kPlanLen;
     int *s_ctx = s_qsl + kPlanLen;
-    uint64_t *kv_full = (uint64_t *)(sm + kUOffBar);  // [stage][producer]
-    uint64_t *kv_empty = kv_full + kUStages * kUProducers;
-    uint64_t *tile_bars = kv_empty + kUStages;
+    uint64_t *k_full = (uint64_t *)(sm + kUOffBar);
+    uint64_t *k_empty = k_full + kUKStages;
+    uint64_t *v_full = k_empty + kUKStages;
+    uint64_t *v_empty = v_full + kUVStages;
+    uint64_t *tile_bars = v_empty + kUVStages;
     uint64_t *mma_done = tile_bars + kUTiles * kUPerTileBars;
     auto tb = [&](int t) {
         uint64_t *q = tile_bars + t * kUPerTileBars;
@@ -172,8 +171,14 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
     __shared__ int s_nitems;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kUStages * kUProducers; ++i) mbar_init(&kv_full[i], 1);
-        for (int s = 0; s < kUStages; ++s) mbar_init(&kv_empty[s], 1);
+        for (int s = 0; s < kUKStages; ++s) {
+            mbar_init(&k_full[s], 2);  // both K producers
+            mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < kUVStages; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
+        }
         for (int t = 0; t < kUTiles; ++t) {
             const UTileBars B = tb(t);
             for (int b = 0; b < 2; ++b) {
@@ -251,8 +256,15 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
 
     if (warp >= kUProd0) {
         // ------------------------------------------------------------ producers
-        // producer 0: K panel 0 of the stage's four 16-key blocks; 1: K panel 1; 2: V
+        // warps 9 and 10: K panel 0 and 1 of the stage's four 16-key blocks into
+        // [panel][64 keys][128 B]; warp 11: V, one 3-D box per block into
+        // [block][panel][16 keys][128 B]
         const int p = warp - kUProd0;
+        const bool is_v = p == 2;
+        const int nst = is_v ? kUVStages : kUKStages;
+        uint64_t *full = is_v ? v_full : k_full;
+        uint64_t *empty = is_v ? v_empty : k_empty;
+        if (lane == 0) prefetch_tmap(is_v ? &tmv3 : &tmk2);
         int n = 0;
         bool ok = true;
         for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
@@ -264,8 +276,8 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
             int cur = lane < nblk ? __ldg(table + lane) : 0;
             int nxt = 32 + lane < nblk ? __ldg(table + 32 + lane) : 0;
             for (int j = 0; j < it.nkt; ++j, ++n) {
-                const int s = n % kUStages;
-                if (n >= kUStages && !mbar_wait(&kv_empty[s], (uint32_t)(n / kUStages - 1) & 1)) {
+                const int s = n % nst;
+                if (n >= nst && !mbar_wait(&empty[s], (uint32_t)(n / nst - 1) & 1)) {
                     ok = false;
                     break;
                 }
@@ -274,7 +286,6 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                     break;
                 }
                 int ys[4];
-                int nload = 0;
 #pragma unroll
                 for (int jb = 0; jb < 4; ++jb) {
                     const int k0 = j * kUKeys + jb * kTile;
@@ -292,22 +303,24 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                             phys = 0;
                         }
                         ys[jb] = (phys * Hkv + it.kvh) * bs + k0 % bs;
-                        ++nload;
                     }
                 }
-                uint64_t *bar = &kv_full[s * kUProducers + p];
                 if (lane == 0) {
-                    uint8_t *ks = sm + kUOffKV + (size_t)s * kUStageBytes;
-                    uint8_t *vs = ks + kUKBytes;
-                    if (nload == 0) {
-                        mbar_arrive(bar);  // keys past the context: nothing to load
+                    uint32_t bytes = 0;
+#pragma unroll
+                    for (int jb = 0; jb < 4; ++jb)
+                        if (ys[jb] >= 0) bytes += is_v ? 4096u : 2048u;
+                    if (bytes == 0) {
+                        mbar_arrive(&full[s]);  // keys past the context: nothing to load
                     } else {
-                        mbar_arrive_expect_tx(bar, (uint32_t)nload * (p == 2 ? 4096u : 2048u));
+                        mbar_arrive_expect_tx(&full[s], bytes);
+                        uint8_t *dst = is_v ? sm + kUOffV + (size_t)s * kUVBytes
+                                            : sm + kUOffK + (size_t)s * kUKBytes + p * 8192;
 #pragma unroll
                         for (int jb = 0; jb < 4; ++jb) {
                             if (ys[jb] < 0) continue;
-                            if (p == 2) tma_load_3d(vs + jb * 4096, &tmv3, 0, ys[jb], 0, bar);
-                            else tma_load_2d(ks + p * 8192 + jb * 2048, &tmk2, p * 64, ys[jb], bar);
+                            if (is_v) tma_load_3d(dst + jb * 4096, &tmv3, 0, ys[jb], 0, &full[s]);
+                            else tma_load_2d(dst + jb * 2048, &tmk2, p * 64, ys[jb], &full[s]);
                         }
                     }
                 }
@@ -319,8 +332,7 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
             *abort_flag = 1;
         }
         // never leave with a copy still writing into this CTA's shared memory
-        for (int m = max(0, n - kUStages); m < n; ++m)
-            mbar_wait(&kv_full[(m % kUStages) * kUProducers + p], (uint32_t)(m / kUStages) & 1);
+        for (int m = max(0, n - nst); m < n; ++m) mbar_wait(&full[m % nst], (uint32_t)(m / nst) & 1);
     } else if (warp < kUMma) {
         // ------------------------------------------------------------ softmax + epilogue
         const int t = warp >> 2;             // row tile of this warpgroup
@@ -432,9 +444,13 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                 const int valid_keys = it.c - k0;
                 if (valid_keys < kUKeys) {
                     // V rows past the context (stale or unloaded) must be zero: P is 0
-                    // there.  Both warpgroups write the same zeros; the MMA thread
-                    // waits for both before either P V.
-                    uint8_t *vs = sm + kUOffKV + (size_t)(n % kUStages) * kUStageBytes + kUKBytes;
+                    // there.  Both warpgroups write the same zeros, after the stage's V
+                    // has landed; the MMA thread waits for both before either P V.
+                    if (!mbar_wait(&v_full[n % kUVStages], (uint32_t)(n / kUVStages) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *vs = sm + kUOffV + (size_t)(n % kUVStages) * kUVBytes;
                     for (int i = r; i < (kUKeys - valid_keys) * 16; i += kURows) {
                         const int key = valid_keys + i / 16, ch = i % 16;
                         *(uint4 *)(vs + (key >> 4) * 4096 + (ch >> 3) * 2048 + (key & 15) * 128 + (ch & 7) * 16) =
@@ -492,9 +508,10 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                     if (!mbar_wait(B.p_full, (uint32_t)nn & 1)) return false;
                     if (first && n_item > 0 && !mbar_wait(B.o_free, (uint32_t)(n_item - 1) & 1)) return false;
                 }
+                const int s = nn % kUVStages;
+                if (!mbar_wait(&v_full[s], (uint32_t)(nn / kUVStages) & 1)) return false;
                 tc_after();
-                const int s = nn % kUStages;
-                const uint32_t va = smem_u32(sm + kUOffKV + (size_t)s * kUStageBytes + kUKBytes);
+                const uint32_t va = smem_u32(sm + kUOffV + (size_t)s * kUVBytes);
                 for (int t = 0; t < kUTiles; ++t) {
                     const uint32_t pa = smem_u32(sm + kUOffP + t * kUPBytes);
 #pragma unroll
@@ -503,7 +520,7 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                                  sdesc(va + kp * 4096, 2048, 1024), kIdescPV, (first && kp == 0) ? 0u : 1u);
                     umma_commit(tb(t).pv_done);
                 }
-                umma_commit(&kv_empty[s]);
+                umma_commit(&v_empty[s]);
                 return true;
             };
             for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++n_item) {
@@ -513,10 +530,8 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                 if (!ok) break;
                 tc_after();
                 for (int j = 0; j < it.nkt; ++j, ++n) {
-                    const int s = n % kUStages, b = n & 1;
-                    bool got = true;
-                    for (int p = 0; p < kUProducers && got; ++p)
-                        got = mbar_wait(&kv_full[s * kUProducers + p], (uint32_t)(n / kUStages) & 1);
+                    const int s = n % kUKStages, b = n & 1;
+                    bool got = mbar_wait(&k_full[s], (uint32_t)(n / kUKStages) & 1);
                     for (int t = 0; t < kUTiles && got; ++t)
                         if (n >= 2) got = mbar_wait(&tb(t).s_free[b], (uint32_t)((n >> 1) - 1) & 1);
                     if (!got || *abort_flag) {
@@ -524,7 +539,7 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                         break;
                     }
                     tc_after();
-                    const uint32_t ka = smem_u32(sm + kUOffKV + (size_t)s * kUStageBytes);
+                    const uint32_t ka = smem_u32(sm + kUOffK + (size_t)s * kUKBytes);
                     for (int t = 0; t < kUTiles; ++t) {
                         const uint32_t qa = smem_u32(sm + kUOffQ + t * kUQBytes);
 #pragma unroll
@@ -535,6 +550,7 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                                      kk > 0 ? 1u : 0u);
                         umma_commit(&tb(t).s_full[b]);
                     }
+                    umma_commit(&k_empty[s]);  // the K slot is free once both S have completed
                     if (j > 0 && !pv(n - 1, j == 1)) {
                         ok = false;
                         break;
