@@ -1,8 +1,9 @@
 // Paged attention for causal prefill chunks on the fifth-generation tensor
-// cores (tcgen05, accumulators in tensor memory): bf16 pools, head_dim 128,
-// block_size a multiple of 16, groups g dividing 128.  Serves every sequence
-// whose query rows (q_b tokens x g heads of a kv group) span more than one
-// 16-row tile; decodes and chunks of a few tokens run in the decode kernel.
+// cores (tcgen05, operands and accumulators in tensor memory): bf16 pools,
+// head_dim 128, block_size a multiple of 16, groups g dividing 128.  Serves
+// every sequence whose query rows (q_b tokens x g heads of a kv group) span more
+// than one 16-row tile; decodes and chunks of a few tokens run in the decode
+// kernel.
 //
 // What is computed ["Batching and PagedAttention", "Continuous batching":
 // long prompts are split into chunks across steps; "PagedAttention & Continuous
@@ -12,25 +13,31 @@
 //
 // Structure.  A work item is 256 query rows (pairs (token, head of the
 // group), token-major) of one (sequence, kv head), as two 128-row tiles; CTA i
-// takes items i, i + gridDim.x, ...  Per 64-key stage:
-//   - three producer warps load the stage's four 16-key blocks by TMA: K as two
+// takes items i, i + gridDim.x, ...  Per 128-key stage:
+//   - three producer warps load the stage's eight 16-key blocks by TMA: K as two
 //     2-D boxes per block (one per 64-column panel; warps 0 and 1) into the
-//     canonical K-major 128-byte-swizzled layout [panel][64 keys][128 B], V as
+//     canonical K-major 128-byte-swizzled layout [panel][128 keys][128 B], V as
 //     one 3-D box per block [block][panel][16 keys][128 B] (warp 2).  K and V
-//     have rings of their own: a K slot is refilled as soon as the stage's S
-//     has completed, a V slot once its P V has, so each load is issued two to
-//     three stages before it is read;
-//   - one thread of the MMA warp issues, per row tile, S = Q K^T (M 128, N 64,
-//     eight K-steps of 16) into one of two tensor-memory buffers, then, when
-//     both tiles' softmax of the previous stage are done, O += P V (M 128,
-//     N 128, four K-steps; V read MN-major);
-//   - per row tile, four softmax warps own one query row per thread (two
-//     warpgroups share each SM sub-partition and hide each other's latency):
-//     they read the row of S
-//     from tensor memory (no shuffles), mask causally, keep the running max m
-//     and sum l in fp32 (the reference m moves, and O is rescaled in tensor
-//     memory, only when a score exceeds it by more than 2^8), and write P as
-//     bf16 into a 128-byte-swizzled shared buffer, the A operand of P V.
+//     have rings of their own: a K slot is refilled once the stage's S has
+//     completed, a V slot once its P V has.  On a stage that runs past the
+//     context the V warp zeroes the rows past it (P is 0 there, the stale rows
+//     may hold anything) before it releases the stage;
+//   - one thread of the MMA warp issues, per row tile t, O_t += P_t V of the
+//     previous stage (A = P_t read from tensor memory, B = V MN-major; M 128,
+//     N 128, eight K-steps) and then S_t = Q_t K^T of this stage (M 128, N 128,
+//     eight K-steps) into the same tensor-memory columns: the tensor core runs
+//     one thread's MMAs in order, so S_t overwrites P_t only after P_t V has
+//     read it.  Tile 1's MMAs run while tile 0's softmax works and the other
+//     way round;
+//   - per row tile, four softmax warps own one query row per thread: they read
+//     the row of S from tensor memory, mask causally, keep the running max m and
+//     sum l in fp32 (the reference m moves, and O is rescaled in tensor memory,
+//     only when a score exceeds it by more than 2^8), and write P as packed bf16
+//     over the first 64 columns of S.  When S_t of a stage is complete, P_t V of
+//     the previous stage is too (its commit covers every earlier MMA), so O_t is
+//     stable for the whole softmax.
+// Each tcgen05.mma has an issue cost of its own, so the stage is 128 keys wide:
+// S MMAs with N = 128 do twice the work per instruction of N = 64 ones.
 // Every wait is bounded (2 s); on expiry the kernel records PK_ERR_TIMEOUT,
 // each warp waits (bounded) for its own copies and tensor-core work, and the
 // CTA releases its tensor memory and returns.  Block ids are range-checked.
@@ -48,53 +55,76 @@ constexpr int kUD = 128;                // head dim
 constexpr int kURows = 128;             // query rows per row tile (UMMA M)
 constexpr int kUTiles = 2;              // row tiles per item: 256 query rows share each KV stage
 constexpr int kUItemRows = kURows * kUTiles;
-constexpr int kUKeys = 64;              // keys per stage
-constexpr int kUKStages = 4;            // K ring: a slot is free once the stage's S = Q K^T has completed
-constexpr int kUVStages = 3;            // V ring: a slot is free once the stage's O += P V has completed
+constexpr int kUKeys = 128;             // keys per stage (UMMA N of S)
+constexpr int kUBlk = kUKeys / 16;      // 16-key blocks per stage
+constexpr int kUKStages = 2;            // K ring: a slot is free once the stage's S = Q K^T has completed
+constexpr int kUVStages = 2;            // V ring: a slot is free once the stage's O += P V has completed
 constexpr int kUMma = 8;                // warp 8: tensor memory and MMA issue
 constexpr int kUProd0 = 9;              // warps 9, 10: K panel 0, 1; warp 11: V
 constexpr int kUThreads = 12 * 32;      // warps 0..3 and 4..7: softmax of row tile 0 and 1
-constexpr uint32_t kUTmemCols = 512;    // S[t][b] at 128 t + 64 b, O[t] at 256 + 128 t
+constexpr uint32_t kUTmemCols = 512;    // S[t] (P[t] over its first 64 columns) at 128 t, O[t] at 256 + 128 t
 constexpr float kURescaleLog2 = 8.f;
+// Register split: the kernel launches with kURegLaunch registers a thread; the
+// two softmax warpgroups then take kURegSoftmax and the MMA / producer warpgroup
+// keeps kURegOther.  The split uses exactly the launch's registers (setmaxnreg
+// can only hand out what the block was launched with), and the host checks the
+// compiled register count before it enables this kernel.
+constexpr int kURegLaunch = 168, kURegSoftmax = 176, kURegOther = 152;
+static_assert(256 * kURegSoftmax + 128 * kURegOther <= kUThreads * kURegLaunch, "register split");
 
 constexpr uint32_t kUQBytes = kURows * kUD * 2;       // per tile: [panel][128 rows][128 B]
-constexpr uint32_t kUKBytes = kUKeys * kUD * 2;       // [panel][64 keys][128 B]
+constexpr uint32_t kUKBytes = kUKeys * kUD * 2;       // [panel][128 keys][128 B]
+constexpr uint32_t kUKPanel = kUKeys * 128;           // bytes of one K panel
 constexpr uint32_t kUVBytes = kUKeys * kUD * 2;       // [block][panel][16 keys][128 B]
-constexpr uint32_t kUPBytes = kURows * kUKeys * 2;    // per tile: [128 rows][128 B]
 constexpr uint32_t kUOffQ = 0;
 constexpr uint32_t kUOffK = kUOffQ + kUTiles * kUQBytes;
 constexpr uint32_t kUOffV = kUOffK + kUKStages * kUKBytes;
-constexpr uint32_t kUOffP = kUOffV + kUVStages * kUVBytes;
-constexpr uint32_t kUOffPlan = kUOffP + kUTiles * kUPBytes;
+constexpr uint32_t kUOffPlan = kUOffV + kUVStages * kUVBytes;
 constexpr uint32_t kUOffBar = kUOffPlan + (3 * kPlanLen * 4 + 15) / 16 * 16;
-// barriers: k_full[K slot], k_empty[K slot], v_full[V slot], v_empty[V slot]; per
-// row tile: s_full[2], s_free[2], p_full, pv_done, q_full, o_full, o_free; mma_done
-constexpr uint32_t kUPerTileBars = 9;
-constexpr uint32_t kUNumBars = 2 * kUKStages + 2 * kUVStages + kUTiles * kUPerTileBars + 1;
+// barriers: k_full[K slot], k_empty[K slot], v_full[V slot], v_empty[V slot],
+// v_tma; per row tile: s_full, p_full, q_full, o_full, o_free; mma_done
+constexpr uint32_t kUPerTileBars = 5;
+constexpr uint32_t kUNumBars = 2 * kUKStages + 2 * kUVStages + 1 + kUTiles * kUPerTileBars + 1;
 constexpr uint32_t kUOffMisc = kUOffBar + kUNumBars * 8;  // tensor memory address, abort flag
 constexpr uint32_t kUSmem = kUOffMisc + 16 + 1024;        // + alignment slack
 static_assert(kUSmem <= 227 * 1024 - 64, "chunk kernel shared memory");
 
-// instruction descriptors (kind::f16): fp32 accumulate, bf16 A and B, M = 128
-constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
+// instruction descriptors (kind::f16): fp32 accumulate, bf16 A and B, M = 128, N = 128
+constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescPV =
     (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);  // B MN-major
 
-// Shared-memory matrix descriptor: 128-byte swizzle, byte offsets lbo / sbo.
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
-    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-    d |= (uint64_t)1 << 46;  // descriptor version of sm_100
-    d |= (uint64_t)2 << 61;  // 128-byte swizzle
-    return d;
+// Shared-memory matrix descriptor (128-byte swizzle) as two 32-bit words: the low
+// word holds the start address and the leading byte offset (both >> 4), the high
+// word the stride byte offset (>> 4, 1024 B here), the descriptor version of
+// sm_100 (bit 46 of the 64-bit value) and the swizzle mode (bits 61..63).  The
+// MMA thread builds the low word of each operand's base once and adds the
+// per-K-step offset (>> 4; addresses stay below 256 KiB, so the 14-bit field
+// never carries).
+__device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo) {
+    return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
 }
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                         uint32_t accumulate) {
+constexpr uint32_t kSdescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+// D (tensor memory) [+]= A (shared) x B (shared)
+__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc,
+                                        uint32_t accumulate) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+        "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\t"
+        "mov.b64 ad, {%1, %5};\n\tmov.b64 bd, {%2, %5};\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, {%6, %6, %6, %6}, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(kSdescHi), "r"(0u));
+}
+// D (tensor memory) [+]= A (tensor memory: row m in lane m, two bf16 per column,
+// the even K index in the low half) x B (shared)
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\t"
+        "mov.b64 bd, {%2, %5};\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %3, {%6, %6, %6, %6}, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(kSdescHi), "r"(0u));
 }
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -126,6 +156,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
                  : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
                  : "memory");
 }
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                 :
+                 : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
 struct UParams {
     const __nv_bfloat16 *q;
     __nv_bfloat16 *out;
@@ -141,7 +177,7 @@ struct UItem {
 
 // Per-row-tile barriers.
 struct UTileBars {
-    uint64_t *s_full, *s_free, *p_full, *pv_done, *q_full, *o_full, *o_free;
+    uint64_t *s_full, *p_full, *q_full, *o_full, *o_free;
 };
 
 __global__ void __launch_bounds__(kUThreads, 1)
@@ -160,11 +196,12 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
     uint64_t *k_empty = k_full + kUKStages;
     uint64_t *v_full = k_empty + kUKStages;
     uint64_t *v_empty = v_full + kUVStages;
-    uint64_t *tile_bars = v_empty + kUVStages;
+    uint64_t *v_tma = v_empty + kUVStages;  // V of a stage that runs past the context
+    uint64_t *tile_bars = v_tma + 1;
     uint64_t *mma_done = tile_bars + kUTiles * kUPerTileBars;
     auto tb = [&](int t) {
         uint64_t *q = tile_bars + t * kUPerTileBars;
-        return UTileBars{q, q + 2, q + 4, q + 5, q + 6, q + 7, q + 8};
+        return UTileBars{q, q + 1, q + 2, q + 3, q + 4};
     };
     uint32_t *tmem_slot = (uint32_t *)(sm + kUOffMisc);
     volatile int *abort_flag = (volatile int *)(sm + kUOffMisc + 4);
@@ -179,14 +216,11 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
             mbar_init(&v_full[s], 1);
             mbar_init(&v_empty[s], 1);
         }
+        mbar_init(v_tma, 1);
         for (int t = 0; t < kUTiles; ++t) {
             const UTileBars B = tb(t);
-            for (int b = 0; b < 2; ++b) {
-                mbar_init(&B.s_full[b], 1);
-                mbar_init(&B.s_free[b], 4);
-            }
+            mbar_init(B.s_full, 1);
             mbar_init(B.p_full, 4);
-            mbar_init(B.pv_done, 1);
             mbar_init(B.q_full, 4);
             mbar_init(B.o_full, 1);
             mbar_init(B.o_free, 4);
@@ -238,6 +272,8 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
     tc_after();
     const uint32_t tmem = *tmem_slot;
     const int n_items = s_nitems;
+    if (warp < kUMma) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kURegSoftmax));
+    else asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kURegOther));
 
     auto item_of = [&](int idx, UItem &it) {
         const int b = find_seq(item_pre, nseq, idx);
@@ -256,8 +292,8 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
 
     if (warp >= kUProd0) {
         // ------------------------------------------------------------ producers
-        // warps 9 and 10: K panel 0 and 1 of the stage's four 16-key blocks into
-        // [panel][64 keys][128 B]; warp 11: V, one 3-D box per block into
+        // warps 9 and 10: K panel 0 and 1 of the stage's eight 16-key blocks into
+        // [panel][128 keys][128 B]; warp 11: V, one 3-D box per block into
         // [block][panel][16 keys][128 B]
         const int p = warp - kUProd0;
         const bool is_v = p == 2;
@@ -265,7 +301,7 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
         uint64_t *full = is_v ? v_full : k_full;
         uint64_t *empty = is_v ? v_empty : k_empty;
         if (lane == 0) prefetch_tmap(is_v ? &tmv3 : &tmk2);
-        int n = 0;
+        int n = 0, ntail = 0;
         bool ok = true;
         for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
             UItem it;
@@ -285,9 +321,9 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                     ok = false;
                     break;
                 }
-                int ys[4];
+                int ys[kUBlk];
 #pragma unroll
-                for (int jb = 0; jb < 4; ++jb) {
+                for (int jb = 0; jb < kUBlk; ++jb) {
                     const int k0 = j * kUKeys + jb * kTile;
                     ys[jb] = -1;
                     if (k0 < it.c) {  // warp-uniform
@@ -305,26 +341,48 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                         ys[jb] = (phys * Hkv + it.kvh) * bs + k0 % bs;
                     }
                 }
+                const int valid_keys = it.c - j * kUKeys;  // warp-uniform
+                const bool tail = is_v && valid_keys < kUKeys;
+                uint8_t *dst = is_v ? sm + kUOffV + (size_t)s * kUVBytes
+                                    : sm + kUOffK + (size_t)s * kUKBytes + p * kUKPanel;
+                uint64_t *bar = tail ? v_tma : &full[s];
                 if (lane == 0) {
                     uint32_t bytes = 0;
 #pragma unroll
-                    for (int jb = 0; jb < 4; ++jb)
+                    for (int jb = 0; jb < kUBlk; ++jb)
                         if (ys[jb] >= 0) bytes += is_v ? 4096u : 2048u;
                     if (bytes == 0) {
-                        mbar_arrive(&full[s]);  // keys past the context: nothing to load
+                        mbar_arrive(bar);  // keys past the context: nothing to load
                     } else {
-                        mbar_arrive_expect_tx(&full[s], bytes);
-                        uint8_t *dst = is_v ? sm + kUOffV + (size_t)s * kUVBytes
-                                            : sm + kUOffK + (size_t)s * kUKBytes + p * 8192;
+                        mbar_arrive_expect_tx(bar, bytes);
 #pragma unroll
-                        for (int jb = 0; jb < 4; ++jb) {
+                        for (int jb = 0; jb < kUBlk; ++jb) {
                             if (ys[jb] < 0) continue;
-                            if (is_v) tma_load_3d(dst + jb * 4096, &tmv3, 0, ys[jb], 0, &full[s]);
-                            else tma_load_2d(dst + jb * 2048, &tmk2, p * 64, ys[jb], &full[s]);
+                            if (is_v) tma_load_3d(dst + jb * 4096, &tmv3, 0, ys[jb], 0, bar);
+                            else tma_load_2d(dst + jb * 2048, &tmk2, p * 64, ys[jb], bar);
                         }
                     }
                 }
                 __syncwarp();
+                if (tail) {
+                    // V rows past the context (stale or never loaded) must be zero, P
+                    // is 0 there: once the stage's V has landed, zero them, then
+                    // release the stage to the MMA thread
+                    const bool landed = mbar_wait(v_tma, (uint32_t)ntail & 1);
+                    ++ntail;
+                    if (!landed) {
+                        ok = false;
+                        break;
+                    }
+                    for (int i = lane; i < (kUKeys - valid_keys) * 16; i += 32) {
+                        const int key = valid_keys + i / 16, ch = i % 16;
+                        *(uint4 *)(dst + (key >> 4) * 4096 + (ch >> 3) * 2048 + (key & 15) * 128 + (ch & 7) * 16) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&full[s]);
+                }
             }
         }
         if (!ok) {
@@ -342,7 +400,6 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
         const uint32_t row_t = tmem + ((uint32_t)(sp * 32) << 16);
         const uint32_t s_col = (uint32_t)(t * 128), o_col = (uint32_t)(256 + t * 128);
         uint8_t *qbuf = sm + kUOffQ + t * kUQBytes;
-        uint8_t *pbuf = sm + kUOffP + t * kUPBytes + r * 128;
         int n = 0, n_item = 0;
         bool ok = true;
         for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++n_item) {
@@ -369,95 +426,80 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
             if (lane == 0) mbar_arrive(B.q_full);
             float m = -INFINITY, l = 0.f;
             for (int j = 0; j < it.nkt; ++j, ++n) {
-                const int b = n & 1;
-                if (!mbar_wait(&B.s_full[b], (uint32_t)(n >> 1) & 1)) {
+                if (!mbar_wait(B.s_full, (uint32_t)n & 1)) {
                     ok = false;
                     break;
                 }
                 tc_after();
-                uint32_t sv[64];
-                tmem_ld64(row_t + s_col + (uint32_t)(b * 64), sv);
+                uint32_t sa[64], sb[64];
+                tmem_ld64(row_t + s_col, sa);
+                tmem_ld64(row_t + s_col + 64u, sb);
                 tmem_wait_ld();
-                tc_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&B.s_free[b]);
                 const int k0 = j * kUKeys;
                 // scores in log2 units are s * scale_log2; the running max is kept in
-                // those units, the raw max (scale > 0) is taken first.  Stages wholly
-                // below every row's diagonal skip the mask.
-                float mx = -INFINITY;
-                if (__all_sync(0xffffffffu, valid && k0 + kUKeys - 1 <= pos)) {
-#pragma unroll
-                    for (int i = 0; i < 64; ++i) mx = fmaxf(mx, __uint_as_float(sv[i]));
-                } else {
+                // those units, the raw max (scale > 0) is taken first, in eight
+                // interleaved chains (the row sum below uses four partial sums).
+                // Stages wholly below every row's diagonal skip the mask.
+                if (!__all_sync(0xffffffffu, valid && k0 + kUKeys - 1 <= pos)) {
 #pragma unroll
                     for (int i = 0; i < 64; ++i) {
-                        const float sc = (valid && k0 + i <= pos) ? __uint_as_float(sv[i]) : -INFINITY;
-                        sv[i] = __float_as_uint(sc);
-                        mx = fmaxf(mx, sc);
+                        if (!(valid && k0 + i <= pos)) sa[i] = __float_as_uint(-INFINITY);
+                        if (!(valid && k0 + 64 + i <= pos)) sb[i] = __float_as_uint(-INFINITY);
                     }
                 }
-                mx *= prm.scale_log2;
-                // the P V of the previous stage has finished: P is free and O is final
-                if (n >= 1 && !mbar_wait(B.pv_done, (uint32_t)(n - 1) & 1)) {
-                    ok = false;
-                    break;
-                }
+                float mt[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mt[i] = fmaxf(__uint_as_float(sa[i]), __uint_as_float(sb[i]));
+#pragma unroll
+                for (int i = 8; i < 64; ++i)
+                    mt[i & 7] = fmaxf(mt[i & 7], fmaxf(__uint_as_float(sa[i]), __uint_as_float(sb[i])));
+#pragma unroll
+                for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+                    for (int i = 0; i < w; ++i) mt[i] = fmaxf(mt[i], mt[i + w]);
+                const float mx = mt[0] * prm.scale_log2;
+                float alpha = 1.f;
+                bool resc = false;
                 if (__any_sync(0xffffffffu, mx > m + kURescaleLog2)) {
                     const float mn = fmaxf(m, mx);
-                    const float alpha = mn == -INFINITY ? 1.f : fast_exp2(m - mn);
-                    if (j > 0) {  // O holds earlier stages: rescale it in place
-                        tc_after();
-#pragma unroll 1
-                        for (int q8 = 0; q8 < 8; ++q8) {
-                            uint32_t ov[16];
-                            tmem_ld16(row_t + o_col + (uint32_t)(q8 * 16), ov);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                            tmem_st16(row_t + o_col + (uint32_t)(q8 * 16), ov);
-                        }
-                        tmem_wait_st();
-                    }
+                    alpha = mn == -INFINITY ? 1.f : fast_exp2(m - mn);
+                    resc = j > 0;  // O holds earlier stages
                     m = mn;
                     l *= alpha;
                 }
                 const float bm = m == -INFINITY ? 0.f : m;
                 const float sl = prm.scale_log2;
-                float ps = 0.f;
+                float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+                // P as bf16 over the first 64 columns of S: keys 16c..16c+15 in
+                // columns 8c..8c+7, two keys per column, the even one in the low half
 #pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
-                    float pv[8];
+                for (int c = 0; c < kUBlk; ++c) {
+                    uint32_t pk[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        pv[i] = fast_exp2(fmaf(__uint_as_float(sv[8 * c8 + i]), sl, -bm));
-                        ps += pv[i];
+                        const int key = 16 * c + 2 * i;
+                        const float x0 = __uint_as_float(key < 64 ? sa[key] : sb[key - 64]);
+                        const float x1 = __uint_as_float(key + 1 < 64 ? sa[key + 1] : sb[key + 1 - 64]);
+                        const float p0 = fast_exp2(fmaf(x0, sl, -bm)), p1 = fast_exp2(fmaf(x1, sl, -bm));
+                        ps4[(2 * i) & 3] += p0;
+                        ps4[(2 * i + 1) & 3] += p1;
+                        pk[i] = pack_bf16(p0, p1);
                     }
-                    uint4 w;
-                    w.x = pack_bf16(pv[0], pv[1]);
-                    w.y = pack_bf16(pv[2], pv[3]);
-                    w.z = pack_bf16(pv[4], pv[5]);
-                    w.w = pack_bf16(pv[6], pv[7]);
-                    *(uint4 *)(pbuf + ((c8 ^ (r & 7)) << 4)) = w;
+                    tmem_st8(row_t + s_col + (uint32_t)(8 * c), pk);
                 }
-                l += ps;
-                const int valid_keys = it.c - k0;
-                if (valid_keys < kUKeys) {
-                    // V rows past the context (stale or unloaded) must be zero: P is 0
-                    // there.  Both warpgroups write the same zeros, after the stage's V
-                    // has landed; the MMA thread waits for both before either P V.
-                    if (!mbar_wait(&v_full[n % kUVStages], (uint32_t)(n / kUVStages) & 1)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t *vs = sm + kUOffV + (size_t)(n % kUVStages) * kUVBytes;
-                    for (int i = r; i < (kUKeys - valid_keys) * 16; i += kURows) {
-                        const int key = valid_keys + i / 16, ch = i % 16;
-                        *(uint4 *)(vs + (key >> 4) * 4096 + (ch >> 3) * 2048 + (key & 15) * 128 + (ch & 7) * 16) =
-                            make_uint4(0u, 0u, 0u, 0u);
+                l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
+                if (resc) {  // O_t is stable: its last P V completed before this S did
+#pragma unroll 1
+                    for (int q8 = 0; q8 < 8; ++q8) {
+                        uint32_t ov[16];
+                        tmem_ld16(row_t + o_col + (uint32_t)(q8 * 16), ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                        tmem_st16(row_t + o_col + (uint32_t)(q8 * 16), ov);
                     }
                 }
-                fence_proxy_async();
+                tmem_wait_st();
                 tc_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(B.p_full);
@@ -501,67 +543,63 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
         if (lane == 0) {
             bool ok = true;
             int n = 0, n_item = 0;
-            // O += P V of stage nn for both row tiles (both softmax warpgroups done)
-            auto pv = [&](int nn, bool first) -> bool {
-                for (int t = 0; t < kUTiles; ++t) {
-                    const UTileBars B = tb(t);
-                    if (!mbar_wait(B.p_full, (uint32_t)nn & 1)) return false;
-                    if (first && n_item > 0 && !mbar_wait(B.o_free, (uint32_t)(n_item - 1) & 1)) return false;
-                }
+            // O_t += P_t V of stage nn (first: the item's first stage, which
+            // overwrites O_t once the previous item's epilogue has read it)
+            auto pv = [&](int t, int nn, bool first) -> bool {
+                const UTileBars B = tb(t);
+                if (!mbar_wait(B.p_full, (uint32_t)nn & 1)) return false;
+                if (first && n_item > 0 && !mbar_wait(B.o_free, (uint32_t)(n_item - 1) & 1)) return false;
                 const int s = nn % kUVStages;
-                if (!mbar_wait(&v_full[s], (uint32_t)(nn / kUVStages) & 1)) return false;
+                if (t == 0 && !mbar_wait(&v_full[s], (uint32_t)(nn / kUVStages) & 1)) return false;
                 tc_after();
-                const uint32_t va = smem_u32(sm + kUOffV + (size_t)s * kUVBytes);
-                for (int t = 0; t < kUTiles; ++t) {
-                    const uint32_t pa = smem_u32(sm + kUOffP + t * kUPBytes);
+                const uint32_t vlo = sdesc_lo(smem_u32(sm + kUOffV + (size_t)s * kUVBytes), 2048);
 #pragma unroll
-                    for (int kp = 0; kp < 4; ++kp)
-                        umma_f16(tmem + 256u + (uint32_t)(t * 128), sdesc(pa + kp * 32, 16, 1024),
-                                 sdesc(va + kp * 4096, 2048, 1024), kIdescPV, (first && kp == 0) ? 0u : 1u);
-                    umma_commit(tb(t).pv_done);
-                }
-                umma_commit(&v_empty[s]);
+                for (int kp = 0; kp < kUBlk; ++kp)
+                    umma_ts(tmem + 256u + (uint32_t)(t * 128), tmem + (uint32_t)(t * 128 + 8 * kp), vlo + kp * 256,
+                            kIdescPV, (first && kp == 0) ? 0u : 1u);
                 return true;
+            };
+            // S_t = Q_t K^T of the stage in K slot s, over S_t's (and P_t's) columns
+            auto s_mma = [&](int t, int s) {
+                const uint32_t klo = sdesc_lo(smem_u32(sm + kUOffK + (size_t)s * kUKBytes), 16);
+                const uint32_t qlo = sdesc_lo(smem_u32(sm + kUOffQ + t * kUQBytes), 16);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ss(tmem + (uint32_t)(t * 128), qlo + (uint32_t)((kk >> 2) * (kURows * 128) + (kk & 3) * 32) / 16,
+                            klo + (uint32_t)((kk >> 2) * kUKPanel + (kk & 3) * 32) / 16, kIdescS, kk > 0 ? 1u : 0u);
+                umma_commit(tb(t).s_full);
             };
             for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++n_item) {
                 UItem it;
                 item_of(idx, it);
                 for (int t = 0; t < kUTiles && ok; ++t) ok = mbar_wait(tb(t).q_full, (uint32_t)n_item & 1);
                 if (!ok) break;
-                tc_after();
                 for (int j = 0; j < it.nkt; ++j, ++n) {
-                    const int s = n % kUKStages, b = n & 1;
-                    bool got = mbar_wait(&k_full[s], (uint32_t)(n / kUKStages) & 1);
-                    for (int t = 0; t < kUTiles && got; ++t)
-                        if (n >= 2) got = mbar_wait(&tb(t).s_free[b], (uint32_t)((n >> 1) - 1) & 1);
-                    if (!got || *abort_flag) {
+                    const int s = n % kUKStages;
+                    if (!mbar_wait(&k_full[s], (uint32_t)(n / kUKStages) & 1) || *abort_flag) {
                         ok = false;
                         break;
                     }
                     tc_after();
-                    const uint32_t ka = smem_u32(sm + kUOffK + (size_t)s * kUKBytes);
                     for (int t = 0; t < kUTiles; ++t) {
-                        const uint32_t qa = smem_u32(sm + kUOffQ + t * kUQBytes);
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            umma_f16(tmem + (uint32_t)(t * 128 + b * 64),
-                                     sdesc(qa + (kk >> 2) * (kURows * 128) + (kk & 3) * 32, 16, 1024),
-                                     sdesc(ka + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), kIdescS,
-                                     kk > 0 ? 1u : 0u);
-                        umma_commit(&tb(t).s_full[b]);
+                        // P_t V of the previous stage, then S_t of this one in the same columns
+                        if (j > 0 && !pv(t, n - 1, j == 1)) {
+                            ok = false;
+                            break;
+                        }
+                        s_mma(t, s);
                     }
+                    if (!ok) break;
                     umma_commit(&k_empty[s]);  // the K slot is free once both S have completed
-                    if (j > 0 && !pv(n - 1, j == 1)) {
-                        ok = false;
-                        break;
-                    }
+                    if (j > 0) umma_commit(&v_empty[(n - 1) % kUVStages]);
                 }
                 if (!ok) break;
-                if (!pv(n - 1, it.nkt == 1)) {
-                    ok = false;
-                    break;
+                for (int t = 0; t < kUTiles && ok; ++t) {
+                    ok = pv(t, n - 1, it.nkt == 1);
+                    if (ok) umma_commit(tb(t).o_full);
                 }
-                for (int t = 0; t < kUTiles; ++t) umma_commit(tb(t).o_full);
+                if (!ok) break;
+                umma_commit(&v_empty[(n - 1) % kUVStages]);
             }
             if (!ok) {
                 record_error(prm.err, PK_ERR_TIMEOUT);
@@ -594,6 +632,11 @@ int chunk_umma_prepare_pool(pk_pool *p) {
     cudaError_t ce = cudaFuncSetAttribute(attention_chunk_umma_kernel,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kUSmem);
     if (ce != cudaSuccess) return cuda_fail(ce, "set chunk (tcgen05) smem size");
+    // the warpgroups' register split assumes this launch register count
+    cudaFuncAttributes fa;
+    ce = cudaFuncGetAttributes(&fa, attention_chunk_umma_kernel);
+    if (ce != cudaSuccess) return cuda_fail(ce, "chunk (tcgen05) attributes");
+    if (fa.numRegs != kURegLaunch) return PK_OK;
     int rc = encode_pool_map(&p->tmap_k2, p->k_base, p, kTile);
     if (rc == PK_OK) rc = encode_pool_map(&p->tmap_v2, p->v_base, p, kTile);
     if (rc != PK_OK) return rc;
