@@ -351,16 +351,20 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
 #pragma unroll
                     for (int jb = 0; jb < kUBlk; ++jb)
                         if (ys[jb] >= 0) bytes += is_v ? 4096u : 2048u;
-                    if (bytes == 0) {
-                        mbar_arrive(bar);  // keys past the context: nothing to load
-                    } else {
-                        mbar_arrive_expect_tx(bar, bytes);
+                    if (bytes == 0) mbar_arrive(bar);  // keys past the context: nothing to load
+                    else mbar_arrive_expect_tx(bar, bytes);
+                }
+                __syncwarp();
+                {
+                    // lane jb issues block jb's box: a warp's TMA instructions issue one
+                    // at a time, so eight lanes start a stage's boxes together
+                    int my = -1;
 #pragma unroll
-                        for (int jb = 0; jb < kUBlk; ++jb) {
-                            if (ys[jb] < 0) continue;
-                            if (is_v) tma_load_3d(dst + jb * 4096, &tmv3, 0, ys[jb], 0, bar);
-                            else tma_load_2d(dst + jb * 2048, &tmk2, p * 64, ys[jb], bar);
-                        }
+                    for (int jb = 0; jb < kUBlk; ++jb)
+                        if (lane == jb) my = ys[jb];
+                    if (my >= 0) {
+                        if (is_v) tma_load_3d(dst + lane * 4096, &tmv3, 0, my, 0, bar);
+                        else tma_load_2d(dst + lane * 2048, &tmk2, p * 64, my, bar);
                     }
                 }
                 __syncwarp();
