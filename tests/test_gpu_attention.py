@@ -120,10 +120,13 @@ def test_chunks_at_successive_offsets(cuda_dev):
         _check(b, Hq, Hkv, d, torch.bfloat16, cuda_dev, f"chunk at {start}")
 
 
-def test_permuted_block_ids_bit_identical(cuda_dev):
+@pytest.mark.parametrize("ql", [[1, 40, 1, 33], [1, 1, 1, 1]], ids=["mixed", "decode_only"])
+def test_permuted_block_ids_bit_identical(cuda_dev, ql):
     # paging must not change attention: same logical K/V under five different
     # physical permutations gives bit-identical GPU output, equal to the oracle
-    ctx, ql, Hkv, Hq, d = [700, 90, 1500, 33], [1, 40, 1, 33], 8, 32, 128
+    # (mixed: chunk and tile-decode kernels; decode_only: block-streaming decode
+    # kernel with its split-K merge)
+    ctx, Hkv, Hq, d = [700, 90, 1500, 33], 8, 32, 128
     g = torch.Generator().manual_seed(21)
     k_seq = [torch.randn((c, Hkv, d), generator=g).to(torch.bfloat16) for c in ctx]
     v_seq = [torch.randn((c, Hkv, d), generator=g).to(torch.bfloat16) for c in ctx]
