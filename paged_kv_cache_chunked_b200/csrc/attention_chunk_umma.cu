@@ -641,8 +641,8 @@ int chunk_umma_prepare_pool(pk_pool *p) {
     ce = cudaFuncGetAttributes(&fa, attention_chunk_umma_kernel);
     if (ce != cudaSuccess) return cuda_fail(ce, "chunk (tcgen05) attributes");
     if (fa.numRegs != kURegLaunch) return PK_OK;
-    int rc = encode_pool_map(&p->tmap_k2, p->k_base, p, kTile);
-    if (rc == PK_OK) rc = encode_pool_map(&p->tmap_v2, p->v_base, p, kTile);
+    // K as 2-D 16-row boxes of one 64-column panel; V uses the pool's 3-D tile map
+    const int rc = encode_pool_map(&p->tmap_k2, p->k_base, p, kTile);
     if (rc != PK_OK) return rc;
     p->umma_ok = true;
     return PK_OK;

@@ -32,7 +32,6 @@ struct pk_pool {
     alignas(64) CUtensorMap tmap_kb;  // 3-D boxes of blk_hs * block_size rows, all panels
     alignas(64) CUtensorMap tmap_vb;
     alignas(64) CUtensorMap tmap_k2;  // 2-D, 16-row boxes: K tiles of the tcgen05 chunk kernel
-    alignas(64) CUtensorMap tmap_v2;  // 2-D, 16-row boxes over V
 };
 
 namespace pk {
