@@ -123,6 +123,26 @@ int pk_block_copy(const pk_pool *pool, const int32_t *src_dst_pairs, int n_pairs
                   pk_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Block swap between the device pool and a host pool  [BP "When blocks run
+ * out": a preempted request's blocks are swapped out to CPU memory and later
+ * back, all blocks of a sequence together]
+ *
+ * host_k, host_v: page-locked host memory of num_host_blocks blocks with the
+ * pool's block geometry and dtype ([H][n_kv_heads][block_size][head_dim]),
+ * mapped for device access (cudaHostAlloc, or pinned torch tensors); the
+ * call checks this with cudaPointerGetAttributes and returns
+ * PK_ERR_INVALID_ARG otherwise.  pairs: device int32 [n_pairs][2]; to_host
+ * != 0: (device block, host block), host block := device block; to_host == 0:
+ * (host block, device block), device block := host block.  Whole blocks, K and
+ * V, bit-exact; the destinations of one call must be distinct.  Ids outside
+ * either pool are recorded as PK_ERR_BAD_INDEX and skipped.  Asynchronous on
+ * the stream: the host pool must stay allocated, and its swapped-out blocks
+ * must not be read on the host, until the stream has passed the call.
+ * ------------------------------------------------------------------------ */
+int pk_swap_blocks(const pk_pool *pool, void *host_k, void *host_v, int num_host_blocks,
+                   const int32_t *pairs, int n_pairs, int to_host, pk_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Paged attention  [SN "Block tables": the kernel gathers through the table;
  * BP "PagedAttention" item 4; BP "Continuous batching": one step mixes
  * prefill chunks and decodes, long prompts are split into chunks]
@@ -210,6 +230,8 @@ typedef struct {
     int64_t alloc_failures;   /* append_slots calls refused with PK_ERR_OOM */
     int64_t tail_waste_slots; /* unwritten slots over all blocks in use, each block once */
     int64_t num_seqs;
+    int64_t host_blocks;      /* host (swap) pool size, 0 until pk_bm_set_host_blocks */
+    int64_t host_free_blocks;
 } pk_bm_stats;
 
 int pk_bm_create(int num_blocks, int block_size, pk_bm **out);
@@ -231,6 +253,28 @@ int pk_bm_blocks_needed(const pk_bm *bm, int64_t seq, int n, int *needed_out);
 int pk_bm_fork(pk_bm *bm, int64_t parent, int64_t *child_out);
 /* Drop seq; blocks no longer referenced return to the free list. */
 int pk_bm_free(pk_bm *bm, int64_t seq);
+/* Swapping [BP "When blocks run out": a preempted request's blocks are
+ * swapped out to CPU memory, or freed and recomputed later; all blocks of a
+ * sequence are evicted together].
+ * pk_bm_set_host_blocks gives the manager a host pool of num_host_blocks
+ * blocks (once; FIFO free list 0..H-1).
+ * pk_bm_swap_out moves every block of a resident seq to the host pool:
+ * pairs_out (int32 [pairs_cap][2]) receives one (device block, host block)
+ * pair per table entry in logical order, the device blocks return to the free
+ * list (last logical block first) and the table now names host blocks.  The
+ * caller runs pk_swap_blocks(..., to_host = 1) on the pairs before anything
+ * else writes those device blocks.  PK_ERR_UNSUPPORTED: the sequence shares a
+ * block (reference count > 1); PK_ERR_OOM: too few free host blocks; nothing
+ * changes in either case.
+ * pk_bm_swap_in is the reverse: (host block, device block) pairs, run with
+ * to_host = 0; PK_ERR_OOM: too few free device blocks, nothing changed.
+ * A swapped sequence accepts only swap_in, free (its host blocks return),
+ * block_table (host ids), seq_len and is_swapped; other calls return
+ * PK_ERR_INVALID_ARG. */
+int pk_bm_set_host_blocks(pk_bm *bm, int num_host_blocks);
+int pk_bm_swap_out(pk_bm *bm, int64_t seq, int32_t *pairs_out, int pairs_cap, int *n_pairs_out);
+int pk_bm_swap_in(pk_bm *bm, int64_t seq, int32_t *pairs_out, int pairs_cap, int *n_pairs_out);
+int pk_bm_is_swapped(const pk_bm *bm, int64_t seq, int *swapped_out);
 /* Copy seq's block table (ceil(len / bs) ids) into out[cap]; *n_out = count. */
 int pk_bm_block_table(const pk_bm *bm, int64_t seq, int32_t *out, int cap, int *n_out);
 /* Fill out[n_seqs][width] (int32, row-major) with the tables of seqs[], -1 padded. */

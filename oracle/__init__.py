@@ -9,11 +9,11 @@ Contents
 ``attention.c`` (float64 C, built here into ``liboracle.so``)
     paged attention with causal chunks and GQA, the plain definition.
 ``kv_ops.py``
-    slot-mapped KV append and whole-block copy (copy-on-write), element by
-    element.
+    slot-mapped KV append, whole-block copy (copy-on-write) and whole-block
+    swaps between the device pool and a host pool.
 ``allocator.py``
     host block manager: free list, block tables, reference counts, fork,
-    copy-on-write, tail-waste accounting.
+    copy-on-write, tail-waste accounting, swapping to a host pool.
 ``capacity.py``
     the capacity arithmetic the pages print (token-slot toy, KV bytes per
     token, sessions per pool).
@@ -22,6 +22,6 @@ Every pin that ties these to the pages lives in ``tests/test_oracle_*.py``.
 """
 
 from .attention import paged_attention, paged_attention_rows, num_threads  # noqa: F401
-from .kv_ops import kv_append, block_copy  # noqa: F401
+from .kv_ops import kv_append, block_copy, swap_blocks  # noqa: F401
 from .allocator import OracleBlockManager, OracleOOM  # noqa: F401
 from . import capacity  # noqa: F401

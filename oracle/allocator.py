@@ -33,6 +33,25 @@ same ones, so block tables can be compared bit for bit):
     allocation failure;
   * tail waste counts every physical block in use once: block_size minus the
     slots written in it.
+
+Swapping [Batching and PagedAttention, "When blocks run out": a preempted
+request's blocks are either swapped out to CPU memory or freed and recomputed
+later; all blocks of a sequence are evicted together]:
+  * a host pool of equal blocks with its own free list, first in, first out
+    from 0, 1, ..., H-1, like the device one;
+  * swap_out(seq) moves every block of seq to the host pool at once: one host
+    block per table entry, taken in logical order; the device blocks are then
+    released from the last logical block to the first; the table now names
+    host blocks and the sequence is "swapped";
+  * swap_in(seq) does the reverse: device blocks taken in logical order, host
+    blocks released last to first; the slots written in each block travel
+    with it;
+  * a sequence holding a shared block (count > 1) is not swapped: its blocks
+    also belong to other sequences, so they cannot all leave with it (the
+    caller recomputes it instead); a swap that cannot be met in full (host or
+    device pool short) changes nothing;
+  * a swapped sequence can only be swapped in or freed (freeing returns its
+    host blocks, last to first).
 """
 
 from collections import deque
@@ -55,6 +74,10 @@ class OracleBlockManager:
         self.lengths = {}                   # seq id -> tokens stored
         self.next_seq = 0
         self.alloc_failures = 0
+        self.host_blocks = 0
+        self.host_free = deque()
+        self.host_filled = []
+        self.swapped = set()
 
     # -- sequences -----------------------------------------------------
     def add_seq(self):
@@ -76,8 +99,15 @@ class OracleBlockManager:
             self.filled[block] = 0
             self.free_list.append(block)
 
+    def _resident(self, seq):
+        if seq not in self.tables:
+            raise KeyError(seq)
+        if seq in self.swapped:
+            raise ValueError(f"sequence {seq} is swapped out")
+
     def blocks_needed(self, seq, n):
         """Blocks an append of n tokens to seq would take from the free list."""
+        self._resident(seq)
         length, table, bs = self.lengths[seq], self.tables[seq], self.block_size
         if n <= 0:
             return 0
@@ -92,8 +122,7 @@ class OracleBlockManager:
         (source, destination) block pairs that must be copied before the
         tokens are written.  Raises OracleOOM with nothing changed.
         """
-        if seq not in self.tables:
-            raise KeyError(seq)
+        self._resident(seq)
         if n < 0:
             raise ValueError("negative token count")
         if self.blocks_needed(seq, n) > len(self.free_list):
@@ -121,8 +150,7 @@ class OracleBlockManager:
 
     def fork(self, parent):
         """New sequence sharing every block of parent (reference counts +1)."""
-        if parent not in self.tables:
-            raise KeyError(parent)
+        self._resident(parent)
         child = self.next_seq
         self.next_seq += 1
         self.tables[child] = list(self.tables[parent])
@@ -132,11 +160,72 @@ class OracleBlockManager:
         return child
 
     def free(self, seq):
-        """Drop seq; blocks whose count reaches zero return to the free list."""
+        """Drop seq; blocks whose count reaches zero return to the free list
+        (a swapped sequence returns its host blocks)."""
         table = self.tables.pop(seq)
         del self.lengths[seq]
+        if seq in self.swapped:
+            self.swapped.discard(seq)
+            for h in reversed(table):
+                self._release_host(h)
+            return
         for block in reversed(table):
             self._release(block)
+
+    # -- swapping ------------------------------------------------------
+    def set_host_blocks(self, n):
+        """Give the manager a host pool of n blocks (once)."""
+        if n < 0 or self.host_blocks:
+            raise ValueError("host pool already set or negative")
+        self.host_blocks = n
+        self.host_free = deque(range(n))
+        self.host_filled = [0] * n
+
+    def _release_host(self, h):
+        self.host_filled[h] = 0
+        self.host_free.append(h)
+
+    def swap_out(self, seq):
+        """Move all of seq's blocks to the host pool.  Returns the (device,
+        host) block pairs to copy, in logical order.  Raises ValueError for a
+        sequence that shares a block or is already swapped, OracleOOM when the
+        host pool is short; nothing changes then."""
+        self._resident(seq)
+        table = self.tables[seq]
+        if any(self.refcount[b] > 1 for b in table):
+            raise ValueError(f"sequence {seq} shares blocks")
+        if len(table) > len(self.host_free):
+            raise OracleOOM(seq)
+        pairs = []
+        for b in table:
+            h = self.host_free.popleft()
+            self.host_filled[h] = self.filled[b]
+            pairs.append((b, h))
+        for b in reversed(table):
+            self._release(b)
+        self.tables[seq] = [h for _, h in pairs]
+        self.swapped.add(seq)
+        return pairs
+
+    def swap_in(self, seq):
+        """Bring a swapped sequence's blocks back to the device pool.  Returns
+        the (host, device) pairs to copy, in logical order.  Raises OracleOOM
+        when the device pool is short (nothing changes then)."""
+        if seq not in self.swapped:
+            raise ValueError(f"sequence {seq} is not swapped out")
+        table = self.tables[seq]
+        if len(table) > len(self.free_list):
+            raise OracleOOM(seq)
+        pairs = []
+        for h in table:
+            b = self._take()
+            self.filled[b] = self.host_filled[h]
+            pairs.append((h, b))
+        for h in reversed(table):
+            self._release_host(h)
+        self.tables[seq] = [b for _, b in pairs]
+        self.swapped.discard(seq)
+        return pairs
 
     # -- views ---------------------------------------------------------
     def block_table(self, seq):
@@ -164,4 +253,6 @@ class OracleBlockManager:
             "alloc_failures": self.alloc_failures,
             "tail_waste_slots": self.tail_waste(),
             "num_seqs": len(self.tables),
+            "host_blocks": self.host_blocks,
+            "host_free_blocks": len(self.host_free),
         }

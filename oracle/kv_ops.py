@@ -12,8 +12,11 @@ block_copy
     writes" [same page, "Copy-on-write"].  The copy moves the whole physical
     block (all heads, all slots, K and V).  All pairs of one call read the
     state from before the call.
+swap_blocks
+    Whole blocks moved between the device pool and a host pool, the swap a
+    preemption may use instead of recomputation.
 
-Both work element by element on CPU torch tensors, in place.
+All work on CPU torch tensors, in place.
 """
 
 import torch
@@ -43,3 +46,20 @@ def block_copy(k_pool, v_pool, src_dst_pairs):
     for src, dst in pairs:
         k_pool[dst] = k_before[src]
         v_pool[dst] = v_before[src]
+
+
+def swap_blocks(k_pool, v_pool, host_k, host_v, pairs, to_host):
+    """Whole-block moves between the device pool and a host pool of the same
+    block geometry [Batching and PagedAttention, "When blocks run out": a
+    preempted request's blocks are swapped out to CPU memory and later back].
+    to_host: pairs are (device block, host block) and host[h] = pool[d];
+    otherwise pairs are (host block, device block) and pool[d] = host[h].
+    K and V alike."""
+    pairs = [(int(a), int(b)) for a, b in torch.as_tensor(pairs).reshape(-1, 2).tolist()]
+    for a, b in pairs:
+        if to_host:
+            host_k[b] = k_pool[a]
+            host_v[b] = v_pool[a]
+        else:
+            k_pool[b] = host_k[a]
+            v_pool[b] = host_v[a]

@@ -31,7 +31,8 @@ class OutOfBlocks(PagedKVError):
 class BmStats(ctypes.Structure):
     _fields_ = [("num_blocks", ctypes.c_int64), ("free_blocks", ctypes.c_int64),
                 ("used_blocks", ctypes.c_int64), ("alloc_failures", ctypes.c_int64),
-                ("tail_waste_slots", ctypes.c_int64), ("num_seqs", ctypes.c_int64)]
+                ("tail_waste_slots", ctypes.c_int64), ("num_seqs", ctypes.c_int64),
+                ("host_blocks", ctypes.c_int64), ("host_free_blocks", ctypes.c_int64)]
 
 
 _lib = None
@@ -50,6 +51,7 @@ SIGNATURES = {
     "pk_check_device_errors": ([_P, _P, _PI], _I),
     "pk_paged_kv_append": ([_P, _P, _P, _P, _I, _P], _I),
     "pk_block_copy": ([_P, _P, _I, _P], _I),
+    "pk_swap_blocks": ([_P, _P, _P, _I, _P, _I, _I, _P], _I),
     "pk_attention_workspace_size": ([_P, _I, _I, _I, _I, _PSZ], _I),
     "pk_paged_attention": ([_P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _F, _P, _SZ, _P], _I),
     "pk_paged_attention_noalloc": ([_P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _F, _P], _I),
@@ -64,6 +66,10 @@ SIGNATURES = {
     "pk_bm_fill_tables": ([_P, _P, _I, _P, _I], _I),
     "pk_bm_seq_len": ([_P, _I64, _PI64], _I),
     "pk_bm_refcount": ([_P, ctypes.c_int32, _PI], _I),
+    "pk_bm_set_host_blocks": ([_P, _I], _I),
+    "pk_bm_swap_out": ([_P, _I64, _P, _I, _PI], _I),
+    "pk_bm_swap_in": ([_P, _I64, _P, _I, _PI], _I),
+    "pk_bm_is_swapped": ([_P, _I64, _PI], _I),
     "pk_bm_get_stats": ([_P, ctypes.POINTER(BmStats)], _I),
 }
 

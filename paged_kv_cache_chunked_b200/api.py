@@ -8,6 +8,8 @@ the library's CUDA kernels.  PyTorch supplies device memory and streams.
     out = paged_attention(q, pool.k_pool, pool.v_pool, block_tables, context_lens,
                           query_start_lens, scale)
     block_copy(src_dst_pairs, pool=pool)
+    host = host_pool_create(num_host_blocks, pool)        # pinned, for swapping
+    swap_blocks(pairs, to_host=True, host_pool=host, pool=pool)
 """
 
 import ctypes
@@ -142,6 +144,34 @@ def block_copy(src_dst_pairs, *, pool):
     check(lib().pk_block_copy(pool.handle, _ptr(src_dst_pairs), src_dst_pairs.shape[0], _stream(d)))
 
 
+class HostPool:
+    """Page-locked host blocks with a device pool's block geometry, the target
+    of swapped-out blocks: k / v [num_host_blocks, n_kv_heads, block_size,
+    head_dim] pinned CPU tensors."""
+
+    def __init__(self, num_host_blocks, pool):
+        shape = (num_host_blocks, pool.n_kv_heads, pool.block_size, pool.head_dim)
+        self.k = torch.zeros(shape, dtype=pool.dtype, pin_memory=True)
+        self.v = torch.zeros(shape, dtype=pool.dtype, pin_memory=True)
+        self.num_blocks = num_host_blocks
+
+
+def host_pool_create(num_host_blocks, pool):
+    return HostPool(num_host_blocks, pool)
+
+
+def swap_blocks(pairs, *, to_host, host_pool, pool):
+    """Move whole blocks between the device pool and a host pool (int32
+    [n, 2] pairs on the pool's device): to_host, (device, host) pairs;
+    otherwise (host, device) pairs.  Asynchronous on the current stream."""
+    d = pool.device
+    _need(pairs, "pairs", torch.int32, d)
+    if pairs.dim() != 2 or pairs.shape[1] != 2:
+        raise ValueError("pairs must be [n, 2]")
+    check(lib().pk_swap_blocks(pool.handle, _ptr(host_pool.k), _ptr(host_pool.v), host_pool.num_blocks,
+                               _ptr(pairs), pairs.shape[0], 1 if to_host else 0, _stream(d)))
+
+
 def paged_attention(q, k_pool, v_pool, block_tables, context_lens, query_start_lens, scale,
                     out=None):
     """Attention of q ([T, Hq, d]) over each sequence's paged K/V.
@@ -210,6 +240,32 @@ class BlockManager:
 
     def free(self, seq):
         check(lib().pk_bm_free(self._h, seq))
+
+    def set_host_blocks(self, num_host_blocks):
+        check(lib().pk_bm_set_host_blocks(self._h, num_host_blocks))
+
+    def _swap(self, fn, seq):
+        cap = self.length(seq) // self.block_size + 2
+        buf = (ctypes.c_int32 * (2 * cap))()
+        n = ctypes.c_int()
+        check(fn(self._h, seq, buf, cap, ctypes.byref(n)))
+        return [(buf[2 * i], buf[2 * i + 1]) for i in range(n.value)]
+
+    def swap_out(self, seq):
+        """Move all of seq's blocks to the host pool; returns the (device, host)
+        pairs to copy.  Raises OutOfBlocks (host pool short) or PagedKVError
+        (shared blocks), with nothing changed."""
+        return self._swap(lib().pk_bm_swap_out, seq)
+
+    def swap_in(self, seq):
+        """Bring a swapped seq back; returns the (host, device) pairs to copy.
+        Raises OutOfBlocks with nothing changed."""
+        return self._swap(lib().pk_bm_swap_in, seq)
+
+    def is_swapped(self, seq):
+        r = ctypes.c_int()
+        check(lib().pk_bm_is_swapped(self._h, seq, ctypes.byref(r)))
+        return bool(r.value)
 
     def block_table(self, seq):
         n = ctypes.c_int()

@@ -200,6 +200,28 @@ int pk_block_copy(const pk_pool *pool, const int32_t *src_dst_pairs, int n_pairs
     return launch_block_copy(pool, src_dst_pairs, n_pairs, (cudaStream_t)stream);
 }
 
+int pk_swap_blocks(const pk_pool *pool, void *host_k, void *host_v, int num_host_blocks,
+                   const int32_t *pairs, int n_pairs, int to_host, pk_stream_t stream) {
+    if (!pool) return fail(PK_ERR_INVALID_ARG, "pool is NULL");
+    if (n_pairs < 0 || num_host_blocks < 0) return fail(PK_ERR_INVALID_ARG, "negative count");
+    if (n_pairs == 0) return PK_OK;
+    if (!pairs || !host_k || !host_v) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    // the kernel reaches the host pool through its device mapping: only
+    // page-locked host memory with one is accepted
+    void *view[2] = {nullptr, nullptr};
+    void *host[2] = {host_k, host_v};
+    for (int i = 0; i < 2; ++i) {
+        cudaPointerAttributes at;
+        const cudaError_t e = cudaPointerGetAttributes(&at, host[i]);
+        if (e != cudaSuccess) return cuda_fail(e, "host pool pointer attributes");
+        if (at.type != cudaMemoryTypeHost || at.devicePointer == nullptr)
+            return fail(PK_ERR_INVALID_ARG, "host pool is not page-locked host memory mapped for the device");
+        view[i] = at.devicePointer;
+    }
+    return launch_swap_blocks(pool, view[0], view[1], num_host_blocks, pairs, n_pairs, to_host != 0,
+                              (cudaStream_t)stream);
+}
+
 int pk_attention_workspace_size(const pk_pool *pool, int num_seqs, int num_tokens,
                                 int n_q_heads, int max_blocks_per_seq, size_t *bytes_out) {
     if (!pool || !bytes_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");

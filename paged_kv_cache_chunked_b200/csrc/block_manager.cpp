@@ -18,6 +18,16 @@
 //  * the operational counters the deep-dive page lists: free and used
 //    blocks, allocation failures, tail waste.
 //
+// Swapping ["Batching and PagedAttention", "When blocks run out": a preempted
+// request's blocks are swapped out to CPU memory or freed and recomputed; all
+// blocks of a sequence are evicted together]: a host pool with its own FIFO
+// free list; swap_out moves every block of a sequence at once (host blocks
+// taken in logical order, device blocks then released last to first; the
+// table then names host blocks), swap_in the reverse.  A sequence that shares
+// a block is not swapped (its blocks also belong to other sequences); a swap
+// that cannot be met in full changes nothing.  A swapped sequence can only be
+// swapped in or freed.
+//
 // Policy details the pages leave open, fixed so that tables are reproducible:
 // FIFO free list starting as 0..N-1 (a released block joins the tail);
 // a sequence's blocks are released from its last logical block to its first;
@@ -44,7 +54,11 @@ struct pk_bm {
     struct Seq {
         std::vector<int32_t> table;
         int64_t len = 0;
+        bool swapped = false;  // table names host blocks
     };
+    int num_host_blocks = 0;
+    std::deque<int32_t> host_free;
+    std::vector<int32_t> host_filled;
     std::unordered_map<int64_t, Seq> seqs;
     int64_t next_seq = 0;
     int64_t alloc_failures = 0;
@@ -72,6 +86,23 @@ struct pk_bm {
 };
 
 using pk::fail;
+
+namespace {
+// the sequence, if it exists and is resident on the device
+pk_bm::Seq *resident(pk_bm *bm, int64_t seq) {
+    auto it = bm->seqs.find(seq);
+    if (it == bm->seqs.end()) {
+        fail(PK_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq);
+        return nullptr;
+    }
+    if (it->second.swapped) {
+        fail(PK_ERR_INVALID_ARG, "sequence %lld is swapped out", (long long)seq);
+        return nullptr;
+    }
+    return &it->second;
+}
+const pk_bm::Seq *resident(const pk_bm *bm, int64_t seq) { return resident(const_cast<pk_bm *>(bm), seq); }
+}  // namespace
 
 extern "C" {
 
@@ -105,20 +136,20 @@ int pk_bm_add_seq(pk_bm *bm, int64_t *seq_out) {
 
 int pk_bm_blocks_needed(const pk_bm *bm, int64_t seq, int n, int *needed_out) {
     if (!bm || !needed_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
-    auto it = bm->seqs.find(seq);
-    if (it == bm->seqs.end()) return fail(PK_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq);
+    const pk_bm::Seq *sq = resident(bm, seq);
+    if (!sq) return PK_ERR_INVALID_ARG;
     if (n < 0) return fail(PK_ERR_INVALID_ARG, "negative token count");
-    *needed_out = (int)bm->needed(it->second, n);
+    *needed_out = (int)bm->needed(*sq, n);
     return PK_OK;
 }
 
 int pk_bm_append_slots(pk_bm *bm, int64_t seq, int n, int64_t *slots_out, int32_t *pairs_out,
                        int pairs_cap, int *n_pairs_out) {
     if (!bm || !n_pairs_out || (n > 0 && !slots_out)) return fail(PK_ERR_INVALID_ARG, "NULL argument");
-    auto it = bm->seqs.find(seq);
-    if (it == bm->seqs.end()) return fail(PK_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq);
+    pk_bm::Seq *sq = resident(bm, seq);
+    if (!sq) return PK_ERR_INVALID_ARG;
     if (n < 0) return fail(PK_ERR_INVALID_ARG, "negative token count");
-    pk_bm::Seq &s = it->second;
+    pk_bm::Seq &s = *sq;
     *n_pairs_out = 0;
     if (n == 0) return PK_OK;
     const int64_t bs = bm->block_size;
@@ -154,9 +185,9 @@ int pk_bm_append_slots(pk_bm *bm, int64_t seq, int n, int64_t *slots_out, int32_
 
 int pk_bm_fork(pk_bm *bm, int64_t parent, int64_t *child_out) {
     if (!bm || !child_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
-    auto it = bm->seqs.find(parent);
-    if (it == bm->seqs.end()) return fail(PK_ERR_INVALID_ARG, "unknown sequence %lld", (long long)parent);
-    pk_bm::Seq child = it->second;  // copy before emplace can rehash
+    const pk_bm::Seq *ps = resident(bm, parent);
+    if (!ps) return PK_ERR_INVALID_ARG;
+    pk_bm::Seq child = *ps;  // copy before emplace can rehash
     for (int32_t b : child.table) ++bm->refcount[b];
     const int64_t id = bm->next_seq++;
     bm->seqs.emplace(id, std::move(child));
@@ -169,8 +200,88 @@ int pk_bm_free(pk_bm *bm, int64_t seq) {
     auto it = bm->seqs.find(seq);
     if (it == bm->seqs.end()) return fail(PK_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq);
     const std::vector<int32_t> &t = it->second.table;
-    for (auto b = t.rbegin(); b != t.rend(); ++b) bm->release(*b);
+    if (it->second.swapped) {  // its host blocks return to the host pool
+        for (auto h = t.rbegin(); h != t.rend(); ++h) {
+            bm->host_filled[*h] = 0;
+            bm->host_free.push_back(*h);
+        }
+    } else {
+        for (auto b = t.rbegin(); b != t.rend(); ++b) bm->release(*b);
+    }
     bm->seqs.erase(it);
+    return PK_OK;
+}
+
+int pk_bm_set_host_blocks(pk_bm *bm, int num_host_blocks) {
+    if (!bm) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    if (num_host_blocks < 0 || bm->num_host_blocks != 0)
+        return fail(PK_ERR_INVALID_ARG, "host pool already set, or negative size");
+    bm->num_host_blocks = num_host_blocks;
+    bm->host_filled.assign(num_host_blocks, 0);
+    for (int32_t h = 0; h < num_host_blocks; ++h) bm->host_free.push_back(h);
+    return PK_OK;
+}
+
+int pk_bm_swap_out(pk_bm *bm, int64_t seq, int32_t *pairs_out, int pairs_cap, int *n_pairs_out) {
+    if (!bm || !n_pairs_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    *n_pairs_out = 0;
+    pk_bm::Seq *sq = resident(bm, seq);
+    if (!sq) return PK_ERR_INVALID_ARG;
+    std::vector<int32_t> &t = sq->table;
+    if ((int64_t)t.size() > pairs_cap || (!pairs_out && !t.empty()))
+        return fail(PK_ERR_INVALID_ARG, "%zu pairs, capacity %d", t.size(), pairs_cap);
+    for (int32_t b : t)
+        if (bm->refcount[b] > 1)
+            return fail(PK_ERR_UNSUPPORTED, "sequence %lld shares block %d", (long long)seq, b);
+    if (t.size() > bm->host_free.size())
+        return fail(PK_ERR_OOM, "need %zu host blocks, %zu free", t.size(), bm->host_free.size());
+    for (size_t i = 0; i < t.size(); ++i) {
+        const int32_t h = bm->host_free.front();
+        bm->host_free.pop_front();
+        bm->host_filled[h] = bm->filled[t[i]];
+        pairs_out[2 * i] = t[i];
+        pairs_out[2 * i + 1] = h;
+    }
+    for (auto b = t.rbegin(); b != t.rend(); ++b) bm->release(*b);
+    for (size_t i = 0; i < t.size(); ++i) t[i] = pairs_out[2 * i + 1];
+    sq->swapped = true;
+    *n_pairs_out = (int)t.size();
+    return PK_OK;
+}
+
+int pk_bm_swap_in(pk_bm *bm, int64_t seq, int32_t *pairs_out, int pairs_cap, int *n_pairs_out) {
+    if (!bm || !n_pairs_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    *n_pairs_out = 0;
+    auto it = bm->seqs.find(seq);
+    if (it == bm->seqs.end()) return fail(PK_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq);
+    pk_bm::Seq &s = it->second;
+    if (!s.swapped) return fail(PK_ERR_INVALID_ARG, "sequence %lld is not swapped out", (long long)seq);
+    std::vector<int32_t> &t = s.table;
+    if ((int64_t)t.size() > pairs_cap || (!pairs_out && !t.empty()))
+        return fail(PK_ERR_INVALID_ARG, "%zu pairs, capacity %d", t.size(), pairs_cap);
+    if (t.size() > bm->free_list.size())
+        return fail(PK_ERR_OOM, "need %zu blocks, %zu free", t.size(), bm->free_list.size());
+    for (size_t i = 0; i < t.size(); ++i) {
+        const int32_t b = bm->take();
+        bm->filled[b] = bm->host_filled[t[i]];
+        pairs_out[2 * i] = t[i];
+        pairs_out[2 * i + 1] = b;
+    }
+    for (auto h = t.rbegin(); h != t.rend(); ++h) {
+        bm->host_filled[*h] = 0;
+        bm->host_free.push_back(*h);
+    }
+    for (size_t i = 0; i < t.size(); ++i) t[i] = pairs_out[2 * i + 1];
+    s.swapped = false;
+    *n_pairs_out = (int)t.size();
+    return PK_OK;
+}
+
+int pk_bm_is_swapped(const pk_bm *bm, int64_t seq, int *swapped_out) {
+    if (!bm || !swapped_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    auto it = bm->seqs.find(seq);
+    if (it == bm->seqs.end()) return fail(PK_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq);
+    *swapped_out = it->second.swapped ? 1 : 0;
     return PK_OK;
 }
 
@@ -190,10 +301,9 @@ int pk_bm_fill_tables(const pk_bm *bm, const int64_t *seqs, int n_seqs, int32_t 
     if (!bm || (n_seqs > 0 && (!seqs || !out)) || n_seqs < 0 || width < 0)
         return fail(PK_ERR_INVALID_ARG, "bad argument");
     for (int i = 0; i < n_seqs; ++i) {
-        auto it = bm->seqs.find(seqs[i]);
-        if (it == bm->seqs.end())
-            return fail(PK_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seqs[i]);
-        const std::vector<int32_t> &t = it->second.table;
+        const pk_bm::Seq *sq = resident(bm, seqs[i]);
+        if (!sq) return PK_ERR_INVALID_ARG;
+        const std::vector<int32_t> &t = sq->table;
         if ((int)t.size() > width)
             return fail(PK_ERR_INVALID_ARG, "table of %zu entries, width %d", t.size(), width);
         int32_t *row = out + (int64_t)i * width;
@@ -230,6 +340,8 @@ int pk_bm_get_stats(const pk_bm *bm, pk_bm_stats *out) {
         if (bm->refcount[b] > 0) waste += bm->block_size - bm->filled[b];
     out->tail_waste_slots = waste;
     out->num_seqs = (int64_t)bm->seqs.size();
+    out->host_blocks = bm->num_host_blocks;
+    out->host_free_blocks = (int64_t)bm->host_free.size();
     return PK_OK;
 }
 

@@ -135,6 +135,37 @@ __global__ void block_copy_scalar(T *kp, T *vp, const int32_t *__restrict__ pair
     }
 }
 
+// Whole blocks between two pools of the same block geometry (the device pool
+// and a host pool, in either direction): CTA work item w copies K (w even) or
+// V (w odd) of pair w / 2, a = source block, b = destination block.  The host
+// side is read or written over the host link through its device mapping.
+template <typename T, int UNROLL>
+__global__ void swap_copy(const T *__restrict__ sk, const T *__restrict__ sv, T *dk, T *dv,
+                          const int32_t *__restrict__ pairs, int n_pairs, int64_t block_chunks,
+                          int n_src, int n_dst, int *err) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    for (int64_t w = blockIdx.x; w < 2LL * n_pairs; w += gridDim.x) {
+        const int pr = (int)(w >> 1);
+        const int a = __ldg(pairs + 2 * pr), b = __ldg(pairs + 2 * pr + 1);
+        if (a < 0 || a >= n_src || b < 0 || b >= n_dst) {
+            if (threadIdx.x == 0) record_error(err, PK_ERR_BAD_INDEX);
+            continue;
+        }
+        const T *src = ((w & 1) ? sv : sk) + (int64_t)a * block_chunks;
+        T *dst = ((w & 1) ? dv : dk) + (int64_t)b * block_chunks;
+        int64_t i = threadIdx.x;
+        // several loads in flight per thread: the host link's latency is long
+        for (; i + (UNROLL - 1) * blockDim.x < block_chunks; i += UNROLL * blockDim.x) {
+            T r[UNROLL];
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) r[u] = src[i + u * blockDim.x];
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) dst[i + u * blockDim.x] = r[u];
+        }
+        for (; i < block_chunks; i += blockDim.x) dst[i] = src[i];
+    }
+}
+
 bool aligned16(const void *p) { return ((uintptr_t)p & 15) == 0; }
 
 int grid_for(int64_t work, int threads, int sm_count) {
@@ -173,6 +204,35 @@ int launch_kv_append(const pk_pool *p, const void *k, const void *v, const int64
     }
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? PK_OK : cuda_fail(e, "kv append launch");
+}
+
+int launch_swap_blocks(const pk_pool *p, void *host_k, void *host_v, int num_host_blocks,
+                       const int32_t *pairs, int n_pairs, bool to_host, cudaStream_t st) {
+    if (n_pairs == 0) return PK_OK;
+    const int elt = p->dtype == PK_BF16 ? 2 : 4;
+    const int64_t block_elems = (int64_t)p->n_kv_heads * p->block_size * p->head_dim;
+    const int64_t block_bytes = block_elems * elt;
+    void *sk = to_host ? p->k_base : host_k, *sv = to_host ? p->v_base : host_v;
+    void *dk = to_host ? host_k : p->k_base, *dv = to_host ? host_v : p->v_base;
+    const int n_src = to_host ? p->num_blocks : num_host_blocks;
+    const int n_dst = to_host ? num_host_blocks : p->num_blocks;
+    const int64_t ctas = 2LL * n_pairs;
+    const int grid = (int)(ctas < (int64_t)p->sm_count * 32 ? ctas : (int64_t)p->sm_count * 32);
+    if (block_bytes % 16 == 0 && aligned16(sk) && aligned16(sv) && aligned16(dk) && aligned16(dv)) {
+        swap_copy<uint4, 4><<<grid, 256, 0, st>>>((const uint4 *)sk, (const uint4 *)sv, (uint4 *)dk,
+                                                  (uint4 *)dv, pairs, n_pairs, block_bytes / 16, n_src,
+                                                  n_dst, p->d_err);
+    } else if (p->dtype == PK_BF16) {
+        swap_copy<uint16_t, 4><<<grid, 256, 0, st>>>((const uint16_t *)sk, (const uint16_t *)sv,
+                                                     (uint16_t *)dk, (uint16_t *)dv, pairs, n_pairs,
+                                                     block_elems, n_src, n_dst, p->d_err);
+    } else {
+        swap_copy<float, 4><<<grid, 256, 0, st>>>((const float *)sk, (const float *)sv, (float *)dk,
+                                                  (float *)dv, pairs, n_pairs, block_elems, n_src,
+                                                  n_dst, p->d_err);
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PK_OK : cuda_fail(e, "block swap launch");
 }
 
 int launch_block_copy(const pk_pool *p, const int32_t *pairs, int n_pairs, cudaStream_t st) {

@@ -52,6 +52,8 @@ constexpr int kTile = 16;        // tokens per KV tile and rows per query tile
 int launch_kv_append(const pk_pool *p, const void *k, const void *v, const int64_t *slots,
                      int num_tokens, cudaStream_t st);
 int launch_block_copy(const pk_pool *p, const int32_t *pairs, int n_pairs, cudaStream_t st);
+int launch_swap_blocks(const pk_pool *p, void *host_k, void *host_v, int num_host_blocks,
+                       const int32_t *pairs, int n_pairs, bool to_host, cudaStream_t st);
 
 struct AttnArgs {
     const void *q;

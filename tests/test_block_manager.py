@@ -8,17 +8,19 @@ import pytest
 
 from oracle import OracleBlockManager, OracleOOM, capacity
 from paged_kv_cache_chunked_b200.api import BlockManager
-from paged_kv_cache_chunked_b200._lib import OutOfBlocks
+from paged_kv_cache_chunked_b200._lib import OutOfBlocks, PagedKVError
 from paged_kv_cache_chunked_b200.workloads import page_toy_lengths
 
 
 def _same_state(bm, ob):
     assert bm.stats() == {"num_blocks": ob.num_blocks, "free_blocks": ob.num_free(),
                           "used_blocks": ob.num_used(), "alloc_failures": ob.alloc_failures,
-                          "tail_waste_slots": ob.tail_waste(), "num_seqs": len(ob.tables)}
+                          "tail_waste_slots": ob.tail_waste(), "num_seqs": len(ob.tables),
+                          "host_blocks": ob.host_blocks, "host_free_blocks": len(ob.host_free)}
     for sid in ob.tables:
         assert bm.block_table(sid) == ob.block_table(sid)
         assert bm.length(sid) == ob.length(sid)
+        assert bm.is_swapped(sid) == (sid in ob.swapped)
     for b in range(ob.num_blocks):
         assert bm.refcount(b) == ob.refcount[b]
 
@@ -28,25 +30,44 @@ def test_random_operations_match_the_oracle(seed):
     rng = random.Random(100 + seed)
     nb, bs = rng.choice([(24, 4), (64, 16), (40, 1), (30, 8)])
     bm, ob = BlockManager(nb, bs), OracleBlockManager(nb, bs)
+    bm.set_host_blocks(nb // 2)
+    ob.set_host_blocks(nb // 2)
     live = []
     for step in range(500):
         op = rng.random()
-        if op < 0.15 or not live:
+        resident = [s for s in live if s not in ob.swapped]
+        if op < 0.15 or not resident:
             a, b = bm.add_seq(), ob.add_seq()
             assert a == b
             live.append(a)
-        elif op < 0.3:
-            p = rng.choice(live)
+        elif op < 0.25:
+            p = rng.choice(resident)
             a, b = bm.fork(p), ob.fork(p)
             assert a == b
             live.append(a)
-        elif op < 0.45:
+        elif op < 0.4:
             s = rng.choice(live)
             live.remove(s)
             bm.free(s)
             ob.free(s)
-        else:
+        elif op < 0.5:
+            # swap out or back in; refusals must match: a shared block
+            # (PK_ERR_UNSUPPORTED), a pool short of blocks (PK_ERR_OOM)
             s = rng.choice(live)
+            ours, theirs = (bm.swap_in, ob.swap_in) if s in ob.swapped else (bm.swap_out, ob.swap_out)
+            try:
+                ref = theirs(s)
+            except OracleOOM:
+                with pytest.raises(OutOfBlocks):
+                    ours(s)
+            except ValueError:
+                with pytest.raises(PagedKVError) as e:
+                    ours(s)
+                assert e.value.code == 3
+            else:
+                assert ours(s) == ref
+        else:
+            s = rng.choice(resident)
             n = rng.randint(0, 3 * bs)
             assert bm.blocks_needed(s, n) == ob.blocks_needed(s, n)
             try:

@@ -120,9 +120,13 @@ def test_oom_changes_nothing():
 
 
 def _check_invariants(bm):
-    referenced = {}
+    referenced, host_referenced = {}, set()
     for sid, table in bm.tables.items():
         assert len(table) == -(-bm.lengths[sid] // bm.block_size)
+        if sid in bm.swapped:           # a swapped table names host blocks, each once
+            assert host_referenced.isdisjoint(table) and len(set(table)) == len(table)
+            host_referenced.update(table)
+            continue
         for b in table:
             referenced[b] = referenced.get(b, 0) + 1
     # a block is in the pool or referenced, never both, never neither
@@ -130,27 +134,45 @@ def _check_invariants(bm):
     assert set(bm.free_list).isdisjoint(referenced)
     for b in range(bm.num_blocks):
         assert bm.refcount[b] == referenced.get(b, 0)
-    # at most one partly filled block per sequence
-    assert bm.tail_waste() <= (bm.block_size - 1) * len(bm.tables)
+    # the same for the host pool
+    assert len(bm.host_free) + len(host_referenced) == bm.host_blocks
+    assert set(bm.host_free).isdisjoint(host_referenced)
+    # at most one partly filled block per sequence on the device
+    assert bm.tail_waste() <= (bm.block_size - 1) * (len(bm.tables) - len(bm.swapped))
 
 
 @pytest.mark.parametrize("seed", range(5))
 def test_random_operation_sequences_keep_invariants(seed):
     rng = random.Random(seed)
     bm = OracleBlockManager(40, rng.choice([1, 4, 16]))
+    bm.set_host_blocks(30)
     live = []
     for _ in range(400):
         op = rng.random()
-        if op < 0.2 or not live:
+        resident = [s for s in live if s not in bm.swapped]
+        if op < 0.2 or not resident:
             live.append(bm.add_seq())
-        elif op < 0.35:
-            live.append(bm.fork(rng.choice(live)))
-        elif op < 0.5:
+        elif op < 0.3:
+            live.append(bm.fork(rng.choice(resident)))
+        elif op < 0.45:
             s = rng.choice(live)
             live.remove(s)
             bm.free(s)
-        else:
+        elif op < 0.55:
             s = rng.choice(live)
+            try:
+                if s in bm.swapped:
+                    table = bm.block_table(s)
+                    pairs = bm.swap_in(s)
+                    assert [h for h, _ in pairs] == table and bm.block_table(s) == [d for _, d in pairs]
+                else:
+                    table = bm.block_table(s)
+                    pairs = bm.swap_out(s)
+                    assert [d for d, _ in pairs] == table and bm.block_table(s) == [h for _, h in pairs]
+            except (OracleOOM, ValueError):
+                pass
+        else:
+            s = rng.choice(resident)
             shared_tail = (bm.length(s) % bm.block_size != 0
                            and bm.refcount[bm.block_table(s)[-1]] > 1)
             try:
@@ -163,3 +185,87 @@ def test_random_operation_sequences_keep_invariants(seed):
     for s in live:
         bm.free(s)
     assert bm.num_free() == bm.num_blocks
+
+
+def test_swap_round_trip_restores_every_sequence_kv():
+    # "a preempted request's blocks are either swapped out to CPU memory or
+    # freed and recomputed" [Batching and PagedAttention, "When blocks run
+    # out"]: after swap-out, reuse of the freed device blocks by another
+    # sequence, and swap-in, both sequences read back exactly what they wrote
+    import torch
+    import oracle
+    bs, H, d = 4, 2, 3
+    bm = OracleBlockManager(6, bs)
+    bm.set_host_blocks(4)
+    kp, vp = torch.zeros(6, H, bs, d), torch.zeros(6, H, bs, d)
+    hk, hv = torch.full((4, H, bs, d), float("nan")), torch.full((4, H, bs, d), float("nan"))
+    written = {}
+
+    def write(seq, n, base):
+        slots, pairs = bm.append_slots(seq, n)
+        assert pairs == []
+        k = base + torch.arange(n * H * d, dtype=torch.float32).reshape(n, H, d)
+        oracle.kv_append(kp, vp, k, -k, torch.tensor(slots))
+        written.setdefault(seq, []).append(k)
+
+    def logical(seq):
+        t = torch.tensor(bm.block_table(seq))
+        n = bm.length(seq)
+        return (kp[t].transpose(1, 2).reshape(-1, H, d)[:n], vp[t].transpose(1, 2).reshape(-1, H, d)[:n])
+
+    a, b = bm.add_seq(), bm.add_seq()
+    write(a, 10, 0.0)                         # blocks 0, 1, 2
+    write(b, 5, 1000.0)                       # blocks 3, 4
+    before_a = logical(a)
+    oracle.swap_blocks(kp, vp, hk, hv, bm.swap_out(a), to_host=True)
+    assert bm.num_free() == 4 and bm.stats()["host_free_blocks"] == 1
+    c = bm.add_seq()
+    write(c, 8, 5000.0)                       # takes block 5 and a's old block 2, overwriting it
+    assert 2 in bm.block_table(c)
+    bm.free(c)
+    oracle.swap_blocks(kp, vp, hk, hv, bm.swap_in(a), to_host=False)
+    assert bm.block_table(a) != [0, 1, 2]      # a lands on other physical blocks
+    for got, want in zip(logical(a), before_a):
+        assert torch.equal(got, want)
+    kb = torch.cat(written[b])
+    assert torch.equal(logical(b)[0], kb) and torch.equal(logical(b)[1], -kb)
+    assert bm.stats()["host_free_blocks"] == 4
+    _check_invariants(bm)
+
+
+def test_swap_refusals_change_nothing():
+    bm = OracleBlockManager(8, 4)
+    bm.set_host_blocks(2)
+    s = bm.add_seq()
+    bm.append_slots(s, 9)                      # 3 blocks
+    c = bm.fork(s)
+    state = lambda: (list(bm.free_list), list(bm.refcount), list(bm.host_free), bm.block_table(s),
+                     set(bm.swapped))
+    before = state()
+    with pytest.raises(ValueError):            # shares blocks with its fork
+        bm.swap_out(s)
+    assert state() == before
+    bm.free(c)
+    before = state()
+    with pytest.raises(OracleOOM):             # 3 blocks, 2 host blocks
+        bm.swap_out(s)
+    assert state() == before
+    with pytest.raises(ValueError):            # not swapped
+        bm.swap_in(s)
+    t = bm.add_seq()
+    bm.append_slots(t, 4)
+    big = OracleBlockManager(3, 4)
+    big.set_host_blocks(3)
+    u = big.add_seq()
+    big.append_slots(u, 12)                    # 3 blocks, pool full
+    big.swap_out(u)
+    v = big.add_seq()
+    big.append_slots(v, 1)                     # the device pool now has 2 free blocks
+    before = (list(big.free_list), list(big.host_free), big.block_table(u))
+    with pytest.raises(OracleOOM):
+        big.swap_in(u)
+    assert (list(big.free_list), list(big.host_free), big.block_table(u)) == before
+    with pytest.raises(ValueError):            # a swapped sequence takes no appends
+        big.append_slots(u, 1)
+    big.free(u)                                # returns its host blocks
+    assert big.stats()["host_free_blocks"] == 3
