@@ -50,7 +50,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="decode64_bf16",
-                   choices=["decode64_bf16", "longdoc_bf16", "chunk512_bf16", "trace", "fork",
+                   choices=["decode64_bf16", "longdoc_bf16", "chunk512_bf16", "trace", "trace_swap", "fork",
                             "fork1028", "append_copy"])
     p.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
     p.add_argument("--no-e2e", action="store_true")
@@ -656,19 +656,27 @@ def run_serving(args, rank, world, device):
     peak, peak_kind = measured_peak()
     kv_tok = 8 * 128 * 2 * 2          # K+V bytes per token per layer (8 kv heads, d 128, bf16)
     recs = []
-    if args.workload == "trace":
-        r = TraceRunner(device)
+    if args.workload in ("trace", "trace_swap"):
+        # trace_swap: preempted requests' blocks go to a pinned host pool of
+        # 8,192 blocks and back instead of being recomputed
+        swap = args.workload == "trace_swap"
+        r = TraceRunner(device, preempt="swap" if swap else "recompute", num_host_blocks=8192 if swap else 0)
         while r.sched.step_no < 300 and (r.pending or r.sched.has_work()):
             rec = r.step()
             if rec is not None:
                 recs.append(rec)
         skip = min(args.warmup, len(recs) // 2)
         recs = recs[skip:]
-        cfg = {"workload": "trace", "steps_run": len(recs) + skip, "warmup_steps": skip,
+        cfg = {"workload": args.workload, "steps_run": len(recs) + skip, "warmup_steps": skip,
                "num_blocks": 8192, "block_size": 16, "n_q_heads": 32, "n_kv_heads": 8,
                "head_dim": 128, "token_budget": 4096, "max_chunk": 512,
+               "preempt": r.sched.preempt_mode,
                "preemptions": r.sched.metrics["preemptions"], "rejected": r.rejected,
                "finished": len(r.sched.finished)}
+        if swap:
+            cfg.update(host_blocks=8192, swaps_out=r.sched.metrics["swaps_out"],
+                       swaps_in=r.sched.metrics["swaps_in"],
+                       swapped_blocks_timed=sum(x.swap_blocks for x in recs))
         ms = [x.gpu_ms for x in recs]
         toks = [x.tokens for x in recs]
         kvb = [x.context_tokens * kv_tok for x in recs]
@@ -702,7 +710,7 @@ def run_serving(args, rank, world, device):
             "tokens_per_step_s": {"p10": pct(0.1), "p50": pct(0.5), "p90": pct(0.9)},
             "kv_gbs": sum(kvb) / (tot_ms * 1e-3) / 1e9,
             "pct_hbm": 100 * sum(kvb) / (tot_ms * 1e-3) / 1e9 / peak,
-            "timing": "per-step CUDA events around copy + append + attention; host scheduling excluded"}
+            "timing": "per-step CUDA events around swaps + copy + append + attention; host scheduling excluded"}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -723,7 +731,7 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                  device_id=device)
     try:
-        if args.workload in ("trace", "fork", "fork1028"):
+        if args.workload in ("trace", "trace_swap", "fork", "fork1028"):
             run_serving(args, rank, world, device)
         elif args.workload == "append_copy":
             run_kvops(args, rank, world, device)

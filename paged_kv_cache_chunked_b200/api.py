@@ -17,7 +17,7 @@ import weakref
 
 import torch
 
-from ._lib import PK_BF16, PK_F32, BmStats, check, lib
+from ._lib import PK_BF16, PK_F32, BmStats, OutOfBlocks, PagedKVError, check, lib  # noqa: F401
 
 _DTYPES = {torch.float32: PK_F32, torch.bfloat16: PK_BF16}
 _pools = weakref.WeakValueDictionary()  # k_pool data_ptr -> KVPool

@@ -2,10 +2,13 @@
 
 TraceRunner   continuous batching over an arrival trace: each iteration the
               scheduler plans a mixed batch (decodes first, then prefill
-              chunks), the kernels run copy -> append -> attention on one
-              stream, finished requests are freed ["PagedAttention &
+              chunks), the kernels run swaps -> copy -> append -> attention on
+              one stream, finished requests are freed ["PagedAttention &
               Continuous Batching" (study notes), "Continuous batching" and
               "Flow"; "Batching and PagedAttention", "Continuous batching"].
+              Preempted requests are recomputed, or with preempt="swap" their
+              blocks go to a pinned host pool and back ["Batching and
+              PagedAttention", "When blocks run out"].
 ForkRunner    n parallel samples of each prompt: prefill, fork (children share
               the prompt's blocks by reference count), then decode steps in
               which the first write into a shared, partly filled tail block
@@ -25,7 +28,7 @@ from .workloads import token_values, trace_requests
 
 class StepRecord:
     __slots__ = ("step", "tokens", "decode_rows", "prefill_tokens", "copies", "gpu_ms",
-                 "context_tokens", "num_seqs")
+                 "context_tokens", "num_seqs", "swap_blocks")
 
     def __init__(self, **kw):
         for k, v in kw.items():
@@ -37,7 +40,7 @@ class TraceRunner:
 
     def __init__(self, device, num_blocks=8192, block_size=16, n_q_heads=32, n_kv_heads=8,
                  head_dim=128, token_budget=4096, max_chunk=512, trace=None, seed=1004,
-                 n_steps=300, dtype=torch.bfloat16):
+                 n_steps=300, dtype=torch.bfloat16, preempt="recompute", num_host_blocks=0):
         self.device = torch.device(device)
         self.Hq, self.Hkv, self.d, self.bs = n_q_heads, n_kv_heads, head_dim, block_size
         self.dtype = dtype
@@ -46,7 +49,11 @@ class TraceRunner:
         self.pool = api.kv_pool_create(num_blocks, block_size, n_kv_heads, head_dim, dtype,
                                        self.device)
         self.bm = api.BlockManager(num_blocks, block_size)
-        self.sched = Scheduler(self.bm, token_budget, max_chunk)
+        self.host = None
+        if preempt == "swap":
+            self.bm.set_host_blocks(num_host_blocks)
+            self.host = api.host_pool_create(num_host_blocks, self.pool)
+        self.sched = Scheduler(self.bm, token_budget, max_chunk, preempt=preempt)
         trace = trace if trace is not None else trace_requests(n_steps=n_steps, seed=seed)
         self.pending = [Request(i, a, p, o) for i, (a, p, o) in enumerate(trace)]
         self.scale = head_dim ** -0.5
@@ -68,10 +75,28 @@ class TraceRunner:
         step = self.sched.step_no
         self._admit_arrivals(step)
         plan = self.sched.schedule()
-        if not plan.requests:
-            self.sched.complete(plan)
-            return None
         dev = self.device
+        swaps = [(to_host, torch.tensor(pairs, dtype=torch.int32).reshape(-1, 2).to(dev))
+                 for to_host, pairs in plan.swap_ops]
+        if not plan.requests:
+            # nothing to run but, possibly, swaps decided while planning (timed:
+            # they are part of the serving work)
+            rec = None
+            if swaps:
+                stream = torch.cuda.current_stream(dev)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                self._run_swaps(swaps)
+                e1.record(stream)
+                if on_step is not None:
+                    on_step(plan, {"swaps": plan.swap_ops}, None)
+                e1.synchronize()
+                rec = StepRecord(step=step, tokens=0, decode_rows=0, prefill_tokens=0, copies=0,
+                                 gpu_ms=e0.elapsed_time(e1), context_tokens=0, num_seqs=0,
+                                 swap_blocks=sum(len(p) for _, p in plan.swap_ops))
+                self.records.append(rec)
+            self.sched.complete(plan)
+            return rec
         rids, pos = [], []
         for req, s, n in zip(plan.requests, plan.starts, plan.counts):
             rids.extend([req.rid] * n)
@@ -91,6 +116,7 @@ class TraceRunner:
         if timed:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
+        self._run_swaps(swaps)
         if d["pairs"].shape[0]:
             api.block_copy(d["pairs"], pool=self.pool)
         api.paged_kv_append(k, v, d["slots"], pool=self.pool)
@@ -99,17 +125,25 @@ class TraceRunner:
         if timed:
             e1.record(stream)
         if on_step is not None:
-            on_step(plan, {"q": q, "k": k, "v": v, **meta}, out)
+            on_step(plan, {"q": q, "k": k, "v": v, "swaps": plan.swap_ops, **meta}, out)
         if timed:
             e1.synchronize()
         n_dec = sum(1 for r, s in zip(plan.requests, plan.starts) if s >= r.target)
         rec = StepRecord(step=step, tokens=plan.num_tokens, decode_rows=n_dec,
                          prefill_tokens=plan.num_tokens - n_dec, copies=len(plan.copy_pairs),
                          gpu_ms=e0.elapsed_time(e1) if timed else None,
-                         context_tokens=sum(plan.context_lens), num_seqs=len(plan.requests))
+                         context_tokens=sum(plan.context_lens), num_seqs=len(plan.requests),
+                         swap_blocks=sum(len(p) for _, p in plan.swap_ops))
         self.sched.complete(plan)
         self.records.append(rec)
         return rec
+
+    def _run_swaps(self, swaps):
+        # in the order the scheduler decided them: a swap-in may reuse blocks a
+        # swap-out of the same step freed, and the reverse on the host
+        for to_host, pairs in swaps:
+            if pairs.shape[0]:
+                api.swap_blocks(pairs, to_host=to_host, host_pool=self.host, pool=self.pool)
 
     def run(self, max_steps=None, on_step=None):
         limit = max_steps if max_steps is not None else self.n_steps

@@ -29,6 +29,19 @@ Readings where the pages give no number or order (listed in the design notes):
   * a request's K/V and queries are a deterministic function of (request id,
     position), so recomputation reproduces the same bits.
 
+Swap mode (preempt="swap") takes the pages' other option for a victim: its
+blocks move to CPU memory, all together, and come back before it runs again
+["Batching and PagedAttention", "When blocks run out"].  Readings:
+  * the victim keeps its state (tokens stored, generated); a victim that
+    shares a block, or that the host pool cannot hold, is recomputed instead;
+  * swapped requests come back first, in arrival order, as soon as their
+    blocks and one more fit (just their blocks when nothing runs), never in
+    the step that swapped them out; while any request is swapped out no new
+    request is admitted;
+  * the swaps of a step run, in the order they were decided, before its
+    copy-on-write copies, appends and attention (a swap-in may land in blocks
+    a swap-out of the same step just freed).
+
 A request with prompt length P and output length O stores P + O - 1 tokens:
 the last prefill chunk yields the first output token, each decode step
 appends the previous output token and yields the next.
@@ -53,6 +66,7 @@ class Request:
     admit_step: int = -1
     finish_step: int = -1
     preemptions: int = 0
+    swapped_step: int = -1
     token_steps: list = field(default_factory=list)
 
     def __post_init__(self):
@@ -76,6 +90,7 @@ class StepPlan:
     context_lens: list      # tokens stored per request after this step's append
     tables: torch.Tensor    # int32 [B, W] block tables (host)
     preempted: list         # requests preempted while planning this step
+    swap_ops: list = field(default_factory=list)  # (to_host, [(src, dst), ...]) in order
 
     @property
     def num_tokens(self):
@@ -89,16 +104,22 @@ class StepPlan:
 
 
 class Scheduler:
-    def __init__(self, bm, token_budget=4096, max_chunk=512):
+    def __init__(self, bm, token_budget=4096, max_chunk=512, preempt="recompute"):
+        if preempt not in ("recompute", "swap"):
+            raise ValueError("preempt must be 'recompute' or 'swap'")
         self.bm = bm
         self.block_size = bm.block_size
         self.token_budget = token_budget
         self.max_chunk = max_chunk
+        self.preempt_mode = preempt
         self.waiting = []    # arrival order
         self.running = []    # arrival order; hold blocks
+        self.swapped = []    # arrival order; blocks in the host pool
         self.finished = []
         self.step_no = 0
-        self.metrics = {"preemptions": 0, "alloc_failures": 0, "admitted": 0}
+        self._swap_ops = []  # swaps decided since the last plan was handed out
+        self.metrics = {"preemptions": 0, "alloc_failures": 0, "admitted": 0, "swaps_out": 0,
+                        "swaps_in": 0}
 
     def add_request(self, req):
         """Queue a request; one that could never fit in the whole pool is
@@ -114,10 +135,25 @@ class Scheduler:
         self.waiting.sort(key=lambda r: (r.arrival, r.rid))
 
     def has_work(self):
-        return bool(self.waiting or self.running)
+        return bool(self.waiting or self.running or self.swapped)
 
     # -- preemption -------------------------------------------------------
+    def _can_swap_out(self, req):
+        table = self.bm.block_table(req.seq)
+        return (self.bm.stats()["host_free_blocks"] >= len(table)
+                and all(self.bm.refcount(b) == 1 for b in table))
+
     def _preempt(self, req):
+        if self.preempt_mode == "swap" and self._can_swap_out(req):
+            self._swap_ops.append((True, self.bm.swap_out(req.seq)))
+            req.preemptions += 1
+            req.swapped_step = self.step_no
+            self.metrics["preemptions"] += 1
+            self.metrics["swaps_out"] += 1
+            self.running.remove(req)
+            self.swapped.append(req)
+            self.swapped.sort(key=lambda r: (r.arrival, r.rid))
+            return
         self.bm.free(req.seq)
         req.seq = -1
         req.stored = 0
@@ -142,9 +178,26 @@ class Scheduler:
             self._preempt(victim)
             plan = self._plan()
             plan.preempted.append(victim)
+        plan.swap_ops, self._swap_ops = self._swap_ops, []
         return plan
 
+    def _swap_in_ready(self):
+        """Bring swapped requests back, in arrival order, while they fit."""
+        for req in list(self.swapped):
+            if req.swapped_step == self.step_no:
+                break
+            need = len(self.bm.block_table(req.seq)) + (1 if self.running else 0)
+            if need > self.bm.num_free():
+                break        # arrival order: later ones wait behind this one
+            self._swap_ops.append((False, self.bm.swap_in(req.seq)))
+            self.swapped.remove(req)
+            self.running.append(req)
+            self.running.sort(key=lambda r: (r.arrival, r.rid))
+            self.metrics["swaps_in"] += 1
+
     def _plan(self):
+        if self.swapped:
+            self._swap_in_ready()
         budget = self.token_budget
         batch, starts, counts, slots, pairs, preempted = [], [], [], [], [], []
 
@@ -172,7 +225,8 @@ class Scheduler:
         # prefill chunks: running requests mid-prefill, then waiting ones (FCFS)
         candidates = [r for r in sorted(self.running, key=lambda r: (r.arrival, r.rid))
                       if r.prefilling and r not in batch]
-        candidates += [r for r in self.waiting if r not in preempted]
+        if not self.swapped:     # nothing new is admitted while a request is swapped out
+            candidates += [r for r in self.waiting if r not in preempted]
         for req in candidates:
             if budget == 0:
                 break
@@ -225,7 +279,8 @@ class Scheduler:
         s = self.bm.stats()
         return {"free_blocks": s["free_blocks"], "used_blocks": s["used_blocks"],
                 "tail_waste_slots": s["tail_waste_slots"], "running": len(self.running),
-                "waiting": len(self.waiting), "preemptions": self.metrics["preemptions"],
+                "waiting": len(self.waiting), "swapped": len(self.swapped),
+                "preemptions": self.metrics["preemptions"],
                 "alloc_failures": self.metrics["alloc_failures"]}
 
 

@@ -26,11 +26,19 @@ pytestmark = pytest.mark.gpu
 
 
 class Mirror:
-    """CPU copy of the pool kept current with the oracle's append and copy."""
+    """CPU copy of the pool (and of the host pool, when swapping) kept current
+    with the oracle's swaps, append and copy."""
 
-    def __init__(self, pool):
+    def __init__(self, pool, host=None):
         self.k = pool.k_pool.cpu()
         self.v = pool.v_pool.cpu()
+        if host is not None:
+            self.hk, self.hv = host.k.clone(), host.v.clone()
+
+    def swaps(self, ops):
+        for to_host, pairs in ops:     # in the order the scheduler decided them
+            if pairs:
+                oracle.swap_blocks(self.k, self.v, self.hk, self.hv, pairs, to_host)
 
     def apply(self, pairs, k, v, slots):
         if pairs.shape[0]:
@@ -136,4 +144,42 @@ def test_fork_copy_on_write(cuda_dev, prompt_len, bs, copies_per_prompt):
     assert runner.unique_blocks() < runner.clone_blocks()
     torch.cuda.synchronize()
     assert torch.equal(runner.pool.k_pool.cpu(), mirror.k)
+    assert runner.pool.check_device_errors() == 0
+
+
+def test_trace_in_swap_mode_matches_the_oracle(cuda_dev):
+    # preempted requests' blocks go to a pinned host pool and come back
+    # ["Batching and PagedAttention", "When blocks run out"]; attention after a
+    # swap-in sees exactly the K/V written before the swap-out
+    trace = trace_requests(n_steps=30, arrivals_per_step=3.0, prompt_median=256, prompt_max=1500,
+                           out_min=20, out_max=120, seed=17)
+    runner = TraceRunner(cuda_dev, num_blocks=250, n_steps=30, trace=trace, token_budget=1024,
+                         max_chunk=256, preempt="swap", num_host_blocks=300)
+    mirror = Mirror(runner.pool, runner.host)
+    gen = torch.Generator().manual_seed(1)
+
+    def on_step(plan, t, out):
+        mirror.swaps(t["swaps"])
+        if out is None:
+            return
+        mirror.apply(t["pairs"], t["k"], t["v"], t["slots"])
+        rows = []
+        qsl = t["qsl"].tolist()
+        for i, (req, s) in enumerate(zip(plan.requests, plan.starts)):
+            toks = list(range(qsl[i], qsl[i + 1]))
+            if s >= req.target or req.preemptions:    # decode rows and resumed requests: all heads
+                rows += [(tk, h) for tk in {toks[0], toks[-1]} for h in range(runner.Hq)]
+            else:
+                pick = {toks[0], toks[-1], toks[int(torch.randint(len(toks), (1,), generator=gen))]}
+                rows += [(tk, int(torch.randint(runner.Hq, (1,), generator=gen))) for tk in pick]
+        _check_rows(mirror, t, out, rows, runner.scale, f"swap trace step {plan.step}")
+        if plan.step % 10 == 0 or t["swaps"]:
+            torch.cuda.synchronize()
+            assert torch.equal(runner.pool.k_pool.cpu(), mirror.k)
+            assert torch.equal(runner.pool.v_pool.cpu(), mirror.v)
+            assert torch.equal(runner.host.k, mirror.hk) and torch.equal(runner.host.v, mirror.hv)
+
+    runner.run(max_steps=60, on_step=on_step)
+    m = runner.sched.metrics
+    assert m["swaps_out"] > 0 and m["swaps_in"] > 0
     assert runner.pool.check_device_errors() == 0

@@ -110,3 +110,53 @@ def test_block_copy_many_pairs(cuda_dev):
     src, dst = pairs[:, 0].long(), pairs[:, 1].long()
     assert torch.equal(pool.k_pool[dst], k0[src]) and torch.equal(pool.v_pool[dst], v0[src])
     assert torch.equal(pool.k_pool[src], k0[src])
+
+
+@pytest.mark.parametrize("geom", GEOMS)
+def test_swap_blocks_round_trip_bit_exact(cuda_dev, geom):
+    # swap-out to a pinned host pool and swap-in to other device blocks
+    # ["Batching and PagedAttention", "When blocks run out"], against the
+    # oracle's whole-block moves; untouched blocks on both sides stay as they were
+    N, bs, Hkv, d, dtype = geom
+    pool = api.kv_pool_create(N, bs, Hkv, d, dtype, cuda_dev)
+    kc, vc = _random_pool(pool, 11)
+    H = N // 2 + 1
+    host = api.host_pool_create(H, pool)
+    g = torch.Generator().manual_seed(12)
+    host.k.copy_(torch.randn(host.k.shape, generator=g).to(dtype))
+    host.v.copy_(torch.randn(host.v.shape, generator=g).to(dtype))
+    hk, hv = host.k.clone(), host.v.clone()
+    n = min(N // 3, H)
+    out_pairs = torch.stack([torch.randperm(N, generator=g)[:n], torch.randperm(H, generator=g)[:n]], 1)
+    out_pairs = out_pairs.to(torch.int32)
+    api.swap_blocks(out_pairs.to(cuda_dev), to_host=True, host_pool=host, pool=pool)
+    oracle.swap_blocks(kc, vc, hk, hv, out_pairs, to_host=True)
+    torch.cuda.synchronize()
+    assert torch.equal(host.k, hk) and torch.equal(host.v, hv)
+    in_pairs = torch.stack([out_pairs[:, 1], torch.randperm(N, generator=g)[:n].to(torch.int32)], 1)
+    api.swap_blocks(in_pairs.to(cuda_dev), to_host=False, host_pool=host, pool=pool)
+    oracle.swap_blocks(kc, vc, hk, hv, in_pairs, to_host=False)
+    torch.cuda.synchronize()
+    assert torch.equal(pool.k_pool.cpu(), kc) and torch.equal(pool.v_pool.cpu(), vc)
+    assert pool.check_device_errors() == 0
+
+
+def test_swap_blocks_checks_ids_and_host_memory(cuda_dev):
+    pool = api.kv_pool_create(16, 16, 2, 64, torch.bfloat16, cuda_dev)
+    _random_pool(pool, 13)
+    host = api.host_pool_create(4, pool)
+    before = host.k.clone()
+    # a host id outside the host pool is recorded and skipped, nothing written
+    api.swap_blocks(torch.tensor([[3, 4], [2, -1]], dtype=torch.int32, device=cuda_dev), to_host=True,
+                    host_pool=host, pool=pool)
+    torch.cuda.synchronize()
+    assert pool.check_device_errors() == 5            # PK_ERR_BAD_INDEX
+    assert torch.equal(host.k, before)
+    # pageable host memory has no device mapping: refused before any launch
+    pageable = api.HostPool.__new__(api.HostPool)
+    pageable.k, pageable.v, pageable.num_blocks = torch.zeros_like(host.k), torch.zeros_like(host.v), 4
+    assert not pageable.k.is_pinned()
+    with pytest.raises(api.PagedKVError) as e:
+        api.swap_blocks(torch.tensor([[0, 0]], dtype=torch.int32, device=cuda_dev), to_host=True,
+                        host_pool=pageable, pool=pool)
+    assert "mapped" in str(e.value)

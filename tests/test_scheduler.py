@@ -37,9 +37,12 @@ class OracleAdapter:
     def stats(self):
         return self.o.stats()
 
+    def refcount(self, block):
+        return self.o.refcount[block]
 
-def _run(bm, trace, n_steps, budget=4096, chunk=512):
-    sched = Scheduler(bm, token_budget=budget, max_chunk=chunk)
+
+def _run(bm, trace, n_steps, budget=4096, chunk=512, preempt="recompute"):
+    sched = Scheduler(bm, token_budget=budget, max_chunk=chunk, preempt=preempt)
     pending = [Request(i, a, p, o) for i, (a, p, o) in enumerate(trace)]
     plans = []
     step = 0
@@ -132,3 +135,73 @@ def test_request_larger_than_pool_is_rejected_early():
         assert "more than the pool" in str(e)
     else:
         raise AssertionError("not rejected")
+
+
+# ---------------------------------------------------------------- swap mode
+def _swap_run(bm, host_blocks=400):
+    bm.set_host_blocks(host_blocks)
+    return _run(bm, _small_trace(), 40, preempt="swap")
+
+
+def test_swap_mode_product_and_oracle_managers_plan_identically():
+    s1, p1 = _swap_run(BlockManager(600, 16))
+    s2, p2 = _swap_run(OracleAdapter(600, 16))
+    assert len(p1) == len(p2)
+    for a, b in zip(p1, p2):
+        assert [r.rid for r in a.requests] == [r.rid for r in b.requests]
+        assert a.counts == b.counts and a.starts == b.starts
+        assert a.slots == b.slots and a.copy_pairs == b.copy_pairs
+        assert a.swap_ops == b.swap_ops
+        assert torch.equal(a.tables, b.tables)
+    assert s1.metrics == s2.metrics
+    assert s1.metrics["swaps_out"] > 0 and s1.metrics["swaps_in"] == s1.metrics["swaps_out"]
+
+
+def test_swap_mode_resumes_without_recomputation_and_drains():
+    # a swapped request keeps its tokens: every request stores exactly
+    # prompt + output - 1 positions, each written once, with no recompute
+    # prefill; every device and host block is back at the end
+    trace = _small_trace()
+    bm = BlockManager(600, 16)
+    sched, plans = _swap_run(bm)
+    assert len(sched.finished) == len(trace)
+    written = {}
+    for plan in plans:
+        for req, s, n in zip(plan.requests, plan.starts, plan.counts):
+            for pos in range(s, s + n):
+                assert (req.rid, pos) not in written, "a position written twice"
+                written[(req.rid, pos)] = plan.step
+    for r in sched.finished:
+        assert r.generated == r.output_len and r.stored == r.prompt_len + r.output_len - 1
+        assert sum(1 for (rid, _) in written if rid == r.rid) == r.stored
+    assert sched.metrics["preemptions"] == sched.metrics["swaps_out"] > 0
+    st = bm.stats()
+    assert st["free_blocks"] == 600 and st["host_free_blocks"] == 400 and st["num_seqs"] == 0
+
+
+def test_swap_ins_bring_back_exactly_what_was_swapped_out():
+    # all blocks of a sequence move together: every swap-in returns the very
+    # host blocks one earlier swap-out filled, and each op names distinct blocks
+    bm = BlockManager(600, 16)
+    sched, plans = _swap_run(bm)
+    on_host = []
+    for plan in plans:
+        for to_host, pairs in plan.swap_ops:
+            src = [a for a, _ in pairs]
+            dst = [b for _, b in pairs]
+            assert len(set(src)) == len(src) and len(set(dst)) == len(dst)
+            if to_host:
+                on_host.append(frozenset(dst))
+            else:
+                assert frozenset(src) in on_host
+                on_host.remove(frozenset(src))
+    assert on_host == []
+
+
+def test_small_host_pool_falls_back_to_recompute():
+    # victims the host pool cannot hold are recomputed, as in recompute mode
+    bm = BlockManager(600, 16)
+    bm.set_host_blocks(8)
+    sched, _ = _run(bm, _small_trace(), 40, preempt="swap")
+    assert len(sched.finished) == len(_small_trace())
+    assert sched.metrics["preemptions"] > sched.metrics["swaps_out"]
