@@ -679,6 +679,7 @@ def run_serving(args, rank, world, device):
                        swapped_blocks_timed=sum(x.swap_blocks for x in recs))
         ms = [x.gpu_ms for x in recs]
         toks = [x.tokens for x in recs]
+        useful = sum(x.new_tokens for x in recs)
         kvb = [x.context_tokens * kv_tok for x in recs]
         copies = sum(x.copies for x in recs)
     else:
@@ -700,6 +701,7 @@ def run_serving(args, rank, world, device):
                "block_size": 16, "n_q_heads": 32, "n_kv_heads": 8, "head_dim": 128,
                "decode_steps_timed": steps, "unique_blocks": r.unique_blocks(),
                "clone_blocks": r.clone_blocks(), "copies": copies}
+        useful = sum(toks)
     tot_ms = sum(ms)
     per_step = sorted(t / (m * 1e-3) for t, m in zip(toks, ms))
     pct = lambda q: per_step[min(len(per_step) - 1, int(q * len(per_step)))]
@@ -708,6 +710,8 @@ def run_serving(args, rank, world, device):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": cfg,
             "tokens_per_step_s": {"p10": pct(0.1), "p50": pct(0.5), "p90": pct(0.9)},
+            # positions stored for the first time: recomputed prefill tokens excluded
+            "useful_tokens_per_s": useful / (tot_ms * 1e-3),
             "kv_gbs": sum(kvb) / (tot_ms * 1e-3) / 1e9,
             "pct_hbm": 100 * sum(kvb) / (tot_ms * 1e-3) / 1e9 / peak,
             "timing": "per-step CUDA events around swaps + copy + append + attention; host scheduling excluded"}

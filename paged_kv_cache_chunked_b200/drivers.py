@@ -28,7 +28,7 @@ from .workloads import token_values, trace_requests
 
 class StepRecord:
     __slots__ = ("step", "tokens", "decode_rows", "prefill_tokens", "copies", "gpu_ms",
-                 "context_tokens", "num_seqs", "swap_blocks")
+                 "context_tokens", "num_seqs", "swap_blocks", "new_tokens")
 
     def __init__(self, **kw):
         for k, v in kw.items():
@@ -59,6 +59,7 @@ class TraceRunner:
         self.scale = head_dim ** -0.5
         self.records = []
         self.rejected = 0
+        self.high_water = {}     # request id -> positions stored at least once
 
     def _admit_arrivals(self, step):
         while self.pending and self.pending[0].arrival <= step:
@@ -93,7 +94,7 @@ class TraceRunner:
                 e1.synchronize()
                 rec = StepRecord(step=step, tokens=0, decode_rows=0, prefill_tokens=0, copies=0,
                                  gpu_ms=e0.elapsed_time(e1), context_tokens=0, num_seqs=0,
-                                 swap_blocks=sum(len(p) for _, p in plan.swap_ops))
+                                 swap_blocks=sum(len(p) for _, p in plan.swap_ops), new_tokens=0)
                 self.records.append(rec)
             self.sched.complete(plan)
             return rec
@@ -129,11 +130,18 @@ class TraceRunner:
         if timed:
             e1.synchronize()
         n_dec = sum(1 for r, s in zip(plan.requests, plan.starts) if s >= r.target)
+        # positions written for the first time (a recompute prefill rewrites
+        # positions a preempted request had already stored)
+        new = 0
+        for req, s, n in zip(plan.requests, plan.starts, plan.counts):
+            hw = self.high_water.get(req.rid, 0)
+            new += max(0, s + n - max(s, hw))
+            self.high_water[req.rid] = max(hw, s + n)
         rec = StepRecord(step=step, tokens=plan.num_tokens, decode_rows=n_dec,
                          prefill_tokens=plan.num_tokens - n_dec, copies=len(plan.copy_pairs),
                          gpu_ms=e0.elapsed_time(e1) if timed else None,
                          context_tokens=sum(plan.context_lens), num_seqs=len(plan.requests),
-                         swap_blocks=sum(len(p) for _, p in plan.swap_ops))
+                         swap_blocks=sum(len(p) for _, p in plan.swap_ops), new_tokens=new)
         self.sched.complete(plan)
         self.records.append(rec)
         return rec
