@@ -232,6 +232,9 @@ typedef struct {
     int64_t num_seqs;
     int64_t host_blocks;      /* host (swap) pool size, 0 until pk_bm_set_host_blocks */
     int64_t host_free_blocks;
+    int64_t prefix_lookups;   /* keys offered to pk_bm_add_seq_cached */
+    int64_t prefix_hits;      /* of which served by a cached block */
+    int64_t cached_blocks;    /* blocks registered in the prefix cache now */
 } pk_bm_stats;
 
 int pk_bm_create(int num_blocks, int block_size, pk_bm **out);
@@ -275,6 +278,24 @@ int pk_bm_set_host_blocks(pk_bm *bm, int num_host_blocks);
 int pk_bm_swap_out(pk_bm *bm, int64_t seq, int32_t *pairs_out, int pairs_cap, int *n_pairs_out);
 int pk_bm_swap_in(pk_bm *bm, int64_t seq, int32_t *pairs_out, int pairs_cap, int *n_pairs_out);
 int pk_bm_is_swapped(const pk_bm *bm, int64_t seq, int *swapped_out);
+/* Prefix cache [BP "Sharing blocks": requests that share a system prompt can
+ * share its blocks; DD: requests with an identical prompt prefix point at the
+ * same read-only blocks, and the prefix hit rate is a metric to watch].
+ * keys[i] is the caller's name for the token prefix 0 .. (i+1)*block_size - 1
+ * (for example a chained hash of the token ids).
+ * pk_bm_cache_blocks registers seq's first n_keys logical blocks, which must
+ * be full (n_keys * block_size <= length; PK_ERR_INVALID_ARG otherwise), under
+ * keys[]; a key already cached, or a block already registered, keeps its
+ * entry.  pk_bm_add_seq_cached creates a sequence that starts on the cached
+ * blocks of the longest cached prefix of keys[] (each count + 1; length
+ * *n_hit_out * block_size); the caller then appends only the tokens after it.
+ * pk_bm_cached_prefix reports that prefix length without changing anything.
+ * An entry lives while its block is referenced: it leaves the cache when the
+ * block returns to the free list.  Cached blocks are full, so appends never
+ * write into them. */
+int pk_bm_cache_blocks(pk_bm *bm, int64_t seq, const uint64_t *keys, int n_keys);
+int pk_bm_cached_prefix(const pk_bm *bm, const uint64_t *keys, int n_keys, int *n_hit_out);
+int pk_bm_add_seq_cached(pk_bm *bm, const uint64_t *keys, int n_keys, int64_t *seq_out, int *n_hit_out);
 /* Copy seq's block table (ceil(len / bs) ids) into out[cap]; *n_out = count. */
 int pk_bm_block_table(const pk_bm *bm, int64_t seq, int32_t *out, int cap, int *n_out);
 /* Fill out[n_seqs][width] (int32, row-major) with the tables of seqs[], -1 padded. */

@@ -52,6 +52,22 @@ later; all blocks of a sequence are evicted together]:
     device pool short) changes nothing;
   * a swapped sequence can only be swapped in or freed (freeing returns its
     host blocks, last to first).
+
+Prefix cache [Batching and PagedAttention, "Sharing blocks": requests that
+share a system prompt can share its blocks, the basis of prefix caching; 7.8
+PagedAttention & continuous batching, "01 Concept": requests with an
+identical prompt prefix can point at the same read-only blocks, and the
+prefix hit rate is one of the metrics to watch]:
+  * a full block of a sequence can be registered under a key that names its
+    whole token prefix (positions 0 up to the block's end); the first block
+    registered under a key keeps it;
+  * a new sequence can start from a list of such keys: it takes, in order,
+    the cached block of every key until the first key not in the cache; each
+    taken block's count goes up, and the sequence starts at hits x block_size
+    tokens; every key offered counts as a lookup, every block taken as a hit;
+  * an entry lives while its block is referenced: when the block's count
+    reaches zero it leaves the cache as the block returns to the free list
+    (the pages fix no retention of unreferenced blocks).
 """
 
 from collections import deque
@@ -78,6 +94,10 @@ class OracleBlockManager:
         self.host_free = deque()
         self.host_filled = []
         self.swapped = set()
+        self.cache = {}                     # key -> physical block
+        self.key_of = {}                    # physical block -> key it is cached under
+        self.prefix_lookups = 0
+        self.prefix_hits = 0
 
     # -- sequences -----------------------------------------------------
     def add_seq(self):
@@ -97,6 +117,8 @@ class OracleBlockManager:
         self.refcount[block] -= 1
         if self.refcount[block] == 0:
             self.filled[block] = 0
+            if block in self.key_of:
+                del self.cache[self.key_of.pop(block)]
             self.free_list.append(block)
 
     def _resident(self, seq):
@@ -171,6 +193,40 @@ class OracleBlockManager:
             return
         for block in reversed(table):
             self._release(block)
+
+    # -- prefix cache --------------------------------------------------
+    def cache_blocks(self, seq, keys):
+        """Register seq's first len(keys) logical blocks (all full) under keys."""
+        self._resident(seq)
+        table, bs = self.tables[seq], self.block_size
+        if len(keys) * bs > self.lengths[seq]:
+            raise ValueError("only full blocks can be cached")
+        for i, key in enumerate(keys):
+            b = table[i]
+            if key not in self.cache and b not in self.key_of:
+                self.cache[key] = b
+                self.key_of[b] = key
+
+    def cached_prefix(self, keys):
+        """Blocks a sequence starting from keys would take from the cache."""
+        n = 0
+        while n < len(keys) and keys[n] in self.cache:
+            n += 1
+        return n
+
+    def add_seq_cached(self, keys):
+        """New sequence starting on the cached blocks of keys' longest cached
+        prefix.  Returns (seq id, blocks hit)."""
+        sid = self.add_seq()
+        hits = self.cached_prefix(keys)
+        for key in keys[:hits]:
+            b = self.cache[key]
+            self.refcount[b] += 1
+            self.tables[sid].append(b)
+        self.lengths[sid] = hits * self.block_size
+        self.prefix_lookups += len(keys)
+        self.prefix_hits += hits
+        return sid, hits
 
     # -- swapping ------------------------------------------------------
     def set_host_blocks(self, n):
@@ -255,4 +311,7 @@ class OracleBlockManager:
             "num_seqs": len(self.tables),
             "host_blocks": self.host_blocks,
             "host_free_blocks": len(self.host_free),
+            "prefix_lookups": self.prefix_lookups,
+            "prefix_hits": self.prefix_hits,
+            "cached_blocks": len(self.cache),
         }

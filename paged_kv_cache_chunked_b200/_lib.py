@@ -32,7 +32,9 @@ class BmStats(ctypes.Structure):
     _fields_ = [("num_blocks", ctypes.c_int64), ("free_blocks", ctypes.c_int64),
                 ("used_blocks", ctypes.c_int64), ("alloc_failures", ctypes.c_int64),
                 ("tail_waste_slots", ctypes.c_int64), ("num_seqs", ctypes.c_int64),
-                ("host_blocks", ctypes.c_int64), ("host_free_blocks", ctypes.c_int64)]
+                ("host_blocks", ctypes.c_int64), ("host_free_blocks", ctypes.c_int64),
+                ("prefix_lookups", ctypes.c_int64), ("prefix_hits", ctypes.c_int64),
+                ("cached_blocks", ctypes.c_int64)]
 
 
 _lib = None
@@ -70,6 +72,9 @@ SIGNATURES = {
     "pk_bm_swap_out": ([_P, _I64, _P, _I, _PI], _I),
     "pk_bm_swap_in": ([_P, _I64, _P, _I, _PI], _I),
     "pk_bm_is_swapped": ([_P, _I64, _PI], _I),
+    "pk_bm_cache_blocks": ([_P, _I64, _P, _I], _I),
+    "pk_bm_cached_prefix": ([_P, _P, _I, _PI], _I),
+    "pk_bm_add_seq_cached": ([_P, _P, _I, ctypes.POINTER(ctypes.c_int64), _PI], _I),
     "pk_bm_get_stats": ([_P, ctypes.POINTER(BmStats)], _I),
 }
 

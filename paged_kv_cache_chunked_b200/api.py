@@ -262,6 +262,27 @@ class BlockManager:
         Raises OutOfBlocks with nothing changed."""
         return self._swap(lib().pk_bm_swap_in, seq)
 
+    @staticmethod
+    def _keys(keys):
+        return (ctypes.c_uint64 * max(len(keys), 1))(*[k & 0xFFFFFFFFFFFFFFFF for k in keys])
+
+    def cache_blocks(self, seq, keys):
+        """Register seq's first len(keys) (full) blocks in the prefix cache."""
+        check(lib().pk_bm_cache_blocks(self._h, seq, self._keys(keys), len(keys)))
+
+    def cached_prefix(self, keys):
+        n = ctypes.c_int()
+        check(lib().pk_bm_cached_prefix(self._h, self._keys(keys), len(keys), ctypes.byref(n)))
+        return n.value
+
+    def add_seq_cached(self, keys):
+        """New sequence on the cached blocks of keys' longest cached prefix;
+        returns (seq id, blocks hit)."""
+        s, n = ctypes.c_int64(), ctypes.c_int()
+        check(lib().pk_bm_add_seq_cached(self._h, self._keys(keys), len(keys), ctypes.byref(s),
+                                         ctypes.byref(n)))
+        return s.value, n.value
+
     def is_swapped(self, seq):
         r = ctypes.c_int()
         check(lib().pk_bm_is_swapped(self._h, seq, ctypes.byref(r)))

@@ -28,6 +28,17 @@
 // that cannot be met in full changes nothing.  A swapped sequence can only be
 // swapped in or freed.
 //
+// Prefix cache ["Batching and PagedAttention", "Sharing blocks": requests that
+// share a system prompt can share its blocks, the basis of prefix caching;
+// "7.8 PagedAttention & continuous batching", "01 Concept": requests with an
+// identical prompt prefix point at the same read-only blocks; prefix hit rate]:
+// a full block can be registered under a caller key naming its whole token
+// prefix (the first registration of a key keeps it); a new sequence can start
+// from a list of keys and takes, in order, the cached block of each key until
+// the first miss (counts + 1, length hits x block_size; every key offered is a
+// lookup, every block taken a hit); an entry lives while its block is
+// referenced and leaves the cache when the block returns to the free list.
+//
 // Policy details the pages leave open, fixed so that tables are reproducible:
 // FIFO free list starting as 0..N-1 (a released block joins the tail);
 // a sequence's blocks are released from its last logical block to its first;
@@ -59,6 +70,9 @@ struct pk_bm {
     int num_host_blocks = 0;
     std::deque<int32_t> host_free;
     std::vector<int32_t> host_filled;
+    std::unordered_map<uint64_t, int32_t> cache;   // key -> physical block
+    std::unordered_map<int32_t, uint64_t> key_of;  // physical block -> its key
+    int64_t prefix_lookups = 0, prefix_hits = 0;
     std::unordered_map<int64_t, Seq> seqs;
     int64_t next_seq = 0;
     int64_t alloc_failures = 0;
@@ -73,8 +87,18 @@ struct pk_bm {
     void release(int32_t b) {
         if (--refcount[b] == 0) {
             filled[b] = 0;
+            auto k = key_of.find(b);
+            if (k != key_of.end()) {
+                cache.erase(k->second);
+                key_of.erase(k);
+            }
             free_list.push_back(b);
         }
+    }
+    int cached_prefix(const uint64_t *keys, int n) const {
+        int h = 0;
+        while (h < n && cache.count(keys[h])) ++h;
+        return h;
     }
     int64_t needed(const Seq &s, int n) const {
         if (n <= 0) return 0;
@@ -277,6 +301,50 @@ int pk_bm_swap_in(pk_bm *bm, int64_t seq, int32_t *pairs_out, int pairs_cap, int
     return PK_OK;
 }
 
+int pk_bm_cache_blocks(pk_bm *bm, int64_t seq, const uint64_t *keys, int n_keys) {
+    if (!bm || (n_keys > 0 && !keys) || n_keys < 0) return fail(PK_ERR_INVALID_ARG, "bad argument");
+    pk_bm::Seq *sq = resident(bm, seq);
+    if (!sq) return PK_ERR_INVALID_ARG;
+    if ((int64_t)n_keys * bm->block_size > sq->len)
+        return fail(PK_ERR_INVALID_ARG, "only full blocks can be cached (%d keys, %lld tokens)", n_keys,
+                    (long long)sq->len);
+    for (int i = 0; i < n_keys; ++i) {
+        const int32_t b = sq->table[i];
+        if (!bm->cache.count(keys[i]) && !bm->key_of.count(b)) {
+            bm->cache.emplace(keys[i], b);
+            bm->key_of.emplace(b, keys[i]);
+        }
+    }
+    return PK_OK;
+}
+
+int pk_bm_cached_prefix(const pk_bm *bm, const uint64_t *keys, int n_keys, int *n_hit_out) {
+    if (!bm || !n_hit_out || (n_keys > 0 && !keys) || n_keys < 0)
+        return fail(PK_ERR_INVALID_ARG, "bad argument");
+    *n_hit_out = bm->cached_prefix(keys, n_keys);
+    return PK_OK;
+}
+
+int pk_bm_add_seq_cached(pk_bm *bm, const uint64_t *keys, int n_keys, int64_t *seq_out, int *n_hit_out) {
+    if (!bm || !seq_out || !n_hit_out || (n_keys > 0 && !keys) || n_keys < 0)
+        return fail(PK_ERR_INVALID_ARG, "bad argument");
+    const int64_t id = bm->next_seq++;
+    pk_bm::Seq s;
+    const int hits = bm->cached_prefix(keys, n_keys);
+    for (int i = 0; i < hits; ++i) {
+        const int32_t b = bm->cache.at(keys[i]);
+        ++bm->refcount[b];
+        s.table.push_back(b);
+    }
+    s.len = (int64_t)hits * bm->block_size;
+    bm->seqs.emplace(id, std::move(s));
+    bm->prefix_lookups += n_keys;
+    bm->prefix_hits += hits;
+    *seq_out = id;
+    *n_hit_out = hits;
+    return PK_OK;
+}
+
 int pk_bm_is_swapped(const pk_bm *bm, int64_t seq, int *swapped_out) {
     if (!bm || !swapped_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
     auto it = bm->seqs.find(seq);
@@ -342,6 +410,9 @@ int pk_bm_get_stats(const pk_bm *bm, pk_bm_stats *out) {
     out->num_seqs = (int64_t)bm->seqs.size();
     out->host_blocks = bm->num_host_blocks;
     out->host_free_blocks = (int64_t)bm->host_free.size();
+    out->prefix_lookups = bm->prefix_lookups;
+    out->prefix_hits = bm->prefix_hits;
+    out->cached_blocks = (int64_t)bm->cache.size();
     return PK_OK;
 }
 

@@ -16,7 +16,9 @@ def _same_state(bm, ob):
     assert bm.stats() == {"num_blocks": ob.num_blocks, "free_blocks": ob.num_free(),
                           "used_blocks": ob.num_used(), "alloc_failures": ob.alloc_failures,
                           "tail_waste_slots": ob.tail_waste(), "num_seqs": len(ob.tables),
-                          "host_blocks": ob.host_blocks, "host_free_blocks": len(ob.host_free)}
+                          "host_blocks": ob.host_blocks, "host_free_blocks": len(ob.host_free),
+                          "prefix_lookups": ob.prefix_lookups, "prefix_hits": ob.prefix_hits,
+                          "cached_blocks": len(ob.cache)}
     for sid in ob.tables:
         assert bm.block_table(sid) == ob.block_table(sid)
         assert bm.length(sid) == ob.length(sid)
@@ -33,13 +35,28 @@ def test_random_operations_match_the_oracle(seed):
     bm.set_host_blocks(nb // 2)
     ob.set_host_blocks(nb // 2)
     live = []
+    prompt_keys = {}
     for step in range(500):
         op = rng.random()
         resident = [s for s in live if s not in ob.swapped]
-        if op < 0.15 or not resident:
+        if op < 0.08 or not resident:
             a, b = bm.add_seq(), ob.add_seq()
             assert a == b
             live.append(a)
+        elif op < 0.15:
+            # a request on one of three shared prompts (keys name prefixes)
+            g = rng.randrange(3)
+            keys = [1000 * g + i for i in range(rng.randint(0, 4))]
+            assert bm.cached_prefix(keys) == ob.cached_prefix(keys)
+            a, b = bm.add_seq_cached(keys), ob.add_seq_cached(keys)
+            assert a == b
+            live.append(a[0])
+            prompt_keys[a[0]] = keys
+        elif op < 0.24 and any(s in prompt_keys for s in resident):
+            s = rng.choice([s for s in resident if s in prompt_keys])
+            full = min(len(prompt_keys[s]), ob.length(s) // bs)
+            bm.cache_blocks(s, prompt_keys[s][:full])
+            ob.cache_blocks(s, prompt_keys[s][:full])
         elif op < 0.25:
             p = rng.choice(resident)
             a, b = bm.fork(p), ob.fork(p)
@@ -80,6 +97,37 @@ def test_random_operations_match_the_oracle(seed):
         if step % 25 == 0:
             _same_state(bm, ob)
     _same_state(bm, ob)
+
+
+def test_prefix_cache_script_matches_the_oracle():
+    # requests on two shared prompts arrive, hit, finish and come back, in
+    # both managers, state compared after every call
+    bm, ob = BlockManager(64, 4), OracleBlockManager(64, 4)
+    keys = {g: [100 * g + i for i in range(5)] for g in (1, 2)}
+    live = {}
+    script = [("new", 1, 18), ("new", 2, 9), ("reg", 0), ("reg", 1), ("new", 1, 22), ("new", 2, 12),
+              ("new", 1, 7), ("free", 0), ("new", 1, 30), ("reg", 4), ("free", 2), ("free", 4),
+              ("new", 1, 20), ("free", 6), ("free", 5), ("new", 1, 20), ("new", 2, 5)]
+    for i, step in enumerate(script):
+        if step[0] == "new":
+            _, g, n = step
+            a, b = bm.add_seq_cached(keys[g]), ob.add_seq_cached(keys[g])
+            assert a == b
+            live[len(live)] = (a[0], g)
+            ref = ob.append_slots(a[0], n)
+            assert bm.append_slots(a[0], n) == (ref[0], ref[1])
+        elif step[0] == "reg":
+            s_, g = live[step[1]]
+            full = min(len(keys[g]), ob.length(s_) // 4)
+            bm.cache_blocks(s_, keys[g][:full])
+            ob.cache_blocks(s_, keys[g][:full])
+        else:
+            s_, _ = live[step[1]]
+            bm.free(s_)
+            ob.free(s_)
+        _same_state(bm, ob)
+    st = bm.stats()
+    assert st["prefix_hits"] == 20 and st["prefix_lookups"] == 5 * 9
 
 
 def test_page_toy_capacity_through_the_product_manager():

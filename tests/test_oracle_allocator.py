@@ -269,3 +269,101 @@ def test_swap_refusals_change_nothing():
         big.append_slots(u, 1)
     big.free(u)                                # returns its host blocks
     assert big.stats()["host_free_blocks"] == 3
+
+
+# ---------------------------------------------------------------- prefix cache
+def test_prefix_cache_shares_a_system_prompt_across_requests():
+    # "requests that share a system prompt can share its blocks too, which is
+    # the basis of prefix caching" [Batching and PagedAttention, "Sharing
+    # blocks"]: the second request reads the first one's prompt blocks, which
+    # were written once, and writes only its own suffix
+    import torch
+    import oracle
+    bs, H, d = 16, 2, 4
+    bm = OracleBlockManager(12, bs)
+    kp, vp = torch.zeros(12, H, bs, d), torch.zeros(12, H, bs, d)
+    keys = ["sys0", "sys1"]                        # two full blocks of system prompt
+    sys_k = torch.randn(32, H, d)
+
+    a, hits = bm.add_seq_cached(keys)
+    assert hits == 0 and bm.length(a) == 0
+    slots, _ = bm.append_slots(a, 40)             # system prompt + 8 own tokens
+    oracle.kv_append(kp, vp, torch.cat([sys_k, torch.randn(8, H, d)]), torch.zeros(40, H, d),
+                     torch.tensor(slots))
+    bm.cache_blocks(a, keys)
+    b, hits = bm.add_seq_cached(keys + ["b-own"])
+    assert hits == 2 and bm.length(b) == 32
+    assert bm.block_table(b) == bm.block_table(a)[:2]
+    assert [bm.refcount[x] for x in bm.block_table(b)] == [2, 2]
+    slots, pairs = bm.append_slots(b, 5)          # b's suffix starts a block of its own
+    assert pairs == [] and all(s // bs not in bm.block_table(a) for s in slots)
+    t = torch.tensor(bm.block_table(b))
+    got = kp[t].transpose(1, 2).reshape(-1, H, d)[:32]
+    assert torch.equal(got, sys_k)
+    assert bm.stats()["prefix_lookups"] == 5 and bm.stats()["prefix_hits"] == 2
+    _check_invariants(bm)
+
+
+def test_prefix_cache_entries_live_while_referenced():
+    bm = OracleBlockManager(8, 4)
+    a, _ = bm.add_seq_cached(["k0", "k1"])
+    bm.append_slots(a, 8)
+    bm.cache_blocks(a, ["k0", "k1"])
+    b, hits = bm.add_seq_cached(["k0", "k1"])
+    assert hits == 2
+    bm.free(a)                                     # b still references both blocks
+    assert bm.cached_prefix(["k0", "k1"]) == 2
+    bm.free(b)                                     # counts reach zero: entries leave
+    assert bm.cached_prefix(["k0"]) == 0 and bm.stats()["cached_blocks"] == 0
+    assert bm.num_free() == 8
+
+
+def test_prefix_cache_first_registration_wins_and_needs_full_blocks():
+    bm = OracleBlockManager(8, 4)
+    a, _ = bm.add_seq_cached([])
+    bm.append_slots(a, 6)
+    with pytest.raises(ValueError):
+        bm.cache_blocks(a, ["x0", "x1"])           # block 1 holds 2 of 4 slots
+    bm.cache_blocks(a, ["x0"])
+    b, _ = bm.add_seq_cached([])
+    bm.append_slots(b, 4)
+    bm.cache_blocks(b, ["x0"])                     # already cached: a's block keeps it
+    c, hits = bm.add_seq_cached(["x0"])
+    assert hits == 1 and bm.block_table(c) == [bm.block_table(a)[0]]
+    _check_invariants(bm)
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_random_operations_with_prefix_cache_keep_invariants(seed):
+    rng = random.Random(50 + seed)
+    bs = rng.choice([4, 16])
+    bm = OracleBlockManager(60, bs)
+    live = []
+    for _ in range(400):
+        op = rng.random()
+        if op < 0.25 or not live:
+            g = rng.randrange(3)                    # one of three shared prompts
+            keys = [f"g{g}b{i}" for i in range(rng.randint(0, 4))]
+            s, hits = bm.add_seq_cached(keys)
+            assert bm.length(s) == hits * bs
+            live.append((s, keys))
+        elif op < 0.4:
+            s, keys = rng.choice(live)
+            full = min(len(keys), bm.length(s) // bs)
+            bm.cache_blocks(s, keys[:full])
+        elif op < 0.55:
+            item = rng.choice(live)
+            live.remove(item)
+            bm.free(item[0])
+        else:
+            s, _ = rng.choice(live)
+            try:
+                bm.append_slots(s, rng.randint(0, 3 * bs))
+            except OracleOOM:
+                pass
+        _check_invariants(bm)
+        for key, b in bm.cache.items():             # cached blocks are referenced and full
+            assert bm.refcount[b] > 0 and bm.filled[b] == bs
+    for s, _ in live:
+        bm.free(s)
+    assert bm.num_free() == 60 and bm.stats()["cached_blocks"] == 0
