@@ -50,7 +50,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="decode64_bf16",
-                   choices=["decode64_bf16", "longdoc_bf16", "chunk512_bf16", "trace", "trace_swap", "fork",
+                   choices=["decode64_bf16", "longdoc_bf16", "chunk512_bf16", "trace", "trace_swap",
+                            "trace_prefix", "trace_prefix_nocache", "fork",
                             "fork1028", "append_copy"])
     p.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
     p.add_argument("--no-e2e", action="store_true")
@@ -656,11 +657,18 @@ def run_serving(args, rank, world, device):
     peak, peak_kind = measured_peak()
     kv_tok = 8 * 128 * 2 * 2          # K+V bytes per token per layer (8 kv heads, d 128, bf16)
     recs = []
-    if args.workload in ("trace", "trace_swap"):
+    if args.workload.startswith("trace"):
         # trace_swap: preempted requests' blocks go to a pinned host pool of
-        # 8,192 blocks and back instead of being recomputed
+        # 8,192 blocks and back instead of being recomputed.  trace_prefix:
+        # every request starts with one of four shared system prompts (1,024,
+        # 512, 2,048 or 256 tokens) whose blocks are shared through the prefix
+        # cache; trace_prefix_nocache runs the same trace without the cache.
+        from paged_kv_cache_chunked_b200.workloads import prefix_trace_requests
         swap = args.workload == "trace_swap"
-        r = TraceRunner(device, preempt="swap" if swap else "recompute", num_host_blocks=8192 if swap else 0)
+        prefix = args.workload.startswith("trace_prefix")
+        r = TraceRunner(device, preempt="swap" if swap else "recompute", num_host_blocks=8192 if swap else 0,
+                        trace=prefix_trace_requests() if prefix else None,
+                        prefix_cache=args.workload == "trace_prefix")
         while r.sched.step_no < 300 and (r.pending or r.sched.has_work()):
             rec = r.step()
             if rec is not None:
@@ -673,6 +681,14 @@ def run_serving(args, rank, world, device):
                "preempt": r.sched.preempt_mode,
                "preemptions": r.sched.metrics["preemptions"], "rejected": r.rejected,
                "finished": len(r.sched.finished)}
+        if prefix:
+            st = r.bm.stats()
+            cfg.update(trace="prefix_trace_requests(seed 1007): system prompts 1024/512/2048/256, user "
+                             "median 256", prefix_cache=r.sched.prefix_cache,
+                       prefix_lookups_blocks=st["prefix_lookups"], prefix_hits_blocks=st["prefix_hits"],
+                       prefix_hit_rate=st["prefix_hits"] / max(st["prefix_lookups"], 1),
+                       prefix_hit_tokens=r.sched.metrics["prefix_hit_tokens"],
+                       gpu_ms_timed_steps=sum(x.gpu_ms for x in recs))
         if swap:
             cfg.update(host_blocks=8192, swaps_out=r.sched.metrics["swaps_out"],
                        swaps_in=r.sched.metrics["swaps_in"],
@@ -735,7 +751,7 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                  device_id=device)
     try:
-        if args.workload in ("trace", "trace_swap", "fork", "fork1028"):
+        if args.workload.startswith("trace") or args.workload in ("fork", "fork1028"):
             run_serving(args, rank, world, device)
         elif args.workload == "append_copy":
             run_kvops(args, rank, world, device)

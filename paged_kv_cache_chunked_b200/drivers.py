@@ -8,7 +8,10 @@ TraceRunner   continuous batching over an arrival trace: each iteration the
               "Flow"; "Batching and PagedAttention", "Continuous batching"].
               Preempted requests are recomputed, or with preempt="swap" their
               blocks go to a pinned host pool and back ["Batching and
-              PagedAttention", "When blocks run out"].
+              PagedAttention", "When blocks run out"].  With prefix_cache and
+              a trace of shared system prompts, a request starts on the
+              blocks of its system prompt that another request already wrote
+              ["Batching and PagedAttention", "Sharing blocks"].
 ForkRunner    n parallel samples of each prompt: prefill, fork (children share
               the prompt's blocks by reference count), then decode steps in
               which the first write into a shared, partly filled tail block
@@ -23,7 +26,7 @@ import torch
 
 from . import api
 from .scheduler import Request, Scheduler
-from .workloads import token_values, trace_requests
+from .workloads import SYS_VID_BASE, token_values, trace_requests
 
 
 class StepRecord:
@@ -40,7 +43,8 @@ class TraceRunner:
 
     def __init__(self, device, num_blocks=8192, block_size=16, n_q_heads=32, n_kv_heads=8,
                  head_dim=128, token_budget=4096, max_chunk=512, trace=None, seed=1004,
-                 n_steps=300, dtype=torch.bfloat16, preempt="recompute", num_host_blocks=0):
+                 n_steps=300, dtype=torch.bfloat16, preempt="recompute", num_host_blocks=0,
+                 prefix_cache=False):
         self.device = torch.device(device)
         self.Hq, self.Hkv, self.d, self.bs = n_q_heads, n_kv_heads, head_dim, block_size
         self.dtype = dtype
@@ -53,9 +57,12 @@ class TraceRunner:
         if preempt == "swap":
             self.bm.set_host_blocks(num_host_blocks)
             self.host = api.host_pool_create(num_host_blocks, self.pool)
-        self.sched = Scheduler(self.bm, token_budget, max_chunk, preempt=preempt)
+        self.sched = Scheduler(self.bm, token_budget, max_chunk, preempt=preempt,
+                               prefix_cache=prefix_cache)
         trace = trace if trace is not None else trace_requests(n_steps=n_steps, seed=seed)
-        self.pending = [Request(i, a, p, o) for i, (a, p, o) in enumerate(trace)]
+        # (arrival, prompt, output) or (arrival, prompt, output, group, system prompt length)
+        self.pending = [Request(i, *t[:3], group=t[3], sys_len=t[4]) if len(t) == 5 else Request(i, *t)
+                        for i, t in enumerate(trace)]
         self.scale = head_dim ** -0.5
         self.records = []
         self.rejected = 0
@@ -100,7 +107,7 @@ class TraceRunner:
             return rec
         rids, pos = [], []
         for req, s, n in zip(plan.requests, plan.starts, plan.counts):
-            rids.extend([req.rid] * n)
+            rids.extend(self.value_ids(req, s, n))
             pos.extend(range(s, s + n))
         meta = {
             "slots": torch.tensor(plan.slots, dtype=torch.int64),
@@ -145,6 +152,15 @@ class TraceRunner:
         self.sched.complete(plan)
         self.records.append(rec)
         return rec
+
+    @staticmethod
+    def value_ids(req, start, n):
+        """Generator key of positions start .. start+n-1 of req: its system
+        prompt's for the shared prefix, its own after it."""
+        if req.group < 0:
+            return [req.rid] * n
+        shared = SYS_VID_BASE + req.group
+        return [shared if p < req.sys_len else req.rid for p in range(start, start + n)]
 
     def _run_swaps(self, swaps):
         # in the order the scheduler decided them: a swap-in may reuse blocks a

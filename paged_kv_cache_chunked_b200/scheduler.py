@@ -42,6 +42,19 @@ blocks move to CPU memory, all together, and come back before it runs again
     copy-on-write copies, appends and attention (a swap-in may land in blocks
     a swap-out of the same step just freed).
 
+Prefix cache (prefix_cache=True): a request whose prompt starts with a shared
+system prompt starts on the cached blocks of that prompt, when another request
+already wrote them, and prefills only the rest ["Batching and PagedAttention",
+"Sharing blocks": requests that share a system prompt can share its blocks,
+the basis of prefix caching].  Readings:
+  * a block is named by (system prompt, block index), which names its whole
+    token prefix; only blocks wholly inside the system prompt are cached, and
+    at least one prompt token is always prefilled (its query yields the first
+    output token);
+  * admission reasons in the blocks the first chunk needs after the hit;
+  * a request's system-prompt blocks enter the cache once the step that
+    filled them has run.
+
 A request with prompt length P and output length O stores P + O - 1 tokens:
 the last prefill chunk yields the first output token, each decode step
 appends the previous output token and yields the next.
@@ -67,6 +80,8 @@ class Request:
     finish_step: int = -1
     preemptions: int = 0
     swapped_step: int = -1
+    group: int = -1          # shared system prompt, -1 for none
+    sys_len: int = 0         # tokens of the shared system prompt at the start of the prompt
     token_steps: list = field(default_factory=list)
 
     def __post_init__(self):
@@ -104,7 +119,7 @@ class StepPlan:
 
 
 class Scheduler:
-    def __init__(self, bm, token_budget=4096, max_chunk=512, preempt="recompute"):
+    def __init__(self, bm, token_budget=4096, max_chunk=512, preempt="recompute", prefix_cache=False):
         if preempt not in ("recompute", "swap"):
             raise ValueError("preempt must be 'recompute' or 'swap'")
         self.bm = bm
@@ -112,6 +127,7 @@ class Scheduler:
         self.token_budget = token_budget
         self.max_chunk = max_chunk
         self.preempt_mode = preempt
+        self.prefix_cache = prefix_cache
         self.waiting = []    # arrival order
         self.running = []    # arrival order; hold blocks
         self.swapped = []    # arrival order; blocks in the host pool
@@ -119,7 +135,7 @@ class Scheduler:
         self.step_no = 0
         self._swap_ops = []  # swaps decided since the last plan was handed out
         self.metrics = {"preemptions": 0, "alloc_failures": 0, "admitted": 0, "swaps_out": 0,
-                        "swaps_in": 0}
+                        "swaps_in": 0, "prefix_hit_tokens": 0}
 
     def add_request(self, req):
         """Queue a request; one that could never fit in the whole pool is
@@ -162,6 +178,14 @@ class Scheduler:
         self.metrics["preemptions"] += 1
         self.running.remove(req)
         self._requeue(req)
+
+    def _prefix_keys(self, req):
+        """Cache keys of the request's blocks that lie wholly inside its system
+        prompt, leaving at least one prompt token to prefill."""
+        if not self.prefix_cache or req.group < 0:
+            return []
+        n = min(req.sys_len, req.prompt_len - 1) // self.block_size
+        return [((req.group + 1) << 32) | i for i in range(n)]
 
     def _latest_running(self):
         return max(self.running, key=lambda r: (r.arrival, r.rid))
@@ -230,19 +254,29 @@ class Scheduler:
         for req in candidates:
             if budget == 0:
                 break
-            n = min(self.max_chunk, req.target - req.stored, budget)
             if req.seq < 0:
-                # admission: reason in blocks before taking any
-                need = -(-n // self.block_size)
+                # admission: reason in blocks before taking any (after the
+                # prefix-cache hit, whose blocks are already in the pool)
+                keys = self._prefix_keys(req)
+                hits = self.bm.cached_prefix(keys) if keys else 0
+                start = hits * self.block_size
+                n = min(self.max_chunk, req.target - start, budget)
+                need = -(-(start + n) // self.block_size) - hits
                 if need > self.bm.num_free():
                     break        # FCFS: later arrivals wait behind this one
-                req.seq = self.bm.add_seq()
+                if keys:
+                    req.seq, hits = self.bm.add_seq_cached(keys)
+                    req.stored = hits * self.block_size
+                    self.metrics["prefix_hit_tokens"] += req.stored
+                else:
+                    req.seq = self.bm.add_seq()
                 if req.admit_step < 0:
                     req.admit_step = self.step_no
                 self.waiting.remove(req)
                 self.running.append(req)
                 self.running.sort(key=lambda r: (r.arrival, r.rid))
                 self.metrics["admitted"] += 1
+            n = min(self.max_chunk, req.target - req.stored, budget)
             if self.bm.blocks_needed(req.seq, n) > self.bm.num_free():
                 break
             reserve(req, n)
@@ -259,6 +293,11 @@ class Scheduler:
         for req, n in zip(plan.requests, plan.counts):
             was_prefill = req.stored < req.target
             req.stored += n
+            if was_prefill and self.prefix_cache and req.group >= 0:
+                keys = self._prefix_keys(req)
+                full = min(len(keys), req.stored // self.block_size)
+                if full:
+                    self.bm.cache_blocks(req.seq, keys[:full])
             if was_prefill:
                 if req.stored == req.target and req.generated == 0:
                     req.generated = 1

@@ -205,3 +205,31 @@ def trace_requests(n_steps=300, arrivals_per_step=4.0, prompt_median=512, prompt
             o = int(rng.integers(out_min, out_max + 1))
             out.append((step, p, o))
     return out
+
+
+# value ids at or above this are shared system prompts, not requests
+SYS_VID_BASE = 1 << 30
+
+
+def prefix_trace_requests(n_steps=300, arrivals_per_step=4.0, sys_lens=(1024, 512, 2048, 256),
+                          user_median=256, user_sigma=1.0, user_max=4096, out_min=10, out_max=500,
+                          seed=1007):
+    """A continuous-batching trace in which every request starts with one of a
+    few shared system prompts ["Batching and PagedAttention", "Sharing
+    blocks": requests that share a system prompt can share its blocks]:
+    Poisson arrivals, a system prompt drawn uniformly from sys_lens, then a
+    lognormal user part (median user_median, clipped to [1, user_max]) and an
+    output length uniform in [out_min, out_max].  Returns (arrival_step,
+    prompt_len, output_len, group, sys_len) tuples in arrival order; a
+    request's tokens before sys_len are its group's, the rest its own."""
+    import numpy as np
+    rng = np.random.Generator(np.random.PCG64(seed))
+    out = []
+    for step in range(n_steps):
+        for _ in range(int(rng.poisson(arrivals_per_step))):
+            g = int(rng.integers(0, len(sys_lens)))
+            u = int(round(float(rng.lognormal(math.log(user_median), user_sigma))))
+            u = min(max(u, 1), user_max)
+            o = int(rng.integers(out_min, out_max + 1))
+            out.append((step, sys_lens[g] + u, o, g, sys_lens[g]))
+    return out

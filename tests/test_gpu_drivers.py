@@ -183,3 +183,39 @@ def test_trace_in_swap_mode_matches_the_oracle(cuda_dev):
     m = runner.sched.metrics
     assert m["swaps_out"] > 0 and m["swaps_in"] > 0
     assert runner.pool.check_device_errors() == 0
+
+
+def test_trace_with_prefix_cache_matches_the_oracle(cuda_dev):
+    # requests on shared system prompts start on the prompt's blocks written by
+    # an earlier request ["Batching and PagedAttention", "Sharing blocks"]:
+    # attention matches the oracle, and every request's K read through its own
+    # table equals, bit for bit, the values its own tokens would have
+    from paged_kv_cache_chunked_b200.workloads import prefix_trace_requests, token_values
+    trace = prefix_trace_requests(n_steps=30, arrivals_per_step=3.0, sys_lens=(200, 64, 320),
+                                  user_median=100, user_max=800, out_min=5, out_max=40, seed=79)
+    runner = TraceRunner(cuda_dev, num_blocks=500, n_steps=30, trace=trace, token_budget=1024,
+                         max_chunk=256, prefix_cache=True)
+    mirror = Mirror(runner.pool)
+    gen = torch.Generator().manual_seed(2)
+
+    def on_step(plan, t, out):
+        mirror.apply(t["pairs"], t["k"], t["v"], t["slots"])
+        rows = []
+        qsl = t["qsl"].tolist()
+        for i, (req, s) in enumerate(zip(plan.requests, plan.starts)):
+            toks = list(range(qsl[i], qsl[i + 1]))
+            pick = {toks[0], toks[-1], toks[int(torch.randint(len(toks), (1,), generator=gen))]}
+            rows += [(tk, h) for tk in pick for h in (0, runner.Hq - 1)]
+        _check_rows(mirror, t, out, rows, runner.scale, f"prefix trace step {plan.step}")
+        for i, req in enumerate(plan.requests):
+            c = plan.context_lens[i]
+            table = t["tables"][i, :-(-c // runner.bs)].long()
+            got = mirror.k[table].transpose(1, 2).reshape(-1, runner.Hkv, runner.d)[:c]
+            want = token_values(runner.seed, 1, runner.value_ids(req, 0, c), list(range(c)),
+                                runner.Hkv, runner.d, runner.dtype)
+            assert torch.equal(got, want), f"request {req.rid}: K through its table differs"
+
+    runner.run(max_steps=60, on_step=on_step)
+    st = runner.bm.stats()
+    assert runner.sched.metrics["prefix_hit_tokens"] > 0 and st["prefix_hits"] > 0
+    assert runner.pool.check_device_errors() == 0

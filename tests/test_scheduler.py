@@ -205,3 +205,64 @@ def test_small_host_pool_falls_back_to_recompute():
     sched, _ = _run(bm, _small_trace(), 40, preempt="swap")
     assert len(sched.finished) == len(_small_trace())
     assert sched.metrics["preemptions"] > sched.metrics["swaps_out"]
+
+
+# ---------------------------------------------------------------- prefix cache
+def _prefix_trace():
+    from paged_kv_cache_chunked_b200.workloads import prefix_trace_requests
+    return prefix_trace_requests(n_steps=40, arrivals_per_step=3.0, sys_lens=(200, 64, 320),
+                                 user_median=100, user_max=800, out_min=5, out_max=60, seed=78)
+
+
+def _prefix_run(bm, prefix_cache=True, n_steps=40):
+    sched = Scheduler(bm, token_budget=4096, max_chunk=512, prefix_cache=prefix_cache)
+    pending = [Request(i, a, p, o, group=g, sys_len=sl) for i, (a, p, o, g, sl) in enumerate(_prefix_trace())]
+    plans = []
+    step = 0
+    while step < n_steps or sched.has_work():
+        while pending and pending[0].arrival <= step:
+            sched.add_request(pending.pop(0))
+        plan = sched.schedule()
+        plans.append(plan)
+        _check_plan(plan, sched, 4096, 512)
+        sched.complete(plan)
+        step += 1
+        assert step < 20 * n_steps, "trace did not drain"
+    return sched, plans
+
+
+def test_prefix_cache_product_and_oracle_managers_plan_identically():
+    s1, p1 = _prefix_run(BlockManager(600, 16))
+    s2, p2 = _prefix_run(OracleAdapter(600, 16))
+    assert len(p1) == len(p2)
+    for a, b in zip(p1, p2):
+        assert [r.rid for r in a.requests] == [r.rid for r in b.requests]
+        assert a.starts == b.starts and a.counts == b.counts and a.slots == b.slots
+        assert torch.equal(a.tables, b.tables)
+    assert s1.metrics == s2.metrics and s1.metrics["prefix_hit_tokens"] > 0
+
+
+def test_prefix_cache_skips_exactly_the_shared_tokens_and_drains():
+    # each request's shared-prompt blocks come from the cache when another
+    # request wrote them; every other position is written exactly once, and
+    # every block (cached ones included) is back in the pool at the end
+    bm = BlockManager(600, 16)
+    sched, plans = _prefix_run(bm)
+    cold, _ = _prefix_run(BlockManager(600, 16), prefix_cache=False)
+    written = {}
+    for plan in plans:
+        for req, s, n in zip(plan.requests, plan.starts, plan.counts):
+            for pos in range(s, s + n):
+                written[(req.rid, pos)] = written.get((req.rid, pos), 0) + 1
+    hit = sched.metrics["prefix_hit_tokens"]
+    assert hit > 0 and len(sched.finished) == len(_prefix_trace())
+    for r in sched.finished:
+        mine = [pos for (rid, pos) in written if rid == r.rid]
+        skipped = r.stored - len(mine)
+        assert skipped % 16 == 0 and skipped <= r.sys_len        # whole shared blocks only
+        assert all(pos >= skipped for pos in mine)               # the skipped part is the prefix
+    if sched.metrics["preemptions"] == 0 and cold.metrics["preemptions"] == 0:
+        tokens = lambda s: sum(r.stored for r in s.finished)
+        assert sum(written.values()) == tokens(sched) - hit
+    st = bm.stats()
+    assert st["free_blocks"] == 600 and st["cached_blocks"] == 0 and st["prefix_hits"] * 16 == hit
