@@ -51,7 +51,7 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="decode64_bf16",
                    choices=["decode64_bf16", "longdoc_bf16", "chunk512_bf16", "trace", "trace_swap",
-                            "trace_prefix", "trace_prefix_nocache", "fork",
+                            "trace_prefix", "trace_prefix_nocache", "policy", "fork",
                             "fork1028", "append_copy"])
     p.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
     p.add_argument("--no-e2e", action="store_true")
@@ -735,6 +735,54 @@ def run_serving(args, rank, world, device):
         print(json.dumps(line), flush=True)
 
 
+def run_policy(args, rank, world, device):
+    """Scheduler policy study ["Batching and PagedAttention", "Scheduling is a
+    policy" and "Static batching"; 7.8 PagedAttention & continuous batching,
+    "01 Concept": queue delay, time to first token, inter-token latency by
+    request class]: one serving trace (about one arrival a step for 300 steps,
+    333 requests) run to completion under continuous batching with token
+    budgets of 1,024, 2,048, 4,096 and 8,192 per step, and under static
+    batching (batches of 64, budget 4,096).  Latencies are in scheduler steps
+    and in GPU ms (per-step CUDA events, summed); value is the tokens/s of the
+    4,096 continuous configuration."""
+    from paged_kv_cache_chunked_b200.drivers import TraceRunner
+    from paged_kv_cache_chunked_b200.scheduler import summary
+    from paged_kv_cache_chunked_b200.workloads import trace_requests
+    trace = trace_requests(n_steps=300, arrivals_per_step=1.0, seed=1004)
+    configs = [("continuous_1024", dict(token_budget=1024)), ("continuous_2048", dict(token_budget=2048)),
+               ("continuous_4096", dict(token_budget=4096)), ("continuous_8192", dict(token_budget=8192)),
+               ("static64_4096", dict(token_budget=4096, static_batch=64))]
+    pick = lambda st, k: None if st is None else {q: st[q] for q in ("p50", "p90")} if k else st
+    study = {}
+    for name, kw in configs:
+        r = TraceRunner(device, trace=trace, **kw)
+        while r.pending or r.sched.has_work():
+            r.step()
+        ms = r.step_ms()
+        tot = sum(ms)
+        summ = summary(r.sched.finished, ms)
+        study[name] = {
+            "steps": r.sched.step_no, "finished": len(r.sched.finished), "gpu_ms": tot,
+            "tokens_per_s": sum(x.tokens for x in r.records) / (tot * 1e-3),
+            "useful_tokens_per_s": sum(x.new_tokens for x in r.records) / (tot * 1e-3),
+            "preemptions": r.sched.metrics["preemptions"],
+            "by_class": {cls: {"requests": v["requests"], "queue_delay_steps": pick(v["queue_delay"], 1),
+                               "ttft_steps": pick(v["ttft"], 1), "ttft_ms": pick(v["ttft_ms"], 1),
+                               "itl_ms": pick(v["itl_ms"], 1)}
+                         for cls, v in summ.items()}}
+    base = study["continuous_4096"]
+    line = {"metric": METRIC, "value": base["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
+            "steps": base["steps"], "warmup": 0, "ms_per_step": base["gpu_ms"] / base["steps"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "policy", "trace": "trace_requests(arrivals 1.0/step, 300 steps, seed 1004)",
+                       "requests": len(trace), "num_blocks": 8192, "block_size": 16, "max_chunk": 512},
+            "study": study,
+            "timing": "per-step CUDA events around copy + append + attention, summed; host scheduling excluded"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -751,7 +799,9 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                  device_id=device)
     try:
-        if args.workload.startswith("trace") or args.workload in ("fork", "fork1028"):
+        if args.workload == "policy":
+            run_policy(args, rank, world, device)
+        elif args.workload.startswith("trace") or args.workload in ("fork", "fork1028"):
             run_serving(args, rank, world, device)
         elif args.workload == "append_copy":
             run_kvops(args, rank, world, device)

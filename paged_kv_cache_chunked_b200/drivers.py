@@ -25,7 +25,7 @@ Both generate queries and K/V with the counter-based generator of
 import torch
 
 from . import api
-from .scheduler import Request, Scheduler
+from .scheduler import Request, Scheduler, StaticScheduler
 from .workloads import SYS_VID_BASE, token_values, trace_requests
 
 
@@ -44,7 +44,7 @@ class TraceRunner:
     def __init__(self, device, num_blocks=8192, block_size=16, n_q_heads=32, n_kv_heads=8,
                  head_dim=128, token_budget=4096, max_chunk=512, trace=None, seed=1004,
                  n_steps=300, dtype=torch.bfloat16, preempt="recompute", num_host_blocks=0,
-                 prefix_cache=False):
+                 prefix_cache=False, max_seqs=None, static_batch=None):
         self.device = torch.device(device)
         self.Hq, self.Hkv, self.d, self.bs = n_q_heads, n_kv_heads, head_dim, block_size
         self.dtype = dtype
@@ -57,8 +57,10 @@ class TraceRunner:
         if preempt == "swap":
             self.bm.set_host_blocks(num_host_blocks)
             self.host = api.host_pool_create(num_host_blocks, self.pool)
-        self.sched = Scheduler(self.bm, token_budget, max_chunk, preempt=preempt,
-                               prefix_cache=prefix_cache)
+        kw = dict(token_budget=token_budget, max_chunk=max_chunk, preempt=preempt,
+                  prefix_cache=prefix_cache, max_seqs=max_seqs)
+        self.sched = (StaticScheduler(self.bm, static_batch, **kw) if static_batch
+                      else Scheduler(self.bm, **kw))
         trace = trace if trace is not None else trace_requests(n_steps=n_steps, seed=seed)
         # (arrival, prompt, output) or (arrival, prompt, output, group, system prompt length)
         self.pending = [Request(i, *t[:3], group=t[3], sys_len=t[4]) if len(t) == 5 else Request(i, *t)
@@ -168,6 +170,13 @@ class TraceRunner:
         for to_host, pairs in swaps:
             if pairs.shape[0]:
                 api.swap_blocks(pairs, to_host=to_host, host_pool=self.host, pool=self.pool)
+
+    def step_ms(self):
+        """GPU ms of every scheduler step so far (0 for steps with no work)."""
+        ms = [0.0] * self.sched.step_no
+        for r in self.records:
+            ms[r.step] = r.gpu_ms or 0.0
+        return ms
 
     def run(self, max_steps=None, on_step=None):
         limit = max_steps if max_steps is not None else self.n_steps

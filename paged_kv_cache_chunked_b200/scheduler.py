@@ -119,7 +119,8 @@ class StepPlan:
 
 
 class Scheduler:
-    def __init__(self, bm, token_budget=4096, max_chunk=512, preempt="recompute", prefix_cache=False):
+    def __init__(self, bm, token_budget=4096, max_chunk=512, preempt="recompute", prefix_cache=False,
+                 max_seqs=None):
         if preempt not in ("recompute", "swap"):
             raise ValueError("preempt must be 'recompute' or 'swap'")
         self.bm = bm
@@ -128,6 +129,7 @@ class Scheduler:
         self.max_chunk = max_chunk
         self.preempt_mode = preempt
         self.prefix_cache = prefix_cache
+        self.max_seqs = max_seqs     # cap on requests holding blocks at once ("slots"); None: memory only
         self.waiting = []    # arrival order
         self.running = []    # arrival order; hold blocks
         self.swapped = []    # arrival order; blocks in the host pool
@@ -178,6 +180,10 @@ class Scheduler:
         self.metrics["preemptions"] += 1
         self.running.remove(req)
         self._requeue(req)
+
+    def _may_admit(self, req):
+        """Continuous batching: any waiting request may join at any step."""
+        return True
 
     def _prefix_keys(self, req):
         """Cache keys of the request's blocks that lie wholly inside its system
@@ -250,11 +256,13 @@ class Scheduler:
         candidates = [r for r in sorted(self.running, key=lambda r: (r.arrival, r.rid))
                       if r.prefilling and r not in batch]
         if not self.swapped:     # nothing new is admitted while a request is swapped out
-            candidates += [r for r in self.waiting if r not in preempted]
+            candidates += [r for r in self.waiting if r not in preempted and self._may_admit(r)]
         for req in candidates:
             if budget == 0:
                 break
             if req.seq < 0:
+                if self.max_seqs is not None and len(self.running) >= self.max_seqs:
+                    break        # every slot is taken
                 # admission: reason in blocks before taking any (after the
                 # prefix-cache hit, whose blocks are already in the pool)
                 keys = self._prefix_keys(req)
@@ -323,11 +331,47 @@ class Scheduler:
                 "alloc_failures": self.metrics["alloc_failures"]}
 
 
-def summary(finished):
+class StaticScheduler(Scheduler):
+    """Static batching, the comparison the pages draw ["Batching and
+    PagedAttention", "Static batching": requests are grouped into a batch that
+    runs until every member has finished, then the next batch starts; slots
+    of finished members sit idle, new arrivals wait for the whole batch].
+
+    Only admission differs from Scheduler: when no request runs and no batch
+    is open, the next batch_size waiting requests (arrival order) become the
+    batch; only its members are admitted (their prefill chunks still follow
+    the token cap), and the batch closes when all of them have finished.
+    Preempted members stay members."""
+
+    def __init__(self, bm, batch_size, **kw):
+        super().__init__(bm, **kw)
+        self.batch_size = batch_size
+        self.batch = set()       # request ids of the open batch
+        self.batches = 0
+
+    def _plan(self):
+        if not self.batch and not self.running and not self.swapped and self.waiting:
+            self.batch = {r.rid for r in self.waiting[:self.batch_size]}
+            self.batches += 1
+        return super()._plan()
+
+    def _may_admit(self, req):
+        return req.rid in self.batch
+
+    def complete(self, plan):
+        super().complete(plan)
+        self.batch -= {r.rid for r in plan.requests if r.finish_step == plan.step}
+
+
+def summary(finished, step_ms=None):
     """Per-request serving metrics over finished requests, in scheduler steps
     [7.8 PagedAttention & continuous batching, "01 Concept": queue delay, time
     to first token, inter-token latency], split by request class (prompt
-    shorter or longer than 512 tokens) so throughput does not hide starvation."""
+    shorter or longer than 512 tokens) so throughput does not hide starvation.
+    With step_ms (GPU ms of each step), time to first token and inter-token
+    latency are also given in ms of GPU time: a request arriving at step a
+    whose first token comes at step f waits from the start of a to the end of
+    f."""
     def stats(xs):
         if not xs:
             return None
@@ -347,6 +391,16 @@ def summary(finished):
                      "ttft": stats([r.first_token_step - r.arrival for r in rs]),
                      "itl": stats(itl),
                      "preempted": sum(1 for r in rs if r.preemptions)}
+        if step_ms is not None:
+            end = [0.0]
+            for m in step_ms:
+                end.append(end[-1] + m)          # end[s + 1]: GPU ms at the end of step s
+            at = lambda s: end[min(s, len(end) - 1)]
+            itl_ms = []
+            for r in rs:
+                itl_ms += [at(b + 1) - at(a + 1) for a, b in zip(r.token_steps, r.token_steps[1:])]
+            out[name]["ttft_ms"] = stats([at(r.first_token_step + 1) - at(r.arrival) for r in rs])
+            out[name]["itl_ms"] = stats(itl_ms)
     return out
 
 

@@ -266,3 +266,81 @@ def test_prefix_cache_skips_exactly_the_shared_tokens_and_drains():
         assert sum(written.values()) == tokens(sched) - hit
     st = bm.stats()
     assert st["free_blocks"] == 600 and st["cached_blocks"] == 0 and st["prefix_hits"] * 16 == hit
+
+
+# ---------------------------------------------------------------- static batching
+from paged_kv_cache_chunked_b200.scheduler import StaticScheduler  # noqa: E402
+
+
+def _run_policy(sched, reqs, limit=5000):
+    pending = sorted(reqs, key=lambda r: (r.arrival, r.rid))
+    step = 0
+    plans = []
+    while pending or sched.has_work():
+        while pending and pending[0].arrival <= step:
+            sched.add_request(pending.pop(0))
+        plan = sched.schedule()
+        plans.append((plan, set(getattr(sched, "batch", set()))))
+        sched.complete(plan)
+        step += 1
+        assert step < limit, "did not drain"
+    return plans
+
+
+def test_static_batching_runs_each_batch_to_its_end():
+    # "a batch that runs until every member has finished, then the next batch
+    # starts" [Batching and PagedAttention, "Static batching"]
+    reqs = [Request(i, a, p, o) for i, (a, p, o) in enumerate(_small_trace())]
+    sched = StaticScheduler(BlockManager(600, 16), batch_size=8, token_budget=4096, max_chunk=512)
+    plans = _run_policy(sched, reqs)
+    batches = []
+    for plan, batch in plans:
+        assert len(batch) <= 8
+        assert {r.rid for r in plan.requests} <= batch
+        if batch and (not batches or batch - batches[-1]):
+            batches.append(set(batch))
+    for a, b in zip(batches, batches[1:]):
+        assert not (a & b)                              # a new batch only after the old one ended
+    assert len(sched.finished) == len(reqs) and sched.batches == len(batches)
+
+
+def _toy(lengths, prompt=16):
+    return [Request(i, 0, prompt, o) for i, o in enumerate(lengths)]
+
+
+def test_continuous_batching_finishes_mixed_lengths_sooner():
+    # [Batching and PagedAttention, "Try it" 1]: 4 slots, mixed output lengths;
+    # the average request finishes sooner with continuous batching
+    lengths = [10, 500, 30, 200, 20, 300, 50, 100, 10, 400, 60, 15]
+    cont = Scheduler(BlockManager(4096, 16), token_budget=4096, max_chunk=512, max_seqs=4)
+    stat = StaticScheduler(BlockManager(4096, 16), batch_size=4, token_budget=4096, max_chunk=512)
+    _run_policy(cont, _toy(lengths))
+    _run_policy(stat, _toy(lengths))
+    mean = lambda s: sum(r.finish_step for r in s.finished) / len(s.finished)
+    assert mean(cont) < 0.8 * mean(stat)
+    assert max(r.finish_step for r in cont.finished) <= max(r.finish_step for r in stat.finished)
+
+
+def test_equal_lengths_make_static_and_continuous_batching_alike():
+    # [Batching and PagedAttention, "Try it" 2]: with similar lengths continuous
+    # batching barely helps; with equal ones every request finishes at the same
+    # step under both policies
+    lengths = [40] * 12
+    cont = Scheduler(BlockManager(4096, 16), token_budget=4096, max_chunk=512, max_seqs=4)
+    stat = StaticScheduler(BlockManager(4096, 16), batch_size=4, token_budget=4096, max_chunk=512)
+    _run_policy(cont, _toy(lengths))
+    _run_policy(stat, _toy(lengths))
+    fin = lambda s: sorted((r.rid, r.finish_step) for r in s.finished)
+    assert fin(cont) == fin(stat)
+
+
+def test_summary_converts_steps_to_gpu_time():
+    # a request arriving at step 0 with tokens at steps 2, 3 and 5, steps of
+    # 1..6 ms: first token at the end of step 2 (1+2+3 = 6 ms), gaps of 4 ms
+    # (step 3) and 5 + 6 = 11 ms (steps 4 and 5)
+    from paged_kv_cache_chunked_b200.scheduler import summary
+    r = Request(0, 0, 100, 3)
+    r.admit_step, r.first_token_step, r.token_steps = 0, 2, [2, 3, 5]
+    out = summary([r], step_ms=[1.0, 2.0, 3.0, 4.0, 5.0, 6.0])["all"]
+    assert out["ttft_ms"]["mean"] == 6.0
+    assert out["itl_ms"]["mean"] == 7.5 and out["ttft"]["mean"] == 2 and out["itl"]["mean"] == 1.5
