@@ -51,7 +51,7 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="decode64_bf16",
                    choices=["decode64_bf16", "longdoc_bf16", "chunk512_bf16", "trace", "trace_swap",
-                            "trace_prefix", "trace_prefix_nocache", "policy", "fork",
+                            "trace_prefix", "trace_prefix_nocache", "trace_hybrid", "policy", "fork",
                             "fork1028", "append_copy"])
     p.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
     p.add_argument("--no-e2e", action="store_true")
@@ -664,11 +664,16 @@ def run_serving(args, rank, world, device):
         # 512, 2,048 or 256 tokens) whose blocks are shared through the prefix
         # cache; trace_prefix_nocache runs the same trace without the cache.
         from paged_kv_cache_chunked_b200.workloads import prefix_trace_requests
+        # trace_hybrid: the same memory as trace's 8,192 blocks split into two
+        # pools, 64 per-sequence state slots of 32 blocks' worth each and 6,144
+        # KV blocks (a hybrid model's fixed-size state beside its paged KV)
         swap = args.workload == "trace_swap"
         prefix = args.workload.startswith("trace_prefix")
+        hybrid = args.workload == "trace_hybrid"
         r = TraceRunner(device, preempt="swap" if swap else "recompute", num_host_blocks=8192 if swap else 0,
                         trace=prefix_trace_requests() if prefix else None,
-                        prefix_cache=args.workload == "trace_prefix")
+                        prefix_cache=args.workload == "trace_prefix",
+                        num_blocks=6144 if hybrid else 8192, state_slots=64 if hybrid else 0)
         while r.sched.step_no < 300 and (r.pending or r.sched.has_work()):
             rec = r.step()
             if rec is not None:
@@ -676,11 +681,14 @@ def run_serving(args, rank, world, device):
         skip = min(args.warmup, len(recs) // 2)
         recs = recs[skip:]
         cfg = {"workload": args.workload, "steps_run": len(recs) + skip, "warmup_steps": skip,
-               "num_blocks": 8192, "block_size": 16, "n_q_heads": 32, "n_kv_heads": 8,
+               "num_blocks": r.bm.num_blocks, "block_size": 16, "n_q_heads": 32, "n_kv_heads": 8,
                "head_dim": 128, "token_budget": 4096, "max_chunk": 512,
                "preempt": r.sched.preempt_mode,
                "preemptions": r.sched.metrics["preemptions"], "rejected": r.rejected,
                "finished": len(r.sched.finished)}
+        if hybrid:
+            cfg.update(state_slots=64, state_slot_blocks_worth=32,
+                       max_running=max(x.num_seqs for x in recs))
         if prefix:
             st = r.bm.stats()
             cfg.update(trace="prefix_trace_requests(seed 1007): system prompts 1024/512/2048/256, user "

@@ -235,11 +235,14 @@ typedef struct {
     int64_t prefix_lookups;   /* keys offered to pk_bm_add_seq_cached */
     int64_t prefix_hits;      /* of which served by a cached block */
     int64_t cached_blocks;    /* blocks registered in the prefix cache now */
+    int64_t state_slots;      /* per-sequence state pool size, 0 without one */
+    int64_t state_free_slots;
 } pk_bm_stats;
 
 int pk_bm_create(int num_blocks, int block_size, pk_bm **out);
 int pk_bm_destroy(pk_bm *bm);
-/* New empty sequence; its id in *seq_out. */
+/* New empty sequence; its id in *seq_out (PK_ERR_OOM: no free state slot,
+ * with a state pool). */
 int pk_bm_add_seq(pk_bm *bm, int64_t *seq_out);
 /* Reserve slots for the next n tokens of seq.  slots_out[n] receives the slot
  * id of each token.  If the sequence's last block is partly filled and shared
@@ -296,6 +299,17 @@ int pk_bm_is_swapped(const pk_bm *bm, int64_t seq, int *swapped_out);
 int pk_bm_cache_blocks(pk_bm *bm, int64_t seq, const uint64_t *keys, int n_keys);
 int pk_bm_cached_prefix(const pk_bm *bm, const uint64_t *keys, int n_keys, int *n_hit_out);
 int pk_bm_add_seq_cached(pk_bm *bm, const uint64_t *keys, int n_keys, int64_t *seq_out, int *n_hit_out);
+/* Two pools [DD: a hybrid model's attention layers keep growing, paged KV,
+ * its other layers a fixed-size state per sequence; the server manages two
+ * pools with different lifecycles].  pk_bm_set_state_slots (once, before any
+ * sequence exists) adds a pool of num_slots state slots: every sequence takes
+ * one when it is created (add_seq, add_seq_cached, fork) and returns it when
+ * freed; with no free slot those calls return PK_ERR_OOM and change nothing.
+ * A fork's slot is new: the caller copies the parent's state into it.  A
+ * swapped-out sequence keeps its slot.  pk_bm_state_slot gives a sequence's
+ * slot (-1 without a state pool). */
+int pk_bm_set_state_slots(pk_bm *bm, int num_slots);
+int pk_bm_state_slot(const pk_bm *bm, int64_t seq, int *slot_out);
 /* Copy seq's block table (ceil(len / bs) ids) into out[cap]; *n_out = count. */
 int pk_bm_block_table(const pk_bm *bm, int64_t seq, int32_t *out, int cap, int *n_out);
 /* Fill out[n_seqs][width] (int32, row-major) with the tables of seqs[], -1 padded. */

@@ -68,6 +68,19 @@ prefix hit rate is one of the metrics to watch]:
   * an entry lives while its block is referenced: when the block's count
     reaches zero it leaves the cache as the block returns to the free list
     (the pages fix no retention of unreferenced blocks).
+
+Two pools [7.8 PagedAttention & continuous batching, "01 Concept": a hybrid
+model's attention layers keep growing, paged KV while its other layers keep a
+fixed-size state per sequence, so the server manages two pools with different
+lifecycles]:
+  * an optional pool of state slots with its own free list (first in, first
+    out from 0, 1, ..., S-1): every sequence takes one slot when it is
+    created (add_seq, add_seq_cached, fork) and keeps it until it is freed,
+    whatever its length; KV blocks keep their on-demand lifecycle;
+  * admission accounts for both pools: creating a sequence with no free slot
+    fails (OracleOOM) and changes nothing; a fork's slot starts as a copy of
+    the parent's state, which the caller makes;
+  * a swapped-out sequence keeps its slot (only KV blocks move).
 """
 
 from collections import deque
@@ -98,14 +111,31 @@ class OracleBlockManager:
         self.key_of = {}                    # physical block -> key it is cached under
         self.prefix_lookups = 0
         self.prefix_hits = 0
+        self.state_slots = 0
+        self.state_free = deque()
+        self.state_of = {}                  # seq id -> state slot
 
     # -- sequences -----------------------------------------------------
     def add_seq(self):
+        if self.state_slots and not self.state_free:
+            raise OracleOOM("no free state slot")
         sid = self.next_seq
         self.next_seq += 1
         self.tables[sid] = []
         self.lengths[sid] = 0
+        if self.state_slots:
+            self.state_of[sid] = self.state_free.popleft()
         return sid
+
+    def set_state_slots(self, n):
+        """Give every sequence a fixed-size state slot from a pool of n (once)."""
+        if n < 0 or self.state_slots or self.tables:
+            raise ValueError("state pool already set, negative, or sequences exist")
+        self.state_slots = n
+        self.state_free = deque(range(n))
+
+    def state_slot(self, seq):
+        return self.state_of.get(seq, -1)
 
     def _take(self):
         block = self.free_list.popleft()
@@ -173,10 +203,14 @@ class OracleBlockManager:
     def fork(self, parent):
         """New sequence sharing every block of parent (reference counts +1)."""
         self._resident(parent)
+        if self.state_slots and not self.state_free:
+            raise OracleOOM("no free state slot")
         child = self.next_seq
         self.next_seq += 1
         self.tables[child] = list(self.tables[parent])
         self.lengths[child] = self.lengths[parent]
+        if self.state_slots:
+            self.state_of[child] = self.state_free.popleft()
         for block in self.tables[child]:
             self.refcount[block] += 1
         return child
@@ -186,6 +220,8 @@ class OracleBlockManager:
         (a swapped sequence returns its host blocks)."""
         table = self.tables.pop(seq)
         del self.lengths[seq]
+        if seq in self.state_of:
+            self.state_free.append(self.state_of.pop(seq))
         if seq in self.swapped:
             self.swapped.discard(seq)
             for h in reversed(table):
@@ -314,4 +350,6 @@ class OracleBlockManager:
             "prefix_lookups": self.prefix_lookups,
             "prefix_hits": self.prefix_hits,
             "cached_blocks": len(self.cache),
+            "state_slots": self.state_slots,
+            "state_free_slots": len(self.state_free),
         }

@@ -34,7 +34,8 @@ class BmStats(ctypes.Structure):
                 ("tail_waste_slots", ctypes.c_int64), ("num_seqs", ctypes.c_int64),
                 ("host_blocks", ctypes.c_int64), ("host_free_blocks", ctypes.c_int64),
                 ("prefix_lookups", ctypes.c_int64), ("prefix_hits", ctypes.c_int64),
-                ("cached_blocks", ctypes.c_int64)]
+                ("cached_blocks", ctypes.c_int64), ("state_slots", ctypes.c_int64),
+                ("state_free_slots", ctypes.c_int64)]
 
 
 _lib = None
@@ -75,6 +76,8 @@ SIGNATURES = {
     "pk_bm_cache_blocks": ([_P, _I64, _P, _I], _I),
     "pk_bm_cached_prefix": ([_P, _P, _I, _PI], _I),
     "pk_bm_add_seq_cached": ([_P, _P, _I, ctypes.POINTER(ctypes.c_int64), _PI], _I),
+    "pk_bm_set_state_slots": ([_P, _I], _I),
+    "pk_bm_state_slot": ([_P, _I64, _PI], _I),
     "pk_bm_get_stats": ([_P, ctypes.POINTER(BmStats)], _I),
 }
 

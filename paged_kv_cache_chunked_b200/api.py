@@ -283,6 +283,15 @@ class BlockManager:
                                          ctypes.byref(n)))
         return s.value, n.value
 
+    def set_state_slots(self, num_slots):
+        """Add a pool of fixed-size per-sequence state slots (two-pool manager)."""
+        check(lib().pk_bm_set_state_slots(self._h, num_slots))
+
+    def state_slot(self, seq):
+        r = ctypes.c_int()
+        check(lib().pk_bm_state_slot(self._h, seq, ctypes.byref(r)))
+        return r.value
+
     def is_swapped(self, seq):
         r = ctypes.c_int()
         check(lib().pk_bm_is_swapped(self._h, seq, ctypes.byref(r)))

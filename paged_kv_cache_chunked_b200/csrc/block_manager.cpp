@@ -39,6 +39,15 @@
 // lookup, every block taken a hit); an entry lives while its block is
 // referenced and leaves the cache when the block returns to the free list.
 //
+// Two pools ["7.8 PagedAttention & continuous batching", "01 Concept": a
+// hybrid model's attention layers keep growing, paged KV while its other
+// layers keep a fixed-size per-sequence state, so the server manages two pools
+// with different lifecycles]: an optional pool of state slots (FIFO free list);
+// every sequence takes a slot when created (add_seq, add_seq_cached, fork; a
+// fork's slot is the caller's copy of the parent's state) and returns it when
+// freed; creating a sequence with no free slot fails and changes nothing; a
+// swapped-out sequence keeps its slot.
+//
 // Policy details the pages leave open, fixed so that tables are reproducible:
 // FIFO free list starting as 0..N-1 (a released block joins the tail);
 // a sequence's blocks are released from its last logical block to its first;
@@ -66,7 +75,10 @@ struct pk_bm {
         std::vector<int32_t> table;
         int64_t len = 0;
         bool swapped = false;  // table names host blocks
+        int32_t state_slot = -1;
     };
+    int num_state_slots = 0;
+    std::deque<int32_t> state_free;
     int num_host_blocks = 0;
     std::deque<int32_t> host_free;
     std::vector<int32_t> host_filled;
@@ -150,11 +162,44 @@ int pk_bm_destroy(pk_bm *bm) {
     return PK_OK;
 }
 
+namespace {
+// a state slot for a new sequence (-1 without a state pool); false: none free
+bool take_state_slot(pk_bm *bm, int32_t *slot) {
+    *slot = -1;
+    if (bm->num_state_slots == 0) return true;
+    if (bm->state_free.empty()) return false;
+    *slot = bm->state_free.front();
+    bm->state_free.pop_front();
+    return true;
+}
+}  // namespace
+
 int pk_bm_add_seq(pk_bm *bm, int64_t *seq_out) {
     if (!bm || !seq_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    int32_t slot;
+    if (!take_state_slot(bm, &slot)) return fail(PK_ERR_OOM, "no free state slot");
     const int64_t id = bm->next_seq++;
-    bm->seqs.emplace(id, pk_bm::Seq());
+    pk_bm::Seq s;
+    s.state_slot = slot;
+    bm->seqs.emplace(id, std::move(s));
     *seq_out = id;
+    return PK_OK;
+}
+
+int pk_bm_set_state_slots(pk_bm *bm, int num_slots) {
+    if (!bm) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    if (num_slots < 0 || bm->num_state_slots != 0 || !bm->seqs.empty())
+        return fail(PK_ERR_INVALID_ARG, "state pool already set, negative, or sequences exist");
+    bm->num_state_slots = num_slots;
+    for (int32_t i = 0; i < num_slots; ++i) bm->state_free.push_back(i);
+    return PK_OK;
+}
+
+int pk_bm_state_slot(const pk_bm *bm, int64_t seq, int *slot_out) {
+    if (!bm || !slot_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    auto it = bm->seqs.find(seq);
+    if (it == bm->seqs.end()) return fail(PK_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq);
+    *slot_out = it->second.state_slot;
     return PK_OK;
 }
 
@@ -211,7 +256,10 @@ int pk_bm_fork(pk_bm *bm, int64_t parent, int64_t *child_out) {
     if (!bm || !child_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
     const pk_bm::Seq *ps = resident(bm, parent);
     if (!ps) return PK_ERR_INVALID_ARG;
+    int32_t slot;
+    if (!take_state_slot(bm, &slot)) return fail(PK_ERR_OOM, "no free state slot");
     pk_bm::Seq child = *ps;  // copy before emplace can rehash
+    child.state_slot = slot;
     for (int32_t b : child.table) ++bm->refcount[b];
     const int64_t id = bm->next_seq++;
     bm->seqs.emplace(id, std::move(child));
@@ -224,6 +272,7 @@ int pk_bm_free(pk_bm *bm, int64_t seq) {
     auto it = bm->seqs.find(seq);
     if (it == bm->seqs.end()) return fail(PK_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq);
     const std::vector<int32_t> &t = it->second.table;
+    if (it->second.state_slot >= 0) bm->state_free.push_back(it->second.state_slot);
     if (it->second.swapped) {  // its host blocks return to the host pool
         for (auto h = t.rbegin(); h != t.rend(); ++h) {
             bm->host_filled[*h] = 0;
@@ -328,8 +377,11 @@ int pk_bm_cached_prefix(const pk_bm *bm, const uint64_t *keys, int n_keys, int *
 int pk_bm_add_seq_cached(pk_bm *bm, const uint64_t *keys, int n_keys, int64_t *seq_out, int *n_hit_out) {
     if (!bm || !seq_out || !n_hit_out || (n_keys > 0 && !keys) || n_keys < 0)
         return fail(PK_ERR_INVALID_ARG, "bad argument");
+    int32_t slot;
+    if (!take_state_slot(bm, &slot)) return fail(PK_ERR_OOM, "no free state slot");
     const int64_t id = bm->next_seq++;
     pk_bm::Seq s;
+    s.state_slot = slot;
     const int hits = bm->cached_prefix(keys, n_keys);
     for (int i = 0; i < hits; ++i) {
         const int32_t b = bm->cache.at(keys[i]);
@@ -413,6 +465,8 @@ int pk_bm_get_stats(const pk_bm *bm, pk_bm_stats *out) {
     out->prefix_lookups = bm->prefix_lookups;
     out->prefix_hits = bm->prefix_hits;
     out->cached_blocks = (int64_t)bm->cache.size();
+    out->state_slots = bm->num_state_slots;
+    out->state_free_slots = (int64_t)bm->state_free.size();
     return PK_OK;
 }
 

@@ -44,7 +44,7 @@ class TraceRunner:
     def __init__(self, device, num_blocks=8192, block_size=16, n_q_heads=32, n_kv_heads=8,
                  head_dim=128, token_budget=4096, max_chunk=512, trace=None, seed=1004,
                  n_steps=300, dtype=torch.bfloat16, preempt="recompute", num_host_blocks=0,
-                 prefix_cache=False, max_seqs=None, static_batch=None):
+                 prefix_cache=False, max_seqs=None, static_batch=None, state_slots=0):
         self.device = torch.device(device)
         self.Hq, self.Hkv, self.d, self.bs = n_q_heads, n_kv_heads, head_dim, block_size
         self.dtype = dtype
@@ -53,6 +53,8 @@ class TraceRunner:
         self.pool = api.kv_pool_create(num_blocks, block_size, n_kv_heads, head_dim, dtype,
                                        self.device)
         self.bm = api.BlockManager(num_blocks, block_size)
+        if state_slots:          # two pools: a fixed-size state slot per sequence beside the KV blocks
+            self.bm.set_state_slots(state_slots)
         self.host = None
         if preempt == "swap":
             self.bm.set_host_blocks(num_host_blocks)

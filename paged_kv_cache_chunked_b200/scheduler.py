@@ -55,6 +55,12 @@ the basis of prefix caching].  Readings:
   * a request's system-prompt blocks enter the cache once the step that
     filled them has run.
 
+Two pools: when the block manager also keeps a fixed-size state slot per
+sequence (hybrid models), admission needs a free slot as well as the first
+chunk's blocks; a recomputed request gives its slot back, a swapped one keeps
+it ["7.8 PagedAttention & continuous batching", "01 Concept": two pools with
+different lifecycles].
+
 A request with prompt length P and output length O stores P + O - 1 tokens:
 the last prefill chunk yields the first output token, each decode step
 appends the previous output token and yields the next.
@@ -263,6 +269,9 @@ class Scheduler:
             if req.seq < 0:
                 if self.max_seqs is not None and len(self.running) >= self.max_seqs:
                     break        # every slot is taken
+                st = self.bm.stats()
+                if st.get("state_slots", 0) and st["state_free_slots"] == 0:
+                    break        # two pools: no free per-sequence state slot
                 # admission: reason in blocks before taking any (after the
                 # prefix-cache hit, whose blocks are already in the pool)
                 keys = self._prefix_keys(req)

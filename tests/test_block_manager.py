@@ -18,11 +18,13 @@ def _same_state(bm, ob):
                           "tail_waste_slots": ob.tail_waste(), "num_seqs": len(ob.tables),
                           "host_blocks": ob.host_blocks, "host_free_blocks": len(ob.host_free),
                           "prefix_lookups": ob.prefix_lookups, "prefix_hits": ob.prefix_hits,
-                          "cached_blocks": len(ob.cache)}
+                          "cached_blocks": len(ob.cache), "state_slots": ob.state_slots,
+                          "state_free_slots": len(ob.state_free)}
     for sid in ob.tables:
         assert bm.block_table(sid) == ob.block_table(sid)
         assert bm.length(sid) == ob.length(sid)
         assert bm.is_swapped(sid) == (sid in ob.swapped)
+        assert bm.state_slot(sid) == ob.state_slot(sid)
     for b in range(ob.num_blocks):
         assert bm.refcount(b) == ob.refcount[b]
 
@@ -128,6 +130,55 @@ def test_prefix_cache_script_matches_the_oracle():
         _same_state(bm, ob)
     st = bm.stats()
     assert st["prefix_hits"] == 20 and st["prefix_lookups"] == 5 * 9
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_two_pool_operations_match_the_oracle(seed):
+    # with a pool of state slots, sequence creation and fork fail cleanly when
+    # no slot is free; slots follow sequences in both managers
+    rng = random.Random(300 + seed)
+    bm, ob = BlockManager(48, 8), OracleBlockManager(48, 8)
+    bm.set_state_slots(5)
+    ob.set_state_slots(5)
+    live = []
+    for step in range(300):
+        op = rng.random()
+        if op < 0.25 or not live:
+            try:
+                b = ob.add_seq()
+            except OracleOOM:
+                with pytest.raises(OutOfBlocks):
+                    bm.add_seq()
+                continue
+            assert bm.add_seq() == b
+            live.append(b)
+        elif op < 0.4:
+            p = rng.choice(live)
+            try:
+                b = ob.fork(p)
+            except OracleOOM:
+                with pytest.raises(OutOfBlocks):
+                    bm.fork(p)
+                continue
+            assert bm.fork(p) == b
+            live.append(b)
+        elif op < 0.6:
+            s_ = rng.choice(live)
+            live.remove(s_)
+            bm.free(s_)
+            ob.free(s_)
+        else:
+            s_ = rng.choice(live)
+            n = rng.randint(0, 20)
+            try:
+                ref = ob.append_slots(s_, n)
+            except OracleOOM:
+                with pytest.raises(OutOfBlocks):
+                    bm.append_slots(s_, n)
+            else:
+                assert bm.append_slots(s_, n) == (ref[0], ref[1])
+        _same_state(bm, ob)
+        assert len(live) <= 5
 
 
 def test_page_toy_capacity_through_the_product_manager():

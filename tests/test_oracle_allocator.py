@@ -367,3 +367,60 @@ def test_random_operations_with_prefix_cache_keep_invariants(seed):
     for s, _ in live:
         bm.free(s)
     assert bm.num_free() == 60 and bm.stats()["cached_blocks"] == 0
+
+
+# ---------------------------------------------------------------- two pools
+def test_two_pools_hold_the_pages_ten_long_document_sessions():
+    # [7.8 PagedAttention & continuous batching, "01 Concept"]: 32,768-token
+    # sessions at 64 KiB of KV per token (2,048 one-MiB blocks of 16 tokens)
+    # plus a 144 MiB per-sequence state, in a 23,859 MiB pool: ten sessions.
+    # Split as ten state slots and the rest in KV blocks, all ten fit and grow
+    # to full length, and an eleventh finds no state slot; with eleven slots
+    # the KV pool is too small for eleven full sessions.
+    gold = capacity.sessions_in_pool(23_859, 32_768, 64 / 1024, 144)
+    assert gold == 10
+    bm = OracleBlockManager(23_859 - 10 * 144, 16)
+    bm.set_state_slots(10)
+    seqs = [bm.add_seq() for _ in range(10)]
+    for s in seqs:
+        bm.append_slots(s, 32_768)
+    assert sorted(bm.state_slot(s) for s in seqs) == list(range(10))
+    with pytest.raises(OracleOOM):
+        bm.add_seq()
+    assert bm.stats()["num_seqs"] == 10
+    bm11 = OracleBlockManager(23_859 - 11 * 144, 16)
+    bm11.set_state_slots(11)
+    grown = 0
+    for _ in range(11):
+        s = bm11.add_seq()
+        try:
+            bm11.append_slots(s, 32_768)
+            grown += 1
+        except OracleOOM:
+            pass
+    assert grown == 10
+
+
+def test_state_slots_follow_sequence_lifetimes():
+    bm = OracleBlockManager(16, 4)
+    bm.set_state_slots(3)
+    a = bm.add_seq()
+    bm.append_slots(a, 9)
+    c = bm.fork(a)                                  # a fork takes its own slot
+    assert bm.state_slot(a) != bm.state_slot(c)
+    b, _ = bm.add_seq_cached([])
+    assert bm.stats()["state_free_slots"] == 0
+    before = (list(bm.free_list), dict(bm.tables), bm.next_seq)
+    with pytest.raises(OracleOOM):
+        bm.fork(a)
+    with pytest.raises(OracleOOM):
+        bm.add_seq_cached(["k"])
+    assert (list(bm.free_list), dict(bm.tables), bm.next_seq) == before
+    assert bm.stats()["prefix_lookups"] == 0
+    bm.free(a)                                      # the slot returns, whatever the length
+    d = bm.add_seq()
+    assert bm.state_slot(d) == 0 and bm.stats()["state_free_slots"] == 0
+    bm.set_host_blocks(8)
+    bm.append_slots(b, 4)
+    bm.swap_out(b)                                  # a swapped sequence keeps its slot
+    assert bm.state_slot(b) >= 0 and bm.stats()["state_free_slots"] == 0

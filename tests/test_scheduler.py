@@ -344,3 +344,20 @@ def test_summary_converts_steps_to_gpu_time():
     out = summary([r], step_ms=[1.0, 2.0, 3.0, 4.0, 5.0, 6.0])["all"]
     assert out["ttft_ms"]["mean"] == 6.0
     assert out["itl_ms"]["mean"] == 7.5 and out["ttft"]["mean"] == 2 and out["itl"]["mean"] == 1.5
+
+
+# ---------------------------------------------------------------- two pools
+def test_two_pool_admission_caps_concurrency_at_the_state_slots():
+    # [7.8 PagedAttention & continuous batching, "01 Concept"]: with a
+    # fixed-size state slot per sequence beside the KV blocks, no more
+    # requests run than there are slots; both managers plan identically
+    def run(bm):
+        bm.set_state_slots(6)
+        sched, plans = _run(bm, _small_trace(), 40)
+        return sched, plans
+    s1, p1 = run(BlockManager(600, 16))
+    s2, p2 = run(OracleAdapter(600, 16))
+    assert [[r.rid for r in a.requests] for a in p1] == [[r.rid for r in b.requests] for b in p2]
+    assert max(len(p.requests) for p in p1) == 6
+    assert len(s1.finished) == len(_small_trace())
+    assert s1.bm.stats()["state_free_slots"] == 6
