@@ -136,6 +136,8 @@ class Scheduler:
         self.preempt_mode = preempt
         self.prefix_cache = prefix_cache
         self.max_seqs = max_seqs     # cap on requests holding blocks at once ("slots"); None: memory only
+        # two pools: the manager's state-slot pool, if it has one (set before the scheduler is made)
+        self._state_pool = bool(bm.stats().get("state_slots", 0))
         self.waiting = []    # arrival order
         self.running = []    # arrival order; hold blocks
         self.swapped = []    # arrival order; blocks in the host pool
@@ -269,8 +271,7 @@ class Scheduler:
             if req.seq < 0:
                 if self.max_seqs is not None and len(self.running) >= self.max_seqs:
                     break        # every slot is taken
-                st = self.bm.stats()
-                if st.get("state_slots", 0) and st["state_free_slots"] == 0:
+                if self._state_pool and self.bm.stats()["state_free_slots"] == 0:
                     break        # two pools: no free per-sequence state slot
                 # admission: reason in blocks before taking any (after the
                 # prefix-cache hit, whose blocks are already in the pool)
