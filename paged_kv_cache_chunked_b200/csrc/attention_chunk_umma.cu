@@ -321,51 +321,44 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                     ok = false;
                     break;
                 }
-                int ys[kUBlk];
-#pragma unroll
-                for (int jb = 0; jb < kUBlk; ++jb) {
-                    const int k0 = j * kUKeys + jb * kTile;
-                    ys[jb] = -1;
-                    if (k0 < it.c) {  // warp-uniform
-                        const int blk = k0 / bs;
-                        while (blk >= base + 32) {
-                            base += 32;
-                            cur = nxt;
-                            nxt = base + 32 + lane < nblk ? __ldg(table + base + 32 + lane) : 0;
-                        }
-                        int phys = __shfl_sync(0xffffffffu, cur, blk - base);
-                        if (phys < 0 || phys >= prm.num_blocks) {
-                            if (lane == 0) record_error(prm.err, PK_ERR_BAD_INDEX);
-                            phys = 0;
-                        }
-                        ys[jb] = (phys * Hkv + it.kvh) * bs + k0 % bs;
-                    }
+                // lane jb (< 8) looks up 16-key block jb of the stage: one division
+                // per lane, all lanes at once.  The table window advances once a
+                // stage, to the stage's first block; a stage spans at most 8 blocks,
+                // so all of them lie in cur (base..) or nxt (base + 32..)
+                const int blk0 = j * kUKeys / bs;  // warp-uniform
+                while (blk0 >= base + 32) {
+                    base += 32;
+                    cur = nxt;
+                    nxt = base + 32 + lane < nblk ? __ldg(table + base + 32 + lane) : 0;
                 }
+                const int k0 = j * kUKeys + lane * kTile;
+                const bool has = lane < kUBlk && k0 < it.c;
+                const int blk = has ? k0 / bs : blk0;
+                const int idx = blk - base;        // 0 .. 39
+                const int pa = __shfl_sync(0xffffffffu, cur, idx & 31);
+                const int pb = __shfl_sync(0xffffffffu, nxt, idx & 31);
+                int phys = idx < 32 ? pa : pb;
+                if (has && (phys < 0 || phys >= prm.num_blocks)) {
+                    record_error(prm.err, PK_ERR_BAD_INDEX);
+                    phys = 0;
+                }
+                const int y = (phys * Hkv + it.kvh) * bs + (k0 - blk * bs);
+                const uint32_t nload = (uint32_t)__popc(__ballot_sync(0xffffffffu, has));
                 const int valid_keys = it.c - j * kUKeys;  // warp-uniform
                 const bool tail = is_v && valid_keys < kUKeys;
                 uint8_t *dst = is_v ? sm + kUOffV + (size_t)s * kUVBytes
                                     : sm + kUOffK + (size_t)s * kUKBytes + p * kUKPanel;
                 uint64_t *bar = tail ? v_tma : &full[s];
                 if (lane == 0) {
-                    uint32_t bytes = 0;
-#pragma unroll
-                    for (int jb = 0; jb < kUBlk; ++jb)
-                        if (ys[jb] >= 0) bytes += is_v ? 4096u : 2048u;
-                    if (bytes == 0) mbar_arrive(bar);  // keys past the context: nothing to load
-                    else mbar_arrive_expect_tx(bar, bytes);
+                    if (nload == 0) mbar_arrive(bar);  // keys past the context: nothing to load
+                    else mbar_arrive_expect_tx(bar, nload * (is_v ? 4096u : 2048u));
                 }
                 __syncwarp();
-                {
-                    // lane jb issues block jb's box: a warp's TMA instructions issue one
-                    // at a time, so eight lanes start a stage's boxes together
-                    int my = -1;
-#pragma unroll
-                    for (int jb = 0; jb < kUBlk; ++jb)
-                        if (lane == jb) my = ys[jb];
-                    if (my >= 0) {
-                        if (is_v) tma_load_3d(dst + lane * 4096, &tmv3, 0, my, 0, bar);
-                        else tma_load_2d(dst + lane * 2048, &tmk2, p * 64, my, bar);
-                    }
+                // lane jb issues block jb's box: a warp's TMA instructions issue one
+                // at a time, so eight lanes start a stage's boxes together
+                if (has) {
+                    if (is_v) tma_load_3d(dst + lane * 4096, &tmv3, 0, y, 0, bar);
+                    else tma_load_2d(dst + lane * 2048, &tmk2, p * 64, y, bar);
                 }
                 __syncwarp();
                 if (tail) {
