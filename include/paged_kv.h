@@ -253,6 +253,13 @@ int pk_bm_add_seq(pk_bm *bm, int64_t *seq_out);
  * changed. */
 int pk_bm_append_slots(pk_bm *bm, int64_t seq, int n, int64_t *slots_out, int32_t *pairs_out,
                        int pairs_cap, int *n_pairs_out);
+/* One token for each of seqs[0..n-1], in order, as append_slots(seq, 1) each:
+ * slots_out[i] its slot, pairs_out (int32 [n][2]) the copy-on-write pairs in
+ * order (*n_pairs_out of them).  Stops, without counting an allocation
+ * failure, at the first sequence whose token needs a block when none is free:
+ * *n_done_out sequences got their token. */
+int pk_bm_append_one_each(pk_bm *bm, const int64_t *seqs, int n, int64_t *slots_out, int32_t *pairs_out,
+                          int *n_pairs_out, int *n_done_out);
 /* Blocks append_slots(seq, n) would take from the free list. */
 int pk_bm_blocks_needed(const pk_bm *bm, int64_t seq, int n, int *needed_out);
 /* New sequence sharing all of parent's blocks (reference counts + 1). */
@@ -317,6 +324,9 @@ int pk_bm_fill_tables(const pk_bm *bm, const int64_t *seqs, int n_seqs, int32_t 
 int pk_bm_seq_len(const pk_bm *bm, int64_t seq, int64_t *len_out);
 int pk_bm_refcount(const pk_bm *bm, int32_t block, int *count_out);
 int pk_bm_get_stats(const pk_bm *bm, pk_bm_stats *out);
+/* Free device blocks now (stats' free_blocks, without the walk over every
+ * block that the tail-waste count needs). */
+int pk_bm_num_free(const pk_bm *bm, int *free_out);
 
 #ifdef __cplusplus
 }

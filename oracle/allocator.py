@@ -200,6 +200,19 @@ class OracleBlockManager:
         self.lengths[seq] = length + n
         return slots, pairs
 
+    def append_one_each(self, seqs):
+        """One token for each of seqs in order, as append_slots(seq, 1), stopping
+        (without an allocation failure) at the first one whose token needs a
+        block while none is free.  Returns (served, slots, pairs)."""
+        slots, pairs = [], []
+        for seq in seqs:
+            if self.blocks_needed(seq, 1) > len(self.free_list):
+                break
+            s, p = self.append_slots(seq, 1)
+            slots += s
+            pairs += p
+        return len(slots), slots, pairs
+
     def fork(self, parent):
         """New sequence sharing every block of parent (reference counts +1)."""
         self._resident(parent)

@@ -79,6 +79,8 @@ SIGNATURES = {
     "pk_bm_set_state_slots": ([_P, _I], _I),
     "pk_bm_state_slot": ([_P, _I64, _PI], _I),
     "pk_bm_get_stats": ([_P, ctypes.POINTER(BmStats)], _I),
+    "pk_bm_num_free": ([_P, _PI], _I),
+    "pk_bm_append_one_each": ([_P, _P, _I, _P, _P, _PI, _PI], _I),
 }
 
 

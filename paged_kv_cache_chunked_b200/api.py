@@ -233,6 +233,20 @@ class BlockManager:
         check(lib().pk_bm_append_slots(self._h, seq, n, slots, pairs, 1, ctypes.byref(npairs)))
         return list(slots[:n]), [(pairs[0], pairs[1])] if npairs.value else []
 
+    def append_one_each(self, seqs):
+        """One token for each seq in order, stopping at the first that needs a
+        block when none is free.  Returns (number served, their slots, the
+        copy-on-write pairs in order)."""
+        n = len(seqs)
+        ids = (ctypes.c_int64 * max(n, 1))(*seqs)
+        slots = (ctypes.c_int64 * max(n, 1))()
+        pairs = (ctypes.c_int32 * max(2 * n, 2))()
+        npairs, done = ctypes.c_int(), ctypes.c_int()
+        check(lib().pk_bm_append_one_each(self._h, ids, n, slots, pairs, ctypes.byref(npairs),
+                                          ctypes.byref(done)))
+        return done.value, list(slots[:done.value]), [(pairs[2 * i], pairs[2 * i + 1])
+                                                      for i in range(npairs.value)]
+
     def fork(self, parent):
         c = ctypes.c_int64()
         check(lib().pk_bm_fork(self._h, parent, ctypes.byref(c)))
@@ -327,7 +341,9 @@ class BlockManager:
         return {name: getattr(s, name) for name, _ in BmStats._fields_}
 
     def num_free(self):
-        return self.stats()["free_blocks"]
+        n = ctypes.c_int()
+        check(lib().pk_bm_num_free(self._h, ctypes.byref(n)))
+        return n.value
 
     def num_used(self):
         return self.stats()["used_blocks"]

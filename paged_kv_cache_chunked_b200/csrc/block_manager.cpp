@@ -252,6 +252,25 @@ int pk_bm_append_slots(pk_bm *bm, int64_t seq, int n, int64_t *slots_out, int32_
     return PK_OK;
 }
 
+int pk_bm_append_one_each(pk_bm *bm, const int64_t *seqs, int n, int64_t *slots_out, int32_t *pairs_out,
+                          int *n_pairs_out, int *n_done_out) {
+    if (!bm || !n_pairs_out || !n_done_out || n < 0 || (n > 0 && (!seqs || !slots_out || !pairs_out)))
+        return fail(PK_ERR_INVALID_ARG, "bad argument");
+    *n_pairs_out = 0;
+    *n_done_out = 0;
+    for (int i = 0; i < n; ++i) {
+        const pk_bm::Seq *sq = resident(bm, seqs[i]);
+        if (!sq) return PK_ERR_INVALID_ARG;
+        if (bm->needed(*sq, 1) > (int64_t)bm->free_list.size()) return PK_OK;  // stop: no block for it
+        int np = 0;
+        const int rc = pk_bm_append_slots(bm, seqs[i], 1, slots_out + i, pairs_out + 2 * *n_pairs_out, 1, &np);
+        if (rc != PK_OK) return rc;
+        *n_pairs_out += np;
+        *n_done_out = i + 1;
+    }
+    return PK_OK;
+}
+
 int pk_bm_fork(pk_bm *bm, int64_t parent, int64_t *child_out) {
     if (!bm || !child_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
     const pk_bm::Seq *ps = resident(bm, parent);
@@ -446,6 +465,12 @@ int pk_bm_refcount(const pk_bm *bm, int32_t block, int *count_out) {
     if (!bm || !count_out || block < 0 || block >= bm->num_blocks)
         return fail(PK_ERR_INVALID_ARG, "bad argument");
     *count_out = bm->refcount[block];
+    return PK_OK;
+}
+
+int pk_bm_num_free(const pk_bm *bm, int *free_out) {
+    if (!bm || !free_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    *free_out = (int)bm->free_list.size();
     return PK_OK;
 }
 

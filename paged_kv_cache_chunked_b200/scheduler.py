@@ -71,7 +71,7 @@ from dataclasses import dataclass, field
 import torch
 
 
-@dataclass
+@dataclass(eq=False)         # a request is itself: identity, not field-wise, equality
 class Request:
     rid: int
     arrival: int
@@ -247,19 +247,31 @@ class Scheduler:
             slots.extend(s)
             pairs.extend(p)
 
-        # decodes first, in arrival order
-        for req in sorted(self.running, key=lambda r: (r.arrival, r.rid)):
-            if req.prefilling or req not in self.running or budget == 0:
-                continue
-            while req in self.running and self.bm.blocks_needed(req.seq, 1) > self.bm.num_free():
-                victim = self._latest_running()
-                self.metrics["alloc_failures"] += 1
-                self._preempt(victim)
-                preempted.append(victim)
-            if req not in self.running:
-                continue
-            reserve(req, 1)
-            budget -= 1
+        # decodes first, in arrival order: one manager call serves them until one
+        # needs a block while none is free; that one preempts the latest arrival
+        # (never a request already served: they all arrived earlier) until it
+        # fits or is itself preempted, and the rest follow
+        decodes = [r for r in sorted(self.running, key=lambda r: (r.arrival, r.rid)) if not r.prefilling]
+        i = 0
+        while i < len(decodes) and budget > 0:
+            todo = decodes[i:i + budget]
+            done, got_slots, got_pairs = self.bm.append_one_each([r.seq for r in todo])
+            for req, slot in zip(todo[:done], got_slots):
+                batch.append(req)
+                starts.append(req.stored)
+                counts.append(1)
+                slots.append(slot)
+            pairs.extend(got_pairs)
+            budget -= done
+            i += done
+            if done < len(todo):
+                req = todo[done]
+                while req in self.running and self.bm.blocks_needed(req.seq, 1) > self.bm.num_free():
+                    victim = self._latest_running()
+                    self.metrics["alloc_failures"] += 1
+                    self._preempt(victim)
+                    preempted.append(victim)
+                decodes = decodes[:i] + [r for r in decodes[i:] if r in self.running]
         # prefill chunks: running requests mid-prefill, then waiting ones (FCFS)
         candidates = [r for r in sorted(self.running, key=lambda r: (r.arrival, r.rid))
                       if r.prefilling and r not in batch]

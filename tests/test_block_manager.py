@@ -85,6 +85,10 @@ def test_random_operations_match_the_oracle(seed):
                 assert e.value.code == 3
             else:
                 assert ours(s) == ref
+        elif op < 0.6:
+            # one token each for a few sequences, stopping where a block is missing
+            seqs = rng.sample(resident, min(len(resident), rng.randint(1, 6)))
+            assert bm.append_one_each(seqs) == ob.append_one_each(seqs)
         else:
             s = rng.choice(resident)
             n = rng.randint(0, 3 * bs)
