@@ -66,6 +66,7 @@ the last prefill chunk yields the first output token, each decode step
 appends the previous output token and yields the next.
 """
 
+import bisect
 from dataclasses import dataclass, field
 
 import torch
@@ -124,6 +125,10 @@ class StepPlan:
         return q
 
 
+def _arrival_order(r):
+    return (r.arrival, r.rid)
+
+
 class Scheduler:
     def __init__(self, bm, token_budget=4096, max_chunk=512, preempt="recompute", prefix_cache=False,
                  max_seqs=None):
@@ -157,8 +162,7 @@ class Scheduler:
         self._requeue(req)
 
     def _requeue(self, req):
-        self.waiting.append(req)
-        self.waiting.sort(key=lambda r: (r.arrival, r.rid))
+        bisect.insort(self.waiting, req, key=_arrival_order)
 
     def has_work(self):
         return bool(self.waiting or self.running or self.swapped)
@@ -177,8 +181,7 @@ class Scheduler:
             self.metrics["preemptions"] += 1
             self.metrics["swaps_out"] += 1
             self.running.remove(req)
-            self.swapped.append(req)
-            self.swapped.sort(key=lambda r: (r.arrival, r.rid))
+            bisect.insort(self.swapped, req, key=_arrival_order)
             return
         self.bm.free(req.seq)
         req.seq = -1
@@ -229,8 +232,7 @@ class Scheduler:
                 break        # arrival order: later ones wait behind this one
             self._swap_ops.append((False, self.bm.swap_in(req.seq)))
             self.swapped.remove(req)
-            self.running.append(req)
-            self.running.sort(key=lambda r: (r.arrival, r.rid))
+            bisect.insort(self.running, req, key=_arrival_order)
             self.metrics["swaps_in"] += 1
 
     def _plan(self):
@@ -251,7 +253,7 @@ class Scheduler:
         # needs a block while none is free; that one preempts the latest arrival
         # (never a request already served: they all arrived earlier) until it
         # fits or is itself preempted, and the rest follow
-        decodes = [r for r in sorted(self.running, key=lambda r: (r.arrival, r.rid)) if not r.prefilling]
+        decodes = [r for r in self.running if not r.prefilling]     # running is kept in arrival order
         i = 0
         while i < len(decodes) and budget > 0:
             todo = decodes[i:i + budget]
@@ -272,14 +274,17 @@ class Scheduler:
                     self._preempt(victim)
                     preempted.append(victim)
                 decodes = decodes[:i] + [r for r in decodes[i:] if r in self.running]
-        # prefill chunks: running requests mid-prefill, then waiting ones (FCFS)
-        candidates = [r for r in sorted(self.running, key=lambda r: (r.arrival, r.rid))
-                      if r.prefilling and r not in batch]
-        if not self.swapped:     # nothing new is admitted while a request is swapped out
-            candidates += [r for r in self.waiting if r not in preempted and self._may_admit(r)]
+        # prefill chunks: running requests mid-prefill, then waiting ones (FCFS);
+        # nothing new is admitted while a request is swapped out
+        in_batch = set(batch)
+        candidates = [r for r in self.running if r.prefilling and r not in in_batch]
+        if not self.swapped:
+            candidates += list(self.waiting)     # filtered below, as they come
         for req in candidates:
             if budget == 0:
                 break
+            if req.seq < 0 and (req in preempted or not self._may_admit(req)):
+                continue
             if req.seq < 0:
                 if self.max_seqs is not None and len(self.running) >= self.max_seqs:
                     break        # every slot is taken
@@ -303,8 +308,7 @@ class Scheduler:
                 if req.admit_step < 0:
                     req.admit_step = self.step_no
                 self.waiting.remove(req)
-                self.running.append(req)
-                self.running.sort(key=lambda r: (r.arrival, r.rid))
+                bisect.insort(self.running, req, key=_arrival_order)
                 self.metrics["admitted"] += 1
             n = min(self.max_chunk, req.target - req.stored, budget)
             if self.bm.blocks_needed(req.seq, n) > self.bm.num_free():
