@@ -361,3 +361,52 @@ def test_two_pool_admission_caps_concurrency_at_the_state_slots():
     assert max(len(p.requests) for p in p1) == 6
     assert len(s1.finished) == len(_small_trace())
     assert s1.bm.stats()["state_free_slots"] == 6
+
+
+# ---------------------------------------------------------------- property test
+from hypothesis import given, settings, HealthCheck, strategies as hst  # noqa: E402
+
+
+@settings(max_examples=40, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(
+    reqs=hst.lists(hst.tuples(hst.integers(0, 12), hst.integers(1, 300), hst.integers(1, 40),
+                              hst.integers(-1, 2), hst.integers(0, 160)), min_size=1, max_size=25),
+    nb=hst.integers(40, 200), bs=hst.sampled_from([4, 16]), budget=hst.sampled_from([64, 256, 1024]),
+    mode=hst.sampled_from(["recompute", "swap"]), prefix=hst.booleans(), static=hst.sampled_from([None, 3]))
+def test_random_traces_plan_identically_and_drain(reqs, nb, bs, budget, mode, prefix, static):
+    # any small trace, pool, budget and mode: the C++ and oracle managers give
+    # the same plans, every plan keeps the invariants, and everything drains
+    reqs = sorted(reqs)
+    trace = []
+    for a, p, o, g, sl in reqs:
+        if -(-(p + o - 1) // bs) > nb:
+            continue                                    # would be rejected at admission
+        trace.append((a, p, o, g, min(sl, p - 1) if g >= 0 else 0))
+    if not trace:
+        return
+
+    def run(bm):
+        if mode == "swap":
+            bm.set_host_blocks(nb)
+        kw = dict(token_budget=budget, max_chunk=min(budget, 128), preempt=mode, prefix_cache=prefix)
+        sched = StaticScheduler(bm, static, **kw) if static else Scheduler(bm, **kw)
+        pending = [Request(i, a, p, o, group=g, sys_len=sl) for i, (a, p, o, g, sl) in enumerate(trace)]
+        plans, step = [], 0
+        while pending or sched.has_work():
+            while pending and pending[0].arrival <= step:
+                sched.add_request(pending.pop(0))
+            plan = sched.schedule()
+            _check_plan(plan, sched, budget, min(budget, 128))
+            plans.append(([r.rid for r in plan.requests], plan.starts, plan.counts, plan.slots,
+                          plan.copy_pairs, plan.swap_ops, plan.tables.tolist()))
+            sched.complete(plan)
+            step += 1
+            assert step < 5000, "did not drain"
+        return sched, plans
+
+    s1, p1 = run(BlockManager(nb, bs))
+    s2, p2 = run(OracleAdapter(nb, bs))
+    assert p1 == p2 and s1.metrics == s2.metrics
+    assert len(s1.finished) == len(trace)
+    st = s1.bm.stats()
+    assert st["free_blocks"] == nb and st["num_seqs"] == 0 and st["cached_blocks"] == 0
