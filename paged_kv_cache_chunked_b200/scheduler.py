@@ -102,7 +102,8 @@ class Request:
 @dataclass
 class StepPlan:
     """One iteration's batch: per scheduled request, `n` new positions starting
-    at `start`; the device tensors the kernels take are built by `tensors()`."""
+    at `start`, with the slots, copy-on-write pairs, swaps and block tables the
+    step's kernels need (the drivers turn them into device tensors)."""
     step: int
     requests: list          # Request objects, batch order
     starts: list            # first new position per request
