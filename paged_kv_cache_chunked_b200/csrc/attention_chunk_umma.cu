@@ -14,11 +14,13 @@
 // Structure.  A work item is 256 query rows (pairs (token, head of the
 // group), token-major) of one (sequence, kv head), as two 128-row tiles; CTA i
 // takes items i, i + gridDim.x, ...  Per 128-key stage:
-//   - three producer warps load the stage's eight 16-key blocks by TMA: K as two
-//     2-D boxes per block (one per 64-column panel; warps 0 and 1) into the
-//     canonical K-major 128-byte-swizzled layout [panel][128 keys][128 B], V as
-//     one 3-D box per block [block][panel][16 keys][128 B] (warp 2).  K and V
-//     have rings of their own: a K slot is refilled once the stage's S has
+//   - three producer warps (9, 10, 11) load the stage's eight 16-key blocks by
+//     TMA: K as two 2-D boxes per block (one per 64-column panel; warps 9 and
+//     10) into the canonical K-major 128-byte-swizzled layout [panel][128
+//     keys][128 B], V as one 3-D box per block [block][panel][16 keys][128 B]
+//     (warp 11).  Lane j of a producer looks up and issues block j, so a
+//     stage's eight table lookups and boxes go out together.  K and V have
+//     rings of their own: a K slot is refilled once the stage's S has
 //     completed, a V slot once its P V has.  On a stage that runs past the
 //     context the V warp zeroes the rows past it (P is 0 there, the stale rows
 //     may hold anything) before it releases the stage;
