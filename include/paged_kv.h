@@ -257,7 +257,9 @@ int pk_bm_append_slots(pk_bm *bm, int64_t seq, int n, int64_t *slots_out, int32_
  * slots_out[i] its slot, pairs_out (int32 [n][2]) the copy-on-write pairs in
  * order (*n_pairs_out of them).  Stops, without counting an allocation
  * failure, at the first sequence whose token needs a block when none is free:
- * *n_done_out sequences got their token. */
+ * *n_done_out sequences got their token.  An unknown or swapped-out sequence
+ * ends the call with PK_ERR_INVALID_ARG; the ones before it keep their tokens
+ * (*n_done_out, *n_pairs_out and their slots and pairs say which). */
 int pk_bm_append_one_each(pk_bm *bm, const int64_t *seqs, int n, int64_t *slots_out, int32_t *pairs_out,
                           int *n_pairs_out, int *n_done_out);
 /* Blocks append_slots(seq, n) would take from the free list. */
