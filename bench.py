@@ -333,6 +333,49 @@ def workload_config(name, batch, l2_note):
 
 
 # ---------------------------------------------------------------- our arm
+def attention_call_ms(call, stream, n):
+    """Device ms of each of n calls, every call between two CUDA events on the
+    stream it is launched on (after 3 untimed calls)."""
+    for _ in range(3):
+        call()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    for a, b in evs:
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def workload_roofline(name, device, n_calls):
+    """Roofline of one pk_paged_attention call on another decode workload (the
+    long-document one rides along with the default line)."""
+    from paged_kv_cache_chunked_b200 import api
+    batch = workload_batch(name, poison_unused=False)
+    attn_b, _, kv_b = step_bytes(batch)
+    N, Hkv, bs, d = batch["k_pool"].shape
+    pool = api.kv_pool_create(N, bs, Hkv, d, torch.bfloat16, device)
+    pool.k_pool.copy_(batch["k_pool"])
+    pool.v_pool.copy_(batch["v_pool"])
+    dq, dt_ = batch["q"].to(device), batch["block_tables"].to(device)
+    dctx, dqsl = batch["context_lens"].to(device), batch["query_start_lens"].to(device)
+    out = torch.empty_like(dq)
+    stream = torch.cuda.current_stream(device)
+    ms = attention_call_ms(lambda: api.paged_attention(dq, pool.k_pool, pool.v_pool, dt_, dctx, dqsl,
+                                                       batch["scale"], out=out), stream, n_calls)
+    assert pool.check_device_errors() == 0
+    peak, kind = measured_peak()
+    avg = statistics.mean(ms)
+    gbs = attn_b / (avg * 1e-3) / 1e9
+    r = roofline_entry(name, attn_b, attention_flops(batch), avg, gbs, None, peak, kind)
+    r.update(calls=n_calls, config=workload_config(name, batch, f"no flush: {kv_b / 1e6:.0f} MB of KV "
+                                                                f"per call, more than the 126 MB L2"))
+    del pool
+    torch.cuda.empty_cache()
+    return r
+
+
 def run_ours(args, rank, world, device):
     from paged_kv_cache_chunked_b200 import api
 
@@ -355,13 +398,12 @@ def run_ours(args, rank, world, device):
     out = torch.empty_like(dq)
     stream = torch.cuda.current_stream(device)
 
-    def step(ev=None):
+    def step():
         api.paged_kv_append(dk, dv, dslots, pool=pool)
-        if ev is not None:
-            ev[0].record(stream)
         api.paged_attention(dq, pool.k_pool, pool.v_pool, dt_, dctx, dqsl, batch["scale"], out=out)
-        if ev is not None:
-            ev[1].record(stream)
+
+    def attention_only():
+        api.paged_attention(dq, pool.k_pool, pool.v_pool, dt_, dctx, dqsl, batch["scale"], out=out)
 
     # append, then per window of 512 sequences: for a batch of decodes only
     # (groups of <= 8 q heads) the block-streaming kernel and its merge kernel,
@@ -385,21 +427,22 @@ def run_ours(args, rank, world, device):
     if not args.profile_run:
         clocks.start()
         time.sleep(0.3)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
         tdist.barrier()
     torch.cuda.synchronize(device)
     start.record(stream)
     for i in range(args.steps):
-        step(evs[i])
+        step()
     end.record(stream)
     torch.cuda.synchronize(device)
     if dist:
         tdist.barrier()
     total_ms = start.elapsed_time(end)
-    attn_ms = [a.elapsed_time(b) for a, b in evs]
+    # the attention call alone, for its roofline: a separate pass, so that no
+    # event sits between the append and the attention of a timed step (the
+    # attention kernels start as programmatic dependents of the append)
+    attn_ms = attention_call_ms(attention_only, stream, max(args.steps, 50))
     # a long enough window for the clock sampler to see the load
     t_extra = time.perf_counter()
     while not args.profile_run and time.perf_counter() - t_extra < 1.0:
@@ -480,9 +523,18 @@ def run_ours(args, rank, world, device):
         "attention_tflops": tflops,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": dict(clk, window="the timed region plus 1 s of the same steps right after it"),
+        "attention_timing": f"{len(attn_ms)} attention calls, each between CUDA events, in a pass "
+                            f"after the timed steps",
     }
     if e2e:
         line["e2e"] = e2e
+    if args.workload == "decode64_bf16" and not args.profile_run and world == 1:
+        clocks2 = ClockSampler(device.index if device.index is not None else 0)
+        clocks2.start()
+        time.sleep(0.3)
+        extra = workload_roofline("longdoc_bf16", device, max(50, min(args.steps, 1000)))
+        extra["clocks"] = clocks2.stop()
+        line["extra_rooflines"] = {"longdoc_bf16": extra}
     if world == 1 and args.cpu_baseline_seconds > 0 and not args.profile_run:
         sec, runs, threads = oracle_step_seconds(batch, args.cpu_baseline_seconds)
         line["cpu_baseline"] = {"value": attn_b / sec / 1e9, "unit": "GB/s", "cores": threads,

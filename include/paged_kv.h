@@ -80,15 +80,31 @@ const char *pk_version(void);
  * torch tensors), 16-byte aligned.  The library owns only the descriptor and
  * a 4-byte device error word, both released by pk_pool_destroy.
  * dtype: PK_F32 or PK_BF16.  head_dim: 1..256 (fast tensor-core path: bf16,
- * head_dim 64/128/256, block_size a multiple of 8; anything else runs a
- * general CUDA kernel).  The current CUDA device at create time is the
- * pool's device; later calls must be made with that device current.
+ * head_dim 64/128/256, block_size a multiple of 8, n_kv_heads <= 64; anything
+ * else runs a general CUDA kernel).  The current CUDA device at create time is
+ * the pool's device; later calls must be made with that device current.
  * ------------------------------------------------------------------------ */
 typedef struct pk_pool pk_pool;
 
 int pk_pool_create(int num_blocks, int block_size, int n_kv_heads, int head_dim, int dtype,
                    void *k_base, void *v_base, pk_pool **out);
 int pk_pool_destroy(pk_pool *pool);
+
+/* Which attention kernels serve this pool, fixed when it was created: a bit
+ * set of the PK_PATH_* values below (0: the general kernel serves every call).
+ *   PK_PATH_TENSOR_CORE    TMA loads and tensor-core attention (bf16 geometries
+ *                          named above)
+ *   PK_PATH_DECODE_BLOCKS  one-token rows stream whole blocks, all kv heads of a
+ *                          group per TMA box (block-streaming decode kernel)
+ *   PK_PATH_CHUNK_TCGEN05  prefill chunks run on tcgen05 with accumulators in
+ *                          tensor memory (head_dim 128, block_size a multiple of
+ *                          16); without it they run on mma.sync.  The library
+ *                          leaves it off when the kernel was not compiled with
+ *                          the register count its warp roles are laid out for,
+ *                          or when PK_CHUNK_MMA_SYNC=1 is set in the environment.
+ * Host only; nothing is launched. */
+enum { PK_PATH_TENSOR_CORE = 1, PK_PATH_DECODE_BLOCKS = 2, PK_PATH_CHUNK_TCGEN05 = 4 };
+int pk_pool_paths(const pk_pool *pool, int *paths_out);
 
 /* Reads and clears the pool's device error word (synchronises `stream`).
  * *code_out = PK_OK or the first PK_ERR_BAD_INDEX / PK_ERR_TIMEOUT recorded. */
@@ -166,11 +182,12 @@ int pk_swap_blocks(const pk_pool *pool, void *host_k, void *host_v, int num_host
  * n_q_heads % n_kv_heads == 0.
  * workspace: device scratch of at least pk_attention_workspace_size bytes,
  *   256-byte aligned, owned by the caller, not shared by calls in flight at
- *   the same time; it holds the work-claim counter, the split-K arrival
- *   counters and the split-K partial results.  It must be zero-filled before
- *   its first use; every call that completes leaves the counters zeroed
- *   again, so a workspace can be reused across calls, batches and pools.
- *   After a call that recorded PK_ERR_TIMEOUT, zero it again.
+ *   the same time (two streams need two workspaces); it holds the work-claim
+ *   counters, the split-K arrival counters and the split-K partial results.
+ *   It must be zero-filled before its first use; every call that completes
+ *   leaves the counters zeroed again, at offsets that are the same for every
+ *   pool and batch, so a workspace can be reused across calls, batches and
+ *   pools.  After a call that recorded PK_ERR_TIMEOUT, zero it again.
  * ------------------------------------------------------------------------ */
 int pk_attention_workspace_size(const pk_pool *pool, int num_seqs, int num_tokens,
                                 int n_q_heads, int max_blocks_per_seq, size_t *bytes_out);
@@ -197,10 +214,12 @@ int pk_paged_attention(const pk_pool *pool, const void *q, void *out,
  * PK_ERR_WORKSPACE before anything is launched.  The first call on a device
  * looks up the array's device address (cudaGetSymbolAddress) with that
  * device current; make that first call before any stream capture.  All calls
- * share the array, which starts zeroed and which every completed call leaves
- * with its counters zeroed: calls whose work overlaps on the GPU (two
- * streams, two host threads) race and corrupt each other's results, so
- * serialise them.
+ * share the array and it keeps the last call's contents; each call starts by
+ * clearing the array's counter region on `stream` (cudaMemsetAsync, which
+ * allocates nothing), so a call that recorded PK_ERR_TIMEOUT leaves nothing
+ * stale for the next one.  Calls whose work overlaps on the GPU (two streams,
+ * two host threads) race on the array and corrupt each other's results, so
+ * serialise them.  num_seqs == 0 returns PK_OK with nothing queued.
  * ------------------------------------------------------------------------ */
 #define PK_NOALLOC_SCRATCH_BYTES (32u << 20)
 

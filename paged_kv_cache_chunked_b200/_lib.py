@@ -16,6 +16,8 @@ PK_OK = 0
 ERRORS = {1: "PK_ERR_INVALID_ARG", 2: "PK_ERR_OOM", 3: "PK_ERR_UNSUPPORTED", 4: "PK_ERR_CUDA",
           5: "PK_ERR_BAD_INDEX", 6: "PK_ERR_WORKSPACE", 7: "PK_ERR_TIMEOUT"}
 PK_F32, PK_BF16 = 0, 1
+PK_ERR_TIMEOUT = 7
+PK_PATH_TENSOR_CORE, PK_PATH_DECODE_BLOCKS, PK_PATH_CHUNK_TCGEN05 = 1, 2, 4
 
 
 class PagedKVError(RuntimeError):
@@ -51,6 +53,7 @@ SIGNATURES = {
     "pk_version": ([], ctypes.c_char_p),
     "pk_pool_create": ([_I, _I, _I, _I, _I, _P, _P, _PP], _I),
     "pk_pool_destroy": ([_P], _I),
+    "pk_pool_paths": ([_P, _PI], _I),
     "pk_check_device_errors": ([_P, _P, _PI], _I),
     "pk_paged_kv_append": ([_P, _P, _P, _P, _I, _P], _I),
     "pk_block_copy": ([_P, _P, _I, _P], _I),

@@ -17,7 +17,9 @@ import weakref
 
 import torch
 
-from ._lib import PK_BF16, PK_F32, BmStats, OutOfBlocks, PagedKVError, check, lib  # noqa: F401
+from ._lib import (PK_BF16, PK_ERR_TIMEOUT, PK_F32, PK_PATH_CHUNK_TCGEN05,  # noqa: F401
+                   PK_PATH_DECODE_BLOCKS, PK_PATH_TENSOR_CORE, BmStats, OutOfBlocks, PagedKVError,
+                   check, lib)
 
 _DTYPES = {torch.float32: PK_F32, torch.bfloat16: PK_BF16}
 _pools = weakref.WeakValueDictionary()  # k_pool data_ptr -> KVPool
@@ -73,7 +75,7 @@ class KVPool:
             check(lib().pk_pool_create(num_blocks, block_size, n_kv_heads, head_dim, _DTYPES[dtype],
                                        _ptr(self.k_pool), _ptr(self.v_pool),
                                        ctypes.byref(self._handle)))
-        self._workspace = None
+        self._workspaces = {}     # CUDA stream handle -> its workspace
         _pools[self.k_pool.data_ptr()] = self
 
     @property
@@ -94,20 +96,40 @@ class KVPool:
         except Exception:
             pass
 
-    def workspace(self, num_seqs, num_tokens, n_q_heads, max_blocks):
-        """Device scratch for one attention call of this shape (kept and grown)."""
+    def workspace(self, num_seqs, num_tokens, n_q_heads, max_blocks, stream=None):
+        """Device scratch for one attention call of this shape on `stream`
+        (default: the current stream), kept and grown.  Calls in flight at the
+        same time must not share scratch, so each stream has its own."""
         n = ctypes.c_size_t()
         check(lib().pk_attention_workspace_size(self.handle, num_seqs, num_tokens, n_q_heads,
                                                 max_blocks, ctypes.byref(n)))
-        if self._workspace is None or self._workspace.numel() < n.value:
-            # zero-filled once; every call leaves its counters zeroed again
-            self._workspace = torch.zeros(max(n.value, 256), dtype=torch.uint8, device=self.device)
-        return self._workspace
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        ws = self._workspaces.get(stream.cuda_stream)
+        if ws is None or ws.numel() < n.value:
+            # zero-filled once, on the stream that uses it; every completed call
+            # leaves its counters zeroed again
+            with torch.cuda.stream(stream):
+                ws = torch.zeros(max(n.value, 256), dtype=torch.uint8, device=self.device)
+            self._workspaces[stream.cuda_stream] = ws
+        return ws
+
+    def paths(self):
+        """The PK_PATH_* bit set of the kernels that serve this pool."""
+        f = ctypes.c_int()
+        check(lib().pk_pool_paths(self.handle, ctypes.byref(f)))
+        return f.value
 
     def check_device_errors(self):
-        """PK_OK or the first device-side error code recorded since the last check."""
+        """PK_OK or the first device-side error code recorded since the last check.
+        After PK_ERR_TIMEOUT every workspace of the pool is zeroed again: a call
+        that gave up on a bounded wait may have left split-K counters set."""
         code = ctypes.c_int()
         check(lib().pk_check_device_errors(self.handle, _stream(self.device), ctypes.byref(code)))
+        if code.value == PK_ERR_TIMEOUT:
+            for ws in self._workspaces.values():
+                ws.zero_()
+            torch.cuda.synchronize(self.device)
         return code.value
 
 

@@ -135,7 +135,8 @@ int pk_pool_create(int num_blocks, int block_size, int n_kv_heads, int head_dim,
     }
     const long long rows = (long long)num_blocks * n_kv_heads * block_size;
     p->tc_path = dtype == PK_BF16 && (head_dim == 64 || head_dim == 128 || head_dim == 256) &&
-                 block_size % 8 == 0 && rows < (1LL << 31) && !force_generic();
+                 block_size % 8 == 0 && n_kv_heads <= kMaxTcKvHeads && rows < (1LL << 31) &&
+                 !force_generic();
     if (p->tc_path) {
         // 16-token tiles of one (block, kv head): one 3-D box brings all head-dim
         // panels when a tile lies in one block (block_size a multiple of 16);
@@ -167,6 +168,18 @@ int pk_pool_destroy(pk_pool *pool) {
     if (dev >= 0 && dev != pool->device) cudaSetDevice(dev);
     delete pool;
     return e == cudaSuccess ? PK_OK : cuda_fail(e, "pool destroy");
+}
+
+int pk_pool_paths(const pk_pool *pool, int *paths_out) {
+    if (!pool || !paths_out) return fail(PK_ERR_INVALID_ARG, "NULL argument");
+    int f = 0;
+    if (pool->tc_path) {
+        f |= PK_PATH_TENSOR_CORE;
+        if (pool->blk_ok) f |= PK_PATH_DECODE_BLOCKS;
+        if (pool->umma_ok) f |= PK_PATH_CHUNK_TCGEN05;
+    }
+    *paths_out = f;
+    return PK_OK;
 }
 
 int pk_check_device_errors(const pk_pool *pool, pk_stream_t stream, int *code_out) {

@@ -11,14 +11,20 @@ namespace pk {
 namespace {
 
 constexpr size_t kHeaderBytes = 256;     // one scheduler header per kernel
-constexpr int kMaxSeqsPerLaunch = 512;   // window of sequences per kernel launch
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Workspace: decode header | chunk header | split-K counters (fixed size) |
-// merge plan (fixed size) | partial log2-sum-exp | partial O.  The headers and counters sit at offsets
-// that do not depend on the batch, so the zeros every call leaves there stay
-// valid when the next call's batch differs.
+// Workspace: decode header | chunk header | split-K counters | merge plan |
+// partial log2-sum-exp | partial O.  The headers and the counter region have
+// the same offsets and sizes for every pool and batch (the counters are sized
+// for kMaxTcKvHeads), so the zeros that every completed call leaves there stay
+// valid for the next call, whatever its pool or batch: a workspace, or the
+// no-allocation entry point's shared array, can move between pools.  Everything
+// after the counters is written before it is read.
+constexpr size_t kCountersOff = 2 * kHeaderBytes;
+constexpr size_t kZeroedBytes =
+    (kCountersOff + (size_t)kMaxSeqsPerLaunch * kMaxTcKvHeads * sizeof(int) + 255) / 256 * 256;
+
 struct Layout {
     size_t hdr_decode, hdr_chunk, counters, merge_plan, partial_lse, partial_o, total;
     int cap_rows;
@@ -39,9 +45,8 @@ Layout layout(const pk_pool *p, int num_seqs, int n_q_heads) {
     L.cap_rows = (int)std::min<long long>(items * std::min(g, kTile), 1LL << 30);
     L.hdr_decode = 0;
     L.hdr_chunk = kHeaderBytes;
-    size_t off = 2 * kHeaderBytes;
-    L.counters = off;
-    off = align_up(off + (size_t)kMaxSeqsPerLaunch * Hkv * sizeof(int), 256);
+    L.counters = kCountersOff;
+    size_t off = kZeroedBytes;
     L.merge_plan = off;  // a count, then an int4 per split (sequence, head group)
     off = align_up(off + (size_t)(4 + 4 * kMaxSeqsPerLaunch * Hkv) * sizeof(int), 256);
     L.partial_lse = off;
@@ -59,6 +64,8 @@ size_t tc_workspace_bytes(const pk_pool *p, int num_seqs, int num_tokens, int n_
     (void)num_tokens;
     return layout(p, num_seqs, n_q_heads).total;
 }
+
+size_t tc_workspace_zeroed_bytes() { return kZeroedBytes; }
 
 int tc_prepare_pool(pk_pool *p) {
     int rc = decode_prepare_pool(p);

@@ -20,12 +20,16 @@
 // capture.
 //
 // All calls share the array and it keeps the last call's contents.  The only
-// state a call relies on at its start is the work-claim counter and the
-// split-K arrival counters, which must be zero: the array starts zeroed (a
-// __device__ variable is zero-initialised) and every completed call leaves
-// them zeroed; everything else is written before it is read.  Two calls whose
-// work overlaps on the GPU (on two streams, or from two host threads) race on
-// the array and corrupt each other's results.  Serialise them.
+// state a call relies on at its start is the work-claim counters and the
+// split-K arrival counters, which must be zero; they sit in a region at the
+// start of the array whose offsets and size are the same for every pool.  A
+// completed call leaves them zeroed, but a call that gave up on a bounded wait
+// (PK_ERR_TIMEOUT) may not, and nobody else can reach the array to clear it:
+// so every call first zeroes that region on its own stream with
+// cudaMemsetAsync (a few hundred KiB; it allocates nothing).  Everything else
+// is written before it is read.  Two calls whose work overlaps on the GPU (on
+// two streams, or from two host threads) race on the array and corrupt each
+// other's results.  Serialise them.
 #include <mutex>
 
 #include "pk_internal.h"
@@ -75,12 +79,21 @@ extern "C" int pk_paged_attention_noalloc(const pk_pool *pool, const void *q, vo
                         "batch needs %zu bytes of scratch; the no-allocation entry point has "
                         "%zu (use pk_paged_attention with a workspace)",
                         need, kNoAllocScratchBytes);
+    if (num_seqs == 0)  // argument checks only; nothing is queued
+        return pk_paged_attention(pool, q, out, block_tables, max_blocks_per_seq, context_lens,
+                                  query_start_lens, num_seqs, num_tokens, n_q_heads, scale, nullptr,
+                                  0, stream);
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev != pool->device)
         return pk::fail(PK_ERR_INVALID_ARG, "the pool's device must be current");
     void *scratch = nullptr;
     rc = scratch_on_current_device(&scratch);
     if (rc != PK_OK) return rc;
+    if (pool->tc_path) {
+        const cudaError_t e =
+            cudaMemsetAsync(scratch, 0, pk::tc_workspace_zeroed_bytes(), (cudaStream_t)stream);
+        if (e != cudaSuccess) return pk::cuda_fail(e, "clearing the scratch counters");
+    }
     return pk_paged_attention(pool, q, out, block_tables, max_blocks_per_seq, context_lens,
                               query_start_lens, num_seqs, num_tokens, n_q_heads, scale, scratch,
                               kNoAllocScratchBytes, stream);

@@ -47,6 +47,11 @@ __device__ __forceinline__ void record_error(int *err, int code) {
 
 constexpr int kMaxHeadDim = 256;
 constexpr int kTile = 16;        // tokens per KV tile and rows per query tile
+constexpr int kMaxSeqsPerLaunch = 512;  // window of sequences per kernel launch
+// Largest n_kv_heads of the tensor-core path: the workspace keeps one split-K
+// arrival counter per (sequence of a launch window, kv head) in a region of
+// fixed size, so that every pool finds its counters at the same offsets.
+constexpr int kMaxTcKvHeads = 64;
 
 // ---- launchers (each returns PK_OK or an error code) ---------------------
 int launch_kv_append(const pk_pool *p, const void *k, const void *v, const int64_t *slots,
@@ -75,6 +80,9 @@ int launch_attention_generic(const pk_pool *p, const AttnArgs &a, cudaStream_t s
 // Tensor-core path: workspace sizing and launch.
 size_t tc_workspace_bytes(const pk_pool *p, int num_seqs, int num_tokens, int n_q_heads,
                           int max_blocks_per_seq);
+// Bytes at the start of every workspace that must be zero when a call starts
+// (scheduler headers and split-K arrival counters); the same for every pool.
+size_t tc_workspace_zeroed_bytes();
 int tc_prepare_pool(pk_pool *p);  // occupancy queries, once per pool
 int launch_attention_tc(const pk_pool *p, const AttnArgs &a, cudaStream_t st);
 

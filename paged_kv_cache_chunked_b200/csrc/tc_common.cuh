@@ -10,7 +10,6 @@ namespace pk {
 namespace tc {
 
 constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded wait: 2 s
-constexpr int kMaxSeqsPerLaunch = 512;
 constexpr int kPlanLen = kMaxSeqsPerLaunch + 1;
 constexpr int kPartitionMinTiles = 4;  // smallest split-K partition (64 tokens)
 

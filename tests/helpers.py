@@ -66,3 +66,26 @@ def sample_rows(num_tokens, n_q_heads, n, seed):
 
 def scale_of(head_dim):
     return 1.0 / math.sqrt(head_dim)
+
+
+def recorded_ops(device, call):
+    """Number of operations (kernels, copies, memsets) that call(stream)
+    queues on a fresh stream: the stream is put in capture mode, so the work
+    is recorded in a CUDA graph, counted and dropped, never run."""
+    import ctypes
+
+    from cuda.bindings import runtime as rt
+    s = torch.cuda.Stream(device)
+    torch.cuda.synchronize(device)
+    (err,) = rt.cudaStreamBeginCapture(rt.cudaStream_t(s.cuda_stream),
+                                       rt.cudaStreamCaptureMode.cudaStreamCaptureModeRelaxed)
+    assert err == rt.cudaError_t.cudaSuccess, err
+    try:
+        rc = call(ctypes.c_void_p(s.cuda_stream))
+    finally:
+        err, graph = rt.cudaStreamEndCapture(rt.cudaStream_t(s.cuda_stream))
+    assert err == rt.cudaError_t.cudaSuccess, err
+    err, _, n = rt.cudaGraphGetNodes(graph, 0)
+    assert err == rt.cudaError_t.cudaSuccess, err
+    rt.cudaGraphDestroy(graph)
+    return rc, n

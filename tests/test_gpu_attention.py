@@ -152,21 +152,60 @@ def test_long_context_split_k(cuda_dev):
 
 
 @pytest.mark.parametrize("name", ["decode64_bf16", "longdoc_bf16"])
-def test_full_size_workloads_sampled_rows(cuda_dev, name):
-    # the bench's workloads at full size: sampled rows against the oracle
+def test_full_size_decode_workloads_every_row(cuda_dev, name):
+    # the bench's decode workloads at full size, in the launch configuration
+    # the bench times: every output row against the oracle
     b = workload_batch(name, poison_unused=False)
-    d = b["q"].shape[2]
-    Hq = b["q"].shape[1]
-    Hkv = b["k_pool"].shape[1]
+    Hkv, d = b["k_pool"].shape[1], b["q"].shape[2]
     pool = gpu_pool_from(b, Hkv, d, torch.bfloat16, cuda_dev)
+    got = run_gpu_attention(b, pool, cuda_dev)
+    assert_close(got, oracle_attention(b), torch.bfloat16, name)
+    assert pool.check_device_errors() == 0
+
+
+def test_full_size_chunk512_sampled_rows(cuda_dev):
+    # sixteen 512-token chunks at context 4,096 (the bench's prefill workload) at
+    # full size: the first and last row of every 256-row work item of the
+    # tcgen05 kernel (rows are (token, group head) pairs, token-major, per
+    # (sequence, kv head)) plus 2,000 random rows, against the oracle
+    b = workload_batch("chunk512_bf16", poison_unused=False)
+    T, Hq, d = b["q"].shape
+    Hkv = b["k_pool"].shape[1]
+    g = Hq // Hkv
+    pool = gpu_pool_from(b, Hkv, d, torch.bfloat16, cuda_dev)
+    assert pool.paths() & api.PK_PATH_CHUNK_TCGEN05
     got = run_gpu_attention(b, pool, cuda_dev).cpu()
-    rows = sample_rows(b["q"].shape[0], Hq, 48, seed=5)
+    rows = sample_rows(T, Hq, 2000, seed=6)
+    qsl = b["query_start_lens"].tolist()
+    for s in range(len(qsl) - 1):
+        qn = qsl[s + 1] - qsl[s]
+        for kvh in range(Hkv):
+            for r0 in range(0, qn * g, 256):
+                for r in (r0, min(r0 + 255, qn * g - 1)):
+                    rows.append([qsl[s] + r // g, kvh * g + r % g])
     ref = oracle.paged_attention_rows(b["q"], b["k_pool"], b["v_pool"], b["block_tables"],
                                       b["context_lens"], b["query_start_lens"], b["scale"], rows)
     got_rows = torch.stack([got[t, h] for t, h in rows])
-    assert_close(got_rows, ref, torch.bfloat16, name)
+    assert_close(got_rows, ref, torch.bfloat16, "chunk512")
     assert torch.isfinite(got).all()
     assert pool.check_device_errors() == 0
+
+
+@pytest.mark.parametrize("Hkv,d,bs,want", [
+    (8, 128, 16, ("TENSOR_CORE", "DECODE_BLOCKS", "CHUNK_TCGEN05")),
+    (4, 256, 16, ("TENSOR_CORE", "DECODE_BLOCKS")),
+    (8, 64, 16, ("TENSOR_CORE", "DECODE_BLOCKS")),
+    (8, 128, 8, ("TENSOR_CORE", "DECODE_BLOCKS")),
+])
+def test_pool_paths(cuda_dev, Hkv, d, bs, want):
+    # the kernels a pool selects are reported, so that losing the tcgen05 chunk
+    # kernel (a register count other than the one its warp roles assume) is
+    # seen rather than silently running every chunk on mma.sync
+    pool = api.kv_pool_create(64, bs, Hkv, d, torch.bfloat16, cuda_dev)
+    bits = {n: getattr(api, "PK_PATH_" + n) for n in ("TENSOR_CORE", "DECODE_BLOCKS", "CHUNK_TCGEN05")}
+    assert {n for n, v in bits.items() if pool.paths() & v} == set(want)
+    fp32 = api.kv_pool_create(64, 16, 8, 64, torch.float32, cuda_dev)
+    assert fp32.paths() == 0
 
 
 def test_single_token_context_returns_its_value(cuda_dev):

@@ -424,3 +424,80 @@ def test_state_slots_follow_sequence_lifetimes():
     bm.append_slots(b, 4)
     bm.swap_out(b)                                  # a swapped sequence keeps its slot
     assert bm.state_slot(b) >= 0 and bm.stats()["state_free_slots"] == 0
+
+
+# ---------------------------------------------------------------- one token for each decode
+def test_append_one_each_worked_example():
+    # four 4-slot blocks, FIFO free list 0..3.  A holds a full block, B two
+    # tokens, C three: one free block left.  Worked by hand from the table rule
+    # ["PagedAttention & Continuous Batching" (study notes), "Block tables":
+    # position p lives in logical block p // bs at offset p % bs; a new block is
+    # taken only when a token starts one].
+    bm = OracleBlockManager(4, 4)
+    a, b, c = bm.add_seq(), bm.add_seq(), bm.add_seq()
+    assert bm.append_slots(a, 4) == ([0, 1, 2, 3], [])
+    assert bm.append_slots(b, 2) == ([4, 5], [])
+    assert bm.append_slots(c, 3) == ([8, 9, 10], [])
+    # B at position 2 (block 1, offset 2), C at 3 (block 2, offset 3), A at 4
+    # starts a block (the free block 3), A at 5 fills it
+    assert bm.append_one_each([b, c, a, a]) == (4, [6, 11, 12, 13], [])
+    assert bm.num_free() == 0
+    # A at 6 and B at 3 fit; C at 4 needs a block and none is free: the call
+    # stops there, counts no allocation failure and leaves C and A's second
+    # request alone
+    assert bm.append_one_each([a, b, c, a]) == (2, [14, 7], [])
+    assert bm.alloc_failures == 0
+    assert (bm.length(a), bm.length(b), bm.length(c)) == (7, 4, 4)
+    assert bm.block_table(c) == [2] and bm.block_table(a) == [0, 3]
+
+
+def test_append_one_each_copy_on_write_and_stop():
+    # a fork shares a partly filled block: the first sharer to write copies it
+    # into a fresh block ["PagedAttention & Continuous Batching" (study notes),
+    # "Copy-on-write"], the last one writes in place; with no block left for a
+    # copy the call stops before that sequence
+    bm = OracleBlockManager(3, 4)
+    p = bm.add_seq()
+    bm.append_slots(p, 6)                       # blocks 0, 1; block 1 holds 2 tokens
+    d = bm.fork(p)
+    assert bm.append_one_each([d, p]) == (2, [10, 6], [(1, 2)])
+    assert bm.block_table(d) == [0, 2] and bm.block_table(p) == [0, 1]
+    e = bm.fork(p)                              # block 1 shared again, 3 tokens in it
+    assert bm.append_one_each([e, p]) == (0, [], [])
+    assert bm.alloc_failures == 0
+    assert bm.block_table(e) == [0, 1] and bm.refcount[1] == 2 and bm.length(e) == 7
+
+
+def test_append_one_each_equals_single_appends_until_the_first_refusal():
+    # the same tokens one append_slots(seq, 1) at a time: identical slots, pairs
+    # and state up to the first append that would be refused; nothing after it
+    import copy
+    rng = random.Random(11)
+    for trial in range(40):
+        bm = OracleBlockManager(rng.randint(6, 30), rng.choice([2, 4, 8]))
+        seqs = []
+        for _ in range(rng.randint(1, 6)):
+            s = bm.add_seq()
+            seqs.append(s)
+            n = rng.randint(0, 3 * bm.block_size)
+            if bm.blocks_needed(s, n) <= bm.num_free():
+                bm.append_slots(s, n)
+        for _ in range(rng.randint(0, 3)):
+            seqs.append(bm.fork(rng.choice(seqs)))
+        order = [rng.choice(seqs) for _ in range(rng.randint(1, 12))]
+        ref = copy.deepcopy(bm)
+        slots, pairs, served = [], [], 0
+        for s in order:
+            failures = ref.alloc_failures
+            try:
+                sl, pr = ref.append_slots(s, 1)
+            except OracleOOM:
+                ref.alloc_failures = failures     # the refused append is not part of the call
+                break
+            slots += sl
+            pairs += pr
+            served += 1
+        assert bm.append_one_each(order) == (served, slots, pairs), trial
+        assert bm.tables == ref.tables and bm.lengths == ref.lengths
+        assert bm.refcount == ref.refcount and list(bm.free_list) == list(ref.free_list)
+        assert bm.alloc_failures == ref.alloc_failures
