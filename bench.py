@@ -50,7 +50,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="decode64_bf16",
-                   choices=["decode64_bf16", "longdoc_bf16", "chunk512_bf16", "trace", "trace_swap",
+                   choices=["decode64_bf16", "longdoc_bf16", "chunk512_bf16", "mixed_bf16", "trace", "trace_swap",
                             "trace_prefix", "trace_prefix_nocache", "trace_hybrid", "policy", "fork",
                             "fork1028", "append_copy"])
     p.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
@@ -308,6 +308,8 @@ def roofline_entry(workload, attn_b, flops, avg_ms, gbs, tflops, hbm_peak, hbm_k
     the tensor pipe for prefill chunks (a dense contraction)."""
     kern = ("paged_attention call: tcgen05 chunk kernel (S and O accumulated in tensor memory)"
             if workload == "chunk512_bf16" else
+            "paged_attention call: block-streaming decode kernel + split-K merge kernel, then the "
+            "tcgen05 chunk kernel" if workload == "mixed_bf16" else
             "paged_attention call: block-streaming decode kernel + split-K merge kernel")
     common = {"kernel": kern,
               "algorithmic_bytes": attn_b, "algorithmic_flops": flops, "avg_ms": avg_ms,
@@ -348,6 +350,49 @@ def attention_call_ms(call, stream, n):
     return [a.elapsed_time(b) for a, b in evs]
 
 
+def sub_batch(batch, idx):
+    """Sequences idx of a batch (same pools), with their query rows."""
+    qsl = batch["query_start_lens"].tolist()
+    toks = torch.cat([torch.arange(qsl[i], qsl[i + 1]) for i in idx])
+    lens = torch.tensor([qsl[i + 1] - qsl[i] for i in idx], dtype=torch.int32)
+    sub = dict(batch)
+    sub["q"] = batch["q"][toks]
+    sub["block_tables"] = batch["block_tables"][idx]
+    sub["context_lens"] = batch["context_lens"][idx]
+    sub["query_start_lens"] = torch.cat([torch.zeros(1, dtype=torch.int32), torch.cumsum(lens, 0)]).to(torch.int32)
+    return sub
+
+
+def mixed_split(batch, pool, device, n_calls, hbm_peak, hbm_kind):
+    """A mixed step's decode rows and chunk rows, each as a call of its own
+    (same pool, same kernels as in the mixed call): the decode rows against
+    the HBM roofline, the chunk rows against the tensor roofline."""
+    from paged_kv_cache_chunked_b200 import api
+    qn = (batch["query_start_lens"][1:] - batch["query_start_lens"][:-1]).tolist()
+    out = {}
+    stream = torch.cuda.current_stream(device)
+    for name, idx in (("decode_rows", [i for i, n in enumerate(qn) if n == 1]),
+                      ("chunk_rows", [i for i, n in enumerate(qn) if n > 1])):
+        sb = sub_batch(batch, idx)
+        dq, dt_ = sb["q"].to(device), sb["block_tables"].to(device)
+        dctx, dqsl = sb["context_lens"].to(device), sb["query_start_lens"].to(device)
+        o = torch.empty_like(dq)
+        ms = statistics.mean(attention_call_ms(lambda: api.paged_attention(
+            dq, pool.k_pool, pool.v_pool, dt_, dctx, dqsl, batch["scale"], out=o), stream, n_calls))
+        ab, _, _ = step_bytes(sb)
+        fl = attention_flops(sb)
+        if name == "decode_rows":
+            gbs = ab / (ms * 1e-3) / 1e9
+            out[name] = {"sequences": len(idx), "ms": ms, "algorithmic_bytes": ab, "achieved": gbs,
+                         "unit": "GB/s", "peak": hbm_peak, "frac": gbs / hbm_peak, "bound": "hbm"}
+        else:
+            tp, _ = measured_tensor_peak()
+            tf = fl / (ms * 1e-3) / 1e12
+            out[name] = {"sequences": len(idx), "ms": ms, "algorithmic_flops": fl, "achieved": tf,
+                         "unit": "TFLOP/s", "peak": tp, "frac": tf / tp, "bound": "tensor"}
+    return out
+
+
 def workload_roofline(name, device, n_calls):
     """Roofline of one pk_paged_attention call on another decode workload (the
     long-document one rides along with the default line)."""
@@ -374,6 +419,51 @@ def workload_roofline(name, device, n_calls):
     del pool
     torch.cuda.empty_cache()
     return r
+
+
+def indirection_cost(batch, pool, dq, dctx, dqsl, device, n_calls):
+    """["Batching and PagedAttention", "The indirection has a cost"]: the same
+    decode batch through the same kernel with each sequence's blocks
+    contiguous and in logical order (identity tables) against the shuffled
+    tables of the workload.  The logical K/V are identical, so the outputs
+    must be bit-identical; the ratio of call times is the price of the scatter."""
+    from paged_kv_cache_chunked_b200 import api
+    tables = batch["block_tables"]
+    ctx = batch["context_lens"].tolist()
+    bs = batch["block_size"]
+    nblk = [-(-c // bs) for c in ctx]
+    old_ids = torch.cat([tables[b, :n].long() for b, n in enumerate(nblk)])
+    contig = torch.full_like(tables, -1)
+    base = 0
+    for b, n in enumerate(nblk):
+        contig[b, :n] = torch.arange(base, base + n, dtype=torch.int32)
+        base += n
+    N, Hkv, _, d = batch["k_pool"].shape
+    cpool = api.kv_pool_create(N, bs, Hkv, d, torch.bfloat16, device)
+    cpool.k_pool[:base] = pool.k_pool[old_ids.to(device)]
+    cpool.v_pool[:base] = pool.v_pool[old_ids.to(device)]
+    dt_s, dt_c = tables.to(device), contig.to(device)
+    o_s, o_c = torch.empty_like(dq), torch.empty_like(dq)
+    stream = torch.cuda.current_stream(device)
+    call_s = lambda: api.paged_attention(dq, pool.k_pool, pool.v_pool, dt_s, dctx, dqsl, batch["scale"], out=o_s)
+    call_c = lambda: api.paged_attention(dq, cpool.k_pool, cpool.v_pool, dt_c, dctx, dqsl, batch["scale"],
+                                         out=o_c)
+    ms_s, ms_c = [], []
+    for _ in range(2):          # alternate, so that both see the same clocks
+        ms_s += attention_call_ms(call_s, stream, n_calls // 2)
+        ms_c += attention_call_ms(call_c, stream, n_calls // 2)
+    torch.cuda.synchronize(device)
+    same = bool(torch.equal(o_s, o_c))
+    assert cpool.check_device_errors() == 0
+    del cpool
+    torch.cuda.empty_cache()
+    t_s, t_c = statistics.mean(ms_s), statistics.mean(ms_c)
+    return {"shuffled_ms": t_s, "contiguous_ms": t_c, "paged_over_contiguous": t_s / t_c,
+            "outputs_bit_identical": same, "calls_each": len(ms_s),
+            "pages_figure": "+20-26% for a paged kernel against an optimised contiguous kernel "
+                            "(hardware not stated)",
+            "how": "one kernel, tables that list each sequence's blocks contiguously in logical order "
+                   "against the workload's randomly permuted tables"}
 
 
 def run_ours(args, rank, world, device):
@@ -409,11 +499,18 @@ def run_ours(args, rank, world, device):
     # (groups of <= 8 q heads) the block-streaming kernel and its merge kernel,
     # else the chunk kernel (when chunks are present) and the tile-streaming
     # decode kernel; the general kernel is one launch
-    tc = pool.dtype == torch.bfloat16 and d in (64, 128, 256) and bs % 8 == 0
+    paths = pool.paths()
+    tc = bool(paths & api.PK_PATH_TENSOR_CORE)
     B = batch["context_lens"].shape[0]
     windows = (B + 511) // 512
-    blocks_path = tc and T == B and Hq // Hkv <= 8
-    per_window = 2 if blocks_path else (2 if T > B or Hq // Hkv > 16 else 1)
+    blocks = bool(paths & api.PK_PATH_DECODE_BLOCKS) and Hq // Hkv <= 8
+    umma = bool(paths & api.PK_PATH_CHUNK_TCGEN05) and 128 % (Hq // Hkv) == 0
+    if blocks and T == B:
+        per_window = 2                  # block-streaming decode + merge
+    elif blocks and umma:
+        per_window = 3                  # block-streaming decode + merge, then the tcgen05 chunk kernel
+    else:
+        per_window = 2 if T > B or Hq // Hkv > 16 else 1
     launches_per_step = 1 + (windows * per_window if tc else 1)
     for _ in range(max(args.warmup, 3)):
         step()
@@ -528,12 +625,24 @@ def run_ours(args, rank, world, device):
     }
     if e2e:
         line["e2e"] = e2e
+    if args.workload == "mixed_bf16" and not args.profile_run:
+        split = mixed_split(batch, pool, device, max(50, min(args.steps, 500)), peak, peak_kind)
+        tp, _ = measured_tensor_peak()
+        ideal_ms = (split["decode_rows"]["algorithmic_bytes"] / (peak * 1e9)
+                    + split["chunk_rows"]["algorithmic_flops"] / (tp * 1e12)) * 1e3
+        line["mixed"] = dict(split, call_ms=attn_avg_ms, ideal_ms=ideal_ms, call_frac=ideal_ms / attn_avg_ms,
+                             how="ideal_ms = decode-row bytes / HBM peak + chunk-row flops / bf16 peak; "
+                                 "each part also timed alone through the same entry point")
     if args.workload == "decode64_bf16" and not args.profile_run and world == 1:
         clocks2 = ClockSampler(device.index if device.index is not None else 0)
         clocks2.start()
         time.sleep(0.3)
-        extra = workload_roofline("longdoc_bf16", device, max(50, min(args.steps, 1000)))
-        extra["clocks"] = clocks2.stop()
+        n_calls = max(50, min(args.steps, 1000))
+        line["indirection"] = indirection_cost(batch, pool, dq, dctx, dqsl, device, 2 * n_calls)
+        extra = workload_roofline("longdoc_bf16", device, n_calls)
+        clk2 = clocks2.stop()
+        extra["clocks"] = clk2
+        line["indirection"]["clocks"] = clk2
         line["extra_rooflines"] = {"longdoc_bf16": extra}
     if world == 1 and args.cpu_baseline_seconds > 0 and not args.profile_run:
         sec, runs, threads = oracle_step_seconds(batch, args.cpu_baseline_seconds)
@@ -700,6 +809,112 @@ def run_kvops(args, rank, world, device):
     print(json.dumps(line), flush=True)
 
 
+class AttentionSplit:
+    """on_step hook of a trace run: after each step's timed region, times the
+    step's attention call again, then its decode rows alone (sequences of one
+    query token) and its chunk rows alone (several query tokens), each between
+    CUDA events on the stream, into scratch outputs (the pool is only read).
+    The pool is the one the step just wrote, so part of it may still sit in L2
+    (a step reads several hundred MB of KV against the 126 MB L2)."""
+
+    def __init__(self, runner, record_steps=0):
+        self.r = runner
+        self.acc = dict(full_ms=0.0, dec_ms=0.0, chunk_ms=0.0, dec_bytes=0, chunk_flops=0, steps=0,
+                        dec_calls=0, chunk_calls=0)
+        self.record_steps = record_steps
+        self.recorded = []
+
+    def _time(self, fn):
+        st = torch.cuda.current_stream(self.r.device)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        fn()
+        b.record(st)
+        b.synchronize()
+        return a.elapsed_time(b)
+
+    def __call__(self, plan, t, out):
+        from paged_kv_cache_chunked_b200 import api
+        if out is None:
+            return
+        r, dev = self.r, self.r.device
+        if len(self.recorded) < self.record_steps:
+            self.recorded.append({k: (v.cpu() if torch.is_tensor(v) else v) for k, v in t.items()})
+        q = t["q"]
+        tables, ctx, qsl = t["tables"], t["ctx"], t["qsl"]
+        qn = (qsl[1:] - qsl[:-1]).tolist()
+        c = ctx.tolist()
+        dtab, dctx, dqsl = tables.to(dev), ctx.to(dev), qsl.to(dev)
+        scratch = torch.empty_like(q)
+        self.acc["full_ms"] += self._time(lambda: api.paged_attention(
+            q, r.pool.k_pool, r.pool.v_pool, dtab, dctx, dqsl, r.scale, out=scratch))
+        kv_tok = r.Hkv * r.d * 2 * 2
+        dec = [i for i, n in enumerate(qn) if n == 1]
+        chk = [i for i, n in enumerate(qn) if n > 1]
+        qs = qsl.tolist()
+        for idx, is_dec in ((dec, True), (chk, False)):
+            if not idx:
+                continue
+            sel = torch.tensor(idx, dtype=torch.int64)
+            toks = torch.cat([torch.arange(qs[i], qs[i + 1]) for i in idx])
+            sq = q[toks.to(dev)]
+            lens = torch.tensor([qn[i] for i in idx], dtype=torch.int32)
+            sqsl = torch.zeros(len(idx) + 1, dtype=torch.int32)
+            sqsl[1:] = torch.cumsum(lens, 0)
+            stab, sctx = dtab[sel.to(dev)], dctx[sel.to(dev)]
+            sqsl = sqsl.to(dev)
+            so = torch.empty_like(sq)
+            ms = self._time(lambda: api.paged_attention(sq, r.pool.k_pool, r.pool.v_pool, stab, sctx,
+                                                        sqsl, r.scale, out=so))
+            if is_dec:
+                self.acc["dec_ms"] += ms
+                self.acc["dec_calls"] += 1
+                self.acc["dec_bytes"] += (sum(c[i] for i in idx) * kv_tok + 2 * len(idx) * r.Hq * r.d * 2
+                                          + sum(-(-c[i] // r.bs) for i in idx) * 4)
+            else:
+                self.acc["chunk_ms"] += ms
+                self.acc["chunk_calls"] += 1
+                keys = sum(qn[i] * (c[i] - qn[i]) + qn[i] * (qn[i] + 1) // 2 for i in idx)
+                self.acc["chunk_flops"] += 4 * r.Hq * r.d * keys
+        self.acc["steps"] += 1
+
+    def summary(self, hbm_peak, tensor_peak):
+        a = self.acc
+        dec_gbs = a["dec_bytes"] / (a["dec_ms"] * 1e-3) / 1e9 if a["dec_ms"] else None
+        ch_tf = a["chunk_flops"] / (a["chunk_ms"] * 1e-3) / 1e12 if a["chunk_ms"] else None
+        return {
+            "decode_rows": {"gbs": dec_gbs, "frac_of_hbm_peak": dec_gbs / hbm_peak if dec_gbs else None,
+                            "algorithmic_bytes": a["dec_bytes"], "ms": a["dec_ms"], "calls": a["dec_calls"]},
+            "chunk_rows": {"tflops": ch_tf, "frac_of_bf16_peak": ch_tf / tensor_peak if ch_tf else None,
+                           "flops": a["chunk_flops"], "ms": a["chunk_ms"], "calls": a["chunk_calls"],
+                           "share_of_attention_ms": a["chunk_ms"] / a["full_ms"] if a["full_ms"] else None},
+            "attention_ms": a["full_ms"], "steps": a["steps"],
+            "how": "after each timed step, its attention call, its decode rows alone and its chunk rows "
+                   "alone, each between CUDA events (a second run of the same trace)"}
+
+
+def oracle_steps_baseline(recorded, pool_shape, dtype, scale, budget_s, k0=None, v0=None):
+    """The oracle as it stands (float64 attention, its append and copy) over the
+    recorded steps in order, on a CPU pool, until budget_s seconds are spent."""
+    import oracle
+    kp = k0.clone() if k0 is not None else torch.zeros(pool_shape, dtype=dtype)
+    vp = v0.clone() if v0 is not None else torch.zeros(pool_shape, dtype=dtype)
+    done, toks, t0 = 0, 0, time.perf_counter()
+    for t in recorded:
+        if t["pairs"].shape[0]:
+            oracle.block_copy(kp, vp, t["pairs"])
+        oracle.kv_append(kp, vp, t["k"], t["v"], t["slots"])
+        oracle.paged_attention(t["q"], kp, vp, t["tables"], t["ctx"], t["qsl"], scale)
+        done += 1
+        toks += t["q"].shape[0]
+        if time.perf_counter() - t0 > budget_s:
+            break
+    sec = time.perf_counter() - t0
+    return {"value": toks / sec, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"the first {done} steps in order: oracle block copy, append and float64 "
+                      f"attention of every row ({toks} tokens, {sec:.1f} s)"}
+
+
 def run_serving(args, rank, world, device):
     """Scheduler-driven workloads: the continuous-batching trace (300
     iterations, Poisson arrivals, chunked prefill, preemption) or n-sample
@@ -707,7 +922,13 @@ def run_serving(args, rank, world, device):
     GPU time of copy + append + attention, and KV GB/s."""
     from paged_kv_cache_chunked_b200.drivers import ForkRunner, TraceRunner
     peak, peak_kind = measured_peak()
+    tpeak, _ = measured_tensor_peak()
     kv_tok = 8 * 128 * 2 * 2          # K+V bytes per token per layer (8 kv heads, d 128, bf16)
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    if not args.profile_run:
+        clocks.start()
+        time.sleep(0.3)
+    extra = {}
     recs = []
     if args.workload.startswith("trace"):
         # trace_swap: preempted requests' blocks go to a pinned host pool of
@@ -722,17 +943,25 @@ def run_serving(args, rank, world, device):
         swap = args.workload == "trace_swap"
         prefix = args.workload.startswith("trace_prefix")
         hybrid = args.workload == "trace_hybrid"
-        r = TraceRunner(device, preempt="swap" if swap else "recompute", num_host_blocks=8192 if swap else 0,
-                        trace=prefix_trace_requests() if prefix else None,
-                        prefix_cache=args.workload == "trace_prefix",
-                        num_blocks=6144 if hybrid else 8192, state_slots=64 if hybrid else 0)
+
+        def runner():
+            return TraceRunner(device, preempt="swap" if swap else "recompute",
+                               num_host_blocks=8192 if swap else 0,
+                               trace=prefix_trace_requests() if prefix else None,
+                               prefix_cache=args.workload == "trace_prefix",
+                               num_blocks=6144 if hybrid else 8192, state_slots=64 if hybrid else 0)
+        r = runner()
+        skip = args.warmup
+        wall = 0.0
         while r.sched.step_no < 300 and (r.pending or r.sched.has_work()):
+            t0 = time.perf_counter()
             rec = r.step()
+            if r.sched.step_no > skip:
+                wall += time.perf_counter() - t0
             if rec is not None:
                 recs.append(rec)
-        skip = min(args.warmup, len(recs) // 2)
-        recs = recs[skip:]
-        cfg = {"workload": args.workload, "steps_run": len(recs) + skip, "warmup_steps": skip,
+        recs = [x for x in recs if x.step >= skip]
+        cfg = {"workload": args.workload, "steps_run": r.sched.step_no, "warmup_steps": skip,
                "num_blocks": r.bm.num_blocks, "block_size": 16, "n_q_heads": 32, "n_kv_heads": 8,
                "head_dim": 128, "token_budget": 4096, "max_chunk": 512,
                "preempt": r.sched.preempt_mode,
@@ -758,26 +987,76 @@ def run_serving(args, rank, world, device):
         useful = sum(x.new_tokens for x in recs)
         kvb = [x.context_tokens * kv_tok for x in recs]
         copies = sum(x.copies for x in recs)
+        extra["wall_clock"] = {
+            "tokens_per_s": sum(toks) / wall, "s": wall,
+            "how": "host time of the timed scheduler steps: planning, host-to-device copies of the "
+                   "step's metadata, the kernels, and the wait for them at the end of each step"}
+        if not args.profile_run:
+            del r
+            torch.cuda.empty_cache()
+            r2 = runner()
+            split = AttentionSplit(r2, record_steps=30 if world == 1 and args.workload == "trace" else 0)
+            while r2.sched.step_no < 300 and (r2.pending or r2.sched.has_work()):
+                r2.step(on_step=split)
+            extra["attention_split"] = split.summary(peak, tpeak)
+            if split.recorded and args.cpu_baseline_seconds > 0:
+                shape = tuple(r2.pool.k_pool.shape)
+                del r2
+                torch.cuda.empty_cache()
+                extra["cpu_baseline"] = oracle_steps_baseline(split.recorded, shape, torch.bfloat16,
+                                                              128 ** -0.5, 2 * args.cpu_baseline_seconds)
     else:
         plen = 1028 if args.workload == "fork1028" else 1024
-        r = ForkRunner(device, prompt_len=plen)
-        r.prefill()
-        for _ in range(min(args.warmup, 8)):
-            r.decode_step()
-        ms, toks, kvb, copies = [], [], [], 0
-        steps = min(args.steps, r.decode_steps - min(args.warmup, 8))
-        for _ in range(steps):
-            before_unique = r.unique_blocks()
-            t, c = r.decode_step()
-            ms.append(t)
-            toks.append(len(r.seqs))
-            kvb.append(before_unique * 16 * kv_tok)     # unique (physical) blocks read
-            copies += c
+
+        def fork_run(bs, n_steps, record=0):
+            r = ForkRunner(device, prompt_len=plen, block_size=bs)
+            r.prefill()
+            for _ in range(min(args.warmup, 8)):
+                r.decode_step()
+            ms, toks, kvb, copies, rec = [], [], [], 0, []
+            steps = min(n_steps, r.decode_steps - min(args.warmup, 8))
+            for _ in range(steps):
+                before_unique = r.unique_blocks()
+                t, c = r.decode_step()
+                ms.append(t)
+                toks.append(len(r.seqs))
+                kvb.append(before_unique * bs * kv_tok)     # unique (physical) blocks read
+                copies += c
+            st = r.bm.stats()
+            info = {"block_size": bs, "tokens_per_s": sum(toks) / (sum(ms) * 1e-3),
+                    "kv_gbs_unique": sum(kvb) / (sum(ms) * 1e-3) / 1e9, "decode_steps_timed": steps,
+                    "unique_blocks": r.unique_blocks(), "clone_blocks": r.clone_blocks(),
+                    "tail_waste_slots": st["tail_waste_slots"], "copies": copies}
+            del r
+            torch.cuda.empty_cache()
+            return ms, toks, kvb, copies, info
+
+        ms, toks, kvb, copies, info = fork_run(16, args.steps)
         cfg = {"workload": args.workload, "prompts": 64, "prompt_len": plen, "samples": 4,
                "block_size": 16, "n_q_heads": 32, "n_kv_heads": 8, "head_dim": 128,
-               "decode_steps_timed": steps, "unique_blocks": r.unique_blocks(),
-               "clone_blocks": r.clone_blocks(), "copies": copies}
+               "decode_steps_timed": info["decode_steps_timed"], "unique_blocks": info["unique_blocks"],
+               "clone_blocks": info["clone_blocks"], "copies": copies}
         useful = sum(toks)
+        if not args.profile_run:
+            # "Choosing the block size": the same fork workload at blocks of 8, 16 and 32
+            extra["block_size_sweep"] = {str(b): (info if b == 16 else fork_run(b, args.steps)[4])
+                                         for b in (8, 16, 32)}
+            if world == 1 and args.cpu_baseline_seconds > 0:
+                # the oracle over the first 8 decode steps after the prefill
+                rb = ForkRunner(device, prompt_len=plen, block_size=16, decode_steps=8)
+                rb.prefill()
+                torch.cuda.synchronize()
+                k0, v0 = rb.pool.k_pool.cpu(), rb.pool.v_pool.cpu()
+                rec = []
+                for _ in range(8):
+                    rb.decode_step(on_step=lambda t, out: rec.append(
+                        {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in t.items()}), timed=False)
+                shape = tuple(rb.pool.k_pool.shape)
+                del rb
+                torch.cuda.empty_cache()
+                extra["cpu_baseline"] = oracle_steps_baseline(rec, shape, torch.bfloat16, 128 ** -0.5,
+                                                              2 * args.cpu_baseline_seconds, k0, v0)
+    clk = clocks.stop() if not args.profile_run else {"sm_mhz": None, "reasons": ["not sampled"]}
     tot_ms = sum(ms)
     per_step = sorted(t / (m * 1e-3) for t, m in zip(toks, ms))
     pct = lambda q: per_step[min(len(per_step) - 1, int(q * len(per_step)))]
@@ -790,7 +1069,12 @@ def run_serving(args, rank, world, device):
             "useful_tokens_per_s": useful / (tot_ms * 1e-3),
             "kv_gbs": sum(kvb) / (tot_ms * 1e-3) / 1e9,
             "pct_hbm": 100 * sum(kvb) / (tot_ms * 1e-3) / 1e9 / peak,
-            "timing": "per-step CUDA events around swaps + copy + append + attention; host scheduling excluded"}
+            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+            else "fallback 6.65 TB/s",
+            "timing": "per-step CUDA events around swaps + copy + append + attention; host scheduling "
+                      "excluded (see wall_clock)",
+            "clocks": dict(clk, window="the whole run: timed steps and the measurement passes after them"),
+            **extra}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -814,6 +1098,9 @@ def run_policy(args, rank, world, device):
                ("static64_4096", dict(token_budget=4096, static_batch=64))]
     pick = lambda st, k: None if st is None else {q: st[q] for q in ("p50", "p90")} if k else st
     study = {}
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    clocks.start()
+    time.sleep(0.3)
     for name, kw in configs:
         r = TraceRunner(device, trace=trace, **kw)
         while r.pending or r.sched.has_work():
@@ -830,6 +1117,7 @@ def run_policy(args, rank, world, device):
                                "ttft_steps": pick(v["ttft"], 1), "ttft_ms": pick(v["ttft_ms"], 1),
                                "itl_ms": pick(v["itl_ms"], 1)}
                          for cls, v in summ.items()}}
+    clk = clocks.stop()
     base = study["continuous_4096"]
     line = {"metric": METRIC, "value": base["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
             "steps": base["steps"], "warmup": 0, "ms_per_step": base["gpu_ms"] / base["steps"],
@@ -838,6 +1126,7 @@ def run_policy(args, rank, world, device):
             "config": {"workload": "policy", "trace": "trace_requests(arrivals 1.0/step, 300 steps, seed 1004)",
                        "requests": len(trace), "num_blocks": 8192, "block_size": 16, "max_chunk": 512},
             "study": study,
+            "clocks": dict(clk, window="every configuration of the study"),
             "timing": "per-step CUDA events around copy + append + attention, summed; host scheduling excluded"}
     if rank == 0:
         print(json.dumps(line), flush=True)

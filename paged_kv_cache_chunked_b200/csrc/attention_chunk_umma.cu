@@ -1,9 +1,10 @@
 // Paged attention for causal prefill chunks on the fifth-generation tensor
 // cores (tcgen05, operands and accumulators in tensor memory): bf16 pools,
 // head_dim 128, block_size a multiple of 16, groups g dividing 128.  Serves
+// every sequence of two or more query tokens when the block-streaming decode
+// kernel takes the one-token rows of the batch (groups of at most 8), else
 // every sequence whose query rows (q_b tokens x g heads of a kv group) span more
-// than one 16-row tile; decodes and chunks of a few tokens run in the decode
-// kernel.
+// than one 16-row tile, the rest running in the tile-streaming decode kernel.
 //
 // What is computed ["Batching and PagedAttention", "Continuous batching":
 // long prompts are split into chunks across steps; "PagedAttention & Continuous
@@ -169,6 +170,7 @@ struct UParams {
     __nv_bfloat16 *out;
     const int32_t *tables, *ctx, *qsl;
     int seq0, nseq, max_blocks, n_q_heads, n_kv_heads, group, block_size, num_blocks, num_tokens;
+    int min_rows;  // a sequence is served when its query rows (tokens x group heads) exceed this
     float scale_log2;
     int *err;
 };
@@ -253,7 +255,7 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                 const int qn = s1 - s0;
                 const bool ok = s0 >= 0 && s1 <= prm.num_tokens && qn >= 1 && c >= qn &&
                                 (long long)(c + bs - 1) / bs <= prm.max_blocks;
-                if (ok && qn * g > kTile) n = (qn * g + kUItemRows - 1) / kUItemRows * Hkv;
+                if (ok && qn * g > prm.min_rows) n = (qn * g + kUItemRows - 1) / kUItemRows * Hkv;
             }
             int inc = n;
 #pragma unroll
@@ -648,7 +650,7 @@ bool chunk_umma_applies(const pk_pool *p, const AttnArgs &a) {
     return p->umma_ok && g >= 1 && kURows % g == 0;
 }
 
-int launch_chunk_umma(const pk_pool *p, const AttnArgs &a, cudaStream_t st) {
+int launch_chunk_umma(const pk_pool *p, const AttnArgs &a, bool all_multi, cudaStream_t st) {
     UParams u;
     u.q = (const __nv_bfloat16 *)a.q;
     u.out = (__nv_bfloat16 *)a.out;
@@ -664,6 +666,7 @@ int launch_chunk_umma(const pk_pool *p, const AttnArgs &a, cudaStream_t st) {
     u.num_tokens = a.num_tokens;
     u.scale_log2 = a.scale * 1.4426950408889634f;
     u.err = p->d_err;
+    u.min_rows = all_multi ? u.group : kTile;
     for (int s0 = 0; s0 < a.num_seqs; s0 += kMaxSeqsPerLaunch) {
         u.seq0 = s0;
         u.nseq = std::min(kMaxSeqsPerLaunch, a.num_seqs - s0);

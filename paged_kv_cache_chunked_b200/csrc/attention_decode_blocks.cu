@@ -1,6 +1,9 @@
-// Paged decode attention for bf16 pools (head_dim 64/128/256) when every
-// sequence of the batch has exactly one query token and a kv head serves at
-// most 8 q heads: the decode step of continuous batching.
+// Paged decode attention for bf16 pools (head_dim 64/128/256) for the
+// sequences of a batch that have exactly one query token, when a kv head
+// serves at most 8 q heads: the decode rows of a continuous-batching step.  In
+// a batch that also holds prefill chunks (several query tokens), those
+// sequences are left to the chunk kernel, launched on the same stream after
+// this kernel and its merge kernel.
 //
 // What is computed ["PagedAttention & Continuous Batching" (study notes),
 // "Block tables"; "Batching and PagedAttention", "PagedAttention" item 4]:
@@ -94,6 +97,7 @@ struct BlkParams {
     __nv_bfloat16 *out;
     const int32_t *tables, *ctx, *qsl;
     int seq0, nseq, max_blocks, n_q_heads, n_kv_heads, group, block_size, num_blocks, num_tokens;
+    int skip_chunks;  // 1: sequences of several query tokens belong to the chunk kernel (skipped)
     int HS, NBS, ST, NPH, NS;  // geometry: heads / blocks / tokens per stage, phases, stages
     int ncta, cap_rows;
     float scale_log2;
@@ -188,10 +192,11 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                 s_qsl[i] = s0;
                 s_ctx[i] = c;
                 if (i == nseq - 1) s_qsl[nseq] = s1;
-                const bool ok = s0 >= 0 && s1 <= prm.num_tokens && s1 - s0 == 1 && c >= 1 &&
-                                (long long)(c + bs - 1) / bs <= prm.max_blocks;
+                const bool ok = s0 >= 0 && s1 <= prm.num_tokens && s1 - s0 >= 1 && c >= s1 - s0 &&
+                                (long long)(c + bs - 1) / bs <= prm.max_blocks &&
+                                (s1 - s0 == 1 || prm.skip_chunks);
                 if (!ok) record_error(prm.err, PK_ERR_BAD_INDEX);
-                else ns = NHG * ((c + ST - 1) / ST);
+                else if (s1 - s0 == 1) ns = NHG * ((c + ST - 1) / ST);
             }
             int inc = ns;
 #pragma unroll
@@ -764,8 +769,9 @@ int blocks_prepare(pk_pool *p) {
 }
 
 template <int D>
-int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, cudaStream_t st) {
+int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, bool skip_chunks, cudaStream_t st) {
     BlkParams tp{};
+    tp.skip_chunks = skip_chunks ? 1 : 0;
     tp.q = (const __nv_bfloat16 *)a.q;
     tp.out = (__nv_bfloat16 *)a.out;
     tp.tables = a.block_tables;
@@ -882,14 +888,15 @@ int decode_blocks_prepare_pool(pk_pool *p) {
 int decode_blocks_chunks_per_cta() { return 1 + kSmallPerCta; }
 
 bool decode_blocks_applies(const pk_pool *p, const AttnArgs &a) {
-    return p->blk_ok && a.num_tokens == a.num_seqs && a.n_q_heads / p->n_kv_heads <= 8;
+    return p->blk_ok && a.n_q_heads / p->n_kv_heads <= 8;
 }
 
-int launch_decode_blocks(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, cudaStream_t st) {
+int launch_decode_blocks(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, bool skip_chunks,
+                         cudaStream_t st) {
     switch (p->head_dim) {
-        case 64: return blocks_launch<64>(p, a, w, st);
-        case 128: return blocks_launch<128>(p, a, w, st);
-        case 256: return blocks_launch<256>(p, a, w, st);
+        case 64: return blocks_launch<64>(p, a, w, skip_chunks, st);
+        case 128: return blocks_launch<128>(p, a, w, skip_chunks, st);
+        case 256: return blocks_launch<256>(p, a, w, skip_chunks, st);
         default: return fail(PK_ERR_UNSUPPORTED, "decode path: head_dim %d", p->head_dim);
     }
 }

@@ -1,8 +1,10 @@
 // Host side of the tensor-core attention path: workspace layout and the
-// dispatch of a call to the chunk kernel (sequences whose query rows need more
-// than one 16-row tile), the block-streaming decode kernel (batches of one
-// query token per sequence and at most 8 q heads per kv head) and the
-// tile-streaming decode kernel (the remaining sequences of one 16-row tile).
+// dispatch of a call.  With at most 8 q heads per kv head, the one-token
+// sequences of a batch (decode rows) run on the block-streaming decode kernel,
+// and the sequences of several query tokens (prefill chunks) on the tcgen05
+// chunk kernel.  Otherwise a chunk kernel (tcgen05, or mma.sync for other head
+// dims) takes the sequences whose query rows need more than one 16-row tile,
+// and the tile-streaming decode kernel the rest.
 #include <algorithm>
 
 #include "pk_internal.h"
@@ -82,14 +84,6 @@ int launch_attention_tc(const pk_pool *p, const AttnArgs &a, cudaStream_t st) {
     if (((uintptr_t)a.workspace & 255) != 0)
         return fail(PK_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     uint8_t *ws = (uint8_t *)a.workspace;
-    // the chunk kernel has work only if some sequence's rows (q_b tokens x g
-    // heads) exceed one 16-row tile: a chunk of several tokens, or g > 16
-    const int g = a.n_q_heads / p->n_kv_heads;
-    if (a.num_tokens > a.num_seqs || g > kTile) {
-        const int rc = chunk_umma_applies(p, a) ? launch_chunk_umma(p, a, st)
-                                                : launch_chunk(p, a, ws + L.hdr_chunk, st);
-        if (rc != PK_OK) return rc;
-    }
     DecodeWs w;
     w.header = ws + L.hdr_decode;
     w.counters = (int *)(ws + L.counters);
@@ -97,7 +91,25 @@ int launch_attention_tc(const pk_pool *p, const AttnArgs &a, cudaStream_t st) {
     w.partial_lse = (float *)(ws + L.partial_lse);
     w.partial_o = (float *)(ws + L.partial_o);
     w.cap_rows = L.cap_rows;
-    if (decode_blocks_applies(p, a)) return launch_decode_blocks(p, a, w, st);
+    const int g = a.n_q_heads / p->n_kv_heads;
+    const bool has_multi = a.num_tokens > a.num_seqs;  // some sequence has several query tokens
+    const bool blocks = decode_blocks_applies(p, a);
+    if (!has_multi && blocks) return launch_decode_blocks(p, a, w, false, st);
+    if (blocks && chunk_umma_applies(p, a)) {
+        // a mixed continuous-batching step: the one-token rows stream whole
+        // blocks (block-streaming kernel + merge), then the tcgen05 kernel
+        // takes every sequence of several query tokens
+        int rc = launch_decode_blocks(p, a, w, true, st);
+        if (rc == PK_OK) rc = launch_chunk_umma(p, a, true, st);
+        return rc;
+    }
+    // otherwise: sequences whose rows (q_b tokens x g heads) exceed one 16-row
+    // tile on a chunk kernel, the rest on the tile-streaming decode kernel
+    if (has_multi || g > kTile) {
+        const int rc = chunk_umma_applies(p, a) ? launch_chunk_umma(p, a, false, st)
+                                                : launch_chunk(p, a, ws + L.hdr_chunk, st);
+        if (rc != PK_OK) return rc;
+    }
     return launch_decode(p, a, w, st);
 }
 

@@ -97,21 +97,27 @@ struct DecodeWs {
 int decode_prepare_pool(pk_pool *p);
 int decode_items_per_cta();
 int launch_decode(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, cudaStream_t st);
-// Block-streaming decode kernel: batches whose sequences all have one query
-// token and groups of at most 8 q heads per kv head.
+// Block-streaming decode kernel: the one-query-token sequences of a batch, for
+// groups of at most 8 q heads per kv head.  skip_chunks: the batch also holds
+// sequences of several query tokens, which the chunk kernel serves (without
+// it such a sequence is recorded as PK_ERR_BAD_INDEX).
 int decode_blocks_prepare_pool(pk_pool *p);
 int decode_blocks_chunks_per_cta();
 bool decode_blocks_applies(const pk_pool *p, const AttnArgs &a);
-int launch_decode_blocks(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, cudaStream_t st);
+int launch_decode_blocks(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, bool skip_chunks,
+                         cudaStream_t st);
 // 2-D TMA view of a pool (rows of head_dim bf16) with boxes of 64 columns x box_rows.
 int encode_pool_map(CUtensorMap *map, void *base, const pk_pool *p, int box_rows);
 // 3-D TMA view (column in panel, row, 64-column panel) with boxes of all panels x box_rows.
 int encode_pool_map3(CUtensorMap *map, void *base, const pk_pool *p, int box_rows);
 int chunk_prepare_pool(pk_pool *p);
 // tcgen05 chunk kernel (head_dim 128, block_size a multiple of 16, g dividing 128).
+// all_multi: serve every sequence of two or more query tokens (the one-token
+// ones go to the block-streaming decode kernel); otherwise every sequence whose
+// rows (query tokens x group heads) exceed one 16-row tile.
 int chunk_umma_prepare_pool(pk_pool *p);
 bool chunk_umma_applies(const pk_pool *p, const AttnArgs &a);
-int launch_chunk_umma(const pk_pool *p, const AttnArgs &a, cudaStream_t st);
+int launch_chunk_umma(const pk_pool *p, const AttnArgs &a, bool all_multi, cudaStream_t st);
 int launch_chunk(const pk_pool *p, const AttnArgs &a, void *header, cudaStream_t st);
 
 }  // namespace pk
