@@ -308,9 +308,11 @@ def roofline_entry(workload, attn_b, flops, avg_ms, gbs, tflops, hbm_peak, hbm_k
     the tensor pipe for prefill chunks (a dense contraction)."""
     kern = ("paged_attention call: tcgen05 chunk kernel (S and O accumulated in tensor memory)"
             if workload == "chunk512_bf16" else
-            "paged_attention call: block-streaming decode kernel + split-K merge kernel, then the "
-            "tcgen05 chunk kernel" if workload == "mixed_bf16" else
-            "paged_attention call: block-streaming decode kernel + split-K merge kernel")
+            "paged_attention call: block-streaming decode kernel (split heads merged by their last "
+            "writer), then the tcgen05 chunk kernel" if workload == "mixed_bf16" else
+            "paged_attention call: block-streaming decode kernel + split-K merge kernel"
+            if workload == "longdoc_bf16" else
+            "paged_attention call: block-streaming decode kernel (split heads merged by their last writer)")
     common = {"kernel": kern,
               "algorithmic_bytes": attn_b, "algorithmic_flops": flops, "avg_ms": avg_ms,
               "traffic": kernel_traffic(workload)}
@@ -495,20 +497,29 @@ def run_ours(args, rank, world, device):
     def attention_only():
         api.paged_attention(dq, pool.k_pool, pool.v_pool, dt_, dctx, dqsl, batch["scale"], out=out)
 
-    # append, then per window of 512 sequences: for a batch of decodes only
-    # (groups of <= 8 q heads) the block-streaming kernel and its merge kernel,
-    # else the chunk kernel (when chunks are present) and the tile-streaming
-    # decode kernel; the general kernel is one launch
+    # append, then per window of 512 sequences: with groups of <= 8 q heads the
+    # block-streaming decode kernel (then, with chunks present, the tcgen05
+    # chunk kernel), else a chunk kernel (when chunks are present) and the
+    # tile-streaming decode kernel; the general kernel is one launch
     paths = pool.paths()
     tc = bool(paths & api.PK_PATH_TENSOR_CORE)
     B = batch["context_lens"].shape[0]
     windows = (B + 511) // 512
     blocks = bool(paths & api.PK_PATH_DECODE_BLOCKS) and Hq // Hkv <= 8
     umma = bool(paths & api.PK_PATH_CHUNK_TCGEN05) and 128 % (Hq // Hkv) == 0
+    # the block-streaming kernel merges split heads itself when a window has at
+    # least a quarter as many (sequence, head group) pairs as SMs, else a merge
+    # kernel follows it; its head group is the largest power of two <= 8 that
+    # divides n_kv_heads and whose block (K + V) fits its 64 KiB stage
+    hs = 8
+    while hs > 1 and (Hkv % hs or hs * bs * d * 4 > 65536):
+        hs //= 2
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    merge_launch = 0 if 4 * min(B, 512) * (Hkv // hs) >= sms else 1
     if blocks and T == B:
-        per_window = 2                  # block-streaming decode + merge
+        per_window = 1 + merge_launch   # block-streaming decode (+ merge kernel)
     elif blocks and umma:
-        per_window = 3                  # block-streaming decode + merge, then the tcgen05 chunk kernel
+        per_window = 2 + merge_launch   # block-streaming decode (+ merge), then the tcgen05 chunk kernel
     else:
         per_window = 2 if T > B or Hq // Hkv > 16 else 1
     launches_per_step = 1 + (windows * per_window if tc else 1)
@@ -556,48 +567,97 @@ def run_ours(args, rank, world, device):
     ms_per_step = total_ms / args.steps
     value = world * (attn_b + app_b) / (ms_per_step * 1e-3) / 1e9
 
-    # end to end through the public API: pinned host inputs in, output back out
+    # end to end through the public API: every step copies its inputs from
+    # pinned host memory and its output back.  Serving overlaps those copies
+    # with the kernels, so the timed loop does too: inputs and outputs are
+    # double-buffered on the device, host-to-device copies run on one stream
+    # and device-to-host copies on another, ordered against the compute stream
+    # by events (a step's copy into a buffer waits for the kernels of the step
+    # two back that read it).  The same steps with every copy serialised on
+    # the compute stream are reported beside it.
     e2e = None
     if not args.no_e2e and not args.profile_run:
-        h_q = batch["q"].pin_memory()
-        h_k, h_v = k_new.pin_memory(), v_new.pin_memory()
-        h_slots = slots.pin_memory()
-        h_t = batch["block_tables"].pin_memory()
-        h_ctx = batch["context_lens"].pin_memory()
-        h_qsl = batch["query_start_lens"].pin_memory()
-        h_out = torch.empty_like(batch["q"]).pin_memory()
-        bufs = [torch.empty_like(x, device=device) for x in (h_q, h_k, h_v, h_slots, h_t, h_ctx, h_qsl)]
-        h2d = sum(x.numel() * x.element_size() for x in (h_q, h_k, h_v, h_slots, h_t, h_ctx, h_qsl))
-        d2h = h_out.numel() * h_out.element_size()
+        h_in = [x.pin_memory() for x in (batch["q"], k_new, v_new, slots, batch["block_tables"],
+                                         batch["context_lens"], batch["query_start_lens"])]
+        h_outs = [torch.empty_like(batch["q"]).pin_memory() for _ in range(2)]
+        sets = [[torch.empty_like(x, device=device) for x in h_in] for _ in range(2)]
+        outs = [torch.empty_like(dq) for _ in range(2)]
+        h2d = sum(x.numel() * x.element_size() for x in h_in)
+        d2h = h_outs[0].numel() * h_outs[0].element_size()
+        h2d_s, d2h_s = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        ev = {k: [torch.cuda.Event(), torch.cuda.Event()] for k in ("h2d", "comp", "d2h")}
+        used = [False, False]
 
-        def e2e_step():
-            for dst, src in zip(bufs, (h_q, h_k, h_v, h_slots, h_t, h_ctx, h_qsl)):
-                dst.copy_(src, non_blocking=True)
+        def kernels(bufs, o):
             api.paged_kv_append(bufs[1], bufs[2], bufs[3], pool=pool)
-            o = api.paged_attention(bufs[0], pool.k_pool, pool.v_pool, bufs[4], bufs[5], bufs[6],
-                                    batch["scale"], out=out)
-            h_out.copy_(o, non_blocking=True)
+            api.paged_attention(bufs[0], pool.k_pool, pool.v_pool, bufs[4], bufs[5], bufs[6],
+                                batch["scale"], out=o)
 
-        for _ in range(3):
-            e2e_step()
-        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if dist:
-            tdist.barrier()
-        torch.cuda.synchronize(device)
-        s2.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e2.record(stream)
-        torch.cuda.synchronize(device)
-        e_ms = s2.elapsed_time(e2)
-        if dist:
-            t = torch.tensor([e_ms], device=device)
-            tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e_ms /= args.steps
+        def e2e_step(i):
+            j = i % 2
+            with torch.cuda.stream(h2d_s):
+                if used[j]:
+                    h2d_s.wait_event(ev["comp"][j])        # the step two back has read set j
+                for dst, src in zip(sets[j], h_in):
+                    dst.copy_(src, non_blocking=True)
+                ev["h2d"][j].record(h2d_s)
+            stream.wait_event(ev["h2d"][j])
+            if used[j]:
+                stream.wait_event(ev["d2h"][j])           # out[j] of the step two back is home
+            kernels(sets[j], outs[j])
+            ev["comp"][j].record(stream)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(ev["comp"][j])
+                h_outs[j].copy_(outs[j], non_blocking=True)
+                ev["d2h"][j].record(d2h_s)
+            used[j] = True
+
+        def timed(fn):
+            s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            if dist:
+                tdist.barrier()
+            torch.cuda.synchronize(device)
+            s2.record(stream)
+            h2d_s.wait_event(s2)
+            d2h_s.wait_event(s2)
+            for i in range(args.steps):
+                fn(i)
+            for x in (h2d_s, d2h_s):
+                done = torch.cuda.Event()
+                done.record(x)
+                stream.wait_event(done)
+            e2.record(stream)
+            torch.cuda.synchronize(device)
+            e_ms = s2.elapsed_time(e2)
+            if dist:
+                t = torch.tensor([e_ms], device=device)
+                tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+                e_ms = float(t.item())
+            return e_ms / args.steps
+
+        def serial_step(i):
+            for dst, src in zip(sets[0], h_in):
+                dst.copy_(src, non_blocking=True)
+            kernels(sets[0], outs[0])
+            h_outs[0].copy_(outs[0], non_blocking=True)
+
+        for i in range(4):
+            e2e_step(i)
+        e_ms = timed(e2e_step)
+        ok = bool(torch.equal(h_outs[0], h_outs[1])) and bool(torch.isfinite(h_outs[0].float()).all())
+        for i in range(3):
+            serial_step(i)
+        s_ms = timed(serial_step)
         e2e = {"value": world * (attn_b + app_b) / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
-               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-        assert torch.isfinite(h_out.float()).all()
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "serialized_ms_per_step": s_ms,
+               "serialized_value": world * (attn_b + app_b) / (s_ms * 1e-3) / 1e9,
+               "how": "per step: host-to-device copies of q, the new K/V, slots, tables, lengths from "
+                      "pinned memory; append + attention; device-to-host copy of the output; copies "
+                      "overlapped with the neighbouring steps' kernels on two copy streams "
+                      "(double-buffered device inputs and outputs); serialized_*: the same with every "
+                      "copy on the compute stream"}
+        assert ok, "end-to-end outputs differ between the two buffers"
 
     if rank != 0:
         return
@@ -615,6 +675,8 @@ def run_ours(args, rank, world, device):
                                   f"more than the 126 MB L2"),
         "pct_hbm": 100.0 * value / world / peak,
         "tokens_per_s": world * T / (ms_per_step * 1e-3),
+        "pool_paths": {n: bool(paths & getattr(api, "PK_PATH_" + n))
+                       for n in ("TENSOR_CORE", "DECODE_BLOCKS", "CHUNK_TCGEN05")},
         "roofline": roofline_entry(args.workload, attn_b, flops, attn_avg_ms, achieved, tflops,
                                    peak, peak_kind),
         "attention_tflops": tflops,
@@ -812,26 +874,32 @@ def run_kvops(args, rank, world, device):
 class AttentionSplit:
     """on_step hook of a trace run: after each step's timed region, times the
     step's attention call again, then its decode rows alone (sequences of one
-    query token) and its chunk rows alone (several query tokens), each between
-    CUDA events on the stream, into scratch outputs (the pool is only read).
-    The pool is the one the step just wrote, so part of it may still sit in L2
-    (a step reads several hundred MB of KV against the 126 MB L2)."""
+    query token) and its chunk rows alone (several query tokens), each run
+    twice back to back between CUDA events on the stream, into scratch outputs
+    (the pool is only read).  The second run is the kernel's figure; the first
+    follows the host's planning gap, as every serving step does, and is kept
+    as the in-loop figure.  A step reads several hundred MB of KV against the
+    126 MB L2, so the repeat finds little of it in L2."""
 
     def __init__(self, runner, record_steps=0):
         self.r = runner
         self.acc = dict(full_ms=0.0, dec_ms=0.0, chunk_ms=0.0, dec_bytes=0, chunk_flops=0, steps=0,
-                        dec_calls=0, chunk_calls=0)
+                        dec_calls=0, chunk_calls=0, dec_first_ms=0.0, chunk_first_ms=0.0)
         self.record_steps = record_steps
         self.recorded = []
+        self._first = 0.0
 
     def _time(self, fn):
         st = torch.cuda.current_stream(self.r.device)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(st)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record(st)
         fn()
-        b.record(st)
-        b.synchronize()
-        return a.elapsed_time(b)
+        ev[1].record(st)
+        fn()
+        ev[2].record(st)
+        ev[2].synchronize()
+        self._first = ev[0].elapsed_time(ev[1])
+        return ev[1].elapsed_time(ev[2])
 
     def __call__(self, plan, t, out):
         from paged_kv_cache_chunked_b200 import api
@@ -868,11 +936,13 @@ class AttentionSplit:
                                                         sqsl, r.scale, out=so))
             if is_dec:
                 self.acc["dec_ms"] += ms
+                self.acc["dec_first_ms"] += self._first
                 self.acc["dec_calls"] += 1
                 self.acc["dec_bytes"] += (sum(c[i] for i in idx) * kv_tok + 2 * len(idx) * r.Hq * r.d * 2
                                           + sum(-(-c[i] // r.bs) for i in idx) * 4)
             else:
                 self.acc["chunk_ms"] += ms
+                self.acc["chunk_first_ms"] += self._first
                 self.acc["chunk_calls"] += 1
                 keys = sum(qn[i] * (c[i] - qn[i]) + qn[i] * (qn[i] + 1) // 2 for i in idx)
                 self.acc["chunk_flops"] += 4 * r.Hq * r.d * keys
@@ -882,15 +952,19 @@ class AttentionSplit:
         a = self.acc
         dec_gbs = a["dec_bytes"] / (a["dec_ms"] * 1e-3) / 1e9 if a["dec_ms"] else None
         ch_tf = a["chunk_flops"] / (a["chunk_ms"] * 1e-3) / 1e12 if a["chunk_ms"] else None
+        first_gbs = a["dec_bytes"] / (a["dec_first_ms"] * 1e-3) / 1e9 if a["dec_first_ms"] else None
         return {
             "decode_rows": {"gbs": dec_gbs, "frac_of_hbm_peak": dec_gbs / hbm_peak if dec_gbs else None,
-                            "algorithmic_bytes": a["dec_bytes"], "ms": a["dec_ms"], "calls": a["dec_calls"]},
+                            "algorithmic_bytes": a["dec_bytes"], "ms": a["dec_ms"], "calls": a["dec_calls"],
+                            "gbs_first_call_after_host_gap": first_gbs},
             "chunk_rows": {"tflops": ch_tf, "frac_of_bf16_peak": ch_tf / tensor_peak if ch_tf else None,
                            "flops": a["chunk_flops"], "ms": a["chunk_ms"], "calls": a["chunk_calls"],
+                           "ms_first_call_after_host_gap": a["chunk_first_ms"],
                            "share_of_attention_ms": a["chunk_ms"] / a["full_ms"] if a["full_ms"] else None},
             "attention_ms": a["full_ms"], "steps": a["steps"],
-            "how": "after each timed step, its attention call, its decode rows alone and its chunk rows "
-                   "alone, each between CUDA events (a second run of the same trace)"}
+            "how": "after each timed step (a second run of the same trace): the step's attention call, "
+                   "then its decode rows alone and its chunk rows alone, each twice back to back between "
+                   "CUDA events; the second of each pair is the kernel figure"}
 
 
 def oracle_steps_baseline(recorded, pool_shape, dtype, scale, budget_s, k0=None, v0=None):
@@ -987,10 +1061,19 @@ def run_serving(args, rank, world, device):
         useful = sum(x.new_tokens for x in recs)
         kvb = [x.context_tokens * kv_tok for x in recs]
         copies = sum(x.copies for x in recs)
+        plan_s = sum(x.host_plan_ms for x in recs) / 1e3
+        values_s = sum(x.host_values_ms for x in recs) / 1e3
+        values_gpu_s = sum(x.values_gpu_ms or 0.0 for x in recs) / 1e3
         extra["wall_clock"] = {
-            "tokens_per_s": sum(toks) / wall, "s": wall,
-            "how": "host time of the timed scheduler steps: planning, host-to-device copies of the "
-                   "step's metadata, the kernels, and the wait for them at the end of each step"}
+            "tokens_per_s": sum(toks) / wall, "s": wall, "steps": len(recs),
+            "host_planning_s": plan_s, "value_generation_launch_s": values_s,
+            "value_generation_gpu_s": values_gpu_s,
+            "tokens_per_s_without_value_generation_gpu_time": sum(toks) / (wall - values_gpu_s),
+            "how": "host time of the timed scheduler steps, each ending in a wait for its kernels: "
+                   "planning (schedule + complete, host_planning_s), launching the generation of the "
+                   "step's synthetic q/k/v on the GPU (a stand-in for the model; its kernels run "
+                   "before the step's timed region), host-to-device copies of the step's metadata, "
+                   "the step's kernels and the wait"}
         if not args.profile_run:
             del r
             torch.cuda.empty_cache()

@@ -1,6 +1,6 @@
 // Paged attention for causal prefill chunks on the fifth-generation tensor
 // cores (tcgen05, operands and accumulators in tensor memory): bf16 pools,
-// head_dim 128, block_size a multiple of 16, groups g dividing 128.  Serves
+// head_dim 64 or 128, block_size a multiple of 16, groups g dividing 128.  Serves
 // every sequence of two or more query tokens when the block-streaming decode
 // kernel takes the one-token rows of the batch (groups of at most 8), else
 // every sequence whose query rows (q_b tokens x g heads of a kv group) span more
@@ -15,11 +15,11 @@
 // Structure.  A work item is 256 query rows (pairs (token, head of the
 // group), token-major) of one (sequence, kv head), as two 128-row tiles; CTA i
 // takes items i, i + gridDim.x, ...  Per 128-key stage:
-//   - three producer warps (9, 10, 11) load the stage's eight 16-key blocks by
-//     TMA: K as two 2-D boxes per block (one per 64-column panel; warps 9 and
-//     10) into the canonical K-major 128-byte-swizzled layout [panel][128
-//     keys][128 B], V as one 3-D box per block [block][panel][16 keys][128 B]
-//     (warp 11).  Lane j of a producer looks up and issues block j, so a
+//   - producer warps load the stage's eight 16-key blocks by TMA: K as one
+//     2-D box per block and 64-column panel (warp 9 panel 0, warp 10 panel 1
+//     at head dim 128) into the canonical K-major 128-byte-swizzled layout
+//     [panel][128 keys][128 B], V as one 3-D box per block [block][panel][16
+//     keys][128 B] (warp 11).  Lane j of a producer looks up and issues block j, so a
 //     stage's eight table lookups and boxes go out together.  K and V have
 //     rings of their own: a K slot is refilled once the stage's S has
 //     completed, a V slot once its P V has.  On a stage that runs past the
@@ -27,8 +27,8 @@
 //     may hold anything) before it releases the stage;
 //   - one thread of the MMA warp issues, per row tile t, O_t += P_t V of the
 //     previous stage (A = P_t read from tensor memory, B = V MN-major; M 128,
-//     N 128, eight K-steps) and then S_t = Q_t K^T of this stage (M 128, N 128,
-//     eight K-steps) into the same tensor-memory columns: the tensor core runs
+//     N = head dim, eight K-steps) and then S_t = Q_t K^T of this stage (M 128,
+//     N 128, head dim / 16 K-steps) into the same tensor-memory columns: the tensor core runs
 //     one thread's MMAs in order, so S_t overwrites P_t only after P_t V has
 //     read it.  Tile 1's MMAs run while tile 0's softmax works and the other
 //     way round;
@@ -54,7 +54,6 @@ namespace {
 
 using namespace tc;
 
-constexpr int kUD = 128;                // head dim
 constexpr int kURows = 128;             // query rows per row tile (UMMA M)
 constexpr int kUTiles = 2;              // row tiles per item: 256 query rows share each KV stage
 constexpr int kUItemRows = kURows * kUTiles;
@@ -63,7 +62,7 @@ constexpr int kUBlk = kUKeys / 16;      // 16-key blocks per stage
 constexpr int kUKStages = 2;            // K ring: a slot is free once the stage's S = Q K^T has completed
 constexpr int kUVStages = 2;            // V ring: a slot is free once the stage's O += P V has completed
 constexpr int kUMma = 8;                // warp 8: tensor memory and MMA issue
-constexpr int kUProd0 = 9;              // warps 9, 10: K panel 0, 1; warp 11: V
+constexpr int kUProd0 = 9;              // warps 9, 10: K panel 0, 1 (head dim 64: warp 9 only); warp 11: V
 constexpr int kUThreads = 12 * 32;      // warps 0..3 and 4..7: softmax of row tile 0 and 1
 constexpr uint32_t kUTmemCols = 512;    // S[t] (P[t] over its first 64 columns) at 128 t, O[t] at 256 + 128 t
 constexpr float kURescaleLog2 = 8.f;
@@ -75,27 +74,34 @@ constexpr float kURescaleLog2 = 8.f;
 constexpr int kURegLaunch = 168, kURegSoftmax = 176, kURegOther = 152;
 static_assert(256 * kURegSoftmax + 128 * kURegOther <= kUThreads * kURegLaunch, "register split");
 
-constexpr uint32_t kUQBytes = kURows * kUD * 2;       // per tile: [panel][128 rows][128 B]
-constexpr uint32_t kUKBytes = kUKeys * kUD * 2;       // [panel][128 keys][128 B]
-constexpr uint32_t kUKPanel = kUKeys * 128;           // bytes of one K panel
-constexpr uint32_t kUVBytes = kUKeys * kUD * 2;       // [block][panel][16 keys][128 B]
-constexpr uint32_t kUOffQ = 0;
-constexpr uint32_t kUOffK = kUOffQ + kUTiles * kUQBytes;
-constexpr uint32_t kUOffV = kUOffK + kUKStages * kUKBytes;
-constexpr uint32_t kUOffPlan = kUOffV + kUVStages * kUVBytes;
-constexpr uint32_t kUOffBar = kUOffPlan + (3 * kPlanLen * 4 + 15) / 16 * 16;
-// barriers: k_full[K slot], k_empty[K slot], v_full[V slot], v_empty[V slot],
-// v_tma; per row tile: s_full, p_full, q_full, o_full, o_free; mma_done
+// Shared-memory layout and instruction descriptors for head dim D (64 or 128).
+template <int D>
+struct UGeo {
+    static constexpr int kPanels = D / 64;                    // 64-column (128-byte) panels
+    static constexpr uint32_t QBytes = kURows * D * 2;        // per tile: [panel][128 rows][128 B]
+    static constexpr uint32_t KBytes = kUKeys * D * 2;        // [panel][128 keys][128 B]
+    static constexpr uint32_t KPanel = kUKeys * 128;          // bytes of one K panel
+    static constexpr uint32_t VBlock = 16 * D * 2;            // one 16-key block of V: [panel][16 keys][128 B]
+    static constexpr uint32_t VBytes = kUKeys * D * 2;        // [block][panel][16 keys][128 B]
+    static constexpr uint32_t OffQ = 0;
+    static constexpr uint32_t OffK = OffQ + kUTiles * QBytes;
+    static constexpr uint32_t OffV = OffK + kUKStages * KBytes;
+    static constexpr uint32_t OffPlan = OffV + kUVStages * VBytes;
+    static constexpr uint32_t OffBar = OffPlan + (3 * kPlanLen * 4 + 15) / 16 * 16;
+    // barriers: k_full[K slot], k_empty[K slot], v_full[V slot], v_empty[V slot],
+    // v_tma; per row tile: s_full, p_full, q_full, o_full, o_free; mma_done
+    static constexpr uint32_t PerTileBars = 5;
+    static constexpr uint32_t NumBars = 2 * kUKStages + 2 * kUVStages + 1 + kUTiles * PerTileBars + 1;
+    static constexpr uint32_t OffMisc = OffBar + NumBars * 8;  // tensor memory address, abort flag
+    static constexpr uint32_t Smem = OffMisc + 16 + 1024;      // + alignment slack
+    static_assert(Smem <= 227 * 1024 - 64, "chunk kernel shared memory");
+    // O += P V (kind::f16): fp32 accumulate, bf16 A and B, B MN-major, M = 128, N = D
+    static constexpr uint32_t IdescPV =
+        (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | (((uint32_t)D >> 3) << 17) | ((128u >> 4) << 24);
+};
 constexpr uint32_t kUPerTileBars = 5;
-constexpr uint32_t kUNumBars = 2 * kUKStages + 2 * kUVStages + 1 + kUTiles * kUPerTileBars + 1;
-constexpr uint32_t kUOffMisc = kUOffBar + kUNumBars * 8;  // tensor memory address, abort flag
-constexpr uint32_t kUSmem = kUOffMisc + 16 + 1024;        // + alignment slack
-static_assert(kUSmem <= 227 * 1024 - 64, "chunk kernel shared memory");
-
-// instruction descriptors (kind::f16): fp32 accumulate, bf16 A and B, M = 128, N = 128
+// S = Q K^T (kind::f16): fp32 accumulate, bf16 A and B, M = 128, N = 128 keys
 constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
-constexpr uint32_t kIdescPV =
-    (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);  // B MN-major
 
 // Shared-memory matrix descriptor (128-byte swizzle) as two 32-bit words: the low
 // word holds the start address and the leading byte offset (both >> 4), the high
@@ -165,6 +171,35 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
                  : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
                  : "memory");
 }
+// ---- packed f32x2 arithmetic ----------------------------------------------
+// The softmax warps are bound by instruction issue, so their per-key work uses
+// the packed two-float forms: one instruction scales and offsets two scores,
+// one adds two probabilities to the row sum.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &a, float &b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 struct UParams {
     const __nv_bfloat16 *q;
     __nv_bfloat16 *out;
@@ -184,19 +219,21 @@ struct UTileBars {
     uint64_t *s_full, *p_full, *q_full, *o_full, *o_free;
 };
 
+template <int D>
 __global__ void __launch_bounds__(kUThreads, 1)
 attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D, 16-row boxes
                             const __grid_constant__ CUtensorMap tmv3,  // V: 3-D, 16 rows x 2 panels
                             const UParams prm) {
+    using G = UGeo<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = prm.group, Hq = prm.n_q_heads, Hkv = prm.n_kv_heads, bs = prm.block_size;
     const int nseq = prm.nseq;
-    int *item_pre = (int *)(sm + kUOffPlan);
+    int *item_pre = (int *)(sm + G::OffPlan);
     int *s_qsl = item_pre + kPlanLen;
     int *s_ctx = s_qsl + kPlanLen;
-    uint64_t *k_full = (uint64_t *)(sm + kUOffBar);
+    uint64_t *k_full = (uint64_t *)(sm + G::OffBar);
     uint64_t *k_empty = k_full + kUKStages;
     uint64_t *v_full = k_empty + kUKStages;
     uint64_t *v_empty = v_full + kUVStages;
@@ -207,13 +244,13 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
         uint64_t *q = tile_bars + t * kUPerTileBars;
         return UTileBars{q, q + 1, q + 2, q + 3, q + 4};
     };
-    uint32_t *tmem_slot = (uint32_t *)(sm + kUOffMisc);
-    volatile int *abort_flag = (volatile int *)(sm + kUOffMisc + 4);
+    uint32_t *tmem_slot = (uint32_t *)(sm + G::OffMisc);
+    volatile int *abort_flag = (volatile int *)(sm + G::OffMisc + 4);
     __shared__ int s_nitems;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kUKStages; ++s) {
-            mbar_init(&k_full[s], 2);  // both K producers
+            mbar_init(&k_full[s], G::kPanels);  // one K producer per panel
             mbar_init(&k_empty[s], 1);
         }
         for (int s = 0; s < kUVStages; ++s) {
@@ -301,13 +338,14 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
         // [block][panel][16 keys][128 B]
         const int p = warp - kUProd0;
         const bool is_v = p == 2;
+        const bool active = is_v || p < G::kPanels;  // head dim 64: one K panel, warp 10 idles
         const int nst = is_v ? kUVStages : kUKStages;
         uint64_t *full = is_v ? v_full : k_full;
         uint64_t *empty = is_v ? v_empty : k_empty;
         if (lane == 0) prefetch_tmap(is_v ? &tmv3 : &tmk2);
         int n = 0, ntail = 0;
         bool ok = true;
-        for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+        for (int idx = blockIdx.x; active && ok && idx < n_items; idx += gridDim.x) {
             UItem it;
             item_of(idx, it);
             const int32_t *table = prm.tables + (long long)(prm.seq0 + it.b) * prm.max_blocks;
@@ -350,18 +388,18 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                 const uint32_t nload = (uint32_t)__popc(__ballot_sync(0xffffffffu, has));
                 const int valid_keys = it.c - j * kUKeys;  // warp-uniform
                 const bool tail = is_v && valid_keys < kUKeys;
-                uint8_t *dst = is_v ? sm + kUOffV + (size_t)s * kUVBytes
-                                    : sm + kUOffK + (size_t)s * kUKBytes + p * kUKPanel;
+                uint8_t *dst = is_v ? sm + G::OffV + (size_t)s * G::VBytes
+                                    : sm + G::OffK + (size_t)s * G::KBytes + p * G::KPanel;
                 uint64_t *bar = tail ? v_tma : &full[s];
                 if (lane == 0) {
                     if (nload == 0) mbar_arrive(bar);  // keys past the context: nothing to load
-                    else mbar_arrive_expect_tx(bar, nload * (is_v ? 4096u : 2048u));
+                    else mbar_arrive_expect_tx(bar, nload * (is_v ? G::VBlock : 2048u));
                 }
                 __syncwarp();
                 // lane jb issues block jb's box: a warp's TMA instructions issue one
                 // at a time, so eight lanes start a stage's boxes together
                 if (has) {
-                    if (is_v) tma_load_3d(dst + lane * 4096, &tmv3, 0, y, 0, bar);
+                    if (is_v) tma_load_3d(dst + lane * G::VBlock, &tmv3, 0, y, 0, bar);
                     else tma_load_2d(dst + lane * 2048, &tmk2, p * 64, y, bar);
                 }
                 __syncwarp();
@@ -375,9 +413,9 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                         ok = false;
                         break;
                     }
-                    for (int i = lane; i < (kUKeys - valid_keys) * 16; i += 32) {
-                        const int key = valid_keys + i / 16, ch = i % 16;
-                        *(uint4 *)(dst + (key >> 4) * 4096 + (ch >> 3) * 2048 + (key & 15) * 128 + (ch & 7) * 16) =
+                    for (int i = lane; i < (kUKeys - valid_keys) * (D / 8); i += 32) {
+                        const int key = valid_keys + i / (D / 8), ch = i % (D / 8);
+                        *(uint4 *)(dst + (key >> 4) * G::VBlock + (ch >> 3) * 2048 + (key & 15) * 128 + (ch & 7) * 16) =
                             make_uint4(0u, 0u, 0u, 0u);
                     }
                     fence_proxy_async();
@@ -400,7 +438,7 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
         const UTileBars B = tb(t);
         const uint32_t row_t = tmem + ((uint32_t)(sp * 32) << 16);
         const uint32_t s_col = (uint32_t)(t * 128), o_col = (uint32_t)(256 + t * 128);
-        uint8_t *qbuf = sm + kUOffQ + t * kUQBytes;
+        uint8_t *qbuf = sm + G::OffQ + t * G::QBytes;
         int n = 0, n_item = 0;
         bool ok = true;
         for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++n_item) {
@@ -410,13 +448,13 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
             const bool valid = R < it.rows;
             const int tok = valid ? R / g : 0, hh = valid ? R % g : 0;
             const int pos = it.c - it.qn + tok;
-            const long long qrow = ((long long)(it.qs0 + tok) * Hq + it.kvh * g + hh) * kUD;
+            const long long qrow = ((long long)(it.qs0 + tok) * Hq + it.kvh * g + hh) * D;
             // Q row into the K-major 128-byte-swizzled layout (the previous item's
             // MMAs have completed: its o_full was seen)
             {
                 const uint4 *src = (const uint4 *)(prm.q + qrow);
 #pragma unroll
-                for (int ch = 0; ch < 16; ++ch) {
+                for (int ch = 0; ch < D / 8; ++ch) {
                     const uint4 v = valid ? __ldg(src + ch) : make_uint4(0u, 0u, 0u, 0u);
                     const int pn = ch >> 3, c8 = ch & 7;
                     *(uint4 *)(qbuf + pn * (kURows * 128) + r * 128 + ((c8 ^ (r & 7)) << 4)) = v;
@@ -453,11 +491,10 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                 for (int i = 0; i < 8; ++i) mt[i] = fmaxf(__uint_as_float(sa[i]), __uint_as_float(sb[i]));
 #pragma unroll
                 for (int i = 8; i < 64; ++i)
-                    mt[i & 7] = fmaxf(mt[i & 7], fmaxf(__uint_as_float(sa[i]), __uint_as_float(sb[i])));
-#pragma unroll
-                for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-                    for (int i = 0; i < w; ++i) mt[i] = fmaxf(mt[i], mt[i + w]);
+                    mt[i & 7] = fmax3(mt[i & 7], __uint_as_float(sa[i]), __uint_as_float(sb[i]));
+                mt[0] = fmax3(mt[0], mt[1], mt[2]);
+                mt[3] = fmax3(mt[3], mt[4], mt[5]);
+                mt[0] = fmax3(mt[0], mt[3], fmaxf(mt[6], mt[7]));
                 const float mx = mt[0] * prm.scale_log2;
                 float alpha = 1.f;
                 bool resc = false;
@@ -470,7 +507,8 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                 }
                 const float bm = m == -INFINITY ? 0.f : m;
                 const float sl = prm.scale_log2;
-                float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+                const uint64_t sl2 = f2_pack(sl, sl), nbm2 = f2_pack(-bm, -bm);
+                uint64_t ps2[2] = {0ull, 0ull};  // two packed partial sums (0.f, 0.f)
                 // P as bf16 over the first 64 columns of S: keys 16c..16c+15 in
                 // columns 8c..8c+7, two keys per column, the even one in the low half
 #pragma unroll
@@ -481,17 +519,24 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                         const int key = 16 * c + 2 * i;
                         const float x0 = __uint_as_float(key < 64 ? sa[key] : sb[key - 64]);
                         const float x1 = __uint_as_float(key + 1 < 64 ? sa[key + 1] : sb[key + 1 - 64]);
-                        const float p0 = fast_exp2(fmaf(x0, sl, -bm)), p1 = fast_exp2(fmaf(x1, sl, -bm));
-                        ps4[(2 * i) & 3] += p0;
-                        ps4[(2 * i + 1) & 3] += p1;
+                        const uint64_t y = f2_fma(f2_pack(x0, x1), sl2, nbm2);  // x * scale - m, log2 units
+                        float y0, y1;
+                        f2_unpack(y, y0, y1);
+                        const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
+                        ps2[i & 1] = f2_add(ps2[i & 1], f2_pack(p0, p1));
                         pk[i] = pack_bf16(p0, p1);
                     }
                     tmem_st8(row_t + s_col + (uint32_t)(8 * c), pk);
                 }
-                l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
+                {
+                    float a0, a1, b0, b1;
+                    f2_unpack(ps2[0], a0, a1);
+                    f2_unpack(ps2[1], b0, b1);
+                    l += (a0 + a1) + (b0 + b1);
+                }
                 if (resc) {  // O_t is stable: its last P V completed before this S did
 #pragma unroll 1
-                    for (int q8 = 0; q8 < 8; ++q8) {
+                    for (int q8 = 0; q8 < D / 16; ++q8) {
                         uint32_t ov[16];
                         tmem_ld16(row_t + o_col + (uint32_t)(q8 * 16), ov);
                         tmem_wait_ld();
@@ -515,7 +560,7 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
             const float inv = l > 0.f ? 1.f / l : 0.f;
             uint4 *dst = (uint4 *)(prm.out + qrow);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
+            for (int q4 = 0; q4 < D / 32; ++q4) {
                 uint32_t ov[32];
                 tmem_ld32(row_t + o_col + (uint32_t)(q4 * 32), ov);
                 tmem_wait_ld();
@@ -553,21 +598,21 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                 const int s = nn % kUVStages;
                 if (t == 0 && !mbar_wait(&v_full[s], (uint32_t)(nn / kUVStages) & 1)) return false;
                 tc_after();
-                const uint32_t vlo = sdesc_lo(smem_u32(sm + kUOffV + (size_t)s * kUVBytes), 2048);
+                const uint32_t vlo = sdesc_lo(smem_u32(sm + G::OffV + (size_t)s * G::VBytes), 2048);
 #pragma unroll
                 for (int kp = 0; kp < kUBlk; ++kp)
-                    umma_ts(tmem + 256u + (uint32_t)(t * 128), tmem + (uint32_t)(t * 128 + 8 * kp), vlo + kp * 256,
-                            kIdescPV, (first && kp == 0) ? 0u : 1u);
+                    umma_ts(tmem + 256u + (uint32_t)(t * 128), tmem + (uint32_t)(t * 128 + 8 * kp),
+                            vlo + kp * (G::VBlock >> 4), G::IdescPV, (first && kp == 0) ? 0u : 1u);
                 return true;
             };
             // S_t = Q_t K^T of the stage in K slot s, over S_t's (and P_t's) columns
             auto s_mma = [&](int t, int s) {
-                const uint32_t klo = sdesc_lo(smem_u32(sm + kUOffK + (size_t)s * kUKBytes), 16);
-                const uint32_t qlo = sdesc_lo(smem_u32(sm + kUOffQ + t * kUQBytes), 16);
+                const uint32_t klo = sdesc_lo(smem_u32(sm + G::OffK + (size_t)s * G::KBytes), 16);
+                const uint32_t qlo = sdesc_lo(smem_u32(sm + G::OffQ + t * G::QBytes), 16);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
+                for (int kk = 0; kk < D / 16; ++kk)  // 16-column K-steps, four per 64-column panel
                     umma_ss(tmem + (uint32_t)(t * 128), qlo + (uint32_t)((kk >> 2) * (kURows * 128) + (kk & 3) * 32) / 16,
-                            klo + (uint32_t)((kk >> 2) * kUKPanel + (kk & 3) * 32) / 16, kIdescS, kk > 0 ? 1u : 0u);
+                            klo + (uint32_t)((kk >> 2) * G::KPanel + (kk & 3) * 32) / 16, kIdescS, kk > 0 ? 1u : 0u);
                 umma_commit(tb(t).s_full);
             };
             for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++n_item) {
@@ -621,26 +666,36 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
     }
 }
 
-}  // namespace
-
-// Serves bf16 pools with head_dim 128 and 16-row tile boxes (block_size a
-// multiple of 16), and groups dividing 128; PK_CHUNK_MMA_SYNC=1 selects the
-// mma.sync chunk kernel instead.
-int chunk_umma_prepare_pool(pk_pool *p) {
-    p->umma_ok = false;
-    const char *e = getenv("PK_CHUNK_MMA_SYNC");
-    if (p->head_dim != kUD || !p->tile_map3d || (e && e[0] == '1')) return PK_OK;
-    cudaError_t ce = cudaFuncSetAttribute(attention_chunk_umma_kernel,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kUSmem);
+template <int D>
+int umma_prepare(pk_pool *p, bool &ok) {
+    ok = false;
+    cudaError_t ce = cudaFuncSetAttribute(attention_chunk_umma_kernel<D>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)UGeo<D>::Smem);
     if (ce != cudaSuccess) return cuda_fail(ce, "set chunk (tcgen05) smem size");
     // the warpgroups' register split assumes this launch register count
     cudaFuncAttributes fa;
-    ce = cudaFuncGetAttributes(&fa, attention_chunk_umma_kernel);
+    ce = cudaFuncGetAttributes(&fa, attention_chunk_umma_kernel<D>);
     if (ce != cudaSuccess) return cuda_fail(ce, "chunk (tcgen05) attributes");
-    if (fa.numRegs != kURegLaunch) return PK_OK;
+    ok = fa.numRegs == kURegLaunch;
+    return PK_OK;
+}
+
+}  // namespace
+
+// Serves bf16 pools with head_dim 64 or 128 and 16-row tile boxes (block_size a
+// multiple of 16), and groups dividing 128; PK_CHUNK_MMA_SYNC=1 selects the
+// mma.sync chunk kernel instead.  Head dim 256 does not fit: two 128-row tiles
+// would need 2 x (128 S + 256 O) tensor-memory columns of the 512.
+int chunk_umma_prepare_pool(pk_pool *p) {
+    p->umma_ok = false;
+    const char *e = getenv("PK_CHUNK_MMA_SYNC");
+    if ((p->head_dim != 64 && p->head_dim != 128) || !p->tile_map3d || (e && e[0] == '1')) return PK_OK;
+    bool ok = false;
+    const int rc = p->head_dim == 64 ? umma_prepare<64>(p, ok) : umma_prepare<128>(p, ok);
+    if (rc != PK_OK || !ok) return rc;
     // K as 2-D 16-row boxes of one 64-column panel; V uses the pool's 3-D tile map
-    const int rc = encode_pool_map(&p->tmap_k2, p->k_base, p, kTile);
-    if (rc != PK_OK) return rc;
+    const int rc2 = encode_pool_map(&p->tmap_k2, p->k_base, p, kTile);
+    if (rc2 != PK_OK) return rc2;
     p->umma_ok = true;
     return PK_OK;
 }
@@ -670,7 +725,10 @@ int launch_chunk_umma(const pk_pool *p, const AttnArgs &a, bool all_multi, cudaS
     for (int s0 = 0; s0 < a.num_seqs; s0 += kMaxSeqsPerLaunch) {
         u.seq0 = s0;
         u.nseq = std::min(kMaxSeqsPerLaunch, a.num_seqs - s0);
-        attention_chunk_umma_kernel<<<p->sm_count, kUThreads, kUSmem, st>>>(p->tmap_k2, p->tmap_v, u);
+        if (p->head_dim == 64)
+            attention_chunk_umma_kernel<64><<<p->sm_count, kUThreads, UGeo<64>::Smem, st>>>(p->tmap_k2, p->tmap_v, u);
+        else
+            attention_chunk_umma_kernel<128><<<p->sm_count, kUThreads, UGeo<128>::Smem, st>>>(p->tmap_k2, p->tmap_v, u);
     }
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? PK_OK : cuda_fail(e, "chunk attention (tcgen05) launch");

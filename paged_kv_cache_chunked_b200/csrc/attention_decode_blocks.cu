@@ -3,7 +3,7 @@
 // serves at most 8 q heads: the decode rows of a continuous-batching step.  In
 // a batch that also holds prefill chunks (several query tokens), those
 // sequences are left to the chunk kernel, launched on the same stream after
-// this kernel and its merge kernel.
+// this kernel.
 //
 // What is computed ["PagedAttention & Continuous Batching" (study notes),
 // "Block tables"; "Batching and PagedAttention", "PagedAttention" item 4]:
@@ -15,7 +15,7 @@
 // four flops per byte: it is bound by HBM.  A pool block holds the K (or V)
 // rows of all kv heads contiguously ([block][kv head][slot][d]), so a block
 // of HS heads is one run of HS * bs rows.  The kernel streams whole blocks:
-//   - one producer warp per CTA claims chunks of work, looks the blocks up in
+//   - one producer warp per CTA walks its chunk of the work, looks the blocks up in
 //     the block tables and loads each block's K and V rows for HS heads with
 //     one TMA box each (all 64-column panels, 128-byte swizzle) into a ring of NS shared-memory
 //     stages, a stage being NBS blocks (ST = NBS * bs tokens, up to 64 KiB);
@@ -26,14 +26,15 @@
 //     O^T += V^T P^T on mma.sync m16n8k16 (bf16 in, fp32 accumulate), with P^T
 //     moved into operand order by movmatrix, and an online softmax in fp32.
 // Work split (flash-decoding-style split-K, balanced like stream-K): the
-// stages of all (sequence, head group) pairs are concatenated and cut into
-// chunks claimed from a global counter: first one large chunk per CTA
-// (kBigEighths / 8 of the work), then small ones (kSmallPerCta per CTA), so a
-// CTA that runs slow sheds the small chunks to the others.  The part of a pair inside one chunk is a partition; a pair
-// cut into several partitions writes (normalised O, log2-sum-exp) rows per
-// partition, and a second kernel, launched as a programmatic dependent of the
-// first, merges them with the whole GPU (no fence, atomic or wait in the
-// streaming kernel).
+// stages of all (sequence, head group) pairs are concatenated and cut into one
+// equal chunk per CTA.  The part of a pair inside one chunk is a partition; a
+// pair cut into several partitions writes (normalised O, log2-sum-exp) rows per
+// partition and kv head, and the consumer warp that writes the last partition
+// of a (sequence, kv head), found by an arrival counter in the workspace,
+// merges that head's rows once its own stages are done (no wait anywhere: a
+// fence and an atomic add per split head).  A chunk holds at most two split
+// partitions (its first and its last pair), so a warp has at most two merges
+// to do.
 //
 // Every wait is bounded (2 s); on expiry the kernel records PK_ERR_TIMEOUT,
 // waits (bounded) for its own copies in flight and returns.  Block ids are
@@ -50,26 +51,22 @@ using namespace tc;
 constexpr int kNC = 8;                        // consumer warps
 constexpr int kBlkThreads = (kNC + 1) * 32;   // + one producer warp
 constexpr int kStageCap = 64 * 1024;          // K + V bytes of one stage
-constexpr int kBigEighths = 8;                // share of the work in the first (large) chunks
-constexpr int kSmallPerCta = 4;               // small chunks per CTA for the rest
 constexpr int kMinChunkStages = 2;            // smallest chunk
 constexpr int kItemSlots = 2;                 // items staged ahead (Q rows + descriptor each)
-constexpr int kMergeListHead = 4;             // merge list: count, pad, then int4 entries
 constexpr float kRescaleLog2 = 8.f;           // lazy softmax rescale threshold (log2 units)
+constexpr int kMaxDeferred = 4;               // split-K merges a consumer warp keeps for its end (2 needed)
+constexpr int kMergeListHead = 4;             // merge kernel's list: count, pad, then int4 entries
 
 enum : int { kFirst = 1, kLast = 2, kEnd = 4 };
 
-// Chunks of the concatenated stages: nb large chunks of cb stages, then small
-// chunks of csm stages up to `total`.
+// Chunks of the concatenated stages: nb chunks of cb stages (the last one
+// shorter), at most one per CTA.
 struct ChunkPlan {
-    int cb, nb, csm, total;
-    __device__ int of(int g) const {  // chunk holding stage g
-        const int big = nb * cb;
-        return g < big ? g / cb : nb + (g - big) / csm;
-    }
-    __device__ int begin(int k) const { return k < nb ? k * cb : nb * cb + (k - nb) * csm; }
-    __device__ int end(int k) const { return min(total, begin(k + 1)); }
-    __device__ int count() const { return nb + (total - nb * cb + csm - 1) / csm; }
+    int cb, nb, total;
+    __device__ int of(int g) const { return g / cb; }  // chunk holding stage g
+    __device__ int begin(int k) const { return k * cb; }
+    __device__ int end(int k) const { return min(total, (k + 1) * cb); }
+    __device__ int count() const { return nb; }
     // partitions of the stages [start, start + n)
     __device__ int parts(int start, int n) const { return of(start + n - 1) - of(start) + 1; }
 };
@@ -77,11 +74,8 @@ struct ChunkPlan {
 __device__ inline ChunkPlan make_chunk_plan(int total, int ncta, int scale) {
     ChunkPlan c;
     c.total = total;
-    c.cb = max(kMinChunkStages, (int)((long long)total * kBigEighths / (8LL * ncta))) * scale;
-    c.nb = min(ncta, total / c.cb);
-    const long long rest = total - (long long)c.nb * c.cb;
-    c.csm = max(kMinChunkStages, (int)((rest + (long long)ncta * kSmallPerCta - 1) /
-                                       ((long long)ncta * kSmallPerCta))) * scale;
+    c.cb = max(kMinChunkStages, (int)(((long long)total + ncta - 1) / ncta)) * scale;
+    c.nb = (total + c.cb - 1) / c.cb;
     return c;
 }
 
@@ -101,12 +95,13 @@ struct BlkParams {
     int HS, NBS, ST, NPH, NS;  // geometry: heads / blocks / tokens per stage, phases, stages
     int ncta, cap_rows;
     float scale_log2;
-    WsHeader *hdr;
-    int *mplan;                      // the plan, for the merge kernel
+    int merge_in_kernel;             // 1: split heads are merged by their last writer; 0: by the merge kernel
+    int *counters;                   // split-K arrivals per (sequence of the window, kv head)
+    int *mplan;                      // merge kernel's list (merge_in_kernel == 0)
     float *partial_o, *partial_lse;  // [row][D], [row]
     int *err;
     // shared-memory layout (byte offsets from the 1024-aligned base)
-    uint32_t stage_bytes, qslot_bytes, off_q, off_scr, off_plan, off_desc, off_info, off_bar, total;
+    uint32_t stage_bytes, qslot_bytes, off_q, off_scr, off_plan, off_desc, off_info, off_defer, off_bar, total;
 };
 
 // Shared-memory layout of one launch.
@@ -127,9 +122,81 @@ void blk_layout(BlkParams &p) {
     off += kItemSlots * sizeof(ItemDesc);
     p.off_info = off;
     off += (uint32_t)p.NS * sizeof(StageInfo);
+    p.off_defer = up(off, 16);
+    off = p.off_defer + (uint32_t)kNC * kMaxDeferred * sizeof(int4);
     p.off_bar = up(off, 8);
     off = p.off_bar + (uint32_t)(2 * p.NS + 2 * kItemSlots + 1) * 8;
     p.total = off + 1024;  // + alignment slack
+}
+
+// Split-K merge of one kv head's g rows [flash-decoding combination]:
+// out = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M), M = max_p lse_p, over
+// the partitions' normalised rows o_p and log2-sum-exps lse_p, written by other
+// CTAs (read from L2).  The g x D outputs are spread over the lanes (with g
+// dividing 32: 32 / g lanes per row, a block of columns each; otherwise row by
+// row) and the loads of up to four partitions are issued before any is used,
+// so a merge costs a few L2 round trips.  Rows prow + p * HS * g + hl * g + q
+// hold partition p of q head q.
+template <int D>
+__device__ __forceinline__ void merge_head(const BlkParams &prm, int prow, int nparts, int qs0, int kvh,
+                                           int hl_, int lane) {
+    const int g = prm.group, HS = prm.HS, Hq = prm.n_q_heads;
+    constexpr int PB = 4;  // partitions per batch of loads
+    const bool by_lane = (32 % g) == 0;
+    const int lq = by_lane ? 32 / g : 32;          // lanes per row
+    const int cols = D / lq;                       // columns per lane and row: 2 .. 64
+    const int cpp = cols < 8 ? cols : 8;           // columns per pass
+    for (int q = by_lane ? lane / lq : 0; q < g; q += by_lane ? g : 1) {
+        const int li = by_lane ? lane % lq : lane;
+        for (int cc = 0; cc < cols; cc += cpp) {
+            const int col = li * cols + cc;
+            float M = -INFINITY, den = 0.f, acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+            for (int p0 = 0; p0 < nparts; p0 += PB) {
+                float l[PB];
+                float2 x[PB][4];
+#pragma unroll
+                for (int i = 0; i < PB; ++i) {
+                    l[i] = -INFINITY;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) x[i][j] = make_float2(0.f, 0.f);
+                    if (p0 + i < nparts) {
+                        const int row = prow + (p0 + i) * HS * g + hl_ * g + q;
+                        l[i] = __ldcg(prm.partial_lse + row);
+                        const float2 *src = (const float2 *)(prm.partial_o + (size_t)row * D + col);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            if (2 * j < cpp) x[i][j] = __ldcg(src + j);
+                    }
+                }
+                float bm = M;
+#pragma unroll
+                for (int i = 0; i < PB; ++i) bm = fmaxf(bm, l[i]);
+                if (bm == -INFINITY) continue;
+                const float a = M == -INFINITY ? 0.f : fast_exp2(M - bm);
+                den *= a;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[j] *= a;
+                M = bm;
+#pragma unroll
+                for (int i = 0; i < PB; ++i) {
+                    const float w = l[i] == -INFINITY ? 0.f : fast_exp2(l[i] - M);
+                    den += w;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        acc[2 * j] += w * x[i][j].x;
+                        acc[2 * j + 1] += w * x[i][j].y;
+                    }
+                }
+            }
+            const float inv = den > 0.f ? 1.f / den : 0.f;
+            __nv_bfloat16 *dst = prm.out + ((long long)qs0 * Hq + kvh * g + q) * D + col;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (2 * j < cpp) *(uint32_t *)(dst + 2 * j) = pack_bf16(acc[2 * j] * inv, acc[2 * j + 1] * inv);
+        }
+    }
 }
 
 template <int D>
@@ -238,7 +305,7 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
             if (attempt < 6) {
                 cp = make_chunk_plan(total, prm.ncta, 2 << attempt);
             } else {
-                cp.cb = cp.csm = max(total, 1);
+                cp.cb = max(total, 1);
                 cp.nb = total > 0 ? 1 : 0;
             }
         }
@@ -247,7 +314,7 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
             s_cp = cp;
         }
         __syncwarp();
-        if (blockIdx.x == 0) {
+        if (!prm.merge_in_kernel && blockIdx.x == 0) {
             // the merge kernel's work list: (sequence, head group, first partial
             // row, partitions) of every pair cut into several partitions
             int n_split = 0;
@@ -269,7 +336,7 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
             if (lane == 0) prm.mplan[0] = n_split;
         }
     }
-    // the merge kernel may be scheduled now; it waits for this grid to finish
+    // a merge kernel, if one follows, may be scheduled now; it waits for this grid to finish
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __syncthreads();
     const ChunkPlan cp = s_cp;
@@ -277,14 +344,8 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
-        // CTA i starts with chunk i; the chunks after the first gridDim.x go to
-        // whoever claims them (the claim for the next one is always in flight)
+        // CTA i takes chunk i
         const int nchunks = cp.count();
-        auto claim = [&]() -> int {
-            int v = 0;
-            if (lane == 0) v = (int)gridDim.x + atomicAdd(&prm.hdr->next_item, 1);
-            return v;
-        };
         int pending = (int)blockIdx.x;
         int n_stage = 0, n_item = 0;
         auto chunk_entry = [&](int b, int blk_base) -> int {
@@ -292,7 +353,7 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
             const int e = blk_base + lane;
             return e < nblk ? __ldg(prm.tables + (long long)(prm.seq0 + b) * prm.max_blocks + e) : 0;
         };
-        // Items (partitions) in claim order.  The next item is found, and its
+        // Items (partitions) in chunk order.  The next item is found, and its
         // first two table chunks requested, while the current one's stages
         // are issued, so the table lookups of an item start without a wait.
         struct PItem {
@@ -301,9 +362,9 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
         int g0 = 0, g1 = 0;
         auto next_item = [&](PItem &it) -> bool {
             while (g0 >= g1) {
-                const int chunk = __shfl_sync(0xffffffffu, pending, 0);
+                const int chunk = pending;
                 if (chunk >= nchunks) return false;
-                pending = claim();  // lane 0's value; broadcast when used
+                pending = nchunks;  // one chunk per CTA
                 g0 = cp.begin(chunk);
                 g1 = cp.end(chunk);
             }
@@ -547,6 +608,9 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                 mma_bf16(ot[mt], a0, a1, a2, a3, b0, b1);
             }
         };
+        // merges this warp found itself last for, run once its stages are done
+        int4 *deferred = (int4 *)(sm + prm.off_defer) + cw * kMaxDeferred;
+        int n_deferred = 0;
         float *scr = (float *)(sm + prm.off_scr);
         constexpr int kScr = KS * 4 + 4;  // floats per lane of one warp's state
         auto finish_item = [&](int slot) -> bool {
@@ -636,6 +700,26 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                         if (va_) pl[ha] = l0 > 0.f ? m0 + __log2f(l0) : -INFINITY;
                         if (vb_) pl[hb] = l1 > 0.f ? m1 + __log2f(l1) : -INFINITY;
                     }
+                    // arrival: the warp that writes the last partition of this
+                    // (sequence, kv head) merges its rows
+                    __threadfence();  // every lane's partial rows, before the arrival
+                    __syncwarp();
+                    int last = 0;
+                    if (prm.merge_in_kernel && lane == 0) {
+                        int *cnt = prm.counters + (size_t)d.b * Hkv + kvh;
+                        last = atomicAdd(cnt, 1) == d.nparts - 1;
+                        if (last) *cnt = 0;  // leave the counter zeroed for the next call
+                    }
+                    if (__shfl_sync(0xffffffffu, last, 0)) {
+                        // a chunk holds at most two split partitions, so the list
+                        // never fills; were it to, the error word says so
+                        if (n_deferred < kMaxDeferred) {
+                            if (lane == 0) deferred[n_deferred] = make_int4(d.prow, d.nparts, d.qs0, kvh);
+                            ++n_deferred;
+                        } else if (lane == 0) {
+                            record_error(prm.err, PK_ERR_UNSUPPORTED);
+                        }
+                    }
                 }
             }
             __syncwarp();
@@ -670,17 +754,23 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                 break;
             }
         }
+        if (ok && n_deferred > 0) {
+            __syncwarp();
+            __threadfence();  // the other partitions' rows after their arrivals
+            for (int i = 0; i < n_deferred; ++i) {
+                const int4 e = deferred[i];
+                merge_head<D>(prm, e.x, e.y, e.z, e.w, hl, lane);
+            }
+        }
         if (!ok && lane == 0) record_error(prm.err, PK_ERR_TIMEOUT);
     }
     __syncthreads();
-    release_counter(prm.hdr);
 }
 
-// The largest dynamic shared memory a launch may ask for: the device's opt-in
-// limit per block less the kernel's static shared memory.
-// Merge of the split-K partitions [flash-decoding combination]: for every
-// (sequence, head group) that the streaming kernel cut into several
-// partitions, each output row (q head hg * HS * g + r of the sequence's token)
+// Merge kernel, for launches whose pairs are cut into many partitions (few
+// long sequences): the merge then needs more of the GPU than the last writer
+// of each head [flash-decoding combination].  For every (sequence, head group)
+// that the streaming kernel cut into several partitions, each output row (q head hg * HS * g + r of the sequence's token)
 // is out = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M), M = max_p lse_p, over
 // the partitions' normalised rows o_p and log2-sum-exps lse_p.
 // The streaming kernel lists the split pairs.  blockIdx.x = list entry,
@@ -754,6 +844,8 @@ __global__ void __launch_bounds__(kMergeThreads) attention_merge_kernel(const Me
     *(uint2 *)(mp.out + orow * D + c4 * 4) = pk;
 }
 
+// The largest dynamic shared memory a launch may ask for: the device's opt-in
+// limit per block less the kernel's static shared memory.
 template <int D>
 int blocks_prepare(pk_pool *p) {
     int optin = 0;
@@ -791,7 +883,7 @@ int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, bool s
     tp.ncta = p->sm_count;
     tp.cap_rows = w.cap_rows;
     tp.scale_log2 = a.scale * 1.4426950408889634f;
-    tp.hdr = (WsHeader *)w.header;
+    tp.counters = w.counters;
     tp.mplan = w.merge_plan;
     tp.partial_o = w.partial_o;
     tp.partial_lse = w.partial_lse;
@@ -807,6 +899,11 @@ int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, bool s
     for (int s0 = 0; s0 < a.num_seqs; s0 += kMaxSeqsPerLaunch) {
         tp.seq0 = s0;
         tp.nseq = std::min(kMaxSeqsPerLaunch, a.num_seqs - s0);
+        // Split heads are merged in the streaming kernel by their last writer
+        // when the window has enough (sequence, head group) pairs for about four
+        // partitions per pair at most; with fewer, longer pairs (each cut into
+        // many partitions) a merge kernel spreads the merging over the GPU.
+        tp.merge_in_kernel = 4LL * tp.nseq * (tp.n_kv_heads / tp.HS) >= tp.ncta ? 1 : 0;
         {
             cudaLaunchConfig_t c0 = {};
             c0.gridDim = dim3(tp.ncta);
@@ -821,6 +918,7 @@ int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, bool s
             const cudaError_t e0 = cudaLaunchKernelEx(&c0, attention_decode_blocks_kernel<D>, p->tmap_kb, p->tmap_vb, tp);
             if (e0 != cudaSuccess) return cuda_fail(e0, "decode attention launch");
         }
+        if (tp.merge_in_kernel) continue;
         MergeParams mp;
         mp.out = tp.out;
         mp.qsl = tp.qsl;
@@ -885,7 +983,7 @@ int decode_blocks_prepare_pool(pk_pool *p) {
     return rc;
 }
 
-int decode_blocks_chunks_per_cta() { return 1 + kSmallPerCta; }
+int decode_blocks_chunks_per_cta() { return 2; }  // split partitions a chunk can hold
 
 bool decode_blocks_applies(const pk_pool *p, const AttnArgs &a) {
     return p->blk_ok && a.n_q_heads / p->n_kv_heads <= 8;

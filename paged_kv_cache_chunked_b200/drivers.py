@@ -22,6 +22,8 @@ Both generate queries and K/V with the counter-based generator of
 `workloads.token_values`, keyed by (request id, position), on the device.
 """
 
+import time
+
 import torch
 
 from . import api
@@ -30,8 +32,14 @@ from .workloads import SYS_VID_BASE, token_values, trace_requests
 
 
 class StepRecord:
+    """One scheduler step: its batch, its GPU time (CUDA events around swaps,
+    copies, append and attention) and its host time split into planning
+    (schedule + complete), launching the generation of the step's synthetic
+    q/k/v (which stands in for the model; values_gpu_ms is its GPU time) and the
+    rest (metadata copies, launches, the wait)."""
     __slots__ = ("step", "tokens", "decode_rows", "prefill_tokens", "copies", "gpu_ms",
-                 "context_tokens", "num_seqs", "swap_blocks", "new_tokens")
+                 "context_tokens", "num_seqs", "swap_blocks", "new_tokens", "host_plan_ms",
+                 "host_values_ms", "values_gpu_ms", "host_total_ms")
 
     def __init__(self, **kw):
         for k, v in kw.items():
@@ -84,9 +92,11 @@ class TraceRunner:
         """One iteration.  on_step(plan, tensors, out) is called after the
         kernels (for parity checks).  Returns the step's record, or None when
         there was nothing to run."""
+        t_start = time.perf_counter()
         step = self.sched.step_no
         self._admit_arrivals(step)
         plan = self.sched.schedule()
+        t_planned = time.perf_counter()
         dev = self.device
         swaps = [(to_host, torch.tensor(pairs, dtype=torch.int32).reshape(-1, 2).to(dev))
                  for to_host, pairs in plan.swap_ops]
@@ -105,9 +115,15 @@ class TraceRunner:
                 e1.synchronize()
                 rec = StepRecord(step=step, tokens=0, decode_rows=0, prefill_tokens=0, copies=0,
                                  gpu_ms=e0.elapsed_time(e1), context_tokens=0, num_seqs=0,
-                                 swap_blocks=sum(len(p) for _, p in plan.swap_ops), new_tokens=0)
+                                 swap_blocks=sum(len(p) for _, p in plan.swap_ops), new_tokens=0,
+                                 host_values_ms=0.0, values_gpu_ms=0.0)
                 self.records.append(rec)
+            t_c = time.perf_counter()
             self.sched.complete(plan)
+            if rec is not None:
+                t_end = time.perf_counter()
+                rec.host_plan_ms = 1e3 * ((t_planned - t_start) + (t_end - t_c))
+                rec.host_total_ms = 1e3 * (t_end - t_start)
             return rec
         rids, pos = [], []
         for req, s, n in zip(plan.requests, plan.starts, plan.counts):
@@ -121,10 +137,17 @@ class TraceRunner:
             "pairs": torch.tensor(plan.copy_pairs, dtype=torch.int32).reshape(-1, 2),
         }
         d = {k: v.to(dev, non_blocking=True) for k, v in meta.items()}
+        stream = torch.cuda.current_stream(dev)
+        t_v = time.perf_counter()
+        if timed:
+            ev_v = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            ev_v[0].record(stream)
         q = token_values(self.seed, 0, rids, pos, self.Hq, self.d, self.dtype, dev)
         k = token_values(self.seed, 1, rids, pos, self.Hkv, self.d, self.dtype, dev)
         v = token_values(self.seed, 2, rids, pos, self.Hkv, self.d, self.dtype, dev)
-        stream = torch.cuda.current_stream(dev)
+        if timed:
+            ev_v[1].record(stream)
+        t_v = time.perf_counter() - t_v
         if timed:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
@@ -152,8 +175,14 @@ class TraceRunner:
                          prefill_tokens=plan.num_tokens - n_dec, copies=len(plan.copy_pairs),
                          gpu_ms=e0.elapsed_time(e1) if timed else None,
                          context_tokens=sum(plan.context_lens), num_seqs=len(plan.requests),
-                         swap_blocks=sum(len(p) for _, p in plan.swap_ops), new_tokens=new)
+                         swap_blocks=sum(len(p) for _, p in plan.swap_ops), new_tokens=new,
+                         host_values_ms=1e3 * t_v,
+                         values_gpu_ms=ev_v[0].elapsed_time(ev_v[1]) if timed else None)
+        t_c = time.perf_counter()
         self.sched.complete(plan)
+        t_end = time.perf_counter()
+        rec.host_plan_ms = 1e3 * ((t_planned - t_start) + (t_end - t_c))
+        rec.host_total_ms = 1e3 * (t_end - t_start)
         self.records.append(rec)
         return rec
 

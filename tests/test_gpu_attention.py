@@ -91,6 +91,10 @@ CHUNK_CASES = [
     ([1100, 96], [600, 96], 64, 8, 128, 32),     # g 8, block 32
     ([2000, 40], [257, 40], 32, 2, 128, 64),     # g 16, block 64
     ([333, 20], [200, 1], 64, 1, 128, 16),       # g 64: one token fills 64 rows; a decode in the batch
+    # d 64, blocks of 16k: the same tcgen05 kernel with one 64-column panel
+    ([600, 77, 900], [300, 77, 1], 16, 4, 64, 16),   # g 4, a decode row on the block-streaming kernel
+    ([1000], [512], 8, 8, 64, 32),                   # g 1, block 32
+    ([333, 40], [200, 40], 64, 1, 64, 16),           # g 64
 ]
 
 
@@ -194,7 +198,7 @@ def test_full_size_chunk512_sampled_rows(cuda_dev):
 @pytest.mark.parametrize("Hkv,d,bs,want", [
     (8, 128, 16, ("TENSOR_CORE", "DECODE_BLOCKS", "CHUNK_TCGEN05")),
     (4, 256, 16, ("TENSOR_CORE", "DECODE_BLOCKS")),
-    (8, 64, 16, ("TENSOR_CORE", "DECODE_BLOCKS")),
+    (8, 64, 16, ("TENSOR_CORE", "DECODE_BLOCKS", "CHUNK_TCGEN05")),
     (8, 128, 8, ("TENSOR_CORE", "DECODE_BLOCKS")),
 ])
 def test_pool_paths(cuda_dev, Hkv, d, bs, want):
