@@ -39,6 +39,7 @@ FALLBACK_HBM_GBS = 6650.0
 CSRC = os.path.join(ROOT, "paged_kv_cache_chunked_b200", "csrc")
 # the source of each workload's dominant kernel (the traffic record is valid for that source only)
 KERNEL_SRC = {"chunk512_bf16": os.path.join(CSRC, "attention_chunk_umma.cu"),
+              "chunk512_d256_bf16": os.path.join(CSRC, "attention_chunk_umma256.cu"),
               "append_copy": os.path.join(CSRC, "kv_copy.cu")}
 DECODE_SRC = os.path.join(CSRC, "attention_decode_blocks.cu")
 
@@ -50,7 +51,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="decode64_bf16",
-                   choices=["decode64_bf16", "longdoc_bf16", "chunk512_bf16", "mixed_bf16", "trace", "trace_swap",
+                   choices=["decode64_bf16", "longdoc_bf16", "chunk512_bf16", "chunk512_d256_bf16", "mixed_bf16",
+                            "trace", "trace_swap",
                             "trace_prefix", "trace_prefix_nocache", "trace_hybrid", "policy", "fork",
                             "fork1028", "append_copy"])
     p.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
@@ -307,7 +309,7 @@ def roofline_entry(workload, attn_b, flops, avg_ms, gbs, tflops, hbm_peak, hbm_k
     """The attention call's roofline: HBM for decode (about 4 flop/byte at GQA 4),
     the tensor pipe for prefill chunks (a dense contraction)."""
     kern = ("paged_attention call: tcgen05 chunk kernel (S and O accumulated in tensor memory)"
-            if workload == "chunk512_bf16" else
+            if workload in ("chunk512_bf16", "chunk512_d256_bf16") else
             "paged_attention call: block-streaming decode kernel (split heads merged by their last "
             "writer), then the tcgen05 chunk kernel" if workload == "mixed_bf16" else
             "paged_attention call: block-streaming decode kernel + split-K merge kernel"
@@ -316,7 +318,7 @@ def roofline_entry(workload, attn_b, flops, avg_ms, gbs, tflops, hbm_peak, hbm_k
     common = {"kernel": kern,
               "algorithmic_bytes": attn_b, "algorithmic_flops": flops, "avg_ms": avg_ms,
               "traffic": kernel_traffic(workload)}
-    if workload == "chunk512_bf16":
+    if workload in ("chunk512_bf16", "chunk512_d256_bf16"):
         peak, kind = measured_tensor_peak()
         return dict(common, bound="tensor", achieved=tflops, peak=peak, unit="TFLOP/s",
                     frac=tflops / peak,
@@ -519,7 +521,7 @@ def run_ours(args, rank, world, device):
     if blocks and T == B:
         per_window = 1 + merge_launch   # block-streaming decode (+ merge kernel)
     elif blocks and umma:
-        per_window = 2 + merge_launch   # block-streaming decode (+ merge), then the tcgen05 chunk kernel
+        per_window = 2                  # block-streaming decode, then the tcgen05 chunk kernel
     else:
         per_window = 2 if T > B or Hq // Hkv > 16 else 1
     launches_per_step = 1 + (windows * per_window if tc else 1)

@@ -97,7 +97,7 @@ int pk_pool_destroy(pk_pool *pool);
  *   PK_PATH_DECODE_BLOCKS  one-token rows stream whole blocks, all kv heads of a
  *                          group per TMA box (block-streaming decode kernel)
  *   PK_PATH_CHUNK_TCGEN05  prefill chunks run on tcgen05 with accumulators in
- *                          tensor memory (head_dim 64 or 128, block_size a
+ *                          tensor memory (head_dim 64, 128 or 256, block_size a
  *                          multiple of 16); without it they run on mma.sync.  The library
  *                          leaves it off when the kernel was not compiled with
  *                          the register count its warp roles are laid out for,

@@ -16,7 +16,7 @@ LIB = os.path.join(HERE, "libpagedkv.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
 SOURCES = ["api.cu", "kv_copy.cu", "attention_generic.cu", "attention_decode.cu", "attention_decode_blocks.cu",
-           "attention_chunk.cu", "attention_chunk_umma.cu", "attention_host.cu", "attention_noalloc.cu", "block_manager.cpp"]
+           "attention_chunk.cu", "attention_chunk_umma.cu", "attention_chunk_umma256.cu", "attention_host.cu", "attention_noalloc.cu", "block_manager.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE,
               "-I", CSRC, "--expt-relaxed-constexpr"]

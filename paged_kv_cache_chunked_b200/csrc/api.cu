@@ -176,7 +176,7 @@ int pk_pool_paths(const pk_pool *pool, int *paths_out) {
     if (pool->tc_path) {
         f |= PK_PATH_TENSOR_CORE;
         if (pool->blk_ok) f |= PK_PATH_DECODE_BLOCKS;
-        if (pool->umma_ok) f |= PK_PATH_CHUNK_TCGEN05;
+        if (pool->umma_ok || pool->umma256_ok) f |= PK_PATH_CHUNK_TCGEN05;
     }
     *paths_out = f;
     return PK_OK;

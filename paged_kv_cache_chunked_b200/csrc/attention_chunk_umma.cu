@@ -44,7 +44,7 @@
 // Every wait is bounded (2 s); on expiry the kernel records PK_ERR_TIMEOUT,
 // each warp waits (bounded) for its own copies and tensor-core work, and the
 // CTA releases its tensor memory and returns.  Block ids are range-checked.
-#include "tc_common.cuh"
+#include "umma_common.cuh"
 
 #include <algorithm>
 #include <cstdlib>
@@ -102,103 +102,6 @@ struct UGeo {
 constexpr uint32_t kUPerTileBars = 5;
 // S = Q K^T (kind::f16): fp32 accumulate, bf16 A and B, M = 128, N = 128 keys
 constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
-
-// Shared-memory matrix descriptor (128-byte swizzle) as two 32-bit words: the low
-// word holds the start address and the leading byte offset (both >> 4), the high
-// word the stride byte offset (>> 4, 1024 B here), the descriptor version of
-// sm_100 (bit 46 of the 64-bit value) and the swizzle mode (bits 61..63).  The
-// MMA thread builds the low word of each operand's base once and adds the
-// per-K-step offset (>> 4; addresses stay below 256 KiB, so the 14-bit field
-// never carries).
-__device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo) {
-    return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
-}
-constexpr uint32_t kSdescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
-// D (tensor memory) [+]= A (shared) x B (shared)
-__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc,
-                                        uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\t"
-        "mov.b64 ad, {%1, %5};\n\tmov.b64 bd, {%2, %5};\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, {%6, %6, %6, %6}, p;\n\t}\n" ::"r"(d_tmem),
-        "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(kSdescHi), "r"(0u));
-}
-// D (tensor memory) [+]= A (tensor memory: row m in lane m, two bf16 per column,
-// the even K index in the low half) x B (shared)
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc,
-                                        uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\t"
-        "mov.b64 bd, {%2, %5};\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %3, {%6, %6, %6, %6}, p;\n\t}\n" ::"r"(d_tmem),
-        "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(kSdescHi), "r"(0u));
-}
-__device__ __forceinline__ void umma_commit(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     smem_u32(bar))
-                 : "memory");
-}
-__device__ __forceinline__ void tc_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
-                 : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-                 : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-                 : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
-                 :
-                 : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
-                 :
-                 : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-                 : "memory");
-}
-// ---- packed f32x2 arithmetic ----------------------------------------------
-// The softmax warps are bound by instruction issue, so their per-key work uses
-// the packed two-float forms: one instruction scales and offsets two scores,
-// one adds two probabilities to the row sum.
-__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-    return r;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float &a, float &b) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-// max(a, b, c) in one instruction
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-    float d;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
 
 struct UParams {
     const __nv_bfloat16 *q;
@@ -682,30 +585,40 @@ int umma_prepare(pk_pool *p, bool &ok) {
 
 }  // namespace
 
-// Serves bf16 pools with head_dim 64 or 128 and 16-row tile boxes (block_size a
-// multiple of 16), and groups dividing 128; PK_CHUNK_MMA_SYNC=1 selects the
-// mma.sync chunk kernel instead.  Head dim 256 does not fit: two 128-row tiles
-// would need 2 x (128 S + 256 O) tensor-memory columns of the 512.
+// Serves bf16 pools with 16-row tile boxes (block_size a multiple of 16) and
+// groups dividing 128: this kernel at head dim 64 or 128, the head-dim-256
+// kernel (attention_chunk_umma256.cu) at 256, where two 128-row tiles would need
+// 2 x (128 S + 256 O) tensor-memory columns of the 512.  PK_CHUNK_MMA_SYNC=1
+// selects the mma.sync chunk kernel instead.
 int chunk_umma_prepare_pool(pk_pool *p) {
-    p->umma_ok = false;
+    p->umma_ok = p->umma256_ok = false;
     const char *e = getenv("PK_CHUNK_MMA_SYNC");
-    if ((p->head_dim != 64 && p->head_dim != 128) || !p->tile_map3d || (e && e[0] == '1')) return PK_OK;
+    if (!p->tile_map3d || (e && e[0] == '1')) return PK_OK;
+    if (p->head_dim != 64 && p->head_dim != 128 && p->head_dim != 256) return PK_OK;
     bool ok = false;
-    const int rc = p->head_dim == 64 ? umma_prepare<64>(p, ok) : umma_prepare<128>(p, ok);
+    int rc = PK_OK;
+    if (p->head_dim == 256) {
+        rc = chunk_umma256_prepare(p);
+        ok = rc == PK_OK;
+    } else {
+        rc = p->head_dim == 64 ? umma_prepare<64>(p, ok) : umma_prepare<128>(p, ok);
+    }
     if (rc != PK_OK || !ok) return rc;
     // K as 2-D 16-row boxes of one 64-column panel; V uses the pool's 3-D tile map
     const int rc2 = encode_pool_map(&p->tmap_k2, p->k_base, p, kTile);
     if (rc2 != PK_OK) return rc2;
-    p->umma_ok = true;
+    if (p->head_dim == 256) p->umma256_ok = true;
+    else p->umma_ok = true;
     return PK_OK;
 }
 
 bool chunk_umma_applies(const pk_pool *p, const AttnArgs &a) {
     const int g = a.n_q_heads / p->n_kv_heads;
-    return p->umma_ok && g >= 1 && kURows % g == 0;
+    return (p->umma_ok || p->umma256_ok) && g >= 1 && kURows % g == 0;
 }
 
 int launch_chunk_umma(const pk_pool *p, const AttnArgs &a, bool all_multi, cudaStream_t st) {
+    if (p->head_dim == 256) return launch_chunk_umma256(p, a, all_multi, st);
     UParams u;
     u.q = (const __nv_bfloat16 *)a.q;
     u.out = (__nv_bfloat16 *)a.out;

@@ -902,8 +902,11 @@ int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, bool s
         // Split heads are merged in the streaming kernel by their last writer
         // when the window has enough (sequence, head group) pairs for about four
         // partitions per pair at most; with fewer, longer pairs (each cut into
-        // many partitions) a merge kernel spreads the merging over the GPU.
-        tp.merge_in_kernel = 4LL * tp.nseq * (tp.n_kv_heads / tp.HS) >= tp.ncta ? 1 : 0;
+        // many partitions) a merge kernel spreads the merging over the GPU.  In
+        // a batch with prefill chunks the decode rows are an unknown part of
+        // the window (often none), so there it is always the last writer.
+        tp.merge_in_kernel =
+            skip_chunks || 4LL * tp.nseq * (tp.n_kv_heads / tp.HS) >= tp.ncta ? 1 : 0;
         {
             cudaLaunchConfig_t c0 = {};
             c0.gridDim = dim3(tp.ncta);

@@ -23,7 +23,8 @@ struct pk_pool {
     int tc_ctas;        // resident CTAs of the decode attention kernel (whole GPU)
     int tc_ctas_chunk;  // resident CTAs of the chunk attention kernel (whole GPU)
     bool tile_map3d;    // tmap_k / tmap_v are 3-D (16-row boxes of all panels), else 2-D (8 rows)
-    bool umma_ok;       // the tcgen05 chunk kernel serves this geometry
+    bool umma_ok;       // the tcgen05 chunk kernel serves this geometry (head dim 64 / 128)
+    bool umma256_ok;    // the head-dim-256 tcgen05 chunk kernel serves it
     bool blk_ok;        // the block-streaming decode kernel serves this geometry
     int blk_hs, blk_nbs;  // its kv heads and blocks per pipeline stage
     int blk_smem_max;     // its largest dynamic shared memory per launch
@@ -118,6 +119,9 @@ int chunk_prepare_pool(pk_pool *p);
 int chunk_umma_prepare_pool(pk_pool *p);
 bool chunk_umma_applies(const pk_pool *p, const AttnArgs &a);
 int launch_chunk_umma(const pk_pool *p, const AttnArgs &a, bool all_multi, cudaStream_t st);
+// head dim 256: one 128-row tile per item, two S buffers in tensor memory
+int chunk_umma256_prepare(pk_pool *p);
+int launch_chunk_umma256(const pk_pool *p, const AttnArgs &a, bool all_multi, cudaStream_t st);
 int launch_chunk(const pk_pool *p, const AttnArgs &a, void *header, cudaStream_t st);
 
 }  // namespace pk

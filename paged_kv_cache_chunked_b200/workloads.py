@@ -15,6 +15,8 @@ Workloads (sizes as the spec configurations name them):
                  heads, head dim 256, pool 1.25x
   chunk512_bf16  16 sequences at context 4096 whose last 512 tokens are this
                  step's prefill chunk (causal), 32 q / 8 kv heads, head dim 128
+  chunk512_d256_bf16  the same chunks at head dim 256 with 16 q / 4 kv heads (the
+                 long-document geometry)
   mixed_bf16     one continuous-batching step: 128 decode sequences with
                  contexts uniform in [128, 2048] and four 512-token prefill
                  chunks at contexts 1024, 2048, 3072 and 4096 (2,176 query
@@ -38,6 +40,9 @@ WORKLOADS = {
     "chunk512_bf16": dict(context_lens=[4096] * 16, query_lens=[512] * 16, block_size=16,
                           n_q_heads=32, n_kv_heads=8, head_dim=128, dtype=torch.bfloat16,
                           pool_factor=1.25, seed=1006),
+    "chunk512_d256_bf16": dict(context_lens=[4096] * 16, query_lens=[512] * 16, block_size=16,
+                               n_q_heads=16, n_kv_heads=4, head_dim=256, dtype=torch.bfloat16,
+                               pool_factor=1.25, seed=1009),
     # decodes first, then the chunks, the order the scheduler emits them
     "mixed_bf16": dict(num_seqs=128, ctx_range=(128, 2048), chunk_contexts=[1024, 2048, 3072, 4096],
                        chunk_len=512, block_size=16, n_q_heads=32, n_kv_heads=8, head_dim=128,

@@ -95,6 +95,10 @@ CHUNK_CASES = [
     ([600, 77, 900], [300, 77, 1], 16, 4, 64, 16),   # g 4, a decode row on the block-streaming kernel
     ([1000], [512], 8, 8, 64, 32),                   # g 1, block 32
     ([333, 40], [200, 40], 64, 1, 64, 16),           # g 64
+    # d 256: the tcgen05 kernel with one 128-row tile and two S buffers
+    ([1500, 300, 900], [700, 300, 1], 16, 4, 256, 16),   # g 4, 64-key stages, a decode row
+    ([1000], [257], 8, 8, 256, 32),                      # g 1, block 32
+    ([400, 50], [200, 50], 64, 1, 256, 16),              # g 64
 ]
 
 
@@ -197,7 +201,8 @@ def test_full_size_chunk512_sampled_rows(cuda_dev):
 
 @pytest.mark.parametrize("Hkv,d,bs,want", [
     (8, 128, 16, ("TENSOR_CORE", "DECODE_BLOCKS", "CHUNK_TCGEN05")),
-    (4, 256, 16, ("TENSOR_CORE", "DECODE_BLOCKS")),
+    (4, 256, 16, ("TENSOR_CORE", "DECODE_BLOCKS", "CHUNK_TCGEN05")),
+    (4, 256, 8, ("TENSOR_CORE", "DECODE_BLOCKS")),
     (8, 64, 16, ("TENSOR_CORE", "DECODE_BLOCKS", "CHUNK_TCGEN05")),
     (8, 128, 8, ("TENSOR_CORE", "DECODE_BLOCKS")),
 ])
