@@ -297,12 +297,15 @@ def run_reference_kvops(args, world):
 
 
 def measured_tensor_peak():
+    """The bf16 tensor peak for a kernel timed over a long loop of calls (seconds
+    under the power cap): the sustained figure of MEASURED_PEAKS.json, else the
+    pool's earlier sustained measurement, about 1.4 PFLOP/s."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
-            return float(json.load(f)["bf16_tflops"]), "measured"
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured"
     except (OSError, KeyError, ValueError):
-        return 1590.0, "fallback"
+        return 1400.0, "fallback"
 
 
 def roofline_entry(workload, attn_b, flops, avg_ms, gbs, tflops, hbm_peak, hbm_kind):
@@ -322,7 +325,9 @@ def roofline_entry(workload, attn_b, flops, avg_ms, gbs, tflops, hbm_peak, hbm_k
         peak, kind = measured_tensor_peak()
         return dict(common, bound="tensor", achieved=tflops, peak=peak, unit="TFLOP/s",
                     frac=tflops / peak,
-                    peak_source=f"{kind} (MEASURED_PEAKS.json bf16_tflops, burst)")
+                    peak_source="measured (MEASURED_PEAKS.json bf16_tflops_sustained)" if kind == "measured"
+                    else "fallback 1.4 PFLOP/s sustained (the calls are timed in a loop of seconds "
+                         "under the power cap)")
     return dict(common, bound="hbm", achieved=gbs, peak=hbm_peak, unit="GB/s",
                 frac=gbs / hbm_peak,
                 peak_source=f"{hbm_kind} (MEASURED_PEAKS.json hbm_gbs)"

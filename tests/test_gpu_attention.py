@@ -152,6 +152,31 @@ def test_permuted_block_ids_bit_identical(cuda_dev, ql):
         assert torch.equal(o, outs[0])
 
 
+def test_in_kernel_merge_bit_identical_under_permutations(cuda_dev):
+    # 48 decode rows of 8 kv heads: enough (sequence, head group) pairs for the
+    # block-streaming kernel to merge split heads itself, by the warp that writes
+    # each head's last partition.  Which warp that is depends on timing; the
+    # merge order (by partition) does not, so the output is bit-identical under
+    # any placement of the blocks, and equal to the oracle
+    g = torch.Generator().manual_seed(31)
+    ctx = torch.randint(200, 2500, (48,), generator=g).tolist()
+    Hkv, Hq, d = 8, 32, 128
+    k_seq = [torch.randn((c, Hkv, d), generator=g).to(torch.bfloat16) for c in ctx]
+    v_seq = [torch.randn((c, Hkv, d), generator=g).to(torch.bfloat16) for c in ctx]
+    q = torch.randn((len(ctx), Hq, d), generator=g).to(torch.bfloat16)
+    qsl = torch.arange(len(ctx) + 1, dtype=torch.int32)
+    outs = []
+    for seed in range(3):
+        kp, vp, tables = contiguous_to_paged(k_seq, v_seq, 16, seed=seed)
+        batch = {"q": q, "k_pool": kp, "v_pool": vp, "block_tables": tables,
+                 "context_lens": torch.tensor(ctx, dtype=torch.int32), "query_start_lens": qsl,
+                 "scale": 1 / math.sqrt(d), "block_size": 16}
+        got, _ = _check(batch, Hq, Hkv, d, torch.bfloat16, cuda_dev, f"perm {seed}")
+        outs.append(got.cpu())
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+
+
 def test_long_context_split_k(cuda_dev):
     # two 8k-token sequences with head dim 256: many split-K partitions
     b = make_batch([8192, 6000], None, block_size=16, n_q_heads=16, n_kv_heads=4, head_dim=256,

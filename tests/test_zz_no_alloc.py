@@ -157,14 +157,20 @@ def test_noalloc_clears_stale_counters(cuda_dev):
     dst, nbytes = int(prm.dst), prm.width * prm.height * prm.elementSize
     assert prm.value == 0 and nbytes >= 512
     rt.cudaGraphDestroy(graph)
-    # non-zero counters, then a normal call
-    (err,) = rt.cudaMemset(dst, 0x01, nbytes)
-    assert err == rt.cudaError_t.cudaSuccess
-    torch.cuda.synchronize(cuda_dev)
-    rc, got = _noalloc(pool, b, cuda_dev)
-    assert rc == 0, lib().pk_last_error()
-    assert_close(got, oracle_attention(b), torch.bfloat16, "no-alloc after stale counters")
-    assert pool.check_device_errors() == 0
+    # non-zero counters, then a normal call: on the tile-streaming decode kernel
+    # (16 q heads per kv head) and on the block-streaming one, whose split heads
+    # are merged through the same counters (48 sequences, 4 q heads per kv head)
+    b2 = make_batch([200 + (i * 97) % 2300 for i in range(48)], None, block_size=16, n_q_heads=32,
+                    n_kv_heads=8, head_dim=128, dtype=torch.bfloat16, seed=57)
+    pool2 = gpu_pool_from(b2, 8, 128, torch.bfloat16, cuda_dev)
+    for pl, bb in ((pool, b), (pool2, b2)):
+        (err,) = rt.cudaMemset(dst, 0x01, nbytes)
+        assert err == rt.cudaError_t.cudaSuccess
+        torch.cuda.synchronize(cuda_dev)
+        rc, got = _noalloc(pl, bb, cuda_dev)
+        assert rc == 0, lib().pk_last_error()
+        assert_close(got, oracle_attention(bb), torch.bfloat16, "no-alloc after stale counters")
+        assert pl.check_device_errors() == 0
 
 
 def test_noalloc_with_no_sequences(cuda_dev):
