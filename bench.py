@@ -109,6 +109,18 @@ def new_token_kv(batch, slots):
     return batch["k_pool"][blk, :, off].contiguous(), batch["v_pool"][blk, :, off].contiguous()
 
 
+# ---------------------------------------------------------------- ranks
+def max_over_ranks(ms, device):
+    """The slowest rank's time: replicas run the same work, and the job is done
+    when the last one is (the one collective of a multi-GPU run)."""
+    import torch.distributed as tdist
+    if not tdist.is_available() or not tdist.is_initialized() or tdist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -567,10 +579,7 @@ def run_ours(args, rank, world, device):
     clk = clocks.stop() if not args.profile_run else {"sm_mhz": None, "reasons": ["not sampled"]}
     assert pool.check_device_errors() == 0
 
-    if dist:
-        t = torch.tensor([total_ms], device=device)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, device)
     ms_per_step = total_ms / args.steps
     value = world * (attn_b + app_b) / (ms_per_step * 1e-3) / 1e9
 
@@ -635,11 +644,7 @@ def run_ours(args, rank, world, device):
                 stream.wait_event(done)
             e2.record(stream)
             torch.cuda.synchronize(device)
-            e_ms = s2.elapsed_time(e2)
-            if dist:
-                t = torch.tensor([e_ms], device=device)
-                tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-                e_ms = float(t.item())
+            e_ms = max_over_ranks(s2.elapsed_time(e2), device)
             return e_ms / args.steps
 
         def serial_step(i):
@@ -791,11 +796,7 @@ def run_kvops(args, rank, world, device):
         step(evs[i])
     end.record(stream)
     torch.cuda.synchronize(device)
-    total_ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([total_ms], device=device)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(start.elapsed_time(end), device)
     t_extra = time.perf_counter()
     while not args.profile_run and time.perf_counter() - t_extra < 1.0:
         for _ in range(20):

@@ -97,8 +97,8 @@ int launch_attention_tc(const pk_pool *p, const AttnArgs &a, cudaStream_t st) {
     if (!has_multi && blocks) return launch_decode_blocks(p, a, w, false, st);
     if (blocks && chunk_umma_applies(p, a)) {
         // a mixed continuous-batching step: the one-token rows stream whole
-        // blocks (block-streaming kernel + merge), then the tcgen05 kernel
-        // takes every sequence of several query tokens
+        // blocks (block-streaming kernel, split heads merged in it), then the
+        // tcgen05 kernel takes every sequence of several query tokens
         int rc = launch_decode_blocks(p, a, w, true, st);
         if (rc == PK_OK) rc = launch_chunk_umma(p, a, true, st);
         return rc;

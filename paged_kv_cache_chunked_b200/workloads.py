@@ -183,25 +183,43 @@ def _mix64(x):
     return x
 
 
+_TABLE_ROWS = 1 << 14
+_tables = {}
+
+
+def _value_table(seed, stream, n_heads, head_dim, dtype, device):
+    """A seeded table of _TABLE_ROWS rows of N(0, 1) values [rows, n_heads,
+    head_dim], drawn on the CPU (so every device holds the same bits) and kept."""
+    device = torch.device(device)
+    key = (seed, stream, n_heads, head_dim, dtype, device)
+    t = _tables.get(key)
+    if t is None:
+        cpu_key = (seed, stream, n_heads, head_dim, dtype, torch.device("cpu"))
+        t = _tables.get(cpu_key)
+        if t is None:
+            g = torch.Generator().manual_seed((seed * 1000003 + stream) * 7919 + n_heads * 1009 + head_dim)
+            t = torch.randn((_TABLE_ROWS, n_heads, head_dim), generator=g).to(dtype)
+            _tables[cpu_key] = t
+        t = t.to(device)
+        _tables[key] = t
+    return t
+
+
 def token_values(seed, stream, rids, positions, n_heads, head_dim, dtype, device="cpu"):
     """Deterministic pseudo-normal values for (request id, position) pairs:
     [len(positions), n_heads, head_dim].  stream separates q / k / v.
 
-    Each element is a sum of four 24-bit uniforms (Irwin-Hall), centred and
-    scaled to unit variance, computed with integer hashing and exact-order
-    float32 operations, so CPU and GPU produce the same bits.  Used so that a
-    preempted request recomputes exactly the K/V it had."""
-    rids = torch.as_tensor(rids, dtype=torch.int64, device=device).reshape(-1, 1, 1)
-    pos = torch.as_tensor(positions, dtype=torch.int64, device=device).reshape(-1, 1, 1)
-    h = torch.arange(n_heads, dtype=torch.int64, device=device).reshape(1, -1, 1)
-    e = torch.arange(head_dim, dtype=torch.int64, device=device).reshape(1, 1, -1)
-    key = (((seed * 1000003 + stream) * 1000003 + rids) * 1048576 + pos) * 4096 + h * head_dim + e
-    acc = torch.zeros(key.shape, dtype=torch.float32, device=device)
-    for j in range(4):
-        x = _mix64(key * 4 + j)
-        u = ((x >> 40) & 0xFFFFFF).to(torch.float32) * (1.0 / 16777216.0)
-        acc = acc + u
-    return ((acc - 2.0) * 1.7320508075688772).to(dtype)
+    A counter-based hash (SplitMix64 finaliser) of (seed, stream, request id,
+    position) picks one row of a seeded N(0, 1) table, so a token's values
+    depend only on its key, CPU and GPU produce the same bits, and one gather
+    on the device makes a whole step's values.  Used so that a preempted
+    request recomputes exactly the K/V it had."""
+    rids = torch.as_tensor(rids, dtype=torch.int64)
+    pos = torch.as_tensor(positions, dtype=torch.int64)
+    key = ((seed * 1000003 + stream) * 1000003 + rids) * 1048576 + pos
+    rows = _mix64(key) & (_TABLE_ROWS - 1)
+    table = _value_table(seed, stream, n_heads, head_dim, dtype, device)
+    return table.index_select(0, rows.to(table.device, non_blocking=True))
 
 
 def trace_requests(n_steps=300, arrivals_per_step=4.0, prompt_median=512, prompt_sigma=1.0,
