@@ -719,11 +719,27 @@ def run_ours(args, rank, world, device):
         line["indirection"]["clocks"] = clk2
         line["extra_rooflines"] = {"longdoc_bf16": extra}
     if world == 1 and args.cpu_baseline_seconds > 0 and not args.profile_run:
+        import oracle
         sec, runs, threads = oracle_step_seconds(batch, args.cpu_baseline_seconds)
         line["cpu_baseline"] = {"value": attn_b / sec / 1e9, "unit": "GB/s", "cores": threads,
                                 "kind": "oracle",
                                 "sample": f"float64 oracle attention over the whole {args.workload} "
                                           f"batch (attention bytes only), {runs} runs"}
+        # the same on one host core, over a leading part of the batch (about a
+        # quarter of the budget's worth of all-core runs, at least one sequence)
+        B1 = batch["context_lens"].shape[0]
+        n1 = max(1, min(B1, int(B1 * min(1.0, args.cpu_baseline_seconds / max(sec * threads, 1e-9)))))
+        sub = subset_batch(batch, n1)
+        sub_b, _, _ = step_bytes(sub)
+        oracle.set_num_threads(1)
+        try:
+            sec1, runs1, threads1 = oracle_step_seconds(sub, args.cpu_baseline_seconds / 2)
+        finally:
+            oracle.set_num_threads(threads)
+        line["cpu_baseline_1core"] = {"value": sub_b / sec1 / 1e9, "unit": "GB/s", "cores": threads1,
+                                      "kind": "oracle",
+                                      "sample": f"float64 oracle attention over the first {n1} of {B1} "
+                                                f"sequences of {args.workload} on one core, {runs1} runs"}
     print(json.dumps(line), flush=True)
 
 

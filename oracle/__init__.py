@@ -21,7 +21,7 @@ Contents
 Every pin that ties these to the pages lives in ``tests/test_oracle_*.py``.
 """
 
-from .attention import paged_attention, paged_attention_rows, num_threads  # noqa: F401
+from .attention import paged_attention, paged_attention_rows, num_threads, set_num_threads  # noqa: F401
 from .kv_ops import kv_append, block_copy, swap_blocks  # noqa: F401
 from .allocator import OracleBlockManager, OracleOOM  # noqa: F401
 from . import capacity  # noqa: F401

@@ -56,6 +56,13 @@ def num_threads():
     return _load().oracle_num_threads()
 
 
+def set_num_threads(n):
+    """Host threads for the oracle calls that follow (OpenMP's own setting, in
+    the library the oracle links; the arithmetic is the same at any count)."""
+    _load()
+    ctypes.CDLL("libgomp.so.1").omp_set_num_threads(int(n))
+
+
 def _cpu(t, dtype=None):
     t = t.detach().to("cpu")
     if dtype is not None:
