@@ -134,39 +134,41 @@ void blk_layout(BlkParams &p) {
 // the partitions' normalised rows o_p and log2-sum-exps lse_p, written by other
 // CTAs (read from L2).  The g x D outputs are spread over the lanes (with g
 // dividing 32: 32 / g lanes per row, a block of columns each; otherwise row by
-// row) and the loads of up to four partitions are issued before any is used,
-// so a merge costs a few L2 round trips.  Rows prow + p * HS * g + hl * g + q
-// hold partition p of q head q.
+// row) and the loads of up to four partitions and sixteen columns are issued
+// before any is used: at d = 128 and g = 4 a merge of up to four partitions is
+// one L2 round trip.  Rows prow + p * HS * g + hl * g + q hold partition p of
+// q head q.
 template <int D>
 __device__ __forceinline__ void merge_head(const BlkParams &prm, int prow, int nparts, int qs0, int kvh,
                                            int hl_, int lane) {
     const int g = prm.group, HS = prm.HS, Hq = prm.n_q_heads;
-    constexpr int PB = 4;  // partitions per batch of loads
+    constexpr int PB = 4;   // partitions per batch of loads
+    constexpr int CW = 16;  // most columns per pass
     const bool by_lane = (32 % g) == 0;
     const int lq = by_lane ? 32 / g : 32;          // lanes per row
     const int cols = D / lq;                       // columns per lane and row: 2 .. 64
-    const int cpp = cols < 8 ? cols : 8;           // columns per pass
+    const int cpp = cols < CW ? cols : CW;         // columns per pass
     for (int q = by_lane ? lane / lq : 0; q < g; q += by_lane ? g : 1) {
         const int li = by_lane ? lane % lq : lane;
         for (int cc = 0; cc < cols; cc += cpp) {
             const int col = li * cols + cc;
-            float M = -INFINITY, den = 0.f, acc[8];
+            float M = -INFINITY, den = 0.f, acc[CW];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+            for (int j = 0; j < CW; ++j) acc[j] = 0.f;
             for (int p0 = 0; p0 < nparts; p0 += PB) {
                 float l[PB];
-                float2 x[PB][4];
+                float2 x[PB][CW / 2];
 #pragma unroll
                 for (int i = 0; i < PB; ++i) {
                     l[i] = -INFINITY;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) x[i][j] = make_float2(0.f, 0.f);
+                    for (int j = 0; j < CW / 2; ++j) x[i][j] = make_float2(0.f, 0.f);
                     if (p0 + i < nparts) {
                         const int row = prow + (p0 + i) * HS * g + hl_ * g + q;
                         l[i] = __ldcg(prm.partial_lse + row);
                         const float2 *src = (const float2 *)(prm.partial_o + (size_t)row * D + col);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
+                        for (int j = 0; j < CW / 2; ++j)
                             if (2 * j < cpp) x[i][j] = __ldcg(src + j);
                     }
                 }
@@ -177,14 +179,14 @@ __device__ __forceinline__ void merge_head(const BlkParams &prm, int prow, int n
                 const float a = M == -INFINITY ? 0.f : fast_exp2(M - bm);
                 den *= a;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) acc[j] *= a;
+                for (int j = 0; j < CW; ++j) acc[j] *= a;
                 M = bm;
 #pragma unroll
                 for (int i = 0; i < PB; ++i) {
                     const float w = l[i] == -INFINITY ? 0.f : fast_exp2(l[i] - M);
                     den += w;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
+                    for (int j = 0; j < CW / 2; ++j) {
                         acc[2 * j] += w * x[i][j].x;
                         acc[2 * j + 1] += w * x[i][j].y;
                     }
@@ -193,7 +195,7 @@ __device__ __forceinline__ void merge_head(const BlkParams &prm, int prow, int n
             const float inv = den > 0.f ? 1.f / den : 0.f;
             __nv_bfloat16 *dst = prm.out + ((long long)qs0 * Hq + kvh * g + q) * D + col;
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < CW / 2; ++j)
                 if (2 * j < cpp) *(uint32_t *)(dst + 2 * j) = pack_bf16(acc[2 * j] * inv, acc[2 * j + 1] * inv);
         }
     }
@@ -206,9 +208,12 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
     constexpr int KS = D / 16;
     constexpr int NPN = D / 64;  // 64-column panels
     extern __shared__ uint8_t smem_raw[];
-    // launched as a programmatic dependent of the previous kernel on the stream
-    // (the KV append): nothing is read before that grid has finished
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // Launched as a programmatic dependent of the previous kernel on the stream
+    // (the KV append or block copy, which write pool rows only).  The plan, the
+    // query rows and the block tables are read while that kernel may still
+    // run; the pool is read, and anything written, only after
+    // griddepcontrol.wait: by the producer before its first K/V copy, by the
+    // consumers at their start.
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int NS = prm.NS, HS = prm.HS, NBS = prm.NBS, ST = prm.ST, NPH = prm.NPH;
@@ -242,6 +247,12 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
         mbar_init(cbar, kNC);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    // the window's query offsets and context lengths, one load per thread
+    for (int i = threadIdx.x; i <= nseq; i += kBlkThreads) {
+        s_qsl[i] = __ldg(prm.qsl + prm.seq0 + i);
+        if (i < nseq) s_ctx[i] = __ldg(prm.ctx + prm.seq0 + i);
+    }
+    __syncthreads();
     // ---------------------------------------------------------------- plan
     // per sequence: S_b = ceil(c_b / ST) stages per head group; chunk size CS;
     // a (sequence, head group) spanning several chunks has one partition per
@@ -254,11 +265,7 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
             const int i = base + lane;
             int ns = 0;
             if (i < nseq) {
-                const int b = prm.seq0 + i;
-                const int s0 = __ldg(prm.qsl + b), s1 = __ldg(prm.qsl + b + 1), c = __ldg(prm.ctx + b);
-                s_qsl[i] = s0;
-                s_ctx[i] = c;
-                if (i == nseq - 1) s_qsl[nseq] = s1;
+                const int s0 = s_qsl[i], s1 = s_qsl[i + 1], c = s_ctx[i];
                 const bool ok = s0 >= 0 && s1 <= prm.num_tokens && s1 - s0 >= 1 && c >= s1 - s0 &&
                                 (long long)(c + bs - 1) / bs <= prm.max_blocks &&
                                 (s1 - s0 == 1 || prm.skip_chunks);
@@ -348,6 +355,8 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
         const int nchunks = cp.count();
         int pending = (int)blockIdx.x;
         int n_stage = 0, n_item = 0;
+        bool waited = false;  // griddepcontrol.wait done
+        const uint64_t stream_pol = l2_evict_first_policy();  // K/V rows are read once
         auto chunk_entry = [&](int b, int blk_base) -> int {
             const int nblk = (s_ctx[b] + bs - 1) / bs;
             const int e = blk_base + lane;
@@ -434,6 +443,10 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                 return phys;
             };
             const int nblk = (c + bs - 1) / bs;
+            if (!waited) {  // the preceding kernel's pool rows are visible from here on
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+                waited = true;
+            }
             for (int st = cur.st0; st < cur.st0 + cur.cnt; ++st) {
                 const int s = n_stage % NS;
                 if (n_stage >= NS && !mbar_wait(&empty[s], ((n_stage / NS) - 1) & 1)) {
@@ -455,8 +468,8 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                     const int phys = table_get(blk0 + j);
                     const int y = (phys * Hkv + hg * HS) * bs;
                     if (lane == 0) {  // all panels of the block's rows: one box for K, one for V
-                        tma_load_3d(kst + j * piece_bytes, &tmk, 0, y, 0, &full[s]);
-                        tma_load_3d(vst + j * piece_bytes, &tmv, 0, y, 0, &full[s]);
+                        tma_load_3d_hint(kst + j * piece_bytes, &tmk, 0, y, 0, &full[s], stream_pol);
+                        tma_load_3d_hint(vst + j * piece_bytes, &tmv, 0, y, 0, &full[s], stream_pol);
                     }
                 }
                 __syncwarp();
@@ -487,6 +500,7 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
         }
     } else {
         // ---------------------------------------------------------- consumers
+        asm volatile("griddepcontrol.wait;" ::: "memory");  // before any write
         const int cw = warp - 1, hl = cw % HS, ph = cw / HS;
         const int qr = lane >> 2, qc = (lane & 3) * 2;
         const int mi = lane >> 3, rr = lane & 7;
@@ -680,6 +694,9 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                         }
                     }
                 } else {
+                    // partial rows are read back by the merge, often at the end of
+                    // the launch: kept in L2 past the K/V stream
+                    const uint64_t keep = l2_evict_last_policy();
                     const int row = d.prow + d.part * HS * g + hl * g;
                     float *pa_ = prm.partial_o + (size_t)(row + ha) * D;
                     float *pb_ = pa_ + D;
@@ -687,18 +704,18 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                     for (int mt = 0; mt < KS; ++mt) {
                         const int d0 = mt * 16 + qr;
                         if (va_) {
-                            pa_[d0] = ot[mt][0] * ia;
-                            pa_[d0 + 8] = ot[mt][2] * ia;
+                            st_l2_keep(pa_ + d0, ot[mt][0] * ia, keep);
+                            st_l2_keep(pa_ + d0 + 8, ot[mt][2] * ia, keep);
                         }
                         if (vb_) {
-                            pb_[d0] = ot[mt][1] * ib;
-                            pb_[d0 + 8] = ot[mt][3] * ib;
+                            st_l2_keep(pb_ + d0, ot[mt][1] * ib, keep);
+                            st_l2_keep(pb_ + d0 + 8, ot[mt][3] * ib, keep);
                         }
                     }
                     if (qr == 0) {
                         float *pl = prm.partial_lse + (size_t)row;
-                        if (va_) pl[ha] = l0 > 0.f ? m0 + __log2f(l0) : -INFINITY;
-                        if (vb_) pl[hb] = l1 > 0.f ? m1 + __log2f(l1) : -INFINITY;
+                        if (va_) st_l2_keep(pl + ha, l0 > 0.f ? m0 + __log2f(l0) : -INFINITY, keep);
+                        if (vb_) st_l2_keep(pl + hb, l1 > 0.f ? m1 + __log2f(l1) : -INFINITY, keep);
                     }
                     // arrival: the warp that writes the last partition of this
                     // (sequence, kv head) merges its rows

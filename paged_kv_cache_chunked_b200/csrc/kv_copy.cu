@@ -17,9 +17,30 @@
 namespace pk {
 namespace {
 
-struct alignas(16) Vec16 {
-    uint4 v;
-};
+// Each kernel here is launched as a programmatic dependent of the previous
+// kernel on the stream (launch_pdl).  It lets its own dependent (the next copy,
+// or the attention kernel, whose plan reads no pool rows) start launching at
+// once, then waits for the previous grid to finish, and its writes to be
+// visible, before it touches any memory: stream order as seen by memory is
+// unchanged, but the launch no longer waits for the previous grid's last CTA.
+__device__ __forceinline__ void pdl_prologue() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int threads, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, ((KArgs)args)...);
+}
 
 // One thread per 16-byte chunk of one (token, head) row of K or V.
 // Grid-stride over num_tokens * n_kv_heads * row_chunks * 2.
@@ -28,9 +49,7 @@ __global__ void kv_append_vec16(const uint4 *__restrict__ k, const uint4 *__rest
                                 const int64_t *__restrict__ slots, int num_tokens, int n_kv_heads,
                                 int block_size, int row_chunks, int64_t num_slots,
                                 int *err) {
-    // a dependent kernel (attention launched with programmatic serialisation)
-    // may start its launch now; it waits for this grid before reading
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    pdl_prologue();
     const int64_t per_side = (int64_t)num_tokens * n_kv_heads * row_chunks;
     const int64_t total = 2 * per_side;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
@@ -61,9 +80,7 @@ __global__ void kv_append_scalar(const T *__restrict__ k, const T *__restrict__ 
                                  const int64_t *__restrict__ slots, int num_tokens,
                                  int n_kv_heads, int block_size, int head_dim,
                                  int64_t num_slots, int *err) {
-    // a dependent kernel (attention launched with programmatic serialisation)
-    // may start its launch now; it waits for this grid before reading
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    pdl_prologue();
     const int64_t per_side = (int64_t)num_tokens * n_kv_heads * head_dim;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < 2 * per_side;
          i += (int64_t)gridDim.x * blockDim.x) {
@@ -88,9 +105,7 @@ __global__ void kv_append_scalar(const T *__restrict__ k, const T *__restrict__ 
 // One CTA per (pair, K or V); the block's bytes are copied as 16-byte vectors.
 __global__ void block_copy_vec16(uint4 *kp, uint4 *vp, const int32_t *__restrict__ pairs,
                                  int n_pairs, int64_t block_chunks, int num_blocks, int *err) {
-    // a dependent kernel (attention launched with programmatic serialisation)
-    // may start its launch now; it waits for this grid before reading
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    pdl_prologue();
     for (int64_t w = blockIdx.x; w < 2LL * n_pairs; w += gridDim.x) {
         const int pr = (int)(w >> 1);
         uint4 *pool = (w & 1) ? vp : kp;
@@ -119,9 +134,7 @@ __global__ void block_copy_vec16(uint4 *kp, uint4 *vp, const int32_t *__restrict
 template <typename T>
 __global__ void block_copy_scalar(T *kp, T *vp, const int32_t *__restrict__ pairs, int n_pairs,
                                   int64_t block_elems, int num_blocks, int *err) {
-    // a dependent kernel (attention launched with programmatic serialisation)
-    // may start its launch now; it waits for this grid before reading
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    pdl_prologue();
     for (int64_t w = blockIdx.x; w < 2LL * n_pairs; w += gridDim.x) {
         const int pr = (int)(w >> 1);
         T *pool = (w & 1) ? vp : kp;
@@ -143,7 +156,7 @@ template <typename T, int UNROLL>
 __global__ void swap_copy(const T *__restrict__ sk, const T *__restrict__ sv, T *dk, T *dv,
                           const int32_t *__restrict__ pairs, int n_pairs, int64_t block_chunks,
                           int n_src, int n_dst, int *err) {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    pdl_prologue();
     for (int64_t w = blockIdx.x; w < 2LL * n_pairs; w += gridDim.x) {
         const int pr = (int)(w >> 1);
         const int a = __ldg(pairs + 2 * pr), b = __ldg(pairs + 2 * pr + 1);
@@ -183,26 +196,25 @@ int launch_kv_append(const pk_pool *p, const void *k, const void *v, const int64
     const int elt = p->dtype == PK_BF16 ? 2 : 4;
     const int64_t row_bytes = (int64_t)p->head_dim * elt;
     const int64_t num_slots = (int64_t)p->num_blocks * p->block_size;
+    cudaError_t e;
     if (row_bytes % 16 == 0 && aligned16(k) && aligned16(v)) {
         const int row_chunks = (int)(row_bytes / 16);
         const int64_t work = 2LL * num_tokens * p->n_kv_heads * row_chunks;
-        kv_append_vec16<<<grid_for(work, 256, p->sm_count), 256, 0, st>>>(
-            (const uint4 *)k, (const uint4 *)v, (uint4 *)p->k_base, (uint4 *)p->v_base, slots,
-            num_tokens, p->n_kv_heads, p->block_size, row_chunks, num_slots, p->d_err);
+        e = launch_pdl(kv_append_vec16, grid_for(work, 256, p->sm_count), 256, st, (const uint4 *)k,
+                       (const uint4 *)v, (uint4 *)p->k_base, (uint4 *)p->v_base, slots, num_tokens,
+                       p->n_kv_heads, p->block_size, row_chunks, num_slots, p->d_err);
     } else {
         const int64_t work = 2LL * num_tokens * p->n_kv_heads * p->head_dim;
+        const int grid = grid_for(work, 256, p->sm_count);
         if (p->dtype == PK_BF16)
-            kv_append_scalar<uint16_t><<<grid_for(work, 256, p->sm_count), 256, 0, st>>>(
-                (const uint16_t *)k, (const uint16_t *)v, (uint16_t *)p->k_base,
-                (uint16_t *)p->v_base, slots, num_tokens, p->n_kv_heads, p->block_size,
-                p->head_dim, num_slots, p->d_err);
+            e = launch_pdl(kv_append_scalar<uint16_t>, grid, 256, st, (const uint16_t *)k,
+                           (const uint16_t *)v, (uint16_t *)p->k_base, (uint16_t *)p->v_base, slots,
+                           num_tokens, p->n_kv_heads, p->block_size, p->head_dim, num_slots, p->d_err);
         else
-            kv_append_scalar<float><<<grid_for(work, 256, p->sm_count), 256, 0, st>>>(
-                (const float *)k, (const float *)v, (float *)p->k_base, (float *)p->v_base,
-                slots, num_tokens, p->n_kv_heads, p->block_size, p->head_dim, num_slots,
-                p->d_err);
+            e = launch_pdl(kv_append_scalar<float>, grid, 256, st, (const float *)k, (const float *)v,
+                           (float *)p->k_base, (float *)p->v_base, slots, num_tokens, p->n_kv_heads,
+                           p->block_size, p->head_dim, num_slots, p->d_err);
     }
-    cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? PK_OK : cuda_fail(e, "kv append launch");
 }
 
@@ -218,20 +230,18 @@ int launch_swap_blocks(const pk_pool *p, void *host_k, void *host_v, int num_hos
     const int n_dst = to_host ? num_host_blocks : p->num_blocks;
     const int64_t ctas = 2LL * n_pairs;
     const int grid = (int)(ctas < (int64_t)p->sm_count * 32 ? ctas : (int64_t)p->sm_count * 32);
-    if (block_bytes % 16 == 0 && aligned16(sk) && aligned16(sv) && aligned16(dk) && aligned16(dv)) {
-        swap_copy<uint4, 4><<<grid, 256, 0, st>>>((const uint4 *)sk, (const uint4 *)sv, (uint4 *)dk,
-                                                  (uint4 *)dv, pairs, n_pairs, block_bytes / 16, n_src,
-                                                  n_dst, p->d_err);
-    } else if (p->dtype == PK_BF16) {
-        swap_copy<uint16_t, 4><<<grid, 256, 0, st>>>((const uint16_t *)sk, (const uint16_t *)sv,
-                                                     (uint16_t *)dk, (uint16_t *)dv, pairs, n_pairs,
-                                                     block_elems, n_src, n_dst, p->d_err);
-    } else {
-        swap_copy<float, 4><<<grid, 256, 0, st>>>((const float *)sk, (const float *)sv, (float *)dk,
-                                                  (float *)dv, pairs, n_pairs, block_elems, n_src,
-                                                  n_dst, p->d_err);
-    }
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e;
+    if (block_bytes % 16 == 0 && aligned16(sk) && aligned16(sv) && aligned16(dk) && aligned16(dv))
+        e = launch_pdl(swap_copy<uint4, 4>, grid, 256, st, (const uint4 *)sk, (const uint4 *)sv,
+                       (uint4 *)dk, (uint4 *)dv, pairs, n_pairs, block_bytes / 16, n_src, n_dst,
+                       p->d_err);
+    else if (p->dtype == PK_BF16)
+        e = launch_pdl(swap_copy<uint16_t, 4>, grid, 256, st, (const uint16_t *)sk,
+                       (const uint16_t *)sv, (uint16_t *)dk, (uint16_t *)dv, pairs, n_pairs,
+                       block_elems, n_src, n_dst, p->d_err);
+    else
+        e = launch_pdl(swap_copy<float, 4>, grid, 256, st, (const float *)sk, (const float *)sv,
+                       (float *)dk, (float *)dv, pairs, n_pairs, block_elems, n_src, n_dst, p->d_err);
     return e == cudaSuccess ? PK_OK : cuda_fail(e, "block swap launch");
 }
 
@@ -242,20 +252,16 @@ int launch_block_copy(const pk_pool *p, const int32_t *pairs, int n_pairs, cudaS
     const int64_t block_bytes = block_elems * elt;
     const int64_t ctas = 2LL * n_pairs;
     const int grid = (int)(ctas < (int64_t)p->sm_count * 32 ? ctas : (int64_t)p->sm_count * 32);
-    if (block_bytes % 16 == 0) {
-        block_copy_vec16<<<grid, 256, 0, st>>>((uint4 *)p->k_base, (uint4 *)p->v_base, pairs,
-                                               n_pairs, block_bytes / 16, p->num_blocks,
-                                               p->d_err);
-    } else if (p->dtype == PK_BF16) {
-        block_copy_scalar<uint16_t><<<grid, 256, 0, st>>>((uint16_t *)p->k_base,
-                                                          (uint16_t *)p->v_base, pairs, n_pairs,
-                                                          block_elems, p->num_blocks, p->d_err);
-    } else {
-        block_copy_scalar<float><<<grid, 256, 0, st>>>((float *)p->k_base, (float *)p->v_base,
-                                                       pairs, n_pairs, block_elems,
-                                                       p->num_blocks, p->d_err);
-    }
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e;
+    if (block_bytes % 16 == 0)
+        e = launch_pdl(block_copy_vec16, grid, 256, st, (uint4 *)p->k_base, (uint4 *)p->v_base, pairs,
+                       n_pairs, block_bytes / 16, p->num_blocks, p->d_err);
+    else if (p->dtype == PK_BF16)
+        e = launch_pdl(block_copy_scalar<uint16_t>, grid, 256, st, (uint16_t *)p->k_base,
+                       (uint16_t *)p->v_base, pairs, n_pairs, block_elems, p->num_blocks, p->d_err);
+    else
+        e = launch_pdl(block_copy_scalar<float>, grid, 256, st, (float *)p->k_base,
+                       (float *)p->v_base, pairs, n_pairs, block_elems, p->num_blocks, p->d_err);
     return e == cudaSuccess ? PK_OK : cuda_fail(e, "block copy launch");
 }
 
