@@ -29,12 +29,13 @@
 // stages of all (sequence, head group) pairs are concatenated and cut into one
 // equal chunk per CTA.  The part of a pair inside one chunk is a partition; a
 // pair cut into several partitions writes (normalised O, log2-sum-exp) rows per
-// partition and kv head, and the consumer warp that writes the last partition
-// of a (sequence, kv head), found by an arrival counter in the workspace,
-// merges that head's rows once its own stages are done (no wait anywhere: a
-// fence and an atomic add per split head).  A chunk holds at most two split
-// partitions (its first and its last pair), so a warp has at most two merges
-// to do.
+// partition and kv head, and a merge kernel, launched behind this one as a
+// programmatic dependent, combines them once the streaming is over.  (Merging
+// inside this kernel, by the last writer of each head, was slower: at the end
+// of a launch the other SMs still stream, and a merge's loads wait behind
+// their traffic for several microseconds.)  A chunk holds at most two split
+// partitions (its first and its last pair), so fewer pairs than chunks are
+// split.
 //
 // Every wait is bounded (2 s); on expiry the kernel records PK_ERR_TIMEOUT,
 // waits (bounded) for its own copies in flight and returns.  Block ids are
@@ -54,7 +55,6 @@ constexpr int kStageCap = 64 * 1024;          // K + V bytes of one stage
 constexpr int kMinChunkStages = 2;            // smallest chunk
 constexpr int kItemSlots = 2;                 // items staged ahead (Q rows + descriptor each)
 constexpr float kRescaleLog2 = 8.f;           // lazy softmax rescale threshold (log2 units)
-constexpr int kMaxDeferred = 4;               // split-K merges a consumer warp keeps for its end (2 needed)
 constexpr int kMergeListHead = 4;             // merge kernel's list: count, pad, then int4 entries
 
 enum : int { kFirst = 1, kLast = 2, kEnd = 4 };
@@ -95,13 +95,11 @@ struct BlkParams {
     int HS, NBS, ST, NPH, NS;  // geometry: heads / blocks / tokens per stage, phases, stages
     int ncta, cap_rows;
     float scale_log2;
-    int merge_in_kernel;             // 1: split heads are merged by their last writer; 0: by the merge kernel
-    int *counters;                   // split-K arrivals per (sequence of the window, kv head)
-    int *mplan;                      // merge kernel's list (merge_in_kernel == 0)
+    int *mplan;                      // the merge kernel's list of split pairs
     float *partial_o, *partial_lse;  // [row][D], [row]
     int *err;
     // shared-memory layout (byte offsets from the 1024-aligned base)
-    uint32_t stage_bytes, qslot_bytes, off_q, off_scr, off_plan, off_desc, off_info, off_defer, off_bar, total;
+    uint32_t stage_bytes, qslot_bytes, off_q, off_scr, off_plan, off_desc, off_info, off_bar, total;
 };
 
 // Shared-memory layout of one launch.
@@ -122,83 +120,9 @@ void blk_layout(BlkParams &p) {
     off += kItemSlots * sizeof(ItemDesc);
     p.off_info = off;
     off += (uint32_t)p.NS * sizeof(StageInfo);
-    p.off_defer = up(off, 16);
-    off = p.off_defer + (uint32_t)kNC * kMaxDeferred * sizeof(int4);
     p.off_bar = up(off, 8);
     off = p.off_bar + (uint32_t)(2 * p.NS + 2 * kItemSlots + 1) * 8;
     p.total = off + 1024;  // + alignment slack
-}
-
-// Split-K merge of one kv head's g rows [flash-decoding combination]:
-// out = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M), M = max_p lse_p, over
-// the partitions' normalised rows o_p and log2-sum-exps lse_p, written by other
-// CTAs (read from L2).  The g x D outputs are spread over the lanes (with g
-// dividing 32: 32 / g lanes per row, a block of columns each; otherwise row by
-// row) and the loads of up to four partitions and sixteen columns are issued
-// before any is used: at d = 128 and g = 4 a merge of up to four partitions is
-// one L2 round trip.  Rows prow + p * HS * g + hl * g + q hold partition p of
-// q head q.
-template <int D>
-__device__ __forceinline__ void merge_head(const BlkParams &prm, int prow, int nparts, int qs0, int kvh,
-                                           int hl_, int lane) {
-    const int g = prm.group, HS = prm.HS, Hq = prm.n_q_heads;
-    constexpr int PB = 4;   // partitions per batch of loads
-    constexpr int CW = 16;  // most columns per pass
-    const bool by_lane = (32 % g) == 0;
-    const int lq = by_lane ? 32 / g : 32;          // lanes per row
-    const int cols = D / lq;                       // columns per lane and row: 2 .. 64
-    const int cpp = cols < CW ? cols : CW;         // columns per pass
-    for (int q = by_lane ? lane / lq : 0; q < g; q += by_lane ? g : 1) {
-        const int li = by_lane ? lane % lq : lane;
-        for (int cc = 0; cc < cols; cc += cpp) {
-            const int col = li * cols + cc;
-            float M = -INFINITY, den = 0.f, acc[CW];
-#pragma unroll
-            for (int j = 0; j < CW; ++j) acc[j] = 0.f;
-            for (int p0 = 0; p0 < nparts; p0 += PB) {
-                float l[PB];
-                float2 x[PB][CW / 2];
-#pragma unroll
-                for (int i = 0; i < PB; ++i) {
-                    l[i] = -INFINITY;
-#pragma unroll
-                    for (int j = 0; j < CW / 2; ++j) x[i][j] = make_float2(0.f, 0.f);
-                    if (p0 + i < nparts) {
-                        const int row = prow + (p0 + i) * HS * g + hl_ * g + q;
-                        l[i] = __ldcg(prm.partial_lse + row);
-                        const float2 *src = (const float2 *)(prm.partial_o + (size_t)row * D + col);
-#pragma unroll
-                        for (int j = 0; j < CW / 2; ++j)
-                            if (2 * j < cpp) x[i][j] = __ldcg(src + j);
-                    }
-                }
-                float bm = M;
-#pragma unroll
-                for (int i = 0; i < PB; ++i) bm = fmaxf(bm, l[i]);
-                if (bm == -INFINITY) continue;
-                const float a = M == -INFINITY ? 0.f : fast_exp2(M - bm);
-                den *= a;
-#pragma unroll
-                for (int j = 0; j < CW; ++j) acc[j] *= a;
-                M = bm;
-#pragma unroll
-                for (int i = 0; i < PB; ++i) {
-                    const float w = l[i] == -INFINITY ? 0.f : fast_exp2(l[i] - M);
-                    den += w;
-#pragma unroll
-                    for (int j = 0; j < CW / 2; ++j) {
-                        acc[2 * j] += w * x[i][j].x;
-                        acc[2 * j + 1] += w * x[i][j].y;
-                    }
-                }
-            }
-            const float inv = den > 0.f ? 1.f / den : 0.f;
-            __nv_bfloat16 *dst = prm.out + ((long long)qs0 * Hq + kvh * g + q) * D + col;
-#pragma unroll
-            for (int j = 0; j < CW / 2; ++j)
-                if (2 * j < cpp) *(uint32_t *)(dst + 2 * j) = pack_bf16(acc[2 * j] * inv, acc[2 * j + 1] * inv);
-        }
-    }
 }
 
 template <int D>
@@ -321,27 +245,6 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
             s_cp = cp;
         }
         __syncwarp();
-        if (!prm.merge_in_kernel && blockIdx.x == 0) {
-            // the merge kernel's work list: (sequence, head group, first partial
-            // row, partitions) of every pair cut into several partitions
-            int n_split = 0;
-            for (int base = 0; base < nseq; base += 32) {
-                const int i = base + lane;
-                const int sb = i < nseq ? (stage_pre[i + 1] - stage_pre[i]) / NHG : 0;
-                int prow = i < nseq ? prow_pre[i] : 0;
-                for (int hg = 0; hg < NHG; ++hg) {
-                    const int n = sb > 0 ? cp.parts(stage_pre[i] + hg * sb, sb) : 1;
-                    const unsigned m = __ballot_sync(0xffffffffu, n > 1);
-                    if (n > 1) {
-                        int4 *e = (int4 *)(prm.mplan + kMergeListHead) + n_split + __popc(m & ((1u << lane) - 1));
-                        *e = make_int4(i, hg, prow, n);
-                        prow += n * HS * g;
-                    }
-                    n_split += __popc(m);
-                }
-            }
-            if (lane == 0) prm.mplan[0] = n_split;
-        }
     }
     // a merge kernel, if one follows, may be scheduled now; it waits for this grid to finish
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -490,6 +393,30 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                 ++n_stage;
             }
         }
+        if (blockIdx.x == 0) {
+            // the merge kernel's work list: (sequence, head group, first partial
+            // row, partitions) of every pair cut into several partitions.  The
+            // previous merge kernel on the stream reads its list until its grid
+            // ends, so this one is written after the wait.
+            if (!waited) asm volatile("griddepcontrol.wait;" ::: "memory");
+            int n_split = 0;
+            for (int base = 0; base < nseq; base += 32) {
+                const int i = base + lane;
+                const int sb = i < nseq ? (stage_pre[i + 1] - stage_pre[i]) / NHG : 0;
+                int prow = i < nseq ? prow_pre[i] : 0;
+                for (int hg = 0; hg < NHG; ++hg) {
+                    const int n = sb > 0 ? cp.parts(stage_pre[i] + hg * sb, sb) : 1;
+                    const unsigned m = __ballot_sync(0xffffffffu, n > 1);
+                    if (n > 1) {
+                        int4 *e = (int4 *)(prm.mplan + kMergeListHead) + n_split + __popc(m & ((1u << lane) - 1));
+                        *e = make_int4(i, hg, prow, n);
+                        prow += n * HS * g;
+                    }
+                    n_split += __popc(m);
+                }
+            }
+            if (lane == 0) prm.mplan[0] = n_split;
+        }
         if (!ok) {
             if (lane == 0) record_error(prm.err, PK_ERR_TIMEOUT);
             // never leave with a copy still writing into this CTA's shared memory
@@ -622,9 +549,6 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                 mma_bf16(ot[mt], a0, a1, a2, a3, b0, b1);
             }
         };
-        // merges this warp found itself last for, run once its stages are done
-        int4 *deferred = (int4 *)(sm + prm.off_defer) + cw * kMaxDeferred;
-        int n_deferred = 0;
         float *scr = (float *)(sm + prm.off_scr);
         constexpr int kScr = KS * 4 + 4;  // floats per lane of one warp's state
         auto finish_item = [&](int slot) -> bool {
@@ -694,8 +618,8 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                         }
                     }
                 } else {
-                    // partial rows are read back by the merge, often at the end of
-                    // the launch: kept in L2 past the K/V stream
+                    // partial rows are read back by the merge kernel: kept in L2
+                    // past the K/V stream that follows them
                     const uint64_t keep = l2_evict_last_policy();
                     const int row = d.prow + d.part * HS * g + hl * g;
                     float *pa_ = prm.partial_o + (size_t)(row + ha) * D;
@@ -716,26 +640,6 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                         float *pl = prm.partial_lse + (size_t)row;
                         if (va_) st_l2_keep(pl + ha, l0 > 0.f ? m0 + __log2f(l0) : -INFINITY, keep);
                         if (vb_) st_l2_keep(pl + hb, l1 > 0.f ? m1 + __log2f(l1) : -INFINITY, keep);
-                    }
-                    // arrival: the warp that writes the last partition of this
-                    // (sequence, kv head) merges its rows
-                    __threadfence();  // every lane's partial rows, before the arrival
-                    __syncwarp();
-                    int last = 0;
-                    if (prm.merge_in_kernel && lane == 0) {
-                        int *cnt = prm.counters + (size_t)d.b * Hkv + kvh;
-                        last = atomicAdd(cnt, 1) == d.nparts - 1;
-                        if (last) *cnt = 0;  // leave the counter zeroed for the next call
-                    }
-                    if (__shfl_sync(0xffffffffu, last, 0)) {
-                        // a chunk holds at most two split partitions, so the list
-                        // never fills; were it to, the error word says so
-                        if (n_deferred < kMaxDeferred) {
-                            if (lane == 0) deferred[n_deferred] = make_int4(d.prow, d.nparts, d.qs0, kvh);
-                            ++n_deferred;
-                        } else if (lane == 0) {
-                            record_error(prm.err, PK_ERR_UNSUPPORTED);
-                        }
                     }
                 }
             }
@@ -771,25 +675,19 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                 break;
             }
         }
-        if (ok && n_deferred > 0) {
-            __syncwarp();
-            __threadfence();  // the other partitions' rows after their arrivals
-            for (int i = 0; i < n_deferred; ++i) {
-                const int4 e = deferred[i];
-                merge_head<D>(prm, e.x, e.y, e.z, e.w, hl, lane);
-            }
-        }
         if (!ok && lane == 0) record_error(prm.err, PK_ERR_TIMEOUT);
     }
     __syncthreads();
 }
 
-// Merge kernel, for launches whose pairs are cut into many partitions (few
-// long sequences): the merge then needs more of the GPU than the last writer
-// of each head [flash-decoding combination].  For every (sequence, head group)
-// that the streaming kernel cut into several partitions, each output row (q head hg * HS * g + r of the sequence's token)
-// is out = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M), M = max_p lse_p, over
-// the partitions' normalised rows o_p and log2-sum-exps lse_p.
+// Merge kernel [flash-decoding combination].  For every (sequence, head
+// group) that the streaming kernel cut into several partitions, each output
+// row (q head hg * HS * g + r of the sequence's token) is
+// out = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M), M = max_p lse_p, over
+// the partitions' normalised rows o_p and log2-sum-exps lse_p.  Launched as a
+// programmatic dependent of the streaming kernel, its CTAs are resident
+// before that grid ends and start the moment it does, when the memory system
+// is quiet and the partial rows are still in L2.
 // The streaming kernel lists the split pairs.  blockIdx.x = list entry,
 // blockIdx.y = a block of kMergeThreads outputs (row, 4 columns) of that
 // pair; one thread per output folds the partitions eight at a time, all of a
@@ -808,7 +706,11 @@ constexpr int kMergeBatch = 8;
 
 template <int D>
 __global__ void __launch_bounds__(kMergeThreads) attention_merge_kernel(const MergeParams mp) {
-    asm volatile("griddepcontrol.wait;" ::: "memory");  // the streaming kernel has finished
+    // the next kernel on the stream may start launching (it waits for this
+    // grid before touching memory); the streaming kernel has finished once
+    // the wait returns
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int HG = mp.HS * mp.group;
     const int unit = blockIdx.y * kMergeThreads + threadIdx.x;
     const int n_split = __ldcg(mp.mplan);
@@ -900,7 +802,6 @@ int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, bool s
     tp.ncta = p->sm_count;
     tp.cap_rows = w.cap_rows;
     tp.scale_log2 = a.scale * 1.4426950408889634f;
-    tp.counters = w.counters;
     tp.mplan = w.merge_plan;
     tp.partial_o = w.partial_o;
     tp.partial_lse = w.partial_lse;
@@ -916,14 +817,6 @@ int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, bool s
     for (int s0 = 0; s0 < a.num_seqs; s0 += kMaxSeqsPerLaunch) {
         tp.seq0 = s0;
         tp.nseq = std::min(kMaxSeqsPerLaunch, a.num_seqs - s0);
-        // Split heads are merged in the streaming kernel by their last writer
-        // when the window has enough (sequence, head group) pairs for about four
-        // partitions per pair at most; with fewer, longer pairs (each cut into
-        // many partitions) a merge kernel spreads the merging over the GPU.  In
-        // a batch with prefill chunks the decode rows are an unknown part of
-        // the window (often none), so there it is always the last writer.
-        tp.merge_in_kernel =
-            skip_chunks || 4LL * tp.nseq * (tp.n_kv_heads / tp.HS) >= tp.ncta ? 1 : 0;
         {
             cudaLaunchConfig_t c0 = {};
             c0.gridDim = dim3(tp.ncta);
@@ -938,7 +831,6 @@ int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, bool s
             const cudaError_t e0 = cudaLaunchKernelEx(&c0, attention_decode_blocks_kernel<D>, p->tmap_kb, p->tmap_vb, tp);
             if (e0 != cudaSuccess) return cuda_fail(e0, "decode attention launch");
         }
-        if (tp.merge_in_kernel) continue;
         MergeParams mp;
         mp.out = tp.out;
         mp.qsl = tp.qsl;
@@ -951,9 +843,11 @@ int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, bool s
         mp.HS = tp.HS;
         const int units = tp.HS * tp.group * (D / 4);
         cudaLaunchConfig_t cfg = {};
-        // one block row per possible split pair (sequence, head group); blocks past
-        // the list's end return at once
-        cfg.gridDim = dim3(tp.nseq * (tp.n_kv_heads / tp.HS), (units + kMergeThreads - 1) / kMergeThreads);
+        // one block row per possible split pair (sequence, head group): each split
+        // pair holds a chunk boundary, so there are fewer than the chunks (at most
+        // one per SM); blocks past the list's end return at once
+        const int pairs = tp.nseq * (tp.n_kv_heads / tp.HS);
+        cfg.gridDim = dim3(std::min(pairs, tp.ncta), (units + kMergeThreads - 1) / kMergeThreads);
         cfg.blockDim = dim3(kMergeThreads);
         cfg.dynamicSmemBytes = 0;
         cfg.stream = st;

@@ -152,12 +152,11 @@ def test_permuted_block_ids_bit_identical(cuda_dev, ql):
         assert torch.equal(o, outs[0])
 
 
-def test_in_kernel_merge_bit_identical_under_permutations(cuda_dev):
-    # 48 decode rows of 8 kv heads: enough (sequence, head group) pairs for the
-    # block-streaming kernel to merge split heads itself, by the warp that writes
-    # each head's last partition.  Which warp that is depends on timing; the
-    # merge order (by partition) does not, so the output is bit-identical under
-    # any placement of the blocks, and equal to the oracle
+def test_split_k_merge_bit_identical_under_permutations(cuda_dev):
+    # 48 decode rows of 8 kv heads on the block-streaming kernel: pairs cut
+    # into partitions at chunk boundaries are combined by the merge kernel in
+    # partition order, whatever CTA finished first, so the output is
+    # bit-identical under any placement of the blocks, and equal to the oracle
     g = torch.Generator().manual_seed(31)
     ctx = torch.randint(200, 2500, (48,), generator=g).tolist()
     Hkv, Hq, d = 8, 32, 128
@@ -175,6 +174,36 @@ def test_in_kernel_merge_bit_identical_under_permutations(cuda_dev):
         outs.append(got.cpu())
     for o in outs[1:]:
         assert torch.equal(o, outs[0])
+
+
+def test_back_to_back_calls_share_one_workspace(cuda_dev):
+    # Calls on one pool and stream reuse one workspace: its split-K partial rows
+    # and the merge kernel's list of split pairs.  A call's kernels start while
+    # the previous call's merge kernel may still run, so four calls with
+    # different split lists are issued without a synchronisation between them;
+    # each must still match the oracle on its own sequences.
+    full = make_batch([100 + (i * 389) % 3900 for i in range(96)], None, block_size=16,
+                      n_q_heads=32, n_kv_heads=8, head_dim=128, dtype=torch.bfloat16, seed=34)
+    pool = gpu_pool_from(full, 8, 128, torch.bfloat16, cuda_dev)
+    subsets = [list(range(96)), list(range(0, 96, 3)), [5, 17, 60], list(range(40, 90))]
+    outs, subs = [], []
+    for idx in subsets:
+        sub = dict(full)
+        sub["q"] = full["q"][idx]
+        sub["block_tables"] = full["block_tables"][idx]
+        sub["context_lens"] = full["context_lens"][idx]
+        sub["query_start_lens"] = torch.arange(len(idx) + 1, dtype=torch.int32)
+        subs.append(sub)
+    dev_in = [(s_["q"].to(cuda_dev), s_["block_tables"].to(cuda_dev), s_["context_lens"].to(cuda_dev),
+               s_["query_start_lens"].to(cuda_dev)) for s_ in subs]
+    torch.cuda.synchronize(cuda_dev)
+    for _ in range(2):
+        outs = [api.paged_attention(q, pool.k_pool, pool.v_pool, bt, ctx, qsl, full["scale"])
+                for q, bt, ctx, qsl in dev_in]
+    torch.cuda.synchronize(cuda_dev)
+    for o, s_, idx in zip(outs, subs, subsets):
+        assert_close(o, oracle_attention(s_), torch.bfloat16, f"{len(idx)} sequences, back to back")
+    assert pool.check_device_errors() == 0
 
 
 def test_long_context_split_k(cuda_dev):

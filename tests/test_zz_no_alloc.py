@@ -158,8 +158,9 @@ def test_noalloc_clears_stale_counters(cuda_dev):
     assert prm.value == 0 and nbytes >= 512
     rt.cudaGraphDestroy(graph)
     # non-zero counters, then a normal call: on the tile-streaming decode kernel
-    # (16 q heads per kv head) and on the block-streaming one, whose split heads
-    # are merged through the same counters (48 sequences, 4 q heads per kv head)
+    # (16 q heads per kv head), whose split heads are merged through those
+    # counters, and on the block-streaming one with its merge kernel (48
+    # sequences, 4 q heads per kv head), which must not depend on them
     b2 = make_batch([200 + (i * 97) % 2300 for i in range(48)], None, block_size=16, n_q_heads=32,
                     n_kv_heads=8, head_dim=128, dtype=torch.bfloat16, seed=57)
     pool2 = gpu_pool_from(b2, 8, 128, torch.bfloat16, cuda_dev)
