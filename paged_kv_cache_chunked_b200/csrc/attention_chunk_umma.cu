@@ -13,8 +13,9 @@
 // of its kv head, each key read through the sequence's block table.
 //
 // Structure.  A work item is 256 query rows (pairs (token, head of the
-// group), token-major) of one (sequence, kv head), as two 128-row tiles; CTA i
-// takes items i, i + gridDim.x, ...  Per 128-key stage:
+// group), token-major) of one (sequence, kv head), as two 128-row tiles; the
+// CTAs take the items sequence by sequence, heaviest sequence first, in the
+// snake order of umma_common.cuh.  Per 128-key stage:
 //   - producer warps load the stage's eight 16-key blocks by TMA: K as one
 //     2-D box per block and 64-column panel (warp 9 panel 0, warp 10 panel 1
 //     at head dim 128) into the canonical K-major 128-byte-swizzled layout
@@ -87,7 +88,7 @@ struct UGeo {
     static constexpr uint32_t OffK = OffQ + kUTiles * QBytes;
     static constexpr uint32_t OffV = OffK + kUKStages * KBytes;
     static constexpr uint32_t OffPlan = OffV + kUVStages * VBytes;
-    static constexpr uint32_t OffBar = OffPlan + (3 * kPlanLen * 4 + 15) / 16 * 16;
+    static constexpr uint32_t OffBar = OffPlan + ((3 * kPlanLen + kOrderInts) * 4 + 15) / 16 * 16;
     // barriers: k_full[K slot], k_empty[K slot], v_full[V slot], v_empty[V slot],
     // v_tma; per row tile: s_full, p_full, q_full, o_full, o_free; mma_done
     static constexpr uint32_t PerTileBars = 5;
@@ -133,9 +134,10 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = prm.group, Hq = prm.n_q_heads, Hkv = prm.n_kv_heads, bs = prm.block_size;
     const int nseq = prm.nseq;
-    int *item_pre = (int *)(sm + G::OffPlan);
-    int *s_qsl = item_pre + kPlanLen;
+    int *grp_pre = (int *)(sm + G::OffPlan);  // groups (256-row blocks) of sequences 0..i-1
+    int *s_qsl = grp_pre + kPlanLen;
     int *s_ctx = s_qsl + kPlanLen;
+    const ChunkOrder order(s_ctx + kPlanLen);
     uint64_t *k_full = (uint64_t *)(sm + G::OffBar);
     uint64_t *k_empty = k_full + kUKStages;
     uint64_t *v_full = k_empty + kUKStages;
@@ -149,7 +151,7 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
     };
     uint32_t *tmem_slot = (uint32_t *)(sm + G::OffMisc);
     volatile int *abort_flag = (volatile int *)(sm + G::OffMisc + 4);
-    __shared__ int s_nitems;
+    __shared__ int s_ngroups, s_nchunk;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kUKStages; ++s) {
@@ -180,9 +182,9 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (warp == kUProd0) {
-        // items: every sequence whose rows need more than one 16-row tile
-        // contributes ceil(rows / 256) items per kv head
-        int run = 0;
+        // groups: every sequence whose rows need more than one 16-row tile
+        // contributes ceil(rows / 256) groups, each of Hkv items (one per kv head)
+        int run = 0, nchunk = 0;
         for (int base = 0; base < nseq; base += 32) {
             const int i = base + lane;
             int n = 0;
@@ -195,7 +197,7 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                 const int qn = s1 - s0;
                 const bool ok = s0 >= 0 && s1 <= prm.num_tokens && qn >= 1 && c >= qn &&
                                 (long long)(c + bs - 1) / bs <= prm.max_blocks;
-                if (ok && qn * g > prm.min_rows) n = (qn * g + kUItemRows - 1) / kUItemRows * Hkv;
+                if (ok && qn * g > prm.min_rows) n = (qn * g + kUItemRows - 1) / kUItemRows;
             }
             int inc = n;
 #pragma unroll
@@ -203,35 +205,46 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                 const int y = __shfl_up_sync(0xffffffffu, inc, o);
                 if (lane >= o) inc += y;
             }
-            if (i < nseq) item_pre[i + 1] = run + inc;
+            if (i < nseq) grp_pre[i + 1] = run + inc;
             run += __shfl_sync(0xffffffffu, inc, 31);
+            // the chunk sequences, in window order, for the ranking
+            const unsigned has = __ballot_sync(0xffffffffu, n > 0);
+            const int pos = nchunk + __popc(has & ((1u << lane) - 1));
+            if (n > 0 && pos < kRankCap) order.cseq[pos] = i;
+            nchunk += __popc(has);
         }
         if (lane == 0) {
-            item_pre[0] = 0;
-            s_nitems = run;
+            grp_pre[0] = 0;
+            s_ngroups = run;
+            s_nchunk = nchunk;
         }
     }
+    __syncthreads();
+    const int n_groups = s_ngroups;
+    const int n_items = n_groups * Hkv;
+    if (s_nchunk <= kRankCap)
+        rank_chunk_seqs<kUItemRows, kUKeys>(order, s_nchunk, grp_pre, s_qsl, s_ctx, g, Hkv, threadIdx.x, kUThreads);
     tc_before();
     __syncthreads();
     tc_after();
     const uint32_t tmem = *tmem_slot;
-    const int n_items = s_nitems;
     if (warp < kUMma) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kURegSoftmax));
     else asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kURegOther));
 
+    // the item at position idx of the ranked list (the chunk-sequence count is
+    // read back from shared memory: kept in a register across the item loops it
+    // would cost the softmax warps a register)
     auto item_of = [&](int idx, UItem &it) {
-        const int b = find_seq(item_pre, nseq, idx);
-        const int local = idx - item_pre[b];
-        it.b = b;
-        it.qs0 = s_qsl[b];
-        it.qn = s_qsl[b + 1] - it.qs0;
-        it.c = s_ctx[b];
-        it.rows = it.qn * g;
-        const int nit = (it.rows + kUItemRows - 1) / kUItemRows;
+        int local;
+        ranked_item(order, s_nchunk, grp_pre, nseq, Hkv, idx, it.b, local);
+        const int nit = grp_pre[it.b + 1] - grp_pre[it.b];
         it.kvh = local / nit;
         it.rt = local - it.kvh * nit;
-        const int last_row = min((it.rt + 1) * kUItemRows, it.rows) - 1;
-        it.nkt = (it.c - it.qn + last_row / g) / kUKeys + 1;
+        it.qs0 = s_qsl[it.b];
+        it.qn = s_qsl[it.b + 1] - it.qs0;
+        it.c = s_ctx[it.b];
+        it.rows = it.qn * g;
+        it.nkt = block_stages<kUItemRows, kUKeys>(it.c, it.qn, g, it.rt);
     };
 
     if (warp >= kUProd0) {
@@ -248,7 +261,8 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
         if (lane == 0) prefetch_tmap(is_v ? &tmv3 : &tmk2);
         int n = 0, ntail = 0;
         bool ok = true;
-        for (int idx = blockIdx.x; active && ok && idx < n_items; idx += gridDim.x) {
+        for (int idx = blockIdx.x; active && ok && idx < n_items;
+             idx = snake_next(idx, blockIdx.x, gridDim.x)) {
             UItem it;
             item_of(idx, it);
             const int32_t *table = prm.tables + (long long)(prm.seq0 + it.b) * prm.max_blocks;
@@ -344,7 +358,8 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
         uint8_t *qbuf = sm + G::OffQ + t * G::QBytes;
         int n = 0, n_item = 0;
         bool ok = true;
-        for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++n_item) {
+        for (int idx = blockIdx.x; ok && idx < n_items;
+             idx = snake_next(idx, blockIdx.x, gridDim.x), ++n_item) {
             UItem it;
             item_of(idx, it);
             const int R = it.rt * kUItemRows + t * kURows + r;
@@ -518,7 +533,8 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
                             klo + (uint32_t)((kk >> 2) * G::KPanel + (kk & 3) * 32) / 16, kIdescS, kk > 0 ? 1u : 0u);
                 umma_commit(tb(t).s_full);
             };
-            for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++n_item) {
+            for (int idx = blockIdx.x; ok && idx < n_items;
+                 idx = snake_next(idx, blockIdx.x, gridDim.x), ++n_item) {
                 UItem it;
                 item_of(idx, it);
                 for (int t = 0; t < kUTiles && ok; ++t) ok = mbar_wait(tb(t).q_full, (uint32_t)n_item & 1);

@@ -18,8 +18,9 @@
 // 32 columns), O at columns 256..511.
 //
 // Structure.  A work item is 128 query rows (pairs (token, head of the group),
-// token-major) of one (sequence, kv head); CTA i takes items i, i + gridDim.x,
-// ...  Per 64-key stage:
+// token-major) of one (sequence, kv head); the CTAs take the items sequence by
+// sequence, heaviest sequence first, in the snake order of umma_common.cuh.
+// Per 64-key stage:
 //   - warp 5 loads K by TMA, one 2-D box per 16-key block and 64-column panel
 //     (16 boxes, one per lane) into [panel][64 keys][128 B]; warp 6 loads V, one
 //     3-D box per block into [block][panel][16 keys][128 B].  K and V have
@@ -70,7 +71,7 @@ constexpr uint32_t kWOffQ = 0;
 constexpr uint32_t kWOffK = kWOffQ + kWQBytes;
 constexpr uint32_t kWOffV = kWOffK + 2 * kWKBytes;
 constexpr uint32_t kWOffPlan = kWOffV + 2 * kWVBytes;
-constexpr uint32_t kWOffBar = kWOffPlan + (3 * kPlanLen * 4 + 15) / 16 * 16;
+constexpr uint32_t kWOffBar = kWOffPlan + ((3 * kPlanLen + kOrderInts) * 4 + 15) / 16 * 16;
 // barriers: k_full[2], k_empty[2], v_full[2], v_empty[2], v_tma, s_full[2],
 // p_full[2], pv_done, q_full, o_full, o_free, mma_done
 constexpr uint32_t kWNumBars = 2 + 2 + 2 + 2 + 1 + 2 + 2 + 1 + 1 + 1 + 1 + 1;
@@ -107,9 +108,10 @@ attention_chunk_umma256_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = prm.group, Hq = prm.n_q_heads, Hkv = prm.n_kv_heads, bs = prm.block_size;
     const int nseq = prm.nseq;
-    int *item_pre = (int *)(sm + kWOffPlan);
-    int *s_qsl = item_pre + kPlanLen;
+    int *grp_pre = (int *)(sm + kWOffPlan);  // groups (128-row blocks) of sequences 0..i-1
+    int *s_qsl = grp_pre + kPlanLen;
     int *s_ctx = s_qsl + kPlanLen;
+    const ChunkOrder order(s_ctx + kPlanLen);
     uint64_t *k_full = (uint64_t *)(sm + kWOffBar);
     uint64_t *k_empty = k_full + 2;
     uint64_t *v_full = k_empty + 2;
@@ -124,7 +126,7 @@ attention_chunk_umma256_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 
     uint64_t *mma_done = o_free + 1;
     uint32_t *tmem_slot = (uint32_t *)(sm + kWOffMisc);
     volatile int *abort_flag = (volatile int *)(sm + kWOffMisc + 4);
-    __shared__ int s_nitems;
+    __shared__ int s_ngroups, s_nchunk;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
@@ -151,8 +153,9 @@ attention_chunk_umma256_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (warp == kWProdK) {
-        // items: every served sequence contributes ceil(rows / 128) items per kv head
-        int run = 0;
+        // groups: every served sequence contributes ceil(rows / 128) groups, each
+        // of Hkv items (one per kv head)
+        int run = 0, nchunk = 0;
         for (int base = 0; base < nseq; base += 32) {
             const int i = base + lane;
             int n = 0;
@@ -165,7 +168,7 @@ attention_chunk_umma256_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 
                 const int qn = s1 - s0;
                 const bool ok = s0 >= 0 && s1 <= prm.num_tokens && qn >= 1 && c >= qn &&
                                 (long long)(c + bs - 1) / bs <= prm.max_blocks;
-                if (ok && qn * g > prm.min_rows) n = (qn * g + kWRows - 1) / kWRows * Hkv;
+                if (ok && qn * g > prm.min_rows) n = (qn * g + kWRows - 1) / kWRows;
             }
             int inc = n;
 #pragma unroll
@@ -173,33 +176,44 @@ attention_chunk_umma256_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 
                 const int y = __shfl_up_sync(0xffffffffu, inc, o);
                 if (lane >= o) inc += y;
             }
-            if (i < nseq) item_pre[i + 1] = run + inc;
+            if (i < nseq) grp_pre[i + 1] = run + inc;
             run += __shfl_sync(0xffffffffu, inc, 31);
+            // the chunk sequences, in window order, for the ranking
+            const unsigned has = __ballot_sync(0xffffffffu, n > 0);
+            const int pos = nchunk + __popc(has & ((1u << lane) - 1));
+            if (n > 0 && pos < kRankCap) order.cseq[pos] = i;
+            nchunk += __popc(has);
         }
         if (lane == 0) {
-            item_pre[0] = 0;
-            s_nitems = run;
+            grp_pre[0] = 0;
+            s_ngroups = run;
+            s_nchunk = nchunk;
         }
     }
+    __syncthreads();
+    const int n_groups = s_ngroups;
+    const int n_items = n_groups * Hkv;
+    if (s_nchunk <= kRankCap)
+        rank_chunk_seqs<kWRows, kWKeys>(order, s_nchunk, grp_pre, s_qsl, s_ctx, g, Hkv, threadIdx.x, kWThreads);
     tc_before();
     __syncthreads();
     tc_after();
     const uint32_t tmem = *tmem_slot;
-    const int n_items = s_nitems;
 
+    // the item at position idx of the ranked list (the chunk-sequence count is
+    // read back from shared memory: kept in a register across the item loops it
+    // would cost the softmax warps a register)
     auto item_of = [&](int idx, WItem &it) {
-        const int b = find_seq(item_pre, nseq, idx);
-        const int local = idx - item_pre[b];
-        it.b = b;
-        it.qs0 = s_qsl[b];
-        it.qn = s_qsl[b + 1] - it.qs0;
-        it.c = s_ctx[b];
-        it.rows = it.qn * g;
-        const int nit = (it.rows + kWRows - 1) / kWRows;
+        int local;
+        ranked_item(order, s_nchunk, grp_pre, nseq, Hkv, idx, it.b, local);
+        const int nit = grp_pre[it.b + 1] - grp_pre[it.b];
         it.kvh = local / nit;
         it.rt = local - it.kvh * nit;
-        const int last_row = min((it.rt + 1) * kWRows, it.rows) - 1;
-        it.nkt = (it.c - it.qn + last_row / g) / kWKeys + 1;
+        it.qs0 = s_qsl[it.b];
+        it.qn = s_qsl[it.b + 1] - it.qs0;
+        it.c = s_ctx[it.b];
+        it.rows = it.qn * g;
+        it.nkt = block_stages<kWRows, kWKeys>(it.c, it.qn, g, it.rt);
     };
 
     if (warp == kWProdK || warp == kWProdV) {
@@ -210,7 +224,8 @@ attention_chunk_umma256_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 
         if (lane == 0) prefetch_tmap(is_v ? &tmv3 : &tmk2);
         int n = 0, ntail = 0;
         bool ok = true;
-        for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+        for (int idx = blockIdx.x; ok && idx < n_items;
+             idx = snake_next(idx, blockIdx.x, gridDim.x)) {
             WItem it;
             item_of(idx, it);
             const int32_t *table = prm.tables + (long long)(prm.seq0 + it.b) * prm.max_blocks;
@@ -301,7 +316,8 @@ attention_chunk_umma256_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 
         uint8_t *qbuf = sm + kWOffQ;
         int n = 0, n_item = 0;
         bool ok = true;
-        for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++n_item) {
+        for (int idx = blockIdx.x; ok && idx < n_items;
+             idx = snake_next(idx, blockIdx.x, gridDim.x), ++n_item) {
             WItem it;
             item_of(idx, it);
             const int R = it.rt * kWRows + r;
@@ -469,7 +485,8 @@ attention_chunk_umma256_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 
                 umma_commit(&k_empty[s]);  // the K slot is free once this S has completed
                 return true;
             };
-            for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x, ++n_item) {
+            for (int idx = blockIdx.x; ok && idx < n_items;
+                 idx = snake_next(idx, blockIdx.x, gridDim.x), ++n_item) {
                 WItem it;
                 item_of(idx, it);
                 if (!mbar_wait(q_full, (uint32_t)n_item & 1)) {

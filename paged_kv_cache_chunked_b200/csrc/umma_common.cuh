@@ -109,5 +109,113 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
+// ---- order of the work items --------------------------------------------
+// A window's chunk work is grouped by sequence; a sequence's items (kv head x
+// row block) are taken in their natural order, so that the row blocks of one
+// (sequence, kv head), which read the same keys, run side by side and share
+// them in L2.  Sequences differ a lot (a chunk at context 4,096 has four times
+// the work of one at 1,024), so taking items round robin in sequence order
+// leaves the CTAs with the longest sequence's items far behind.  Every CTA
+// instead ranks the window's chunk sequences by work, heaviest first (ties by
+// index: the same order in every CTA), and CTA i takes the positions of the
+// ranked item list in snake order, i, 2P - 1 - i, 2P + i, ... (P CTAs):
+// greedy balancing of the longest-first kind, without a shared counter.
+// Windows of more than kRankCap chunk sequences, where round robin already
+// spreads the work, keep the natural order.
+constexpr int kRankCap = 256;
+constexpr int kOrderInts = 5 * kRankCap + 1;  // shared-memory ints of a ChunkOrder
+
+struct ChunkOrder {
+    int *cseq;       // [kRankCap] chunk sequences (window index), in window order
+    int *key;        // [kRankCap] their key stages summed over row blocks
+    int *ord;        // [kRankCap] rank -> position in cseq
+    int *rank_seq;   // [kRankCap] rank -> window index
+    int *rank_pre;   // [kRankCap + 1] items of the ranks before
+    __device__ explicit ChunkOrder(int *base)
+        : cseq(base), key(base + kRankCap), ord(base + 2 * kRankCap), rank_seq(base + 3 * kRankCap),
+          rank_pre(base + 4 * kRankCap) {}
+};
+
+// Key stages of row block rt of a chunk of qn tokens at context c: those of its
+// last query row (token-major rows of g heads, ROWS rows a block, KEYS keys a
+// stage).
+template <int ROWS, int KEYS>
+__device__ __forceinline__ int block_stages(int c, int qn, int g, int rt) {
+    const int last_row = min((rt + 1) * ROWS, qn * g) - 1;
+    return (c - qn + last_row / g) / KEYS + 1;
+}
+
+// Ranks the m chunk sequences listed in order.cseq (m <= kRankCap) and fills
+// order.rank_seq / rank_pre.  grp_pre[i] = row blocks of window sequences
+// before i.  Called by every thread of the CTA (it holds barriers).
+template <int ROWS, int KEYS>
+__device__ void rank_chunk_seqs(const ChunkOrder &o, int m, const int *grp_pre, const int *s_qsl,
+                                const int *s_ctx, int g, int Hkv, int tid, int nthreads) {
+    for (int j = tid; j < m; j += nthreads) {
+        const int b = o.cseq[j];
+        const int qn = s_qsl[b + 1] - s_qsl[b], nb = grp_pre[b + 1] - grp_pre[b];
+        int w = 0;
+        for (int rt = 0; rt < nb; ++rt) w += block_stages<ROWS, KEYS>(s_ctx[b], qn, g, rt);
+        o.key[j] = w;
+    }
+    __syncthreads();
+    for (int i = tid; i < m; i += nthreads) {
+        const int ki = o.key[i];
+        int r = 0;
+        for (int j = 0; j < m; ++j) {
+            const int kj = o.key[j];
+            r += (kj > ki) | ((kj == ki) & (j < i));
+        }
+        o.ord[r] = i;
+    }
+    __syncthreads();
+    if (tid < 32) {
+        int run = 0;
+        for (int base = 0; base < m; base += 32) {
+            const int r = base + tid;
+            int n = 0;
+            if (r < m) {
+                const int b = o.cseq[o.ord[r]];
+                o.rank_seq[r] = b;
+                n = (grp_pre[b + 1] - grp_pre[b]) * Hkv;
+            }
+            int inc = n;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, inc, d);
+                if (tid >= d) inc += y;
+            }
+            if (r < m) o.rank_pre[r + 1] = run + inc;
+            run += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (tid == 0) o.rank_pre[0] = 0;
+    }
+}
+
+// The item at position idx of the ranked list (or of the natural list when the
+// window has more than kRankCap chunk sequences): window sequence b and its
+// local item (kv head x row blocks + row block).
+__device__ __forceinline__ void ranked_item(const ChunkOrder &o, int m, const int *grp_pre, int nseq,
+                                            int Hkv, int idx, int &b, int &local) {
+    if (m <= kRankCap) {
+        const int r = find_seq(o.rank_pre, m, idx);
+        b = o.rank_seq[r];
+        local = idx - o.rank_pre[r];
+    } else {
+        b = find_seq(grp_pre, nseq, idx / Hkv);
+        local = idx - grp_pre[b] * Hkv;
+    }
+}
+
+// position of CTA cta's item of round r in the ranked list (in
+// [r * ncta, (r + 1) * ncta), so strictly increasing in r)
+__device__ __forceinline__ int snake_pos(int r, int cta, int ncta) {
+    return r * ncta + ((r & 1) ? ncta - 1 - cta : cta);
+}
+// the position after pos = snake_pos(r, cta, ncta)
+__device__ __forceinline__ int snake_next(int pos, int cta, int ncta) {
+    return snake_pos(pos / ncta + 1, cta, ncta);
+}
+
 }  // namespace
 }  // namespace pk
