@@ -37,11 +37,22 @@ from paged_kv_cache_chunked_b200.workloads import WORKLOADS, workload_batch  # n
 METRIC = "paged decode attention KV GB/s (% of HBM peak) and tokens/s per scheduler step"
 FALLBACK_HBM_GBS = 6650.0
 CSRC = os.path.join(ROOT, "paged_kv_cache_chunked_b200", "csrc")
-# the source of each workload's dominant kernel (the traffic record is valid for that source only)
-KERNEL_SRC = {"chunk512_bf16": os.path.join(CSRC, "attention_chunk_umma.cu"),
-              "chunk512_d256_bf16": os.path.join(CSRC, "attention_chunk_umma256.cu"),
-              "append_copy": os.path.join(CSRC, "kv_copy.cu")}
-DECODE_SRC = os.path.join(CSRC, "attention_decode_blocks.cu")
+# the sources of each workload's dominant kernel, its local headers included
+# (the traffic record is valid for those sources only)
+_TC = ["tc_common.cuh", "pk_internal.h"]
+KERNEL_SRC = {"chunk512_bf16": ["attention_chunk_umma.cu", "umma_common.cuh"] + _TC,
+              "chunk512_d256_bf16": ["attention_chunk_umma256.cu", "umma_common.cuh"] + _TC,
+              "append_copy": ["kv_copy.cu", "pk_internal.h"]}
+DECODE_SRC = ["attention_decode_blocks.cu"] + _TC
+
+
+def kernel_source_hash(workload):
+    """sha256 (first 16 hex digits) of the dominant kernel's sources, in order."""
+    h = hashlib.sha256()
+    for name in KERNEL_SRC.get(workload, DECODE_SRC):
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def parse():
@@ -187,10 +198,8 @@ def kernel_traffic(workload):
             rec = json.load(f)
     except (OSError, ValueError):
         return None
-    with open(KERNEL_SRC.get(workload, DECODE_SRC), "rb") as f:
-        src_hash = hashlib.sha256(f.read()).hexdigest()[:16]
     entry = rec.get(workload)
-    if not entry or entry.get("kernel_sha256_16") != src_hash:
+    if not entry or entry.get("kernel_sha256_16") != kernel_source_hash(workload):
         return None
     return entry.get("dram_bytes_per_call")
 
