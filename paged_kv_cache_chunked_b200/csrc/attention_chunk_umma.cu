@@ -228,6 +228,13 @@ attention_chunk_umma_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 2-D
     __syncthreads();
     tc_after();
     const uint32_t tmem = *tmem_slot;
+    // Launched as a programmatic dependent of the kernel before it on the stream
+    // (in a mixed batch, the decode rows' merge kernel): the plan above reads
+    // only the query offsets and lengths, which no kernel of the call writes;
+    // the pool, the queries, the tables and the output are touched only after
+    // this wait, which also covers every kernel before that one
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (warp < kUMma) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kURegSoftmax));
     else asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kURegOther));
 
@@ -654,10 +661,13 @@ int launch_chunk_umma(const pk_pool *p, const AttnArgs &a, bool all_multi, cudaS
     for (int s0 = 0; s0 < a.num_seqs; s0 += kMaxSeqsPerLaunch) {
         u.seq0 = s0;
         u.nseq = std::min(kMaxSeqsPerLaunch, a.num_seqs - s0);
-        if (p->head_dim == 64)
-            attention_chunk_umma_kernel<64><<<p->sm_count, kUThreads, UGeo<64>::Smem, st>>>(p->tmap_k2, p->tmap_v, u);
-        else
-            attention_chunk_umma_kernel<128><<<p->sm_count, kUThreads, UGeo<128>::Smem, st>>>(p->tmap_k2, p->tmap_v, u);
+        const cudaError_t e =
+            p->head_dim == 64
+                ? launch_dependent(attention_chunk_umma_kernel<64>, dim3(p->sm_count), kUThreads, UGeo<64>::Smem, st,
+                                   p->tmap_k2, p->tmap_v, u)
+                : launch_dependent(attention_chunk_umma_kernel<128>, dim3(p->sm_count), kUThreads, UGeo<128>::Smem,
+                                   st, p->tmap_k2, p->tmap_v, u);
+        if (e != cudaSuccess) return cuda_fail(e, "chunk attention (tcgen05) launch");
     }
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? PK_OK : cuda_fail(e, "chunk attention (tcgen05) launch");

@@ -199,6 +199,13 @@ attention_chunk_umma256_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 
     __syncthreads();
     tc_after();
     const uint32_t tmem = *tmem_slot;
+    // Launched as a programmatic dependent of the kernel before it on the stream
+    // (in a mixed batch, the decode rows' merge kernel): the plan above reads
+    // only the query offsets and lengths, which no kernel of the call writes;
+    // the pool, the queries, the tables and the output are touched only after
+    // this wait, which also covers every kernel before that one
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // the item at position idx of the ranked list (the chunk-sequence count is
     // read back from shared memory: kept in a register across the item loops it
@@ -566,7 +573,9 @@ int launch_chunk_umma256(const pk_pool *p, const AttnArgs &a, bool all_multi, cu
     for (int s0 = 0; s0 < a.num_seqs; s0 += kMaxSeqsPerLaunch) {
         u.seq0 = s0;
         u.nseq = std::min(kMaxSeqsPerLaunch, a.num_seqs - s0);
-        attention_chunk_umma256_kernel<<<p->sm_count, kWThreads, kWSmem, st>>>(p->tmap_k2, p->tmap_v, u);
+        const cudaError_t e = launch_dependent(attention_chunk_umma256_kernel, dim3(p->sm_count), kWThreads, kWSmem, st,
+                                               p->tmap_k2, p->tmap_v, u);
+        if (e != cudaSuccess) return cuda_fail(e, "chunk attention (tcgen05, head dim 256) launch");
     }
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? PK_OK : cuda_fail(e, "chunk attention (tcgen05, head dim 256) launch");

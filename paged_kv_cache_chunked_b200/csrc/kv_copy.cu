@@ -18,9 +18,9 @@ namespace pk {
 namespace {
 
 // Each kernel here is launched as a programmatic dependent of the previous
-// kernel on the stream (launch_pdl).  It lets its own dependent (the next copy,
-// or the attention kernel, whose plan reads no pool rows) start launching at
-// once, then waits for the previous grid to finish, and its writes to be
+// kernel on the stream (launch_dependent).  It lets its own dependent (the next
+// copy, or the attention kernel, whose plan reads no pool rows) start launching
+// at once, then waits for the previous grid to finish, and its writes to be
 // visible, before it touches any memory: stream order as seen by memory is
 // unchanged, but the launch no longer waits for the previous grid's last CTA.
 __device__ __forceinline__ void pdl_prologue() {
@@ -28,19 +28,6 @@ __device__ __forceinline__ void pdl_prologue() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int threads, cudaStream_t st, Args... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(threads);
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, ((KArgs)args)...);
-}
 
 // One thread per 16-byte chunk of one (token, head) row of K or V.
 // Grid-stride over num_tokens * n_kv_heads * row_chunks * 2.
@@ -200,18 +187,18 @@ int launch_kv_append(const pk_pool *p, const void *k, const void *v, const int64
     if (row_bytes % 16 == 0 && aligned16(k) && aligned16(v)) {
         const int row_chunks = (int)(row_bytes / 16);
         const int64_t work = 2LL * num_tokens * p->n_kv_heads * row_chunks;
-        e = launch_pdl(kv_append_vec16, grid_for(work, 256, p->sm_count), 256, st, (const uint4 *)k,
+        e = launch_dependent(kv_append_vec16, dim3(grid_for(work, 256, p->sm_count)), 256, 0, st, (const uint4 *)k,
                        (const uint4 *)v, (uint4 *)p->k_base, (uint4 *)p->v_base, slots, num_tokens,
                        p->n_kv_heads, p->block_size, row_chunks, num_slots, p->d_err);
     } else {
         const int64_t work = 2LL * num_tokens * p->n_kv_heads * p->head_dim;
         const int grid = grid_for(work, 256, p->sm_count);
         if (p->dtype == PK_BF16)
-            e = launch_pdl(kv_append_scalar<uint16_t>, grid, 256, st, (const uint16_t *)k,
+            e = launch_dependent(kv_append_scalar<uint16_t>, dim3(grid), 256, 0, st, (const uint16_t *)k,
                            (const uint16_t *)v, (uint16_t *)p->k_base, (uint16_t *)p->v_base, slots,
                            num_tokens, p->n_kv_heads, p->block_size, p->head_dim, num_slots, p->d_err);
         else
-            e = launch_pdl(kv_append_scalar<float>, grid, 256, st, (const float *)k, (const float *)v,
+            e = launch_dependent(kv_append_scalar<float>, dim3(grid), 256, 0, st, (const float *)k, (const float *)v,
                            (float *)p->k_base, (float *)p->v_base, slots, num_tokens, p->n_kv_heads,
                            p->block_size, p->head_dim, num_slots, p->d_err);
     }
@@ -232,15 +219,15 @@ int launch_swap_blocks(const pk_pool *p, void *host_k, void *host_v, int num_hos
     const int grid = (int)(ctas < (int64_t)p->sm_count * 32 ? ctas : (int64_t)p->sm_count * 32);
     cudaError_t e;
     if (block_bytes % 16 == 0 && aligned16(sk) && aligned16(sv) && aligned16(dk) && aligned16(dv))
-        e = launch_pdl(swap_copy<uint4, 4>, grid, 256, st, (const uint4 *)sk, (const uint4 *)sv,
+        e = launch_dependent(swap_copy<uint4, 4>, dim3(grid), 256, 0, st, (const uint4 *)sk, (const uint4 *)sv,
                        (uint4 *)dk, (uint4 *)dv, pairs, n_pairs, block_bytes / 16, n_src, n_dst,
                        p->d_err);
     else if (p->dtype == PK_BF16)
-        e = launch_pdl(swap_copy<uint16_t, 4>, grid, 256, st, (const uint16_t *)sk,
+        e = launch_dependent(swap_copy<uint16_t, 4>, dim3(grid), 256, 0, st, (const uint16_t *)sk,
                        (const uint16_t *)sv, (uint16_t *)dk, (uint16_t *)dv, pairs, n_pairs,
                        block_elems, n_src, n_dst, p->d_err);
     else
-        e = launch_pdl(swap_copy<float, 4>, grid, 256, st, (const float *)sk, (const float *)sv,
+        e = launch_dependent(swap_copy<float, 4>, dim3(grid), 256, 0, st, (const float *)sk, (const float *)sv,
                        (float *)dk, (float *)dv, pairs, n_pairs, block_elems, n_src, n_dst, p->d_err);
     return e == cudaSuccess ? PK_OK : cuda_fail(e, "block swap launch");
 }
@@ -254,13 +241,13 @@ int launch_block_copy(const pk_pool *p, const int32_t *pairs, int n_pairs, cudaS
     const int grid = (int)(ctas < (int64_t)p->sm_count * 32 ? ctas : (int64_t)p->sm_count * 32);
     cudaError_t e;
     if (block_bytes % 16 == 0)
-        e = launch_pdl(block_copy_vec16, grid, 256, st, (uint4 *)p->k_base, (uint4 *)p->v_base, pairs,
+        e = launch_dependent(block_copy_vec16, dim3(grid), 256, 0, st, (uint4 *)p->k_base, (uint4 *)p->v_base, pairs,
                        n_pairs, block_bytes / 16, p->num_blocks, p->d_err);
     else if (p->dtype == PK_BF16)
-        e = launch_pdl(block_copy_scalar<uint16_t>, grid, 256, st, (uint16_t *)p->k_base,
+        e = launch_dependent(block_copy_scalar<uint16_t>, dim3(grid), 256, 0, st, (uint16_t *)p->k_base,
                        (uint16_t *)p->v_base, pairs, n_pairs, block_elems, p->num_blocks, p->d_err);
     else
-        e = launch_pdl(block_copy_scalar<float>, grid, 256, st, (float *)p->k_base,
+        e = launch_dependent(block_copy_scalar<float>, dim3(grid), 256, 0, st, (float *)p->k_base,
                        (float *)p->v_base, pairs, n_pairs, block_elems, p->num_blocks, p->d_err);
     return e == cudaSuccess ? PK_OK : cuda_fail(e, "block copy launch");
 }

@@ -54,6 +54,26 @@ constexpr int kMaxSeqsPerLaunch = 512;  // window of sequences per kernel launch
 // fixed size, so that every pool finds its counters at the same offsets.
 constexpr int kMaxTcKvHeads = 64;
 
+// Launches kernel as a programmatic dependent of the previous kernel on the
+// stream: it may start while that kernel drains, so it must execute
+// griddepcontrol.wait before it reads what earlier work on the stream wrote
+// (or writes what that work reads).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, int threads, size_t smem, cudaStream_t st,
+                             Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, ((KArgs)args)...);
+}
+
 // ---- launchers (each returns PK_OK or an error code) ---------------------
 int launch_kv_append(const pk_pool *p, const void *k, const void *v, const int64_t *slots,
                      int num_tokens, cudaStream_t st);
