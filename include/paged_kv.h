@@ -32,6 +32,17 @@
  *     pk_check_device_errors reads.  Results of such a call are undefined.
  *   - Bounded waits: a pipeline wait that exceeds its iteration limit records
  *     PK_ERR_TIMEOUT in the same word and the kernel returns.
+ *   - Stream order holds as for plain launches.  The kernels are launched as
+ *     programmatic dependents of the kernel before them on `stream`, so a
+ *     call's kernels may start while that kernel drains.  They wait for it
+ *     (griddepcontrol.wait) before they touch the pool, the output or any
+ *     scratch. Before that wait the attention kernels read only their plan
+ *     inputs: q, the block tables, the context lengths and the query offsets.
+ *     One obligation on the caller follows. A kernel of its own that
+ *     immediately precedes an attention call on `stream` and signals its
+ *     dependents early (griddepcontrol.launch_dependents) must not write
+ *     those four arrays after the signal. Kernels that never signal, copies
+ *     and events are unaffected.
  *   - Threading: calls on different pools may run concurrently; calls on
  *     one pk_bm must be serialised by the caller.
  */
