@@ -29,35 +29,56 @@ __device__ __forceinline__ void pdl_prologue() {
 }
 
 
-// One thread per 16-byte chunk of one (token, head) row of K or V.
-// Grid-stride over num_tokens * n_kv_heads * row_chunks * 2.
+// One warp per token: the token's slot is read and split into (block, offset)
+// once, then the lanes move the token's K and V rows of all kv heads
+// (n_kv_heads * row_chunks 16-byte chunks each), four chunks of K and four of V
+// a lane, all loads issued before the first store.  Consecutive lanes touch
+// consecutive chunks of one (block, head) row, so every warp access is a
+// contiguous 512-byte run.  Grid-stride over the tokens.
+constexpr int kAppendUnroll = 4;
 __global__ void kv_append_vec16(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
                                 uint4 *__restrict__ kp, uint4 *__restrict__ vp,
                                 const int64_t *__restrict__ slots, int num_tokens, int n_kv_heads,
                                 int block_size, int row_chunks, int64_t num_slots,
                                 int *err) {
     pdl_prologue();
-    const int64_t per_side = (int64_t)num_tokens * n_kv_heads * row_chunks;
-    const int64_t total = 2 * per_side;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const bool is_v = i >= per_side;
-        const int64_t j = is_v ? i - per_side : i;
-        const int c = (int)(j % row_chunks);
-        const int64_t th = j / row_chunks;  // token * n_kv_heads + head
-        const int h = (int)(th % n_kv_heads);
-        const int64_t t = th / n_kv_heads;
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    const int per_side = n_kv_heads * row_chunks;  // chunks of one token's K (or V)
+    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < num_tokens; t += warps) {
         const int64_t slot = __ldg(slots + t);
         if (slot < 0) continue;
         if (slot >= num_slots) {
-            record_error(err, PK_ERR_BAD_INDEX);
+            if (lane == 0) record_error(err, PK_ERR_BAD_INDEX);
             continue;
         }
         const int64_t blk = slot / block_size;
-        const int off = (int)(slot % block_size);
-        const int64_t dst = ((blk * n_kv_heads + h) * block_size + off) * row_chunks + c;
-        const uint4 val = __ldcs((is_v ? v : k) + j);
-        __stcs((is_v ? vp : kp) + dst, val);
+        const int off = (int)(slot - blk * block_size);
+        // chunk c = h * row_chunks + e of the token goes to ((blk * Hkv + h) * bs + off) * row_chunks + e
+        const int64_t base = (blk * n_kv_heads * block_size + off) * row_chunks;
+        const int64_t head_stride = (int64_t)block_size * row_chunks;
+        const uint4 *ks = k + (int64_t)t * per_side, *vs = v + (int64_t)t * per_side;
+        for (int c0 = 0; c0 < per_side; c0 += 32 * kAppendUnroll) {
+            uint4 a[kAppendUnroll], b[kAppendUnroll];
+#pragma unroll
+            for (int u = 0; u < kAppendUnroll; ++u) {
+                const int c = c0 + u * 32 + lane;
+                if (c < per_side) {
+                    a[u] = __ldcs(ks + c);
+                    b[u] = __ldcs(vs + c);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kAppendUnroll; ++u) {
+                const int c = c0 + u * 32 + lane;
+                if (c < per_side) {
+                    const int h = c / row_chunks;
+                    const int64_t dst = base + h * head_stride + (c - h * row_chunks);
+                    __stcs(kp + dst, a[u]);
+                    __stcs(vp + dst, b[u]);
+                }
+            }
+        }
     }
 }
 
@@ -186,8 +207,8 @@ int launch_kv_append(const pk_pool *p, const void *k, const void *v, const int64
     cudaError_t e;
     if (row_bytes % 16 == 0 && aligned16(k) && aligned16(v)) {
         const int row_chunks = (int)(row_bytes / 16);
-        const int64_t work = 2LL * num_tokens * p->n_kv_heads * row_chunks;
-        e = launch_dependent(kv_append_vec16, dim3(grid_for(work, 256, p->sm_count)), 256, 0, st, (const uint4 *)k,
+        // one warp per token, eight warps a CTA
+        e = launch_dependent(kv_append_vec16, dim3(grid_for(32LL * num_tokens, 256, p->sm_count)), 256, 0, st, (const uint4 *)k,
                        (const uint4 *)v, (uint4 *)p->k_base, (uint4 *)p->v_base, slots, num_tokens,
                        p->n_kv_heads, p->block_size, row_chunks, num_slots, p->d_err);
     } else {
