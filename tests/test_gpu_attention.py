@@ -206,6 +206,17 @@ def test_back_to_back_calls_share_one_workspace(cuda_dev):
     assert pool.check_device_errors() == 0
 
 
+@pytest.mark.parametrize("Hq,Hkv,d", [(32, 8, 128), (16, 4, 256)])
+def test_chunk_order_past_the_rank_cap(cuda_dev, Hq, Hkv, d):
+    # 300 sequences of 3-token chunks: more chunk sequences than the tcgen05
+    # kernels rank by work (256), so their items are taken in window order;
+    # every row against the oracle
+    ctx = [20 + (i * 37) % 400 for i in range(300)]
+    b = make_batch(ctx, [3] * len(ctx), block_size=16, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d,
+                   dtype=torch.bfloat16, seed=35)
+    _check(b, Hq, Hkv, d, torch.bfloat16, cuda_dev, f"300 chunk sequences, d {d}")
+
+
 def test_long_context_split_k(cuda_dev):
     # two 8k-token sequences with head dim 256: many split-K partitions
     b = make_batch([8192, 6000], None, block_size=16, n_q_heads=16, n_kv_heads=4, head_dim=256,
