@@ -535,7 +535,15 @@ def run_ours(args, rank, world, device):
     out = torch.empty_like(dq)
     stream = torch.cuda.current_stream(device)
 
+    # a step: the new tokens' K/V stored and attention over them, in one call
+    # (pk_paged_attention_append; where the block-streaming kernel serves the
+    # batch, the attention kernel stores them itself)
     def step():
+        api.paged_attention_append(dq, dk, dv, pool.k_pool, pool.v_pool, dt_, dctx, dqsl, batch["scale"],
+                                   out=out)
+
+    # the same step as two calls: the append kernel, then attention
+    def step_two_calls():
         api.paged_kv_append(dk, dv, dslots, pool=pool)
         api.paged_attention(dq, pool.k_pool, pool.v_pool, dt_, dctx, dqsl, batch["scale"], out=out)
 
@@ -559,7 +567,10 @@ def run_ours(args, rank, world, device):
         per_window = 3                  # block-streaming decode, merge kernel, tcgen05 chunk kernel
     else:
         per_window = 2 if T > B or Hq // Hkv > 16 else 1
-    launches_per_step = 1 + (windows * per_window if tc else 1)
+    # the new K/V are stored by the block-streaming kernel where it serves the
+    # batch, else by the position append kernel
+    stored_in_kernel = blocks and (T == B or umma)
+    launches_per_step = (0 if stored_in_kernel else 1) + (windows * per_window if tc else 1)
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize(device)
@@ -584,13 +595,14 @@ def run_ours(args, rank, world, device):
     if dist:
         tdist.barrier()
     total_ms = start.elapsed_time(end)
-    # the attention call alone, for its roofline: a separate pass, so that no
-    # event sits between the append and the attention of a timed step (the
-    # attention kernels start as programmatic dependents of the append)
+    # the attention call alone, for its roofline: a separate pass after the
+    # timed steps (a step's kernels start as programmatic dependents of the
+    # previous ones, and no event sits between them)
     n_attn = max(args.steps, 50)
     attn_avg_ms = attention_run_ms(attention_only, stream, n_attn)
     attn_iso_each = attention_call_ms(attention_only, stream, n_attn)
     attn_iso_ms = statistics.mean(attn_iso_each)
+    two_call_ms = attention_run_ms(step_two_calls, stream, n_attn)
     # a long enough window for the clock sampler to see the load
     t_extra = time.perf_counter()
     while not args.profile_run and time.perf_counter() - t_extra < 1.0:
@@ -614,7 +626,7 @@ def run_ours(args, rank, world, device):
     # the compute stream are reported beside it.
     e2e = None
     if not args.no_e2e and not args.profile_run:
-        h_in = [x.pin_memory() for x in (batch["q"], k_new, v_new, slots, batch["block_tables"],
+        h_in = [x.pin_memory() for x in (batch["q"], k_new, v_new, batch["block_tables"],
                                          batch["context_lens"], batch["query_start_lens"])]
         h_outs = [torch.empty_like(batch["q"]).pin_memory() for _ in range(2)]
         sets = [[torch.empty_like(x, device=device) for x in h_in] for _ in range(2)]
@@ -626,9 +638,8 @@ def run_ours(args, rank, world, device):
         used = [False, False]
 
         def kernels(bufs, o):
-            api.paged_kv_append(bufs[1], bufs[2], bufs[3], pool=pool)
-            api.paged_attention(bufs[0], pool.k_pool, pool.v_pool, bufs[4], bufs[5], bufs[6],
-                                batch["scale"], out=o)
+            api.paged_attention_append(bufs[0], bufs[1], bufs[2], pool.k_pool, pool.v_pool, bufs[3], bufs[4],
+                                       bufs[5], batch["scale"], out=o)
 
         def e2e_step(i):
             j = i % 2
@@ -685,8 +696,8 @@ def run_ours(args, rank, world, device):
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "serialized_ms_per_step": s_ms,
                "serialized_value": world * (attn_b + app_b) / (s_ms * 1e-3) / 1e9,
-               "how": "per step: host-to-device copies of q, the new K/V, slots, tables, lengths from "
-                      "pinned memory; append + attention; device-to-host copy of the output; copies "
+               "how": "per step: host-to-device copies of q, the new K/V, tables, lengths from "
+                      "pinned memory; pk_paged_attention_append; device-to-host copy of the output; copies "
                       "overlapped with the neighbouring steps' kernels on two copy streams "
                       "(double-buffered device inputs and outputs); serialized_*: the same with every "
                       "copy on the compute stream"}
@@ -718,6 +729,12 @@ def run_ours(args, rank, world, device):
                             f"pass after the timed steps (roofline avg_ms); the same calls each "
                             f"between their own events: isolated_call_ms",
     }
+    line["step_call"] = ("pk_paged_attention_append: the new K/V stored "
+                         + ("by the block-streaming decode kernel" if stored_in_kernel
+                            else "by the position append kernel") + ", then attention")
+    line["two_call_ms_per_step"] = two_call_ms
+    line["two_call_value"] = world * (attn_b + app_b) / (two_call_ms * 1e-3) / 1e9
+    line["two_call"] = "pk_paged_kv_append with slots, then pk_paged_attention, back to back"
     line["roofline"]["isolated_call_ms"] = attn_iso_ms
     line["roofline"]["isolated_call_median_ms"] = statistics.median(attn_iso_each)
     if e2e:

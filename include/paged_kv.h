@@ -210,6 +210,34 @@ int pk_paged_attention(const pk_pool *pool, const void *q, void *out,
                        void *workspace, size_t workspace_bytes, pk_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Append, then attend, in one call ([SN] "Flow": the step's new K/V go into
+ * the blocks their table maps them to; [BP] "PagedAttention" item 4).
+ *
+ * The same as pk_paged_kv_append of the query rows' own K/V, followed by
+ * pk_paged_attention with the same arguments. Query row t = query_start_lens[b]
+ * + i of sequence b holds the K/V rows k[t], v[t] ([num_tokens][n_kv_heads]
+ * [head_dim], the pool's dtype, contiguous, 16-byte aligned). They are stored
+ * at position c_b - q_b + i, in block block_tables[b][pos / bs] at offset
+ * pos % bs, before any attention reads them.
+ *
+ * The slots follow from the tables, so no slot_mapping is taken.
+ *   - Block-streaming path (bf16 decode rows, groups of at most 8): the decode
+ *     kernel stores each decode row's K/V just before it loads the block
+ *     holding it, and a mixed step's chunk rows before its chunk kernel
+ *     starts. No append kernel runs.
+ *   - Other geometries: an append kernel runs first, then attention.
+ * Results, and the pool afterwards, equal those of the two separate calls.
+ * A table entry outside the pool is recorded (PK_ERR_BAD_INDEX) and its row
+ * is not stored. Errors: as pk_paged_attention, and PK_ERR_INVALID_ARG for
+ * k or v NULL or misaligned.
+ * ------------------------------------------------------------------------ */
+int pk_paged_attention_append(const pk_pool *pool, const void *q, const void *k, const void *v,
+                              void *out, const int32_t *block_tables, int max_blocks_per_seq,
+                              const int32_t *context_lens, const int32_t *query_start_lens,
+                              int num_seqs, int num_tokens, int n_q_heads, float scale,
+                              void *workspace, size_t workspace_bytes, pk_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Paged attention without a caller workspace.  The pages have no
  * counterpart to this call; it exists for callers that cannot allocate
  * device memory, such as a C host program with no caching allocator, or a

@@ -60,6 +60,7 @@ SIGNATURES = {
     "pk_swap_blocks": ([_P, _P, _P, _I, _P, _I, _I, _P], _I),
     "pk_attention_workspace_size": ([_P, _I, _I, _I, _I, _PSZ], _I),
     "pk_paged_attention": ([_P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _F, _P, _SZ, _P], _I),
+    "pk_paged_attention_append": ([_P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _F, _P, _SZ, _P], _I),
     "pk_paged_attention_noalloc": ([_P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _F, _P], _I),
     "pk_bm_create": ([_I, _I, _PP], _I),
     "pk_bm_destroy": ([_P], _I),

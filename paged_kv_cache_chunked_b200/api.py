@@ -224,6 +224,39 @@ def paged_attention(q, k_pool, v_pool, block_tables, context_lens, query_start_l
     return out
 
 
+def paged_attention_append(q, k, v, k_pool, v_pool, block_tables, context_lens, query_start_lens, scale,
+                           out=None):
+    """Store the query rows' own K/V (k, v: [T, Hkv, d]) at their positions
+    (position c_b - q_b + i of sequence b, slot from its block table), then
+    attend: the same as paged_kv_append with the slots the tables give,
+    followed by paged_attention, in one call."""
+    pool = _pool_of(k_pool, v_pool)
+    d = pool.device
+    _need(q, "q", pool.dtype, d)
+    _need(k, "k", pool.dtype, d)
+    _need(v, "v", pool.dtype, d)
+    _need(block_tables, "block_tables", torch.int32, d)
+    _need(context_lens, "context_lens", torch.int32, d)
+    _need(query_start_lens, "query_start_lens", torch.int32, d)
+    T, Hq, hd = q.shape
+    B = context_lens.shape[0]
+    if hd != pool.head_dim or block_tables.dim() != 2 or block_tables.shape[0] != B or \
+            query_start_lens.shape != (B + 1,) or tuple(k.shape) != (T, pool.n_kv_heads, hd) or \
+            k.shape != v.shape:
+        raise ValueError("inconsistent shapes")
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _need(out, "out", pool.dtype, d)
+    W = block_tables.shape[1]
+    ws = pool.workspace(B, T, Hq, W)
+    check(lib().pk_paged_attention_append(pool.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                          _ptr(block_tables), W, _ptr(context_lens),
+                                          _ptr(query_start_lens), B, T, Hq, float(scale), _ptr(ws),
+                                          ws.numel(), _stream(d)))
+    return out
+
+
 class BlockManager:
     """Host block manager (free list, tables, reference counts, fork, copy-on-write)."""
 

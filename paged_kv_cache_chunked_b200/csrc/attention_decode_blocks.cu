@@ -96,6 +96,11 @@ struct BlkParams {
     int ncta, cap_rows;
     float scale_log2;
     int *mplan;                      // the merge kernel's list of split pairs
+    // the query rows' own K/V ([num_tokens, n_kv_heads, D]) to store at their
+    // positions before they are read, and the pool they go to; k_new == nullptr:
+    // nothing to store
+    const __nv_bfloat16 *k_new, *v_new;
+    __nv_bfloat16 *kpool, *vpool;
     float *partial_o, *partial_lse;  // [row][D], [row]
     int *err;
     // shared-memory layout (byte offsets from the 1024-aligned base)
@@ -265,6 +270,22 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
             const int e = blk_base + lane;
             return e < nblk ? __ldg(prm.tables + (long long)(prm.seq0 + b) * prm.max_blocks + e) : 0;
         };
+        // the token of sequence b's (one) query row
+        auto d_tok = [&](int b) -> int { return s_qsl[b]; };
+        // query token tok's K and V rows of kv heads h0 .. h0 + nh - 1 into block
+        // phys at offset off (16-byte vectors over the warp's lanes)
+        auto store_row = [&](int tok, int phys, int off, int h0, int nh) {
+            constexpr int RC = D / 8;  // 16-byte chunks of a row
+            const uint4 *ks = (const uint4 *)prm.k_new, *vs = (const uint4 *)prm.v_new;
+            uint4 *kd = (uint4 *)prm.kpool, *vd = (uint4 *)prm.vpool;
+            for (int i = lane; i < nh * RC; i += 32) {
+                const int h = h0 + i / RC, e = i % RC;
+                const long long src = ((long long)tok * Hkv + h) * RC + e;
+                const long long dst = (((long long)phys * Hkv + h) * bs + off) * RC + e;
+                kd[dst] = __ldg(ks + src);
+                vd[dst] = __ldg(vs + src);
+            }
+        };
         // Items (partitions) in chunk order.  The next item is found, and its
         // first two table chunks requested, while the current one's stages
         // are issued, so the table lookups of an item start without a wait.
@@ -332,20 +353,26 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
             // block table lookups: this lane holds entry cur_base + lane; the
             // following 32 entries are in flight
             int cur_base = (cur.st0 * NBS) & ~31, cur_tab = cur.tab0, nxt_tab = cur.tab1;
+            // the table entry of block blk (non-decreasing over the item); a bad id
+            // is recorded and comes back as -1
             auto table_get = [&](int blk) -> int {
                 while (blk >= cur_base + 32) {
                     cur_base += 32;
                     cur_tab = nxt_tab;
                     nxt_tab = chunk_entry(b, cur_base + 32);
                 }
-                int phys = __shfl_sync(0xffffffffu, cur_tab, blk - cur_base);
+                const int phys = __shfl_sync(0xffffffffu, cur_tab, blk - cur_base);
                 if (phys < 0 || phys >= prm.num_blocks) {
                     if (lane == 0) record_error(prm.err, PK_ERR_BAD_INDEX);
-                    phys = 0;
+                    return -1;
                 }
                 return phys;
             };
             const int nblk = (c + bs - 1) / bs;
+            // with an append, the row's own K/V go to position c - 1 (block
+            // new_blk, offset new_off) before that block is loaded
+            const int new_blk = prm.k_new != nullptr ? (c - 1) / bs : -1;
+            const int new_off = (c - 1) - new_blk * bs;
             if (!waited) {  // the preceding kernel's pool rows are visible from here on
                 asm volatile("griddepcontrol.wait;" ::: "memory");
                 waited = true;
@@ -368,7 +395,14 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                 uint8_t *kst = sm + (size_t)s * prm.stage_bytes;
                 uint8_t *vst = kst + (size_t)NBS * piece_bytes;
                 for (int j = 0; j < np; ++j) {
-                    const int phys = table_get(blk0 + j);
+                    const int raw = table_get(blk0 + j);
+                    const int phys = raw < 0 ? 0 : raw;
+                    if (blk0 + j == new_blk) {
+                        if (raw >= 0) store_row(d_tok(b), raw, new_off, hg * HS, HS);
+                        // the generic-proxy stores before the TMA box that reads them
+                        asm volatile("fence.proxy.async.global;" ::: "memory");
+                        __syncwarp();
+                    }
                     const int y = (phys * Hkv + hg * HS) * bs;
                     if (lane == 0) {  // all panels of the block's rows: one box for K, one for V
                         tma_load_3d_hint(kst + j * piece_bytes, &tmk, 0, y, 0, &full[s], stream_pol);
@@ -391,6 +425,28 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                     mbar_arrive(&full[s]);
                 }
                 ++n_stage;
+            }
+        }
+        if (ok && prm.k_new != nullptr && prm.skip_chunks) {
+            // the chunk rows' K/V (sequences of several query tokens), for the chunk
+            // kernel that follows: token t of the window by CTA t % grid, all kv heads
+            if (!waited) {
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+                waited = true;
+            }
+            for (int t = s_qsl[0] + (int)blockIdx.x; t < s_qsl[nseq]; t += (int)gridDim.x) {
+                const int b = find_seq(s_qsl, nseq, t);
+                const int qb = s_qsl[b + 1] - s_qsl[b];
+                if (qb < 2) continue;  // a decode row: stored before its block was loaded
+                const int pos = s_ctx[b] - qb + (t - s_qsl[b]);
+                const int jb = pos / bs;
+                if (pos < 0 || jb >= prm.max_blocks) continue;  // recorded by the plan
+                const int phys = __ldg(prm.tables + (long long)(prm.seq0 + b) * prm.max_blocks + jb);
+                if (phys < 0 || phys >= prm.num_blocks) {
+                    if (lane == 0) record_error(prm.err, PK_ERR_BAD_INDEX);
+                    continue;
+                }
+                store_row(t, phys, pos - jb * bs, 0, Hkv);
             }
         }
         if (blockIdx.x == 0) {
@@ -803,6 +859,10 @@ int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, bool s
     tp.cap_rows = w.cap_rows;
     tp.scale_log2 = a.scale * 1.4426950408889634f;
     tp.mplan = w.merge_plan;
+    tp.k_new = (const __nv_bfloat16 *)a.k_new;
+    tp.v_new = (const __nv_bfloat16 *)a.v_new;
+    tp.kpool = (__nv_bfloat16 *)p->k_base;
+    tp.vpool = (__nv_bfloat16 *)p->v_base;
     tp.partial_o = w.partial_o;
     tp.partial_lse = w.partial_lse;
     tp.err = p->d_err;

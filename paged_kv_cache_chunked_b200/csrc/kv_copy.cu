@@ -82,6 +82,51 @@ __global__ void kv_append_vec16(const uint4 *__restrict__ k, const uint4 *__rest
     }
 }
 
+// The query rows' K/V of an attention call stored at their positions: token t
+// of sequence b (t = qsl[b] + i) sits at position ctx[b] - (qsl[b + 1] - qsl[b])
+// + i, in block tables[b][pos / bs] at offset pos % bs.  One warp per token;
+// the sequence is found by a binary search over the query offsets.  A row is
+// row_elems elements of T (16-byte vectors when the row allows, else scalars).
+template <typename T>
+__global__ void kv_append_at_positions(const T *__restrict__ k, const T *__restrict__ v, T *kp, T *vp,
+                                       const int32_t *__restrict__ tables, int max_blocks,
+                                       const int32_t *__restrict__ ctx, const int32_t *__restrict__ qsl,
+                                       int num_seqs, int num_tokens, int n_kv_heads, int block_size,
+                                       int row_elems, int num_blocks, int *err) {
+    pdl_prologue();
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    const int per_side = n_kv_heads * row_elems;
+    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < num_tokens; t += warps) {
+        int lo = 0, hi = num_seqs - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(qsl + mid + 1) > t) hi = mid;
+            else lo = mid + 1;
+        }
+        const int b = lo;
+        const int s0 = __ldg(qsl + b), s1 = __ldg(qsl + b + 1), c = __ldg(ctx + b);
+        const int pos = c - (s1 - s0) + (t - s0);
+        if (t < s0 || t >= s1 || pos < 0 || pos >= max_blocks * block_size) {
+            if (lane == 0) record_error(err, PK_ERR_BAD_INDEX);
+            continue;
+        }
+        const int blk = __ldg(tables + (int64_t)b * max_blocks + pos / block_size);
+        if (blk < 0 || blk >= num_blocks) {
+            if (lane == 0) record_error(err, PK_ERR_BAD_INDEX);
+            continue;
+        }
+        const int off = pos % block_size;
+        const T *ks = k + (int64_t)t * per_side, *vs = v + (int64_t)t * per_side;
+        for (int c2 = lane; c2 < per_side; c2 += 32) {
+            const int h = c2 / row_elems;
+            const int64_t dst = (((int64_t)blk * n_kv_heads + h) * block_size + off) * row_elems + (c2 - h * row_elems);
+            kp[dst] = ks[c2];
+            vp[dst] = vs[c2];
+        }
+    }
+}
+
 // Element-wise fallback for rows that are not a multiple of 16 bytes.
 template <typename T>
 __global__ void kv_append_scalar(const T *__restrict__ k, const T *__restrict__ v, T *kp, T *vp,
@@ -224,6 +269,30 @@ int launch_kv_append(const pk_pool *p, const void *k, const void *v, const int64
                            p->block_size, p->head_dim, num_slots, p->d_err);
     }
     return e == cudaSuccess ? PK_OK : cuda_fail(e, "kv append launch");
+}
+
+int launch_kv_append_at_positions(const pk_pool *p, const AttnArgs &a, cudaStream_t st) {
+    if (a.num_tokens == 0 || a.num_seqs == 0) return PK_OK;
+    const int elt = p->dtype == PK_BF16 ? 2 : 4;
+    const int64_t row_bytes = (int64_t)p->head_dim * elt;
+    const int grid = grid_for(32LL * a.num_tokens, 256, p->sm_count);  // one warp per token
+    cudaError_t e;
+    if (row_bytes % 16 == 0 && aligned16(a.k_new) && aligned16(a.v_new))
+        e = launch_dependent(kv_append_at_positions<uint4>, dim3(grid), 256, 0, st, (const uint4 *)a.k_new,
+                             (const uint4 *)a.v_new, (uint4 *)p->k_base, (uint4 *)p->v_base, a.block_tables,
+                             a.max_blocks_per_seq, a.context_lens, a.query_start_lens, a.num_seqs, a.num_tokens,
+                             p->n_kv_heads, p->block_size, (int)(row_bytes / 16), p->num_blocks, p->d_err);
+    else if (p->dtype == PK_BF16)
+        e = launch_dependent(kv_append_at_positions<uint16_t>, dim3(grid), 256, 0, st, (const uint16_t *)a.k_new,
+                             (const uint16_t *)a.v_new, (uint16_t *)p->k_base, (uint16_t *)p->v_base,
+                             a.block_tables, a.max_blocks_per_seq, a.context_lens, a.query_start_lens, a.num_seqs,
+                             a.num_tokens, p->n_kv_heads, p->block_size, p->head_dim, p->num_blocks, p->d_err);
+    else
+        e = launch_dependent(kv_append_at_positions<float>, dim3(grid), 256, 0, st, (const float *)a.k_new,
+                             (const float *)a.v_new, (float *)p->k_base, (float *)p->v_base, a.block_tables,
+                             a.max_blocks_per_seq, a.context_lens, a.query_start_lens, a.num_seqs, a.num_tokens,
+                             p->n_kv_heads, p->block_size, p->head_dim, p->num_blocks, p->d_err);
+    return e == cudaSuccess ? PK_OK : cuda_fail(e, "kv append at positions launch");
 }
 
 int launch_swap_blocks(const pk_pool *p, void *host_k, void *host_v, int num_host_blocks,

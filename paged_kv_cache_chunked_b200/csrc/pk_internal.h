@@ -94,7 +94,14 @@ struct AttnArgs {
     float scale;
     void *workspace;
     size_t workspace_bytes;
+    // the query rows' own K/V rows ([num_tokens, n_kv_heads, head_dim], pool dtype),
+    // stored at their positions before they are read; nullptr: no append
+    const void *k_new = nullptr, *v_new = nullptr;
 };
+
+// The query rows' K/V of an attention call (a.k_new, a.v_new) stored at their
+// positions (slot from the block table), one warp per token.
+int launch_kv_append_at_positions(const pk_pool *p, const AttnArgs &a, cudaStream_t st);
 
 int launch_attention_generic(const pk_pool *p, const AttnArgs &a, cudaStream_t st);
 
