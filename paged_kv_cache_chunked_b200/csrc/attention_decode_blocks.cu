@@ -377,6 +377,24 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                 asm volatile("griddepcontrol.wait;" ::: "memory");
                 waited = true;
             }
+            // when this item reaches the new row's block, that row's K/V (heads of
+            // this group, contiguous in k_new) are loaded now and stored there
+            constexpr int RCd = D / 8, UP = 4;
+            const int nrow = HS * RCd;
+            const bool pre = new_blk >= 0 && new_blk / NBS >= cur.st0 && new_blk / NBS < cur.st0 + cur.cnt &&
+                             nrow <= 32 * UP;
+            uint4 pk[UP], pv[UP];
+            if (pre) {
+                const long long src0 = ((long long)d_tok(b) * Hkv + hg * HS) * RCd;
+#pragma unroll
+                for (int u = 0; u < UP; ++u) {
+                    const int i = u * 32 + lane;
+                    if (i < nrow) {
+                        pk[u] = __ldg((const uint4 *)prm.k_new + src0 + i);
+                        pv[u] = __ldg((const uint4 *)prm.v_new + src0 + i);
+                    }
+                }
+            }
             for (int st = cur.st0; st < cur.st0 + cur.cnt; ++st) {
                 const int s = n_stage % NS;
                 if (n_stage >= NS && !mbar_wait(&empty[s], ((n_stage / NS) - 1) & 1)) {
@@ -398,7 +416,21 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                     const int raw = table_get(blk0 + j);
                     const int phys = raw < 0 ? 0 : raw;
                     if (blk0 + j == new_blk) {
-                        if (raw >= 0) store_row(d_tok(b), raw, new_off, hg * HS, HS);
+                        if (raw >= 0 && pre) {
+                            uint4 *kd = (uint4 *)prm.kpool, *vd = (uint4 *)prm.vpool;
+#pragma unroll
+                            for (int u = 0; u < UP; ++u) {
+                                const int i = u * 32 + lane;
+                                if (i < nrow) {
+                                    const long long dst =
+                                        (((long long)raw * Hkv + hg * HS + i / RCd) * bs + new_off) * RCd + i % RCd;
+                                    kd[dst] = pk[u];
+                                    vd[dst] = pv[u];
+                                }
+                            }
+                        } else if (raw >= 0) {
+                            store_row(d_tok(b), raw, new_off, hg * HS, HS);
+                        }
                         // the generic-proxy stores before the TMA box that reads them
                         asm volatile("fence.proxy.async.global;" ::: "memory");
                         __syncwarp();
@@ -425,28 +457,6 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
                     mbar_arrive(&full[s]);
                 }
                 ++n_stage;
-            }
-        }
-        if (ok && prm.k_new != nullptr && prm.skip_chunks) {
-            // the chunk rows' K/V (sequences of several query tokens), for the chunk
-            // kernel that follows: token t of the window by CTA t % grid, all kv heads
-            if (!waited) {
-                asm volatile("griddepcontrol.wait;" ::: "memory");
-                waited = true;
-            }
-            for (int t = s_qsl[0] + (int)blockIdx.x; t < s_qsl[nseq]; t += (int)gridDim.x) {
-                const int b = find_seq(s_qsl, nseq, t);
-                const int qb = s_qsl[b + 1] - s_qsl[b];
-                if (qb < 2) continue;  // a decode row: stored before its block was loaded
-                const int pos = s_ctx[b] - qb + (t - s_qsl[b]);
-                const int jb = pos / bs;
-                if (pos < 0 || jb >= prm.max_blocks) continue;  // recorded by the plan
-                const int phys = __ldg(prm.tables + (long long)(prm.seq0 + b) * prm.max_blocks + jb);
-                if (phys < 0 || phys >= prm.num_blocks) {
-                    if (lane == 0) record_error(prm.err, PK_ERR_BAD_INDEX);
-                    continue;
-                }
-                store_row(t, phys, pos - jb * bs, 0, Hkv);
             }
         }
         if (blockIdx.x == 0) {
@@ -485,6 +495,50 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
         // ---------------------------------------------------------- consumers
         asm volatile("griddepcontrol.wait;" ::: "memory");  // before any write
         const int cw = warp - 1, hl = cw % HS, ph = cw / HS;
+        if (prm.k_new != nullptr && prm.skip_chunks) {
+            // the chunk rows' own K/V (sequences of several query tokens), for
+            // the chunk kernel that follows, stored while this CTA's first
+            // stages are in flight: one consumer warp per token, all kv heads,
+            // every load of a pass issued before its stores
+            constexpr int RC = D / 8, U = 4;  // 16-byte chunks of a head's row; chunks per lane and pass
+            const int n = Hkv * RC;
+            const uint4 *ks = (const uint4 *)prm.k_new, *vs = (const uint4 *)prm.v_new;
+            uint4 *kd = (uint4 *)prm.kpool, *vd = (uint4 *)prm.vpool;
+            for (int t = s_qsl[0] + (int)blockIdx.x * kNC + cw; t < s_qsl[nseq]; t += (int)gridDim.x * kNC) {
+                const int b = find_seq(s_qsl, nseq, t);
+                const int qb = s_qsl[b + 1] - s_qsl[b];
+                if (qb < 2) continue;  // a decode row: the producer stores it before its block is loaded
+                const int pos = s_ctx[b] - qb + (t - s_qsl[b]);
+                const int jb = pos / bs;
+                if (pos < 0 || jb >= prm.max_blocks) continue;  // recorded by the plan
+                const int phys = __ldg(prm.tables + (long long)(prm.seq0 + b) * prm.max_blocks + jb);
+                if (phys < 0 || phys >= prm.num_blocks) {
+                    if (lane == 0) record_error(prm.err, PK_ERR_BAD_INDEX);
+                    continue;
+                }
+                const long long row = ((long long)phys * Hkv * bs + (pos - jb * bs)) * RC;
+                for (int i0 = 0; i0 < n; i0 += 32 * U) {
+                    uint4 kr[U], vr[U];
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int i = i0 + u * 32 + lane;
+                        if (i < n) {
+                            kr[u] = __ldg(ks + (long long)t * n + i);
+                            vr[u] = __ldg(vs + (long long)t * n + i);
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int i = i0 + u * 32 + lane;
+                        if (i < n) {  // kv head i / RC: (block, head, offset) rows are bs * RC apart
+                            const long long dst = row + (long long)(i / RC) * bs * RC + i % RC;
+                            kd[dst] = kr[u];
+                            vd[dst] = vr[u];
+                        }
+                    }
+                }
+            }
+        }
         const int qr = lane >> 2, qc = (lane & 3) * 2;
         const int mi = lane >> 3, rr = lane & 7;
         const int a_row = (mi & 1) * 8 + rr, a_col = (mi >> 1) * 8;  // K rows (A of S^T)
