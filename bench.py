@@ -1,13 +1,15 @@
 #!/usr/bin/env python
 """Benchmark of one step of the paged-KV hot path on B200.
 
-A step is one decode iteration of the named workload: append each sequence's
-new token's K/V into its block (paged_kv_append), then paged attention of
-every sequence's query over its whole paged context (plan + attention +
-split-K reduce kernels).  The workload has no forks, so the copy-on-write
-block copy has no work in it.  Every step leaves the pool in the same state
-(the appended rows are the values already stored at those slots), so all
-steps are the same work.
+A step is one decode iteration of the named workload in one call
+(paged_attention_append): each sequence's new token's K/V stored at its
+position through the block table, then paged attention of every sequence's
+query over its whole paged context (the block-streaming kernel stores the new
+rows itself; its split-K merge kernel follows).  The same step as two calls
+(paged_kv_append with slots, then paged_attention) is timed beside it.  The
+workload has no forks, so the copy-on-write block copy has no work in it.
+Every step leaves the pool in the same state (the appended rows are the values
+already stored at those slots), so all steps are the same work.
 
 Prints one JSON line.  `value` is the step's algorithmic bytes (KV read once
 per sequence and kv head, Q and output, block tables, the append's reads and
@@ -1220,7 +1222,8 @@ def run_serving(args, rank, world, device):
             "pct_hbm": 100 * sum(kvb) / (tot_ms * 1e-3) / 1e9 / peak,
             "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
             else "fallback 6.65 TB/s",
-            "timing": "per-step CUDA events around swaps + copy + append + attention; host scheduling "
+            "timing": "per-step CUDA events around swaps + copy + append and attention (trace: one "
+                      "pk_paged_attention_append call; fork: append, then attention); host scheduling "
                       "excluded (see wall_clock)",
             "clocks": dict(clk, window="the whole run: timed steps and the measurement passes after them"),
             **extra}

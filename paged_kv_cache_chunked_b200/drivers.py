@@ -2,8 +2,8 @@
 
 TraceRunner   continuous batching over an arrival trace: each iteration the
               scheduler plans a mixed batch (decodes first, then prefill
-              chunks), the kernels run swaps -> copy -> append -> attention on
-              one stream, finished requests are freed ["PagedAttention &
+              chunks), the kernels run swaps -> copy -> append + attention
+              (one call) on one stream, finished requests are freed ["PagedAttention &
               Continuous Batching" (study notes), "Continuous batching" and
               "Flow"; "Batching and PagedAttention", "Continuous batching"].
               Preempted requests are recomputed, or with preempt="swap" their
@@ -136,7 +136,9 @@ class TraceRunner:
             "qsl": torch.tensor(plan.query_start_lens(), dtype=torch.int32),
             "pairs": torch.tensor(plan.copy_pairs, dtype=torch.int32).reshape(-1, 2),
         }
-        d = {k: v.to(dev, non_blocking=True) for k, v in meta.items()}
+        # the slots stay on the host (the step records them): the fused call
+        # stores each row at position c_b - q_b + i through the block tables
+        d = {k: v.to(dev, non_blocking=True) for k, v in meta.items() if k != "slots"}
         stream = torch.cuda.current_stream(dev)
         t_v = time.perf_counter()
         if timed:
@@ -154,9 +156,8 @@ class TraceRunner:
         self._run_swaps(swaps)
         if d["pairs"].shape[0]:
             api.block_copy(d["pairs"], pool=self.pool)
-        api.paged_kv_append(k, v, d["slots"], pool=self.pool)
-        out = api.paged_attention(q, self.pool.k_pool, self.pool.v_pool, d["tables"], d["ctx"],
-                                  d["qsl"], self.scale)
+        out = api.paged_attention_append(q, k, v, self.pool.k_pool, self.pool.v_pool, d["tables"], d["ctx"],
+                                         d["qsl"], self.scale)
         if timed:
             e1.record(stream)
         if on_step is not None:
