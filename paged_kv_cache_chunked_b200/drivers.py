@@ -24,6 +24,7 @@ Both generate queries and K/V with the counter-based generator of
 
 import time
 
+import numpy as np
 import torch
 
 from . import api
@@ -125,20 +126,18 @@ class TraceRunner:
                 rec.host_plan_ms = 1e3 * ((t_planned - t_start) + (t_end - t_c))
                 rec.host_total_ms = 1e3 * (t_end - t_start)
             return rec
-        rids, pos = [], []
-        for req, s, n in zip(plan.requests, plan.starts, plan.counts):
-            rids.extend(self.value_ids(req, s, n))
-            pos.extend(range(s, s + n))
+        rids, pos = self.value_keys(plan)
         meta = {
-            "slots": torch.tensor(plan.slots, dtype=torch.int64),
             "tables": plan.tables,
             "ctx": torch.tensor(plan.context_lens, dtype=torch.int32),
             "qsl": torch.tensor(plan.query_start_lens(), dtype=torch.int32),
             "pairs": torch.tensor(plan.copy_pairs, dtype=torch.int32).reshape(-1, 2),
         }
-        # the slots stay on the host (the step records them): the fused call
-        # stores each row at position c_b - q_b + i through the block tables
-        d = {k: v.to(dev, non_blocking=True) for k, v in meta.items() if k != "slots"}
+        # the fused call stores each row at position c_b - q_b + i through the
+        # block tables, so the slots are not sent; a step hook gets them
+        d = {k: v.to(dev, non_blocking=True) for k, v in meta.items()}
+        if on_step is not None:
+            meta["slots"] = torch.tensor(plan.slots, dtype=torch.int64)
         stream = torch.cuda.current_stream(dev)
         t_v = time.perf_counter()
         if timed:
@@ -195,6 +194,21 @@ class TraceRunner:
             return [req.rid] * n
         shared = SYS_VID_BASE + req.group
         return [shared if p < req.sys_len else req.rid for p in range(start, start + n)]
+
+    @staticmethod
+    def value_keys(plan):
+        """Generator keys of the step's rows, in batch order: (value id,
+        position) per row, value_ids of every request concatenated, built with
+        array operations (a chunked step has thousands of rows)."""
+        counts = np.asarray(plan.counts, dtype=np.int64)
+        first = np.repeat(np.cumsum(counts) - counts, counts)
+        pos = np.repeat(np.asarray(plan.starts, dtype=np.int64), counts) + (np.arange(int(counts.sum())) - first)
+        reqs = plan.requests
+        rid = np.repeat(np.asarray([r.rid for r in reqs], dtype=np.int64), counts)
+        grp = np.repeat(np.asarray([r.group for r in reqs], dtype=np.int64), counts)
+        sys_len = np.repeat(np.asarray([r.sys_len for r in reqs], dtype=np.int64), counts)
+        vid = np.where((grp >= 0) & (pos < sys_len), SYS_VID_BASE + grp, rid)
+        return torch.from_numpy(vid), torch.from_numpy(pos)
 
     def _run_swaps(self, swaps):
         # in the order the scheduler decided them: a swap-in may reuse blocks a

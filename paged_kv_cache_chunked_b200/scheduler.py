@@ -259,11 +259,11 @@ class Scheduler:
         while i < len(decodes) and budget > 0:
             todo = decodes[i:i + budget]
             done, got_slots, got_pairs = self.bm.append_one_each([r.seq for r in todo])
-            for req, slot in zip(todo[:done], got_slots):
-                batch.append(req)
-                starts.append(req.stored)
-                counts.append(1)
-                slots.append(slot)
+            served = todo[:done]
+            batch.extend(served)
+            starts.extend([r.stored for r in served])
+            counts.extend([1] * done)
+            slots.extend(got_slots)
             pairs.extend(got_pairs)
             budget -= done
             i += done

@@ -410,3 +410,31 @@ def test_random_traces_plan_identically_and_drain(reqs, nb, bs, budget, mode, pr
     assert len(s1.finished) == len(trace)
     st = s1.bm.stats()
     assert st["free_blocks"] == nb and st["num_seqs"] == 0 and st["cached_blocks"] == 0
+
+
+def test_step_value_keys_match_the_per_request_keys():
+    # The serving driver builds a step's generator keys with array operations.
+    # They must equal, row by row in batch order, the per-request keys: a
+    # request's own id past its shared system prompt, the prompt's id inside it.
+    from paged_kv_cache_chunked_b200.drivers import TraceRunner
+    from paged_kv_cache_chunked_b200.workloads import SYS_VID_BASE, prefix_trace_requests
+    trace = prefix_trace_requests()[:60]
+    sched = Scheduler(BlockManager(2048, 16), token_budget=1024, max_chunk=256, prefix_cache=True)
+    pending = [Request(i, *t[:3], group=t[3], sys_len=t[4]) for i, t in enumerate(trace)]
+    step = checked = shared = 0
+    while (pending or sched.has_work()) and step < 400:
+        while pending and pending[0].arrival <= step:
+            sched.add_request(pending.pop(0))
+        plan = sched.schedule()
+        if plan.requests:
+            vid, pos = TraceRunner.value_keys(plan)
+            want_v, want_p = [], []
+            for req, s, n in zip(plan.requests, plan.starts, plan.counts):
+                want_v += TraceRunner.value_ids(req, s, n)
+                want_p += list(range(s, s + n))
+            assert vid.tolist() == want_v and pos.tolist() == want_p
+            checked += 1
+            shared += int((vid >= SYS_VID_BASE).sum())
+        sched.complete(plan)
+        step += 1
+    assert checked > 20 and shared > 0
