@@ -1279,7 +1279,8 @@ def run_policy(args, rank, world, device):
                        "requests": len(trace), "num_blocks": 8192, "block_size": 16, "max_chunk": 512},
             "study": study,
             "clocks": dict(clk, window="every configuration of the study"),
-            "timing": "per-step CUDA events around copy + append + attention, summed; host scheduling excluded"}
+            "timing": "per-step CUDA events around the block copy and the append + attention call, summed; "
+                      "host scheduling excluded"}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
