@@ -80,6 +80,7 @@ class TraceRunner:
         self.records = []
         self.rejected = 0
         self.high_water = {}     # request id -> positions stored at least once
+        self._inflight = []      # (record, events) of steps whose GPU time is not read yet
 
     def _admit_arrivals(self, step):
         while self.pending and self.pending[0].arrival <= step:
@@ -89,18 +90,24 @@ class TraceRunner:
             except ValueError:
                 self.rejected += 1
 
-    def step(self, on_step=None, timed=True):
+    def step(self, on_step=None, timed=True, wait=True):
         """One iteration.  on_step(plan, tensors, out) is called after the
         kernels (for parity checks).  Returns the step's record, or None when
-        there was nothing to run."""
+        there was nothing to run.
+
+        wait=False (no on_step): the step returns once its kernels are
+        launched, and its GPU time is read at the next step or in finish().
+        The host then plans and launches step n + 1 while step n runs, as a
+        serving loop does; the scheduler's state never depends on a step's
+        results, only on its plan.  At most one step is left in flight."""
         t_start = time.perf_counter()
         step = self.sched.step_no
         self._admit_arrivals(step)
         plan = self.sched.schedule()
         t_planned = time.perf_counter()
         dev = self.device
-        swaps = [(to_host, torch.tensor(pairs, dtype=torch.int32).reshape(-1, 2).to(dev))
-                 for to_host, pairs in plan.swap_ops]
+        swaps = [(to_host, torch.tensor(pairs, dtype=torch.int32).reshape(-1, 2).pin_memory().to(
+                     dev, non_blocking=True)) for to_host, pairs in plan.swap_ops]
         if not plan.requests:
             # nothing to run but, possibly, swaps decided while planning (timed:
             # they are part of the serving work)
@@ -135,7 +142,9 @@ class TraceRunner:
         }
         # the fused call stores each row at position c_b - q_b + i through the
         # block tables, so the slots are not sent; a step hook gets them
-        d = {k: v.to(dev, non_blocking=True) for k, v in meta.items()}
+        # staged through pinned memory: a copy from pageable memory would first
+        # wait for the stream, and with it for the step still running
+        d = {k: v.pin_memory().to(dev, non_blocking=True) for k, v in meta.items()}
         if on_step is not None:
             meta["slots"] = torch.tensor(plan.slots, dtype=torch.int64)
         stream = torch.cuda.current_stream(dev)
@@ -161,8 +170,6 @@ class TraceRunner:
             e1.record(stream)
         if on_step is not None:
             on_step(plan, {"q": q, "k": k, "v": v, "swaps": plan.swap_ops, **meta}, out)
-        if timed:
-            e1.synchronize()
         n_dec = sum(1 for r, s in zip(plan.requests, plan.starts) if s >= r.target)
         # positions written for the first time (a recompute prefill rewrites
         # positions a preempted request had already stored)
@@ -173,11 +180,12 @@ class TraceRunner:
             self.high_water[req.rid] = max(hw, s + n)
         rec = StepRecord(step=step, tokens=plan.num_tokens, decode_rows=n_dec,
                          prefill_tokens=plan.num_tokens - n_dec, copies=len(plan.copy_pairs),
-                         gpu_ms=e0.elapsed_time(e1) if timed else None,
-                         context_tokens=sum(plan.context_lens), num_seqs=len(plan.requests),
+                         gpu_ms=None, context_tokens=sum(plan.context_lens), num_seqs=len(plan.requests),
                          swap_blocks=sum(len(p) for _, p in plan.swap_ops), new_tokens=new,
-                         host_values_ms=1e3 * t_v,
-                         values_gpu_ms=ev_v[0].elapsed_time(ev_v[1]) if timed else None)
+                         host_values_ms=1e3 * t_v, values_gpu_ms=None)
+        if timed:
+            self._inflight.append((rec, e0, e1, ev_v))
+            self._settle(0 if wait or on_step is not None else 1)
         t_c = time.perf_counter()
         self.sched.complete(plan)
         t_end = time.perf_counter()
@@ -224,10 +232,24 @@ class TraceRunner:
             ms[r.step] = r.gpu_ms or 0.0
         return ms
 
-    def run(self, max_steps=None, on_step=None):
+    def _settle(self, keep):
+        """Read the GPU times of all but the last `keep` steps in flight (each
+        waits for its step's kernels)."""
+        while len(self._inflight) > keep:
+            rec, e0, e1, ev_v = self._inflight.pop(0)
+            e1.synchronize()
+            rec.gpu_ms = e0.elapsed_time(e1)
+            rec.values_gpu_ms = ev_v[0].elapsed_time(ev_v[1])
+
+    def finish(self):
+        """Wait for the steps in flight and fill in their GPU times."""
+        self._settle(0)
+
+    def run(self, max_steps=None, on_step=None, wait=True):
         limit = max_steps if max_steps is not None else self.n_steps
         while self.sched.step_no < limit and (self.pending or self.sched.has_work()):
-            self.step(on_step)
+            self.step(on_step, wait=wait)
+        self.finish()
         return self.records
 
 

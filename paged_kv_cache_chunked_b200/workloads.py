@@ -219,6 +219,8 @@ def token_values(seed, stream, rids, positions, n_heads, head_dim, dtype, device
     key = ((seed * 1000003 + stream) * 1000003 + rids) * 1048576 + pos
     rows = _mix64(key) & (_TABLE_ROWS - 1)
     table = _value_table(seed, stream, n_heads, head_dim, dtype, device)
+    if table.is_cuda:
+        rows = rows.pin_memory()   # a copy from pageable memory would wait for the stream
     return table.index_select(0, rows.to(table.device, non_blocking=True))
 
 

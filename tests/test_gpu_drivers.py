@@ -206,6 +206,31 @@ def test_trace_steps_match_the_oracle(cuda_dev):
     assert runner.pool.check_device_errors() == 0
 
 
+def test_trace_with_the_host_a_step_ahead_ends_in_the_same_pool(cuda_dev):
+    # TraceRunner.step(wait=False) plans and launches step n + 1 while step n
+    # runs.  The same trace run both ways (with preemption and swaps to the host
+    # pool) must plan the same steps and leave both pools bit-identical, and
+    # every step of the overlapped run gets its GPU time after finish().
+    trace = trace_requests(n_steps=30, arrivals_per_step=3.0, prompt_median=256, prompt_max=1500,
+                           out_min=20, out_max=120, seed=17)
+
+    def run(wait):
+        r = TraceRunner(cuda_dev, num_blocks=250, n_steps=30, trace=trace, token_budget=1024,
+                        max_chunk=256, preempt="swap", num_host_blocks=300)
+        r.run(max_steps=80, wait=wait)
+        torch.cuda.synchronize()
+        return r
+
+    a, b = run(True), run(False)
+    assert [(x.step, x.tokens, x.copies, x.swap_blocks) for x in a.records] == \
+        [(x.step, x.tokens, x.copies, x.swap_blocks) for x in b.records]
+    assert a.sched.metrics["swaps_out"] > 0 and a.sched.metrics == b.sched.metrics
+    assert torch.equal(a.pool.k_pool.view(torch.int16), b.pool.k_pool.view(torch.int16))
+    assert torch.equal(a.pool.v_pool.view(torch.int16), b.pool.v_pool.view(torch.int16))
+    assert all(x.gpu_ms is not None and x.gpu_ms > 0 for x in b.records)
+    assert a.pool.check_device_errors() == 0 and b.pool.check_device_errors() == 0
+
+
 def test_recompute_reproduces_the_same_kv(cuda_dev):
     # a request preempted and re-prefilled holds bit-identical K/V afterwards
     trace = [(0, 40, 30), (0, 40, 30), (1, 40, 30)]
