@@ -236,12 +236,14 @@ def test_full_size_decode_workloads_every_row(cuda_dev, name):
     assert pool.check_device_errors() == 0
 
 
-def test_full_size_chunk512_sampled_rows(cuda_dev):
-    # sixteen 512-token chunks at context 4,096 (the bench's prefill workload) at
-    # full size: the first and last row of every 256-row work item of the
-    # tcgen05 kernel (rows are (token, group head) pairs, token-major, per
-    # (sequence, kv head)) plus 2,000 random rows, against the oracle
-    b = workload_batch("chunk512_bf16", poison_unused=False)
+@pytest.mark.parametrize("workload,item_rows", [("chunk512_bf16", 256), ("chunk512_d256_bf16", 128)])
+def test_full_size_chunk512_sampled_rows(cuda_dev, workload, item_rows):
+    # sixteen 512-token chunks at context 4,096 (the bench's prefill workloads,
+    # head dim 128 and 256) at full size: the first and last row of every work
+    # item of the tcgen05 kernel (256 rows at head dim 128, 128 at 256; rows are
+    # (token, group head) pairs, token-major, per (sequence, kv head)) plus
+    # 2,000 random rows, against the oracle
+    b = workload_batch(workload, poison_unused=False)
     T, Hq, d = b["q"].shape
     Hkv = b["k_pool"].shape[1]
     g = Hq // Hkv
@@ -253,13 +255,13 @@ def test_full_size_chunk512_sampled_rows(cuda_dev):
     for s in range(len(qsl) - 1):
         qn = qsl[s + 1] - qsl[s]
         for kvh in range(Hkv):
-            for r0 in range(0, qn * g, 256):
-                for r in (r0, min(r0 + 255, qn * g - 1)):
+            for r0 in range(0, qn * g, item_rows):
+                for r in (r0, min(r0 + item_rows - 1, qn * g - 1)):
                     rows.append([qsl[s] + r // g, kvh * g + r % g])
     ref = oracle.paged_attention_rows(b["q"], b["k_pool"], b["v_pool"], b["block_tables"],
                                       b["context_lens"], b["query_start_lens"], b["scale"], rows)
     got_rows = torch.stack([got[t, h] for t, h in rows])
-    assert_close(got_rows, ref, torch.bfloat16, "chunk512")
+    assert_close(got_rows, ref, torch.bfloat16, workload)
     assert torch.isfinite(got).all()
     assert pool.check_device_errors() == 0
 
