@@ -67,9 +67,21 @@ def test_attention_over_zero_sequences(cuda_dev, dtype, d):
                                         NULL, ctypes.c_void_p(qsl.data_ptr()), 0, 0, 32,
                                         ctypes.c_float(0.1), ctypes.c_void_p(ws.data_ptr()), 256, s)
     assert recorded_ops(cuda_dev, call) == (0, 0)
+
+    def call_append(s):   # the one-call step: no rows to store, nothing to attend
+        return lib().pk_paged_attention_append(pool.handle, NULL, NULL, NULL, ctypes.c_void_p(out.data_ptr()),
+                                               NULL, 1, NULL, ctypes.c_void_p(qsl.data_ptr()), 0, 0, 32,
+                                               ctypes.c_float(0.1), ctypes.c_void_p(ws.data_ptr()), 256, s)
+    assert recorded_ops(cuda_dev, call_append) == (0, 0)
     got = api.paged_attention(torch.empty((0, 32, d), dtype=dtype, device=cuda_dev), pool.k_pool,
                               pool.v_pool, torch.empty((0, 1), dtype=torch.int32, device=cuda_dev),
                               torch.empty((0,), dtype=torch.int32, device=cuda_dev), qsl, 0.1)
+    assert got.shape == (0, 32, d)
+    empty_kv = torch.empty((0, 8, d), dtype=dtype, device=cuda_dev)
+    got = api.paged_attention_append(torch.empty((0, 32, d), dtype=dtype, device=cuda_dev), empty_kv,
+                                     empty_kv, pool.k_pool, pool.v_pool,
+                                     torch.empty((0, 1), dtype=torch.int32, device=cuda_dev),
+                                     torch.empty((0,), dtype=torch.int32, device=cuda_dev), qsl, 0.1)
     assert got.shape == (0, 32, d)
     assert torch.isnan(out.float()).all()
     _unchanged(pool, k0, v0)

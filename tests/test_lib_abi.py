@@ -41,6 +41,8 @@ def test_pool_create_rejects_unsupported(args):
 def test_null_pool_is_rejected():
     L = _lib.lib()
     assert L.pk_paged_attention(None, None, None, None, 1, None, None, 1, 1, 1, 1.0, None, 0, None) == 1
+    assert L.pk_paged_attention_append(None, None, None, None, None, None, 1, None, None, 1, 1, 1, 1.0,
+                                       None, 0, None) == 1
     assert L.pk_paged_kv_append(None, None, None, None, 1, None) == 1
     assert L.pk_block_copy(None, None, 1, None) == 1
     assert L.pk_swap_blocks(None, None, None, 4, None, 1, 1, None) == 1
