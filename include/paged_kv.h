@@ -229,7 +229,8 @@ int pk_paged_attention(const pk_pool *pool, const void *q, void *out,
  * Results, and the pool afterwards, equal those of the two separate calls.
  * A table entry outside the pool is recorded (PK_ERR_BAD_INDEX) and its row
  * is not stored. Errors: as pk_paged_attention, and PK_ERR_INVALID_ARG for
- * k or v NULL or misaligned.
+ * k or v NULL or misaligned when num_seqs > 0. With num_seqs == 0 the call
+ * queues no work and may be given NULL arrays, as pk_paged_attention may.
  * ------------------------------------------------------------------------ */
 int pk_paged_attention_append(const pk_pool *pool, const void *q, const void *k, const void *v,
                               void *out, const int32_t *block_tables, int max_blocks_per_seq,

@@ -251,9 +251,10 @@ int pk_attention_workspace_size(const pk_pool *pool, int num_seqs, int num_token
 
 namespace {
 
-// Checks and launch shared by the two attention entry points; k_new / v_new
-// nullptr: no append.
-int attention_call(const pk_pool *pool, const void *q, const void *k_new, const void *v_new, void *out,
+// Checks and launch shared by the two attention entry points; append: the
+// query rows' own K/V (k_new, v_new) are stored first.
+int attention_call(const pk_pool *pool, const void *q, bool append, const void *k_new, const void *v_new,
+                   void *out,
                    const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
                    const int32_t *query_start_lens, int num_seqs, int num_tokens, int n_q_heads, float scale,
                    void *workspace, size_t workspace_bytes, pk_stream_t stream) {
@@ -270,8 +271,7 @@ int attention_call(const pk_pool *pool, const void *q, const void *k_new, const 
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(block_tables, 4) ||
         !aligned(context_lens, 4) || !aligned(query_start_lens, 4))
         return fail(PK_ERR_INVALID_ARG, "misaligned pointer argument");
-    const bool append = k_new != nullptr || v_new != nullptr;
-    if (append && (!k_new || !v_new)) return fail(PK_ERR_INVALID_ARG, "k and v must both be given");
+    if (append && (!k_new || !v_new)) return fail(PK_ERR_INVALID_ARG, "NULL k or v");
     if (append && (!aligned(k_new, 16) || !aligned(v_new, 16)))
         return fail(PK_ERR_INVALID_ARG, "misaligned k or v");
     if (!(scale > 0.f) || scale != scale) return fail(PK_ERR_INVALID_ARG, "scale must be > 0");
@@ -294,7 +294,7 @@ int pk_paged_attention(const pk_pool *pool, const void *q, void *out,
                        const int32_t *context_lens, const int32_t *query_start_lens,
                        int num_seqs, int num_tokens, int n_q_heads, float scale,
                        void *workspace, size_t workspace_bytes, pk_stream_t stream) {
-    return attention_call(pool, q, nullptr, nullptr, out, block_tables, max_blocks_per_seq, context_lens,
+    return attention_call(pool, q, false, nullptr, nullptr, out, block_tables, max_blocks_per_seq, context_lens,
                           query_start_lens, num_seqs, num_tokens, n_q_heads, scale, workspace,
                           workspace_bytes, stream);
 }
@@ -304,8 +304,7 @@ int pk_paged_attention_append(const pk_pool *pool, const void *q, const void *k,
                               const int32_t *context_lens, const int32_t *query_start_lens,
                               int num_seqs, int num_tokens, int n_q_heads, float scale,
                               void *workspace, size_t workspace_bytes, pk_stream_t stream) {
-    if (!k || !v) return fail(PK_ERR_INVALID_ARG, "NULL k or v");
-    return attention_call(pool, q, k, v, out, block_tables, max_blocks_per_seq, context_lens,
+    return attention_call(pool, q, true, k, v, out, block_tables, max_blocks_per_seq, context_lens,
                           query_start_lens, num_seqs, num_tokens, n_q_heads, scale, workspace,
                           workspace_bytes, stream);
 }
