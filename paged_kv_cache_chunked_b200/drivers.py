@@ -258,8 +258,11 @@ class ForkRunner:
 
     def __init__(self, device, n_prompts=64, prompt_len=1024, n_samples=4, block_size=16,
                  n_q_heads=32, n_kv_heads=8, head_dim=128, decode_steps=256, seed=1005,
-                 dtype=torch.bfloat16, chunk=512):
+                 dtype=torch.bfloat16, chunk=512, fused=False):
         self.device = torch.device(device)
+        # fused: a decode step's append and attention as one call (the copy-on-
+        # write copies first; the rows then go through the updated tables)
+        self.fused = fused
         self.Hq, self.Hkv, self.d, self.bs = n_q_heads, n_kv_heads, head_dim, block_size
         self.dtype, self.seed, self.chunk = dtype, seed, chunk
         self.n_prompts, self.prompt_len, self.n_samples = n_prompts, prompt_len, n_samples
@@ -336,9 +339,13 @@ class ForkRunner:
             e0.record(stream)
         if dd["pairs"].shape[0]:
             api.block_copy(dd["pairs"], pool=self.pool)
-        api.paged_kv_append(k, v, dd["slots"], pool=self.pool)
-        out = api.paged_attention(q, self.pool.k_pool, self.pool.v_pool, dd["tables"], dd["ctx"],
-                                  dd["qsl"], self.scale)
+        if self.fused:
+            out = api.paged_attention_append(q, k, v, self.pool.k_pool, self.pool.v_pool, dd["tables"],
+                                             dd["ctx"], dd["qsl"], self.scale)
+        else:
+            api.paged_kv_append(k, v, dd["slots"], pool=self.pool)
+            out = api.paged_attention(q, self.pool.k_pool, self.pool.v_pool, dd["tables"], dd["ctx"],
+                                      dd["qsl"], self.scale)
         if timed:
             e1.record(stream)
         if on_step is not None:

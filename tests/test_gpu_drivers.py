@@ -257,12 +257,16 @@ def test_recompute_reproduces_the_same_kv(cuda_dev):
     assert any(getattr(r, "checked", False) for r in runner.sched.finished + runner.sched.running)
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["append+attention", "one call"])
 @pytest.mark.parametrize("prompt_len,bs,copies_per_prompt", [(100, 16, 3), (96, 16, 0), (37, 8, 3),
                                                               (64, 32, 0)])
-def test_fork_copy_on_write(cuda_dev, prompt_len, bs, copies_per_prompt):
+def test_fork_copy_on_write(cuda_dev, prompt_len, bs, copies_per_prompt, fused):
+    # fused: each decode step is one pk_paged_attention_append call after the
+    # copy-on-write copies, so the new rows go where the updated tables point;
+    # the mirror appends them with the manager's slots
     n_prompts, n_samples = 4, 4
     runner = ForkRunner(cuda_dev, n_prompts=n_prompts, prompt_len=prompt_len,
-                        n_samples=n_samples, block_size=bs, decode_steps=6)
+                        n_samples=n_samples, block_size=bs, decode_steps=6, fused=fused)
     runner.prefill()
     torch.cuda.synchronize()
     shared = runner.unique_blocks()
@@ -282,6 +286,8 @@ def test_fork_copy_on_write(cuda_dev, prompt_len, bs, copies_per_prompt):
 
     for _ in range(runner.decode_steps):
         runner.decode_step(on_step)
+    torch.cuda.synchronize()
+    assert torch.equal(runner.pool.k_pool.cpu(), mirror.k) and torch.equal(runner.pool.v_pool.cpu(), mirror.v)
     assert copies[0] == n_prompts * copies_per_prompt and sum(copies[1:]) == 0
     # after diverging, siblings differ only in the blocks written since the fork
     for i in range(n_prompts):
