@@ -329,10 +329,11 @@ def test_split_k_partition_count_leaves_the_result_to_rounding(cuda_dev, Hq, Hkv
     # sequences, the same sequence, with the same pool, table and query, spans
     # only a few. The merge combines the partitions in fp32, but each partition
     # rounds its P to bf16 for the tensor core against its own reference max,
-    # so the two outputs agree to P's rounding (2^-8 per weight), not to fp32:
-    # each (row, head) within a 2^-7 share of its largest output magnitude. A
-    # merge that dropped or misweighted a partition moves outputs by about
-    # their own size.
+    # so the two outputs agree to P's rounding (2^-9 per weight) and the
+    # output's own bf16 rounding, not to fp32: each (row, head) within 2^-6 of
+    # its largest output magnitude (six seeds at d 128 and 256 reached at most
+    # half of that). A merge that dropped or misweighted one of a hundred
+    # partitions moves outputs by about a fifth of that magnitude.
     ctx = [8000] + [200 + (i * 97) % 1800 for i in range(300)]
     b = make_batch(ctx, None, block_size=16, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d,
                    dtype=torch.bfloat16, seed=71, poison_unused=False)
@@ -341,7 +342,7 @@ def test_split_k_partition_count_leaves_the_result_to_rounding(cuda_dev, Hq, Hkv
     alone = dict(b, q=b["q"][:1], block_tables=b["block_tables"][:1], context_lens=b["context_lens"][:1],
                  query_start_lens=b["query_start_lens"][:2])
     one = run_gpu_attention(alone, pool, cuda_dev)[0].float()
-    bound = torch.maximum(many.abs(), one.abs()).amax(dim=-1, keepdim=True) * 2.0 ** -7
+    bound = torch.maximum(many.abs(), one.abs()).amax(dim=-1, keepdim=True) * 2.0 ** -6
     assert ((many - one).abs() <= bound).all(), float(((many - one).abs() / bound).max())
     ref = oracle.paged_attention(alone["q"], b["k_pool"], b["v_pool"], alone["block_tables"],
                                  alone["context_lens"], alone["query_start_lens"], b["scale"])[0]
