@@ -29,7 +29,7 @@ import torch
 
 from . import api
 from .scheduler import Request, Scheduler, StaticScheduler
-from .workloads import SYS_VID_BASE, token_values, trace_requests
+from .workloads import SYS_VID_BASE, token_values_qkv, trace_requests
 
 
 class StepRecord:
@@ -152,9 +152,7 @@ class TraceRunner:
         if timed:
             ev_v = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             ev_v[0].record(stream)
-        q = token_values(self.seed, 0, rids, pos, self.Hq, self.d, self.dtype, dev)
-        k = token_values(self.seed, 1, rids, pos, self.Hkv, self.d, self.dtype, dev)
-        v = token_values(self.seed, 2, rids, pos, self.Hkv, self.d, self.dtype, dev)
+        q, k, v = token_values_qkv(self.seed, rids, pos, self.Hq, self.Hkv, self.d, self.dtype, dev)
         if timed:
             ev_v[1].record(stream)
         t_v = time.perf_counter() - t_v
@@ -280,9 +278,7 @@ class ForkRunner:
 
     def _values(self, keys, pos):
         dev = self.device
-        q = token_values(self.seed, 0, keys, pos, self.Hq, self.d, self.dtype, dev)
-        k = token_values(self.seed, 1, keys, pos, self.Hkv, self.d, self.dtype, dev)
-        v = token_values(self.seed, 2, keys, pos, self.Hkv, self.d, self.dtype, dev)
+        q, k, v = token_values_qkv(self.seed, keys, pos, self.Hq, self.Hkv, self.d, self.dtype, dev)
         return q, k, v
 
     def prefill(self):

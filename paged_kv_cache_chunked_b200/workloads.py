@@ -224,6 +224,23 @@ def token_values(seed, stream, rids, positions, n_heads, head_dim, dtype, device
     return table.index_select(0, rows.to(table.device, non_blocking=True))
 
 
+def token_values_qkv(seed, rids, positions, n_q_heads, n_kv_heads, head_dim, dtype, device="cpu"):
+    """token_values of streams 0, 1 and 2 (q, k, v) for the same keys, with one
+    hash pass over a [3, T] key tensor and one host-to-device copy of the rows:
+    the same values as three token_values calls."""
+    rids = torch.as_tensor(rids, dtype=torch.int64)
+    pos = torch.as_tensor(positions, dtype=torch.int64)
+    streams = torch.arange(3, dtype=torch.int64)[:, None]
+    key = ((seed * 1000003 + streams) * 1000003 + rids[None, :]) * 1048576 + pos[None, :]
+    rows = _mix64(key) & (_TABLE_ROWS - 1)
+    tables = [_value_table(seed, st, h, head_dim, dtype, device)
+              for st, h in ((0, n_q_heads), (1, n_kv_heads), (2, n_kv_heads))]
+    if tables[0].is_cuda:
+        rows = rows.pin_memory()   # a copy from pageable memory would wait for the stream
+    rows = rows.to(tables[0].device, non_blocking=True)
+    return tuple(t.index_select(0, rows[i]) for i, t in enumerate(tables))
+
+
 def trace_requests(n_steps=300, arrivals_per_step=4.0, prompt_median=512, prompt_sigma=1.0,
                    prompt_max=8192, out_min=10, out_max=500, seed=1004):
     """Continuous-batching trace: Poisson arrivals per step, lognormal prompt

@@ -438,3 +438,17 @@ def test_step_value_keys_match_the_per_request_keys():
         sched.complete(plan)
         step += 1
     assert checked > 20 and shared > 0
+
+
+def test_step_values_in_one_pass_equal_the_per_stream_values():
+    # the drivers draw a step's q, k and v with one hash pass over the keys;
+    # each must be bit for bit the per-stream generator's output
+    from paged_kv_cache_chunked_b200.workloads import SYS_VID_BASE, token_values, token_values_qkv
+    g = torch.Generator().manual_seed(5)
+    rids = torch.randint(0, 400, (257,), generator=g)
+    rids[::7] = SYS_VID_BASE + 3
+    pos = torch.randint(0, 9000, (257,), generator=g)
+    q, k, v = token_values_qkv(1004, rids, pos, 32, 8, 128, torch.bfloat16)
+    for stream, (got, heads) in enumerate(((q, 32), (k, 8), (v, 8))):
+        want = token_values(1004, stream, rids, pos, heads, 128, torch.bfloat16)
+        assert torch.equal(got.view(torch.int16), want.view(torch.int16))
