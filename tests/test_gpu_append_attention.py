@@ -39,6 +39,8 @@ CASES = [
     ([300, 45, 1111], None, 32, 2, 128, 16, torch.bfloat16, "decode, 16 q heads per kv head"),
     ([100, 260], [1, 40], 32, 8, 128, 8, torch.bfloat16, "mixed, block size 8"),
     ([50, 333, 9], [1, 7, 1], 8, 8, 64, 16, torch.float32, "fp32 pool"),
+    ([100, 700, 33, 1], None, 32, 8, 128, 32, torch.bfloat16, "decode, block size 32"),
+    ([50, 3000, 129], [1, 200, 64], 16, 4, 128, 64, torch.bfloat16, "mixed, block size 64"),
     ([1 + (i * 53) % 300 for i in range(600)], None, 8, 2, 64, 16, torch.bfloat16,
      "600 sequences, two launch windows"),
 ]
