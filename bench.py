@@ -566,12 +566,12 @@ def run_ours(args, rank, world, device):
     if blocks and T == B:
         per_window = 2                  # block-streaming decode, merge kernel
     elif blocks and umma:
-        per_window = 3                  # block-streaming decode, merge kernel, tcgen05 chunk kernel
+        per_window = 3                  # tcgen05 chunk kernel, block-streaming decode behind it, merge kernel
     else:
         per_window = 2 if T > B or Hq // Hkv > 16 else 1
-    # the new K/V are stored by the block-streaming kernel where it serves the
-    # batch, else by the position append kernel
-    stored_in_kernel = blocks and (T == B or umma)
+    # the new K/V are stored by the block-streaming kernel where it serves a
+    # decode-only batch, else by the position append kernel
+    stored_in_kernel = blocks and T == B
     launches_per_step = (0 if stored_in_kernel else 1) + (windows * per_window if tc else 1)
     for _ in range(max(args.warmup, 3)):
         step()

@@ -221,11 +221,11 @@ int pk_paged_attention(const pk_pool *pool, const void *q, void *out,
  * pos % bs, before any attention reads them.
  *
  * The slots follow from the tables, so no slot_mapping is taken.
- *   - Block-streaming path (bf16 decode rows, groups of at most 8): the decode
- *     kernel stores each decode row's K/V just before it loads the block
- *     holding it, and a mixed step's chunk rows before its chunk kernel
- *     starts. No append kernel runs.
- *   - Other geometries: an append kernel runs first, then attention.
+ *   - A decode-only batch on the block-streaming path (bf16, groups of at
+ *     most 8): the decode kernel stores each row's K/V just before it loads
+ *     the block holding it. No append kernel runs.
+ *   - Otherwise (batches with prefill chunks, other geometries): an append
+ *     kernel stores every row first, then attention runs.
  * Results, and the pool afterwards, equal those of the two separate calls.
  * A table entry outside the pool is recorded (PK_ERR_BAD_INDEX) and its row
  * is not stored. Errors: as pk_paged_attention, and PK_ERR_INVALID_ARG for

@@ -199,13 +199,15 @@ attention_chunk_umma256_kernel(const __grid_constant__ CUtensorMap tmk2,  // K: 
     __syncthreads();
     tc_after();
     const uint32_t tmem = *tmem_slot;
-    // Launched as a programmatic dependent of the kernel before it on the stream
-    // (in a mixed batch, the decode rows' merge kernel): the plan above reads
-    // only the query offsets and lengths, which no kernel of the call writes;
-    // the pool, the queries, the tables and the output are touched only after
-    // this wait, which also covers every kernel before that one
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // Launched as a programmatic dependent of the kernel before it on the stream:
+    // the plan above reads only the query offsets and lengths, which no kernel
+    // of the call writes; the pool, the queries, the tables and the output are
+    // touched only after this wait, which also covers every kernel before that
+    // one.  Dependents are signalled after the wait, so a kernel launched behind
+    // this one (the decode rows of a mixed step) may start work at once: the
+    // step's rows and everything before this kernel are complete by then.
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // the item at position idx of the ranked list (the chunk-sequence count is
     // read back from shared memory: kept in a register across the item loops it

@@ -92,13 +92,20 @@ struct BlkParams {
     const int32_t *tables, *ctx, *qsl;
     int seq0, nseq, max_blocks, n_q_heads, n_kv_heads, group, block_size, num_blocks, num_tokens;
     int skip_chunks;  // 1: sequences of several query tokens belong to the chunk kernel (skipped)
+    // 1: launched behind the chunk kernel of a mixed step, which signals its
+    // dependents only once its own wait has returned (the step's rows and the
+    // previous call are complete by then).  This grid then reads and writes
+    // without a wait of its own, so its CTAs work on the SMs the chunk kernel
+    // frees, and waits for the chunk grid only before it exits: the grids
+    // after it on the stream still find both finished.
+    int behind_chunk;
     int HS, NBS, ST, NPH, NS;  // geometry: heads / blocks / tokens per stage, phases, stages
     int ncta, cap_rows;
     float scale_log2;
     int *mplan;                      // the merge kernel's list of split pairs
-    // the query rows' own K/V ([num_tokens, n_kv_heads, D]) to store at their
-    // positions before they are read, and the pool they go to; k_new == nullptr:
-    // nothing to store
+    // the decode rows' own K/V ([num_tokens, n_kv_heads, D]) to store at their
+    // positions before their blocks are read, and the pool they go to (a
+    // decode-only batch); k_new == nullptr: nothing to store
     const __nv_bfloat16 *k_new, *v_new;
     __nv_bfloat16 *kpool, *vpool;
     float *partial_o, *partial_lse;  // [row][D], [row]
@@ -263,7 +270,7 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
         const int nchunks = cp.count();
         int pending = (int)blockIdx.x;
         int n_stage = 0, n_item = 0;
-        bool waited = false;  // griddepcontrol.wait done
+        bool waited = prm.behind_chunk != 0;  // griddepcontrol.wait done (or not needed)
         const uint64_t stream_pol = l2_evict_first_policy();  // K/V rows are read once
         auto chunk_entry = [&](int b, int blk_base) -> int {
             const int nblk = (s_ctx[b] + bs - 1) / bs;
@@ -493,52 +500,8 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
         }
     } else {
         // ---------------------------------------------------------- consumers
-        asm volatile("griddepcontrol.wait;" ::: "memory");  // before any write
+        if (!prm.behind_chunk) asm volatile("griddepcontrol.wait;" ::: "memory");  // before any write
         const int cw = warp - 1, hl = cw % HS, ph = cw / HS;
-        if (prm.k_new != nullptr && prm.skip_chunks) {
-            // the chunk rows' own K/V (sequences of several query tokens), for
-            // the chunk kernel that follows, stored while this CTA's first
-            // stages are in flight: one consumer warp per token, all kv heads,
-            // every load of a pass issued before its stores
-            constexpr int RC = D / 8, U = 4;  // 16-byte chunks of a head's row; chunks per lane and pass
-            const int n = Hkv * RC;
-            const uint4 *ks = (const uint4 *)prm.k_new, *vs = (const uint4 *)prm.v_new;
-            uint4 *kd = (uint4 *)prm.kpool, *vd = (uint4 *)prm.vpool;
-            for (int t = s_qsl[0] + (int)blockIdx.x * kNC + cw; t < s_qsl[nseq]; t += (int)gridDim.x * kNC) {
-                const int b = find_seq(s_qsl, nseq, t);
-                const int qb = s_qsl[b + 1] - s_qsl[b];
-                if (qb < 2) continue;  // a decode row: the producer stores it before its block is loaded
-                const int pos = s_ctx[b] - qb + (t - s_qsl[b]);
-                const int jb = pos / bs;
-                if (pos < 0 || jb >= prm.max_blocks) continue;  // recorded by the plan
-                const int phys = __ldg(prm.tables + (long long)(prm.seq0 + b) * prm.max_blocks + jb);
-                if (phys < 0 || phys >= prm.num_blocks) {
-                    if (lane == 0) record_error(prm.err, PK_ERR_BAD_INDEX);
-                    continue;
-                }
-                const long long row = ((long long)phys * Hkv * bs + (pos - jb * bs)) * RC;
-                for (int i0 = 0; i0 < n; i0 += 32 * U) {
-                    uint4 kr[U], vr[U];
-#pragma unroll
-                    for (int u = 0; u < U; ++u) {
-                        const int i = i0 + u * 32 + lane;
-                        if (i < n) {
-                            kr[u] = __ldg(ks + (long long)t * n + i);
-                            vr[u] = __ldg(vs + (long long)t * n + i);
-                        }
-                    }
-#pragma unroll
-                    for (int u = 0; u < U; ++u) {
-                        const int i = i0 + u * 32 + lane;
-                        if (i < n) {  // kv head i / RC: (block, head, offset) rows are bs * RC apart
-                            const long long dst = row + (long long)(i / RC) * bs * RC + i % RC;
-                            kd[dst] = kr[u];
-                            vd[dst] = vr[u];
-                        }
-                    }
-                }
-            }
-        }
         const int qr = lane >> 2, qc = (lane & 3) * 2;
         const int mi = lane >> 3, rr = lane & 7;
         const int a_row = (mi & 1) * 8 + rr, a_col = (mi >> 1) * 8;  // K rows (A of S^T)
@@ -788,6 +751,8 @@ attention_decode_blocks_kernel(const __grid_constant__ CUtensorMap tmk,
         if (!ok && lane == 0) record_error(prm.err, PK_ERR_TIMEOUT);
     }
     __syncthreads();
+    // behind a chunk kernel: the CTA leaves only once the chunk grid has finished
+    if (prm.behind_chunk && threadIdx.x == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // Merge kernel [flash-decoding combination].  For every (sequence, head
@@ -890,7 +855,8 @@ int blocks_prepare(pk_pool *p) {
 }
 
 template <int D>
-int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, bool skip_chunks, cudaStream_t st) {
+int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, bool skip_chunks, bool behind_chunk,
+                  cudaStream_t st) {
     BlkParams tp{};
     tp.skip_chunks = skip_chunks ? 1 : 0;
     tp.q = (const __nv_bfloat16 *)a.q;
@@ -931,6 +897,7 @@ int blocks_launch(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, bool s
     for (int s0 = 0; s0 < a.num_seqs; s0 += kMaxSeqsPerLaunch) {
         tp.seq0 = s0;
         tp.nseq = std::min(kMaxSeqsPerLaunch, a.num_seqs - s0);
+        tp.behind_chunk = behind_chunk && s0 == 0 ? 1 : 0;  // later windows follow a merge kernel
         {
             cudaLaunchConfig_t c0 = {};
             c0.gridDim = dim3(tp.ncta);
@@ -1018,11 +985,11 @@ bool decode_blocks_applies(const pk_pool *p, const AttnArgs &a) {
 }
 
 int launch_decode_blocks(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, bool skip_chunks,
-                         cudaStream_t st) {
+                         bool behind_chunk, cudaStream_t st) {
     switch (p->head_dim) {
-        case 64: return blocks_launch<64>(p, a, w, skip_chunks, st);
-        case 128: return blocks_launch<128>(p, a, w, skip_chunks, st);
-        case 256: return blocks_launch<256>(p, a, w, skip_chunks, st);
+        case 64: return blocks_launch<64>(p, a, w, skip_chunks, behind_chunk, st);
+        case 128: return blocks_launch<128>(p, a, w, skip_chunks, behind_chunk, st);
+        case 256: return blocks_launch<256>(p, a, w, skip_chunks, behind_chunk, st);
         default: return fail(PK_ERR_UNSUPPORTED, "decode path: head_dim %d", p->head_dim);
     }
 }

@@ -94,17 +94,25 @@ int launch_attention_tc(const pk_pool *p, const AttnArgs &a, cudaStream_t st) {
     const int g = a.n_q_heads / p->n_kv_heads;
     const bool has_multi = a.num_tokens > a.num_seqs;  // some sequence has several query tokens
     const bool blocks = decode_blocks_applies(p, a);
-    // With an append (a.k_new), the block-streaming kernel stores the query
-    // rows' K/V itself: a decode row's just before its block is loaded, the
-    // chunk rows before the chunk kernel starts.  The other paths run the
-    // position append kernel first.
-    if (!has_multi && blocks) return launch_decode_blocks(p, a, w, false, st);
+    // With an append (a.k_new), the block-streaming kernel of a decode-only
+    // batch stores the query rows' K/V itself, each just before its block is
+    // loaded.  The other paths run the position append kernel first.
+    if (!has_multi && blocks) return launch_decode_blocks(p, a, w, false, false, st);
     if (blocks && chunk_umma_applies(p, a)) {
-        // a mixed continuous-batching step: the one-token rows stream whole
-        // blocks (block-streaming kernel and its merge kernel), then the
-        // tcgen05 kernel takes every sequence of several query tokens
-        int rc = launch_decode_blocks(p, a, w, true, st);
+        // a mixed continuous-batching step: the tcgen05 kernel takes every
+        // sequence of several query tokens, then the one-token rows stream
+        // whole blocks (block-streaming kernel and its merge kernel).  The
+        // chunk kernel's CTAs finish unevenly (its items differ in work); the
+        // decode kernel, launched behind it, starts its CTAs on the SMs they
+        // free and waits for the chunk grid only before it exits.
+        int rc = PK_OK;
+        if (a.k_new != nullptr) rc = launch_kv_append_at_positions(p, a, st);
         if (rc == PK_OK) rc = launch_chunk_umma(p, a, true, st);
+        if (rc == PK_OK) {
+            AttnArgs d = a;
+            d.k_new = d.v_new = nullptr;  // stored above
+            rc = launch_decode_blocks(p, d, w, true, true, st);
+        }
         return rc;
     }
     if (a.k_new != nullptr) {

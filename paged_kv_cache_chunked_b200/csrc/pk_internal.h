@@ -133,7 +133,7 @@ int decode_blocks_prepare_pool(pk_pool *p);
 int decode_blocks_chunks_per_cta();
 bool decode_blocks_applies(const pk_pool *p, const AttnArgs &a);
 int launch_decode_blocks(const pk_pool *p, const AttnArgs &a, const DecodeWs &w, bool skip_chunks,
-                         cudaStream_t st);
+                         bool behind_chunk, cudaStream_t st);
 // 2-D TMA view of a pool (rows of head_dim bf16) with boxes of 64 columns x box_rows.
 int encode_pool_map(CUtensorMap *map, void *base, const pk_pool *p, int box_rows);
 // 3-D TMA view (column in panel, row, 64-column panel) with boxes of all panels x box_rows.
