@@ -22,6 +22,7 @@ from ._lib import (PK_BF16, PK_ERR_TIMEOUT, PK_F32, PK_PATH_CHUNK_TCGEN05,  # no
                    check, lib)
 
 _DTYPES = {torch.float32: PK_F32, torch.bfloat16: PK_BF16}
+_WINDOW_SEQS = 512   # sequences per kernel launch window (the attention scratch stops growing there)
 _pools = weakref.WeakValueDictionary()  # k_pool data_ptr -> KVPool
 
 
@@ -107,10 +108,17 @@ class KVPool:
             stream = torch.cuda.current_stream(self.device)
         ws = self._workspaces.get(stream.cuda_stream)
         if ws is None or ws.numel() < n.value:
+            # sized at once for a full launch window of sequences (the size stops
+            # growing there; a few tens of MiB at most), so that a serving loop
+            # whose batches grow does not allocate, and wait on the allocator, in
+            # the middle of its steps
+            full = ctypes.c_size_t()
+            check(lib().pk_attention_workspace_size(self.handle, max(num_seqs, _WINDOW_SEQS), num_tokens,
+                                                    n_q_heads, max_blocks, ctypes.byref(full)))
             # zero-filled once, on the stream that uses it; every completed call
             # leaves its counters zeroed again
             with torch.cuda.stream(stream):
-                ws = torch.zeros(max(n.value, 256), dtype=torch.uint8, device=self.device)
+                ws = torch.zeros(max(n.value, full.value, 256), dtype=torch.uint8, device=self.device)
             self._workspaces[stream.cuda_stream] = ws
         return ws
 
