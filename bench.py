@@ -552,9 +552,10 @@ def run_ours(args, rank, world, device):
     def attention_only():
         api.paged_attention(dq, pool.k_pool, pool.v_pool, dt_, dctx, dqsl, batch["scale"], out=out)
 
-    # append, then per window of 512 sequences: with groups of <= 8 q heads the
-    # block-streaming decode kernel (then, with chunks present, the tcgen05
-    # chunk kernel), else a chunk kernel (when chunks are present) and the
+    # the append (unless the decode kernel stores the rows), then per window of
+    # 512 sequences: with groups of <= 8 q heads the block-streaming decode
+    # kernel and its merge kernel, behind the tcgen05 chunk kernel when chunks
+    # are present; else a chunk kernel (when chunks are present) and the
     # tile-streaming decode kernel; the general kernel is one launch
     paths = pool.paths()
     tc = bool(paths & api.PK_PATH_TENSOR_CORE)
