@@ -43,6 +43,8 @@ CASES = [
     ([50, 3000, 129], [1, 200, 64], 16, 4, 128, 64, torch.bfloat16, "mixed, block size 64"),
     ([1 + (i * 53) % 300 for i in range(600)], None, 8, 2, 64, 16, torch.bfloat16,
      "600 sequences, two launch windows"),
+    ([max(64, 1 + (i * 53) % 300) for i in range(600)], [40 if i % 50 == 0 else 1 for i in range(600)],
+     32, 8, 128, 16, torch.bfloat16, "600 sequences with chunks, two launch windows"),
 ]
 
 
